@@ -1,0 +1,335 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each check is chosen so that a plausible mistake in the oracle (a wrong
+gather index, a transposed head mapping, a sign or scale slip in the softmax,
+a dropped merge term, a bad f16/bf16 decoding) fails at least one of them:
+
+* library routines: torch's scaled_dot_product_attention (float64, with its
+  own GQA grouping), numpy's float16 and torch's bfloat16 widening;
+* closed forms: one token, zero query / zero scale, constant and shifted V,
+  the large-scale limit (the arg-max row);
+* an unshifted brute force (no max subtraction) on tiny inputs;
+* invariance under any relabelling of physical blocks; one-block tables;
+* the split/merge identity for any partition size;
+* the worked examples printed on the pages (tests/golden).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_418_b200.workloads import (BF16, F16, F32, nan_fill, round_to_storage,
+                                               storage_to_float64)
+
+RNG = np.random.default_rng
+
+
+def _paged_from_contiguous(kc_list, vc_list, bs, dtype, rng, extra_blocks=3):
+    """Scatter per-sequence contiguous K/V ([ctx, Hkv, D] storage arrays) into a
+    NaN-poisoned pool through a random permutation of block ids (block-wise
+    reshapes, independent of the oracle's per-token gather)."""
+    B = len(kc_list)
+    hkv, d = kc_list[0].shape[1:]
+    nblk = [(len(k) + bs - 1) // bs for k in kc_list]
+    nb = sum(nblk) + extra_blocks
+    perm = rng.permutation(nb)
+    kp, vp = nan_fill((nb, bs, hkv, d), dtype), nan_fill((nb, bs, hkv, d), dtype)
+    tables = np.full((B, max(max(nblk), 1)), -1, dtype=np.int32)
+    used = 0
+    for b in range(B):
+        ids = perm[used:used + nblk[b]]
+        used += nblk[b]
+        tables[b, :nblk[b]] = ids
+        n = len(kc_list[b])
+        padk = nan_fill((nblk[b] * bs, hkv, d), dtype)
+        padv = nan_fill((nblk[b] * bs, hkv, d), dtype)
+        padk[:n], padv[:n] = kc_list[b], vc_list[b]
+        kp[ids] = padk.reshape(nblk[b], bs, hkv, d)
+        vp[ids] = padv.reshape(nblk[b], bs, hkv, d)
+    return kp, vp, tables
+
+
+def _rand(rng, shape, dtype, scale=1.0):
+    return round_to_storage(rng.standard_normal(shape).astype(np.float32) * scale, dtype)
+
+
+def _sdpa(q64, k64, v64, scale):
+    """torch SDPA in float64: q [Hq, D], k/v [ctx, Hkv, D] -> [Hq, D]."""
+    q = torch.from_numpy(q64)[None, :, None, :]
+    k = torch.from_numpy(np.ascontiguousarray(k64.transpose(1, 0, 2)))[None]
+    v = torch.from_numpy(np.ascontiguousarray(v64.transpose(1, 0, 2)))[None]
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=scale,
+                                                         enable_gqa=q.shape[1] != k.shape[1])
+    return o[0, :, 0, :].numpy()
+
+
+# -- element decoding ---------------------------------------------------------
+def test_widen_f16_every_bit_pattern_matches_numpy():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.widen(bits.view(np.float16), oracle.F16)
+    ref = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(ref)
+    assert (np.isnan(ours) == nan).all()
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+def test_widen_bf16_every_bit_pattern_matches_torch():
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = oracle.widen(bits, oracle.BF16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert (np.isnan(ours) == nan).all()
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+# -- gather: the pages' worked examples ------------------------------------------
+def test_gather_follows_the_block_table_example(golden_dir):
+    """Block table 0->17, 1->42, 2->8 ("五十三" section 8), 16-token blocks."""
+    g = json.load(open(os.path.join(golden_dir, "block_table_example.json")))
+    bs, table = g["block_size"], np.array(g["logical_to_physical"], dtype=np.int32)
+    nb = 64
+    pool = np.zeros((nb, bs, 1, 2), dtype=np.float32)
+    pool[:, :, 0, 0] = np.arange(nb)[:, None]          # each row knows its block
+    pool[:, :, 0, 1] = np.arange(bs)[None, :]          # ... and its row in the block
+    rows = oracle.gather(pool, oracle.F32, table, 40)[:, 0, :]
+    # token 0 -> block 17 row 0; token 20 -> block 42 row 4; token 35 -> block 8 row 3
+    assert tuple(rows[0]) == (17, 0) and tuple(rows[20]) == (42, 4) and tuple(rows[35]) == (8, 3)
+    assert tuple(rows[15]) == (17, 15) and tuple(rows[16]) == (42, 0)
+
+
+def test_gather_rejects_out_of_range_block():
+    pool = np.zeros((4, 2, 1, 1), dtype=np.float32)
+    with pytest.raises(oracle.OracleError):
+        oracle.gather(pool, oracle.F32, np.array([0, 4]), 3)
+    with pytest.raises(oracle.OracleError):
+        oracle.gather(pool, oracle.F32, np.array([0, -1]), 3)
+
+
+# -- decode vs a library routine -------------------------------------------------
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", [(F32, 4, 4, 64, 16), (F16, 8, 2, 32, 4),
+                                              (BF16, 8, 1, 16, 8), (BF16, 16, 2, 128, 16)])
+def test_decode_matches_torch_sdpa(dtype, Hq, Hkv, D, bs):
+    rng = RNG(11 + dtype + Hq)
+    ctxs = [1, 5, bs, bs + 1, 3 * bs - 1, 37]
+    kc = [_rand(rng, (n, Hkv, D), dtype) for n in ctxs]
+    vc = [_rand(rng, (n, Hkv, D), dtype) for n in ctxs]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, bs, dtype, rng)
+    q = _rand(rng, (len(ctxs), Hq, D), dtype)
+    scale = 1.0 / math.sqrt(D)
+    out = oracle.decode(q, kp, vp, dtype, tables, np.array(ctxs), scale)
+    for b in range(len(ctxs)):
+        ref = _sdpa(storage_to_float64(q[b], dtype), storage_to_float64(kc[b], dtype),
+                    storage_to_float64(vc[b], dtype), scale)
+        np.testing.assert_allclose(out[b], ref, rtol=0, atol=1e-12)
+
+
+def test_decode_rows_subset_equals_full():
+    rng = RNG(3)
+    kc = [_rand(rng, (n, 2, 16), BF16) for n in (7, 30)]
+    vc = [_rand(rng, (n, 2, 16), BF16) for n in (7, 30)]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, 8, BF16, rng)
+    q = _rand(rng, (2, 6, 16), BF16)
+    full = oracle.decode(q, kp, vp, BF16, tables, np.array([7, 30]), 0.25)
+    rows = np.array([[1, 5], [0, 0], [1, 2]])
+    sub = oracle.decode(q, kp, vp, BF16, tables, np.array([7, 30]), 0.25, rows=rows)
+    for i, (b, h) in enumerate(rows):
+        assert np.array_equal(sub[i], full[b, h])
+
+
+# -- closed forms -------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", [F32, F16, BF16])
+def test_one_token_returns_its_v_row_exactly(dtype):
+    rng = RNG(5)
+    kc = [_rand(rng, (1, 2, 32), dtype, 3.0) for _ in range(3)]
+    vc = [_rand(rng, (1, 2, 32), dtype) for _ in range(3)]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, 4, dtype, rng)
+    q = _rand(rng, (3, 4, 32), dtype, 5.0)
+    out = oracle.decode(q, kp, vp, dtype, tables, np.ones(3), 0.17)
+    for b in range(3):
+        for hq in range(4):
+            assert np.array_equal(out[b, hq], storage_to_float64(vc[b][0, hq // 2], dtype))
+
+
+def test_zero_query_or_zero_scale_gives_mean_of_v():
+    rng = RNG(6)
+    n = 23
+    kc, vc = [_rand(rng, (n, 1, 8), F32)], [_rand(rng, (n, 1, 8), F32)]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, 4, F32, rng)
+    mean = vc[0][:, 0, :].astype(np.float64).mean(axis=0)
+    q0 = np.zeros((1, 1, 8), dtype=np.float32)
+    np.testing.assert_allclose(oracle.decode(q0, kp, vp, F32, tables, [n], 1.0)[0, 0], mean,
+                               rtol=0, atol=1e-14)
+    q = _rand(rng, (1, 1, 8), F32)
+    np.testing.assert_allclose(oracle.decode(q, kp, vp, F32, tables, [n], 0.0)[0, 0], mean,
+                               rtol=0, atol=1e-14)
+
+
+def test_constant_and_shifted_v():
+    rng = RNG(8)
+    n, D = 19, 8
+    k = _rand(rng, (n, 1, D), F32)
+    c = rng.standard_normal(D).astype(np.float32)
+    vconst = np.broadcast_to(c, (n, 1, D)).copy()
+    # bf16-representable values in f32 storage, so that v + 0.5 is exact
+    v = storage_to_float64(_rand(rng, (n, 1, D), BF16), BF16).astype(np.float32)
+    q = _rand(rng, (1, 1, D), F32)
+    kp, vp, t = _paged_from_contiguous([k], [vconst], 4, F32, RNG(1))
+    np.testing.assert_allclose(oracle.decode(q, kp, vp, F32, t, [n], 0.5)[0, 0], c, atol=1e-14, rtol=0)
+    kp1, vp1, t1 = _paged_from_contiguous([k], [v], 4, F32, RNG(2))
+    kp2, vp2, t2 = _paged_from_contiguous([k], [v + np.float32(0.5)], 4, F32, RNG(2))
+    o1 = oracle.decode(q, kp1, vp1, F32, t1, [n], 0.5)[0, 0]
+    o2 = oracle.decode(q, kp2, vp2, F32, t2, [n], 0.5)[0, 0]
+    np.testing.assert_allclose(o2, o1 + 0.5, rtol=0, atol=1e-14)
+
+
+def test_large_scale_limit_picks_the_argmax_row():
+    """softmax(scale * s) -> one-hot at arg max s; a sign slip picks the arg min."""
+    rng = RNG(9)
+    n, D = 40, 16
+    k = _rand(rng, (n, 1, D), F32)
+    v = _rand(rng, (n, 1, D), F32)
+    q = _rand(rng, (1, 1, D), F32)
+    kp, vp, t = _paged_from_contiguous([k], [v], 8, F32, rng)
+    s = k[:, 0, :].astype(np.float64) @ q[0, 0].astype(np.float64)
+    i = int(np.argmax(s))
+    gap = np.sort(s)[-1] - np.sort(s)[-2]
+    out = oracle.decode(q, kp, vp, F32, t, [n], 800.0 / gap)[0, 0]
+    np.testing.assert_allclose(out, v[i, 0], rtol=0, atol=1e-12)
+
+
+def test_unshifted_brute_force_on_tiny_inputs():
+    """exp(s_i) without the max shift, summed with math.fsum, on small scores."""
+    rng = RNG(10)
+    for trial in range(20):
+        bs = int(rng.choice([1, 2, 4]))
+        n = int(rng.integers(1, 21))
+        D = int(rng.integers(1, 9))
+        Hkv, G = int(rng.integers(1, 3)), int(rng.integers(1, 3))
+        k = _rand(rng, (n, Hkv, D), F32, 0.5)
+        v = _rand(rng, (n, Hkv, D), F32)
+        q = _rand(rng, (1, Hkv * G, D), F32, 0.5)
+        kp, vp, t = _paged_from_contiguous([k], [v], bs, F32, rng)
+        out = oracle.decode(q, kp, vp, F32, t, [n], 0.3)[0]
+        for hq in range(Hkv * G):
+            h = hq // G
+            w = [math.exp(0.3 * math.fsum(float(q[0, hq, d]) * float(k[i, h, d]) for d in range(D)))
+                 for i in range(n)]
+            den = math.fsum(w)
+            ref = [math.fsum(w[i] * float(v[i, h, d]) for i in range(n)) / den for d in range(D)]
+            np.testing.assert_allclose(out[hq], ref, rtol=0, atol=1e-12)
+
+
+def test_empty_context_is_zero():
+    rng = RNG(12)
+    kp = _rand(rng, (4, 4, 1, 8), F32)
+    out = oracle.decode(_rand(rng, (2, 1, 8), F32), kp, kp, F32,
+                        np.array([[0], [1]], dtype=np.int32), [0, 3], 1.0)
+    assert np.array_equal(out[0, 0], np.zeros(8))
+
+
+# -- paging invariances -------------------------------------------------------------
+def test_relabelling_physical_blocks_is_bit_exact():
+    rng = RNG(13)
+    ctxs = [9, 33, 2]
+    kc = [_rand(rng, (n, 2, 16), F16) for n in ctxs]
+    vc = [_rand(rng, (n, 2, 16), F16) for n in ctxs]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, 4, F16, rng)
+    q = _rand(rng, (3, 4, 16), F16)
+    o1 = oracle.decode(q, kp, vp, F16, tables, ctxs, 0.25)
+    pi = rng.permutation(kp.shape[0])          # block b moves to pi[b]
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[pi], vp2[pi] = kp, vp
+    t2 = np.where(tables >= 0, pi[np.maximum(tables, 0)], -1).astype(np.int32)
+    o2 = oracle.decode(q, kp2, vp2, F16, t2, ctxs, 0.25)
+    assert np.array_equal(o1, o2)
+
+
+def test_one_block_per_sequence_equals_unpaged_attention():
+    rng = RNG(14)
+    n = 27
+    k, v = _rand(rng, (n, 2, 16), BF16), _rand(rng, (n, 2, 16), BF16)
+    q = _rand(rng, (1, 4, 16), BF16)
+    kp, vp = k.reshape(1, n, 2, 16), v.reshape(1, n, 2, 16)
+    out = oracle.decode(q, kp, vp, BF16, np.zeros((1, 1), dtype=np.int32), [n], 0.25)[0]
+    ref = _sdpa(storage_to_float64(q[0], BF16), storage_to_float64(k, BF16),
+                storage_to_float64(v, BF16), 0.25)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+# -- split / merge ------------------------------------------------------------------
+@pytest.mark.parametrize("psize", [1, 3, 8, 16, 64, 1000])
+def test_partitioned_merge_equals_single_pass(psize):
+    rng = RNG(15)
+    ctxs = [1, 17, 64, 100]
+    kc = [_rand(rng, (n, 2, 8), BF16, 2.0) for n in ctxs]
+    vc = [_rand(rng, (n, 2, 8), BF16) for n in ctxs]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, 4, BF16, rng)
+    q = _rand(rng, (4, 4, 8), BF16)
+    ref = oracle.decode(q, kp, vp, BF16, tables, ctxs, 0.7)
+    out, m, l, acc = oracle.decode_partitioned(q, kp, vp, BF16, tables, ctxs, 0.7, psize)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    # partials: each partition's own max / sum / weighted sum, empty ones marked
+    for b, n in enumerate(ctxs):
+        for hq in range(4):
+            k64 = storage_to_float64(kc[b][:, hq // 2], BF16)
+            v64 = storage_to_float64(vc[b][:, hq // 2], BF16)
+            s = 0.7 * (k64 @ storage_to_float64(q[b, hq], BF16))
+            for j in range(m.shape[2]):
+                lo, hi = j * psize, min((j + 1) * psize, n)
+                if lo >= n:
+                    assert m[b, hq, j] == -np.inf and l[b, hq, j] == 0.0
+                    continue
+                assert m[b, hq, j] == s[lo:hi].max()
+                w = np.exp(s[lo:hi] - s[lo:hi].max())
+                np.testing.assert_allclose(l[b, hq, j], w.sum(), rtol=1e-13)
+                np.testing.assert_allclose(acc[b, hq, j], w @ v64[lo:hi], rtol=0, atol=1e-12)
+
+
+# -- reshape_and_cache / copy_blocks ------------------------------------------------
+def test_reshape_and_cache_writes_exactly_the_named_slots():
+    rng = RNG(16)
+    nb, bs, hkv, d = 6, 16, 2, 8
+    kp, vp = nan_fill((nb, bs, hkv, d), BF16), nan_fill((nb, bs, hkv, d), BF16)
+    key, val = _rand(rng, (4, hkv, d), BF16), _rand(rng, (4, hkv, d), BF16)
+    slots = np.array([37, -1, 0, 95], dtype=np.int64)
+    k0, v0 = kp.copy(), vp.copy()
+    oracle.reshape_and_cache(kp, vp, key, val, slots, BF16)
+    # slot 37 = block 2 row 5; slot 0 = block 0 row 0; slot 95 = block 5 row 15
+    assert np.array_equal(kp[2, 5], key[0]) and np.array_equal(vp[2, 5], val[0])
+    assert np.array_equal(kp[0, 0], key[2]) and np.array_equal(vp[5, 15], val[3])
+    touched = np.zeros((nb, bs), dtype=bool)
+    touched[2, 5] = touched[0, 0] = touched[5, 15] = True
+    assert np.array_equal(kp[~touched], k0[~touched]) and np.array_equal(vp[~touched], v0[~touched])
+    with pytest.raises(oracle.OracleError):
+        oracle.reshape_and_cache(kp, vp, key[:1], val[:1], np.array([96]), BF16)
+
+
+def test_reshape_then_one_token_decode_returns_written_row():
+    rng = RNG(17)
+    kp, vp = nan_fill((5, 4, 2, 8), F16), nan_fill((5, 4, 2, 8), F16)
+    key, val = _rand(rng, (1, 2, 8), F16), _rand(rng, (1, 2, 8), F16)
+    oracle.reshape_and_cache(kp, vp, key, val, np.array([3 * 4]), F16)
+    out = oracle.decode(_rand(rng, (1, 4, 8), F16), kp, vp, F16,
+                        np.array([[3]], dtype=np.int32), [1], 0.3)
+    for hq in range(4):
+        assert np.array_equal(out[0, hq], val[0, hq // 2].astype(np.float64))
+
+
+def test_copy_blocks_copies_whole_blocks_from_a_snapshot():
+    rng = RNG(18)
+    kp, vp = _rand(rng, (8, 4, 2, 8), F32), _rand(rng, (8, 4, 2, 8), F32)
+    k0, v0 = kp.copy(), vp.copy()
+    pairs = np.array([[1, 5], [5, 6], [2, 7]], dtype=np.int64)   # 5 is a src and a dst
+    oracle.copy_blocks(kp, vp, pairs, F32)
+    assert np.array_equal(kp[5], k0[1]) and np.array_equal(vp[5], v0[1])
+    assert np.array_equal(kp[6], k0[5]) and np.array_equal(vp[6], v0[5])   # old contents
+    assert np.array_equal(kp[7], k0[2])
+    for b in (0, 1, 2, 3, 4):
+        assert np.array_equal(kp[b], k0[b]) and np.array_equal(vp[b], v0[b])
+    with pytest.raises(oracle.OracleError):
+        oracle.copy_blocks(kp, vp, np.array([[0, 8]]), F32)
