@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode step: reshape_and_cache (+ copy_blocks when the
+step has copy-on-write pairs) + paged decode attention, on synthetic workloads.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|ID]
+                    [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch: the step's
+copy_blocks, then reshape_and_cache of the new tokens, then decode attention
+of every sequence's new query over its paged context (inputs resident in HBM).
+The default workload is the Llama-2-7B-shaped fp16 batch (64 sequences, 32
+heads x 128, contexts U[128, 2048], 16-token blocks, pool of 8192 blocks).
+
+Under torchrun (N > 1) every rank runs its own replica of the workload on its
+own GPU (weak scaling; the path has no exchange step, so there is no
+collective on the data path). Timing is on the device with CUDA events, max
+over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only other implementation
+there is) on a bounded sample of the same workload, on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_418_b200 import workloads as W  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "paged decode attention KV GB/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="llama2-7b-fp16")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=None)
+    return p.parse_args()
+
+
+def workload_id(x) -> int:
+    return int(x) if str(x).isdigit() else W.WORKLOAD_IDS[x]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def config_of(w: W.Workload, world: int, l2_note: str):
+    return {
+        "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.D,
+        "block_size": w.block_size, "num_blocks": w.num_blocks, "dtype": W.DTYPE_NAMES[w.dtype],
+        "context_lens": {"sum": int(w.context_lens.sum()), "mean": float(w.context_lens.mean()),
+                         "max": int(w.context_lens.max())},
+        "new_tokens": int(len(w.slot_mapping)), "cow_pairs": int(len(w.block_mapping)),
+        "partition_size": w.partition_size or "auto",
+        "kv_bytes_per_step": w.kv_bytes(), "seed": w.seed,
+        "parallelism": f"replicas x{world} (no collective on the data path)",
+        "l2": l2_note,
+    }
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_smi_id(local_rank: int) -> str:
+    """The id nvidia-smi knows this process's GPU by (UUID when torch exposes it)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(local_rank).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[local_rank].strip()
+        return str(local_rank)
+
+
+# ----------------------------------------------------------------------------
+# reference arm / CPU baseline: the fp64 oracle on a bounded sample
+# ----------------------------------------------------------------------------
+def oracle_sample_rows(w: W.Workload, budget_s: float, rng_seed: int = 0):
+    """Pick (b, hq) rows, longest-first interleaved with random, until the
+    estimated oracle time reaches the budget (calibrated on a few rows)."""
+    import oracle
+    rng = np.random.default_rng(rng_seed)
+    all_rows = np.array([(b, h) for b in range(w.B) for h in range(w.Hq)], dtype=np.int32)
+    order = rng.permutation(len(all_rows))
+    probe = all_rows[order[:8]]
+    t = time.perf_counter()
+    oracle.decode(w.q, w.k_cache, w.v_cache, w.dtype, w.block_tables, w.context_lens, w.scale,
+                  rows=probe)
+    dt = max(time.perf_counter() - t, 1e-4)
+    tok = float(w.context_lens[probe[:, 0]].sum())
+    per_token = dt / tok
+    budget_tokens = budget_s / per_token
+    chosen, acc = [], 0.0
+    for i in order:
+        if acc >= budget_tokens:
+            break
+        chosen.append(all_rows[i])
+        acc += float(w.context_lens[all_rows[i][0]])
+    return np.array(chosen, dtype=np.int32)
+
+
+def run_oracle(w: W.Workload, rows: np.ndarray, reps: int = 1):
+    """Time the oracle's share of a step: the step's cache ops on host pools and
+    decode of the sampled rows. Returns (seconds, kv_bytes_equivalent)."""
+    import oracle
+    kc, vc = w.k_cache, w.v_cache                       # in place; the step is idempotent
+    total = 0.0
+    for _ in range(reps):
+        t = time.perf_counter()
+        if len(w.block_mapping):
+            oracle.copy_blocks(kc, vc, w.block_mapping, w.dtype)
+        oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
+        oracle.decode(w.q, kc, vc, w.dtype, w.block_tables, w.context_lens, w.scale, rows=rows)
+        total += time.perf_counter() - t
+    frac = float(w.context_lens[rows[:, 0]].sum()) / (w.Hq * float(w.context_lens.sum()))
+    return total, w.kv_bytes() * frac * reps
+
+
+def reference_arm(args, w: W.Workload, rank: int, world: int):
+    if rank != 0:
+        return None
+    import oracle
+    cores = oracle.max_threads()
+    rows = oracle_sample_rows(w, budget_s=3.0)
+    for _ in range(max(0, min(args.warmup, 1))):
+        run_oracle(w, rows[:4])
+    secs, byts = run_oracle(w, rows, reps=args.steps)
+    value = byts / secs / 1e9
+    sample = (f"{len(rows)} of {w.B * w.Hq} (sequence, query head) rows per step "
+              f"({100.0 * len(rows) / (w.B * w.Hq):.1f}%), plus the step's full "
+              f"reshape_and_cache/copy_blocks; value scaled by the rows' share of KV bytes")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, 1, "host memory"),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def traffic_record(kernel_hash: str, w: W.Workload):
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    rec = d.get(w.name)
+    if not rec or rec.get("source_hash") != kernel_hash:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_418_b200 import _build, ops
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    t = W.to_torch(w, dev)
+    tdt = t["torch_dtype"]
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=tdt, device=dev)
+    ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len, w.partition_size)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    kernel, P, psize = ops.pa_decode_plan(w.dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
+                                          w.max_context_len, w.partition_size)
+    launches_per_step = (1 if len(w.block_mapping) else 0) + 1 + 1 + (1 if P > 1 else 0)
+    unique = w.unique_kv_bytes()
+    flush = unique < 2 * L2_BYTES
+    l2_note = ("L2 flushed before every step (workload smaller than 2x L2)" if flush else
+               f"inputs larger than L2 (KV {unique / 1e9:.2f} GB distinct > 126 MB)")
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
+
+    def step(ev=None):
+        if len(w.block_mapping):
+            ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err, stream)
+        ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                 t["slot_mapping"], err, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                      t["context_lens"], w.scale, w.max_context_len, w.partition_size, ws, err,
+                      stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())} during warm-up")
+
+    K = args.steps
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)] if flush else None
+    sampler = ClockSampler(gpu_smi_id(local_rank))
+    if rank == 0:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        if flush:
+            flush_buf.zero_()
+            step_ev[i][0].record(stream)
+        step(dec_ev[i])
+        if flush:
+            step_ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    if flush:
+        ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    else:
+        ms = t_start.elapsed_time(t_end)
+    dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / K
+    if world > 1:
+        tt = torch.tensor([ms, dec_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, dec_ms = float(tt[0]), float(tt[1])
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())} during timing")
+
+    # end to end through the public API: pinned host inputs -> device -> step -> host result
+    host = {k: v.cpu().pin_memory() for k, v in t.items()
+            if k in ("q", "new_key", "new_value", "slot_mapping", "block_tables",
+                     "context_lens", "block_mapping")}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out.numel() * out.element_size()
+    Ke = args.e2e_steps or max(1, min(K, 200))
+    for _ in range(2):
+        for k, v in host.items():
+            t[k].copy_(v, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_ms = 0.0
+    for i in range(Ke):
+        if flush:
+            flush_buf.zero_()
+        e0.record(stream)
+        for k, v in host.items():
+            t[k].copy_(v, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e_ms += e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt[0])
+    barrier()
+    if rank != 0:
+        return None
+
+    kv = w.kv_bytes()
+    value = kv * K * world / (ms / 1e3) / 1e9
+    peak, peak_src = peaks()
+    achieved = kv / (dec_ms / 1e3) / 1e9
+    kernel_hash = _build._hash()
+    traffic = traffic_record(kernel_hash, w)
+    e2e_value = kv * Ke * world / (e_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": W.DTYPE_NAMES[w.dtype], "data": "synthetic",
+        "config": config_of(w, world, l2_note),
+        "pct_of_hbm_peak": round(100.0 * (value / world) / peak, 2),
+        "seq_steps_per_s": round(w.B * K * world / (ms / 1e3), 1),
+        "decode_us": round(dec_ms * 1e3, 2),
+        "decode_plan": {"kernel": {1: "cuda-core", 2: "tcgen05"}[kernel], "partitions": P,
+                        "partition_tokens": psize},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_source": f"hbm_gbs ({peak_src})",
+                     "kernel": "pa_decode (partition pass + merge), per launch",
+                     "algorithmic_bytes": kv},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke},
+    }
+    return line
+
+
+def cpu_baseline(w: W.Workload):
+    import oracle
+    rows = oracle_sample_rows(w, budget_s=12.0)
+    secs, byts = run_oracle(w, rows, reps=1)
+    return {"value": round(byts / secs / 1e9, 4), "unit": "GB/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": (f"{len(rows)} of {w.B * w.Hq} (sequence, query head) rows "
+                       f"({100.0 * len(rows) / (w.B * w.Hq):.1f}%) of one step plus its cache "
+                       f"ops, {secs:.1f} s; scaled by the rows' share of KV bytes")}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    k = workload_id(args.workload)
+    seed = 1000 + k + 7919 * rank
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        w = W.make_workload(k, seed=seed)
+        line = reference_arm(args, w, rank, world)
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    w = W.make_workload(k, seed=seed)
+    try:
+        line = ours_arm(args, w, rank, world, local_rank)
+        if rank == 0 and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w)
+        elif rank == 0:
+            line["cpu_baseline"] = {"value": None, "unit": "GB/s", "cores": 0, "kind": "oracle",
+                                    "sample": "timed at N=1 only"}
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

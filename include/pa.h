@@ -1,0 +1,170 @@
+/*
+ * pa.h -- C ABI of libpa.so: paged KV-cache decode attention for NVIDIA B200
+ * (sm_100a), and the two kernels that keep the paged cache current.
+ *
+ * The problem, as the pages on PagedAttention state it: a pool of fixed-size
+ * physical KV blocks, shaped [num_blocks, block_size, ...] ("17. vLLM
+ * PagedAttention", Step 3: the physical block pool), and per sequence a block
+ * table mapping logical block i to a physical block id, not contiguous
+ * ("五十三：vLLM-PagedAttention" section 8; "vLLM 与 LLM 推理部署实战" section
+ * 2.1). The attention kernel finds each sequence's history through its block
+ * table and attends the current query to it ("17. vLLM PagedAttention",
+ * Step 2; "vLLM 与 LLM 推理部署实战" section 2.3).
+ *
+ * Conventions shared by every entry point
+ *  - All array arguments are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory. Arrays are dense, row-major, in the layouts
+ *    written beside each argument, and 16-byte aligned (element arrays).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream). The return value covers only what the host can see
+ *    before launching: a nonzero pa_status means nothing was launched.
+ *  - Errors that depend on device data (a block id or slot out of range, a
+ *    context length beyond the table) never fault and never trap: the
+ *    offending element is skipped and a bit is OR-ed into *err_flag (if
+ *    err_flag is not NULL). err_flag is a device uint32 the caller zeroes and
+ *    reads back when it wants to know.
+ *  - Element types: PA_F32, PA_F16 (IEEE binary16), PA_BF16. Pools, queries
+ *    and new K/V rows share one element type per call.
+ *  - Shapes: head size D in {64, 128}; block_size in {16, 32}; Hq a multiple
+ *    of Hkv with G = Hq / Hkv in {1, 2, 4, 8, 16}. Query head hq reads KV head
+ *    hq / G (contiguous groups; the pages do not say, this is the usual GQA
+ *    grouping).
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_NULL = 1,        /* a required pointer is NULL */
+  PA_ERR_SHAPE = 2,       /* a size is negative or inconsistent */
+  PA_ERR_DTYPE = 3,       /* unknown element type, or out_dtype not F32 / dtype */
+  PA_ERR_UNSUPPORTED = 4, /* D, block_size or G outside the supported set */
+  PA_ERR_WORKSPACE = 5,   /* workspace missing or smaller than pa_workspace_size() */
+  PA_ERR_CUDA = 6,        /* a CUDA call failed (launch error, no device, ...) */
+  PA_ERR_ALIGN = 7        /* an element array is not 16-byte aligned */
+} pa_status;
+
+/* Bits OR-ed into *err_flag by the kernels (never a trap). */
+#define PA_DEV_BAD_BLOCK_ID 1u /* a needed block-table entry is outside [0, num_blocks):
+                                  that block's tokens are left out of the softmax */
+#define PA_DEV_BAD_CTX 2u      /* context_lens[b] < 0, > max_blocks_per_seq * block_size or
+                                  > max_context_len: sequence b's output rows are zeros */
+#define PA_DEV_BAD_SLOT 4u     /* slot >= num_blocks * block_size: that token is not written */
+#define PA_DEV_BAD_PAIR 8u     /* src or dst outside [0, num_blocks): that pair is skipped */
+
+/*
+ * pa_workspace_size -- bytes of scratch pa_decode needs for these sizes.
+ *
+ * The split-context pass (used when contexts are long or the batch is too
+ * small to fill the GPU) writes, per (sequence, query head, partition), the
+ * partition's running max m, exp-sum l and unnormalised output (fp32), and a
+ * merge kernel combines them: M = max m_j, L = sum l_j e^(m_j - M),
+ * o = sum e^(m_j - M) o_j / L. This is not on the pages; it is the algebra of
+ * splitting one softmax sum. Returns 0 when pa_decode will not split.
+ * partition_size: 0 = let the library choose, else the partition length in
+ * tokens (a multiple of block_size, used as given). Same arguments as the
+ * pa_decode call it sizes; never fails (nonsense sizes give 0).
+ */
+size_t pa_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len,
+                         int partition_size);
+
+/*
+ * pa_decode -- one decode step of attention for B sequences, one new query
+ * token each, against their paged KV history.
+ *
+ *   out[b, hq, :] = sum_i softmax_i(scale * q[b,hq,:] . K_b[i]) V_b[i],  i < context_lens[b]
+ *   with K_b[i] = key_cache[block_tables[b, i / block_size], i % block_size, hq / G, :]
+ *   and  V_b[i] likewise from value_cache.
+ *
+ * out           [B, Hq, D] of out_dtype (PA_F32, or the same type as dtype);
+ *               written, rounded to nearest even from fp32.
+ * query         [B, Hq, D] of dtype.
+ * key_cache,
+ * value_cache   [num_blocks, block_size, Hkv, D] of dtype; read only.
+ * block_tables  [B, max_blocks_per_seq] int32; entries past
+ *               ceil(context_lens[b] / block_size) are never read.
+ * context_lens  [B] int32: tokens attended per sequence (0 gives a zero row).
+ * scale         softmax scale (usually 1/sqrt(D)).
+ * max_context_len  host-side upper bound of context_lens (no device read is
+ *               needed to size the launch); a larger length is an error bit.
+ * partition_size   0 = auto, else split into partitions of this many tokens.
+ * workspace     device scratch of at least pa_workspace_size(...) bytes, or
+ *               NULL when that size is 0. Overwritten; the caller owns it.
+ * err_flag      nullable device uint32, see PA_DEV_*.
+ * stream        cudaStream_t.
+ *
+ * Arithmetic: products and sums in fp32, online softmax with exp2, fp32
+ * accumulation; the GQA tensor-core path multiplies in the input type with
+ * fp32 accumulators (tcgen05, TMEM).
+ */
+int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache,
+              const void* value_cache, int dtype, const int32_t* block_tables,
+              int max_blocks_per_seq, const int32_t* context_lens, int B, int Hq, int Hkv,
+              int D, int block_size, int num_blocks, float scale, int max_context_len,
+              int partition_size, void* workspace, size_t workspace_bytes,
+              uint32_t* err_flag, void* stream);
+
+/*
+ * pa_reshape_and_cache -- write the K and V rows of T new tokens into the
+ * pool: key_cache[s / block_size, s % block_size, :, :] = key[t, :, :] with
+ * s = slot_mapping[t] (the same for value). A negative slot means "no
+ * token" (padding) and is skipped. This is the write the exercise page's
+ * allocate_for_decode prepares ("17. vLLM PagedAttention", Step 4: the new
+ * token goes into the sequence's current block, a new block when it is full).
+ *
+ * key, value    [T, Hkv, D] of dtype.
+ * key_cache,
+ * value_cache   [num_blocks, block_size, Hkv, D]; written in place.
+ * slot_mapping  [T] int64. Two tokens naming the same slot is a caller
+ *               error (which one lands is unspecified).
+ * Bit-exact copy; no arithmetic on the values.
+ */
+int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                         int dtype, const int64_t* slot_mapping, int T, int Hkv, int D,
+                         int block_size, int num_blocks, uint32_t* err_flag, void* stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write: for each pair p, copy the whole physical
+ * block block_mapping[p][0] (all block_size rows, all Hkv heads) to block
+ * block_mapping[p][1], in both pools. A write into a block that several
+ * sequences share first copies that block whole ("vLLM 与 LLM 推理部署实战"
+ * section 2.2; "五十三：vLLM-PagedAttention" sections 10 and 17).
+ *
+ * block_mapping [num_pairs, 2] int64 (src, dst). Destinations must be
+ *               distinct and must not appear as a source in the same call
+ *               (the block manager guarantees it: a fresh block is never
+ *               shared); otherwise the result is unspecified.
+ * Bit-exact copy.
+ */
+int pa_copy_blocks(void* key_cache, void* value_cache, int dtype, const int64_t* block_mapping,
+                   int num_pairs, int Hkv, int D, int block_size, int num_blocks,
+                   uint32_t* err_flag, void* stream);
+
+/* Static text for a pa_status value. */
+const char* pa_status_string(int status);
+
+/*
+ * pa_decode_plan -- what pa_decode will launch for these arguments, for
+ * tools and tests: *kernel = 1 (CUDA-core path) or 2 (tcgen05 GQA path),
+ * *num_partitions = partitions per sequence in the split pass (1 = no split),
+ * *partition_tokens = their length. Any pointer may be NULL. Returns a
+ * pa_status (PA_ERR_UNSUPPORTED etc. for the same reasons pa_decode would).
+ */
+int pa_decode_plan(int dtype, int B, int Hq, int Hkv, int D, int block_size,
+                   int max_context_len, int partition_size, int* kernel, int* num_partitions,
+                   int* partition_tokens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,314 @@
+// decode_simt.cu -- paged decode attention on the CUDA cores.
+//
+// One CTA = one (partition j, KV head h, chunk of GC query heads, sequence b).
+// Its four warps walk the partition's tokens in tiles; a tile is TILE rows of
+// one physical block (the whole block for 16-bit D=128, half of it for fp32
+// D=128). For every tile a warp
+//   1. reads the physical block id from the block table (prefetched one tile
+//      ahead, so the table read is off the critical path),
+//   2. issues all of the tile's K and V row loads at once: 16-byte vectors,
+//      LPR lanes per row, RPI rows per warp instruction, so each row is one
+//      fully used, contiguous 128 / 256-byte segment,
+//   3. forms the GC scores of each row as fp32 partial dots reduced over the
+//      row's LPR lanes with xor shuffles,
+//   4. applies the online-softmax update (running max m, running sum l,
+//      rescale by exp2(m_old - m_new)) and accumulates p * V in fp32.
+// Rows past the context length are never loaded and never enter the sums (a
+// select, not a multiply by zero, because unused slots may hold NaN).
+// At the end the four warps' (m, l, acc) are merged through shared memory.
+// A sequence whose context fits in one partition is written to the output
+// directly; otherwise the partition's (m, l, acc) go to the workspace and the
+// merge kernel combines them.
+//
+// The pages describe this kernel only as FlashAttention changed to read
+// non-contiguous blocks ("vLLM 与 LLM 推理部署实战", section 2.3) and list
+// block prefetch, shared-memory reuse and asynchronous copies as its
+// optimisations ("vLLM与PagedAttention：大模型推理内存优化技术解析", section
+// 3.2); the tiling and vector layout here are this library's own.
+#include <math_constants.h>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kWarps = 4;
+
+template <typename T, int D, int BS, int GC>
+__global__ void __launch_bounds__(kWarps * 32)
+decode_simt_kernel(const DecodeArgs a) {
+  constexpr int VEC = Vec<T>::N;               // elements per 16-byte vector
+  constexpr int LPR = D / VEC;                 // lanes per K/V row: 8, 16 or 32
+  constexpr int RPI = 32 / LPR;                // rows per warp instruction: 4, 2 or 1
+  constexpr int RG = (BS / RPI) < 8 ? (BS / RPI) : 8;   // row groups per tile
+  constexpr int TILE = RG * RPI;               // tokens per tile (divides BS)
+  static_assert(BS % TILE == 0, "tile must divide the block");
+
+  __shared__ float sm_acc[kWarps][GC][D];
+  __shared__ float sm_m[kWarps][GC];
+  __shared__ float sm_l[kWarps][GC];
+
+  const int G = a.Hq / a.Hkv;
+  const int chunks = G / GC;
+  const int j = blockIdx.x / chunks;
+  const int chunk = blockIdx.x - j * chunks;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int hq0 = h * G + chunk * GC;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int ctx = a.context_lens[b];
+  const bool bad_ctx = ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len;
+  const int tok_begin = j * a.psize;
+  if (bad_ctx || ctx == 0) {
+    // zero rows, written once (by partition 0); the merge kernel skips them
+    if (j == 0) {
+      if (bad_ctx && threadIdx.x == 0 && chunk == 0 && h == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
+      for (int i = threadIdx.x; i < GC * D; i += blockDim.x)
+        store_out(a.out, ((size_t)b * a.Hq + hq0 + i / D) * D + i % D, 0.f, a.out_dtype);
+    }
+    return;
+  }
+  if (tok_begin >= ctx) return;                 // partition past this sequence's end
+  const int tok_end = min(ctx, tok_begin + a.psize);
+  const int nparts = (ctx + a.psize - 1) / a.psize;
+
+  // query vectors of this chunk, pre-scaled so scores come out as scale*log2(e)*q.k
+  const int ci = lane % LPR;                    // which 16-byte vector of a row
+  const int rs = lane / LPR;                    // which row of an RPI-row group
+  float qf[GC][VEC];
+#pragma unroll
+  for (int g = 0; g < GC; ++g) {
+    uint4 raw = *reinterpret_cast<const uint4*>(
+        reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + hq0 + g) * D + ci * VEC);
+    widen16<T>(raw, qf[g]);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) qf[g][e] *= a.scale_log2;
+  }
+
+  float m[GC], l[GC], acc[GC][VEC];
+#pragma unroll
+  for (int g = 0; g < GC; ++g) {
+    m[g] = -CUDART_INF_F;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[g][e] = 0.f;
+  }
+
+  const int32_t* table = a.block_tables + (size_t)b * a.max_blocks;
+  const T* kc = reinterpret_cast<const T*>(a.k_cache);
+  const T* vc = reinterpret_cast<const T*>(a.v_cache);
+  const size_t row_stride = (size_t)a.Hkv * D;          // elements between token rows
+  const int tile_begin = tok_begin / TILE;
+  const int tile_end = (tok_end + TILE - 1) / TILE;
+
+  int t = tile_begin + warp;
+  int phys_next = t < tile_end ? __ldg(table + (t * TILE) / BS) : 0;
+  for (; t < tile_end; t += kWarps) {
+    const int phys = phys_next;
+    const int tn = t + kWarps;
+    if (tn < tile_end) phys_next = __ldg(table + (tn * TILE) / BS);
+    const int token0 = t * TILE;
+    if (phys < 0 || phys >= a.num_blocks) {
+      if (lane == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+      continue;
+    }
+    const size_t base =
+        ((size_t)phys * BS + (token0 % BS)) * row_stride + (size_t)h * D + ci * VEC;
+
+    uint4 kr[RG], vr[RG];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      const int row = r * RPI + rs;
+      if (token0 + row < tok_end) {
+        kr[r] = ld_stream16(kc + base + row * row_stride);
+        vr[r] = ld_stream16(vc + base + row * row_stride);
+      } else {
+        kr[r] = make_uint4(0, 0, 0, 0);
+        vr[r] = make_uint4(0, 0, 0, 0);
+      }
+    }
+
+    // scores of the lane's RG rows, reduced over the row's LPR lanes
+    float s[RG][GC];
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      float kf[VEC];
+      widen16<T>(kr[r], kf);
+#pragma unroll
+      for (int g = 0; g < GC; ++g) {
+        float d0 = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) d0 = fmaf(qf[g][e], kf[e], d0);
+        s[r][g] = d0;
+      }
+    }
+#pragma unroll
+    for (int o = LPR / 2; o >= 1; o >>= 1)
+#pragma unroll
+      for (int r = 0; r < RG; ++r)
+#pragma unroll
+        for (int g = 0; g < GC; ++g) s[r][g] += __shfl_xor_sync(0xffffffffu, s[r][g], o);
+
+    // online softmax over the tile (max over all TILE rows of the warp)
+#pragma unroll
+    for (int g = 0; g < GC; ++g) {
+      float tmax = -CUDART_INF_F;
+#pragma unroll
+      for (int r = 0; r < RG; ++r)
+        if (token0 + r * RPI + rs < tok_end) tmax = fmaxf(tmax, s[r][g]);
+#pragma unroll
+      for (int o = LPR; o < 32; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+      const float m_new = fmaxf(m[g], tmax);
+      const float alpha = exp2f(m[g] - m_new);
+      m[g] = m_new;
+      l[g] *= alpha;
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[g][e] *= alpha;
+#pragma unroll
+      for (int r = 0; r < RG; ++r) {
+        const bool valid = token0 + r * RPI + rs < tok_end;
+        s[r][g] = valid ? exp2f(s[r][g] - m_new) : 0.f;
+        l[g] += s[r][g];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < RG; ++r) {
+      float vf[VEC];
+      widen16<T>(vr[r], vf);
+#pragma unroll
+      for (int g = 0; g < GC; ++g)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[g][e] = fmaf(s[r][g], vf[e], acc[g][e]);
+    }
+  }
+
+  // combine the RPI row slots of the warp (same vector index, different rows)
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int g = 0; g < GC; ++g) {
+      l[g] += __shfl_xor_sync(0xffffffffu, l[g], o);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], o);
+    }
+  if (lane < LPR) {
+#pragma unroll
+    for (int g = 0; g < GC; ++g)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) sm_acc[warp][g][ci * VEC + e] = acc[g][e];
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < GC; ++g) { sm_m[warp][g] = m[g]; sm_l[warp][g] = l[g]; }
+  }
+  __syncthreads();
+
+  // merge the warps: M = max m_w, L = sum l_w 2^(m_w - M), O = sum acc_w 2^(m_w - M)
+  for (int i = threadIdx.x; i < GC * D; i += blockDim.x) {
+    const int g = i / D, d = i - g * D;
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][g]);
+    float L = 0.f, O = 0.f;
+    if (M != -CUDART_INF_F) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float c = exp2f(sm_m[w][g] - M);
+        L = fmaf(sm_l[w][g], c, L);
+        O = fmaf(sm_acc[w][g][d], c, O);
+      }
+    }
+    const size_t row = (size_t)b * a.Hq + hq0 + g;
+    if (nparts == 1) {
+      store_out(a.out, row * D + d, L > 0.f ? O / L : 0.f, a.out_dtype);
+    } else {
+      const size_t pj = row * a.P + j;
+      a.ws_acc[pj * D + d] = O;
+      if (d == 0) { a.ws_m[pj] = M; a.ws_l[pj] = L; }
+    }
+  }
+}
+
+template <typename T, int D, int BS, int GC>
+int launch_t(const DecodeArgs& a, cudaStream_t stream) {
+  const int chunks = (a.Hq / a.Hkv) / GC;
+  dim3 grid((unsigned)(a.P * chunks), (unsigned)a.Hkv, (unsigned)a.B);
+  decode_simt_kernel<T, D, BS, GC><<<grid, kWarps * 32, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D, int BS>
+int launch_gc(const DecodeArgs& a, cudaStream_t stream) {
+  const int G = a.Hq / a.Hkv;
+  if (G == 1) return launch_t<T, D, BS, 1>(a, stream);
+  if (G == 2) return launch_t<T, D, BS, 2>(a, stream);
+  return launch_t<T, D, BS, 4>(a, stream);      // G = 4, 8, 16: chunks of 4 heads
+}
+
+template <typename T, int D>
+int launch_bs(const DecodeArgs& a, cudaStream_t stream) {
+  return a.bs == 16 ? launch_gc<T, D, 16>(a, stream) : launch_gc<T, D, 32>(a, stream);
+}
+
+template <typename T>
+int launch_d(const DecodeArgs& a, cudaStream_t stream) {
+  return a.D == 64 ? launch_bs<T, 64>(a, stream) : launch_bs<T, 128>(a, stream);
+}
+
+// Merge of the split pass: one warp per (b, hq) row with more than one partition.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
+  constexpr int PER = D / 32;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= a.B * a.Hq) return;
+  const int b = row / a.Hq;
+  const int ctx = a.context_lens[b];
+  if (ctx <= 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len) return;
+  const int nparts = (ctx + a.psize - 1) / a.psize;
+  if (nparts <= 1) return;
+  const float* pm = a.ws_m + (size_t)row * a.P;
+  const float* pl = a.ws_l + (size_t)row * a.P;
+  float M = -CUDART_INF_F;
+  for (int jj = lane; jj < nparts; jj += 32) M = fmaxf(M, pm[jj]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f, O[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) O[e] = 0.f;
+  if (M != -CUDART_INF_F) {
+    for (int jj = 0; jj < nparts; ++jj) {
+      const float c = exp2f(pm[jj] - M);          // empty partitions: m = -inf, c = 0
+      L = fmaf(pl[jj], c, L);
+      const float* src = a.ws_acc + ((size_t)row * a.P + jj) * D + lane * PER;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) O[e] = fmaf(src[e], c, O[e]);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) store_out(a.out, (size_t)row * D + lane * PER + e, O[e] * inv, a.out_dtype);
+}
+
+}  // namespace
+
+int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream) {
+  switch (dtype) {
+    case PA_F32: return launch_d<float>(a, stream);
+    case PA_F16: return launch_d<__half>(a, stream);
+    case PA_BF16: return launch_d<__nv_bfloat16>(a, stream);
+  }
+  return PA_ERR_DTYPE;
+}
+
+int launch_merge(const DecodeArgs& a, cudaStream_t stream) {
+  const long long rows = (long long)a.B * a.Hq;
+  const unsigned blocks = (unsigned)((rows + 3) / 4);
+  if (a.D == 64) merge_kernel<64><<<blocks, 128, 0, stream>>>(a);
+  else merge_kernel<128><<<blocks, 128, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace pa

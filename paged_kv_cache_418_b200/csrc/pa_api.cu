@@ -1,0 +1,189 @@
+// pa_api.cu -- the extern "C" boundary of libpa.so: argument checks, launch
+// planning (split or not, which kernel), workspace carve-up, launches.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr int kDefaultPartition = 512;
+
+bool supported_shape(int Hq, int Hkv, int D, int bs) {
+  if (Hkv <= 0 || Hq <= 0 || Hq % Hkv) return false;
+  const int G = Hq / Hkv;
+  return (D == 64 || D == 128) && (bs == 16 || bs == 32) &&
+         (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
+}
+
+int esize_of(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Kernel override for A/B measurements: PA_DECODE_KERNEL=simt|tc (unset = auto).
+int kernel_override() {
+  const char* s = std::getenv("PA_DECODE_KERNEL");
+  if (!s) return 0;
+  if (!std::strcmp(s, "simt")) return 1;
+  if (!std::strcmp(s, "tc")) return 2;
+  return 0;
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max_ctx,
+                       int partition_size) {
+  DecodePlan p{1, 1, 0};
+  int psize = partition_size;
+  if (psize <= 0) {
+    // Auto: one pass when every context fits one default partition; else
+    // fixed partitions, so no CTA streams more than 512 tokens and the tail
+    // of a ragged batch stays short.
+    psize = kDefaultPartition;
+  }
+  const int mc = max_ctx > 0 ? max_ctx : 1;
+  p.P = (mc + psize - 1) / psize;
+  if (p.P <= 1) {
+    p.P = 1;
+    p.psize = ((mc + bs - 1) / bs) * bs;
+  } else {
+    p.psize = psize;
+  }
+  const int ov = kernel_override();
+  const bool tc = tc_supported(dtype, Hq, Hkv, D, bs);
+  p.kernel = ov == 1 ? 1 : (ov == 2 ? (tc ? 2 : 1) : (tc ? 2 : 1));
+  (void)B;
+  return p;
+}
+
+size_t workspace_bytes_for(int B, int Hq, int D, int P) {
+  if (P <= 1 || B <= 0) return 0;
+  const size_t rows = (size_t)B * Hq * P;
+  // acc [rows, D] then m [rows] then l [rows], each 256-byte aligned
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return up(rows * D * 4) + up(rows * 4) + up(rows * 4);
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+size_t pa_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len, int partition_size) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_context_len <= 0 || partition_size < 0)
+    return 0;
+  DecodePlan p = plan_decode(PA_F32, B, Hq, Hkv, D, 16, max_context_len, partition_size);
+  return workspace_bytes_for(B, Hq, D, p.P);
+}
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_NULL: return "a required pointer is NULL";
+    case PA_ERR_SHAPE: return "a size is negative or inconsistent";
+    case PA_ERR_DTYPE: return "unsupported element type or output type";
+    case PA_ERR_UNSUPPORTED: return "head size, block size or group size not supported";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_ALIGN: return "element array not 16-byte aligned";
+  }
+  return "unknown status";
+}
+
+int pa_decode_plan(int dtype, int B, int Hq, int Hkv, int D, int block_size, int max_context_len,
+                   int partition_size, int* kernel, int* num_partitions, int* partition_tokens) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (B < 0 || max_context_len < 0 || partition_size < 0) return PA_ERR_SHAPE;
+  if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (partition_size > 0 && partition_size % block_size) return PA_ERR_SHAPE;
+  DecodePlan p = plan_decode(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  if (kernel) *kernel = p.kernel;
+  if (num_partitions) *num_partitions = p.P;
+  if (partition_tokens) *partition_tokens = p.psize;
+  return PA_OK;
+}
+
+int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache,
+              const void* value_cache, int dtype, const int32_t* block_tables,
+              int max_blocks_per_seq, const int32_t* context_lens, int B, int Hq, int Hkv, int D,
+              int block_size, int num_blocks, float scale, int max_context_len,
+              int partition_size, void* workspace, size_t workspace_bytes, uint32_t* err_flag,
+              void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_DTYPE;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0 ||
+      max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+    return PA_ERR_SHAPE;
+  if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (partition_size > 0 && partition_size % block_size) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (B > 65535 || Hkv > 65535) return PA_ERR_UNSUPPORTED;
+  if (B == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
+    return PA_ERR_NULL;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_ALIGN;
+
+  DecodePlan p = plan_decode(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  DecodeArgs a{};
+  a.out = out; a.out_dtype = out_dtype; a.q = query;
+  a.k_cache = key_cache; a.v_cache = value_cache;
+  a.block_tables = block_tables; a.max_blocks = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.bs = block_size; a.num_blocks = num_blocks;
+  a.scale_log2 = scale * kLog2e;
+  a.max_context_len = max_context_len;
+  a.P = p.P; a.psize = p.psize;
+  a.err_flag = err_flag;
+  if (p.P > 1) {
+    const size_t need = workspace_bytes_for(B, Hq, D, p.P);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return PA_ERR_WORKSPACE;
+    const size_t rows = (size_t)B * Hq * p.P;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    char* w = static_cast<char*>(workspace);
+    a.ws_acc = reinterpret_cast<float*>(w);
+    a.ws_m = reinterpret_cast<float*>(w + up(rows * D * 4));
+    a.ws_l = reinterpret_cast<float*>(w + up(rows * D * 4) + up(rows * 4));
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, s) : launch_decode_simt(a, dtype, s);
+  if (rc == PA_OK && p.P > 1) rc = launch_merge(a, s);
+  return rc;
+}
+
+int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                         int dtype, const int64_t* slot_mapping, int T, int Hkv, int D,
+                         int block_size, int num_blocks, uint32_t* err_flag, void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (T < 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0) return PA_ERR_SHAPE;
+  if (!supported_shape(Hkv, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (T == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_ALIGN;
+  return launch_reshape_and_cache(key, value, key_cache, value_cache, esize_of(dtype),
+                                  slot_mapping, T, Hkv, D, block_size, num_blocks, err_flag,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+int pa_copy_blocks(void* key_cache, void* value_cache, int dtype, const int64_t* block_mapping,
+                   int num_pairs, int Hkv, int D, int block_size, int num_blocks,
+                   uint32_t* err_flag, void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (num_pairs < 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0)
+    return PA_ERR_SHAPE;
+  if (!supported_shape(Hkv, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!key_cache || !value_cache || !block_mapping) return PA_ERR_NULL;
+  if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_ALIGN;
+  return launch_copy_blocks(key_cache, value_cache, esize_of(dtype), block_mapping, num_pairs,
+                            Hkv, D, block_size, num_blocks, err_flag,
+                            static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// pa_common.cuh -- element types, 16-byte vector helpers and device error bits
+// shared by the libpa kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pa.h"
+
+namespace pa {
+
+constexpr int kSMs = 148;           // B200: 2 dies x 74 SMs
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Number of T elements in one 16-byte vector.
+template <typename T> struct Vec { static constexpr int N = 16 / sizeof(T); };
+
+// Widen the 16-byte vector `v` (N elements of T) to fp32.
+template <typename T> __device__ __forceinline__ void widen16(const uint4& v, float* f);
+
+template <> __device__ __forceinline__ void widen16<float>(const uint4& v, float* f) {
+  f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+  f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+}
+template <> __device__ __forceinline__ void widen16<__half>(const uint4& v, float* f) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __half22float2(h[i]);
+    f[2 * i] = t.x; f[2 * i + 1] = t.y;
+  }
+}
+template <> __device__ __forceinline__ void widen16<__nv_bfloat16>(const uint4& v, float* f) {
+  // bf16 -> fp32 is exact: the bf16 pattern is the top half of the fp32 one.
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Round fp32 to the output type (round to nearest even) and store.
+__device__ __forceinline__ void store_out(void* base, size_t i, float x, int out_dtype) {
+  if (out_dtype == PA_F32) reinterpret_cast<float*>(base)[i] = x;
+  else if (out_dtype == PA_F16) reinterpret_cast<__half*>(base)[i] = __float2half_rn(x);
+  else reinterpret_cast<__nv_bfloat16*>(base)[i] = __float2bfloat16_rn(x);
+}
+
+// Streaming 16-byte load of data read exactly once (K/V rows): keep L1 clean.
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void flag_error(uint32_t* err_flag, uint32_t bit) {
+  if (err_flag) atomicOr(err_flag, bit);
+}
+
+}  // namespace pa

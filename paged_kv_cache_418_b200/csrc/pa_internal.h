@@ -1,0 +1,56 @@
+// pa_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+// Everything a decode launch needs, resolved by the host layer.
+struct DecodeArgs {
+  void* out;
+  int out_dtype;
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;
+  int B, Hq, Hkv, D, bs, num_blocks;
+  float scale_log2;     // softmax scale * log2(e): scores live in the log2 domain
+  int max_context_len;
+  int P;                // partitions per sequence (grid extent); 1 = single pass
+  int psize;            // tokens per partition (a multiple of bs)
+  float* ws_acc;        // [B, Hq, P, D] unnormalised partial outputs (P > 1)
+  float* ws_m;          // [B, Hq, P] partial max, log2 domain
+  float* ws_l;          // [B, Hq, P] partial sum of exp2(s - m)
+  uint32_t* err_flag;
+};
+
+struct DecodePlan {
+  int kernel;           // 1 = CUDA-core path, 2 = tcgen05 GQA path
+  int P;
+  int psize;
+};
+
+// Host planning shared by pa_workspace_size, pa_decode_plan and pa_decode.
+DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max_ctx,
+                       int partition_size);
+size_t workspace_bytes_for(int B, int Hq, int D, int P);
+
+int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream);
+int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream);
+bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
+int launch_merge(const DecodeArgs& a, cudaStream_t stream);
+
+int launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                             void* value_cache, int esize, const int64_t* slot_mapping, int T,
+                             int Hkv, int D, int block_size, int num_blocks, uint32_t* err_flag,
+                             cudaStream_t stream);
+int launch_copy_blocks(void* key_cache, void* value_cache, int esize,
+                       const int64_t* block_mapping, int num_pairs, int Hkv, int D,
+                       int block_size, int num_blocks, uint32_t* err_flag, cudaStream_t stream);
+
+}  // namespace pa

@@ -1,0 +1,142 @@
+"""ctypes binding of libpa.so (the C ABI declared in include/pa.h).
+
+Argument marshalling only: every function here checks nothing the library does
+not check itself, reads the sizes off torch tensor shapes, passes raw device
+pointers and the current CUDA stream, and turns a nonzero status into
+``PAError``. All of the computing happens in the CUDA kernels. There is no
+fallback: if the library cannot be built or loaded, importing this module
+raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _build
+
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+PA_OK = 0
+PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_CTX, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR = 1, 2, 4, 8
+_TORCH_TO_PA = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+
+
+class PAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {pa_status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.ensure_built()
+    lib = ctypes.CDLL(path)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    IP = ctypes.POINTER(ctypes.c_int)
+    lib.pa_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.pa_workspace_size.restype = S
+    lib.pa_decode.argtypes = [P, I, P, P, P, I, P, I, P, I, I, I, I, I, I, F, I, I, P, S, P, P]
+    lib.pa_decode.restype = I
+    lib.pa_reshape_and_cache.argtypes = [P, P, P, P, I, P, I, I, I, I, I, P, P]
+    lib.pa_reshape_and_cache.restype = I
+    lib.pa_copy_blocks.argtypes = [P, P, I, P, I, I, I, I, I, P, P]
+    lib.pa_copy_blocks.restype = I
+    lib.pa_status_string.argtypes = [I]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_decode_plan.argtypes = [I, I, I, I, I, I, I, I, IP, IP, IP]
+    lib.pa_decode_plan.restype = I
+    return lib
+
+
+LIB = _load()
+LIB_PATH = _build.LIB
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def pa_dtype(t: torch.Tensor) -> int:
+    try:
+        return _TORCH_TO_PA[t.dtype]
+    except KeyError:
+        raise PAError("pa_dtype", 3) from None
+
+
+def pa_status_string(status: int) -> str:
+    return LIB.pa_status_string(int(status)).decode()
+
+
+def pa_workspace_size(B: int, Hq: int, Hkv: int, D: int, max_context_len: int,
+                      partition_size: int = 0) -> int:
+    return int(LIB.pa_workspace_size(B, Hq, Hkv, D, max_context_len, partition_size))
+
+
+def pa_decode_plan(dtype: int, B: int, Hq: int, Hkv: int, D: int, block_size: int,
+                   max_context_len: int, partition_size: int = 0) -> Tuple[int, int, int]:
+    k, p, t = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    rc = LIB.pa_decode_plan(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size,
+                            ctypes.byref(k), ctypes.byref(p), ctypes.byref(t))
+    if rc:
+        raise PAError("pa_decode_plan", rc)
+    return k.value, p.value, t.value
+
+
+def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+              value_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+              scale: float, max_context_len: int, partition_size: int = 0,
+              workspace: Optional[torch.Tensor] = None, err_flag: Optional[torch.Tensor] = None,
+              stream=None) -> None:
+    """out [B,Hq,D] <- paged decode attention (see pa_decode in include/pa.h)."""
+    B, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    rc = LIB.pa_decode(
+        _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+        B, Hq, Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
+        int(partition_size), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_decode", rc)
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                         value_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                         err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Scatter new K/V rows [T,Hkv,D] into the pools at slot_mapping [T] (int64)."""
+    num_blocks, block_size, Hkv, D = key_cache.shape
+    T = slot_mapping.shape[0]
+    rc = LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache),
+                                  pa_dtype(key_cache), _ptr(slot_mapping), T, Hkv, D,
+                                  block_size, num_blocks, _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_reshape_and_cache", rc)
+
+
+def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor,
+                   block_mapping: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                   stream=None) -> None:
+    """Copy whole blocks src -> dst for each (src, dst) row of block_mapping [P,2] (int64)."""
+    num_blocks, block_size, Hkv, D = key_cache.shape
+    P = block_mapping.shape[0]
+    rc = LIB.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), pa_dtype(key_cache),
+                            _ptr(block_mapping), P, Hkv, D, block_size, num_blocks,
+                            _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_copy_blocks", rc)
+
+
+def workspace_for(query: torch.Tensor, key_cache: torch.Tensor, max_context_len: int,
+                  partition_size: int = 0) -> Optional[torch.Tensor]:
+    """A device byte tensor big enough for pa_decode, or None when none is needed."""
+    B, Hq, D = query.shape
+    n = pa_workspace_size(B, Hq, key_cache.shape[2], D, max_context_len, partition_size)
+    return None if n == 0 else torch.empty(n, dtype=torch.uint8, device=query.device)
