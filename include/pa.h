@@ -60,6 +60,8 @@ typedef enum {
                                   > max_context_len: sequence b's output rows are zeros */
 #define PA_DEV_BAD_SLOT 4u     /* slot >= num_blocks * block_size: that token is not written */
 #define PA_DEV_BAD_PAIR 8u     /* src or dst outside [0, num_blocks): that pair is skipped */
+#define PA_DEV_TIMEOUT 16u     /* a pipeline wait inside the tensor-core decode kernel gave up
+                                  (bounded at 1 s): outputs of that launch are unspecified */
 
 /*
  * pa_workspace_size -- bytes of scratch pa_decode needs for these sizes.

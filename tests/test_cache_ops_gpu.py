@@ -90,7 +90,7 @@ def test_copy_blocks_bad_pair_is_flagged_and_skipped():
 
 
 def test_many_pairs_and_tokens():
-    """More pairs than a grid's y/z extent and a long token list."""
+    """More pairs than a grid's y/z extent (65535) would allow, and a long token list."""
     rng = np.random.default_rng(2)
     nb, bs, Hkv, D = 4096, 16, 1, 64
     kc = W.round_to_storage(rng.standard_normal((nb, bs, Hkv, D)).astype(np.float32), W.F16)
@@ -100,7 +100,7 @@ def test_many_pairs_and_tokens():
     dk, dv = torch.from_numpy(kc).cuda(), torch.from_numpy(vc).cuda()
     ops.pa_copy_blocks(dk, dv, torch.from_numpy(pairs).cuda())
     oracle.copy_blocks(kc, vc, pairs, W.F16)
-    T = 70000
+    T = 60000                                             # < num_blocks * bs slots
     key = W.round_to_storage(rng.standard_normal((T, Hkv, D)).astype(np.float32), W.F16)
     slots = rng.choice(nb * bs, size=T, replace=False).astype(np.int64)
     ops.pa_reshape_and_cache(torch.from_numpy(key).cuda(), torch.from_numpy(key).cuda(), dk, dv,
