@@ -53,6 +53,8 @@ def parse():
     p.add_argument("--workload", default="llama2-7b-fp16")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=None)
+    p.add_argument("--batch", type=int, default=None,
+                   help="fewer sequences of the same workload (profiling captures)")
     return p.parse_args()
 
 
@@ -415,7 +417,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        w = W.make_workload(k, seed=seed)
+        w = W.make_workload(k, seed=seed, batch=args.batch)
         line = reference_arm(args, w, rank, world)
         print(json.dumps(line), flush=True)
         return 0
@@ -426,7 +428,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                 device_id=torch.device("cuda", local_rank))
-    w = W.make_workload(k, seed=seed)
+    w = W.make_workload(k, seed=seed, batch=args.batch)
     try:
         line = ours_arm(args, w, rank, world, local_rank)
         if rank == 0 and world == 1:

@@ -332,11 +332,18 @@ WORKLOADS = {
 WORKLOAD_IDS = {v: k for k, v in WORKLOADS.items()}
 
 
-def make_workload(which, seed: Optional[int] = None) -> Workload:
-    """Build workload ``which`` (1..5 or its name); seed defaults to 1000 + id."""
+def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None) -> Workload:
+    """Build workload ``which`` (1..5 or its name); seed defaults to 1000 + id.
+
+    ``batch`` (profiling runs) keeps every distribution and shape but uses that
+    many sequences (groups of 16 for the shared-prefix workload) and a pool
+    scaled down with them.
+    """
     k = WORKLOAD_IDS[which] if isinstance(which, str) else int(which)
     seed = 1000 + k if seed is None else int(seed)
-    name = WORKLOADS[k]
+    name = WORKLOADS[k] if batch is None else f"{WORKLOADS[k]}-b{int(batch)}"
+    if batch is not None and k in (2, 3, 4, 5):
+        return _make_batch(k, name, seed, int(batch))
     if k == 1:
         return build_decode_case(name, F32, B=4, Hq=4, Hkv=4, D=64, block_size=16,
                                  num_blocks=64, context_lens=[1, 15, 16, 33], seed=seed,
@@ -364,6 +371,29 @@ def make_workload(which, seed: Optional[int] = None) -> Workload:
                                         block_size=16, num_blocks=8192, max_suffix=512,
                                         seed=seed)
     raise KeyError(which)
+
+
+def _make_batch(k: int, name: str, seed: int, B: int) -> Workload:
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if k == 2:
+        ctx = rng.integers(128, 2049, size=B)
+        return build_decode_case(name, F16, B=B, Hq=32, Hkv=32, D=128, block_size=16,
+                                 num_blocks=B * 128, context_lens=ctx, seed=seed, rng=rng,
+                                 max_blocks=128)
+    if k == 3:
+        ln = rng.lognormal(mean=math.log(1200.0), sigma=0.8, size=B)
+        ctx = np.clip(np.rint(ln), 16, 8192).astype(np.int64)
+        return build_decode_case(name, BF16, B=B, Hq=64, Hkv=8, D=128, block_size=16,
+                                 num_blocks=max(512, 2 * int(sum((c + 15) // 16 for c in ctx))),
+                                 context_lens=ctx, seed=seed, rng=rng, max_blocks=512)
+    if k == 4:
+        return build_decode_case(name, BF16, B=B, Hq=64, Hkv=8, D=128, block_size=32,
+                                 num_blocks=B * 2048, context_lens=[32768] * B, seed=seed,
+                                 rng=rng, max_blocks=1024, partition_size=512,
+                                 k_boost_frac=0.01)
+    return build_shared_prefix_case(name, BF16, groups=B, children=16, prefix_blocks=64,
+                                    Hq=32, Hkv=8, D=128, block_size=16,
+                                    num_blocks=max(1024, 512 * B), max_suffix=512, seed=seed)
 
 
 def shrink_workload(which, seed: int, B: Optional[int] = None, max_ctx: Optional[int] = None):
