@@ -151,6 +151,33 @@ int pa_copy_blocks(void* key_cache, void* value_cache, int dtype, const int64_t*
                    int num_pairs, int Hkv, int D, int block_size, int num_blocks,
                    uint32_t* err_flag, void* stream);
 
+/*
+ * pa_decode_static -- pa_decode without a workspace argument, for callers
+ * that cannot allocate device memory (a plugin inside an engine that owns all
+ * device memory, a program with a fixed device budget, a framework that
+ * forbids allocation inside its step). The pages have no counterpart: this
+ * entry point exists only for such callers.
+ *
+ * Same arguments, meaning and results as pa_decode, minus workspace and
+ * workspace_bytes. The scratch is a device array of PA_STATIC_SCRATCH_BYTES
+ * inside libpa.so: the library calls no allocator (no cudaMalloc, no cudaFree).
+ *  - Sizes whose pa_workspace_size(...) exceeds PA_STATIC_SCRATCH_BYTES are
+ *    rejected with PA_ERR_WORKSPACE before anything is launched.
+ *  - Every GPU that loads the array keeps those bytes until the process exits.
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address; make that first call before any stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero); calls that overlap on
+ *    the GPU race on it, so order them (one stream, or events).
+ * Returns a pa_status like pa_decode (PA_ERR_CUDA if the address lookup fails).
+ */
+#define PA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int pa_decode_static(void* out, int out_dtype, const void* query, const void* key_cache,
+                     const void* value_cache, int dtype, const int32_t* block_tables,
+                     int max_blocks_per_seq, const int32_t* context_lens, int B, int Hq, int Hkv,
+                     int D, int block_size, int num_blocks, float scale, int max_context_len,
+                     int partition_size, uint32_t* err_flag, void* stream);
+
 /* Static text for a pa_status value. */
 const char* pa_status_string(int status);
 

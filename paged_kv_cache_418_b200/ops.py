@@ -46,6 +46,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_decode_plan.argtypes = [I, I, I, I, I, I, I, I, IP, IP, IP]
     lib.pa_decode_plan.restype = I
+    lib.pa_decode_static.argtypes = [P, I, P, P, P, I, P, I, P, I, I, I, I, I, I, F, I, I, P, P]
+    lib.pa_decode_static.restype = I
     return lib
 
 
@@ -106,6 +108,28 @@ def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
         _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode", rc)
+
+
+PA_STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def pa_decode_static(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                     value_cache: torch.Tensor, block_tables: torch.Tensor,
+                     context_lens: torch.Tensor, scale: float, max_context_len: int,
+                     partition_size: int = 0, err_flag: Optional[torch.Tensor] = None,
+                     stream=None) -> None:
+    """pa_decode with the library's own device scratch instead of a workspace
+    argument, for callers that cannot allocate device memory (see pa_decode_static
+    in include/pa.h: one shared scratch per device, calls must not overlap)."""
+    B, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    rc = LIB.pa_decode_static(
+        _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+        B, Hq, Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
+        int(partition_size), _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_decode_static", rc)
 
 
 def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
