@@ -57,6 +57,8 @@ constexpr int kQBytes = 2 * kNS * 128;          // Q operand: 2 d-halves x 16 ro
 constexpr int kThreads = 192;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kTmemCols = 128;
+constexpr int kMaxUnits = 512;                  // work units one CTA can hold in its list
+constexpr int kScanChunk = 4096;                // sequences scanned per pass (stage 0 as scratch)
 
 template <int G> struct TcShape {
   static constexpr int NO = ((2 * G + 15) / 16) * 16;      // N of the PV MMA
@@ -67,9 +69,11 @@ template <int G> struct TcShape {
   static constexpr int NBAR = 2 * kStages + 15;
   static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;
   static constexpr int OFF_REDL = OFF_RED + 2 * 4 * 16 * 4;
-  static constexpr int OFF_MISC = OFF_REDL + 4 * 16 * 4;
-  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int OFF_REC = (OFF_REDL + 4 * 16 * 4 + 15) / 16 * 16;
+  static constexpr int OFF_MISC = OFF_REC + kMaxUnits * 16;
+  static constexpr int BYTES = OFF_MISC + 32;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
 };
 
 // barrier indices
@@ -208,33 +212,104 @@ template <int FMT> __device__ __forceinline__ void split_16(float p, uint16_t& h
 }
 
 // ---------------------------------------------------------------- work units
-struct Unit {
-  int b, h, j, ctx, t0, t1, ntiles;
-  bool work, zero, bad;
+// A unit is (sequence b, KV head h, partition j). Units exist only for
+// partitions that hold tokens; they are numbered sequence by sequence
+// (k = (units before b) * Hkv + j * Hkv + h) and CTA c takes k = c, c + grid,
+// ... Every CTA builds its own list at start, in shared memory, so the roles
+// never touch global memory to find their next unit.
+struct __align__(16) URec {
+  int b, h, j, ctx;
 };
 
-template <int BS>
-__device__ __forceinline__ Unit unit_of(const DecodeArgs& a, int u) {
+struct Unit {
+  int b, h, j, ctx, t0, t1, ntiles, nparts;
+};
+
+__device__ __forceinline__ Unit unit_from(const URec& r, int psize) {
   Unit x;
-  x.j = u % a.P;
-  const int bh = u / a.P;
-  x.h = bh % a.Hkv;
-  x.b = bh / a.Hkv;
-  x.ctx = a.context_lens[x.b];
-  x.bad = x.ctx < 0 || x.ctx > a.max_blocks * BS || x.ctx > a.max_context_len;
-  x.t0 = x.j * a.psize;
-  x.zero = (x.bad || x.ctx == 0) && x.j == 0;
-  x.work = !x.bad && x.t0 < x.ctx;
-  x.t1 = min(x.ctx, x.t0 + a.psize);
-  x.ntiles = x.work ? (x.t1 - x.t0 + kTile - 1) / kTile : 0;
+  x.b = r.b; x.h = r.h; x.j = r.j; x.ctx = r.ctx;
+  x.t0 = r.j * psize;
+  x.t1 = min(r.ctx, x.t0 + psize);
+  x.ntiles = (x.t1 - x.t0 + kTile - 1) / kTile;
+  x.nparts = (r.ctx + psize - 1) / psize;
   return x;
+}
+
+// Build this CTA's unit list (128 threads of warps 0-3). Sequences with no
+// tokens (or a context length the table cannot hold) get no units; their
+// output rows are zeroed here by the CTA that owns them.
+template <int BS>
+__device__ void build_unit_list(const DecodeArgs& a, uint8_t* scratch, URec* recs, int* carry_s,
+                                int* wsum, int* my_units) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int* np_s = reinterpret_cast<int*>(scratch);
+  int* ctx_s = np_s + kScanChunk;
+  constexpr int PER = kScanChunk / 128;
+  if (tid == 0) *carry_s = 0;
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  for (int b0 = 0; b0 < a.B; b0 += kScanChunk) {
+    const int n = min(kScanChunk, a.B - b0);
+    for (int i = tid; i < kScanChunk; i += 128) {
+      int np = 0, ctx = 0;
+      if (i < n) {
+        ctx = __ldg(a.context_lens + b0 + i);
+        const bool bad = ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len;
+        np = (bad || ctx == 0) ? 0 : (ctx + a.psize - 1) / a.psize;
+        if (bad && ((b0 + i) % (int)gridDim.x) == (int)blockIdx.x) flag_error(a.err_flag, PA_DEV_BAD_CTX);
+      }
+      np_s[i] = np;
+      ctx_s[i] = ctx;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int sum = 0;
+    for (int e = 0; e < PER; ++e) sum += np_s[tid * PER + e];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int wpre = 0;
+    for (int w = 0; w < warp; ++w) wpre += wsum[w];
+    const int base = *carry_s;
+    int pre = base + wpre + incl - sum;                 // partitions before my first sequence
+    for (int e = 0; e < PER; ++e) {
+      const int li = tid * PER + e, np = np_s[li];
+      if (np > 0) {
+        const long long start = (long long)pre * a.Hkv, end = start + (long long)np * a.Hkv;
+        long long k = start + (((long long)blockIdx.x - start % gridDim.x) + gridDim.x) % gridDim.x;
+        for (; k < end; k += gridDim.x) {
+          const int idx = (int)((k - blockIdx.x) / gridDim.x);
+          const int local = (int)(k - start);
+          if (idx < kMaxUnits) recs[idx] = URec{b0 + li, local % a.Hkv, local / a.Hkv, ctx_s[li]};
+        }
+      }
+      pre += np;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // zero the output rows of empty / bad sequences this CTA owns
+    for (int li = 0; li < n; ++li) {
+      const int b = b0 + li;
+      if (np_s[li] != 0 || (b % (int)gridDim.x) != (int)blockIdx.x) continue;
+      for (int i = tid; i < a.Hq * kD; i += 128)
+        store_out(a.out, (size_t)b * a.Hq * kD + i, 0.f, a.out_dtype);
+    }
+    if (tid == 127) *carry_s = pre;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
+  if (tid == 0) {
+    const long long U = (long long)(*carry_s) * a.Hkv;
+    const long long mine = U > blockIdx.x ? (U - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    *my_units = (int)(mine < kMaxUnits ? mine : kMaxUnits);
+  }
 }
 
 template <int FMT, int BS, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ,
-                 int total_units) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ) {
   using S = TcShape<G>;
   constexpr int NO = S::NO;
   constexpr uint32_t IDESC_S = make_idesc(FMT, 0, 0, kNS, 128);
@@ -249,8 +324,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   float* red = reinterpret_cast<float*>(smem + S::OFF_RED);     // [2][4][16]
   float* red_l = reinterpret_cast<float*>(smem + S::OFF_REDL);  // [4][16]
+  const URec* recs = reinterpret_cast<const URec*>(smem + S::OFF_REC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::OFF_MISC + 4);
+  int* my_units_s = reinterpret_cast<int*>(smem + S::OFF_MISC + 8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -271,9 +348,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     mbar_init(bar(B_DONE), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    fence_proxy_async();
   }
-  if (warp == 4) {
+  if (warp < 4) {
+    build_unit_list<BS>(a, smem, const_cast<URec*>(recs), reinterpret_cast<int*>(smem + S::OFF_MISC + 12),
+                        reinterpret_cast<int*>(smem + S::OFF_MISC + 16), my_units_s);
+    fence_proxy_async();                 // stage 0 served as scratch; TMA writes it next
+  } else if (warp == 4) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kTmemCols)
@@ -286,6 +366,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_s = tmem;                 // S buffers: columns [0,16) and [16,32)
   const uint32_t tmem_o = tmem + 2 * kNS;       // O buffers: [32, 32+NO) and [32+NO, 32+2NO)
+  const int nu = *my_units_s;
   auto give_up = [&]() {
     *abort_flag = 1u;
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
@@ -294,45 +375,52 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int tc = 0, uc = 0;
-      int issued = 0;                                   // stage loads issued so far
-      for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-        const Unit x = unit_of<BS>(a, u);
-        if (!x.work) continue;
-        const int qi = uc & 1;
-        if (!mbar_wait(bar(B_QEMPTY + qi), ((uc >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+      int tc = 0, issued = 0;
+      int phys_next[BPT];
+      // block ids of tile k of unit i, loaded one tile ahead of their use
+      auto load_ids = [&](int i, int k, int* ph) {
+        const Unit x = unit_from(recs[i], a.psize);
+        const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
+        const int nb = (te - ts + BS - 1) / BS;
+        const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks + ts / BS;
+#pragma unroll
+        for (int q = 0; q < BPT; ++q) ph[q] = q < nb ? __ldg(table + q) : -1;
+      };
+      if (nu > 0) load_ids(0, 0, phys_next);
+      for (int i = 0; i < nu; ++i) {
+        const Unit x = unit_from(recs[i], a.psize);
+        const int qi = i & 1;
+        if (!mbar_wait(bar(B_QEMPTY + qi), ((i >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
         mbar_expect_tx(bar(B_QFULL + qi), 2u * G * 128u);
         for (int hh = 0; hh < 2; ++hh)
           tma_load_2d(sbase + S::OFF_Q + qi * kQBytes + hh * (kNS * 128), &tmQ, hh * 64,
                       x.b * a.Hq + x.h * G, bar(B_QFULL + qi));
-        const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
         for (int k = 0; k < x.ntiles; ++k) {
-          const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
-          const int nb = (te - ts + BS - 1) / BS;
           int phys[BPT];
           uint32_t bytes = 0;
 #pragma unroll
-          for (int i = 0; i < BPT; ++i) {
-            phys[i] = i < nb ? __ldg(table + ts / BS + i) : -1;
-            if (phys[i] >= 0 && phys[i] < a.num_blocks) bytes += 2u * BS * 128u;
+          for (int q = 0; q < BPT; ++q) {
+            phys[q] = phys_next[q];
+            if (phys[q] >= 0 && phys[q] < a.num_blocks) bytes += 2u * BS * 128u;
           }
+          if (k + 1 < x.ntiles) load_ids(i, k + 1, phys_next);
+          else if (i + 1 < nu) load_ids(i + 1, 0, phys_next);
           for (int kv = 0; kv < 2; ++kv) {
             const int seq = 2 * tc + kv, s = seq % kStages;
             if (!mbar_wait(bar(B_EMPTY + s), ((seq / kStages) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
             mbar_expect_tx(bar(B_FULL + s), bytes);
             const uint32_t dst = sbase + s * kStageBytes;
 #pragma unroll
-            for (int i = 0; i < BPT; ++i) {
-              if (phys[i] < 0 || phys[i] >= a.num_blocks) continue;
+            for (int q = 0; q < BPT; ++q) {
+              if (phys[q] < 0 || phys[q] >= a.num_blocks) continue;
               for (int hh = 0; hh < 2; ++hh)
-                tma_load_4d(dst + hh * kHalf + i * BS * 128, kv ? &tmV : &tmK, hh * 64, x.h, 0,
-                            phys[i], bar(B_FULL + s));
+                tma_load_4d(dst + hh * kHalf + q * BS * 128, kv ? &tmV : &tmK, hh * 64, x.h, 0,
+                            phys[q], bar(B_FULL + s));
             }
             ++issued;
           }
           ++tc;
         }
-        ++uc;
       }
     prod_done:
       // never leave with copies in flight: wait (bounded) for the last loads of every stage
@@ -345,7 +433,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int tc = 0, uc = 0;
+      int tc = 0;
       bool ok = true;
       auto issue_pv = [&](int tt, int nb) -> bool {
         const int pb = tt & 1;
@@ -368,11 +456,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         mma_commit(bar(B_OFULL + pb));
         return true;
       };
-      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const Unit x = unit_of<BS>(a, u);
-        if (!x.work) continue;
-        const int qi = uc & 1;
-        if (!mbar_wait(bar(B_QFULL + qi), (uc >> 1) & 1, abort_flag)) { ok = false; break; }
+      for (int i = 0; i < nu && ok; ++i) {
+        const Unit x = unit_from(recs[i], a.psize);
+        const int qi = i & 1;
+        if (!mbar_wait(bar(B_QFULL + qi), (i >> 1) & 1, abort_flag)) { ok = false; break; }
         const uint32_t qst = sbase + S::OFF_Q + qi * kQBytes;
         int prev_nb = 0;
         for (int k = 0; k < x.ntiles; ++k) {
@@ -398,7 +485,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         }
         if (!ok) break;
         if (!issue_pv(tc - 1, prev_nb)) { ok = false; break; }
-        ++uc;
       }
       if (!ok) give_up();
       // all issued MMAs must finish before tensor memory is released
@@ -412,16 +498,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     int tc = 0;
     bool failed = false;
-    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-      const Unit x = unit_of<BS>(a, u);
-      if (x.zero) {
-        if (x.bad && x.h == 0 && row == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-          store_out(a.out, ((size_t)x.b * a.Hq + x.h * G + g) * kD + row, 0.f, a.out_dtype);
-      }
-      if (!x.work) continue;
-      const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
+    // this thread's block id for tile k of unit i (its token row), one tile ahead
+    auto row_id = [&](int i, int k) -> int {
+      const Unit x = unit_from(recs[i], a.psize);
+      const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
+      const int nb = (te - ts + BS - 1) / BS;
+      return row < nb * BS ? __ldg(a.block_tables + (size_t)x.b * a.max_blocks + ts / BS + row / BS)
+                           : -1;
+    };
+    int phys_next = nu > 0 ? row_id(0, 0) : -1;
+    for (int i = 0; i < nu; ++i) {
+      const Unit x = unit_from(recs[i], a.psize);
       float m[G], l[G], O[G], al_prev[G], al[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -444,7 +531,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
         const int nb = (te - ts + BS - 1) / BS;
         const bool in_range = row < nb * BS;
-        const int phys = in_range ? __ldg(table + ts / BS + row / BS) : -1;
+        const int phys = phys_next;
+        if (k + 1 < x.ntiles) phys_next = row_id(i, k + 1);
+        else if (i + 1 < nu) phys_next = row_id(i + 1, 0);
         const bool blk_ok = phys >= 0 && phys < a.num_blocks;
         const bool valid = in_range && blk_ok && ts + row < te;
         if (in_range && !blk_ok && (row % BS) == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
@@ -511,12 +600,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         if (lane == 0) red_l[warp * 16 + g] = v;
       }
       if (wg_vote_or(failed)) break;
-      const int nparts = (x.ctx + a.psize - 1) / a.psize;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float L = red_l[g] + red_l[16 + g] + red_l[32 + g] + red_l[48 + g];
         const size_t orow = (size_t)x.b * a.Hq + x.h * G + g;
-        if (nparts == 1) {
+        if (x.nparts == 1) {
           store_out(a.out, orow * kD + row, L > 0.f ? O[g] / L : 0.f, a.out_dtype);
         } else {
           const size_t pj = orow * a.P + x.j;
@@ -600,11 +688,13 @@ int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
       return PA_ERR_CUDA;
     attr = true;
   }
+  // Units that hold tokens number at most B * Hkv * P; a CTA's list holds kMaxUnits.
   const long long units = (long long)a.B * a.Hkv * a.P;
   if (units <= 0) return PA_OK;
-  if (units > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-  const int grid = (int)(units < sm_count() ? units : sm_count());
-  kern<<<grid, kThreads, smem, stream>>>(a, k, v, q, (int)units);
+  long long grid = units < sm_count() ? units : sm_count();
+  if ((units + grid - 1) / grid > kMaxUnits) grid = (units + kMaxUnits - 1) / kMaxUnits;
+  if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  kern<<<(unsigned)grid, kThreads, smem, stream>>>(a, k, v, q);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
