@@ -224,13 +224,30 @@ def reference_arm(args, w: W.Workload, rank: int, world: int):
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
-def traffic_record(kernel_hash: str, w: W.Workload):
+KERNEL_SOURCES = {
+    "cuda-core": ["decode_simt.cu"],
+    "tcgen05": ["decode_tc.cu", "decode_simt.cu"],      # the merge kernel lives in decode_simt.cu
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources a decode path is built from (its kernels + shared headers)."""
+    csrc = os.path.join(ROOT, "paged_kv_cache_418_b200", "csrc")
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel] + ["pa_common.cuh", "pa_internal.h"]:
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    h.update(open(os.path.join(ROOT, "include", "pa.h"), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, w: W.Workload):
+    """DRAM bytes per pa_decode launch from a committed ncu summary, or None when
+    there is none for this workload or the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path))
-    rec = d.get(w.name)
-    if not rec or rec.get("source_hash") != kernel_hash:
+    rec = json.load(open(path)).get(w.name)
+    if not rec or rec.get("kernel") != kernel or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -356,8 +373,8 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     value = kv * K * world / (ms / 1e3) / 1e9
     peak, peak_src = peaks()
     achieved = kv / (dec_ms / 1e3) / 1e9
-    kernel_hash = _build._hash()
-    traffic = traffic_record(kernel_hash, w)
+    kname = {1: "cuda-core", 2: "tcgen05"}[kernel]
+    traffic = traffic_record(kname, w)
     e2e_value = kv * Ke * world / (e_ms / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
