@@ -1,42 +1,50 @@
 // decode_tc.cu -- grouped-query paged decode attention on the 5th-generation
 // tensor cores (tcgen05, accumulators in tensor memory), for 16-bit K/V with
-// head size 128 and G = Hq / Hkv in {4, 8, 16} query heads per KV head.
+// head size 128, G = Hq / Hkv in {4, 8, 16} query heads per KV head, and KV
+// heads in groups of HG = 4.
 //
 // Why tensor cores here: the G query heads that share a KV head turn the
-// per-token work into a small dense contraction (G x 128 against 128-token
-// tiles). On the CUDA cores that is ~4 FMAs per byte of K/V at G = 8, close to
-// the FP32 pipe's limit at HBM speed; on tcgen05 it is a few MMAs per tile.
+// per-token work into a small dense contraction. On the CUDA cores that is ~4
+// FMAs per byte of K/V at G = 8, close to the FP32 pipe's limit at HBM speed;
+// on tcgen05 it is a few MMAs per tile.
 //
-// Shapes (swap-AB, so the 128-token tile fills the MMA's M = 128):
-//   scores  S^T[128 tok x 16]  = K_tile[128 tok x 128 d] . Q^T      (Q rows padded to 16)
-//   output  O^T[128 d x NO]   += V_tile^T[128 d x 128 tok] . P^T     (P = [P_hi; P_lo])
-// P is split into two 16-bit parts, p = hi + lo with hi = RN(p), lo = RN(p - hi),
-// stacked as 2G rows of the B operand, so the products keep ~16 significant
-// bits of the softmax weights instead of 8 (bf16); the two column groups of O
-// are summed in fp32 afterwards. K/V products are exact and accumulate in fp32.
+// Work unit = (sequence, partition of the context, group of HG KV heads).
+// Tile = 128 rows of K (or V): HG heads x Rt = 128 / HG tokens, taken from
+// whole physical blocks. A 5-D TMA tensor map views the pool as
+// [num_blocks][2 d-halves][Hkv][block_size][64 d] (strides of the real
+// [num_blocks, block_size, Hkv, D] layout), so one TMA box brings Rb token
+// rows of all HG heads for one 64-wide d-half: 8-16 KB per instruction, in the
+// canonical 128-byte-swizzled layout the MMA reads (rows = (head, token),
+// 128 B each; the two d-halves 16 KB apart). Bigger boxes matter: streaming
+// the same bytes as 2-4 KB per-head boxes is limited by TMA issue, not HBM.
 //
-// Data movement: a 4-D TMA tensor map over the pool [num_blocks, bs, Hkv, D]
-// loads, for one physical block and one KV head, bs rows x 64 d (128 bytes)
-// with 128-byte swizzling, which is exactly the canonical SW128 K-major
-// layout the MMA reads for K, and the MN-major layout it reads for V^T. One
-// tile = 128 / bs such block loads per d-half, written side by side.
+// Per tile (swap-AB, rows of the tile on the MMA's M = 128):
+//   scores  S^T[128 x HG*G]   = K_tile . Q_grp^T         (all query heads of the group)
+//   output  O^T_h[128 d x 2G] += V_h^T . [P_hi; P_lo]_h^T  one MMA per head and 16 tokens
+// Each row (head h, token) keeps only its own head's G scores. The softmax
+// weights enter the output product as two 16-bit parts, p = hi + lo with
+// hi = RN(p), lo = RN(p - hi), so the products keep ~16 significant bits
+// instead of 8 (bf16); O accumulates in fp32 in TMEM for the whole unit.
+// The online softmax rescales O lazily: a query head's reference max moves
+// only when a tile's max exceeds it by more than 2^64 (weights up to 2^64 are
+// far from fp32 overflow in l and O, and relative precision does not depend
+// on scale), which after the first tile is rare; then the affected TMEM
+// columns are read, scaled and written back. Exact in real arithmetic: O and
+// l always share the same reference.
 //
-// CTA = 6 warps, persistent over work units (sequence, KV head, partition):
-//   warps 0-3  softmax + output: read S from TMEM (one token row per thread),
-//              online softmax over the tile (running max per head), write
-//              P_hi/P_lo to shared memory, then fold the tile's O (one d row
-//              per thread) into fp32 registers with the rescale factor;
-//   warp 4     TMA producer (one lane): Q of the unit, then K and V tiles
-//              through a 6-stage ring (192 KB in flight per SM);
-//   warp 5     MMA issuer (one lane): S(t), then O(t-1), committing each to
-//              mbarriers that release ring stages and hand results over.
-// S and O each have two TMEM buffers and P two shared buffers, so the softmax
-// of tile t overlaps the PV product of tile t-1 and the loads of later tiles.
-//
+// CTA = 10 warps, persistent over its list of units:
+//   warps 0-7  two softmax groups; group w takes tiles t with t % 2 == w, so
+//              every SM sub-partition runs two independent softmax warps; at
+//              the end of a unit the group that did not take its last tile
+//              hands its reference maxima and exp-sums to the other (mbarrier
+//              hand-off), which merges both TMEM accumulators and writes;
+//   warp 8     TMA producer (one lane): Q of the unit, K and V tiles through a
+//              ring of 32 KB stages;
+//   warp 9     MMA issuer (one lane): S(t), then O(t-1).
 // Every pipeline wait is bounded (1 s); a wait that gives up sets the
 // PA_DEV_TIMEOUT bit, raises a CTA-wide abort flag, and all roles leave their
-// loops (the softmax warps only together, at a named-barrier vote), wait for
-// their own asynchronous work, free tensor memory and return.
+// loops (the softmax warps of a group only together, at a named-barrier vote),
+// wait for their own asynchronous work, free tensor memory and return.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -48,38 +56,50 @@ namespace pa {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kTile = 128;                      // tokens per tile
-constexpr int kHalf = kTile * 128;              // bytes of one 64-wide d-half of a tile
+constexpr int kRows = 128;                      // rows per tile (the MMA's M)
+constexpr int kHalf = kRows * 128;              // bytes of one 64-wide d-half of a tile
 constexpr int kStageBytes = 2 * kHalf;          // one K or V tile: 32 KB
-constexpr int kStages = 6;
-constexpr int kNS = 16;                         // N of the score MMA
-constexpr int kQBytes = 2 * kNS * 128;          // Q operand: 2 d-halves x 16 rows x 128 B
-constexpr int kThreads = 192;
+constexpr int kHG = 4;                          // KV heads per unit
+constexpr int kRt = kRows / kHG;                // tokens per head per tile (32)
+constexpr int kThreads = 320;
 constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr int kTmemCols = 128;
-constexpr int kMaxUnits = 512;                  // work units one CTA can hold in its list
+constexpr int kMaxUnits = 320;                  // work units one CTA can hold in its list
 constexpr int kScanChunk = 4096;                // sequences scanned per pass (stage 0 as scratch)
+constexpr float kRescaleLog2 = 64.f;            // lazy rescale threshold (log2 units): p <= 2^64,
+                                                // far from fp32 overflow in l and O
 
 template <int G> struct TcShape {
-  static constexpr int NO = ((2 * G + 15) / 16) * 16;      // N of the PV MMA
-  static constexpr int kPBytes = NO * 2 * 128;               // per tile: 2 token-halves
+  static constexpr int NS = kHG * G;                         // N of the score MMA
+  static constexpr int NOH = ((2 * G + 15) / 16) * 16;       // N of a head's output MMA
+  static constexpr int NO = kHG * NOH;                       // output columns per group
+  static constexpr int kStages = G <= 8 ? 6 : 5;
+  static constexpr int kTmemCols = 2 * NS + 2 * NO <= 256 ? 256 : 512;
+  static constexpr int kQBytes = 2 * NS * 128;               // Q operand: 2 d-halves x NS rows
+  static constexpr int kPBytes = 2 * NOH * 128;              // P operand of one tile: 2 lines
   static constexpr int OFF_Q = kStages * kStageBytes;
   static constexpr int OFF_P = OFF_Q + 2 * kQBytes;
-  static constexpr int OFF_BAR = OFF_P + 2 * kPBytes;
-  static constexpr int NBAR = 2 * kStages + 15;
-  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;
-  static constexpr int OFF_REDL = OFF_RED + 2 * 4 * 16 * 4;
-  static constexpr int OFF_REC = (OFF_REDL + 4 * 16 * 4 + 15) / 16 * 16;
+  static constexpr int OFF_X = OFF_P + 2 * kPBytes;          // [2][2][NS] reference max, exp-sum
+  static constexpr int OFF_BAR = OFF_X + 2 * 2 * NS * 4 + 16;
+  static constexpr int NBAR = 2 * kStages + 19;
+  static constexpr int GP = G < 8 ? 8 : G;                  // per-chunk stride of the reductions
+  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;         // [group][2][8 chunks][GP] maxima
+  static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
+  static constexpr int OFF_MREF = OFF_REDL + 2 * 2 * 8 * GP * 4;  // [group][3][NS] references
+  static constexpr int OFF_REC = (OFF_MREF + 2 * 3 * NS * 4 + 15) / 16 * 16;
   static constexpr int OFF_MISC = OFF_REC + kMaxUnits * 16;
   static constexpr int BYTES = OFF_MISC + 32;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(2 * NS + 2 * NO <= 512, "tensor memory columns");
 };
 
-// barrier indices
-constexpr int B_FULL = 0, B_EMPTY = kStages, B_QFULL = 2 * kStages, B_QEMPTY = B_QFULL + 2,
-              B_SFULL = B_QEMPTY + 2, B_SFREE = B_SFULL + 2, B_PREADY = B_SFREE + 2,
-              B_OFULL = B_PREADY + 2, B_OFREE = B_OFULL + 2, B_DONE = B_OFREE + 2;
+// barrier indices (the ring's full/empty pairs come first)
+template <int NST> struct Bars {
+  static constexpr int FULL = 0, EMPTY = NST, QFULL = 2 * NST, QEMPTY = QFULL + 2,
+                       SFULL = QEMPTY + 2, SFREE = SFULL + 2, PREADY = SFREE + 2,
+                       OFULL = PREADY + 2, XFULL = OFULL + 2, XFREE = XFULL + 2,
+                       ODONE = XFREE + 2, DONE = ODONE + 1;
+};
 
 // ---------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -131,12 +151,12 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, uint32_t bar) {
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, int c4, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
@@ -185,14 +205,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-// Vote over the 128 softmax threads (named barrier 1): OR of every thread's flag.
-__device__ __forceinline__ bool wg_vote_or(bool x) {
+// Vote over the 128 threads of one softmax group (named barrier 1 + group):
+// OR of every thread's flag; also a barrier for the group's shared memory.
+__device__ __forceinline__ bool wg_vote_or(bool x, int group) {
   uint32_t r;
   asm volatile(
-      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, 1, 128, pi;"
+      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, %2, 128, pi;"
       " selp.u32 %0, 1, 0, po; }"
       : "=r"(r)
-      : "r"((uint32_t)x)
+      : "r"((uint32_t)x), "r"(1 + group)
       : "memory");
   return r != 0;
 }
@@ -211,10 +232,29 @@ template <int FMT> __device__ __forceinline__ void split_16(float p, uint16_t& h
   }
 }
 
+// Store 16 consecutive fp32 columns of this thread's TMEM lane; waits for the store.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
+  __syncwarp();
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      "\n\ttcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15]))
+      : "memory");
+}
+// Plain named-barrier sync of one softmax group.
+__device__ __forceinline__ void wg_sync(int group) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + group) : "memory");
+}
+
 // ---------------------------------------------------------------- work units
-// A unit is (sequence b, KV head h, partition j). Units exist only for
-// partitions that hold tokens; they are numbered sequence by sequence
-// (k = (units before b) * Hkv + j * Hkv + h) and CTA c takes k = c, c + grid,
+// A unit is (sequence b, partition j, group h of kHG KV heads). Units exist
+// only for partitions that hold tokens; they are numbered sequence by sequence
+// (k = (partitions before b) * NHG + j * NHG + h, NHG = Hkv / kHG) and CTA c takes k = c, c + grid,
 // ... Every CTA builds its own list at start, in shared memory, so the roles
 // never touch global memory to find their next unit.
 struct __align__(16) URec {
@@ -230,7 +270,7 @@ __device__ __forceinline__ Unit unit_from(const URec& r, int psize) {
   x.b = r.b; x.h = r.h; x.j = r.j; x.ctx = r.ctx;
   x.t0 = r.j * psize;
   x.t1 = min(r.ctx, x.t0 + psize);
-  x.ntiles = (x.t1 - x.t0 + kTile - 1) / kTile;
+  x.ntiles = (x.t1 - x.t0 + kRt - 1) / kRt;
   x.nparts = (r.ctx + psize - 1) / psize;
   return x;
 }
@@ -239,8 +279,8 @@ __device__ __forceinline__ Unit unit_from(const URec& r, int psize) {
 // tokens (or a context length the table cannot hold) get no units; their
 // output rows are zeroed here by the CTA that owns them.
 template <int BS>
-__device__ void build_unit_list(const DecodeArgs& a, uint8_t* scratch, URec* recs, int* carry_s,
-                                int* wsum, int* my_units) {
+__device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, URec* recs,
+                                int* carry_s, int* wsum, int* my_units) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int* np_s = reinterpret_cast<int*>(scratch);
   int* ctx_s = np_s + kScanChunk;
@@ -278,12 +318,12 @@ __device__ void build_unit_list(const DecodeArgs& a, uint8_t* scratch, URec* rec
     for (int e = 0; e < PER; ++e) {
       const int li = tid * PER + e, np = np_s[li];
       if (np > 0) {
-        const long long start = (long long)pre * a.Hkv, end = start + (long long)np * a.Hkv;
+        const long long start = (long long)pre * nhg, end = start + (long long)np * nhg;
         long long k = start + (((long long)blockIdx.x - start % gridDim.x) + gridDim.x) % gridDim.x;
         for (; k < end; k += gridDim.x) {
           const int idx = (int)((k - blockIdx.x) / gridDim.x);
           const int local = (int)(k - start);
-          if (idx < kMaxUnits) recs[idx] = URec{b0 + li, local % a.Hkv, local / a.Hkv, ctx_s[li]};
+          if (idx < kMaxUnits) recs[idx] = URec{b0 + li, local % nhg, local / nhg, ctx_s[li]};
         }
       }
       pre += np;
@@ -300,21 +340,35 @@ __device__ void build_unit_list(const DecodeArgs& a, uint8_t* scratch, URec* rec
     asm volatile("bar.sync 1, 128;" ::: "memory");
   }
   if (tid == 0) {
-    const long long U = (long long)(*carry_s) * a.Hkv;
+    const long long U = (long long)(*carry_s) * nhg;
     const long long mine = U > blockIdx.x ? (U - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     *my_units = (int)(mine < kMaxUnits ? mine : kMaxUnits);
   }
 }
+
+// Advance (i, k) to the next tile of the CTA's unit list (i == nu: past the end).
+__device__ __forceinline__ void next_tile(const URec* recs, int nu, int psize, int& i, int& k) {
+  if (i >= nu) return;
+  const Unit x = unit_from(recs[i], psize);
+  if (++k >= x.ntiles) { k = 0; ++i; }
+}
+
 
 template <int FMT, int BS, int G>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ) {
   using S = TcShape<G>;
-  constexpr int NO = S::NO;
-  constexpr uint32_t IDESC_S = make_idesc(FMT, 0, 0, kNS, 128);
-  constexpr uint32_t IDESC_O = make_idesc(FMT, 1, 0, NO, 128);
-  constexpr int BPT = kTile / BS;                       // physical blocks per tile
+  constexpr int NST = S::kStages;
+  using Bx = Bars<NST>;
+  constexpr int NS = S::NS, NOH = S::NOH, NO = S::NO;
+  constexpr int RB = BS < kRt ? BS : kRt;        // token rows per TMA box (per head)
+  constexpr int NQ = kRt / RB;                   // boxes per d-half per tile
+  constexpr int KS = kRt / 16;                   // output-MMA K steps per head per tile
+  constexpr int NCH = NQ * kHG;                  // (box, head) row chunks per tile
+  constexpr uint32_t IDESC_S = make_idesc(FMT, 0, 0, NS, 128);
+  constexpr uint32_t IDESC_O = make_idesc(FMT, 1, 0, NOH, 128);
+  static_assert(NCH * RB == kRows && NCH <= 8, "tile geometry");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -322,41 +376,43 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + S::OFF_BAR;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  float* red = reinterpret_cast<float*>(smem + S::OFF_RED);     // [2][4][16]
-  float* red_l = reinterpret_cast<float*>(smem + S::OFF_REDL);  // [4][16]
   const URec* recs = reinterpret_cast<const URec*>(smem + S::OFF_REC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::OFF_MISC + 4);
   int* my_units_s = reinterpret_cast<int*>(smem + S::OFF_MISC + 8);
+  const int nhg = a.Hkv / kHG;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(B_FULL + s), 1);
-      mbar_init(bar(B_EMPTY + s), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar(Bx::FULL + s), 1);
+      mbar_init(bar(Bx::EMPTY + s), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(B_QFULL + i), 1);
-      mbar_init(bar(B_QEMPTY + i), 1);
-      mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_SFREE + i), 128);
-      mbar_init(bar(B_PREADY + i), 128);
-      mbar_init(bar(B_OFULL + i), 1);
-      mbar_init(bar(B_OFREE + i), 128);
+      mbar_init(bar(Bx::QFULL + i), 1);
+      mbar_init(bar(Bx::QEMPTY + i), 1);
+      mbar_init(bar(Bx::SFULL + i), 1);
+      mbar_init(bar(Bx::SFREE + i), 128);
+      mbar_init(bar(Bx::PREADY + i), 128);
+      mbar_init(bar(Bx::OFULL + i), 1);
+      mbar_init(bar(Bx::XFULL + i), 128);
+      mbar_init(bar(Bx::XFREE + i), 128);
     }
-    mbar_init(bar(B_DONE), 1);
+    mbar_init(bar(Bx::ODONE), 128);
+    mbar_init(bar(Bx::DONE), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp < 4) {
-    build_unit_list<BS>(a, smem, const_cast<URec*>(recs), reinterpret_cast<int*>(smem + S::OFF_MISC + 12),
+    build_unit_list<BS>(a, nhg, smem, const_cast<URec*>(recs),
+                        reinterpret_cast<int*>(smem + S::OFF_MISC + 12),
                         reinterpret_cast<int*>(smem + S::OFF_MISC + 16), my_units_s);
     fence_proxy_async();                 // stage 0 served as scratch; TMA writes it next
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
-                 "r"(kTmemCols)
+                 "r"(S::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -364,58 +420,66 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem;                 // S buffers: columns [0,16) and [16,32)
-  const uint32_t tmem_o = tmem + 2 * kNS;       // O buffers: [32, 32+NO) and [32+NO, 32+2NO)
+  const uint32_t tmem_s = tmem;                 // S buffers: [0, NS) and [NS, 2NS)
+  const uint32_t tmem_o = tmem + 2 * NS;        // O accumulators: [2NS, 2NS+NO), [2NS+NO, 2NS+2NO)
   const int nu = *my_units_s;
   auto give_up = [&]() {
     *abort_flag = 1u;
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
   };
+  // token range of tile k of a unit, and how many of its boxes hold tokens
+  auto tile_span = [&](const Unit& x, int k, int& ts, int& te, int& nql) {
+    ts = x.t0 + k * kRt;
+    te = min(x.t1, ts + kRt);
+    nql = (te - ts + RB - 1) / RB;
+  };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int tc = 0, issued = 0;
-      int phys_next[BPT];
-      // block ids of tile k of unit i, loaded one tile ahead of their use
+      int phys_next[NQ];
       auto load_ids = [&](int i, int k, int* ph) {
         const Unit x = unit_from(recs[i], a.psize);
-        const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
-        const int nb = (te - ts + BS - 1) / BS;
-        const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks + ts / BS;
+        int ts, te, nql;
+        tile_span(x, k, ts, te, nql);
+        const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
 #pragma unroll
-        for (int q = 0; q < BPT; ++q) ph[q] = q < nb ? __ldg(table + q) : -1;
+        for (int q = 0; q < NQ; ++q) ph[q] = q < nql ? __ldg(table + (ts + q * RB) / BS) : -1;
       };
       if (nu > 0) load_ids(0, 0, phys_next);
       for (int i = 0; i < nu; ++i) {
         const Unit x = unit_from(recs[i], a.psize);
         const int qi = i & 1;
-        if (!mbar_wait(bar(B_QEMPTY + qi), ((i >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-        mbar_expect_tx(bar(B_QFULL + qi), 2u * G * 128u);
+        if (!mbar_wait(bar(Bx::QEMPTY + qi), ((i >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+        mbar_expect_tx(bar(Bx::QFULL + qi), 2u * NS * 128u);
         for (int hh = 0; hh < 2; ++hh)
-          tma_load_2d(sbase + S::OFF_Q + qi * kQBytes + hh * (kNS * 128), &tmQ, hh * 64,
-                      x.b * a.Hq + x.h * G, bar(B_QFULL + qi));
+          tma_load_2d(sbase + S::OFF_Q + qi * S::kQBytes + hh * (NS * 128), &tmQ, hh * 64,
+                      x.b * a.Hq + x.h * kHG * G, bar(Bx::QFULL + qi));
         for (int k = 0; k < x.ntiles; ++k) {
-          int phys[BPT];
+          int ts, te, nql;
+          tile_span(x, k, ts, te, nql);
+          int phys[NQ];
           uint32_t bytes = 0;
 #pragma unroll
-          for (int q = 0; q < BPT; ++q) {
+          for (int q = 0; q < NQ; ++q) {
             phys[q] = phys_next[q];
-            if (phys[q] >= 0 && phys[q] < a.num_blocks) bytes += 2u * BS * 128u;
+            if (phys[q] >= 0 && phys[q] < a.num_blocks) bytes += 2u * RB * kHG * 128u;
           }
           if (k + 1 < x.ntiles) load_ids(i, k + 1, phys_next);
           else if (i + 1 < nu) load_ids(i + 1, 0, phys_next);
           for (int kv = 0; kv < 2; ++kv) {
-            const int seq = 2 * tc + kv, s = seq % kStages;
-            if (!mbar_wait(bar(B_EMPTY + s), ((seq / kStages) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-            mbar_expect_tx(bar(B_FULL + s), bytes);
+            const int seq = 2 * tc + kv, s = seq % NST;
+            if (!mbar_wait(bar(Bx::EMPTY + s), ((seq / NST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+            mbar_expect_tx(bar(Bx::FULL + s), bytes);
             const uint32_t dst = sbase + s * kStageBytes;
 #pragma unroll
-            for (int q = 0; q < BPT; ++q) {
+            for (int q = 0; q < NQ; ++q) {
               if (phys[q] < 0 || phys[q] >= a.num_blocks) continue;
+              const int r0 = (ts + q * RB) % BS;
               for (int hh = 0; hh < 2; ++hh)
-                tma_load_4d(dst + hh * kHalf + q * BS * 128, kv ? &tmV : &tmK, hh * 64, x.h, 0,
-                            phys[q], bar(B_FULL + s));
+                tma_load_5d(dst + hh * kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, r0,
+                            x.h * kHG, hh, phys[q], bar(Bx::FULL + s));
             }
             ++issued;
           }
@@ -424,193 +488,314 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       }
     prod_done:
       // never leave with copies in flight: wait (bounded) for the last loads of every stage
-      for (int seq = max(0, issued - kStages); seq < issued; ++seq) {
-        const int s = seq % kStages;
+      for (int seq = max(0, issued - NST); seq < issued; ++seq) {
+        const int s = seq % NST;
         const uint64_t t0 = globaltimer();
-        while (!mbar_try(bar(B_FULL + s), (seq / kStages) & 1) && globaltimer() - t0 < kWaitNs) {}
+        while (!mbar_try(bar(Bx::FULL + s), (seq / NST) & 1) && globaltimer() - t0 < kWaitNs) {}
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int tc = 0;
       bool ok = true;
-      auto issue_pv = [&](int tt, int nb) -> bool {
+      // output product of tile tt (unit ui, tile kk of the unit, nql boxes with tokens)
+      auto issue_pv = [&](int tt, int ui, int kk, int nql) -> bool {
         const int pb = tt & 1;
-        if (!mbar_wait(bar(B_PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(bar(B_OFREE + pb), ((tt >> 1) & 1) ^ 1, abort_flag)) return false;
-        const int seq = 2 * tt + 1, s = seq % kStages;
-        if (!mbar_wait(bar(B_FULL + s), (seq / kStages) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(Bx::PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
+        const bool first = kk <= 1;                   // this group's first tile of the unit
+        if (first && ui > 0 && !mbar_wait(bar(Bx::ODONE), (ui - 1) & 1, abort_flag)) return false;
+        const int seq = 2 * tt + 1, s = seq % NST;
+        if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vst = sbase + s * kStageBytes;
         const uint32_t pst = sbase + S::OFF_P + pb * S::kPBytes;
-        const int nsteps = nb * BS / 16;
-        for (int ks = 0; ks < nsteps; ++ks) {
-          // A = V^T, MN-major: 16 token rows (2 KB) per K step, d-halves 16 KB apart
-          const uint64_t ad = sw128_desc(vst + ks * 2048, kHalf, 1024);
-          // B = [P_hi; P_lo], K-major: token-halves NO*128 B apart, 32 B per K step
-          const uint64_t bd = sw128_desc(pst + (ks >> 2) * (NO * 128) + (ks & 3) * 32, 16, 1024);
-          mma_f16(tmem_o + pb * NO, ad, bd, IDESC_O, ks > 0 ? 1u : 0u);
+#pragma unroll
+        for (int h = 0; h < kHG; ++h) {
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            if (ks * 16 >= nql * RB) continue;       // no tokens loaded there
+            const int q = (ks * 16) / RB;
+            const int row0 = q * (kHG * RB) + h * RB + (ks * 16) % RB;
+            const int c = h * KS + ks;                // 32-byte chunk of the P operand
+            // A = V^T (MN-major): 16 rows of head h from row0; d-halves 16 KB apart
+            const uint64_t ad = sw128_desc(vst + row0 * 128, kHalf, 1024);
+            // B = [P_hi; P_lo] of head h, K-major, chunk c of the 2-line P tile
+            const uint64_t bd = sw128_desc(pst + (c >> 2) * (NOH * 128) + (c & 3) * 32, 16, 1024);
+            mma_f16(tmem_o + pb * NO + h * NOH, ad, bd, IDESC_O, (first && ks == 0) ? 0u : 1u);
+          }
         }
-        mma_commit(bar(B_EMPTY + s));
-        mma_commit(bar(B_OFULL + pb));
+        mma_commit(bar(Bx::EMPTY + s));
+        mma_commit(bar(Bx::OFULL + pb));
         return true;
       };
+      int pui = 0, pkk = 0, pnql = 0;                // the tile waiting for its output product
       for (int i = 0; i < nu && ok; ++i) {
         const Unit x = unit_from(recs[i], a.psize);
         const int qi = i & 1;
-        if (!mbar_wait(bar(B_QFULL + qi), (i >> 1) & 1, abort_flag)) { ok = false; break; }
-        const uint32_t qst = sbase + S::OFF_Q + qi * kQBytes;
-        int prev_nb = 0;
+        if (!mbar_wait(bar(Bx::QFULL + qi), (i >> 1) & 1, abort_flag)) { ok = false; break; }
+        const uint32_t qst = sbase + S::OFF_Q + qi * S::kQBytes;
         for (int k = 0; k < x.ntiles; ++k) {
-          const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
+          int ts, te, nql;
+          tile_span(x, k, ts, te, nql);
           const int sb = tc & 1;
-          if (!mbar_wait(bar(B_SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          const int seq = 2 * tc, s = seq % kStages;
-          if (!mbar_wait(bar(B_FULL + s), (seq / kStages) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int seq = 2 * tc, s = seq % NST;
+          if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + s * kStageBytes;
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint64_t ad = sw128_desc(kst + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(qst + (ks >> 2) * (kNS * 128) + (ks & 3) * 32, 16, 1024);
-            mma_f16(tmem_s + sb * kNS, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+            const uint64_t bd = sw128_desc(qst + (ks >> 2) * (NS * 128) + (ks & 3) * 32, 16, 1024);
+            mma_f16(tmem_s + sb * NS, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
           }
-          mma_commit(bar(B_EMPTY + s));
-          mma_commit(bar(B_SFULL + sb));
-          if (k == x.ntiles - 1) mma_commit(bar(B_QEMPTY + qi));
-          if (k > 0 && !issue_pv(tc - 1, prev_nb)) { ok = false; break; }
-          prev_nb = (te - ts + BS - 1) / BS;
+          mma_commit(bar(Bx::EMPTY + s));
+          mma_commit(bar(Bx::SFULL + sb));
+          if (k == x.ntiles - 1) mma_commit(bar(Bx::QEMPTY + qi));
+          if (tc > 0 && !issue_pv(tc - 1, pui, pkk, pnql)) { ok = false; break; }
+          pui = i; pkk = k; pnql = nql;
           ++tc;
         }
-        if (!ok) break;
-        if (!issue_pv(tc - 1, prev_nb)) { ok = false; break; }
       }
+      if (ok && tc > 0 && !issue_pv(tc - 1, pui, pkk, pnql)) ok = false;
       if (!ok) give_up();
       // all issued MMAs must finish before tensor memory is released
-      mma_commit(bar(B_DONE));
+      mma_commit(bar(Bx::DONE));
       const uint64_t t0 = globaltimer();
-      while (!mbar_try(bar(B_DONE), 0) && globaltimer() - t0 < kWaitNs) {}
+      while (!mbar_try(bar(Bx::DONE), 0) && globaltimer() - t0 < kWaitNs) {}
     }
-  } else {
-    // ------------------------------------------------------------ softmax / output warps
-    const int row = threadIdx.x;                   // token row of S, d row of O
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    int tc = 0;
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax / output groups
+    const int grp = warp >> 2;                     // group: tiles t with t % 2 == grp
+    const int wq = warp & 3;                       // TMEM lane quadrant of this warp
+    const int row = threadIdx.x & 127;             // tile row (head, token) for S; d row for O
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+    const int rq = row / (kHG * RB), rh = (row / RB) % kHG, rr = row % RB;
+    const int tt_row = rq * RB + rr;               // this row's token within its head's tile
+    const int col0 = ((32 * wq / RB) % kHG) * G;   // first S column this warp reads
+    float* red = reinterpret_cast<float*>(smem + S::OFF_RED) + grp * 16 * S::GP;     // [2][8][GP]
+    float* red_l = reinterpret_cast<float*>(smem + S::OFF_REDL) + grp * 16 * S::GP;  // [2][8][GP]
+    float* mold = reinterpret_cast<float*>(smem + S::OFF_MREF) + grp * 3 * NS;      // [NS]
+    float* mnew = mold + NS;                                                         // [NS]
+    float* mown = mnew + NS;                                                         // [NS]
+    float* xbuf = reinterpret_cast<float*>(smem + S::OFF_X);                   // [2][2][NS] + flags
+    int* xflag = reinterpret_cast<int*>(smem + S::OFF_X + 2 * 2 * NS * 4);    // [2]
+    uint8_t* pbuf = smem + S::OFF_P + grp * S::kPBytes;
+    // P address of this row: head rh, K step tt_row / 16, element tt_row % 16
+    const int pc = rh * KS + tt_row / 16, pe = tt_row % 16;
+    uint8_t* prow = pbuf + (pc >> 2) * (NOH * 128);
+    const int pchunk = (pc & 3) * 2 + (pe >> 3), pbyte = (pe & 7) * 2;
     bool failed = false;
-    // this thread's block id for tile k of unit i (its token row), one tile ahead
+    int tc = 0;                                    // global tile index
     auto row_id = [&](int i, int k) -> int {
       const Unit x = unit_from(recs[i], a.psize);
-      const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
-      const int nb = (te - ts + BS - 1) / BS;
-      return row < nb * BS ? __ldg(a.block_tables + (size_t)x.b * a.max_blocks + ts / BS + row / BS)
-                           : -1;
+      int ts, te, nql;
+      tile_span(x, k, ts, te, nql);
+      return rq < nql ? __ldg(a.block_tables + (size_t)x.b * a.max_blocks + (ts + rq * RB) / BS) : -1;
     };
-    int phys_next = nu > 0 ? row_id(0, 0) : -1;
-    for (int i = 0; i < nu; ++i) {
+    int ni = 0, nk = 0;
+    if (nu > 0 && grp == 1) next_tile(recs, nu, a.psize, ni, nk);       // group 1 starts at tile 1
+    int phys_next = (nu > 0 && ni < nu) ? row_id(ni, nk) : -1;
+    bool stop = false;
+    for (int i = 0; i < nu && !stop; ++i) {
       const Unit x = unit_from(recs[i], a.psize);
-      float m[G], l[G], O[G], al_prev[G], al[G];
+      float mo[G], l[G];                           // this row's head: reference max, exp-sum
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        m[g] = -CUDART_INF_F; l[g] = 0.f; O[g] = 0.f; al_prev[g] = 0.f;
-      }
-      auto accumulate = [&](int tt, const float* alpha) {
-        const int pb = tt & 1;
-        if (!mbar_wait(bar(B_OFULL + pb), (tt >> 1) & 1, abort_flag)) failed = true;
-        tc_fence_after();
-        float o[NO];
-#pragma unroll
-        for (int c = 0; c < NO; c += 16) tmem_ld16(tmem_o + lane_off + pb * NO + c, o + c);
-        tc_fence_before();
-        mbar_arrive(bar(B_OFREE + pb));
-#pragma unroll
-        for (int g = 0; g < G; ++g) O[g] = fmaf(O[g], alpha[g], o[g] + o[G + g]);
-      };
-      bool stop = false;
-      for (int k = 0; k < x.ntiles; ++k) {
-        const int ts = x.t0 + k * kTile, te = min(x.t1, ts + kTile);
-        const int nb = (te - ts + BS - 1) / BS;
-        const bool in_range = row < nb * BS;
+      for (int g = 0; g < G; ++g) { mo[g] = -CUDART_INF_F; l[g] = 0.f; }
+      int my_last = -1;
+      for (int k = 0; k < x.ntiles; ++k, ++tc) {
+        if ((tc & 1) != grp) continue;
+        int ts, te, nql;
+        tile_span(x, k, ts, te, nql);
+        const bool in_range = rq < nql;
         const int phys = phys_next;
-        if (k + 1 < x.ntiles) phys_next = row_id(i, k + 1);
-        else if (i + 1 < nu) phys_next = row_id(i + 1, 0);
+        next_tile(recs, nu, a.psize, ni, nk);                 // two tiles ahead: the next own tile
+        next_tile(recs, nu, a.psize, ni, nk);
+        if (ni < nu) phys_next = row_id(ni, nk);
         const bool blk_ok = phys >= 0 && phys < a.num_blocks;
-        const bool valid = in_range && blk_ok && ts + row < te;
-        if (in_range && !blk_ok && (row % BS) == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+        const bool valid = in_range && blk_ok && ts + tt_row < te;
+        if (in_range && !blk_ok && rr == 0 && rh == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+        const bool first = my_last < 0;
 
-        const int sb = tc & 1;
-        if (!mbar_wait(bar(B_SFULL + sb), (tc >> 1) & 1, abort_flag)) failed = true;
+        const int par = (tc >> 1) & 1;                        // use count of this group's buffers
+        if (!mbar_wait(bar(Bx::SFULL + grp), par, abort_flag)) failed = true;
         tc_fence_after();
-        float s[16];
-        tmem_ld16(tmem_s + lane_off + sb * kNS, s);
+        constexpr int SVN = ((32 / RB) * G + 15) / 16 * 16;  // S columns this warp loads
+        float sv[SVN];
+#pragma unroll
+        for (int c = 0; c < SVN; c += 16) tmem_ld16(tmem_s + lane_off + grp * NS + col0 + c, sv + c);
         tc_fence_before();
-        mbar_arrive(bar(B_SFREE + sb));
+        mbar_arrive(bar(Bx::SFREE + grp));
 
-        float* rb = red + (tc & 1) * 64;
+        float s[G];
+        const bool second = rh * G != col0;                   // this row's head is the 2nd loaded
+        float* rb = red + par * 8 * S::GP;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          s[g] = valid ? s[g] * a.scale_log2 : -CUDART_INF_F;
+          const float raw = (RB < 32 && second) ? sv[(RB < 32 ? G : 0) + g] : sv[g];
+          s[g] = valid ? raw * a.scale_log2 : -CUDART_INF_F;
           float v = s[g];
 #pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (lane == 0) rb[warp * 16 + g] = v;
+          for (int o = RB / 2; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+          if (rr == 0) rb[(rq * kHG + rh) * S::GP + g] = v;
         }
-        if (wg_vote_or(failed)) { stop = true; break; }
-        const int pb = tc & 1;
-        uint8_t* pbase = smem + S::OFF_P + pb * S::kPBytes + (row >> 6) * (NO * 128);
-        const int chunk = (row & 63) >> 3, e = row & 7;
+        if (wg_vote_or(failed, grp)) { stop = true; break; }
+        // this head's tile maxima; lazy update of the references (uniform per group)
+        float tm[G], ao[G];
+        bool exceed = false;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const float tmax = fmaxf(fmaxf(rb[g], rb[16 + g]), fmaxf(rb[32 + g], rb[48 + g]));
-          const float m_new = fmaxf(m[g], tmax);
-          al[g] = m_new == -CUDART_INF_F ? 1.f : exp2f(m[g] - m_new);
-          const float p = valid ? exp2f(s[g] - m_new) : 0.f;
-          l[g] = fmaf(l[g], al[g], p);
-          m[g] = m_new;
+          tm[g] = -CUDART_INF_F;
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) tm[g] = fmaxf(tm[g], rb[(q * kHG + rh) * S::GP + g]);
+          ao[g] = 1.f;
+          if (first) mo[g] = tm[g];
+          else exceed |= tm[g] > mo[g] + kRescaleLog2;
+        }
+        if (!first && wg_vote_or(exceed, grp)) {
+          // rare: O holds earlier tiles' products; publish old and new references,
+          // wait for the last product, rescale the moved columns in TMEM
+          if (rq == 0 && rr == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              mold[rh * G + g] = mo[g];
+              mnew[rh * G + g] = tm[g] > mo[g] + kRescaleLog2 ? tm[g] : mo[g];
+            }
+          }
+          wg_sync(grp);
+          if (!mbar_wait(bar(Bx::OFULL + grp), par ^ 1, abort_flag)) failed = true;
+          tc_fence_after();
+#pragma unroll
+          for (int h = 0; h < kHG; ++h) {
+#pragma unroll
+            for (int c = 0; c < NOH; c += 16) {
+              float o[16];
+              const uint32_t ta = tmem_o + lane_off + grp * NO + h * NOH + c;
+              tmem_ld16(ta, o);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int cc = c + e;             // hi columns [0, G), lo columns [G, 2G)
+                if (cc >= 2 * G) continue;
+                const int n = h * G + (cc < G ? cc : cc - G);
+                if (mnew[n] != mold[n] && mold[n] != -CUDART_INF_F) o[e] *= exp2f(mold[n] - mnew[n]);
+              }
+              tmem_st16(ta, o);
+            }
+          }
+          tc_fence_before();
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            if (tm[g] > mo[g] + kRescaleLog2) {
+              ao[g] = mo[g] == -CUDART_INF_F ? 1.f : exp2f(mo[g] - tm[g]);
+              mo[g] = tm[g];
+            }
+          }
+          wg_sync(grp);                           // mold / mnew may be rewritten next tile
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float p = valid ? exp2f(s[g] - mo[g]) : 0.f;
+          l[g] = fmaf(l[g], ao[g], p);
           uint16_t hi, lo;
           split_16<FMT>(p, hi, lo);
-          *reinterpret_cast<uint16_t*>(pbase + g * 128 + ((chunk ^ (g & 7)) << 4) + e * 2) = hi;
-          *reinterpret_cast<uint16_t*>(pbase + (G + g) * 128 + (((chunk ^ ((G + g) & 7))) << 4) + e * 2) = lo;
+          *reinterpret_cast<uint16_t*>(prow + g * 128 + ((pchunk ^ (g & 7)) << 4) + pbyte) = hi;
+          *reinterpret_cast<uint16_t*>(prow + (G + g) * 128 + ((pchunk ^ ((G + g) & 7)) << 4) + pbyte) = lo;
         }
         if (in_range && !valid) {
-          // this V row enters the PV product with weight 0: it must hold finite values
-          const int seq = 2 * tc + 1, sv = seq % kStages;
-          if (!mbar_wait(bar(B_FULL + sv), (seq / kStages) & 1, abort_flag)) failed = true;
-          uint4* r0 = reinterpret_cast<uint4*>(smem + sv * kStageBytes + row * 128);
-          uint4* r1 = reinterpret_cast<uint4*>(smem + sv * kStageBytes + kHalf + row * 128);
+          // this V row enters the output product with weight 0: it must hold finite values
+          const int seq = 2 * tc + 1, sv_ = seq % NST;
+          if (!mbar_wait(bar(Bx::FULL + sv_), (seq / NST) & 1, abort_flag)) failed = true;
+          uint4* r0 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + row * 128);
+          uint4* r1 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + kHalf + row * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) { r0[c] = make_uint4(0, 0, 0, 0); r1[c] = make_uint4(0, 0, 0, 0); }
         }
         fence_proxy_async();
-        mbar_arrive(bar(B_PREADY + pb));
-        if (k > 0) accumulate(tc - 1, al_prev);
-#pragma unroll
-        for (int g = 0; g < G; ++g) al_prev[g] = al[g];
-        ++tc;
+        mbar_arrive(bar(Bx::PREADY + grp));
+        my_last = tc;
       }
       if (stop) break;
-      accumulate(tc - 1, al_prev);
 
-      // epilogue: total exp-sum per head, then the unit's output rows
+      // ---- end of unit i: exp-sums per query head, then one group merges both accumulators
+      float* rl = red_l + (i & 1) * 8 * S::GP;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float v = l[g];
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red_l[warp * 16 + g] = v;
+        for (int o = RB / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (rr == 0) rl[(rq * kHG + rh) * S::GP + g] = v;
       }
-      if (wg_vote_or(failed)) break;
+      if (wg_vote_or(failed, grp)) break;
+      const int xi = i & 1, xpar = (i >> 1) & 1;
+      float* xm = xbuf + xi * 2 * NS;
+      float* xl = xm + NS;
+      const int last_grp = (tc - 1) & 1;                    // group of the unit's last tile
+      if (grp != last_grp) {
+        if (my_last >= 0 && !mbar_wait(bar(Bx::OFULL + grp), (my_last >> 1) & 1, abort_flag)) failed = true;
+        if (!mbar_wait(bar(Bx::XFREE + xi), xpar ^ 1, abort_flag)) failed = true;
+        if (row < NS) {
+          float L = 0.f;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float L = red_l[g] + red_l[16 + g] + red_l[32 + g] + red_l[48 + g];
-        const size_t orow = (size_t)x.b * a.Hq + x.h * G + g;
-        if (x.nparts == 1) {
-          store_out(a.out, orow * kD + row, L > 0.f ? O[g] / L : 0.f, a.out_dtype);
-        } else {
-          const size_t pj = orow * a.P + x.j;
-          a.ws_acc[pj * kD + row] = O[g];
-          if (row == 0) { a.ws_m[pj] = m[g]; a.ws_l[pj] = L; }
+          for (int q = 0; q < NQ; ++q) L += rl[(q * kHG + row / G) * S::GP + row % G];
+          xl[row] = L;
         }
+        if (rq == 0 && rr == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) xm[rh * G + g] = mo[g];
+        }
+        if (row == 0) xflag[xi] = my_last >= 0 ? 1 : 0;
+        tc_fence_before();
+        mbar_arrive(bar(Bx::XFULL + xi));
+      } else {
+        if (!mbar_wait(bar(Bx::OFULL + grp), (my_last >> 1) & 1, abort_flag)) failed = true;
+        if (!mbar_wait(bar(Bx::XFULL + xi), xpar, abort_flag)) failed = true;
+        if (rq == 0 && rr == 0) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) mown[rh * G + g] = mo[g];
+        }
+        wg_sync(grp);
+        tc_fence_after();
+        const bool has_p = xflag[xi] != 0;
+#pragma unroll
+        for (int h = 0; h < kHG; ++h) {
+          float own[16 > NOH ? 16 : NOH], part[16 > NOH ? 16 : NOH];
+#pragma unroll
+          for (int c = 0; c < NOH; c += 16) {
+            tmem_ld16(tmem_o + lane_off + grp * NO + h * NOH + c, own + c);
+            tmem_ld16(tmem_o + lane_off + (1 - grp) * NO + h * NOH + c, part + c);
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const int n = h * G + g;
+            float L = 0.f;
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) L += rl[(q * kHG + h) * S::GP + g];
+            const float mp = has_p ? xm[n] : -CUDART_INF_F;
+            const float mine = mown[n];
+            const float M = fmaxf(mine, mp);
+            float c = 0.f, cp = 0.f;
+            if (M != -CUDART_INF_F) {
+              c = exp2f(mine - M);
+              if (has_p) cp = exp2f(mp - M);
+            }
+            const int lo = NOH == 2 * G ? G + g : G + g;
+            const float Lt = L * c + (has_p ? xl[n] * cp : 0.f);
+            const float Ot = (own[g] + own[lo]) * c + (has_p ? (part[g] + part[lo]) * cp : 0.f);
+            const size_t orow = (size_t)x.b * a.Hq + (size_t)(x.h * kHG + h) * G + g;
+            if (x.nparts == 1) {
+              store_out(a.out, orow * kD + row, Lt > 0.f ? Ot / Lt : 0.f, a.out_dtype);
+            } else {
+              const size_t pj = orow * a.P + x.j;
+              a.ws_acc[pj * kD + row] = Ot;
+              if (row == 0) { a.ws_m[pj] = M; a.ws_l[pj] = Lt; }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(Bx::XFREE + xi));
+        mbar_arrive(bar(Bx::ODONE));
+        wg_sync(grp);                             // mown is rewritten at the next merge
       }
     }
     if (failed) give_up();
@@ -618,9 +803,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(S::kTmemCols)
                  : "memory");
   }
 }
@@ -647,21 +833,23 @@ bool make_maps(const DecodeArgs& a, int dtype, int G, CUtensorMap* k, CUtensorMa
   if (!enc || a.num_blocks <= 0) return false;
   const CUtensorMapDataType dt =
       dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.Hkv, (cuuint64_t)a.bs,
-                              (cuuint64_t)a.num_blocks};
-  const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)a.Hkv * kD * 2,
+  // the pool [num_blocks][bs][Hkv][D] seen as [num_blocks][2][Hkv][bs][64]: a box of
+  // RB rows x kHG heads x 64 d lands head-major, 128 B per row, 128-byte swizzled
+  const int rb = a.bs < kRt ? a.bs : kRt;
+  const cuuint64_t dims[5] = {64, (cuuint64_t)a.bs, (cuuint64_t)a.Hkv, 2, (cuuint64_t)a.num_blocks};
+  const cuuint64_t strides[4] = {(cuuint64_t)a.Hkv * kD * 2, (cuuint64_t)kD * 2, 128,
                                  (cuuint64_t)a.bs * a.Hkv * kD * 2};
-  const cuuint32_t box[4] = {64, 1, (cuuint32_t)a.bs, 1};
-  const cuuint32_t es[4] = {1, 1, 1, 1};
+  const cuuint32_t box[5] = {64, (cuuint32_t)rb, (cuuint32_t)kHG, 1, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   for (int i = 0; i < 2; ++i) {
-    CUresult r = enc(i == 0 ? k : v, dt, 4, const_cast<void*>(i == 0 ? a.k_cache : a.v_cache), dims,
+    CUresult r = enc(i == 0 ? k : v, dt, 5, const_cast<void*>(i == 0 ? a.k_cache : a.v_cache), dims,
                      strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
   }
   const cuuint64_t qdims[2] = {(cuuint64_t)kD, (cuuint64_t)a.B * a.Hq};
   const cuuint64_t qstr[1] = {(cuuint64_t)kD * 2};
-  const cuuint32_t qbox[2] = {64, (cuuint32_t)G};
+  const cuuint32_t qbox[2] = {64, (cuuint32_t)(kHG * G)};
   const cuuint32_t qes[2] = {1, 1};
   return enc(q, dt, 2, const_cast<void*>(a.q), qdims, qstr, qbox, qes,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -688,8 +876,8 @@ int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
       return PA_ERR_CUDA;
     attr = true;
   }
-  // Units that hold tokens number at most B * Hkv * P; a CTA's list holds kMaxUnits.
-  const long long units = (long long)a.B * a.Hkv * a.P;
+  // Units that hold tokens number at most B * (Hkv / kHG) * P; a CTA's list holds kMaxUnits.
+  const long long units = (long long)a.B * (a.Hkv / kHG) * a.P;
   if (units <= 0) return PA_OK;
   long long grid = units < sm_count() ? units : sm_count();
   if ((units + grid - 1) / grid > kMaxUnits) grid = (units + kMaxUnits - 1) / kMaxUnits;
@@ -713,7 +901,7 @@ int launch_tc_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
 
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs) {
   if (dtype != PA_F16 && dtype != PA_BF16) return false;
-  if (D != kD || (bs != 16 && bs != 32) || Hkv <= 0 || Hq % Hkv) return false;
+  if (D != kD || (bs != 16 && bs != 32) || Hkv <= 0 || Hq % Hkv || Hkv % kHG) return false;
   const int G = Hq / Hkv;
   return G == 4 || G == 8 || G == 16;
 }
