@@ -224,7 +224,7 @@ decode_simt_kernel(const DecodeArgs a) {
     if (nparts == 1) {
       store_out(a.out, row * D + d, L > 0.f ? O / L : 0.f, a.out_dtype);
     } else {
-      const size_t pj = row * a.P + j;
+      const size_t pj = ((size_t)b * a.P + j) * a.Hq + hq0 + g;   // [B][P][Hq] slot
       a.ws_acc[pj * D + d] = O;
       if (d == 0) { a.ws_m[pj] = M; a.ws_l[pj] = L; }
     }
@@ -269,10 +269,13 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
   if (ctx <= 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len) return;
   const int nparts = (ctx + a.psize - 1) / a.psize;
   if (nparts <= 1) return;
-  const float* pm = a.ws_m + (size_t)row * a.P;
-  const float* pl = a.ws_l + (size_t)row * a.P;
+  // partials of (b, hq) sit at [B][P][Hq] slots: partition stride Hq
+  const int hq = row - b * a.Hq;
+  const size_t base = (size_t)b * a.P * a.Hq + hq;
+  const float* pm = a.ws_m + base;
+  const float* pl = a.ws_l + base;
   float M = -CUDART_INF_F;
-  for (int jj = lane; jj < nparts; jj += 32) M = fmaxf(M, pm[jj]);
+  for (int jj = lane; jj < nparts; jj += 32) M = fmaxf(M, pm[(size_t)jj * a.Hq]);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.f, O[PER];
@@ -280,9 +283,9 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
   for (int e = 0; e < PER; ++e) O[e] = 0.f;
   if (M != -CUDART_INF_F) {
     for (int jj = 0; jj < nparts; ++jj) {
-      const float c = exp2f(pm[jj] - M);          // empty partitions: m = -inf, c = 0
-      L = fmaf(pl[jj], c, L);
-      const float* src = a.ws_acc + ((size_t)row * a.P + jj) * D + lane * PER;
+      const float c = exp2f(pm[(size_t)jj * a.Hq] - M);   // empty partitions: m = -inf, c = 0
+      L = fmaf(pl[(size_t)jj * a.Hq], c, L);
+      const float* src = a.ws_acc + (base + (size_t)jj * a.Hq) * D + lane * PER;
 #pragma unroll
       for (int e = 0; e < PER; ++e) O[e] = fmaf(src[e], c, O[e]);
     }

@@ -1,7 +1,8 @@
 // decode_tc.cu -- grouped-query paged decode attention on the 5th-generation
 // tensor cores (tcgen05, accumulators in tensor memory), for 16-bit K/V with
-// head size 128, G = Hq / Hkv in {4, 8, 16} query heads per KV head, and KV
-// heads in groups of HG = 4.
+// head size 128, G = Hq / Hkv in {4, 8} query heads per KV head, and KV
+// heads in groups of HG = 4. (G = 16 would need 640 tensor-memory columns for
+// the double-buffered accumulators below; it runs on the CUDA-core kernel.)
 //
 // Why tensor cores here: the G query heads that share a KV head turn the
 // per-token work into a small dense contraction. On the CUDA cores that is ~4
@@ -37,7 +38,11 @@
 //              every SM sub-partition runs two independent softmax warps; at
 //              the end of a unit the group that did not take its last tile
 //              hands its reference maxima and exp-sums to the other (mbarrier
-//              hand-off), which merges both TMEM accumulators and writes;
+//              hand-off), which merges both TMEM accumulators into a shared-
+//              memory staging buffer and sends the unit's rows (contiguous in
+//              the output and in the workspace) out with bulk asynchronous
+//              copies; the accumulators are double-buffered by unit parity,
+//              so the next unit's products do not wait for this merge;
 //   warp 8     TMA producer (one lane): Q of the unit, K and V tiles through a
 //              ring of 32 KB stages;
 //   warp 9     MMA issuer (one lane): S(t), then O(t-1).
@@ -72,15 +77,17 @@ template <int G> struct TcShape {
   static constexpr int NS = kHG * G;                         // N of the score MMA
   static constexpr int NOH = ((2 * G + 15) / 16) * 16;       // N of a head's output MMA
   static constexpr int NO = kHG * NOH;                       // output columns per group
-  static constexpr int kStages = G <= 8 ? 6 : 5;
-  static constexpr int kTmemCols = 2 * NS + 2 * NO <= 256 ? 256 : 512;
+  static constexpr int kStages = 5;
+  static constexpr int kTmemCols = 512;                      // S x2, O x (2 units x 2 groups)
   static constexpr int kQBytes = 2 * NS * 128;               // Q operand: 2 d-halves x NS rows
   static constexpr int kPBytes = 2 * NOH * 128;              // P operand of one tile: 2 lines
+  static constexpr int kStgBytes = NS * kD * 4;              // one group's merged rows (fp32)
   static constexpr int OFF_Q = kStages * kStageBytes;
   static constexpr int OFF_P = OFF_Q + 2 * kQBytes;
-  static constexpr int OFF_X = OFF_P + 2 * kPBytes;          // [2][2][NS] reference max, exp-sum
+  static constexpr int OFF_STG = OFF_P + 2 * kPBytes;        // [2 groups] output staging
+  static constexpr int OFF_X = OFF_STG + 2 * kStgBytes;      // [2][2][NS] reference max, exp-sum
   static constexpr int OFF_BAR = OFF_X + 2 * 2 * NS * 4 + 16;
-  static constexpr int NBAR = 2 * kStages + 19;
+  static constexpr int NBAR = 2 * kStages + 20;
   static constexpr int GP = G < 8 ? 8 : G;                  // per-chunk stride of the reductions
   static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;         // [group][2][8 chunks][GP] maxima
   static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
@@ -90,7 +97,8 @@ template <int G> struct TcShape {
   static constexpr int BYTES = OFF_MISC + 32;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-  static_assert(2 * NS + 2 * NO <= 512, "tensor memory columns");
+  static_assert(2 * NS + 4 * NO <= kTmemCols, "tensor memory columns");
+  static_assert(OFF_STG % 128 == 0, "bulk-copy source alignment");
 };
 
 // barrier indices (the ring's full/empty pairs come first)
@@ -98,7 +106,7 @@ template <int NST> struct Bars {
   static constexpr int FULL = 0, EMPTY = NST, QFULL = 2 * NST, QEMPTY = QFULL + 2,
                        SFULL = QEMPTY + 2, SFREE = SFULL + 2, PREADY = SFREE + 2,
                        OFULL = PREADY + 2, XFULL = OFULL + 2, XFREE = XFULL + 2,
-                       ODONE = XFREE + 2, DONE = ODONE + 1;
+                       ODONE = XFREE + 2, DONE = ODONE + 2;
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -250,6 +258,22 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
 __device__ __forceinline__ void wg_sync(int group) {
   asm volatile("bar.sync %0, 128;" ::"r"(1 + group) : "memory");
 }
+// Bulk asynchronous copy shared -> global (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// The staging buffer may be rewritten once the copies have read it.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- work units
 // A unit is (sequence b, partition j, group h of kHG KV heads). Units exist
@@ -400,6 +424,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       mbar_init(bar(Bx::XFREE + i), 128);
     }
     mbar_init(bar(Bx::ODONE), 128);
+    mbar_init(bar(Bx::ODONE + 1), 128);
     mbar_init(bar(Bx::DONE), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -421,7 +446,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_s = tmem;                 // S buffers: [0, NS) and [NS, 2NS)
-  const uint32_t tmem_o = tmem + 2 * NS;        // O accumulators: [2NS, 2NS+NO), [2NS+NO, 2NS+2NO)
+  // O accumulators from column 2NS: [unit parity][group], NO columns each, so the
+  // next unit accumulates while the previous one is merged
+  const uint32_t tmem_o = tmem + 2 * NS;
+  auto obuf = [&](int ui, int g) { return tmem_o + (uint32_t)((2 * (ui & 1) + g) * NO); };
   const int nu = *my_units_s;
   auto give_up = [&]() {
     *abort_flag = 1u;
@@ -504,7 +532,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         const int pb = tt & 1;
         if (!mbar_wait(bar(Bx::PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
         const bool first = kk <= 1;                   // this group's first tile of the unit
-        if (first && ui > 0 && !mbar_wait(bar(Bx::ODONE), (ui - 1) & 1, abort_flag)) return false;
+        // the unit's accumulators were last used by unit ui - 2: wait for its merge
+        if (first && ui >= 2 && !mbar_wait(bar(Bx::ODONE + (ui & 1)), ((ui - 2) >> 1) & 1, abort_flag))
+          return false;
         const int seq = 2 * tt + 1, s = seq % NST;
         if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag)) return false;
         tc_fence_after();
@@ -522,7 +552,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             const uint64_t ad = sw128_desc(vst + row0 * 128, kHalf, 1024);
             // B = [P_hi; P_lo] of head h, K-major, chunk c of the 2-line P tile
             const uint64_t bd = sw128_desc(pst + (c >> 2) * (NOH * 128) + (c & 3) * 32, 16, 1024);
-            mma_f16(tmem_o + pb * NO + h * NOH, ad, bd, IDESC_O, (first && ks == 0) ? 0u : 1u);
+            mma_f16(obuf(ui, pb) + h * NOH, ad, bd, IDESC_O, (first && ks == 0) ? 0u : 1u);
           }
         }
         mma_commit(bar(Bx::EMPTY + s));
@@ -588,6 +618,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     const int pchunk = (pc & 3) * 2 + (pe >> 3), pbyte = (pe & 7) * 2;
     bool failed = false;
     int tc = 0;                                    // global tile index
+    // Wait for the output product of this group's tile t, the latest tile it
+    // handed over. A parity wait is exact here: the barrier cannot pass t's
+    // phase before the group hands over tile t + 2, and it has already passed
+    // the phase before t's (the group has seen S of a tile >= t, and the
+    // issuer puts S(t) after O(t - 2) on the same in-order tensor pipe).
+    auto wait_pv = [&](int t) {
+      if (!mbar_wait(bar(Bx::OFULL + grp), (t >> 1) & 1, abort_flag)) failed = true;
+    };
     auto row_id = [&](int i, int k) -> int {
       const Unit x = unit_from(recs[i], a.psize);
       int ts, te, nql;
@@ -664,14 +702,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             }
           }
           wg_sync(grp);
-          if (!mbar_wait(bar(Bx::OFULL + grp), par ^ 1, abort_flag)) failed = true;
+          wait_pv(tc - 2);
           tc_fence_after();
 #pragma unroll
           for (int h = 0; h < kHG; ++h) {
 #pragma unroll
             for (int c = 0; c < NOH; c += 16) {
               float o[16];
-              const uint32_t ta = tmem_o + lane_off + grp * NO + h * NOH + c;
+              const uint32_t ta = obuf(i, grp) + lane_off + h * NOH + c;
               tmem_ld16(ta, o);
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
@@ -732,7 +770,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       float* xl = xm + NS;
       const int last_grp = (tc - 1) & 1;                    // group of the unit's last tile
       if (grp != last_grp) {
-        if (my_last >= 0 && !mbar_wait(bar(Bx::OFULL + grp), (my_last >> 1) & 1, abort_flag)) failed = true;
+        if (my_last >= 0) wait_pv(my_last);
         if (!mbar_wait(bar(Bx::XFREE + xi), xpar ^ 1, abort_flag)) failed = true;
         if (row < NS) {
           float L = 0.f;
@@ -748,22 +786,31 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         tc_fence_before();
         mbar_arrive(bar(Bx::XFULL + xi));
       } else {
-        if (!mbar_wait(bar(Bx::OFULL + grp), (my_last >> 1) & 1, abort_flag)) failed = true;
+        wait_pv(my_last);
         if (!mbar_wait(bar(Bx::XFULL + xi), xpar, abort_flag)) failed = true;
         if (rq == 0 && rr == 0) {
 #pragma unroll
           for (int g = 0; g < G; ++g) mown[rh * G + g] = mo[g];
         }
+        if (row == 0) bulk_wait_read();           // the group's previous rows have left staging
         wg_sync(grp);
         tc_fence_after();
         const bool has_p = xflag[xi] != 0;
+        // merged rows go to shared memory first, then out in one bulk copy per head:
+        // the unit's NS output rows are contiguous in out [B, Hq, D] and in the
+        // workspace [B, P, Hq, D]
+        const bool final_out = x.nparts == 1;
+        const int osz = final_out && a.out_dtype != PA_F32 ? 2 : 4;
+        uint8_t* stg = smem + S::OFF_STG + grp * S::kStgBytes;
+        const size_t row0 = final_out ? (size_t)x.b * a.Hq + (size_t)x.h * NS
+                                      : ((size_t)x.b * a.P + x.j) * a.Hq + (size_t)x.h * NS;
 #pragma unroll
         for (int h = 0; h < kHG; ++h) {
           float own[16 > NOH ? 16 : NOH], part[16 > NOH ? 16 : NOH];
 #pragma unroll
           for (int c = 0; c < NOH; c += 16) {
-            tmem_ld16(tmem_o + lane_off + grp * NO + h * NOH + c, own + c);
-            tmem_ld16(tmem_o + lane_off + (1 - grp) * NO + h * NOH + c, part + c);
+            tmem_ld16(obuf(i, grp) + lane_off + h * NOH + c, own + c);
+            tmem_ld16(obuf(i, 1 - grp) + lane_off + h * NOH + c, part + c);
           }
 #pragma unroll
           for (int g = 0; g < G; ++g) {
@@ -779,25 +826,32 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
               c = exp2f(mine - M);
               if (has_p) cp = exp2f(mp - M);
             }
-            const int lo = NOH == 2 * G ? G + g : G + g;
             const float Lt = L * c + (has_p ? xl[n] * cp : 0.f);
-            const float Ot = (own[g] + own[lo]) * c + (has_p ? (part[g] + part[lo]) * cp : 0.f);
-            const size_t orow = (size_t)x.b * a.Hq + (size_t)(x.h * kHG + h) * G + g;
-            if (x.nparts == 1) {
-              store_out(a.out, orow * kD + row, Lt > 0.f ? Ot / Lt : 0.f, a.out_dtype);
+            const float Ot = (own[g] + own[G + g]) * c + (has_p ? (part[g] + part[G + g]) * cp : 0.f);
+            if (final_out) {
+              store_out(stg, (size_t)n * kD + row, Lt > 0.f ? Ot / Lt : 0.f, a.out_dtype);
             } else {
-              const size_t pj = orow * a.P + x.j;
-              a.ws_acc[pj * kD + row] = Ot;
-              if (row == 0) { a.ws_m[pj] = M; a.ws_l[pj] = Lt; }
+              reinterpret_cast<float*>(stg)[n * kD + row] = Ot;
+              if (row == n) { a.ws_m[row0 + n] = M; a.ws_l[row0 + n] = Lt; }
             }
           }
         }
         tc_fence_before();
         mbar_arrive(bar(Bx::XFREE + xi));
-        mbar_arrive(bar(Bx::ODONE));
-        wg_sync(grp);                             // mown is rewritten at the next merge
+        mbar_arrive(bar(Bx::ODONE + (i & 1)));
+        fence_proxy_async();                      // staging writes -> the bulk copy's proxy
+        wg_sync(grp);                             // (mown is rewritten at the next merge, too)
+        if (row == 0) {
+          uint8_t* dst = final_out ? static_cast<uint8_t*>(a.out) + row0 * kD * osz
+                                   : reinterpret_cast<uint8_t*>(a.ws_acc) + row0 * kD * 4;
+          const uint32_t hb = (uint32_t)(G * kD * osz);
+#pragma unroll
+          for (int h = 0; h < kHG; ++h) bulk_store(dst + h * hb, smem_addr(stg) + h * hb, hb);
+          bulk_commit();
+        }
       }
     }
+    if (row == 0) bulk_wait_all();               // no copy outlives the kernel
     if (failed) give_up();
   }
 
@@ -892,7 +946,6 @@ int launch_tc_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
   switch (a.Hq / a.Hkv) {
     case 4: return launch_tc_t<FMT, BS, 4>(a, k, v, q, stream);
     case 8: return launch_tc_t<FMT, BS, 8>(a, k, v, q, stream);
-    case 16: return launch_tc_t<FMT, BS, 16>(a, k, v, q, stream);
   }
   return PA_ERR_UNSUPPORTED;
 }
@@ -903,7 +956,7 @@ bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs) {
   if (dtype != PA_F16 && dtype != PA_BF16) return false;
   if (D != kD || (bs != 16 && bs != 32) || Hkv <= 0 || Hq % Hkv || Hkv % kHG) return false;
   const int G = Hq / Hkv;
-  return G == 4 || G == 8 || G == 16;
+  return G == 4 || G == 8;
 }
 
 int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream) {

@@ -23,9 +23,9 @@ struct DecodeArgs {
   int max_context_len;
   int P;                // partitions per sequence (grid extent); 1 = single pass
   int psize;            // tokens per partition (a multiple of bs)
-  float* ws_acc;        // [B, Hq, P, D] unnormalised partial outputs (P > 1)
-  float* ws_m;          // [B, Hq, P] partial max, log2 domain
-  float* ws_l;          // [B, Hq, P] partial sum of exp2(s - m)
+  float* ws_acc;        // [B, P, Hq, D] unnormalised partial outputs (P > 1)
+  float* ws_m;          // [B, P, Hq] partial max, log2 domain
+  float* ws_l;          // [B, P, Hq] partial sum of exp2(s - m)
   uint32_t* err_flag;
 };
 

@@ -134,9 +134,12 @@ def test_split_partials_match_the_oracle_partials(kernel_choice):
     rows = B * Hq * P
     up = lambda x: (x + 255) // 256 * 256
     ws = t["workspace"].cpu().numpy()
-    acc = ws[:rows * D * 4].view(np.float32).reshape(B, Hq, P, D)
-    m2 = ws[up(rows * D * 4):up(rows * D * 4) + rows * 4].view(np.float32).reshape(B, Hq, P)
-    l = ws[up(rows * D * 4) + up(rows * 4):][:rows * 4].view(np.float32).reshape(B, Hq, P)
+    # workspace layout: acc [B, P, Hq, D], then m and l [B, P, Hq]
+    acc = ws[:rows * D * 4].view(np.float32).reshape(B, P, Hq, D).transpose(0, 2, 1, 3)
+    m2 = ws[up(rows * D * 4):up(rows * D * 4) + rows * 4].view(np.float32).reshape(B, P, Hq)
+    m2 = m2.transpose(0, 2, 1)
+    l = ws[up(rows * D * 4) + up(rows * 4):][:rows * 4].view(np.float32).reshape(B, P, Hq)
+    l = l.transpose(0, 2, 1)
     log2e = 1.0 / math.log(2.0)
     for b in range(B):
         nparts = -(-ctx[b] // psize)
