@@ -92,13 +92,15 @@ template <int G> struct TcShape {
   static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;         // [group][2][8 chunks][GP] maxima
   static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
   static constexpr int OFF_MREF = OFF_REDL + 2 * 2 * 8 * GP * 4;  // [group][3][NS] references
-  static constexpr int OFF_REC = (OFF_MREF + 2 * 3 * NS * 4 + 15) / 16 * 16;
+  static constexpr int OFF_COEF = OFF_MREF + 2 * 3 * NS * 4;   // [group][2][NS] merge weights
+  static constexpr int OFF_REC = (OFF_COEF + 2 * 2 * NS * 4 + 15) / 16 * 16;
   static constexpr int OFF_MISC = OFF_REC + kMaxUnits * 16;
   static constexpr int BYTES = OFF_MISC + 32;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   static_assert(2 * NS + 4 * NO <= kTmemCols, "tensor memory columns");
   static_assert(OFF_STG % 128 == 0, "bulk-copy source alignment");
+  static_assert(OFF_COEF % 16 == 0, "vector loads of the merge weights");
 };
 
 // barrier indices (the ring's full/empty pairs come first)
@@ -132,6 +134,16 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
@@ -560,6 +572,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         return true;
       };
       int pui = 0, pkk = 0, pnql = 0;                // the tile waiting for its output product
+      bool pending = false;                          // tile tc - 1 still needs its output product
       for (int i = 0; i < nu && ok; ++i) {
         const Unit x = unit_from(recs[i], a.psize);
         const int qi = i & 1;
@@ -569,8 +582,26 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           int ts, te, nql;
           tile_span(x, k, ts, te, nql);
           const int sb = tc & 1;
-          if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
           const int seq = 2 * tc, s = seq % NST;
+          if (pending) {
+            // whichever comes first: the softmax of tile tc - 1 (issue its output
+            // product now, so its V stage and its group are released early) or
+            // the inputs of S(tc)
+            const uint64_t t0 = globaltimer();
+            while (true) {
+              if (mbar_test(bar(Bx::PREADY + ((tc - 1) & 1)), ((tc - 1) >> 1) & 1)) {
+                if (!issue_pv(tc - 1, pui, pkk, pnql)) ok = false;
+                pending = false;
+                break;
+              }
+              if (mbar_test(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1) &&
+                  mbar_test(bar(Bx::FULL + s), (seq / NST) & 1))
+                break;
+              if (*abort_flag || globaltimer() - t0 > kWaitNs) { ok = false; break; }
+            }
+            if (!ok) break;
+          }
+          if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
           if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + s * kStageBytes;
@@ -583,12 +614,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           mma_commit(bar(Bx::EMPTY + s));
           mma_commit(bar(Bx::SFULL + sb));
           if (k == x.ntiles - 1) mma_commit(bar(Bx::QEMPTY + qi));
-          if (tc > 0 && !issue_pv(tc - 1, pui, pkk, pnql)) { ok = false; break; }
+          if (pending && !issue_pv(tc - 1, pui, pkk, pnql)) { ok = false; break; }
+          pending = true;
           pui = i; pkk = k; pnql = nql;
           ++tc;
         }
       }
-      if (ok && tc > 0 && !issue_pv(tc - 1, pui, pkk, pnql)) ok = false;
+      if (ok && pending && !issue_pv(tc - 1, pui, pkk, pnql)) ok = false;
       if (!ok) give_up();
       // all issued MMAs must finish before tensor memory is released
       mma_commit(bar(Bx::DONE));
@@ -794,7 +826,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         }
         if (row == 0) bulk_wait_read();           // the group's previous rows have left staging
         wg_sync(grp);
-        tc_fence_after();
         const bool has_p = xflag[xi] != 0;
         // merged rows go to shared memory first, then out in one bulk copy per head:
         // the unit's NS output rows are contiguous in out [B, Hq, D] and in the
@@ -804,36 +835,56 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         uint8_t* stg = smem + S::OFF_STG + grp * S::kStgBytes;
         const size_t row0 = final_out ? (size_t)x.b * a.Hq + (size_t)x.h * NS
                                       : ((size_t)x.b * a.P + x.j) * a.Hq + (size_t)x.h * NS;
+        float* coef = reinterpret_cast<float*>(smem + S::OFF_COEF) + grp * 2 * NS;
+        if (row < NS) {
+          // query head n: combined max and exp-sum, and the weights of the two
+          // accumulators (divided by the exp-sum when this is the final output)
+          const int n = row, h = n / G, g = n - h * G;
+          float L = 0.f;
 #pragma unroll
+          for (int q = 0; q < NQ; ++q) L += rl[(q * kHG + h) * S::GP + g];
+          const float mp = has_p ? xm[n] : -CUDART_INF_F;
+          const float mine = mown[n];
+          const float M = fmaxf(mine, mp);
+          float c = 0.f, cp = 0.f;
+          if (M != -CUDART_INF_F) {
+            c = exp2f(mine - M);
+            if (has_p) cp = exp2f(mp - M);
+          }
+          const float Lt = L * c + (has_p ? xl[n] * cp : 0.f);
+          if (final_out) {
+            const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+            c *= inv;
+            cp *= inv;
+          } else {
+            a.ws_m[row0 + n] = M;
+            a.ws_l[row0 + n] = Lt;
+          }
+          coef[n] = c;
+          coef[NS + n] = cp;
+        }
+        wg_sync(grp);
+        tc_fence_after();
+#pragma unroll 1
         for (int h = 0; h < kHG; ++h) {
-          float own[16 > NOH ? 16 : NOH], part[16 > NOH ? 16 : NOH];
+          float own[16 > NOH ? 16 : NOH], part[16 > NOH ? 16 : NOH], w[G], wp[G];
 #pragma unroll
           for (int c = 0; c < NOH; c += 16) {
             tmem_ld16(obuf(i, grp) + lane_off + h * NOH + c, own + c);
             tmem_ld16(obuf(i, 1 - grp) + lane_off + h * NOH + c, part + c);
           }
 #pragma unroll
+          for (int g = 0; g < G; g += 4) {
+            *reinterpret_cast<float4*>(w + g) = *reinterpret_cast<const float4*>(coef + h * G + g);
+            *reinterpret_cast<float4*>(wp + g) = *reinterpret_cast<const float4*>(coef + NS + h * G + g);
+          }
+#pragma unroll
           for (int g = 0; g < G; ++g) {
             const int n = h * G + g;
-            float L = 0.f;
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) L += rl[(q * kHG + h) * S::GP + g];
-            const float mp = has_p ? xm[n] : -CUDART_INF_F;
-            const float mine = mown[n];
-            const float M = fmaxf(mine, mp);
-            float c = 0.f, cp = 0.f;
-            if (M != -CUDART_INF_F) {
-              c = exp2f(mine - M);
-              if (has_p) cp = exp2f(mp - M);
-            }
-            const float Lt = L * c + (has_p ? xl[n] * cp : 0.f);
-            const float Ot = (own[g] + own[G + g]) * c + (has_p ? (part[g] + part[G + g]) * cp : 0.f);
-            if (final_out) {
-              store_out(stg, (size_t)n * kD + row, Lt > 0.f ? Ot / Lt : 0.f, a.out_dtype);
-            } else {
-              reinterpret_cast<float*>(stg)[n * kD + row] = Ot;
-              if (row == n) { a.ws_m[row0 + n] = M; a.ws_l[row0 + n] = Lt; }
-            }
+            float v = (own[g] + own[G + g]) * w[g];
+            if (has_p) v = fmaf(part[g] + part[G + g], wp[g], v);   // no partner: its TMEM is stale
+            if (final_out) store_out(stg, (size_t)n * kD + row, v, a.out_dtype);
+            else reinterpret_cast<float*>(stg)[n * kD + row] = v;
           }
         }
         tc_fence_before();
