@@ -257,42 +257,120 @@ int launch_d(const DecodeArgs& a, cudaStream_t stream) {
   return a.D == 64 ? launch_bs<T, 64>(a, stream) : launch_bs<T, 128>(a, stream);
 }
 
-// Merge of the split pass: one warp per (b, hq) row with more than one partition.
-template <int D>
+// Merge of the split pass, for each (b, hq) row with more than one partition:
+// M = max_j m_j, L = sum_j l_j 2^(m_j - M), o = sum_j 2^(m_j - M) acc_j / L.
+// NW warps share a row (NW = 4 when rows have many partitions, else 1); warp w
+// takes partitions w, w + NW, ... Its lanes first find the maximum over the
+// warp's partitions (one partition per lane), then each lane computes the
+// weight of its partition and the warp streams the acc rows eight partitions
+// at a time, so eight loads are in flight per lane. The NW warps of a row
+// combine their (M, L, o) through shared memory.
+template <int PER> struct VecF;
+template <> struct VecF<4> { using T = float4; };
+template <> struct VecF<2> { using T = float2; };
+
+template <int D, int NW>
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
-  constexpr int PER = D / 32;
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  constexpr int PER = D / 32;                  // floats per lane: one 16- or 8-byte vector
+  constexpr int RPB = 4 / NW;                  // rows per block
+  using V = typename VecF<PER>::T;
+  __shared__ float sm_m[NW], sm_l[NW];
+  __shared__ float sm_o[NW][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * RPB + warp / NW;
+  const int sub = warp % NW;
+  // the NW warps of a row take the same branch here (for NW > 1 the block is one row)
   if (row >= a.B * a.Hq) return;
-  const int b = row / a.Hq;
+  const int b = row / a.Hq, hq = row - b * a.Hq;
   const int ctx = a.context_lens[b];
   if (ctx <= 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len) return;
   const int nparts = (ctx + a.psize - 1) / a.psize;
   if (nparts <= 1) return;
   // partials of (b, hq) sit at [B][P][Hq] slots: partition stride Hq
-  const int hq = row - b * a.Hq;
   const size_t base = (size_t)b * a.P * a.Hq + hq;
   const float* pm = a.ws_m + base;
   const float* pl = a.ws_l + base;
-  float M = -CUDART_INF_F;
-  for (int jj = lane; jj < nparts; jj += 32) M = fmaxf(M, pm[(size_t)jj * a.Hq]);
+  // one batch (the usual case): each lane keeps its partition's m and l
+  const bool one = nparts <= 32 * NW;
+  float M = -CUDART_INF_F, mj = -CUDART_INF_F, lj = 0.f;
+  if (one) {
+    const int jl = sub + lane * NW;
+    if (jl < nparts) { mj = pm[(size_t)jl * a.Hq]; lj = pl[(size_t)jl * a.Hq]; }
+    M = mj;
+  } else {
+    for (int jj = sub + lane * NW; jj < nparts; jj += 32 * NW) M = fmaxf(M, pm[(size_t)jj * a.Hq]);
+  }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.f, O[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) O[e] = 0.f;
-  if (M != -CUDART_INF_F) {
-    for (int jj = 0; jj < nparts; ++jj) {
-      const float c = exp2f(pm[(size_t)jj * a.Hq] - M);   // empty partitions: m = -inf, c = 0
-      L = fmaf(pl[(size_t)jj * a.Hq], c, L);
-      const float* src = a.ws_acc + (base + (size_t)jj * a.Hq) * D + lane * PER;
+  if (M != -CUDART_INF_F) {                    // a warp with no partitions keeps M = -inf
+    for (int j0 = sub; j0 < nparts; j0 += 32 * NW) {
+      const int jl = j0 + lane * NW;           // this lane's partition of the batch
+      float c = 0.f;
+      if (jl < nparts) {
+        c = exp2f((one ? mj : pm[(size_t)jl * a.Hq]) - M);
+        L = fmaf(one ? lj : pl[(size_t)jl * a.Hq], c, L);
+      }
+      const int cnt = min(32, (nparts - j0 + NW - 1) / NW);
+      for (int t0 = 0; t0 < cnt; t0 += 8) {
+        V v[8];
+        float ct[8];
 #pragma unroll
-      for (int e = 0; e < PER; ++e) O[e] = fmaf(src[e], c, O[e]);
+        for (int u = 0; u < 8; ++u) {
+          ct[u] = __shfl_sync(0xffffffffu, c, (t0 + u) & 31);
+          if (t0 + u < cnt)
+            v[u] = *reinterpret_cast<const V*>(
+                a.ws_acc + (base + (size_t)(j0 + (t0 + u) * NW) * a.Hq) * D + lane * PER);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (t0 + u < cnt) {
+            const float* f = reinterpret_cast<const float*>(&v[u]);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) O[e] = fmaf(f[e], ct[u], O[e]);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  if (NW > 1) {
+    if (lane == 0) { sm_m[sub] = M; sm_l[sub] = L; }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) sm_o[sub][lane * PER + e] = O[e];
+    __syncthreads();
+    if (sub != 0) return;
+    float Mx = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, sm_m[w]);
+    L = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) O[e] = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float c = sm_m[w] == -CUDART_INF_F ? 0.f : exp2f(sm_m[w] - Mx);
+      L = fmaf(sm_l[w], c, L);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) O[e] = fmaf(sm_o[w][lane * PER + e], c, O[e]);
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
   for (int e = 0; e < PER; ++e) store_out(a.out, (size_t)row * D + lane * PER + e, O[e] * inv, a.out_dtype);
+}
+
+template <int D>
+int launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
+  const long long rows = (long long)a.B * a.Hq;
+  if (a.P >= 16) {
+    merge_kernel<D, 4><<<(unsigned)rows, 128, 0, stream>>>(a);
+  } else {
+    merge_kernel<D, 1><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace
@@ -307,11 +385,7 @@ int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream) {
 }
 
 int launch_merge(const DecodeArgs& a, cudaStream_t stream) {
-  const long long rows = (long long)a.B * a.Hq;
-  const unsigned blocks = (unsigned)((rows + 3) / 4);
-  if (a.D == 64) merge_kernel<64><<<blocks, 128, 0, stream>>>(a);
-  else merge_kernel<128><<<blocks, 128, 0, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return a.D == 64 ? launch_merge_d<64>(a, stream) : launch_merge_d<128>(a, stream);
 }
 
 }  // namespace pa

@@ -69,7 +69,7 @@ constexpr int kRt = kRows / kHG;                // tokens per head per tile (32)
 constexpr int kThreads = 320;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kMaxUnits = 320;                  // work units one CTA can hold in its list
-constexpr int kScanChunk = 4096;                // sequences scanned per pass (stage 0 as scratch)
+constexpr int kScanChunk = 2048;                // sequences scanned per pass (stage 0 as scratch)
 constexpr float kRescaleLog2 = 64.f;            // lazy rescale threshold (log2 units): p <= 2^64,
                                                 // far from fp32 overflow in l and O
 
@@ -289,10 +289,13 @@ __device__ __forceinline__ void bulk_wait_all() {
 
 // ---------------------------------------------------------------- work units
 // A unit is (sequence b, partition j, group h of kHG KV heads). Units exist
-// only for partitions that hold tokens; they are numbered sequence by sequence
-// (k = (partitions before b) * NHG + j * NHG + h, NHG = Hkv / kHG) and CTA c takes k = c, c + grid,
-// ... Every CTA builds its own list at start, in shared memory, so the roles
-// never touch global memory to find their next unit.
+// only for partitions that hold tokens. Units are spread over the CTAs like
+// longest-first list scheduling: they are ranked by size class (16 classes of
+// tile count, whole partitions first), and rank r goes to round r / grid of a
+// zig-zag over the CTAs (even rounds CTA 0, 1, ..., odd rounds backwards), so
+// every CTA gets its big units first and the small ones even out the end.
+// Every CTA builds its own list at start, in shared memory, so the roles never
+// touch global memory to find their next unit.
 struct __align__(16) URec {
   int b, h, j, ctx;
 };
@@ -311,74 +314,132 @@ __device__ __forceinline__ Unit unit_from(const URec& r, int psize) {
   return x;
 }
 
-// Build this CTA's unit list (128 threads of warps 0-3). Sequences with no
-// tokens (or a context length the table cannot hold) get no units; their
-// output rows are zeroed here by the CTA that owns them.
+// Build this CTA's unit list (128 threads of warps 0-3, stage 0 as scratch).
+// Sequences with no tokens (or a context length the table cannot hold) get no
+// units; their output rows are zeroed here by CTA b % grid. Thread t of a pass
+// over kScanChunk sequences owns sequences t, t + 128, ... of the chunk, and
+// ranks within a class follow (pass, thread, sequence) order. Every loop here
+// is short and independent across threads: this runs before any K/V moves.
 template <int BS>
 __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, URec* recs,
-                                int* carry_s, int* wsum, int* my_units) {
+                                int* my_units) {
+  constexpr int NC = 16;                                  // size classes
+  constexpr int PER = kScanChunk / 128;                   // sequences per thread and pass
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int* np_s = reinterpret_cast<int*>(scratch);
-  int* ctx_s = np_s + kScanChunk;
-  constexpr int PER = kScanChunk / 128;
-  if (tid == 0) *carry_s = 0;
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
+  int* ctx_s = reinterpret_cast<int*>(scratch);           // [kScanChunk]
+  int* next_s = ctx_s + kScanChunk;                       // [NC][128] next rank per class
+  int* hist = next_s + NC * 128;                          // [NC] units per class
+  int* cbase = hist + NC;                                 // [NC] first rank of each class
+  int* carry = cbase + NC;                                // [NC] ranks used by earlier passes
+  int* wsum = carry + NC;                                 // [4][NC]
+  int* nempty = wsum + 4 * NC;                            // sequences to zero in this pass
+  int* empty_s = nempty + 4;                              // [kScanChunk]
+  const int TP = (a.psize + kRt - 1) / kRt;               // tiles of a whole partition
+  // partitions of a sequence and tiles of its last one; false: no units
+  auto shape = [&](int ctx, int& np, int& tl) -> bool {
+    if (ctx <= 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len) return false;
+    np = (ctx + a.psize - 1) / a.psize;
+    tl = (ctx - (np - 1) * a.psize + kRt - 1) / kRt;
+    return true;
+  };
+  auto cls = [&](int nt) { return min(NC - 1, (nt * NC + TP - 1) / TP - 1); };
+  auto bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+
+  if (tid < NC) { hist[tid] = 0; carry[tid] = 0; }
+  bar();
+  for (int b = tid; b < a.B; b += 128) {
+    int np, tl;
+    if (!shape(__ldg(a.context_lens + b), np, tl)) continue;
+    if (np > 1) atomicAdd(&hist[NC - 1], (np - 1) * nhg);
+    atomicAdd(&hist[cls(tl)], nhg);
+  }
+  bar();
+  if (tid == 0) {
+    int r = 0;
+    for (int q = NC - 1; q >= 0; --q) { cbase[q] = r; r += hist[q]; }
+    const int full = r / grid, rem = r - full * grid;
+    const bool extra = rem > 0 && ((full & 1) ? cta >= grid - rem : cta < rem);
+    *my_units = min(full + (extra ? 1 : 0), kMaxUnits);
+  }
   for (int b0 = 0; b0 < a.B; b0 += kScanChunk) {
     const int n = min(kScanChunk, a.B - b0);
-    for (int i = tid; i < kScanChunk; i += 128) {
-      int np = 0, ctx = 0;
-      if (i < n) {
-        ctx = __ldg(a.context_lens + b0 + i);
-        const bool bad = ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len;
-        np = (bad || ctx == 0) ? 0 : (ctx + a.psize - 1) / a.psize;
-        if (bad && ((b0 + i) % (int)gridDim.x) == (int)blockIdx.x) flag_error(a.err_flag, PA_DEV_BAD_CTX);
-      }
-      np_s[i] = np;
-      ctx_s[i] = ctx;
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    int sum = 0;
-    for (int e = 0; e < PER; ++e) sum += np_s[tid * PER + e];
-    int incl = sum;
+    if (tid == 0) *nempty = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    int wpre = 0;
-    for (int w = 0; w < warp; ++w) wpre += wsum[w];
-    const int base = *carry_s;
-    int pre = base + wpre + incl - sum;                 // partitions before my first sequence
     for (int e = 0; e < PER; ++e) {
-      const int li = tid * PER + e, np = np_s[li];
-      if (np > 0) {
-        const long long start = (long long)pre * nhg, end = start + (long long)np * nhg;
-        long long k = start + (((long long)blockIdx.x - start % gridDim.x) + gridDim.x) % gridDim.x;
-        for (; k < end; k += gridDim.x) {
-          const int idx = (int)((k - blockIdx.x) / gridDim.x);
-          const int local = (int)(k - start);
-          if (idx < kMaxUnits) recs[idx] = URec{b0 + li, local % nhg, local / nhg, ctx_s[li]};
+      const int i = e * 128 + tid;
+      ctx_s[i] = i < n ? __ldg(a.context_lens + b0 + i) : 0;
+    }
+    bar();
+    // units per class of this thread's sequences, then a block-wide scan per class
+    int v[NC];
+#pragma unroll
+    for (int q = 0; q < NC; ++q) v[q] = 0;
+    for (int e = 0; e < PER; ++e) {
+      int np, tl;
+      const int i = e * 128 + tid;
+      if (!shape(ctx_s[i], np, tl)) {
+        if (i < n && ((b0 + i) % grid) == cta) empty_s[atomicAdd(nempty, 1)] = i;
+        continue;
+      }
+      const int c = cls(tl);
+#pragma unroll
+      for (int q = 0; q < NC; ++q) v[q] += (q == NC - 1 ? (np - 1) * nhg : 0) + (q == c ? nhg : 0);
+    }
+    int incl[NC];
+#pragma unroll
+    for (int q = 0; q < NC; ++q) {
+      incl[q] = v[q];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl[q], o);
+        if (lane >= o) incl[q] += t;
+      }
+      if (lane == 31) wsum[warp * NC + q] = incl[q];
+    }
+    bar();
+#pragma unroll
+    for (int q = 0; q < NC; ++q) {
+      int wpre = 0;
+      for (int w = 0; w < warp; ++w) wpre += wsum[w * NC + q];
+      next_s[q * 128 + tid] = cbase[q] + carry[q] + wpre + incl[q] - v[q];
+    }
+    bar();
+    if (tid < NC) carry[tid] += wsum[tid] + wsum[NC + tid] + wsum[2 * NC + tid] + wsum[3 * NC + tid];
+    // walk the units in the order they were counted; keep the ones that land here
+    for (int e = 0; e < PER; ++e) {
+      const int li = e * 128 + tid;
+      int np, tl;
+      if (!shape(ctx_s[li], np, tl)) continue;
+      if (np > 1) {
+        // whole partitions: consecutive ranks r0 .. r0 + nf - 1 (unit j * nhg + h);
+        // visit only the rounds they span and this CTA's slot in each
+        int* nx = next_s + (NC - 1) * 128 + tid;
+        const int r0 = *nx, nf = (np - 1) * nhg;
+        *nx = r0 + nf;
+        for (int round = r0 / grid; round * grid < r0 + nf && round < kMaxUnits; ++round) {
+          const int r = round * grid + ((round & 1) ? grid - 1 - cta : cta);
+          if (r < r0 || r >= r0 + nf) continue;
+          recs[round] = URec{b0 + li, (r - r0) % nhg, (r - r0) / nhg, ctx_s[li]};
         }
       }
-      pre += np;
+      int* nx = next_s + cls(tl) * 128 + tid;               // the last partition
+      for (int h = 0; h < nhg; ++h) {
+        const int r = (*nx)++;
+        const int round = r / grid, pos = r - round * grid;
+        const int owner = (round & 1) ? grid - 1 - pos : pos;
+        if (owner == cta && round < kMaxUnits) recs[round] = URec{b0 + li, h, np - 1, ctx_s[li]};
+      }
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
     // zero the output rows of empty / bad sequences this CTA owns
-    for (int li = 0; li < n; ++li) {
-      const int b = b0 + li;
-      if (np_s[li] != 0 || (b % (int)gridDim.x) != (int)blockIdx.x) continue;
+    bar();
+    for (int k = 0; k < *nempty; ++k) {
+      const int li = empty_s[k], b = b0 + li;
+      if (ctx_s[li] != 0 && tid == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
       for (int i = tid; i < a.Hq * kD; i += 128)
         store_out(a.out, (size_t)b * a.Hq * kD + i, 0.f, a.out_dtype);
     }
-    if (tid == 127) *carry_s = pre;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-  }
-  if (tid == 0) {
-    const long long U = (long long)(*carry_s) * nhg;
-    const long long mine = U > blockIdx.x ? (U - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    *my_units = (int)(mine < kMaxUnits ? mine : kMaxUnits);
+    bar();
   }
 }
 
@@ -442,9 +503,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp < 4) {
-    build_unit_list<BS>(a, nhg, smem, const_cast<URec*>(recs),
-                        reinterpret_cast<int*>(smem + S::OFF_MISC + 12),
-                        reinterpret_cast<int*>(smem + S::OFF_MISC + 16), my_units_s);
+    build_unit_list<BS>(a, nhg, smem, const_cast<URec*>(recs), my_units_s);
     fence_proxy_async();                 // stage 0 served as scratch; TMA writes it next
   } else if (warp == 8) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
