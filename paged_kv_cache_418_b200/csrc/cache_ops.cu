@@ -19,6 +19,8 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
                                          uint4* __restrict__ value_cache,
                                          const int64_t* __restrict__ slot_mapping, int T,
                                          int row16, long long num_slots, uint32_t* err_flag) {
+  pdl_trigger();
+  pdl_wait();
   long long n = (long long)T * row16;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
@@ -42,6 +44,8 @@ __global__ void reshape_and_cache_kernel(const uint4* __restrict__ key,
 __global__ void copy_blocks_kernel(uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
                                    const int64_t* __restrict__ block_mapping, int block16,
                                    int num_blocks, uint32_t* err_flag) {
+  pdl_trigger();
+  pdl_wait();
   int p = blockIdx.x;
   int64_t src = block_mapping[2 * p], dst = block_mapping[2 * p + 1];
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -65,10 +69,11 @@ int launch_reshape_and_cache(const void* key, const void* value, void* key_cache
   int threads = 256;
   long long blocks = (n + threads - 1) / threads;
   if (blocks > 8 * kSMs) blocks = 8 * kSMs;
-  reshape_and_cache_kernel<<<(int)blocks, threads, 0, stream>>>(
+  const cudaError_t e = launch_k(
+      reshape_and_cache_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream,
       (const uint4*)key, (const uint4*)value, (uint4*)key_cache, (uint4*)value_cache,
       slot_mapping, T, row16, (long long)num_blocks * block_size, err_flag);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int launch_copy_blocks(void* key_cache, void* value_cache, int esize,
@@ -80,9 +85,10 @@ int launch_copy_blocks(void* key_cache, void* value_cache, int esize,
   int yb = (block16 + threads * 4 - 1) / (threads * 4);   // ~4 vectors per thread
   if (yb < 1) yb = 1;
   dim3 grid(num_pairs, yb, 2);
-  copy_blocks_kernel<<<grid, threads, 0, stream>>>((uint4*)key_cache, (uint4*)value_cache,
-                                                   block_mapping, block16, num_blocks, err_flag);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = launch_k(copy_blocks_kernel, grid, dim3(threads), 0, stream,
+                                 (uint4*)key_cache, (uint4*)value_cache, block_mapping, block16,
+                                 num_blocks, err_flag);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace pa

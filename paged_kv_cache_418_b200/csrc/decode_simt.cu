@@ -48,6 +48,8 @@ decode_simt_kernel(const DecodeArgs a) {
   __shared__ float sm_acc[kWarps][GC][D];
   __shared__ float sm_m[kWarps][GC];
   __shared__ float sm_l[kWarps][GC];
+  pdl_trigger();
+  pdl_wait();
 
   const int G = a.Hq / a.Hkv;
   const int chunks = G / GC;
@@ -235,8 +237,9 @@ template <typename T, int D, int BS, int GC>
 int launch_t(const DecodeArgs& a, cudaStream_t stream) {
   const int chunks = (a.Hq / a.Hkv) / GC;
   dim3 grid((unsigned)(a.P * chunks), (unsigned)a.Hkv, (unsigned)a.B);
-  decode_simt_kernel<T, D, BS, GC><<<grid, kWarps * 32, 0, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  const cudaError_t e = launch_k(decode_simt_kernel<T, D, BS, GC>, grid, dim3(kWarps * 32), 0,
+                                 stream, a);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <typename T, int D, int BS>
@@ -276,26 +279,31 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
   using V = typename VecF<PER>::T;
   __shared__ float sm_m[NW], sm_l[NW];
   __shared__ float sm_o[NW][D];
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * RPB + warp / NW;
   const int sub = warp % NW;
   // the NW warps of a row take the same branch here (for NW > 1 the block is one row)
   if (row >= a.B * a.Hq) return;
   const int b = row / a.Hq, hq = row - b * a.Hq;
-  const int ctx = a.context_lens[b];
-  if (ctx <= 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len) return;
-  const int nparts = (ctx + a.psize - 1) / a.psize;
-  if (nparts <= 1) return;
   // partials of (b, hq) sit at [B][P][Hq] slots: partition stride Hq
   const size_t base = (size_t)b * a.P * a.Hq + hq;
   const float* pm = a.ws_m + base;
   const float* pl = a.ws_l + base;
-  // one batch (the usual case): each lane keeps its partition's m and l
-  const bool one = nparts <= 32 * NW;
+  // when one batch of lanes covers every partition of the grid (the usual
+  // case), each lane loads its partition's m and l together with the context
+  // length, and partitions past this row's end are masked once it is known
+  const bool one = a.P <= 32 * NW;
+  const int jl = sub + lane * NW;
   float M = -CUDART_INF_F, mj = -CUDART_INF_F, lj = 0.f;
+  if (one && jl < a.P) { mj = pm[(size_t)jl * a.Hq]; lj = pl[(size_t)jl * a.Hq]; }
+  const int ctx = a.context_lens[b];
+  if (ctx <= 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len) return;
+  const int nparts = (ctx + a.psize - 1) / a.psize;
+  if (nparts <= 1) return;
   if (one) {
-    const int jl = sub + lane * NW;
-    if (jl < nparts) { mj = pm[(size_t)jl * a.Hq]; lj = pl[(size_t)jl * a.Hq]; }
+    if (jl >= nparts) { mj = -CUDART_INF_F; lj = 0.f; }
     M = mj;
   } else {
     for (int jj = sub + lane * NW; jj < nparts; jj += 32 * NW) M = fmaxf(M, pm[(size_t)jj * a.Hq]);
@@ -366,11 +374,11 @@ template <int D>
 int launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
   const long long rows = (long long)a.B * a.Hq;
   if (a.P >= 16) {
-    merge_kernel<D, 4><<<(unsigned)rows, 128, 0, stream>>>(a);
-  } else {
-    merge_kernel<D, 1><<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(a);
+    return launch_k(merge_kernel<D, 4>, dim3((unsigned)rows), dim3(128), 0, stream, a) ==
+                   cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return launch_k(merge_kernel<D, 1>, dim3((unsigned)((rows + 3) / 4)), dim3(128), 0, stream, a) ==
+                 cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 }  // namespace

@@ -480,6 +480,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   const int nhg = a.Hkv / kHG;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
@@ -502,15 +503,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp < 4) {
-    build_unit_list<BS>(a, nhg, smem, const_cast<URec*>(recs), my_units_s);
-    fence_proxy_async();                 // stage 0 served as scratch; TMA writes it next
-  } else if (warp == 8) {
+  if (warp == 8) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(S::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();                            // global memory from here on
+  if (warp < 4) {
+    build_unit_list<BS>(a, nhg, smem, const_cast<URec*>(recs), my_units_s);
+    fence_proxy_async();                 // stage 0 served as scratch; TMA writes it next
   }
   tc_fence_before();
   __syncthreads();
@@ -1046,8 +1049,8 @@ int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
   long long grid = units < sm_count() ? units : sm_count();
   if ((units + grid - 1) / grid > kMaxUnits) grid = (units + kMaxUnits - 1) / kMaxUnits;
   if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(a, k, v, q);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return launch_k(kern, dim3((unsigned)grid), dim3(kThreads), smem, stream, a, k, v, q) ==
+                 cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <int FMT, int BS>

@@ -8,6 +8,14 @@
 
 namespace pa {
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("PA_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 namespace {
 
 constexpr int kDefaultPartition = 512;

@@ -61,4 +61,35 @@ __device__ __forceinline__ void flag_error(uint32_t* err_flag, uint32_t bit) {
   if (err_flag) atomicOr(err_flag, bit);
 }
 
+// Programmatic dependent launch. Every kernel of the library lets the next
+// kernel in its stream be scheduled as soon as all of its own CTAs are running
+// (pdl_trigger), and touches global memory only after the previous kernel has
+// completed and its writes are visible (pdl_wait). Without the launch
+// attribute both are no-ops and the stream serialises as usual.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Launch with the programmatic-stream-serialisation attribute (unless the
+// environment sets PA_PDL=0).
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 }  // namespace pa
