@@ -326,10 +326,7 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     else:
         ms = t_start.elapsed_time(t_end)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / K
-    if world > 1:
-        tt = torch.tensor([ms, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, dec_ms = float(tt[0]), float(tt[1])
+    ms, dec_ms = max_over_ranks([ms, dec_ms], world, dev)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error flag {int(err.item())} during timing")
 
@@ -361,21 +358,18 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
         e1.record(stream)
         e1.synchronize()
         e_ms += e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt[0])
+    (e_ms,) = max_over_ranks([e_ms], world, dev)
     barrier()
     if rank != 0:
         return None
 
     kv = w.kv_bytes()
-    value = kv * K * world / (ms / 1e3) / 1e9
+    value = job_value(kv, K, world, ms)
     peak, peak_src = peaks()
     achieved = kv / (dec_ms / 1e3) / 1e9
     kname = {1: "cuda-core", 2: "tcgen05"}[kernel]
     traffic = traffic_record(kname, w)
-    e2e_value = kv * Ke * world / (e_ms / 1e3) / 1e9
+    e2e_value = job_value(kv, Ke, world, e_ms)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(ms / K, 5),
@@ -398,6 +392,28 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
                 "d2h_bytes_per_step": d2h, "steps": Ke},
     }
     return line
+
+
+def rank_seed(k: int, rank: int) -> int:
+    """Seed of workload k on one rank: every replica gets its own batch."""
+    return 1000 + k + 7919 * rank
+
+
+def max_over_ranks(vals, world: int, device):
+    """Elementwise max of per-rank timings (ms) over all ranks; identity at N=1."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    tt = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return [float(v) for v in tt.tolist()]
+
+
+def job_value(kv_bytes_per_step: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job algorithmic GB/s: every rank streams its own batch of kv_bytes per
+    step (weak scaling), and the job takes the slowest rank's time."""
+    return kv_bytes_per_step * steps * world / (ms / 1e3) / 1e9
 
 
 def cpu_baseline(w: W.Workload, budget_s: float = 10.0):
@@ -430,7 +446,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     k = workload_id(args.workload)
-    seed = 1000 + k + 7919 * rank
+    seed = rank_seed(k, rank)
     if args.impl == "reference":
         if rank != 0:
             return 0
