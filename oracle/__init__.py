@@ -6,8 +6,9 @@ and the CUDA package imports nothing from it; what both see is the arrays the
 seeded workload generator produces.
 
 Every function takes host numpy arrays in their storage types (float32,
-float16, or uint16 bit patterns for bf16) plus a dtype code: 0 = f32,
-1 = f16, 2 = bf16. What each one computes, and the passage it follows, is in
+float16, uint16 bit patterns for bf16, uint8 codes for FP8 E4M3 pools) plus a
+dtype code: 0 = f32, 1 = f16, 2 = bf16, 3 = fp8 (E4M3 codes, read times the
+pool's scale). What each one computes, and the passage it follows, is in
 the header comment of ``oracle.c``. Parity status: every function is pinned by
 the ``tests/test_oracle.py`` checks (library routines, closed forms,
 invariances, the pages' worked examples); none is "parity unpinned".
@@ -29,7 +30,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _STAMP = _LIB + ".src-sha256"
 _lib = None
 
-F32, F16, BF16 = 0, 1, 2
+F32, F16, BF16, FP8 = 0, 1, 2, 3
 _ERRORS = {1: "bad argument", 2: "block id out of range", 3: "slot out of range",
            4: "copy pair out of range", 5: "out of memory"}
 
@@ -73,9 +74,16 @@ def _load():
         lib.oracle_copy_blocks.argtypes = [P, P, P, I, I, I, I, I, I]
         lib.oracle_widen.argtypes = [P, P, LL, I]
         lib.oracle_max_threads.argtypes = []
+        lib.oracle_decode_kv.argtypes = [P, P, I, P, P, I, D, D, P, I, P, I, I, I, I, I, I, D,
+                                         P, I, I]
+        lib.oracle_reshape_and_cache_fp8.argtypes = [P, P, P, P, I, ctypes.c_float,
+                                                     ctypes.c_float, P, I, I, I, I, I]
+        lib.oracle_fp8_encode.argtypes = [P, P, LL]
+        lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, I, ctypes.c_size_t, I, I]
         for fn in ("oracle_gather", "oracle_decode", "oracle_decode_partitioned",
                    "oracle_reshape_and_cache", "oracle_copy_blocks", "oracle_widen",
-                   "oracle_max_threads"):
+                   "oracle_max_threads", "oracle_decode_kv", "oracle_reshape_and_cache_fp8",
+                   "oracle_fp8_encode", "oracle_swap_blocks"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -99,7 +107,7 @@ def max_threads() -> int:
 
 
 def widen(a: np.ndarray, dtype: int) -> np.ndarray:
-    """Exact float64 values of stored f32 / f16 / bf16 elements."""
+    """Exact float64 values of stored f32 / f16 / bf16 elements or E4M3 codes."""
     a = _c(a)
     out = np.empty(a.shape, dtype=np.float64)
     _check(_load().oracle_widen(_ptr(out), _ptr(a), a.size, dtype))
@@ -175,3 +183,59 @@ def copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray, block_mapping, dtype: 
     nb, bs, hkv, d = k_cache.shape
     _check(_load().oracle_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(bm), bm.shape[0],
                                       hkv, d, bs, nb, dtype))
+
+
+def decode_kv(q, q_dtype: int, k_cache, v_cache, kv_dtype: int, k_scale: float, v_scale: float,
+              block_tables, context_lens, scale: float, rows=None, n_threads: int = 0
+              ) -> np.ndarray:
+    """Attention with the query in q_dtype and the pools in kv_dtype (FP8 codes are
+    read times k_scale / v_scale): [B, Hq, D] float64, or [len(rows), D]."""
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    bt, cl = _c(block_tables, np.int32), _c(context_lens, np.int32)
+    B, Hq, D = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    assert d2 == D and v_cache.shape == k_cache.shape and bt.shape[0] == B
+    if rows is None:
+        out = np.empty((B, Hq, D), dtype=np.float64)
+        rp, nr = None, 0
+    else:
+        rows = _c(rows, np.int32).reshape(-1, 2)
+        out = np.empty((rows.shape[0], D), dtype=np.float64)
+        rp, nr = _ptr(rows), rows.shape[0]
+    _check(_load().oracle_decode_kv(_ptr(out), _ptr(q), q_dtype, _ptr(k_cache), _ptr(v_cache),
+                                    kv_dtype, float(k_scale), float(v_scale), _ptr(bt),
+                                    bt.shape[1], _ptr(cl), B, Hq, hkv, D, bs, nb, float(scale),
+                                    rp, nr, int(n_threads)))
+    return out
+
+
+def fp8_encode(x) -> np.ndarray:
+    """E4M3 codes (uint8) of float32 values: nearest even, saturating at +-448."""
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    _check(_load().oracle_fp8_encode(_ptr(out), _ptr(x), x.size))
+    return out
+
+
+def reshape_and_cache_fp8(k_codes: np.ndarray, v_codes: np.ndarray, key, value, src_dtype: int,
+                          k_scale: float, v_scale: float, slot_mapping) -> None:
+    """In place on uint8 code pools [NB, bs, Hkv, D]: code = E4M3(float(x) / scale)."""
+    assert k_codes.flags.c_contiguous and v_codes.flags.c_contiguous
+    assert k_codes.dtype == np.uint8 and v_codes.dtype == np.uint8
+    key, value, sm = _c(key), _c(value), _c(slot_mapping, np.int64)
+    nb, bs, hkv, d = k_codes.shape
+    _check(_load().oracle_reshape_and_cache_fp8(
+        _ptr(k_codes), _ptr(v_codes), _ptr(key), _ptr(value), src_dtype, float(k_scale),
+        float(v_scale), _ptr(sm), sm.shape[0], hkv, d, bs, nb))
+
+
+def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k: np.ndarray, src_v: np.ndarray,
+                block_mapping) -> None:
+    """Copy whole blocks src pool -> dst pool for each (src id, dst id) pair, in place."""
+    assert dst_k.flags.c_contiguous and dst_v.flags.c_contiguous
+    src_k, src_v = _c(src_k), _c(src_v)
+    bm = _c(block_mapping, np.int64).reshape(-1, 2)
+    blk = src_k[0].nbytes if src_k.shape[0] else 0
+    assert dst_k[0].nbytes == blk and dst_k.dtype == src_k.dtype
+    _check(_load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
+                                      _ptr(bm), bm.shape[0], blk, src_k.shape[0], dst_k.shape[0]))

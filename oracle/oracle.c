@@ -43,6 +43,24 @@
  *                     src block (all rows, all heads) of K and V to dst, all
  *                     sources read before any write. "vLLM 与 LLM 推理部署实战"
  *                     section 2.2 (a write to a shared block copies it whole).
+ *  oracle_swap_blocks The same whole-block copy between two different pools
+ *                     (host and device memory): preemption by swapping moves
+ *                     a sequence's blocks to CPU memory and back. "vLLM与
+ *                     PagedAttention：大模型推理内存优化技术解析" section 三
+ *                     (preemption: swapping blocks to CPU memory).
+ *  FP8 KV cache       The pools may hold 8-bit codes instead of 16/32-bit
+ *                     values: halving the bytes per token is the stated
+ *                     point ("vLLM与PagedAttention：大模型推理内存优化技术解析"
+ *                     section 6.2; "vLLM 与 LLM 推理部署实战" section 6.1,
+ *                     which also names fp8 K with bf16 V). The pages fix no
+ *                     format; the reading here is OCP FP8 E4M3 (bias 7, no
+ *                     infinities, 448 the largest finite value) with one
+ *                     float scale per pool: stored code = E4M3(x / scale),
+ *                     the quotient taken in binary32 and rounded to nearest
+ *                     even, saturating at +-448; value read = code * scale.
+ *                     oracle_reshape_and_cache_fp8 quantises that way and
+ *                     oracle_decode_kv reads the codes times their scale
+ *                     (exact in double).
  *
  * Inputs are read exactly: f32 as is; f16 and bf16 are widened to double from
  * their bit patterns by the IEEE-754 definitions of those formats.
@@ -55,7 +73,7 @@
 #include <omp.h>
 #endif
 
-enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
+enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2, OR_FP8 = 3 };
 enum { OR_OK = 0, OR_ERR_ARG = 1, OR_ERR_BLOCK = 2, OR_ERR_SLOT = 3, OR_ERR_PAIR = 4,
        OR_ERR_NOMEM = 5 };
 
@@ -80,22 +98,58 @@ static double bf16_to_double(uint16_t b) {
   return (double)x;
 }
 
-static int esize_of(int dtype) { return dtype == OR_F32 ? 4 : 2; }
+/* E4M3: 1 sign, 4 exponent (bias 7), 3 fraction bits; exponent 15 with
+   fraction 7 is NaN, there are no infinities. */
+static double e4m3_to_double(uint8_t c) {
+  int sign = c >> 7, e = (c >> 3) & 15, f = c & 7;
+  double v;
+  if (e == 15 && f == 7)
+    v = NAN;
+  else if (e == 0)
+    v = ldexp((double)f, -9);                  /* subnormal: f/8 * 2^(1-7) */
+  else
+    v = ldexp((double)(8 + f), e - 10);        /* (1 + f/8) * 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* binary32 -> E4M3, round to nearest even on the E4M3 grid, saturating:
+   |y| >= 448 (or rounding to above 448) gives +-448, NaN gives 0x7F. */
+static uint8_t e4m3_from_float(float y) {
+  if (isnan(y)) return 0x7F;
+  uint8_t sign = signbit(y) ? 0x80 : 0;
+  double a = fabs((double)y);
+  if (a >= 448.0) return sign | 0x7E;
+  int ex;
+  frexp(a, &ex);                                /* a in [2^(ex-1), 2^ex) */
+  int binade = ex - 1 < -6 ? -6 : ex - 1;       /* below 2^-6 the grid is uniform */
+  double step = ldexp(1.0, binade - 3);         /* 3 fraction bits */
+  double v = rint(a / step) * step;             /* ties to even (default mode) */
+  if (v == 0.0) return sign;
+  frexp(v, &ex);
+  int be = ex - 1;
+  if (be < -6) return sign | (uint8_t)(v / ldexp(1.0, -9));           /* subnormal */
+  return sign | (uint8_t)((be + 7) << 3) | (uint8_t)((v / ldexp(1.0, be) - 1.0) * 8.0);
+}
+
+static int esize_of(int dtype) { return dtype == OR_F32 ? 4 : (dtype == OR_FP8 ? 1 : 2); }
 
 static double elem(const void* base, size_t i, int dtype) {
   if (dtype == OR_F32) return (double)((const float*)base)[i];
+  if (dtype == OR_FP8) return e4m3_to_double(((const uint8_t*)base)[i]);
   uint16_t h = ((const uint16_t*)base)[i];
   return dtype == OR_F16 ? f16_to_double(h) : bf16_to_double(h);
 }
 
-/* out[i, d] = pool[table[i / bs], i % bs, h, d] for i < ctx (one KV head). */
-static int gather_head(double* out, const void* pool, int dtype, const int32_t* table,
-                       int ctx, int Hkv, int h, int D, int bs, int num_blocks) {
+/* out[i, d] = pool[table[i / bs], i % bs, h, d] * pscale for i < ctx (one KV
+   head); pscale is 1 for 16/32-bit pools, the pool's scale for FP8 codes. */
+static int gather_head(double* out, const void* pool, int dtype, double pscale,
+                       const int32_t* table, int ctx, int Hkv, int h, int D, int bs,
+                       int num_blocks) {
   for (int i = 0; i < ctx; ++i) {
     int32_t blk = table[i / bs];
     if (blk < 0 || blk >= num_blocks) return OR_ERR_BLOCK;
     size_t row = (((size_t)blk * bs + (size_t)(i % bs)) * Hkv + h) * (size_t)D;
-    for (int d = 0; d < D; ++d) out[(size_t)i * D + d] = elem(pool, row + d, dtype);
+    for (int d = 0; d < D; ++d) out[(size_t)i * D + d] = elem(pool, row + d, dtype) * pscale;
   }
   return OR_OK;
 }
@@ -116,9 +170,10 @@ int oracle_gather(double* out, const void* pool, int dtype, const int32_t* table
 }
 
 /* One (b, hq) output row by the textbook two-pass softmax. */
-static int attend_row(double* o, const void* q, const void* kpool, const void* vpool,
-                      int dtype, const int32_t* table, int ctx, int Hq, int Hkv, int D,
-                      int bs, int num_blocks, double scale, int b, int hq) {
+static int attend_row(double* o, const void* q, int qdt, const void* kpool, const void* vpool,
+                      int kvdt, double kscale, double vscale, const int32_t* table, int ctx,
+                      int Hq, int Hkv, int D, int bs, int num_blocks, double scale, int b,
+                      int hq) {
   int G = Hq / Hkv, h = hq / G;
   for (int d = 0; d < D; ++d) o[d] = 0.0;
   if (ctx <= 0) return OR_OK;
@@ -128,11 +183,12 @@ static int attend_row(double* o, const void* q, const void* kpool, const void* v
   double* qv = (double*)malloc(sizeof(double) * (size_t)D);
   int rc = OR_ERR_NOMEM;
   if (K && V && s && qv) {
-    rc = gather_head(K, kpool, dtype, table, ctx, Hkv, h, D, bs, num_blocks);
-    if (rc == OR_OK) rc = gather_head(V, vpool, dtype, table, ctx, Hkv, h, D, bs, num_blocks);
+    rc = gather_head(K, kpool, kvdt, kscale, table, ctx, Hkv, h, D, bs, num_blocks);
+    if (rc == OR_OK)
+      rc = gather_head(V, vpool, kvdt, vscale, table, ctx, Hkv, h, D, bs, num_blocks);
   }
   if (rc == OR_OK) {
-    for (int d = 0; d < D; ++d) qv[d] = elem(q, ((size_t)b * Hq + hq) * D + d, dtype);
+    for (int d = 0; d < D; ++d) qv[d] = elem(q, ((size_t)b * Hq + hq) * D + d, qdt);
     double m = -INFINITY;
     for (int i = 0; i < ctx; ++i) {
       double dot = 0.0;
@@ -156,7 +212,7 @@ static int check_decode_args(const void* q, const void* kp, const void* vp, int 
                              const int32_t* bt, int MB, const int32_t* cl, int B, int Hq,
                              int Hkv, int D, int bs) {
   if (!q || !kp || !vp || !bt || !cl) return OR_ERR_ARG;
-  if (dtype < OR_F32 || dtype > OR_BF16 || B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0)
+  if (dtype < OR_F32 || dtype > OR_FP8 || B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0)
     return OR_ERR_ARG;
   if (Hq % Hkv) return OR_ERR_ARG;
   for (int b = 0; b < B; ++b)
@@ -169,11 +225,13 @@ static int check_decode_args(const void* q, const void* kp, const void* vp, int 
  *      [B, Hq, D] (rows == NULL).
  * Returns OR_OK, or an error code (first error wins); n_threads <= 0 = all.
  */
-int oracle_decode(double* out, const void* q, const void* kpool, const void* vpool, int dtype,
-                  const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
-                  int B, int Hq, int Hkv, int D, int bs, int num_blocks, double scale,
-                  const int32_t* rows, int n_rows, int n_threads) {
-  int rc = check_decode_args(q, kpool, vpool, dtype, block_tables, max_blocks, context_lens,
+int oracle_decode_kv(double* out, const void* q, int q_dtype, const void* kpool,
+                     const void* vpool, int kv_dtype, double k_scale, double v_scale,
+                     const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                     int B, int Hq, int Hkv, int D, int bs, int num_blocks, double scale,
+                     const int32_t* rows, int n_rows, int n_threads) {
+  if (q_dtype < OR_F32 || q_dtype > OR_BF16) return OR_ERR_ARG;
+  int rc = check_decode_args(q, kpool, vpool, kv_dtype, block_tables, max_blocks, context_lens,
                              B, Hq, Hkv, D, bs);
   if (rc != OR_OK || !out) return rc ? rc : OR_ERR_ARG;
   long long n = rows ? n_rows : (long long)B * Hq;
@@ -188,8 +246,9 @@ int oracle_decode(double* out, const void* q, const void* kpool, const void* vpo
     int e;
     if (b < 0 || b >= B || hq < 0 || hq >= Hq) e = OR_ERR_ARG;
     else
-      e = attend_row(out + r * D, q, kpool, vpool, dtype, block_tables + (size_t)b * max_blocks,
-                     context_lens[b], Hq, Hkv, D, bs, num_blocks, scale, b, hq);
+      e = attend_row(out + r * D, q, q_dtype, kpool, vpool, kv_dtype, k_scale, v_scale,
+                     block_tables + (size_t)b * max_blocks, context_lens[b], Hq, Hkv, D, bs,
+                     num_blocks, scale, b, hq);
     if (e != OR_OK) {
 #ifdef _OPENMP
 #pragma omp critical
@@ -198,6 +257,17 @@ int oracle_decode(double* out, const void* q, const void* kpool, const void* vpo
     }
   }
   return err;
+}
+
+/* Same element type for q, K and V (16/32-bit pools). */
+int oracle_decode(double* out, const void* q, const void* kpool, const void* vpool, int dtype,
+                  const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                  int B, int Hq, int Hkv, int D, int bs, int num_blocks, double scale,
+                  const int32_t* rows, int n_rows, int n_threads) {
+  if (dtype == OR_FP8) return OR_ERR_ARG;
+  return oracle_decode_kv(out, q, dtype, kpool, vpool, dtype, 1.0, 1.0, block_tables,
+                          max_blocks, context_lens, B, Hq, Hkv, D, bs, num_blocks, scale, rows,
+                          n_rows, n_threads);
 }
 
 /*
@@ -215,7 +285,7 @@ int oracle_decode_partitioned(double* out, double* part_m, double* part_l, doubl
   int rc = check_decode_args(q, kpool, vpool, dtype, block_tables, max_blocks, context_lens,
                              B, Hq, Hkv, D, bs);
   if (rc != OR_OK || !out) return rc ? rc : OR_ERR_ARG;
-  if (partition_size <= 0) return OR_ERR_ARG;
+  if (partition_size <= 0 || dtype == OR_FP8) return OR_ERR_ARG;
   int maxc = 0;
   for (int b = 0; b < B; ++b) if (context_lens[b] > maxc) maxc = context_lens[b];
   int P = (maxc + partition_size - 1) / partition_size;
@@ -235,8 +305,8 @@ int oracle_decode_partitioned(double* out, double* part_m, double* part_l, doubl
     double* lj = (double*)malloc(sizeof(double) * ((size_t)P + 1));
     double* aj = (double*)calloc(((size_t)P + 1) * D, sizeof(double));
     int e = (K && V && qv && mj && lj && aj) ? OR_OK : OR_ERR_NOMEM;
-    if (e == OR_OK) e = gather_head(K, kpool, dtype, table, ctx, Hkv, h, D, bs, num_blocks);
-    if (e == OR_OK) e = gather_head(V, vpool, dtype, table, ctx, Hkv, h, D, bs, num_blocks);
+    if (e == OR_OK) e = gather_head(K, kpool, dtype, 1.0, table, ctx, Hkv, h, D, bs, num_blocks);
+    if (e == OR_OK) e = gather_head(V, vpool, dtype, 1.0, table, ctx, Hkv, h, D, bs, num_blocks);
     if (e == OR_OK) {
       for (int d = 0; d < D; ++d) qv[d] = elem(q, ((size_t)b * Hq + hq) * D + d, dtype);
       for (int j = 0; j < P; ++j) {
@@ -306,6 +376,58 @@ int oracle_reshape_and_cache(void* kpool, void* vpool, const void* key, const vo
     size_t dst = (blk * bs + off) * row;
     memcpy((char*)kpool + dst, (const char*)key + (size_t)t * row, row);
     memcpy((char*)vpool + dst, (const char*)value + (size_t)t * row, row);
+  }
+  return OR_OK;
+}
+
+/* Scatter with quantisation to E4M3 codes: code = E4M3(float(x) / scale), the
+   quotient in binary32 (x is exact in binary32 for every source type). */
+int oracle_reshape_and_cache_fp8(uint8_t* kpool, uint8_t* vpool, const void* key,
+                                 const void* value, int src_dtype, float k_scale, float v_scale,
+                                 const int64_t* slot_mapping, int T, int Hkv, int D, int bs,
+                                 int num_blocks) {
+  if (!kpool || !vpool || (T > 0 && (!key || !value || !slot_mapping))) return OR_ERR_ARG;
+  if (T < 0 || Hkv <= 0 || D <= 0 || bs <= 0 || num_blocks <= 0) return OR_ERR_ARG;
+  if (src_dtype < OR_F32 || src_dtype > OR_BF16 || !(k_scale > 0.f) || !(v_scale > 0.f))
+    return OR_ERR_ARG;
+  size_t row = (size_t)Hkv * D;
+  long long nslots = (long long)num_blocks * bs;
+  for (int t = 0; t < T; ++t)
+    if (slot_mapping[t] >= nslots) return OR_ERR_SLOT;
+  for (int t = 0; t < T; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s < 0) continue;
+    for (size_t i = 0; i < row; ++i) {
+      float kx = (float)elem(key, (size_t)t * row + i, src_dtype);
+      float vx = (float)elem(value, (size_t)t * row + i, src_dtype);
+      kpool[(size_t)s * row + i] = e4m3_from_float(kx / k_scale);
+      vpool[(size_t)s * row + i] = e4m3_from_float(vx / v_scale);
+    }
+  }
+  return OR_OK;
+}
+
+/* E4M3 codes of n binary32 values (the quantiser above, exported for pinning). */
+int oracle_fp8_encode(uint8_t* out, const float* x, long long n) {
+  if (!out || !x || n < 0) return OR_ERR_ARG;
+  for (long long i = 0; i < n; ++i) out[i] = e4m3_from_float(x[i]);
+  return OR_OK;
+}
+
+/* Block copies between two pools (src_pool -> dst_pool, pairs of block ids). */
+int oracle_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                       const int64_t* block_mapping, int num_pairs, size_t block_bytes,
+                       int src_blocks, int dst_blocks) {
+  if (!dst_k || !dst_v || !src_k || !src_v || num_pairs < 0 || (num_pairs > 0 && !block_mapping))
+    return OR_ERR_ARG;
+  for (int p = 0; p < num_pairs; ++p) {
+    int64_t s = block_mapping[2 * p], d = block_mapping[2 * p + 1];
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) return OR_ERR_PAIR;
+  }
+  for (int p = 0; p < num_pairs; ++p) {
+    size_t s = (size_t)block_mapping[2 * p], d = (size_t)block_mapping[2 * p + 1];
+    memcpy((char*)dst_k + d * block_bytes, (const char*)src_k + s * block_bytes, block_bytes);
+    memcpy((char*)dst_v + d * block_bytes, (const char*)src_v + s * block_bytes, block_bytes);
   }
   return OR_OK;
 }

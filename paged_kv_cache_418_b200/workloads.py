@@ -16,6 +16,12 @@ Value recipe (all workloads)
     sequence's last block, and the slots the step is about to write) are
     NaN, so a kernel that reads outside what it should shows it in its output.
   * Unused block-table entries are -1.
+  * FP8 pools (E4M3 codes, one byte each) are drawn as bit fields, not by
+    quantising anything: sign ~ U{0,1}, exponent field ~ round(N(7, 1.5))
+    clipped to [0, 15], fraction ~ U{0..7} (the NaN pattern 15/7 becomes
+    15/6), so cached values sit around 1 in magnitude before the pool's
+    scale. Empty slots hold the NaN code 0x7F. The new K/V rows of the step
+    stay N(0, 1) in the query's type: reshape_and_cache_fp8 quantises them.
 
 Layout recipe
   * Physical blocks come from a ``BlockManager`` whose free list is a seeded
@@ -44,11 +50,11 @@ import numpy as np
 
 from .block_manager import BlockManager
 
-F32, F16, BF16 = 0, 1, 2
-DTYPE_NAMES = {F32: "f32", F16: "f16", BF16: "bf16"}
-ESIZE = {F32: 4, F16: 2, BF16: 2}
-_STORAGE = {F32: np.float32, F16: np.float16, BF16: np.uint16}
-_NAN_BITS = {F16: 0x7E00, BF16: 0x7FC0}
+F32, F16, BF16, FP8 = 0, 1, 2, 3
+DTYPE_NAMES = {F32: "f32", F16: "f16", BF16: "bf16", FP8: "fp8e4m3"}
+ESIZE = {F32: 4, F16: 2, BF16: 2, FP8: 1}
+_STORAGE = {F32: np.float32, F16: np.float16, BF16: np.uint16, FP8: np.uint8}
+_NAN_BITS = {F16: 0x7E00, BF16: 0x7FC0, FP8: 0x7F}
 
 
 def round_to_storage(x: np.ndarray, dtype: int) -> np.ndarray:
@@ -76,7 +82,18 @@ def storage_to_float64(a: np.ndarray, dtype: int) -> np.ndarray:
 def nan_fill(shape, dtype: int) -> np.ndarray:
     if dtype == F32:
         return np.full(shape, np.nan, dtype=np.float32)
+    if dtype == FP8:
+        return np.full(shape, _NAN_BITS[FP8], dtype=np.uint8)
     return np.full(shape, _NAN_BITS[dtype], dtype=np.uint16).view(_STORAGE[dtype])
+
+
+def random_e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """E4M3 codes drawn field by field (see the module notes); never NaN."""
+    sign = rng.integers(0, 2, size=shape, dtype=np.int64)
+    ex = np.clip(np.rint(rng.normal(7.0, 1.5, size=shape)), 0, 15).astype(np.int64)
+    frac = rng.integers(0, 8, size=shape, dtype=np.int64)
+    frac = np.where((ex == 15) & (frac == 7), 6, frac)
+    return ((sign << 7) | (ex << 3) | frac).astype(np.uint8)
 
 
 @dataclass
@@ -105,10 +122,22 @@ class Workload:
     block_mapping: np.ndarray   # [P, 2] int64 (src, dst) copy-on-write pairs
     seed: int = 0
     meta: Dict = field(default_factory=dict)
+    kv_dtype: int = -1          # pool element type: dtype, or FP8 (codes times the scales)
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+
+    def __post_init__(self):
+        if self.kv_dtype < 0:
+            self.kv_dtype = self.dtype
+
+    @property
+    def fp8(self) -> bool:
+        return self.kv_dtype == FP8
 
     @property
     def esize(self) -> int:
-        return ESIZE[self.dtype]
+        """Bytes per cached K/V element."""
+        return ESIZE[self.kv_dtype]
 
     @property
     def G(self) -> int:
@@ -160,8 +189,14 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
                       seed: int, rng: Optional[np.random.Generator] = None,
                       max_blocks: Optional[int] = None, scale: Optional[float] = None,
                       partition_size: int = 0, shuffle: bool = True,
-                      k_boost_frac: float = 0.0, k_boost: float = 8.0) -> Workload:
-    """Independent sequences, each prefilled with ctx-1 tokens plus one append."""
+                      k_boost_frac: float = 0.0, k_boost: float = 8.0,
+                      kv_fp8: bool = False, k_scale: float = 0.3,
+                      v_scale: float = 0.7) -> Workload:
+    """Independent sequences, each prefilled with ctx-1 tokens plus one append.
+
+    kv_fp8: the pools hold E4M3 codes (value = code * k_scale / v_scale,
+    scales rounded to float32); the query and the new rows keep ``dtype``.
+    """
     if Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
     rng = rng if rng is not None else np.random.Generator(np.random.PCG64(seed))
@@ -187,11 +222,16 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
         tables[b, :len(tb)] = tb
 
     st = _STORAGE[dtype]
+    kvdt = FP8 if kv_fp8 else dtype
     q = round_to_storage(rng.standard_normal((B, Hq, D), dtype=np.float32), dtype).view(st)
-    kc = nan_fill((num_blocks, block_size, Hkv, D), dtype)
-    vc = nan_fill((num_blocks, block_size, Hkv, D), dtype)
+    kc = nan_fill((num_blocks, block_size, Hkv, D), kvdt)
+    vc = nan_fill((num_blocks, block_size, Hkv, D), kvdt)
     for b in range(B):
         n = int(ctx[b]) - 1
+        if kv_fp8:
+            _fill_rows(kc, tables[b], block_size, 0, random_e4m3_codes(rng, (n, Hkv, D)))
+            _fill_rows(vc, tables[b], block_size, 0, random_e4m3_codes(rng, (n, Hkv, D)))
+            continue
         k = rng.standard_normal((n, Hkv, D), dtype=np.float32)
         if k_boost_frac > 0.0:
             k *= np.where(rng.random((n, Hkv, 1)) < k_boost_frac, np.float32(k_boost),
@@ -207,7 +247,9 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
         scale=float(1.0 / math.sqrt(D)) if scale is None else float(scale),
         partition_size=int(partition_size), q=q, k_cache=kc, v_cache=vc,
         block_tables=tables, context_lens=ctx.astype(np.int32), new_key=nk, new_value=nv,
-        slot_mapping=slots, block_mapping=np.zeros((0, 2), dtype=np.int64), seed=seed)
+        slot_mapping=slots, block_mapping=np.zeros((0, 2), dtype=np.int64), seed=seed,
+        kv_dtype=kvdt, k_scale=float(np.float32(k_scale)) if kv_fp8 else 1.0,
+        v_scale=float(np.float32(v_scale)) if kv_fp8 else 1.0)
 
 
 # --------------------------------------------------------------------------
@@ -328,6 +370,7 @@ WORKLOADS = {
     3: "llama3-70b-gqa-bf16",
     4: "long-context-splitk-bf16",
     5: "shared-prefix-sampling-bf16",
+    6: "llama2-7b-fp8kv",
 }
 WORKLOAD_IDS = {v: k for k, v in WORKLOADS.items()}
 
@@ -342,7 +385,7 @@ def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None
     k = WORKLOAD_IDS[which] if isinstance(which, str) else int(which)
     seed = 1000 + k if seed is None else int(seed)
     name = WORKLOADS[k] if batch is None else f"{WORKLOADS[k]}-b{int(batch)}"
-    if batch is not None and k in (2, 3, 4, 5):
+    if batch is not None and k in (2, 3, 4, 5, 6):
         return _make_batch(k, name, seed, int(batch))
     if k == 1:
         return build_decode_case(name, F32, B=4, Hq=4, Hkv=4, D=64, block_size=16,
@@ -370,16 +413,22 @@ def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None
                                         prefix_blocks=64, Hq=32, Hkv=8, D=128,
                                         block_size=16, num_blocks=8192, max_suffix=512,
                                         seed=seed)
+    if k == 6:
+        # the Llama-2-7B batch with an FP8 E4M3 cache: half the bytes per token
+        ctx = rng.integers(128, 2049, size=64)
+        return build_decode_case(name, F16, B=64, Hq=32, Hkv=32, D=128, block_size=16,
+                                 num_blocks=8192, context_lens=ctx, seed=seed, rng=rng,
+                                 max_blocks=128, kv_fp8=True)
     raise KeyError(which)
 
 
 def _make_batch(k: int, name: str, seed: int, B: int) -> Workload:
     rng = np.random.Generator(np.random.PCG64(seed))
-    if k == 2:
+    if k in (2, 6):
         ctx = rng.integers(128, 2049, size=B)
         return build_decode_case(name, F16, B=B, Hq=32, Hkv=32, D=128, block_size=16,
                                  num_blocks=B * 128, context_lens=ctx, seed=seed, rng=rng,
-                                 max_blocks=128)
+                                 max_blocks=128, kv_fp8=k == 6)
     if k == 3:
         ln = rng.lognormal(mean=math.log(1200.0), sigma=0.8, size=B)
         ctx = np.clip(np.rint(ln), 16, 8192).astype(np.int64)
@@ -433,6 +482,14 @@ def shrink_workload(which, seed: int, B: Optional[int] = None, max_ctx: Optional
                                         children=4, prefix_blocks=4, Hq=32, Hkv=8, D=128,
                                         block_size=16, num_blocks=96, max_suffix=40,
                                         seed=seed)
+    if k == 6:
+        B = B or 6
+        hi = max_ctx or 300
+        ctx = rng.integers(1, hi + 1, size=B)
+        nb = int(sum((c + 15) // 16 for c in ctx)) + 7
+        return build_decode_case("llama2-7b-fp8kv-small", F16, B=B, Hq=32, Hkv=32, D=128,
+                                 block_size=16, num_blocks=nb, context_lens=ctx, seed=seed,
+                                 rng=rng, kv_fp8=True)
     raise KeyError(which)
 
 
@@ -448,6 +505,8 @@ def to_torch(w: Workload, device="cpu") -> Dict[str, "object"]:
 
     def el(a):
         t = torch.from_numpy(np.ascontiguousarray(a))
+        if t.dtype == torch.uint8:                 # FP8 codes stay bytes
+            return t.to(device)
         if w.dtype == BF16:
             t = t.view(torch.int16).view(torch.bfloat16) if t.dtype != torch.bfloat16 else t
         return t.to(device)

@@ -333,3 +333,133 @@ def test_copy_blocks_copies_whole_blocks_from_a_snapshot():
         assert np.array_equal(kp[b], k0[b]) and np.array_equal(vp[b], v0[b])
     with pytest.raises(oracle.OracleError):
         oracle.copy_blocks(kp, vp, np.array([[0, 8]]), F32)
+
+
+# -- FP8 (E4M3) pools ------------------------------------------------------------
+def _torch_e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+def test_fp8_decoding_of_every_code_matches_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    got, ref = oracle.widen(codes, oracle.FP8), _torch_e4m3_to_f64(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+    assert np.isnan(got[[0x7F, 0xFF]]).all() and np.isnan(got).sum() == 2
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_fp8_encoding_matches_torch_rounding_in_range():
+    rng = RNG(41)
+    x = np.concatenate([rng.standard_normal(40000).astype(np.float32) * np.float32(s)
+                        for s in (2.0 ** -12, 1e-3, 0.05, 1.0, 20.0, 150.0)])
+    # exact midpoints between neighbouring codes (ties go to the even code)
+    vals = oracle.widen(np.arange(0x7E, dtype=np.uint8), oracle.FP8)
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids])
+    x = x[np.abs(x) < 448]
+    got = oracle.fp8_encode(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+
+
+def test_fp8_encoding_saturates_and_round_trips():
+    special = np.array([448, 449, 463.9, 464, 1e6, np.inf, -448, -1e30, -np.inf, 0.0, -0.0,
+                        2.0 ** -10, 2.0 ** -10 * 1.001, 3 * 2.0 ** -10], dtype=np.float32)
+    assert oracle.fp8_encode(special).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE,
+                                                    0xFE, 0xFE, 0x00, 0x80, 0x00, 0x01, 0x02]
+    assert oracle.fp8_encode(np.array([np.nan], dtype=np.float32))[0] == 0x7F
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    back = oracle.fp8_encode(oracle.widen(finite, oracle.FP8).astype(np.float32))
+    assert np.array_equal(back, finite)
+
+
+def test_reshape_and_cache_fp8_quantises_the_named_slots():
+    rng = RNG(42)
+    nb, bs, hkv, d, T = 6, 16, 2, 32, 5
+    ks, vs = np.float32(0.37), np.float32(0.005)          # V quotients reach past 448
+    for src in (F32, F16, BF16):
+        kp = np.full((nb, bs, hkv, d), 0x7F, dtype=np.uint8)
+        vp = kp.copy()
+        key = _rand(rng, (T, hkv, d), src, scale=3.0)
+        val = _rand(rng, (T, hkv, d), src)
+        slots = np.array([37, -1, 0, 95, 50], dtype=np.int64)
+        oracle.reshape_and_cache_fp8(kp, vp, key, val, src, float(ks), float(vs), slots)
+        # independent path: numpy float32 division, torch's E4M3 cast (saturation by clipping)
+        kx = (storage_to_float64(key, src).astype(np.float32) / ks).clip(-448, 448)
+        vx = (storage_to_float64(val, src).astype(np.float32) / vs).clip(-448, 448)
+        kq = torch.from_numpy(kx).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        vq = torch.from_numpy(vx).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        touched = np.zeros((nb, bs), dtype=bool)
+        for t, s in enumerate(slots):
+            if s < 0:
+                continue
+            assert np.array_equal(kp[s // bs, s % bs], kq[t])
+            assert np.array_equal(vp[s // bs, s % bs], vq[t])
+            touched[s // bs, s % bs] = True
+        assert (kp[~touched] == 0x7F).all() and (vp[~touched] == 0x7F).all()
+        assert np.isin(vp[touched], [0x7E, 0xFE]).any()      # saturated codes occur
+    with pytest.raises(oracle.OracleError):
+        oracle.reshape_and_cache_fp8(kp, vp, key, val, F32, 0.0, 1.0, slots)
+
+
+@pytest.mark.parametrize("qdt,Hq,Hkv,D,bs", [(F16, 8, 2, 32, 4), (BF16, 4, 4, 16, 8),
+                                            (F32, 16, 2, 128, 16)])
+def test_decode_kv_over_fp8_pools_matches_torch_sdpa(qdt, Hq, Hkv, D, bs):
+    from paged_kv_cache_418_b200.workloads import random_e4m3_codes
+    rng = RNG(43 + Hq + D)
+    ctxs = [1, 7, bs, bs + 3, 40]
+    kc = [random_e4m3_codes(rng, (n, Hkv, D)) for n in ctxs]
+    vc = [random_e4m3_codes(rng, (n, Hkv, D)) for n in ctxs]
+    # a paged layout of code pools (block-wise, NaN code in the gaps)
+    nblk = [(n + bs - 1) // bs for n in ctxs]
+    nb = sum(nblk) + 2
+    perm = rng.permutation(nb)
+    kp = np.full((nb, bs, Hkv, D), 0x7F, dtype=np.uint8)
+    vp = kp.copy()
+    tables = np.full((len(ctxs), max(nblk)), -1, dtype=np.int32)
+    used = 0
+    for b, n in enumerate(ctxs):
+        ids = perm[used:used + nblk[b]]
+        used += nblk[b]
+        tables[b, :nblk[b]] = ids
+        pk = np.full((nblk[b] * bs, Hkv, D), 0x7F, dtype=np.uint8)
+        pv = pk.copy()
+        pk[:n], pv[:n] = kc[b], vc[b]
+        kp[ids], vp[ids] = pk.reshape(-1, bs, Hkv, D), pv.reshape(-1, bs, Hkv, D)
+    q = _rand(rng, (len(ctxs), Hq, D), qdt)
+    ks, vs, scale = float(np.float32(0.3)), float(np.float32(0.7)), 1.0 / math.sqrt(D)
+    out = oracle.decode_kv(q, qdt, kp, vp, oracle.FP8, ks, vs, tables, np.array(ctxs), scale)
+    for b in range(len(ctxs)):
+        ref = _sdpa(storage_to_float64(q[b], qdt), _torch_e4m3_to_f64(kc[b]) * ks,
+                    _torch_e4m3_to_f64(vc[b]) * vs, scale)
+        np.testing.assert_allclose(out[b], ref, rtol=0, atol=1e-12)
+
+
+def test_decode_kv_with_one_type_equals_decode():
+    rng = RNG(44)
+    kc = [_rand(rng, (n, 2, 16), BF16) for n in (3, 9)]
+    vc = [_rand(rng, (n, 2, 16), BF16) for n in (3, 9)]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, 4, BF16, rng)
+    q = _rand(rng, (2, 4, 16), BF16)
+    a = oracle.decode(q, kp, vp, BF16, tables, [3, 9], 0.25)
+    b = oracle.decode_kv(q, BF16, kp, vp, BF16, 1.0, 1.0, tables, [3, 9], 0.25)
+    assert np.array_equal(a, b)
+
+
+# -- swap_blocks ---------------------------------------------------------------------
+def test_swap_blocks_moves_whole_blocks_between_pools():
+    rng = RNG(45)
+    src_k, src_v = _rand(rng, (9, 4, 2, 8), F16), _rand(rng, (9, 4, 2, 8), F16)
+    dst_k, dst_v = _rand(rng, (5, 4, 2, 8), F16), _rand(rng, (5, 4, 2, 8), F16)
+    d0k, d0v = dst_k.copy(), dst_v.copy()
+    pairs = np.array([[8, 0], [3, 4], [3, 2]], dtype=np.int64)
+    oracle.swap_blocks(dst_k, dst_v, src_k, src_v, pairs)
+    for s, d in pairs:
+        assert np.array_equal(dst_k[d], src_k[s]) and np.array_equal(dst_v[d], src_v[s])
+    assert np.array_equal(dst_k[[1]], d0k[[1]]) and np.array_equal(dst_v[[1]], d0v[[1]])
+    with pytest.raises(oracle.OracleError):
+        oracle.swap_blocks(dst_k, dst_v, src_k, src_v, np.array([[9, 0]]))
+    with pytest.raises(oracle.OracleError):
+        oracle.swap_blocks(dst_k, dst_v, src_k, src_v, np.array([[0, 5]]))
