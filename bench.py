@@ -71,7 +71,9 @@ def peaks():
 
 
 def config_of(w: W.Workload, world: int, l2_note: str):
-    return {
+    extra = ({"kv_cache": W.DTYPE_NAMES[w.kv_dtype], "k_scale": w.k_scale, "v_scale": w.v_scale}
+             if w.fp8 else {})
+    return {**extra,
         "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.D,
         "block_size": w.block_size, "num_blocks": w.num_blocks, "dtype": W.DTYPE_NAMES[w.dtype],
         "context_lens": {"sum": int(w.context_lens.sum()), "mean": float(w.context_lens.mean()),
@@ -162,8 +164,7 @@ def oracle_sample_rows(w: W.Workload, budget_s: float, rng_seed: int = 0):
     order = rng.permutation(len(all_rows))
     probe = all_rows[order[:8]]
     t = time.perf_counter()
-    oracle.decode(w.q, w.k_cache, w.v_cache, w.dtype, w.block_tables, w.context_lens, w.scale,
-                  rows=probe)
+    oracle_decode_rows(w, w.k_cache, w.v_cache, probe)
     dt = max(time.perf_counter() - t, 1e-4)
     tok = float(w.context_lens[probe[:, 0]].sum())
     per_token = dt / tok
@@ -177,6 +178,27 @@ def oracle_sample_rows(w: W.Workload, budget_s: float, rng_seed: int = 0):
     return np.array(chosen, dtype=np.int32)
 
 
+def oracle_cache_ops(w: W.Workload, kc, vc):
+    """The step's copy_blocks and reshape_and_cache on host pools (oracle)."""
+    import oracle
+    if len(w.block_mapping):
+        oracle.copy_blocks(kc, vc, w.block_mapping, w.kv_dtype)
+    if w.fp8:
+        oracle.reshape_and_cache_fp8(kc, vc, w.new_key, w.new_value, w.dtype, w.k_scale,
+                                     w.v_scale, w.slot_mapping)
+    else:
+        oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
+
+
+def oracle_decode_rows(w: W.Workload, kc, vc, rows):
+    import oracle
+    if w.fp8:
+        return oracle.decode_kv(w.q, w.dtype, kc, vc, oracle.FP8, w.k_scale, w.v_scale,
+                                w.block_tables, w.context_lens, w.scale, rows=rows)
+    return oracle.decode(w.q, kc, vc, w.dtype, w.block_tables, w.context_lens, w.scale,
+                         rows=rows)
+
+
 def run_oracle(w: W.Workload, rows: np.ndarray, reps: int = 1):
     """Time the oracle's share of a step: the step's cache ops on host pools and
     decode of the sampled rows. Returns (seconds, kv_bytes_equivalent)."""
@@ -185,10 +207,8 @@ def run_oracle(w: W.Workload, rows: np.ndarray, reps: int = 1):
     total = 0.0
     for _ in range(reps):
         t = time.perf_counter()
-        if len(w.block_mapping):
-            oracle.copy_blocks(kc, vc, w.block_mapping, w.dtype)
-        oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
-        oracle.decode(w.q, kc, vc, w.dtype, w.block_tables, w.context_lens, w.scale, rows=rows)
+        oracle_cache_ops(w, kc, vc)
+        oracle_decode_rows(w, kc, vc, rows)
         total += time.perf_counter() - t
     frac = float(w.context_lens[rows[:, 0]].sum()) / (w.Hq * float(w.context_lens.sum()))
     return total, w.kv_bytes() * frac * reps
@@ -265,7 +285,7 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     out = torch.empty((w.B, w.Hq, w.D), dtype=tdt, device=dev)
     ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len, w.partition_size)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
-    kernel, P, psize = ops.pa_decode_plan(w.dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
+    kernel, P, psize = ops.pa_decode_plan(w.kv_dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
                                           w.max_context_len, w.partition_size)
     launches_per_step = (1 if len(w.block_mapping) else 0) + 1 + 1 + (1 if P > 1 else 0)
     unique = w.unique_kv_bytes()
@@ -277,13 +297,22 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     def step(ev=None):
         if len(w.block_mapping):
             ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err, stream)
-        ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
-                                 t["slot_mapping"], err, stream)
+        if w.fp8:
+            ops.pa_reshape_and_cache_fp8(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                         w.k_scale, w.v_scale, t["slot_mapping"], err, stream)
+        else:
+            ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                     t["slot_mapping"], err, stream)
         if ev is not None:
             ev[0].record(stream)
-        ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                      t["context_lens"], w.scale, w.max_context_len, w.partition_size, ws, err,
-                      stream)
+        if w.fp8:
+            ops.pa_decode_fp8(out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
+                              t["block_tables"], t["context_lens"], w.scale, w.max_context_len,
+                              w.partition_size, ws, err, stream)
+        else:
+            ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                          t["context_lens"], w.scale, w.max_context_len, w.partition_size, ws,
+                          err, stream)
         if ev is not None:
             ev[1].record(stream)
 

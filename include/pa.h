@@ -24,7 +24,8 @@
  *    err_flag is not NULL). err_flag is a device uint32 the caller zeroes and
  *    reads back when it wants to know.
  *  - Element types: PA_F32, PA_F16 (IEEE binary16), PA_BF16. Pools, queries
- *    and new K/V rows share one element type per call.
+ *    and new K/V rows share one element type per call, except in the FP8
+ *    entry points below, whose pools hold PA_FP8_E4M3 codes.
  *  - Shapes: head size D in {64, 128}; block_size in {16, 32}; Hq a multiple
  *    of Hkv with G = Hq / Hkv in {1, 2, 4, 8, 16}. Query head hq reads KV head
  *    hq / G (contiguous groups; the pages do not say, this is the usual GQA
@@ -145,7 +146,7 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
  *               distinct and must not appear as a source in the same call
  *               (the block manager guarantees it: a fresh block is never
  *               shared); otherwise the result is unspecified.
- * Bit-exact copy.
+ * dtype may also be PA_FP8_E4M3 (pools of codes). Bit-exact copy.
  */
 int pa_copy_blocks(void* key_cache, void* value_cache, int dtype, const int64_t* block_mapping,
                    int num_pairs, int Hkv, int D, int block_size, int num_blocks,
@@ -178,12 +179,88 @@ int pa_decode_static(void* out, int out_dtype, const void* query, const void* ke
                      int D, int block_size, int num_blocks, float scale, int max_context_len,
                      int partition_size, uint32_t* err_flag, void* stream);
 
+/*
+ * FP8 KV cache. The pages give halving the bytes per cached token as the
+ * reason to keep K and V in 8 bits ("vLLM与PagedAttention：大模型推理内存优化
+ * 技术解析" section 6.2; "vLLM 与 LLM 推理部署实战" section 6.1) and fix no
+ * format. Here an FP8 pool holds OCP FP8 E4M3 codes, one byte per element
+ * (sign, 4-bit exponent with bias 7, 3 fraction bits, no infinities, largest
+ * finite value 448), with one float scale per pool: code c stands for
+ * value(c) * scale.
+ */
+#define PA_FP8_E4M3 3 /* pool element type for the FP8 entry points, copy_blocks and swap_blocks */
+
+/*
+ * pa_reshape_and_cache_fp8 -- pa_reshape_and_cache into FP8 pools.
+ * key, value    [T, Hkv, D] of src_dtype (PA_F32, PA_F16 or PA_BF16);
+ * key_cache, value_cache
+ *               [num_blocks, block_size, Hkv, D] uint8 E4M3 codes;
+ * k_scale, v_scale
+ *               positive finite scales: code = E4M3(float(x) / scale), the
+ *               quotient rounded to binary32 (IEEE division) and then to the
+ *               nearest E4M3 value, ties to even, saturating at +-448 (an
+ *               infinite quotient gives +-448, a NaN one 0x7F);
+ * slot_mapping, T, Hkv, D, block_size, num_blocks, err_flag, stream
+ *               as pa_reshape_and_cache.
+ * Returns PA_ERR_SHAPE for a scale that is not positive and finite, otherwise
+ * as pa_reshape_and_cache.
+ */
+int pa_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype, void* key_cache,
+                             void* value_cache, float k_scale, float v_scale,
+                             const int64_t* slot_mapping, int T, int Hkv, int D, int block_size,
+                             int num_blocks, uint32_t* err_flag, void* stream);
+
+/*
+ * pa_decode_fp8 -- pa_decode over FP8 pools: each K element attended is
+ * value(code) * k_scale and each V element value(code) * v_scale.
+ * query         [B, Hq, D] of q_dtype (PA_F32, PA_F16 or PA_BF16);
+ * out           [B, Hq, D] of out_dtype (PA_F32 or q_dtype);
+ * key_cache, value_cache
+ *               [num_blocks, block_size, Hkv, D] uint8 E4M3 codes;
+ * k_scale, v_scale
+ *               positive finite scales (else PA_ERR_SHAPE).
+ * Every other argument, the workspace (sized by pa_workspace_size), the
+ * supported shapes and the error behaviour are those of pa_decode. All shapes
+ * run on the CUDA-core decode kernel.
+ */
+int pa_decode_fp8(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                  const void* value_cache, float k_scale, float v_scale,
+                  const int32_t* block_tables, int max_blocks_per_seq,
+                  const int32_t* context_lens, int B, int Hq, int Hkv, int D, int block_size,
+                  int num_blocks, float scale, int max_context_len, int partition_size,
+                  void* workspace, size_t workspace_bytes, uint32_t* err_flag, void* stream);
+
+/*
+ * pa_swap_blocks -- preemption by swapping: copy whole blocks (K and V)
+ * between two pools, typically the device pool and a pool in page-locked host
+ * memory ("vLLM与PagedAttention：大模型推理内存优化技术解析" section 三: under
+ * memory pressure the block manager moves blocks out to CPU memory, and back).
+ * dst_key, dst_value  [dst_blocks, block_size, Hkv, D] destination pools;
+ * src_key, src_value  [src_blocks, block_size, Hkv, D] source pools;
+ *               each pool is device memory or page-locked host memory that
+ *               the device can address (cudaHostAlloc, torch pin_memory);
+ *               the kernel reads and writes both directly (one launch, no
+ *               copy-engine calls). Source and destination pools must not
+ *               overlap, and the dst ids must be distinct.
+ * dtype         element type of both pools (PA_F32, PA_F16, PA_BF16 or
+ *               PA_FP8_E4M3; only its size matters);
+ * block_mapping [num_pairs, 2] int64 (src id, dst id), device or page-locked
+ *               host memory; a pair with an id out of range is skipped and
+ *               sets PA_DEV_BAD_PAIR.
+ * Returns a pa_status like pa_copy_blocks.
+ */
+int pa_swap_blocks(void* dst_key, void* dst_value, const void* src_key, const void* src_value,
+                   int dtype, const int64_t* block_mapping, int num_pairs, int Hkv, int D,
+                   int block_size, int src_blocks, int dst_blocks, uint32_t* err_flag,
+                   void* stream);
+
 /* Static text for a pa_status value. */
 const char* pa_status_string(int status);
 
 /*
  * pa_decode_plan -- what pa_decode will launch for these arguments, for
- * tools and tests: *kernel = 1 (CUDA-core path) or 2 (tcgen05 GQA path),
+ * tools and tests (dtype = PA_FP8_E4M3 plans pa_decode_fp8, whose pools hold
+ * codes): *kernel = 1 (CUDA-core path) or 2 (tcgen05 GQA path),
  * *num_partitions = partitions per sequence in the split pass (1 = no split),
  * *partition_tokens = their length. Any pointer may be NULL. Returns a
  * pa_status (PA_ERR_UNSUPPORTED etc. for the same reasons pa_decode would).

@@ -35,13 +35,25 @@ namespace {
 
 constexpr int kWarps = 4;
 
-template <typename T, int D, int BS, int GC>
+// VEC consecutive query elements of type TQ, widened to fp32 (16-byte loads).
+template <typename TQ, int VEC>
+__device__ __forceinline__ void load_q(const TQ* p, float* f) {
+  constexpr int N = Vec<TQ>::N;
+  static_assert(VEC % N == 0, "query chunk");
+#pragma unroll
+  for (int c = 0; c < VEC / N; ++c) widen16<TQ>(*reinterpret_cast<const uint4*>(p + c * N), f + c * N);
+}
+
+// TQ: query element type; TC: pool element type (TQ, or FP8 E4M3 codes).
+template <typename TQ, typename TC, int D, int BS, int GC>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_simt_kernel(const DecodeArgs a) {
+  using T = TC;
   constexpr int VEC = Vec<T>::N;               // elements per 16-byte vector
-  constexpr int LPR = D / VEC;                 // lanes per K/V row: 8, 16 or 32
-  constexpr int RPI = 32 / LPR;                // rows per warp instruction: 4, 2 or 1
-  constexpr int RG = (BS / RPI) < 8 ? (BS / RPI) : 8;   // row groups per tile
+  constexpr int LPR = D / VEC;                 // lanes per K/V row: 4, 8, 16 or 32
+  constexpr int RPI = 32 / LPR;                // rows per warp instruction: 8, 4, 2 or 1
+  constexpr int RGMAX = sizeof(T) == 1 ? 4 : 8;           // registers: 16 floats per vector for FP8
+  constexpr int RG = (BS / RPI) < RGMAX ? (BS / RPI) : RGMAX;   // row groups per tile
   constexpr int TILE = RG * RPI;               // tokens per tile (divides BS)
   static_assert(BS % TILE == 0, "tile must divide the block");
 
@@ -82,9 +94,8 @@ decode_simt_kernel(const DecodeArgs a) {
   float qf[GC][VEC];
 #pragma unroll
   for (int g = 0; g < GC; ++g) {
-    uint4 raw = *reinterpret_cast<const uint4*>(
-        reinterpret_cast<const T*>(a.q) + ((size_t)b * a.Hq + hq0 + g) * D + ci * VEC);
-    widen16<T>(raw, qf[g]);
+    load_q<TQ, VEC>(reinterpret_cast<const TQ*>(a.q) + ((size_t)b * a.Hq + hq0 + g) * D + ci * VEC,
+                    qf[g]);
 #pragma unroll
     for (int e = 0; e < VEC; ++e) qf[g][e] *= a.scale_log2;
   }
@@ -223,6 +234,7 @@ decode_simt_kernel(const DecodeArgs a) {
       }
     }
     const size_t row = (size_t)b * a.Hq + hq0 + g;
+    O *= a.v_scale;                              // 1 unless the V pool holds FP8 codes
     if (nparts == 1) {
       store_out(a.out, row * D + d, L > 0.f ? O / L : 0.f, a.out_dtype);
     } else {
@@ -233,31 +245,31 @@ decode_simt_kernel(const DecodeArgs a) {
   }
 }
 
-template <typename T, int D, int BS, int GC>
+template <typename TQ, typename TC, int D, int BS, int GC>
 int launch_t(const DecodeArgs& a, cudaStream_t stream) {
   const int chunks = (a.Hq / a.Hkv) / GC;
   dim3 grid((unsigned)(a.P * chunks), (unsigned)a.Hkv, (unsigned)a.B);
-  const cudaError_t e = launch_k(decode_simt_kernel<T, D, BS, GC>, grid, dim3(kWarps * 32), 0,
-                                 stream, a);
+  const cudaError_t e = launch_k(decode_simt_kernel<TQ, TC, D, BS, GC>, grid, dim3(kWarps * 32),
+                                 0, stream, a);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <typename T, int D, int BS>
+template <typename TQ, typename TC, int D, int BS>
 int launch_gc(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
-  if (G == 1) return launch_t<T, D, BS, 1>(a, stream);
-  if (G == 2) return launch_t<T, D, BS, 2>(a, stream);
-  return launch_t<T, D, BS, 4>(a, stream);      // G = 4, 8, 16: chunks of 4 heads
+  if (G == 1) return launch_t<TQ, TC, D, BS, 1>(a, stream);
+  if (G == 2 || sizeof(TC) == 1) return launch_t<TQ, TC, D, BS, 2>(a, stream);   // FP8: pairs
+  return launch_t<TQ, TC, D, BS, 4>(a, stream);  // G = 4, 8, 16: chunks of 4 heads
 }
 
-template <typename T, int D>
+template <typename TQ, typename TC, int D>
 int launch_bs(const DecodeArgs& a, cudaStream_t stream) {
-  return a.bs == 16 ? launch_gc<T, D, 16>(a, stream) : launch_gc<T, D, 32>(a, stream);
+  return a.bs == 16 ? launch_gc<TQ, TC, D, 16>(a, stream) : launch_gc<TQ, TC, D, 32>(a, stream);
 }
 
-template <typename T>
+template <typename TQ, typename TC>
 int launch_d(const DecodeArgs& a, cudaStream_t stream) {
-  return a.D == 64 ? launch_bs<T, 64>(a, stream) : launch_bs<T, 128>(a, stream);
+  return a.D == 64 ? launch_bs<TQ, TC, 64>(a, stream) : launch_bs<TQ, TC, 128>(a, stream);
 }
 
 // Merge of the split pass, for each (b, hq) row with more than one partition:
@@ -385,9 +397,18 @@ int launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
 
 int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   switch (dtype) {
-    case PA_F32: return launch_d<float>(a, stream);
-    case PA_F16: return launch_d<__half>(a, stream);
-    case PA_BF16: return launch_d<__nv_bfloat16>(a, stream);
+    case PA_F32: return launch_d<float, float>(a, stream);
+    case PA_F16: return launch_d<__half, __half>(a, stream);
+    case PA_BF16: return launch_d<__nv_bfloat16, __nv_bfloat16>(a, stream);
+  }
+  return PA_ERR_DTYPE;
+}
+
+int launch_decode_simt_fp8(const DecodeArgs& a, int q_dtype, cudaStream_t stream) {
+  switch (q_dtype) {
+    case PA_F32: return launch_d<float, __nv_fp8_e4m3>(a, stream);
+    case PA_F16: return launch_d<__half, __nv_fp8_e4m3>(a, stream);
+    case PA_BF16: return launch_d<__nv_bfloat16, __nv_fp8_e4m3>(a, stream);
   }
   return PA_ERR_DTYPE;
 }

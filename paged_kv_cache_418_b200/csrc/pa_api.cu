@@ -27,7 +27,7 @@ bool supported_shape(int Hq, int Hkv, int D, int bs) {
          (G == 1 || G == 2 || G == 4 || G == 8 || G == 16);
 }
 
-int esize_of(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+int esize_of(int dtype) { return dtype == PA_F32 ? 4 : (dtype == PA_FP8_E4M3 ? 1 : 2); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -104,7 +104,7 @@ const char* pa_status_string(int status) {
 
 int pa_decode_plan(int dtype, int B, int Hq, int Hkv, int D, int block_size, int max_context_len,
                    int partition_size, int* kernel, int* num_partitions, int* partition_tokens) {
-  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (dtype < PA_F32 || dtype > PA_FP8_E4M3) return PA_ERR_DTYPE;
   if (B < 0 || max_context_len < 0 || partition_size < 0) return PA_ERR_SHAPE;
   if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
   if (partition_size > 0 && partition_size % block_size) return PA_ERR_SHAPE;
@@ -115,20 +115,28 @@ int pa_decode_plan(int dtype, int B, int Hq, int Hkv, int D, int block_size, int
   return PA_OK;
 }
 
-int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache,
-              const void* value_cache, int dtype, const int32_t* block_tables,
-              int max_blocks_per_seq, const int32_t* context_lens, int B, int Hq, int Hkv, int D,
-              int block_size, int num_blocks, float scale, int max_context_len,
-              int partition_size, void* workspace, size_t workspace_bytes, uint32_t* err_flag,
-              void* stream) {
-  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
-  if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_DTYPE;
+}  // extern "C"
+
+namespace {
+
+bool scale_ok(float x) { return std::isfinite(x) && x > 0.f; }
+
+// Shared body of pa_decode and pa_decode_fp8. q_dtype: query element type;
+// kv_dtype: pool element type (q_dtype itself, or PA_FP8_E4M3 with scales).
+int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                const void* value_cache, int kv_dtype, float k_scale, float v_scale,
+                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                int B, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+                int max_context_len, int partition_size, void* workspace,
+                size_t workspace_bytes, uint32_t* err_flag, void* stream) {
+  if (q_dtype < PA_F32 || q_dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (out_dtype != PA_F32 && out_dtype != q_dtype) return PA_ERR_DTYPE;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0 ||
       max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
     return PA_ERR_SHAPE;
   if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
   if (partition_size > 0 && partition_size % block_size) return PA_ERR_SHAPE;
-  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale) || !scale_ok(k_scale) || !scale_ok(v_scale)) return PA_ERR_SHAPE;
   if (B > 65535 || Hkv > 65535) return PA_ERR_UNSUPPORTED;
   if (B == 0) return PA_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
@@ -136,14 +144,16 @@ int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_ALIGN;
 
-  DecodePlan p = plan_decode(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  DecodePlan p =
+      plan_decode(kv_dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
   DecodeArgs a{};
   a.out = out; a.out_dtype = out_dtype; a.q = query;
   a.k_cache = key_cache; a.v_cache = value_cache;
   a.block_tables = block_tables; a.max_blocks = max_blocks_per_seq;
   a.context_lens = context_lens;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.bs = block_size; a.num_blocks = num_blocks;
-  a.scale_log2 = scale * kLog2e;
+  a.scale_log2 = scale * kLog2e * k_scale;      // k_scale = 1 unless K holds FP8 codes
+  a.v_scale = v_scale;
   a.max_context_len = max_context_len;
   a.P = p.P; a.psize = p.psize;
   a.err_flag = err_flag;
@@ -159,9 +169,75 @@ int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache
     a.ws_l = reinterpret_cast<float*>(w + up(rows * D * 4) + up(rows * 4));
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, s) : launch_decode_simt(a, dtype, s);
+  int rc;
+  if (kv_dtype == PA_FP8_E4M3) rc = launch_decode_simt_fp8(a, q_dtype, s);
+  else rc = p.kernel == 2 ? launch_decode_tc(a, q_dtype, s) : launch_decode_simt(a, q_dtype, s);
   if (rc == PA_OK && p.P > 1) rc = launch_merge(a, s);
   return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache,
+              const void* value_cache, int dtype, const int32_t* block_tables,
+              int max_blocks_per_seq, const int32_t* context_lens, int B, int Hq, int Hkv, int D,
+              int block_size, int num_blocks, float scale, int max_context_len,
+              int partition_size, void* workspace, size_t workspace_bytes, uint32_t* err_flag,
+              void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  return decode_impl(out, out_dtype, query, dtype, key_cache, value_cache, dtype, 1.f, 1.f,
+                     block_tables, max_blocks_per_seq, context_lens, B, Hq, Hkv, D, block_size,
+                     num_blocks, scale, max_context_len, partition_size, workspace,
+                     workspace_bytes, err_flag, stream);
+}
+
+int pa_decode_fp8(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                  const void* value_cache, float k_scale, float v_scale,
+                  const int32_t* block_tables, int max_blocks_per_seq,
+                  const int32_t* context_lens, int B, int Hq, int Hkv, int D, int block_size,
+                  int num_blocks, float scale, int max_context_len, int partition_size,
+                  void* workspace, size_t workspace_bytes, uint32_t* err_flag, void* stream) {
+  return decode_impl(out, out_dtype, query, q_dtype, key_cache, value_cache, PA_FP8_E4M3,
+                     k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens, B, Hq,
+                     Hkv, D, block_size, num_blocks, scale, max_context_len, partition_size,
+                     workspace, workspace_bytes, err_flag, stream);
+}
+
+int pa_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype, void* key_cache,
+                             void* value_cache, float k_scale, float v_scale,
+                             const int64_t* slot_mapping, int T, int Hkv, int D, int block_size,
+                             int num_blocks, uint32_t* err_flag, void* stream) {
+  if (src_dtype < PA_F32 || src_dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (T < 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0) return PA_ERR_SHAPE;
+  if (!scale_ok(k_scale) || !scale_ok(v_scale)) return PA_ERR_SHAPE;
+  if (!supported_shape(Hkv, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (T == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_ALIGN;
+  return launch_reshape_and_cache_fp8(key, value, src_dtype, key_cache, value_cache, k_scale,
+                                      v_scale, slot_mapping, T, Hkv, D, block_size, num_blocks,
+                                      err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int pa_swap_blocks(void* dst_key, void* dst_value, const void* src_key, const void* src_value,
+                   int dtype, const int64_t* block_mapping, int num_pairs, int Hkv, int D,
+                   int block_size, int src_blocks, int dst_blocks, uint32_t* err_flag,
+                   void* stream) {
+  if (dtype < PA_F32 || dtype > PA_FP8_E4M3) return PA_ERR_DTYPE;
+  if (num_pairs < 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || src_blocks < 0 ||
+      dst_blocks < 0)
+    return PA_ERR_SHAPE;
+  if (!supported_shape(Hkv, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_key || !dst_value || !src_key || !src_value || !block_mapping) return PA_ERR_NULL;
+  if (!aligned16(dst_key) || !aligned16(dst_value) || !aligned16(src_key) || !aligned16(src_value))
+    return PA_ERR_ALIGN;
+  return launch_swap_blocks(dst_key, dst_value, src_key, src_value, esize_of(dtype),
+                            block_mapping, num_pairs, Hkv, D, block_size, src_blocks, dst_blocks,
+                            err_flag, static_cast<cudaStream_t>(stream));
 }
 
 int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
@@ -182,7 +258,7 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
 int pa_copy_blocks(void* key_cache, void* value_cache, int dtype, const int64_t* block_mapping,
                    int num_pairs, int Hkv, int D, int block_size, int num_blocks,
                    uint32_t* err_flag, void* stream) {
-  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (dtype < PA_F32 || dtype > PA_FP8_E4M3) return PA_ERR_DTYPE;
   if (num_pairs < 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0)
     return PA_ERR_SHAPE;
   if (!supported_shape(Hkv, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;

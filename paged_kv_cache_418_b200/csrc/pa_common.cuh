@@ -4,6 +4,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,6 +40,23 @@ template <> __device__ __forceinline__ void widen16<__nv_bfloat16>(const uint4& 
   for (int i = 0; i < 4; ++i) {
     f[2 * i] = __uint_as_float(w[i] << 16);
     f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+template <> __device__ __forceinline__ void widen16<__nv_fp8_e4m3>(const uint4& v, float* f) {
+  // E4M3 -> binary16 is exact (every E4M3 value, subnormals included, is a
+  // normal or subnormal half), and half -> fp32 is exact.
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+          static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * k)) & 0xffffu), __NV_E4M3);
+      const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&h));
+      f[4 * i + 2 * k] = t.x;
+      f[4 * i + 2 * k + 1] = t.y;
+    }
   }
 }
 

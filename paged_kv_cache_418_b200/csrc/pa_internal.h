@@ -26,6 +26,7 @@ struct DecodeArgs {
   float* ws_acc;        // [B, P, Hq, D] unnormalised partial outputs (P > 1)
   float* ws_m;          // [B, P, Hq] partial max, log2 domain
   float* ws_l;          // [B, P, Hq] partial sum of exp2(s - m)
+  float v_scale;        // value of one V unit (FP8 pools; 1 otherwise); K's is in scale_log2
   uint32_t* err_flag;
 };
 
@@ -41,6 +42,8 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max
 size_t workspace_bytes_for(int B, int Hq, int D, int P);
 
 int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream);
+// FP8 E4M3 pools, query of q_dtype
+int launch_decode_simt_fp8(const DecodeArgs& a, int q_dtype, cudaStream_t stream);
 int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream);
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 int launch_merge(const DecodeArgs& a, cudaStream_t stream);
@@ -52,5 +55,14 @@ int launch_reshape_and_cache(const void* key, const void* value, void* key_cache
 int launch_copy_blocks(void* key_cache, void* value_cache, int esize,
                        const int64_t* block_mapping, int num_pairs, int Hkv, int D,
                        int block_size, int num_blocks, uint32_t* err_flag, cudaStream_t stream);
+int launch_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype,
+                                 void* key_cache, void* value_cache, float k_scale,
+                                 float v_scale, const int64_t* slot_mapping, int T, int Hkv,
+                                 int D, int block_size, int num_blocks, uint32_t* err_flag,
+                                 cudaStream_t stream);
+int launch_swap_blocks(void* dst_key, void* dst_value, const void* src_key,
+                       const void* src_value, int esize, const int64_t* block_mapping,
+                       int num_pairs, int Hkv, int D, int block_size, int src_blocks,
+                       int dst_blocks, uint32_t* err_flag, cudaStream_t stream);
 
 }  // namespace pa

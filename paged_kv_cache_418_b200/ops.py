@@ -17,10 +17,11 @@ import torch
 
 from . import _build
 
-PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+PA_F32, PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2, 3
 PA_OK = 0
 PA_DEV_BAD_BLOCK_ID, PA_DEV_BAD_CTX, PA_DEV_BAD_SLOT, PA_DEV_BAD_PAIR = 1, 2, 4, 8
-_TORCH_TO_PA = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}
+_TORCH_TO_PA = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16,
+                torch.uint8: PA_FP8_E4M3, torch.float8_e4m3fn: PA_FP8_E4M3}
 
 
 class PAError(RuntimeError):
@@ -48,6 +49,13 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_plan.restype = I
     lib.pa_decode_static.argtypes = [P, I, P, P, P, I, P, I, P, I, I, I, I, I, I, F, I, I, P, P]
     lib.pa_decode_static.restype = I
+    lib.pa_decode_fp8.argtypes = [P, I, P, I, P, P, F, F, P, I, P, I, I, I, I, I, I, F, I, I, P, S,
+                                  P, P]
+    lib.pa_decode_fp8.restype = I
+    lib.pa_reshape_and_cache_fp8.argtypes = [P, P, I, P, P, F, F, P, I, I, I, I, I, P, P]
+    lib.pa_reshape_and_cache_fp8.restype = I
+    lib.pa_swap_blocks.argtypes = [P, P, P, P, I, P, I, I, I, I, I, I, P, P]
+    lib.pa_swap_blocks.restype = I
     return lib
 
 
@@ -156,6 +164,56 @@ def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor,
                             _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_copy_blocks", rc)
+
+
+def pa_decode_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                  value_cache: torch.Tensor, k_scale: float, v_scale: float,
+                  block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                  max_context_len: int, partition_size: int = 0,
+                  workspace: Optional[torch.Tensor] = None,
+                  err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out [B,Hq,D] <- paged decode attention over FP8 E4M3 pools (uint8 codes)."""
+    B, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    rc = LIB.pa_decode_fp8(
+        _ptr(out), pa_dtype(out), _ptr(query), pa_dtype(query), _ptr(key_cache),
+        _ptr(value_cache), float(k_scale), float(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, block_size, num_blocks,
+        float(scale), int(max_context_len), int(partition_size), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_decode_fp8", rc)
+
+
+def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                             value_cache: torch.Tensor, k_scale: float, v_scale: float,
+                             slot_mapping: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                             stream=None) -> None:
+    """Quantise new K/V rows [T,Hkv,D] to E4M3 codes and scatter them into the pools."""
+    num_blocks, block_size, Hkv, D = key_cache.shape
+    T = slot_mapping.shape[0]
+    rc = LIB.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), pa_dtype(key), _ptr(key_cache),
+                                      _ptr(value_cache), float(k_scale), float(v_scale),
+                                      _ptr(slot_mapping), T, Hkv, D, block_size, num_blocks,
+                                      _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_reshape_and_cache_fp8", rc)
+
+
+def pa_swap_blocks(dst_key: torch.Tensor, dst_value: torch.Tensor, src_key: torch.Tensor,
+                   src_value: torch.Tensor, block_mapping: torch.Tensor,
+                   err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Copy whole blocks src pool -> dst pool ((src id, dst id) rows of block_mapping);
+    either pool may be pinned host memory."""
+    src_blocks, block_size, Hkv, D = src_key.shape
+    dst_blocks = dst_key.shape[0]
+    P = block_mapping.shape[0]
+    rc = LIB.pa_swap_blocks(_ptr(dst_key), _ptr(dst_value), _ptr(src_key), _ptr(src_value),
+                            pa_dtype(src_key), _ptr(block_mapping), P, Hkv, D, block_size,
+                            src_blocks, dst_blocks, _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_swap_blocks", rc)
 
 
 def workspace_for(query: torch.Tensor, key_cache: torch.Tensor, max_context_len: int,

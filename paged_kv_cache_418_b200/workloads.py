@@ -17,10 +17,10 @@ Value recipe (all workloads)
     NaN, so a kernel that reads outside what it should shows it in its output.
   * Unused block-table entries are -1.
   * FP8 pools (E4M3 codes, one byte each) are drawn as bit fields, not by
-    quantising anything: sign ~ U{0,1}, exponent field ~ round(N(7, 1.5))
-    clipped to [0, 15], fraction ~ U{0..7} (the NaN pattern 15/7 becomes
-    15/6), so cached values sit around 1 in magnitude before the pool's
-    scale. Empty slots hold the NaN code 0x7F. The new K/V rows of the step
+    quantising anything: sign ~ U{0,1}, exponent field ~ round(N(7, 1))
+    clipped to [3, 10], fraction ~ U{0..7}, so cached values lie in
+    [2^-4, 16) in magnitude, around 1, before the pool's scale (like the
+    N(0, 1) values of the 16-bit pools). Empty slots hold the NaN code 0x7F. The new K/V rows of the step
     stay N(0, 1) in the query's type: reshape_and_cache_fp8 quantises them.
 
 Layout recipe
@@ -87,10 +87,13 @@ def nan_fill(shape, dtype: int) -> np.ndarray:
     return np.full(shape, _NAN_BITS[dtype], dtype=np.uint16).view(_STORAGE[dtype])
 
 
-def random_e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
-    """E4M3 codes drawn field by field (see the module notes); never NaN."""
+def random_e4m3_codes(rng: np.random.Generator, shape, lo: int = 3, hi: int = 10) -> np.ndarray:
+    """E4M3 codes drawn field by field (see the module notes); never NaN.
+
+    The exponent field lies in [lo, hi]; lo=0, hi=15 reaches every finite code.
+    """
     sign = rng.integers(0, 2, size=shape, dtype=np.int64)
-    ex = np.clip(np.rint(rng.normal(7.0, 1.5, size=shape)), 0, 15).astype(np.int64)
+    ex = np.clip(np.rint(rng.normal(7.0, 1.0, size=shape)), lo, hi).astype(np.int64)
     frac = rng.integers(0, 8, size=shape, dtype=np.int64)
     frac = np.where((ex == 15) & (frac == 7), 6, frac)
     return ((sign << 7) | (ex << 3) | frac).astype(np.uint8)

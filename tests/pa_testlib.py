@@ -6,7 +6,9 @@ for fp16 / bf16 inputs when the kernel writes fp32 output. When it writes the
 input type, the fp32 result within that bound is then rounded once more, so
 |out - oracle| <= ATOL + ulp(out) / 2 (a correctly rounded 16-bit output can by
 itself be more than 4e-3 from the exact value: bf16 values in [2, 4) are 2^-6
-apart).
+apart). With FP8 pools the bound is the query type's: the oracle reads the
+very codes the kernel reads (times the same scales), so only the kernel's
+fp32 arithmetic and the output rounding separate the two.
 """
 
 from __future__ import annotations
@@ -16,7 +18,7 @@ import torch
 
 import oracle
 from paged_kv_cache_418_b200 import ops
-from paged_kv_cache_418_b200.workloads import BF16, F16, F32, Workload, to_torch
+from paged_kv_cache_418_b200.workloads import BF16, F16, F32, FP8, Workload, to_torch
 
 ATOL = {F32: 1e-5, F16: 4e-3, BF16: 4e-3}
 TORCH_DT = {F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}
@@ -35,15 +37,24 @@ def device_step(w: Workload, t=None, out_dtype=None, partition_size=None, err=No
     if do_cache_ops:
         if len(w.block_mapping):
             ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err, stream)
-        ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
-                                 t["slot_mapping"], err, stream)
+        if w.fp8:
+            ops.pa_reshape_and_cache_fp8(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                         w.k_scale, w.v_scale, t["slot_mapping"], err, stream)
+        else:
+            ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                     t["slot_mapping"], err, stream)
     odt = TORCH_DT[w.dtype] if out_dtype is None else out_dtype
     out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=odt, device=dev)
     psize = w.partition_size if partition_size is None else partition_size
     mcl = w.max_context_len if max_context_len is None else max_context_len
     ws = ops.workspace_for(t["q"], t["k_cache"], mcl, psize)
-    ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                  t["context_lens"], w.scale, mcl, psize, ws, err, stream)
+    if w.fp8:
+        ops.pa_decode_fp8(out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
+                          t["block_tables"], t["context_lens"], w.scale, mcl, psize, ws, err,
+                          stream)
+    else:
+        ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                      t["context_lens"], w.scale, mcl, psize, ws, err, stream)
     t["workspace"] = ws
     t["err"] = err
     return out, t
@@ -54,9 +65,18 @@ def oracle_step(w: Workload, rows=None, do_cache_ops=True):
     kc, vc = w.k_cache.copy(), w.v_cache.copy()
     if do_cache_ops:
         if len(w.block_mapping):
-            oracle.copy_blocks(kc, vc, w.block_mapping, w.dtype)
-        oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
-    out = oracle.decode(w.q, kc, vc, w.dtype, w.block_tables, w.context_lens, w.scale, rows=rows)
+            oracle.copy_blocks(kc, vc, w.block_mapping, w.kv_dtype)
+        if w.fp8:
+            oracle.reshape_and_cache_fp8(kc, vc, w.new_key, w.new_value, w.dtype, w.k_scale,
+                                         w.v_scale, w.slot_mapping)
+        else:
+            oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
+    if w.fp8:
+        out = oracle.decode_kv(w.q, w.dtype, kc, vc, FP8, w.k_scale, w.v_scale, w.block_tables,
+                               w.context_lens, w.scale, rows=rows)
+    else:
+        out = oracle.decode(w.q, kc, vc, w.dtype, w.block_tables, w.context_lens, w.scale,
+                            rows=rows)
     return out, kc, vc
 
 
@@ -82,10 +102,14 @@ def assert_attention_close(got: torch.Tensor, ref: np.ndarray, dtype: int, what=
 
 def bits(t: torch.Tensor) -> torch.Tensor:
     """Bit pattern view for exact comparisons (NaN payloads included)."""
+    if t.dtype == torch.uint8:
+        return t
     return t.view(torch.int32) if t.dtype == torch.float32 else t.view(torch.int16)
 
 
 def host_bits(a: np.ndarray) -> torch.Tensor:
+    if a.dtype == np.uint8:
+        return torch.from_numpy(np.ascontiguousarray(a))
     v = a.view(np.int32) if a.dtype == np.float32 else a.view(np.int16)
     return torch.from_numpy(np.ascontiguousarray(v))
 
