@@ -18,6 +18,10 @@ over ranks. Rank 0 prints one JSON line.
 
 --impl reference times the fp64 CPU oracle (the only other implementation
 there is) on a bounded sample of the same workload, on rank 0.
+
+--swap measures swap_blocks instead (preemption by swapping): whole blocks of
+the Llama-2-7B-shaped pool moved device -> page-locked host and back, against
+a plain cudaMemcpyAsync of the same bytes timed in the same run.
 """
 
 from __future__ import annotations
@@ -55,6 +59,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=None)
     p.add_argument("--batch", type=int, default=None,
                    help="fewer sequences of the same workload (profiling captures)")
+    p.add_argument("--swap", action="store_true",
+                   help="measure swap_blocks (device <-> pinned host) instead of the decode step")
     return p.parse_args()
 
 
@@ -251,12 +257,17 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources a decode path is built from (its kernels + shared headers)."""
+    """Hash of what a decode path's device code is built from: its kernel files,
+    the device helpers, and the launch-argument struct (declarations of other
+    entry points do not change the kernels, so they are left out)."""
+    import re
     csrc = os.path.join(ROOT, "paged_kv_cache_418_b200", "csrc")
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES[kernel] + ["pa_common.cuh", "pa_internal.h"]:
+    for f in KERNEL_SOURCES[kernel] + ["pa_common.cuh"]:
         h.update(open(os.path.join(csrc, f), "rb").read())
-    h.update(open(os.path.join(ROOT, "include", "pa.h"), "rb").read())
+    internal = open(os.path.join(csrc, "pa_internal.h")).read()
+    m = re.search(r"struct DecodeArgs \{.*?\};", internal, re.S)
+    h.update((m.group(0) if m else internal).encode())
     return h.hexdigest()[:16]
 
 
@@ -469,8 +480,103 @@ def cpu_baseline(w: W.Workload, budget_s: float = 10.0):
                        f"by the rows' share of KV bytes")}
 
 
+SWAP_METRIC = "swap_blocks GB/s (device <-> page-locked host)"
+
+
+def swap_arm(args, rank: int, world: int, local_rank: int):
+    """Blocks of the Llama-2-7B-shaped pool (16 tokens x 32 heads x 128, fp16:
+    128 KiB per block per pool) swapped out to a pinned host pool and back in."""
+    import torch
+    from paged_kv_cache_418_b200 import ops
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    nd, nh, bs, hkv, d = 8192, 2048, 16, 32, 128
+    rng = np.random.default_rng(rank_seed(7, rank))
+    dk = torch.randn((nd, bs, hkv, d), dtype=torch.float16, device=dev)
+    dv = torch.randn((nd, bs, hkv, d), dtype=torch.float16, device=dev)
+    hk = torch.empty((nh, bs, hkv, d), dtype=torch.float16).pin_memory()
+    hv = torch.empty((nh, bs, hkv, d), dtype=torch.float16).pin_memory()
+    out_map = np.stack([rng.choice(nd, nh, replace=False), rng.permutation(nh)], 1)
+    in_map = np.stack([rng.permutation(nh), rng.choice(nd, nh, replace=False)], 1)
+    out_map = torch.from_numpy(out_map.astype(np.int64)).to(dev)
+    in_map = torch.from_numpy(in_map.astype(np.int64)).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    moved = 2 * nh * bs * hkv * d * 2                 # K + V bytes per direction
+
+    def timed(fn, reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    swap_out = lambda: ops.pa_swap_blocks(hk, hv, dk, dv, out_map, err, stream)
+    swap_in = lambda: ops.pa_swap_blocks(dk, dv, hk, hv, in_map, err, stream)
+    flat_d = dk[:nh].view(-1)
+    flat_h = hk.view(-1)
+    copy_out = lambda: (flat_h.copy_(flat_d, non_blocking=True), hv.view(-1).copy_(dv[:nh].view(-1), non_blocking=True))
+    copy_in = lambda: (flat_d.copy_(flat_h, non_blocking=True), dv[:nh].view(-1).copy_(hv.view(-1), non_blocking=True))
+    K = max(1, min(args.steps, 20))
+    for _ in range(max(3, args.warmup)):
+        swap_out(); swap_in()
+    torch.cuda.synchronize(dev)
+    t_out, t_in = timed(swap_out, K), timed(swap_in, K)
+    c_out, c_in = timed(copy_out, K), timed(copy_in, K)
+    torch.cuda.synchronize(dev)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+    (t_out, t_in) = max_over_ranks([t_out, t_in], world, dev)
+    g = lambda ms: moved / (ms / 1e3) / 1e9
+    value = 2 * moved * world / ((t_out + t_in) / 1e3) / 1e9
+    peak = 2 * moved / ((c_out + c_in) / 1e3) / 1e9
+    # oracle: the same block copies between two host pools, on a sample of blocks
+    import oracle
+    n_s = 256
+    sk, sv = hk[:n_s].numpy(), hv[:n_s].numpy()
+    tk, tv = np.empty_like(sk), np.empty_like(sv)
+    pairs = np.stack([np.arange(n_s), np.random.default_rng(0).permutation(n_s)], 1)
+    t0, reps = time.perf_counter(), 0
+    while time.perf_counter() - t0 < 2.0:
+        oracle.swap_blocks(tk, tv, sk, sv, pairs)
+        reps += 1
+    cpu = 2 * n_s * bs * hkv * d * 2 * reps / (time.perf_counter() - t0) / 1e9
+    return {
+        "metric": SWAP_METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": max(3, args.warmup), "ms_per_step": round(t_out + t_in, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": "swap llama2-7b-shaped blocks", "blocks_per_direction": nh,
+                   "block_bytes_k_plus_v": 2 * bs * hkv * d * 2, "device_pool_blocks": nd,
+                   "mapping": "random distinct device ids <-> permuted host ids"},
+        "swap_out_gbs": round(g(t_out), 2), "swap_in_gbs": round(g(t_in), 2),
+        "roofline": {"bound": "host-link", "achieved": round(2 * moved / ((t_out + t_in) / 1e3) / 1e9, 2),
+                     "peak": round(peak, 2), "unit": "GB/s",
+                     "frac": round(peak and (2 * moved / ((t_out + t_in) / 1e3) / 1e9) / peak, 4),
+                     "traffic": None,
+                     "peak_source": "cudaMemcpyAsync of the same bytes (contiguous, copy engine), this run",
+                     "memcpy_out_gbs": round(g(c_out), 2), "memcpy_in_gbs": round(g(c_in), 2)},
+        "gpu_launches": 2 * K,
+        "e2e": {"value": round(value, 2), "unit": "GB/s", "h2d_bytes_per_step": moved,
+                "d2h_bytes_per_step": moved},
+        "cpu_baseline": {"value": round(cpu, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{n_s} blocks host->host, {reps} repetitions in 2 s"},
+    }
+
+
 def main():
     args = parse()
+    if args.swap:
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if args.impl == "reference" or world > 1:
+            return 0 if rank else (print(json.dumps({"impl": args.impl, "unavailable":
+                "swap measurement runs on one GPU with --impl ours"})) or 0)
+        line = swap_arm(args, rank, world, int(os.environ.get("LOCAL_RANK", "0")))
+        print(json.dumps(line), flush=True)
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -35,6 +35,16 @@ namespace {
 
 constexpr int kWarps = 4;
 
+// Packed fp32x2 FMA (two lanes of fp32 per instruction on sm_100).
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  uint64_t d = (uint64_t)__float_as_uint(d0) | ((uint64_t)__float_as_uint(d1) << 32);
+  const uint64_t a = (uint64_t)__float_as_uint(a0) | ((uint64_t)__float_as_uint(a1) << 32);
+  const uint64_t b = (uint64_t)__float_as_uint(b0) | ((uint64_t)__float_as_uint(b1) << 32);
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+  d0 = __uint_as_float((uint32_t)d);
+  d1 = __uint_as_float((uint32_t)(d >> 32));
+}
+
 // VEC consecutive query elements of type TQ, widened to fp32 (16-byte loads).
 template <typename TQ, int VEC>
 __device__ __forceinline__ void load_q(const TQ* p, float* f) {
@@ -151,10 +161,18 @@ decode_simt_kernel(const DecodeArgs a) {
       widen16<T>(kr[r], kf);
 #pragma unroll
       for (int g = 0; g < GC; ++g) {
-        float d0 = 0.f;
+        if constexpr (sizeof(T) == 1) {
+          // FP8 rows carry twice the elements per byte: packed FMAs halve the issue
+          float d0 = 0.f, d1 = 0.f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) d0 = fmaf(qf[g][e], kf[e], d0);
-        s[r][g] = d0;
+          for (int e = 0; e < VEC; e += 2) fma2(d0, d1, qf[g][e], qf[g][e + 1], kf[e], kf[e + 1]);
+          s[r][g] = d0 + d1;
+        } else {
+          float d0 = 0.f;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) d0 = fmaf(qf[g][e], kf[e], d0);
+          s[r][g] = d0;
+        }
       }
     }
 #pragma unroll
@@ -191,9 +209,16 @@ decode_simt_kernel(const DecodeArgs a) {
       float vf[VEC];
       widen16<T>(vr[r], vf);
 #pragma unroll
-      for (int g = 0; g < GC; ++g)
+      for (int g = 0; g < GC; ++g) {
+        if constexpr (sizeof(T) == 1) {
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[g][e] = fmaf(s[r][g], vf[e], acc[g][e]);
+          for (int e = 0; e < VEC; e += 2)
+            fma2(acc[g][e], acc[g][e + 1], s[r][g], s[r][g], vf[e], vf[e + 1]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[g][e] = fmaf(s[r][g], vf[e], acc[g][e]);
+        }
+      }
     }
   }
 
@@ -258,8 +283,12 @@ template <typename TQ, typename TC, int D, int BS>
 int launch_gc(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   if (G == 1) return launch_t<TQ, TC, D, BS, 1>(a, stream);
-  if (G == 2 || sizeof(TC) == 1) return launch_t<TQ, TC, D, BS, 2>(a, stream);   // FP8: pairs
-  return launch_t<TQ, TC, D, BS, 4>(a, stream);  // G = 4, 8, 16: chunks of 4 heads
+  if constexpr (sizeof(TC) == 1) {
+    return launch_t<TQ, TC, D, BS, 2>(a, stream);   // FP8: pairs of heads (registers)
+  } else {
+    if (G == 2) return launch_t<TQ, TC, D, BS, 2>(a, stream);
+    return launch_t<TQ, TC, D, BS, 4>(a, stream);   // G = 4, 8, 16: chunks of 4 heads
+  }
 }
 
 template <typename TQ, typename TC, int D>
