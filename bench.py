@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=None)
     p.add_argument("--batch", type=int, default=None,
                    help="fewer sequences of the same workload (profiling captures)")
+    p.add_argument("--shared-prefix", action="store_true",
+                   help="decode the shared-prefix workload with pa_decode_shared_prefix")
     p.add_argument("--swap", action="store_true",
                    help="measure swap_blocks (device <-> pinned host) instead of the decode step")
     return p.parse_args()
@@ -294,11 +296,23 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     tdt = t["torch_dtype"]
     stream = torch.cuda.current_stream(dev)
     out = torch.empty((w.B, w.Hq, w.D), dtype=tdt, device=dev)
-    ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len, w.partition_size)
+    cascade = bool(getattr(args, "shared_prefix", False))
+    if cascade:
+        if "prefix_blocks" not in w.meta:
+            raise SystemExit("--shared-prefix needs a workload with groups (shared-prefix-sampling-bf16)")
+        ng, nc, pb = w.meta["groups"], w.meta["children"], w.meta["prefix_blocks"]
+        g_off = torch.arange(0, ng * nc + 1, nc, dtype=torch.int32, device=dev)
+        g_mem = torch.arange(ng * nc, dtype=torch.int32, device=dev)
+        g_shared = torch.full((w.B,), pb, dtype=torch.int32, device=dev)
+        ws = ops.shared_prefix_workspace_for(t["q"], t["k_cache"], w.max_context_len, pb,
+                                             w.partition_size)
+    else:
+        ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len, w.partition_size)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     kernel, P, psize = ops.pa_decode_plan(w.kv_dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
                                           w.max_context_len, w.partition_size)
-    launches_per_step = (1 if len(w.block_mapping) else 0) + 1 + 1 + (1 if P > 1 else 0)
+    launches_per_step = (1 if len(w.block_mapping) else 0) + 1 + 1 + (1 if P > 1 or cascade else 0) \
+        + (1 if cascade else 0)
     unique = w.unique_kv_bytes()
     flush = unique < 2 * L2_BYTES
     l2_note = ("L2 flushed before every step (workload smaller than 2x L2)" if flush else
@@ -316,7 +330,11 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
                                      t["slot_mapping"], err, stream)
         if ev is not None:
             ev[0].record(stream)
-        if w.fp8:
+        if cascade:
+            ops.pa_decode_shared_prefix(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                        t["context_lens"], g_shared, g_off, g_mem, nc, pb, w.scale,
+                                        w.max_context_len, w.partition_size, ws, err, stream)
+        elif w.fp8:
             ops.pa_decode_fp8(out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
                               t["block_tables"], t["context_lens"], w.scale, w.max_context_len,
                               w.partition_size, ws, err, stream)
@@ -406,8 +424,10 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     kv = w.kv_bytes()
     value = job_value(kv, K, world, ms)
     peak, peak_src = peaks()
-    achieved = kv / (dec_ms / 1e3) / 1e9
-    kname = {1: "cuda-core", 2: "tcgen05"}[kernel]
+    kname = {1: "cuda-core", 2: "tcgen05"}[kernel] if not cascade else "shared-prefix"
+    # the cascade reads each distinct K/V byte once: its algorithmic bytes are the distinct ones
+    alg = w.unique_kv_bytes() if cascade else kv
+    achieved = alg / (dec_ms / 1e3) / 1e9
     traffic = traffic_record(kname, w)
     e2e_value = job_value(kv, Ke, world, e_ms)
     line = {
@@ -419,13 +439,15 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
         "pct_of_hbm_peak": round(100.0 * (value / world) / peak, 2),
         "seq_steps_per_s": round(w.B * K * world / (ms / 1e3), 1),
         "decode_us": round(dec_ms * 1e3, 2),
-        "decode_plan": {"kernel": {1: "cuda-core", 2: "tcgen05"}[kernel], "partitions": P,
+        "decode_plan": {"kernel": kname if cascade else {1: "cuda-core", 2: "tcgen05"}[kernel],
+                        "partitions": P,
                         "partition_tokens": psize},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_source": f"hbm_gbs ({peak_src})",
-                     "kernel": "pa_decode (partition pass + merge), per launch",
-                     "algorithmic_bytes": kv},
+                     "kernel": ("pa_decode_shared_prefix (suffix pass + prefix pass + merge)"
+                                if cascade else "pa_decode (partition pass + merge)") + ", per launch",
+                     "algorithmic_bytes": alg},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,

@@ -254,6 +254,46 @@ int pa_swap_blocks(void* dst_key, void* dst_value, const void* src_key, const vo
                    int block_size, int src_blocks, int dst_blocks, uint32_t* err_flag,
                    void* stream);
 
+/*
+ * pa_decode_shared_prefix -- pa_decode for a batch whose sequences come in
+ * groups that share the leading blocks of their block tables: the sequences
+ * forked from one prompt for parallel sampling share its blocks
+ * ("五十三：vLLM-PagedAttention" section 17; the copy-on-write sharing of
+ * "vLLM 与 LLM 推理部署实战" section 2.2). The shared blocks are read once per
+ * group, for the queries of all its members together (tensor cores), each
+ * sequence's own blocks once, and the two parts are merged (split-context
+ * merge). The result is pa_decode's on the same arguments.
+ *
+ * Every argument of pa_decode, with the same meaning and layout, plus:
+ * shared_blocks   [B] int32: the first shared_blocks[b] entries of sequence
+ *                 b's table are its group's shared prefix (the same entries
+ *                 in every member's table; 0 = nothing shared);
+ * num_groups, group_offsets [num_groups + 1] int32, group_members [B] int32:
+ *                 group g is group_members[group_offsets[g] ..
+ *                 group_offsets[g + 1]); every sequence is in exactly one
+ *                 group and all members of a group have the same
+ *                 shared_blocks value (a lone sequence is a group of one);
+ * max_group_size  the largest group (host-side bound, >= 1);
+ * max_shared_blocks  the largest shared_blocks value (host-side bound);
+ * workspace       of pa_shared_prefix_workspace_size(...) bytes.
+ * Groups that break the contract give unspecified (finite) results. A
+ * sequence whose shared blocks hold more tokens than its context length is a
+ * bad context (PA_DEV_BAD_CTX, zero row). Element types other than f16 / bf16,
+ * D = 64, or G > 64 (and max_shared_blocks = 0) run as plain pa_decode.
+ */
+size_t pa_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len,
+                                       int partition_size, int block_size,
+                                       int max_shared_blocks);
+int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const void* key_cache,
+                            const void* value_cache, int dtype, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* context_lens,
+                            const int32_t* shared_blocks, int num_groups,
+                            const int32_t* group_offsets, const int32_t* group_members,
+                            int max_group_size, int max_shared_blocks, int B, int Hq, int Hkv,
+                            int D, int block_size, int num_blocks, float scale,
+                            int max_context_len, int partition_size, void* workspace,
+                            size_t workspace_bytes, uint32_t* err_flag, void* stream);
+
 /* Static text for a pa_status value. */
 const char* pa_status_string(int status);
 

@@ -1,0 +1,578 @@
+// decode_prefix_tc.cu -- decode attention of a group of sequences over the
+// blocks they share (the group's common prefix), on the 5th-generation tensor
+// cores: every shared block is streamed once per group, not once per sequence.
+//
+// Parallel sampling forks one prompt into sequences that share its physical
+// blocks ("五十三：vLLM-PagedAttention" section 17; the copy-on-write sharing of
+// "vLLM 与 LLM 推理部署实战" section 2.2). The decode queries of all of them
+// attend those blocks. For every query row of a group this kernel computes the
+// softmax state (m, l, acc) of each prefix partition (a multiple of 128 tokens);
+// the merge kernel combines it with the partials of each sequence's own
+// suffix (decode_simt.cu / decode_tc.cu in their split-only mode).
+//
+// Work unit = (group g, chunk c of the group's members, KV head h, prefix
+// partition j). Rows of a unit = the chunk's members x the G query heads of
+// KV head h, NQ <= kNQ = 64 (padded to NQP, a multiple of 16). Tile = 128
+// tokens of KV head h: one TMA box per physical block and 64-wide d-half.
+//   S^T[128 tokens x NQP] = K_tile . Q^T
+//   O^T[128 d x NQP]     += V^T . P_hi^T + V^T . P_lo^T   (weights split in two
+//                           16-bit parts, as in the per-sequence kernel)
+// A softmax thread owns one token row of S^T. The reference max of a query
+// column is set on the unit's first tile (an exact column max) and moves only
+// when a score passes it by 2^64 (then O's columns are rescaled in TMEM), so a
+// tile needs no reduction across threads; the column sums l are per-thread
+// partial sums reduced once per unit.
+//
+// CTA = 6 warps, persistent over units u = blockIdx.x + k * gridDim.x:
+// warps 0-3 softmax and epilogue (TMEM lanes 0-127), warp 4 TMA producer,
+// warp 5 MMA issuer (it also owns the tensor memory). Every wait is bounded;
+// one that gives up sets PA_DEV_TIMEOUT and the CTA drains and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include "pa_internal.h"
+#include "tc_ptx.cuh"
+
+namespace pa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 128;
+constexpr int kHalf = 128 * 128;                // one 64-wide d-half of a 128-row tile
+constexpr int kStage = 2 * kHalf;               // one K or V tile: 32 KB
+constexpr int kNST = 4;                         // ring stages
+constexpr int kNQ = 64;                         // query rows per unit (max)
+constexpr int kTile = 128;                      // tokens per tile
+constexpr int kThreads = 192;
+constexpr float kRescaleLog2 = 64.f;
+
+constexpr int OFF_Q = kNST * kStage;            // Q: 2 d-halves x kNQ rows x 128 B
+constexpr int kQBytes = 2 * kNQ * 128;
+constexpr int OFF_P = OFF_Q + kQBytes;          // P: [2 buffers][hi, lo][2 token halves][kNQ][128 B]
+constexpr int kPPart = 2 * kNQ * 128;
+constexpr int kPBuf = 2 * kPPart;
+constexpr int OFF_MREF = OFF_P + 2 * kPBuf;     // [3][kNQ] reference, old, new maxima
+constexpr int OFF_RED = OFF_MREF + 3 * kNQ * 4; // [4 warps][kNQ]
+constexpr int OFF_BAR = OFF_RED + 4 * kNQ * 4;
+enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY, B_SFULL, B_SFREE = B_SFULL + 2,
+       B_PREADY = B_SFREE + 2, B_OFULL = B_PREADY + 2, B_ODONE = B_OFULL + 2, B_DONE, B_COUNT };
+constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
+constexpr int kSmem = OFF_MISC + 32 + 1024;
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+constexpr int kTmemCols = 256;                  // S x2 (2 * kNQ) + O (kNQ), rounded up
+
+struct PrefixArgs {
+  const void* q;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* shared_blocks;                 // [B] blocks each sequence shares with its group
+  const int32_t* group_offsets;                 // [num_groups + 1]
+  const int32_t* group_members;                 // [B]
+  int num_groups, chunks, parts;                // chunks per group, prefix partitions
+  int part_tokens;                              // tokens per prefix partition (multiple of 128)
+  int B, Hq, Hkv, bs, num_blocks;
+  float scale_log2;
+  int P;                                        // workspace slots per sequence
+  float* ws_acc;
+  float* ws_m;
+  float* ws_l;
+  uint32_t* err_flag;
+};
+
+struct PUnit {
+  int g, mbeg, nm, h, j, b0, t0, t1, ntiles, nq, nqp;
+};
+
+// Decode unit u; nm <= 0 means the unit has no rows (every role skips it).
+__device__ __forceinline__ PUnit prefix_unit(const PrefixArgs& a, int G, int mc, long long u) {
+  PUnit x;
+  x.j = (int)(u % a.parts);
+  long long t = u / a.parts;
+  x.h = (int)(t % a.Hkv);
+  t /= a.Hkv;
+  const int c = (int)(t % a.chunks);
+  x.g = (int)(t / a.chunks);
+  const int gb = __ldg(a.group_offsets + x.g), ge = __ldg(a.group_offsets + x.g + 1);
+  x.mbeg = gb + c * mc;
+  x.nm = min(ge, x.mbeg + mc) - x.mbeg;
+  x.b0 = gb < ge ? __ldg(a.group_members + gb) : 0;
+  int sb = x.nm > 0 ? __ldg(a.shared_blocks + x.b0) : 0;
+  if (sb < 0 || sb > a.max_blocks) sb = 0;      // never read past the table (the suffix pass flags it)
+  const int ptoks = sb * a.bs;
+  x.t0 = x.j * a.part_tokens;
+  x.t1 = min(ptoks, x.t0 + a.part_tokens);
+  x.ntiles = x.t1 > x.t0 ? (x.t1 - x.t0 + kTile - 1) / kTile : 0;
+  x.nq = x.nm * G;
+  x.nqp = (x.nq + 15) / 16 * 16;
+  return x;
+}
+
+// Named barrier of the 128 softmax threads; vote = OR of every thread's flag.
+__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool sm_vote(bool x) { return wg_vote_or(x, 0); }
+
+template <int FMT, int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV) {
+  constexpr int NB_T = kTile / BS;              // physical blocks per tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = a.Hq / a.Hkv;
+  const int mc = kNQ / G;                       // members per chunk
+  const long long U = (long long)a.num_groups * a.chunks * a.Hkv * a.parts;
+  pdl_trigger();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNST; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_QFULL), 128);
+    mbar_init(bar(B_QEMPTY), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_SFULL + i), 1);
+      mbar_init(bar(B_SFREE + i), 128);
+      mbar_init(bar(B_PREADY + i), 128);
+      mbar_init(bar(B_OFULL + i), 1);
+    }
+    mbar_init(bar(B_ODONE), 128);
+    mbar_init(bar(B_DONE), 1);
+    *abort_flag = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s = tmem;                 // S buffers: columns [0, kNQ), [kNQ, 2 kNQ)
+  const uint32_t tmem_o = tmem + 2 * kNQ;       // O: [2 kNQ, 3 kNQ)
+  auto give_up = [&]() {
+    *abort_flag = 1u;
+    flag_error(a.err_flag, PA_DEV_TIMEOUT);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int tc_ = 0, issued = 0;
+      for (long long u = blockIdx.x; u < U; u += gridDim.x) {
+        const PUnit x = prefix_unit(a, G, mc, u);
+        if (x.nm <= 0 || x.ntiles == 0) continue;
+        const int32_t* table = a.block_tables + (size_t)x.b0 * a.max_blocks;
+        // block ids of tile k of this unit (-1: no block there)
+        auto load_ids = [&](int k, int* ph) {
+          const int ts = x.t0 + k * kTile;
+          const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+#pragma unroll
+          for (int q = 0; q < NB_T; ++q) ph[q] = q < nblk ? __ldg(table + ts / BS + q) : -1;
+        };
+        int phys_next[NB_T];
+        load_ids(0, phys_next);
+        for (int k = 0; k < x.ntiles; ++k, ++tc_) {
+          const int ts = x.t0 + k * kTile;
+          const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+          int phys[NB_T];
+          uint32_t bytes = 0;
+#pragma unroll
+          for (int q = 0; q < NB_T; ++q) phys[q] = phys_next[q];
+          if (k + 1 < x.ntiles) load_ids(k + 1, phys_next);   // a tile ahead: off the issue path
+#pragma unroll
+          for (int q = 0; q < NB_T; ++q) {
+            if (q < nblk && (phys[q] < 0 || phys[q] >= a.num_blocks)) {
+              flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+              phys[q] = -1;
+            }
+            if (phys[q] >= 0) bytes += 2u * BS * 128u;
+          }
+          for (int kv = 0; kv < 2; ++kv) {
+            const int seq = 2 * tc_ + kv, s = seq % kNST;
+            if (!mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+            mbar_expect_tx(bar(B_FULL + s), bytes);
+            const uint32_t dst = sbase + s * kStage;
+#pragma unroll
+            for (int q = 0; q < NB_T; ++q) {
+              if (phys[q] < 0) continue;
+              for (int hh = 0; hh < 2; ++hh)
+                tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
+                            phys[q], bar(B_FULL + s));
+            }
+            ++issued;
+          }
+        }
+      }
+    prod_done:
+      for (int seq = max(0, issued - kNST); seq < issued; ++seq) {
+        const int s = seq % kNST;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(bar(B_FULL + s), (seq / kNST) & 1) && globaltimer() - t0 < kWaitNs) {}
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int tc_ = 0, ua = 0;
+      bool ok = true;
+      for (long long u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const PUnit x = prefix_unit(a, G, mc, u);
+        if (x.nm <= 0 || x.ntiles == 0) continue;
+        const uint32_t idesc_s = make_idesc(FMT, 0, 0, x.nqp, 128);
+        const uint32_t idesc_o = make_idesc(FMT, 1, 0, x.nqp, 128);
+        if (!mbar_wait(bar(B_QFULL), ua & 1, abort_flag)) { ok = false; break; }
+        const uint32_t qst = sbase + OFF_Q;
+        auto issue_pv = [&](int tt, bool first) -> bool {
+          const int pb = tt & 1;
+          if (!mbar_wait(bar(B_PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
+          if (first && ua > 0 && !mbar_wait(bar(B_ODONE), (ua - 1) & 1, abort_flag)) return false;
+          const int seq = 2 * tt + 1, s = seq % kNST;
+          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t vst = sbase + s * kStage;
+          const uint32_t pst = sbase + OFF_P + pb * kPBuf;
+#pragma unroll
+          for (int ks = 0; ks < kTile / 16; ++ks) {
+            const uint64_t ad = sw128_desc(vst + ks * 16 * 128, kHalf, 1024);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+              const uint64_t bd =
+                  sw128_desc(pst + part * kPPart + (ks >> 2) * (kNQ * 128) + (ks & 3) * 32, 16, 1024);
+              mma_f16(tmem_o, ad, bd, idesc_o, (first && ks == 0 && part == 0) ? 0u : 1u);
+            }
+          }
+          mma_commit(bar(B_EMPTY + s));
+          mma_commit(bar(B_OFULL + pb));
+          return true;
+        };
+        for (int k = 0; k < x.ntiles; ++k) {
+          const int sb = tc_ & 1;
+          if (!mbar_wait(bar(B_SFREE + sb), ((tc_ >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int seq = 2 * tc_, s = seq % kNST;
+          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kst = sbase + s * kStage;
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint64_t ad = sw128_desc(kst + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(qst + (ks >> 2) * (kNQ * 128) + (ks & 3) * 32, 16, 1024);
+            mma_f16(tmem_s + sb * kNQ, ad, bd, idesc_s, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(B_EMPTY + s));
+          mma_commit(bar(B_SFULL + sb));
+          if (k == x.ntiles - 1) mma_commit(bar(B_QEMPTY));
+          if (k > 0 && !issue_pv(tc_ - 1, k == 1)) { ok = false; break; }
+          ++tc_;
+        }
+        if (ok && !issue_pv(tc_ - 1, x.ntiles == 1)) ok = false;
+        ++ua;
+      }
+      if (!ok) give_up();
+      mma_commit(bar(B_DONE));
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(bar(B_DONE), 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int r = threadIdx.x;                   // token row of S^T; d row of O^T
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    float* mref = reinterpret_cast<float*>(smem + OFF_MREF);
+    float* mold = mref + kNQ;
+    float* mnew = mold + kNQ;
+    float* red = reinterpret_cast<float*>(smem + OFF_RED);
+    bool failed = false, stop = false;
+    int tc_ = 0, ua = 0;
+    auto wait_pv = [&](int t) {                  // output product of tile t has completed
+      if (!mbar_wait(bar(B_OFULL + (t & 1)), (t >> 1) & 1, abort_flag)) failed = true;
+    };
+    // exact column maxima of s[] over the 128 rows -> dst[q]
+    auto col_max = [&](const float* s, float* dst) {
+#pragma unroll
+      for (int q = 0; q < kNQ; ++q) {
+        float v = s[q];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) red[warp * kNQ + q] = v;
+      }
+      sm_sync();
+      if (r < kNQ) dst[r] = fmaxf(fmaxf(red[r], red[kNQ + r]), fmaxf(red[2 * kNQ + r], red[3 * kNQ + r]));
+      sm_sync();
+    };
+    for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
+      const PUnit x = prefix_unit(a, G, mc, u);
+      if (x.nm <= 0) continue;
+      // rows of the unit: q = m * G + gg -> (sequence, query head) slot of partition j
+      auto slot_row = [&](int q) -> size_t {
+        const int b = __ldg(a.group_members + x.mbeg + q / G);
+        return ((size_t)b * a.P + x.j) * a.Hq + (size_t)x.h * G + (q % G);
+      };
+      if (x.ntiles == 0) {
+        // this partition of the prefix holds no tokens: an empty partial
+        for (int q = 0; q < x.nq; ++q) a.ws_acc[slot_row(q) * kD + r] = 0.f;
+        if (r < x.nq) {
+          a.ws_m[slot_row(r)] = -CUDART_INF_F;
+          a.ws_l[slot_row(r)] = 0.f;
+        }
+        continue;
+      }
+      // Q rows of the unit into the K-major 128-byte-swizzled operand
+      if (ua > 0 && !mbar_wait(bar(B_QEMPTY), (ua - 1) & 1, abort_flag)) failed = true;
+      for (int c = r; c < x.nqp * 16; c += 128) {
+        const int q = c >> 4, k16 = c & 15, hh = k16 >> 3, kk = k16 & 7;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (q < x.nq) {
+          const int b = __ldg(a.group_members + x.mbeg + q / G);
+          const size_t row = (size_t)b * a.Hq + (size_t)x.h * G + (q % G);
+          v = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.q) + row * (kD * 2) +
+                                              k16 * 16);
+        }
+        *reinterpret_cast<uint4*>(smem + OFF_Q + hh * (kNQ * 128) + q * 128 + ((kk ^ (q & 7)) << 4)) = v;
+      }
+      fence_proxy_async();
+      mbar_arrive(bar(B_QFULL));
+
+      float l[kNQ];
+#pragma unroll
+      for (int q = 0; q < kNQ; ++q) l[q] = 0.f;
+      const int32_t* table = a.block_tables + (size_t)x.b0 * a.max_blocks;
+      for (int k = 0; k < x.ntiles; ++k, ++tc_) {
+        const int ts = x.t0 + k * kTile;
+        const int tok = ts + r;
+        bool valid = tok < x.t1;
+        if (valid) {
+          const int32_t p = __ldg(table + tok / BS);
+          valid = p >= 0 && p < a.num_blocks;
+        }
+        if (!mbar_wait(bar(B_SFULL + (tc_ & 1)), (tc_ >> 1) & 1, abort_flag)) failed = true;
+        tc_fence_after();
+        float s[kNQ];
+#pragma unroll
+        for (int c = 0; c < kNQ; c += 16) tmem_ld16(tmem_s + lane_off + (tc_ & 1) * kNQ + c, s + c);
+        tc_fence_before();
+        mbar_arrive(bar(B_SFREE + (tc_ & 1)));
+#pragma unroll
+        for (int q = 0; q < kNQ; ++q) s[q] = (valid && q < x.nq) ? s[q] * a.scale_log2 : -CUDART_INF_F;
+        if (sm_vote(failed)) { stop = true; break; }
+        if (k == 0) {
+          col_max(s, mref);
+        } else {
+          bool exceed = false;
+#pragma unroll
+          for (int q = 0; q < kNQ; ++q) exceed |= s[q] > mref[q] + kRescaleLog2;
+          if (sm_vote(exceed)) {
+            // rare: move the references of the columns that passed them, and
+            // rescale those columns of O (all earlier products included) and l
+            col_max(s, mnew);
+            if (r < kNQ) {
+              mold[r] = mref[r];
+              mnew[r] = mnew[r] > mref[r] + kRescaleLog2 ? mnew[r] : mref[r];
+            }
+            sm_sync();
+            wait_pv(tc_ - 1);
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < kNQ; c += 16) {
+              float o[16];
+              tmem_ld16(tmem_o + lane_off + c, o);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int q = c + e;
+                if (mnew[q] != mold[q] && mold[q] != -CUDART_INF_F) {
+                  const float f = exp2f(mold[q] - mnew[q]);
+                  o[e] *= f;
+                  l[q] *= f;
+                }
+              }
+              tmem_st16(tmem_o + lane_off + c, o);
+            }
+            tc_fence_before();
+            sm_sync();
+            if (r < kNQ) mref[r] = mnew[r];
+            sm_sync();
+          }
+        }
+        // the P buffer of this tile was last read by the output product of tile tc - 2
+        if (tc_ >= 2) wait_pv(tc_ - 2);
+        uint8_t* pb = smem + OFF_P + (tc_ & 1) * kPBuf + (r >> 6) * (kNQ * 128);
+        const int pc = (r & 63) >> 3, pbyte = (r & 7) * 2;
+#pragma unroll
+        for (int q = 0; q < kNQ; ++q) {
+          const float m = mref[q];
+          const float p = (s[q] != -CUDART_INF_F && m != -CUDART_INF_F) ? exp2f(s[q] - m) : 0.f;
+          l[q] += p;
+          uint16_t hi, lo;
+          split_16<FMT>(p, hi, lo);
+          const int off = q * 128 + ((pc ^ (q & 7)) << 4) + pbyte;
+          *reinterpret_cast<uint16_t*>(pb + off) = hi;
+          *reinterpret_cast<uint16_t*>(pb + kPPart + off) = lo;
+        }
+        if (!valid) {
+          // a row with weight 0 still enters the product: it must hold finite values
+          const int seq = 2 * tc_ + 1, sv = seq % kNST;
+          if (!mbar_wait(bar(B_FULL + sv), (seq / kNST) & 1, abort_flag)) failed = true;
+          uint4* r0 = reinterpret_cast<uint4*>(smem + sv * kStage + r * 128);
+          uint4* r1 = reinterpret_cast<uint4*>(smem + sv * kStage + kHalf + r * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) { r0[c] = make_uint4(0, 0, 0, 0); r1[c] = make_uint4(0, 0, 0, 0); }
+        }
+        fence_proxy_async();
+        mbar_arrive(bar(B_PREADY + (tc_ & 1)));
+      }
+      if (stop) break;
+
+      // ---- end of the unit: column sums, then O and (m, l) to the workspace
+      wait_pv(tc_ - 1);
+      if (sm_vote(failed)) break;
+#pragma unroll
+      for (int q = 0; q < kNQ; ++q) {
+        float v = l[q];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[warp * kNQ + q] = v;
+      }
+      sm_sync();
+      if (r < x.nq) {
+        const size_t sr = slot_row(r);
+        a.ws_m[sr] = mref[r];
+        a.ws_l[sr] = red[r] + red[kNQ + r] + red[2 * kNQ + r] + red[3 * kNQ + r];
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < kNQ; c += 16) {
+        float o[16];
+        tmem_ld16(tmem_o + lane_off + c, o);
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (c + e < x.nq) a.ws_acc[slot_row(c + e) * kD + r] = o[e];
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_ODONE));
+      sm_sync();                                 // red and mref are rewritten by the next unit
+      ++ua;
+    }
+    if (failed) give_up();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// The pool [NB][bs][Hkv][D] seen as [NB][2][Hkv][bs][64]: a box of one block's
+// bs rows of one head and one d-half, 128-byte swizzled.
+bool make_prefix_maps(const void* k_cache, const void* v_cache, int dtype, int bs, int Hkv,
+                      int num_blocks, CUtensorMap* k, CUtensorMap* v) {
+  auto enc = encode_fn();
+  if (!enc || num_blocks <= 0) return false;
+  const CUtensorMapDataType dt =
+      dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t dims[5] = {64, (cuuint64_t)bs, (cuuint64_t)Hkv, 2, (cuuint64_t)num_blocks};
+  const cuuint64_t strides[4] = {(cuuint64_t)Hkv * kD * 2, (cuuint64_t)kD * 2, 128,
+                                 (cuuint64_t)bs * Hkv * kD * 2};
+  const cuuint32_t box[5] = {64, (cuuint32_t)bs, 1, 1, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r = enc(i == 0 ? k : v, dt, 5, const_cast<void*>(i == 0 ? k_cache : v_cache), dims,
+                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+  }
+  return true;
+}
+
+template <int FMT, int BS>
+int launch_prefix_t(const PrefixArgs& a, const CUtensorMap& k, const CUtensorMap& v,
+                    cudaStream_t stream) {
+  auto kern = prefix_tc_kernel<FMT, BS>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    attr = true;
+  }
+  const long long U = (long long)a.num_groups * a.chunks * a.Hkv * a.parts;
+  if (U <= 0) return PA_OK;
+  int dev = 0, sms = kSMs;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = U < sms ? U : sms;
+  return launch_k(kern, dim3((unsigned)grid), dim3(kThreads), kSmem, stream, a, k, v) ==
+                 cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+bool prefix_tc_supported(int dtype, int Hq, int Hkv, int D, int bs) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return false;
+  if (D != kD || (bs != 16 && bs != 32) || Hkv <= 0 || Hq % Hkv) return false;
+  return Hq / Hkv <= kNQ;
+}
+
+int prefix_chunks(int max_group_size, int G) {
+  const int mc = kNQ / G;
+  return (max_group_size + mc - 1) / mc;
+}
+
+int launch_prefix_tc(const DecodeArgs& d, int dtype, const int32_t* group_offsets,
+                     const int32_t* group_members, int num_groups, int max_group_size,
+                     int parts, int part_tokens, cudaStream_t stream) {
+  CUtensorMap k, v;
+  if (!make_prefix_maps(d.k_cache, d.v_cache, dtype, d.bs, d.Hkv, d.num_blocks, &k, &v))
+    return PA_ERR_CUDA;
+  PrefixArgs a{};
+  a.q = d.q;
+  a.block_tables = d.block_tables;
+  a.max_blocks = d.max_blocks;
+  a.shared_blocks = d.start_blocks;
+  a.group_offsets = group_offsets;
+  a.group_members = group_members;
+  a.num_groups = num_groups;
+  a.chunks = prefix_chunks(max_group_size, d.Hq / d.Hkv);
+  a.parts = parts;
+  a.part_tokens = part_tokens;
+  a.B = d.B; a.Hq = d.Hq; a.Hkv = d.Hkv; a.bs = d.bs; a.num_blocks = d.num_blocks;
+  a.scale_log2 = d.scale_log2;
+  a.P = d.P;
+  a.ws_acc = d.ws_acc; a.ws_m = d.ws_m; a.ws_l = d.ws_l;
+  a.err_flag = d.err_flag;
+  if (dtype == PA_BF16)
+    return d.bs == 16 ? launch_prefix_t<1, 16>(a, k, v, stream) : launch_prefix_t<1, 32>(a, k, v, stream);
+  return d.bs == 16 ? launch_prefix_t<0, 16>(a, k, v, stream) : launch_prefix_t<0, 32>(a, k, v, stream);
+}
+
+}  // namespace pa

@@ -83,20 +83,24 @@ decode_simt_kernel(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int ctx = a.context_lens[b];
-  const bool bad_ctx = ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len;
-  const int tok_begin = j * a.psize;
-  if (bad_ctx || ctx == 0) {
+  const int start = a.start_blocks ? a.start_blocks[b] * BS : 0;   // first token of this pass
+  const bool bad_ctx = ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len ||
+                       start < 0 || start > ctx;
+  const int tok_begin = start + j * a.psize;
+  if (bad_ctx || ctx == start) {
     // zero rows, written once (by partition 0); the merge kernel skips them
+    // (in the split-only pass the merge writes every row)
     if (j == 0) {
       if (bad_ctx && threadIdx.x == 0 && chunk == 0 && h == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
-      for (int i = threadIdx.x; i < GC * D; i += blockDim.x)
-        store_out(a.out, ((size_t)b * a.Hq + hq0 + i / D) * D + i % D, 0.f, a.out_dtype);
+      if (!a.force_split)
+        for (int i = threadIdx.x; i < GC * D; i += blockDim.x)
+          store_out(a.out, ((size_t)b * a.Hq + hq0 + i / D) * D + i % D, 0.f, a.out_dtype);
     }
     return;
   }
   if (tok_begin >= ctx) return;                 // partition past this sequence's end
   const int tok_end = min(ctx, tok_begin + a.psize);
-  const int nparts = (ctx + a.psize - 1) / a.psize;
+  const int nparts = (ctx - start + a.psize - 1) / a.psize;
 
   // query vectors of this chunk, pre-scaled so scores come out as scale*log2(e)*q.k
   const int ci = lane % LPR;                    // which 16-byte vector of a row
@@ -260,10 +264,10 @@ decode_simt_kernel(const DecodeArgs a) {
     }
     const size_t row = (size_t)b * a.Hq + hq0 + g;
     O *= a.v_scale;                              // 1 unless the V pool holds FP8 codes
-    if (nparts == 1) {
+    if (nparts == 1 && !a.force_split) {
       store_out(a.out, row * D + d, L > 0.f ? O / L : 0.f, a.out_dtype);
     } else {
-      const size_t pj = ((size_t)b * a.P + j) * a.Hq + hq0 + g;   // [B][P][Hq] slot
+      const size_t pj = ((size_t)b * a.P + a.slot_base + j) * a.Hq + hq0 + g;   // [B][P][Hq] slot
       a.ws_acc[pj * D + d] = O;
       if (d == 0) { a.ws_m[pj] = M; a.ws_l[pj] = L; }
     }
@@ -340,9 +344,17 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeArgs a) {
   float M = -CUDART_INF_F, mj = -CUDART_INF_F, lj = 0.f;
   if (one && jl < a.P) { mj = pm[(size_t)jl * a.Hq]; lj = pl[(size_t)jl * a.Hq]; }
   const int ctx = a.context_lens[b];
-  if (ctx <= 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len) return;
-  const int nparts = (ctx + a.psize - 1) / a.psize;
-  if (nparts <= 1) return;
+  const int start = a.start_blocks ? a.start_blocks[b] * a.bs : 0;
+  if (ctx < 0 || ctx > a.max_blocks * a.bs || ctx > a.max_context_len || start < 0 || start > ctx ||
+      (!a.force_split && ctx == 0)) {
+    if (a.force_split && sub == 0)                 // split-only pass: the merge owns every row
+      for (int e = lane; e < D; e += 32) store_out(a.out, (size_t)row * D + e, 0.f, a.out_dtype);
+    return;
+  }
+  // partitions of this row: slots [0, slot_base) hold earlier passes' partials
+  // (the shared prefix), then ceil((ctx - start) / psize) of this pass
+  const int nparts = a.slot_base + (ctx - start + a.psize - 1) / a.psize;
+  if (nparts <= 1 && !a.force_split) return;
   if (one) {
     if (jl >= nparts) { mj = -CUDART_INF_F; lj = 0.f; }
     M = mj;

@@ -55,10 +55,13 @@
 #include <math_constants.h>
 
 #include "pa_internal.h"
+#include "tc_ptx.cuh"
 
 namespace pa {
 
 namespace {
+
+using namespace tc;
 
 constexpr int kD = 128;
 constexpr int kRows = 128;                      // rows per tile (the MMA's M)
@@ -67,9 +70,8 @@ constexpr int kStageBytes = 2 * kHalf;          // one K or V tile: 32 KB
 constexpr int kHG = 4;                          // KV heads per unit
 constexpr int kRt = kRows / kHG;                // tokens per head per tile (32)
 constexpr int kThreads = 320;
-constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kMaxUnits = 320;                  // work units one CTA can hold in its list
-constexpr int kScanChunk = 2048;                // sequences scanned per pass (stage 0 as scratch)
+constexpr int kScanChunk = 1024;                // sequences scanned per pass (stage 0 as scratch)
 constexpr float kRescaleLog2 = 64.f;            // lazy rescale threshold (log2 units): p <= 2^64,
                                                 // far from fp32 overflow in l and O
 
@@ -111,182 +113,6 @@ template <int NST> struct Bars {
                        ODONE = XFREE + 2, DONE = ODONE + 2;
 };
 
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Non-blocking probe: has the phase with the given parity completed?
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait for the phase with the given parity; false = gave up (timeout or abort).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile uint32_t* abort_flag) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitNs) return false;
-  }
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            int c2, int c3, int c4, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-// Shared-memory matrix descriptor, 128-byte swizzle (tcgen05 format: version 1 at bit 46).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor of kind::f16 with fp32 accumulation.
-__host__ __device__ constexpr uint32_t make_idesc(int fmt, int a_mn, int b_mn, int N, int M) {
-  return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((uint32_t)a_mn << 15) |
-         ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.u32 p, %4, 0;"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-// 16 consecutive fp32 columns of this thread's TMEM lane; waits for the load.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  __syncwarp();
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15},"
-      " [%16];\n\ttcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-// Vote over the 128 threads of one softmax group (named barrier 1 + group):
-// OR of every thread's flag; also a barrier for the group's shared memory.
-__device__ __forceinline__ bool wg_vote_or(bool x, int group) {
-  uint32_t r;
-  asm volatile(
-      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, %2, 128, pi;"
-      " selp.u32 %0, 1, 0, po; }"
-      : "=r"(r)
-      : "r"((uint32_t)x), "r"(1 + group)
-      : "memory");
-  return r != 0;
-}
-
-template <int FMT> __device__ __forceinline__ void split_16(float p, uint16_t& hi, uint16_t& lo) {
-  if (FMT == 1) {
-    __nv_bfloat16 h = __float2bfloat16_rn(p);
-    __nv_bfloat16 l = __float2bfloat16_rn(p - __bfloat162float(h));
-    hi = __bfloat16_as_ushort(h);
-    lo = __bfloat16_as_ushort(l);
-  } else {
-    __half h = __float2half_rn(p);
-    __half l = __float2half_rn(p - __half2float(h));
-    hi = __half_as_ushort(h);
-    lo = __half_as_ushort(l);
-  }
-}
-
-// Store 16 consecutive fp32 columns of this thread's TMEM lane; waits for the store.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
-  __syncwarp();
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-      "\n\ttcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15]))
-      : "memory");
-}
-// Plain named-barrier sync of one softmax group.
-__device__ __forceinline__ void wg_sync(int group) {
-  asm volatile("bar.sync %0, 128;" ::"r"(1 + group) : "memory");
-}
-// Bulk asynchronous copy shared -> global (16-byte aligned, size a multiple of 16).
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst),
-               "r"(ssrc), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// The staging buffer may be rewritten once the copies have read it.
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // ---------------------------------------------------------------- work units
 // A unit is (sequence b, partition j, group h of kHG KV heads). Units exist
 // only for partitions that hold tokens. Units are spread over the CTAs like
@@ -297,7 +123,7 @@ __device__ __forceinline__ void bulk_wait_all() {
 // Every CTA builds its own list at start, in shared memory, so the roles never
 // touch global memory to find their next unit.
 struct __align__(16) URec {
-  int b, h, j, ctx;
+  int b, hj, ctx, start;      // hj = KV-head group | partition << 16; start = first token of the pass
 };
 
 struct Unit {
@@ -306,11 +132,11 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_from(const URec& r, int psize) {
   Unit x;
-  x.b = r.b; x.h = r.h; x.j = r.j; x.ctx = r.ctx;
-  x.t0 = r.j * psize;
+  x.b = r.b; x.h = r.hj & 0xffff; x.j = r.hj >> 16; x.ctx = r.ctx;
+  x.t0 = r.start + x.j * psize;
   x.t1 = min(r.ctx, x.t0 + psize);
   x.ntiles = (x.t1 - x.t0 + kRt - 1) / kRt;
-  x.nparts = (r.ctx + psize - 1) / psize;
+  x.nparts = (r.ctx - r.start + psize - 1) / psize;
   return x;
 }
 
@@ -328,7 +154,8 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
   int* ctx_s = reinterpret_cast<int*>(scratch);           // [kScanChunk]
-  int* next_s = ctx_s + kScanChunk;                       // [NC][128] next rank per class
+  int* start_s = ctx_s + kScanChunk;                      // [kScanChunk] first token of the pass
+  int* next_s = start_s + kScanChunk;                     // [NC][128] next rank per class
   int* hist = next_s + NC * 128;                          // [NC] units per class
   int* cbase = hist + NC;                                 // [NC] first rank of each class
   int* carry = cbase + NC;                                // [NC] ranks used by earlier passes
@@ -336,13 +163,19 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
   int* nempty = wsum + 4 * NC;                            // sequences to zero in this pass
   int* empty_s = nempty + 4;                              // [kScanChunk]
   const int TP = (a.psize + kRt - 1) / kRt;               // tiles of a whole partition
-  // partitions of a sequence and tiles of its last one; false: no units
-  auto shape = [&](int ctx, int& np, int& tl) -> bool {
-    if (ctx <= 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len) return false;
-    np = (ctx + a.psize - 1) / a.psize;
-    tl = (ctx - (np - 1) * a.psize + kRt - 1) / kRt;
+  // a context length (or pass start) the table cannot hold
+  auto bad = [&](int ctx, int start) {
+    return ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len || start < 0 ||
+           start > ctx;
+  };
+  // partitions of the pass [start, ctx) and tiles of its last one; false: no units
+  auto shape = [&](int ctx, int start, int& np, int& tl) -> bool {
+    if (bad(ctx, start) || ctx == start) return false;
+    np = (ctx - start + a.psize - 1) / a.psize;
+    tl = (ctx - start - (np - 1) * a.psize + kRt - 1) / kRt;
     return true;
   };
+  auto start_of = [&](int b) { return a.start_blocks ? __ldg(a.start_blocks + b) * BS : 0; };
   auto cls = [&](int nt) { return min(NC - 1, (nt * NC + TP - 1) / TP - 1); };
   auto bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
 
@@ -350,7 +183,7 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
   bar();
   for (int b = tid; b < a.B; b += 128) {
     int np, tl;
-    if (!shape(__ldg(a.context_lens + b), np, tl)) continue;
+    if (!shape(__ldg(a.context_lens + b), start_of(b), np, tl)) continue;
     if (np > 1) atomicAdd(&hist[NC - 1], (np - 1) * nhg);
     atomicAdd(&hist[cls(tl)], nhg);
   }
@@ -369,6 +202,7 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
     for (int e = 0; e < PER; ++e) {
       const int i = e * 128 + tid;
       ctx_s[i] = i < n ? __ldg(a.context_lens + b0 + i) : 0;
+      start_s[i] = i < n ? start_of(b0 + i) : 0;
     }
     bar();
     // units per class of this thread's sequences, then a block-wide scan per class
@@ -378,7 +212,7 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
     for (int e = 0; e < PER; ++e) {
       int np, tl;
       const int i = e * 128 + tid;
-      if (!shape(ctx_s[i], np, tl)) {
+      if (!shape(ctx_s[i], start_s[i], np, tl)) {
         if (i < n && ((b0 + i) % grid) == cta) empty_s[atomicAdd(nempty, 1)] = i;
         continue;
       }
@@ -410,7 +244,7 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
     for (int e = 0; e < PER; ++e) {
       const int li = e * 128 + tid;
       int np, tl;
-      if (!shape(ctx_s[li], np, tl)) continue;
+      if (!shape(ctx_s[li], start_s[li], np, tl)) continue;
       if (np > 1) {
         // whole partitions: consecutive ranks r0 .. r0 + nf - 1 (unit j * nhg + h);
         // visit only the rounds they span and this CTA's slot in each
@@ -420,7 +254,8 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
         for (int round = r0 / grid; round * grid < r0 + nf && round < kMaxUnits; ++round) {
           const int r = round * grid + ((round & 1) ? grid - 1 - cta : cta);
           if (r < r0 || r >= r0 + nf) continue;
-          recs[round] = URec{b0 + li, (r - r0) % nhg, (r - r0) / nhg, ctx_s[li]};
+          recs[round] = URec{b0 + li, ((r - r0) % nhg) | (((r - r0) / nhg) << 16), ctx_s[li],
+                             start_s[li]};
         }
       }
       int* nx = next_s + cls(tl) * 128 + tid;               // the last partition
@@ -428,16 +263,18 @@ __device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, 
         const int r = (*nx)++;
         const int round = r / grid, pos = r - round * grid;
         const int owner = (round & 1) ? grid - 1 - pos : pos;
-        if (owner == cta && round < kMaxUnits) recs[round] = URec{b0 + li, h, np - 1, ctx_s[li]};
+        if (owner == cta && round < kMaxUnits)
+          recs[round] = URec{b0 + li, h | ((np - 1) << 16), ctx_s[li], start_s[li]};
       }
     }
     // zero the output rows of empty / bad sequences this CTA owns
     bar();
     for (int k = 0; k < *nempty; ++k) {
       const int li = empty_s[k], b = b0 + li;
-      if (ctx_s[li] != 0 && tid == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
-      for (int i = tid; i < a.Hq * kD; i += 128)
-        store_out(a.out, (size_t)b * a.Hq * kD + i, 0.f, a.out_dtype);
+      if (bad(ctx_s[li], start_s[li]) && tid == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
+      if (!a.force_split)                 // the split-only pass leaves every row to the merge
+        for (int i = tid; i < a.Hq * kD; i += 128)
+          store_out(a.out, (size_t)b * a.Hq * kD + i, 0.f, a.out_dtype);
     }
     bar();
   }
@@ -892,11 +729,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         // merged rows go to shared memory first, then out in one bulk copy per head:
         // the unit's NS output rows are contiguous in out [B, Hq, D] and in the
         // workspace [B, P, Hq, D]
-        const bool final_out = x.nparts == 1;
+        const bool final_out = x.nparts == 1 && !a.force_split;
         const int osz = final_out && a.out_dtype != PA_F32 ? 2 : 4;
         uint8_t* stg = smem + S::OFF_STG + grp * S::kStgBytes;
         const size_t row0 = final_out ? (size_t)x.b * a.Hq + (size_t)x.h * NS
-                                      : ((size_t)x.b * a.P + x.j) * a.Hq + (size_t)x.h * NS;
+                                      : ((size_t)x.b * a.P + a.slot_base + x.j) * a.Hq +
+                                            (size_t)x.h * NS;
         float* coef = reinterpret_cast<float*>(smem + S::OFF_COEF) + grp * 2 * NS;
         if (row < NS) {
           // query head n: combined max and exp-sum, and the weights of the two

@@ -1,5 +1,6 @@
 // pa_api.cu -- the extern "C" boundary of libpa.so: argument checks, launch
 // planning (split or not, which kernel), workspace carve-up, launches.
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -30,6 +31,22 @@ bool supported_shape(int Hq, int Hkv, int D, int bs) {
 int esize_of(int dtype) { return dtype == PA_F32 ? 4 : (dtype == PA_FP8_E4M3 ? 1 : 2); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Upper bound of the prefix partitions of a shared-prefix decode (one per tile).
+int max_prefix_slots(int max_shared_blocks, int block_size) {
+  return (max_shared_blocks * block_size + kPrefixTile - 1) / kPrefixTile;
+}
+
+int sm_count_cached() {
+  static int n = 0;
+  if (n <= 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = kSMs;
+  }
+  return n;
+}
 
 // Kernel override for A/B measurements: PA_DECODE_KERNEL=simt|tc (unset = auto).
 int kernel_override() {
@@ -220,6 +237,91 @@ int pa_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype, 
   return launch_reshape_and_cache_fp8(key, value, src_dtype, key_cache, value_cache, k_scale,
                                       v_scale, slot_mapping, T, Hkv, D, block_size, num_blocks,
                                       err_flag, static_cast<cudaStream_t>(stream));
+}
+
+size_t pa_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len,
+                                        int partition_size, int block_size,
+                                        int max_shared_blocks) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_context_len <= 0 || partition_size < 0 ||
+      block_size <= 0 || max_shared_blocks < 0)
+    return 0;
+  if (max_shared_blocks == 0) return pa_workspace_size(B, Hq, Hkv, D, max_context_len, partition_size);
+  DecodePlan p = plan_decode(PA_F32, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  return workspace_bytes_for(B, Hq, D, max_prefix_slots(max_shared_blocks, block_size) + p.P);
+}
+
+int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const void* key_cache,
+                            const void* value_cache, int dtype, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* context_lens,
+                            const int32_t* shared_blocks, int num_groups,
+                            const int32_t* group_offsets, const int32_t* group_members,
+                            int max_group_size, int max_shared_blocks, int B, int Hq, int Hkv,
+                            int D, int block_size, int num_blocks, float scale,
+                            int max_context_len, int partition_size, void* workspace,
+                            size_t workspace_bytes, uint32_t* err_flag, void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0) return PA_ERR_SHAPE;
+  if (max_shared_blocks > max_blocks_per_seq) return PA_ERR_SHAPE;
+  const bool share = max_shared_blocks > 0 && num_groups > 0 && B > 0 &&
+                     prefix_tc_supported(dtype, Hq, Hkv, D, block_size);
+  if (!share)   // nothing shared, or a shape the prefix kernel does not take: plain decode
+    return decode_impl(out, out_dtype, query, dtype, key_cache, value_cache, dtype, 1.f, 1.f,
+                       block_tables, max_blocks_per_seq, context_lens, B, Hq, Hkv, D, block_size,
+                       num_blocks, scale, max_context_len, partition_size, workspace,
+                       workspace_bytes, err_flag, stream);
+  if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_DTYPE;
+  if (Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0 ||
+      max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0 || max_group_size < 1)
+    return PA_ERR_SHAPE;
+  if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (partition_size > 0 && partition_size % block_size) return PA_ERR_SHAPE;
+  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (B > 65535 || Hkv > 65535) return PA_ERR_UNSUPPORTED;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
+      !shared_blocks || !group_offsets || !group_members)
+    return PA_ERR_NULL;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_ALIGN;
+
+  DecodePlan p = plan_decode(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  // Prefix partitions: as many as keep every (group, member chunk, KV head)
+  // unit of all of them in one wave over the SMs, at least one tile each.
+  const int tiles = max_prefix_slots(max_shared_blocks, block_size);
+  const long long per_part =
+      (long long)num_groups * prefix_chunks(max_group_size, Hq / Hkv) * Hkv;
+  int parts = (int)std::max(1LL, std::min<long long>(tiles, sm_count_cached() / std::max(1LL, per_part)));
+  const int part_tokens = (tiles + parts - 1) / parts * kPrefixTile;
+  parts = (max_shared_blocks * block_size + part_tokens - 1) / part_tokens;
+  DecodeArgs a{};
+  a.out = out; a.out_dtype = out_dtype; a.q = query;
+  a.k_cache = key_cache; a.v_cache = value_cache;
+  a.block_tables = block_tables; a.max_blocks = max_blocks_per_seq;
+  a.context_lens = context_lens;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.bs = block_size; a.num_blocks = num_blocks;
+  a.scale_log2 = scale * kLog2e;
+  a.v_scale = 1.f;
+  a.max_context_len = max_context_len;
+  a.P = tiles + p.P; a.psize = p.psize;    // slot stride as sized by the workspace query
+  a.err_flag = err_flag;
+  a.start_blocks = shared_blocks;        // the suffix pass starts after the shared blocks
+  a.slot_base = parts;                   // slots [0, parts) hold the prefix partials
+  a.force_split = 1;
+  const size_t need = workspace_bytes_for(B, Hq, D, a.P);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PA_ERR_WORKSPACE;
+  const size_t rows = (size_t)B * Hq * a.P;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  char* w = static_cast<char*>(workspace);
+  a.ws_acc = reinterpret_cast<float*>(w);
+  a.ws_m = reinterpret_cast<float*>(w + up(rows * D * 4));
+  a.ws_l = reinterpret_cast<float*>(w + up(rows * D * 4) + up(rows * 4));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, st) : launch_decode_simt(a, dtype, st);
+  if (rc == PA_OK)
+    rc = launch_prefix_tc(a, dtype, group_offsets, group_members, num_groups, max_group_size,
+                          parts, part_tokens, st);
+  if (rc == PA_OK) rc = launch_merge(a, st);
+  return rc;
 }
 
 int pa_swap_blocks(void* dst_key, void* dst_value, const void* src_key, const void* src_value,

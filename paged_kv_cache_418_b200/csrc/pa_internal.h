@@ -28,7 +28,20 @@ struct DecodeArgs {
   float* ws_l;          // [B, P, Hq] partial sum of exp2(s - m)
   float v_scale;        // value of one V unit (FP8 pools; 1 otherwise); K's is in scale_log2
   uint32_t* err_flag;
+  // Shared-prefix (cascade) suffix pass: sequence b attends tokens
+  // [start_blocks[b] * bs, ctx_b) only (start_blocks NULL = all tokens),
+  // partition j goes to workspace slot slot_base + j, and with force_split
+  // every partition is left as a partial for the merge (which then also
+  // writes empty and bad rows).
+  const int32_t* start_blocks;
+  int slot_base;
+  int force_split;
 };
+
+// Shared-prefix decode: the prefix is cut into partitions of a multiple of
+// kPrefixTile tokens (one tensor-core tile); a sequence's workspace slots
+// [0, slot_base) hold its prefix partials, at most ceil(prefix / kPrefixTile).
+constexpr int kPrefixTile = 128;
 
 struct DecodePlan {
   int kernel;           // 1 = CUDA-core path, 2 = tcgen05 GQA path
@@ -47,6 +60,11 @@ int launch_decode_simt_fp8(const DecodeArgs& a, int q_dtype, cudaStream_t stream
 int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream);
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 int launch_merge(const DecodeArgs& a, cudaStream_t stream);
+bool prefix_tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
+int prefix_chunks(int max_group_size, int G);
+int launch_prefix_tc(const DecodeArgs& a, int dtype, const int32_t* group_offsets,
+                     const int32_t* group_members, int num_groups, int max_group_size, int parts,
+                     int part_tokens, cudaStream_t stream);
 
 int launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
                              void* value_cache, int esize, const int64_t* slot_mapping, int T,

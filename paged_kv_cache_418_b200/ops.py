@@ -56,6 +56,11 @@ def _load() -> ctypes.CDLL:
     lib.pa_reshape_and_cache_fp8.restype = I
     lib.pa_swap_blocks.argtypes = [P, P, P, P, I, P, I, I, I, I, I, I, P, P]
     lib.pa_swap_blocks.restype = I
+    lib.pa_shared_prefix_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+    lib.pa_shared_prefix_workspace_size.restype = S
+    lib.pa_decode_shared_prefix.argtypes = [P, I, P, P, P, I, P, I, P, P, I, P, P, I, I, I, I, I,
+                                            I, I, I, F, I, I, P, S, P, P]
+    lib.pa_decode_shared_prefix.restype = I
     return lib
 
 
@@ -214,6 +219,47 @@ def pa_swap_blocks(dst_key: torch.Tensor, dst_value: torch.Tensor, src_key: torc
                             src_blocks, dst_blocks, _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_swap_blocks", rc)
+
+
+def pa_shared_prefix_workspace_size(B: int, Hq: int, Hkv: int, D: int, max_context_len: int,
+                                    partition_size: int, block_size: int,
+                                    max_shared_blocks: int) -> int:
+    return int(LIB.pa_shared_prefix_workspace_size(B, Hq, Hkv, D, max_context_len,
+                                                   partition_size, block_size,
+                                                   max_shared_blocks))
+
+
+def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                            value_cache: torch.Tensor, block_tables: torch.Tensor,
+                            context_lens: torch.Tensor, shared_blocks: torch.Tensor,
+                            group_offsets: torch.Tensor, group_members: torch.Tensor,
+                            max_group_size: int, max_shared_blocks: int, scale: float,
+                            max_context_len: int, partition_size: int = 0,
+                            workspace: Optional[torch.Tensor] = None,
+                            err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pa_decode for groups of sequences sharing their leading blocks (see
+    pa_decode_shared_prefix in include/pa.h): shared blocks read once per group."""
+    B, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    rc = LIB.pa_decode_shared_prefix(
+        _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+        _ptr(shared_blocks), group_offsets.shape[0] - 1, _ptr(group_offsets), _ptr(group_members),
+        int(max_group_size), int(max_shared_blocks), B, Hq, Hkv, D, block_size, num_blocks,
+        float(scale), int(max_context_len), int(partition_size), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_decode_shared_prefix", rc)
+
+
+def shared_prefix_workspace_for(query: torch.Tensor, key_cache: torch.Tensor,
+                                max_context_len: int, max_shared_blocks: int,
+                                partition_size: int = 0) -> Optional[torch.Tensor]:
+    B, Hq, D = query.shape
+    n = pa_shared_prefix_workspace_size(B, Hq, key_cache.shape[2], D, max_context_len,
+                                        partition_size, key_cache.shape[1], max_shared_blocks)
+    return None if n == 0 else torch.empty(n, dtype=torch.uint8, device=query.device)
 
 
 def workspace_for(query: torch.Tensor, key_cache: torch.Tensor, max_context_len: int,

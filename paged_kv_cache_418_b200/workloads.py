@@ -361,7 +361,8 @@ def build_shared_prefix_case(name: str, dtype: int, groups: int, children: int,
         context_lens=ctx.astype(np.int32), new_key=nk, new_value=nv, slot_mapping=slots,
         block_mapping=np.asarray(pairs, dtype=np.int64).reshape(-1, 2), seed=seed,
         meta={"groups": groups, "children": children, "suffix": suffix,
-              "parent_len": parent_len, "pre_tables": pre_tables})
+              "parent_len": parent_len, "pre_tables": pre_tables,
+              "prefix_blocks": prefix_blocks})
 
 
 # --------------------------------------------------------------------------
