@@ -80,10 +80,11 @@ def _load():
                                                      ctypes.c_float, P, I, I, I, I, I]
         lib.oracle_fp8_encode.argtypes = [P, P, LL]
         lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, I, ctypes.c_size_t, I, I]
+        lib.oracle_prefill.argtypes = [P, P, P, P, I, P, I, P, P, I, I, I, I, I, I, D, I]
         for fn in ("oracle_gather", "oracle_decode", "oracle_decode_partitioned",
                    "oracle_reshape_and_cache", "oracle_copy_blocks", "oracle_widen",
                    "oracle_max_threads", "oracle_decode_kv", "oracle_reshape_and_cache_fp8",
-                   "oracle_fp8_encode", "oracle_swap_blocks"):
+                   "oracle_fp8_encode", "oracle_swap_blocks", "oracle_prefill"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -239,3 +240,19 @@ def swap_blocks(dst_k: np.ndarray, dst_v: np.ndarray, src_k: np.ndarray, src_v: 
     assert dst_k[0].nbytes == blk and dst_k.dtype == src_k.dtype
     _check(_load().oracle_swap_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
                                       _ptr(bm), bm.shape[0], blk, src_k.shape[0], dst_k.shape[0]))
+
+
+def prefill(q, k_cache, v_cache, dtype: int, block_tables, context_lens, query_start,
+            scale: float, n_threads: int = 0) -> np.ndarray:
+    """Causal prefill attention in float64: [T, Hq, D] for the packed new tokens."""
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    bt, cl, qs = _c(block_tables, np.int32), _c(context_lens, np.int32), _c(query_start, np.int32)
+    T, Hq, D = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    B = cl.shape[0]
+    assert qs.shape[0] == B + 1 and int(qs[-1]) == T
+    out = np.empty((T, Hq, D), dtype=np.float64)
+    _check(_load().oracle_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), dtype,
+                                  _ptr(bt), bt.shape[1], _ptr(cl), _ptr(qs), B, Hq, hkv, D, bs, nb,
+                                  float(scale), int(n_threads)))
+    return out

@@ -43,6 +43,14 @@
  *                     src block (all rows, all heads) of K and V to dst, all
  *                     sources read before any write. "vLLM 与 LLM 推理部署实战"
  *                     section 2.2 (a write to a shared block copies it whole).
+ *  oracle_prefill     Prompt (chunked-prefill) attention: new token i of
+ *                     sequence b, at position p = ctx_b - n_b + i, attends the
+ *                     cached tokens 0 .. p (causal) through the block table,
+ *                     by the same two-pass softmax as oracle_decode.
+ *                     "推理引擎内部机制——PagedAttention、连续批处理、分块预填充"
+ *                     (chunked prefill: a long prompt's chunks attend the
+ *                     paged cache). Causality is the plain reading of a
+ *                     prompt's self-attention.
  *  oracle_swap_blocks The same whole-block copy between two different pools
  *                     (host and device memory): preemption by swapping moves
  *                     a sequence's blocks to CPU memory and back. "vLLM与
@@ -249,6 +257,47 @@ int oracle_decode_kv(double* out, const void* q, int q_dtype, const void* kpool,
       e = attend_row(out + r * D, q, q_dtype, kpool, vpool, kv_dtype, k_scale, v_scale,
                      block_tables + (size_t)b * max_blocks, context_lens[b], Hq, Hkv, D, bs,
                      num_blocks, scale, b, hq);
+    if (e != OR_OK) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+      { if (err == OR_OK) err = e; }
+    }
+  }
+  return err;
+}
+
+/*
+ * Causal prefill: out [T, Hq, D]; query [T, Hq, D] (packed new tokens, rows
+ * query_start[b] .. query_start[b+1] of sequence b); context_lens after the chunk.
+ */
+int oracle_prefill(double* out, const void* q, const void* kpool, const void* vpool, int dtype,
+                   const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                   const int32_t* query_start, int B, int Hq, int Hkv, int D, int bs,
+                   int num_blocks, double scale, int n_threads) {
+  if (!out || !query_start) return OR_ERR_ARG;
+  int rc = check_decode_args(q, kpool, vpool, dtype, block_tables, max_blocks, context_lens, B,
+                             Hq, Hkv, D, bs);
+  if (rc != OR_OK || dtype == OR_FP8) return rc ? rc : OR_ERR_ARG;
+  for (int b = 0; b < B; ++b) {
+    int n = query_start[b + 1] - query_start[b];
+    if (n < 0 || n > context_lens[b]) return OR_ERR_ARG;
+  }
+  long long T = query_start[B];
+  int err = OR_OK;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (long long r = 0; r < T * Hq; ++r) {
+    long long t = r / Hq;
+    int hq = (int)(r % Hq), b = 0;
+    while (query_start[b + 1] <= t) ++b;                /* the sequence of query row t */
+    int n = query_start[b + 1] - query_start[b];
+    int pos = context_lens[b] - n + (int)(t - query_start[b]);
+    int e = attend_row(out + r * D, q, dtype, kpool, vpool, dtype, 1.0, 1.0,
+                       block_tables + (size_t)b * max_blocks, pos + 1, Hq, Hkv, D, bs,
+                       num_blocks, scale, (int)t, hq);
     if (e != OR_OK) {
 #ifdef _OPENMP
 #pragma omp critical

@@ -366,6 +366,105 @@ def build_shared_prefix_case(name: str, dtype: int, groups: int, children: int,
 
 
 # --------------------------------------------------------------------------
+# chunked prefill: a chunk of new tokens per sequence, already in the cache
+# --------------------------------------------------------------------------
+@dataclass
+class PrefillCase:
+    """Inputs of one prefill attention call (host arrays in storage types)."""
+
+    name: str
+    dtype: int
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    block_size: int
+    num_blocks: int
+    max_blocks: int
+    scale: float
+    q: np.ndarray               # [T, Hq, D] new tokens, packed by sequence
+    k_cache: np.ndarray         # [num_blocks, block_size, Hkv, D], new tokens included
+    v_cache: np.ndarray
+    block_tables: np.ndarray    # [B, max_blocks] int32
+    context_lens: np.ndarray    # [B] int32, prior + new
+    query_start: np.ndarray     # [B + 1] int32
+    seed: int = 0
+
+    @property
+    def T(self) -> int:
+        return int(self.query_start[-1])
+
+    @property
+    def max_query_len(self) -> int:
+        return int(np.diff(self.query_start).max()) if self.B else 0
+
+    @property
+    def max_context_len(self) -> int:
+        return int(self.context_lens.max()) if self.B else 0
+
+    def attention_flops(self) -> int:
+        """4 * D flops per (query head, attended key): the QK and PV products."""
+        n = np.diff(self.query_start)
+        prior = self.context_lens - n
+        keys = sum(int(n[b]) * int(prior[b]) + int(n[b]) * (int(n[b]) + 1) // 2
+                   for b in range(self.B))
+        return 4 * self.D * self.Hq * keys
+
+
+def build_prefill_case(name: str, dtype: int, Hq: int, Hkv: int, D: int, block_size: int,
+                       prior_lens: Seq[int], new_lens: Seq[int], seed: int,
+                       extra_blocks: int = 3) -> PrefillCase:
+    """Sequences with prior_lens[b] cached tokens and a chunk of new_lens[b] tokens
+    whose K/V rows are already in the pool (written by reshape_and_cache)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    prior = np.asarray(prior_lens, dtype=np.int64)
+    new = np.asarray(new_lens, dtype=np.int64)
+    B = len(prior)
+    ctx = prior + new
+    bs = block_size
+    num_blocks = int(sum((c + bs - 1) // bs for c in ctx)) + extra_blocks
+    bm = BlockManager(num_blocks, bs, rng.permutation(num_blocks))
+    for b in range(B):
+        bm.allocate_prefill(b, int(ctx[b]))
+    MB = max(1, max(len(bm.seqs[b].block_table) for b in range(B)))
+    tables = np.full((B, MB), -1, dtype=np.int32)
+    for b in range(B):
+        tb = bm.seqs[b].block_table
+        tables[b, :len(tb)] = tb
+    st = _STORAGE[dtype]
+    T = int(new.sum())
+    q = round_to_storage(rng.standard_normal((T, Hq, D), dtype=np.float32), dtype).view(st)
+    kc = nan_fill((num_blocks, bs, Hkv, D), dtype)
+    vc = nan_fill((num_blocks, bs, Hkv, D), dtype)
+    for b in range(B):
+        n = int(ctx[b])
+        k = round_to_storage(rng.standard_normal((n, Hkv, D), dtype=np.float32), dtype).view(st)
+        v = round_to_storage(rng.standard_normal((n, Hkv, D), dtype=np.float32), dtype).view(st)
+        _fill_rows(kc, tables[b], bs, 0, k)
+        _fill_rows(vc, tables[b], bs, 0, v)
+    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    return PrefillCase(name=name, dtype=dtype, B=B, Hq=Hq, Hkv=Hkv, D=D, block_size=bs,
+                       num_blocks=num_blocks, max_blocks=MB, scale=float(1.0 / math.sqrt(D)),
+                       q=q, k_cache=kc, v_cache=vc, block_tables=tables,
+                       context_lens=ctx.astype(np.int32), query_start=qs, seed=seed)
+
+
+def prefill_to_torch(c: PrefillCase, device="cpu") -> Dict[str, "object"]:
+    import torch
+
+    def el(a):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if c.dtype == BF16:
+            t = t.view(torch.int16).view(torch.bfloat16)
+        return t.to(device)
+
+    ix = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    return {"q": el(c.q), "k_cache": el(c.k_cache), "v_cache": el(c.v_cache),
+            "block_tables": ix(c.block_tables), "context_lens": ix(c.context_lens),
+            "query_start": ix(c.query_start)}
+
+
+# --------------------------------------------------------------------------
 # the five named workloads
 # --------------------------------------------------------------------------
 WORKLOADS = {

@@ -463,3 +463,47 @@ def test_swap_blocks_moves_whole_blocks_between_pools():
         oracle.swap_blocks(dst_k, dst_v, src_k, src_v, np.array([[9, 0]]))
     with pytest.raises(oracle.OracleError):
         oracle.swap_blocks(dst_k, dst_v, src_k, src_v, np.array([[0, 5]]))
+
+
+# -- chunked prefill ---------------------------------------------------------------
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", [(F16, 8, 2, 32, 4), (BF16, 4, 4, 16, 8),
+                                              (F32, 6, 3, 64, 16)])
+def test_prefill_matches_sdpa_with_a_bottom_right_causal_mask(dtype, Hq, Hkv, D, bs):
+    from paged_kv_cache_418_b200.workloads import build_prefill_case
+    c = build_prefill_case("pf", dtype, Hq, Hkv, D, bs, prior_lens=[0, 5, 17, 0],
+                           new_lens=[7, 1, 9, 0], seed=50 + D)
+    out = oracle.prefill(c.q, c.k_cache, c.v_cache, dtype, c.block_tables, c.context_lens,
+                         c.query_start, c.scale)
+    for b in range(c.B):
+        n = int(c.query_start[b + 1] - c.query_start[b])
+        if n == 0:
+            continue
+        ctx = int(c.context_lens[b])
+        # contiguous K/V by block-wise reshape of the table's blocks (not per token)
+        blk = c.block_tables[b, :(ctx + bs - 1) // bs]
+        k64 = storage_to_float64(c.k_cache[blk].reshape(-1, Hkv, D)[:ctx], dtype)
+        v64 = storage_to_float64(c.v_cache[blk].reshape(-1, Hkv, D)[:ctx], dtype)
+        q64 = storage_to_float64(c.q[c.query_start[b]:c.query_start[b + 1]], dtype)
+        pos = ctx - n + np.arange(n)
+        mask = torch.from_numpy(np.arange(ctx)[None, :] <= pos[:, None])     # [n, ctx]
+        qt = torch.from_numpy(np.ascontiguousarray(q64.transpose(1, 0, 2)))[None]
+        kt = torch.from_numpy(np.ascontiguousarray(k64.transpose(1, 0, 2)))[None]
+        vt = torch.from_numpy(np.ascontiguousarray(v64.transpose(1, 0, 2)))[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, attn_mask=mask, scale=c.scale, enable_gqa=Hq != Hkv)[0].numpy()
+        got = out[c.query_start[b]:c.query_start[b + 1]].transpose(1, 0, 2)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_prefill_first_token_of_an_empty_sequence_is_its_v_row():
+    from paged_kv_cache_418_b200.workloads import build_prefill_case
+    c = build_prefill_case("pf1", BF16, 8, 2, 16, 4, prior_lens=[0], new_lens=[5], seed=3)
+    out = oracle.prefill(c.q, c.k_cache, c.v_cache, BF16, c.block_tables, c.context_lens,
+                         c.query_start, c.scale)
+    v0 = storage_to_float64(c.v_cache[c.block_tables[0, 0], 0], BF16)     # token 0, [Hkv, D]
+    for hq in range(8):
+        assert np.array_equal(out[0, hq], v0[hq // 4])
+    with pytest.raises(oracle.OracleError):
+        bad = c.context_lens.copy()
+        bad[0] = 3                                   # fewer tokens than the chunk holds
+        oracle.prefill(c.q, c.k_cache, c.v_cache, BF16, c.block_tables, bad, c.query_start, c.scale)
