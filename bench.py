@@ -61,6 +61,8 @@ def parse():
                    help="fewer sequences of the same workload (profiling captures)")
     p.add_argument("--shared-prefix", action="store_true",
                    help="decode the shared-prefix workload with pa_decode_shared_prefix")
+    p.add_argument("--prefill", action="store_true",
+                   help="measure paged prefill attention (causal chunks) instead of decode")
     p.add_argument("--swap", action="store_true",
                    help="measure swap_blocks (device <-> pinned host) instead of the decode step")
     return p.parse_args()
@@ -588,8 +590,112 @@ def swap_arm(args, rank: int, world: int, local_rank: int):
     }
 
 
+PREFILL_METRIC = "paged prefill attention TFLOP/s"
+
+
+def prefill_case(rank: int):
+    """Chunked prefill of a Llama-3-70B-shaped batch: 8 sequences with U[0, 2048]
+    cached tokens each take a 512-token chunk (64 query heads over 8 KV heads,
+    D = 128, bf16, 16-token blocks)."""
+    rng = np.random.default_rng(rank_seed(8, rank))
+    prior = rng.integers(0, 2049, size=8)
+    return W.build_prefill_case("prefill-chunk512-llama3-70b-bf16", W.BF16, Hq=64, Hkv=8, D=128,
+                                block_size=16, prior_lens=prior, new_lens=[512] * 8,
+                                seed=rank_seed(8, rank))
+
+
+def prefill_arm(args, rank: int, world: int, local_rank: int):
+    import torch
+    import oracle
+    from paged_kv_cache_418_b200 import ops
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    c = prefill_case(rank)
+    t = W.prefill_to_torch(c, dev)
+    out = torch.empty((c.T, c.Hq, c.D), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    run = lambda: ops.pa_prefill(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                 t["context_lens"], t["query_start"], c.max_query_len, c.scale,
+                                 c.max_context_len, err, stream)
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize(dev)
+    K = max(1, min(args.steps, 200))
+    sampler = ClockSampler(gpu_smi_id(local_rank))
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        run()
+    e1.record(stream)
+    e1.synchronize()
+    clocks = sampler.stop()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error flag {int(err.item())}")
+    ms = e0.elapsed_time(e1) / K
+    (ms,) = max_over_ranks([ms], world, dev)
+    flops = c.attention_flops()
+    tflops = flops / (ms / 1e3) / 1e12
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak = float(json.load(open(path))["bf16_tflops"]) if os.path.exists(path) else 1590.0
+    # end to end: query and tables from pinned host memory, output back, every call
+    hq = t["q"].cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    for _ in range(K):
+        t["q"].copy_(hq, non_blocking=True)
+        run()
+        hout.copy_(out, non_blocking=True)
+    e3.record(stream)
+    e3.synchronize()
+    e_ms = e2.elapsed_time(e3) / K
+    # oracle on the host cores: the first sequence's chunk (a bounded sample)
+    sub = W.build_prefill_case("sample", W.BF16, Hq=64, Hkv=8, D=128, block_size=16,
+                               prior_lens=[int(c.context_lens[0]) - 512], new_lens=[64],
+                               seed=1)
+    t0 = time.perf_counter()
+    oracle.prefill(sub.q, sub.k_cache, sub.v_cache, W.BF16, sub.block_tables, sub.context_lens,
+                   sub.query_start, sub.scale)
+    cpu_s = time.perf_counter() - t0
+    return {
+        "metric": PREFILL_METRIC, "value": round(tflops * world, 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": K, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": c.name, "B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "head_dim": c.D,
+                   "block_size": c.block_size, "new_tokens": c.T,
+                   "prior_tokens": int((c.context_lens - 512).sum()),
+                   "flops_per_step": flops, "l2": "K/V of the batch read once per 8-token "
+                   "query chunk; inputs resident, no flush (compute-bound)"},
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                     "peak_source": "bf16_tflops (measured, burst)",
+                     "kernel": "multi_query_tc_kernel (prefill), per launch; algorithmic flops "
+                               "4*D per (query head, attended key)"},
+        "gpu_launches": K,
+        "clocks": clocks,
+        "e2e": {"value": round(flops / (e_ms / 1e3) / 1e12 * world, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "cpu_baseline": {"value": round(sub.attention_flops() / cpu_s / 1e12, 6),
+                         "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"64 of the first sequence's 512 new tokens, {cpu_s:.1f} s"},
+    }
+
+
 def main():
     args = parse()
+    if args.prefill:
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if args.impl == "reference" or world > 1:
+            return 0 if rank else (print(json.dumps({"impl": args.impl, "unavailable":
+                "prefill measurement runs on one GPU with --impl ours"})) or 0)
+        print(json.dumps(prefill_arm(args, rank, world, int(os.environ.get("LOCAL_RANK", "0")))),
+              flush=True)
+        return 0
     if args.swap:
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -294,6 +294,37 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
                             int max_context_len, int partition_size, void* workspace,
                             size_t workspace_bytes, uint32_t* err_flag, void* stream);
 
+/*
+ * pa_prefill -- paged prefill (prompt or chunked-prefill) attention: each new
+ * query token attends, causally, to its sequence's cached tokens up to and
+ * including itself. Long prompts are cut into chunks that run between decode
+ * steps ("推理引擎内部机制——PagedAttention、连续批处理、分块预填充", chunked
+ * prefill); a chunk's K/V rows are written into the pool first
+ * (pa_reshape_and_cache), then its queries attend through the block table.
+ *
+ * query        [T, Hq, D] of dtype: the new tokens of all sequences, packed;
+ *              sequence b's are rows [query_start[b], query_start[b + 1]);
+ * query_start  [B + 1] int32, non-decreasing, query_start[B] = T;
+ * context_lens [B] int32: tokens of sequence b in the pool after the chunk,
+ *              its new tokens included; new token i of b (0-based) sits at
+ *              position context_lens[b] - n_b + i and attends positions
+ *              0 .. that position (n_b = query_start[b + 1] - query_start[b]);
+ * max_query_len the largest n_b (host-side bound);
+ * out          [T, Hq, D] of out_dtype (PA_F32 or dtype);
+ * key_cache, value_cache, block_tables, max_blocks_per_seq, block_size,
+ * num_blocks, scale, max_context_len, err_flag, stream: as pa_decode.
+ * Supported: 16-bit K/V (PA_F16, PA_BF16), D = 128, the pa_decode block and
+ * group sizes; otherwise PA_ERR_UNSUPPORTED. A sequence with n_b >
+ * context_lens[b] (or a context the table cannot hold) sets PA_DEV_BAD_CTX and
+ * its rows are not written. No workspace.
+ */
+int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cache,
+               const void* value_cache, int dtype, const int32_t* block_tables,
+               int max_blocks_per_seq, const int32_t* context_lens, const int32_t* query_start,
+               int B, int T, int max_query_len, int Hq, int Hkv, int D, int block_size,
+               int num_blocks, float scale, int max_context_len, uint32_t* err_flag,
+               void* stream);
+
 /* Static text for a pa_status value. */
 const char* pa_status_string(int status);
 

@@ -23,6 +23,14 @@
 // tile needs no reduction across threads; the column sums l are per-thread
 // partial sums reduced once per unit.
 //
+// The same kernel runs paged prefill (PF = true): a chunk of a sequence's new
+// query tokens attends, causally, to the sequence's own blocks — the prompt
+// phase before decode (the lesson, "分块预填充": long prompts are cut into
+// chunks that run beside decode steps). There a unit is (sequence b, chunk c
+// of up to kNQ / G new tokens, KV head h); row q = (token q / G, query head
+// q % G) at position pos0 + q / G attends keys [0, pos0 + q / G]; the unit
+// covers all of them and writes the normalised output rows directly.
+//
 // CTA = 6 warps, persistent over units u = blockIdx.x + k * gridDim.x:
 // warps 0-3 softmax and epilogue (TMEM lanes 0-127), warp 4 TMA producer,
 // warp 5 MMA issuer (it also owns the tensor memory). Every wait is bounded;
@@ -56,7 +64,8 @@ constexpr int kPPart = 2 * kNQ * 128;
 constexpr int kPBuf = 2 * kPPart;
 constexpr int OFF_MREF = OFF_P + 2 * kPBuf;     // [3][kNQ] reference, old, new maxima
 constexpr int OFF_RED = OFF_MREF + 3 * kNQ * 4; // [4 warps][kNQ]
-constexpr int OFF_BAR = OFF_RED + 4 * kNQ * 4;
+constexpr int OFF_LIM = OFF_RED + 4 * kNQ * 4;  // [kNQ] prefill causal limits
+constexpr int OFF_BAR = OFF_LIM + kNQ * 4;
 enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY, B_SFULL, B_SFREE = B_SFULL + 2,
        B_PREADY = B_SFREE + 2, B_OFULL = B_PREADY + 2, B_ODONE = B_OFULL + 2, B_DONE, B_COUNT };
 constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
@@ -80,11 +89,40 @@ struct PrefixArgs {
   float* ws_m;
   float* ws_l;
   uint32_t* err_flag;
+  // prefill mode
+  const int32_t* query_start;                   // [B + 1]: new tokens of b are query rows [qs_b, qs_{b+1})
+  const int32_t* context_lens;                  // [B]: tokens in the cache, the new ones included
+  int max_context_len;
+  void* out;                                    // [T, Hq, D] of out_dtype
+  int out_dtype;
 };
 
 struct PUnit {
   int g, mbeg, nm, h, j, b0, t0, t1, ntiles, nq, nqp;
+  int qrow0, pos0;                              // prefill: first query row, its position
+  bool bad;                                     // prefill: the sequence's lengths are inconsistent
 };
+
+// Prefill unit u = (sequence b, chunk c, KV head h): nm = tokens of the chunk.
+__device__ __forceinline__ PUnit prefill_unit(const PrefixArgs& a, int G, int mc, long long u) {
+  PUnit x;
+  x.h = (int)(u % a.Hkv);
+  const long long t = u / a.Hkv;
+  const int c = (int)(t % a.chunks);
+  const int b = (int)(t / a.chunks);
+  const int qs = __ldg(a.query_start + b), qe = __ldg(a.query_start + b + 1);
+  const int n = qe - qs, ctx = __ldg(a.context_lens + b);
+  x.bad = n < 0 || ctx < n || ctx > a.max_blocks * a.bs || ctx > a.max_context_len;
+  x.g = b; x.mbeg = 0; x.j = 0; x.b0 = b; x.t0 = 0;
+  x.nm = x.bad ? 0 : min(mc, n - c * mc);
+  x.qrow0 = qs + c * mc;
+  x.pos0 = ctx - n + c * mc;
+  x.t1 = x.nm > 0 ? x.pos0 + x.nm : 0;          // keys of the chunk's last token, inclusive
+  x.ntiles = (x.t1 + kTile - 1) / kTile;
+  x.nq = x.nm * G;
+  x.nqp = (x.nq + 15) / 16 * 16;
+  return x;
+}
 
 // Decode unit u; nm <= 0 means the unit has no rows (every role skips it).
 __device__ __forceinline__ PUnit prefix_unit(const PrefixArgs& a, int G, int mc, long long u) {
@@ -107,17 +145,23 @@ __device__ __forceinline__ PUnit prefix_unit(const PrefixArgs& a, int G, int mc,
   x.ntiles = x.t1 > x.t0 ? (x.t1 - x.t0 + kTile - 1) / kTile : 0;
   x.nq = x.nm * G;
   x.nqp = (x.nq + 15) / 16 * 16;
+  x.qrow0 = 0; x.pos0 = 0; x.bad = false;
   return x;
+}
+
+template <bool PF>
+__device__ __forceinline__ PUnit mq_unit(const PrefixArgs& a, int G, int mc, long long u) {
+  return PF ? prefill_unit(a, G, mc, u) : prefix_unit(a, G, mc, u);
 }
 
 // Named barrier of the 128 softmax threads; vote = OR of every thread's flag.
 __device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 __device__ __forceinline__ bool sm_vote(bool x) { return wg_vote_or(x, 0); }
 
-template <int FMT, int BS>
+template <int FMT, int BS, bool PF>
 __global__ void __launch_bounds__(kThreads, 1)
-prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV) {
+multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV) {
   constexpr int NB_T = kTile / BS;              // physical blocks per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -128,8 +172,9 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.Hq / a.Hkv;
-  const int mc = kNQ / G;                       // members per chunk
-  const long long U = (long long)a.num_groups * a.chunks * a.Hkv * a.parts;
+  const int mc = kNQ / G;                       // members (prefill: tokens) per chunk
+  const long long U = PF ? (long long)a.B * a.chunks * a.Hkv
+                         : (long long)a.num_groups * a.chunks * a.Hkv * a.parts;
   pdl_trigger();
 
   if (threadIdx.x == 0) {
@@ -174,7 +219,7 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
     if (lane == 0) {
       int tc_ = 0, issued = 0;
       for (long long u = blockIdx.x; u < U; u += gridDim.x) {
-        const PUnit x = prefix_unit(a, G, mc, u);
+        const PUnit x = mq_unit<PF>(a, G, mc, u);
         if (x.nm <= 0 || x.ntiles == 0) continue;
         const int32_t* table = a.block_tables + (size_t)x.b0 * a.max_blocks;
         // block ids of tile k of this unit (-1: no block there)
@@ -231,7 +276,7 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
       int tc_ = 0, ua = 0;
       bool ok = true;
       for (long long u = blockIdx.x; u < U && ok; u += gridDim.x) {
-        const PUnit x = prefix_unit(a, G, mc, u);
+        const PUnit x = mq_unit<PF>(a, G, mc, u);
         if (x.nm <= 0 || x.ntiles == 0) continue;
         const uint32_t idesc_s = make_idesc(FMT, 0, 0, x.nqp, 128);
         const uint32_t idesc_o = make_idesc(FMT, 1, 0, x.nqp, 128);
@@ -295,6 +340,7 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
     float* mold = mref + kNQ;
     float* mnew = mold + kNQ;
     float* red = reinterpret_cast<float*>(smem + OFF_RED);
+    int* lim = reinterpret_cast<int*>(smem + OFF_LIM);   // prefill: last key of each column
     bool failed = false, stop = false;
     int tc_ = 0, ua = 0;
     auto wait_pv = [&](int t) {                  // output product of tile t has completed
@@ -314,14 +360,21 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
       sm_sync();
     };
     for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
-      const PUnit x = prefix_unit(a, G, mc, u);
+      const PUnit x = mq_unit<PF>(a, G, mc, u);
+      if (PF && x.bad && x.h == 0 && r == 0 && (u / a.Hkv) % a.chunks == 0)
+        flag_error(a.err_flag, PA_DEV_BAD_CTX);
       if (x.nm <= 0) continue;
+      // the (query token, head) row q of the unit in the query matrix
+      auto q_row = [&](int q) -> size_t {
+        const int tokrow = PF ? x.qrow0 + q / G : __ldg(a.group_members + x.mbeg + q / G);
+        return (size_t)tokrow * a.Hq + (size_t)x.h * G + (q % G);
+      };
       // rows of the unit: q = m * G + gg -> (sequence, query head) slot of partition j
       auto slot_row = [&](int q) -> size_t {
         const int b = __ldg(a.group_members + x.mbeg + q / G);
         return ((size_t)b * a.P + x.j) * a.Hq + (size_t)x.h * G + (q % G);
       };
-      if (x.ntiles == 0) {
+      if (!PF && x.ntiles == 0) {
         // this partition of the prefix holds no tokens: an empty partial
         for (int q = 0; q < x.nq; ++q) a.ws_acc[slot_row(q) * kD + r] = 0.f;
         if (r < x.nq) {
@@ -335,16 +388,15 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
       for (int c = r; c < x.nqp * 16; c += 128) {
         const int q = c >> 4, k16 = c & 15, hh = k16 >> 3, kk = k16 & 7;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (q < x.nq) {
-          const int b = __ldg(a.group_members + x.mbeg + q / G);
-          const size_t row = (size_t)b * a.Hq + (size_t)x.h * G + (q % G);
-          v = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.q) + row * (kD * 2) +
+        if (q < x.nq)
+          v = *reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.q) + q_row(q) * (kD * 2) +
                                               k16 * 16);
-        }
         *reinterpret_cast<uint4*>(smem + OFF_Q + hh * (kNQ * 128) + q * 128 + ((kk ^ (q & 7)) << 4)) = v;
       }
+      if (PF && r < kNQ) lim[r] = x.pos0 + r / G;   // causal: the last key of column r
       fence_proxy_async();
       mbar_arrive(bar(B_QFULL));
+      if (PF) sm_sync();
 
       float l[kNQ];
 #pragma unroll
@@ -366,7 +418,8 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
         tc_fence_before();
         mbar_arrive(bar(B_SFREE + (tc_ & 1)));
 #pragma unroll
-        for (int q = 0; q < kNQ; ++q) s[q] = (valid && q < x.nq) ? s[q] * a.scale_log2 : -CUDART_INF_F;
+        for (int q = 0; q < kNQ; ++q)
+          s[q] = (valid && q < x.nq && (!PF || tok <= lim[q])) ? s[q] * a.scale_log2 : -CUDART_INF_F;
         if (sm_vote(failed)) { stop = true; break; }
         if (k == 0) {
           col_max(s, mref);
@@ -446,7 +499,11 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
         if (lane == 0) red[warp * kNQ + q] = v;
       }
       sm_sync();
-      if (r < x.nq) {
+      if (PF) {
+        // prefill: each column's exp-sum, then normalised rows straight to the output
+        if (r < kNQ) mold[r] = red[r] + red[kNQ + r] + red[2 * kNQ + r] + red[3 * kNQ + r];
+        sm_sync();
+      } else if (r < x.nq) {
         const size_t sr = slot_row(r);
         a.ws_m[sr] = mref[r];
         a.ws_l[sr] = red[r] + red[kNQ + r] + red[2 * kNQ + r] + red[3 * kNQ + r];
@@ -457,8 +514,15 @@ prefix_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
         float o[16];
         tmem_ld16(tmem_o + lane_off + c, o);
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          if (c + e < x.nq) a.ws_acc[slot_row(c + e) * kD + r] = o[e];
+        for (int e = 0; e < 16; ++e) {
+          if (c + e >= x.nq) continue;
+          if (PF) {
+            const float L = mold[c + e];
+            store_out(a.out, q_row(c + e) * kD + r, L > 0.f ? o[e] / L : 0.f, a.out_dtype);
+          } else {
+            a.ws_acc[slot_row(c + e) * kD + r] = o[e];
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(bar(B_ODONE));
@@ -515,10 +579,10 @@ bool make_prefix_maps(const void* k_cache, const void* v_cache, int dtype, int b
   return true;
 }
 
-template <int FMT, int BS>
-int launch_prefix_t(const PrefixArgs& a, const CUtensorMap& k, const CUtensorMap& v,
-                    cudaStream_t stream) {
-  auto kern = prefix_tc_kernel<FMT, BS>;
+template <int FMT, int BS, bool PF>
+int launch_mq_t(const PrefixArgs& a, const CUtensorMap& k, const CUtensorMap& v,
+                cudaStream_t stream) {
+  auto kern = multi_query_tc_kernel<FMT, BS, PF>;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
@@ -526,7 +590,8 @@ int launch_prefix_t(const PrefixArgs& a, const CUtensorMap& k, const CUtensorMap
       return PA_ERR_CUDA;
     attr = true;
   }
-  const long long U = (long long)a.num_groups * a.chunks * a.Hkv * a.parts;
+  const long long U = PF ? (long long)a.B * a.chunks * a.Hkv
+                         : (long long)a.num_groups * a.chunks * a.Hkv * a.parts;
   if (U <= 0) return PA_OK;
   int dev = 0, sms = kSMs;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -571,8 +636,35 @@ int launch_prefix_tc(const DecodeArgs& d, int dtype, const int32_t* group_offset
   a.ws_acc = d.ws_acc; a.ws_m = d.ws_m; a.ws_l = d.ws_l;
   a.err_flag = d.err_flag;
   if (dtype == PA_BF16)
-    return d.bs == 16 ? launch_prefix_t<1, 16>(a, k, v, stream) : launch_prefix_t<1, 32>(a, k, v, stream);
-  return d.bs == 16 ? launch_prefix_t<0, 16>(a, k, v, stream) : launch_prefix_t<0, 32>(a, k, v, stream);
+    return d.bs == 16 ? launch_mq_t<1, 16, false>(a, k, v, stream)
+                      : launch_mq_t<1, 32, false>(a, k, v, stream);
+  return d.bs == 16 ? launch_mq_t<0, 16, false>(a, k, v, stream)
+                    : launch_mq_t<0, 32, false>(a, k, v, stream);
+}
+
+int launch_prefill_tc(const PrefillLaunch& p, cudaStream_t stream) {
+  CUtensorMap k, v;
+  if (!make_prefix_maps(p.k_cache, p.v_cache, p.dtype, p.bs, p.Hkv, p.num_blocks, &k, &v))
+    return PA_ERR_CUDA;
+  PrefixArgs a{};
+  a.q = p.q;
+  a.block_tables = p.block_tables;
+  a.max_blocks = p.max_blocks;
+  a.query_start = p.query_start;
+  a.context_lens = p.context_lens;
+  a.max_context_len = p.max_context_len;
+  a.out = p.out;
+  a.out_dtype = p.out_dtype;
+  a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.bs = p.bs; a.num_blocks = p.num_blocks;
+  a.scale_log2 = p.scale_log2;
+  a.chunks = (p.max_query_len + kNQ / (p.Hq / p.Hkv) - 1) / (kNQ / (p.Hq / p.Hkv));
+  a.parts = 1;
+  a.err_flag = p.err_flag;
+  if (p.dtype == PA_BF16)
+    return p.bs == 16 ? launch_mq_t<1, 16, true>(a, k, v, stream)
+                      : launch_mq_t<1, 32, true>(a, k, v, stream);
+  return p.bs == 16 ? launch_mq_t<0, 16, true>(a, k, v, stream)
+                    : launch_mq_t<0, 32, true>(a, k, v, stream);
 }
 
 }  // namespace pa

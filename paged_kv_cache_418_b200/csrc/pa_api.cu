@@ -324,6 +324,39 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   return rc;
 }
 
+int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cache,
+               const void* value_cache, int dtype, const int32_t* block_tables,
+               int max_blocks_per_seq, const int32_t* context_lens, const int32_t* query_start,
+               int B, int T, int max_query_len, int Hq, int Hkv, int D, int block_size,
+               int num_blocks, float scale, int max_context_len, uint32_t* err_flag,
+               void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_DTYPE;
+  if (B < 0 || T < 0 || max_query_len < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 ||
+      num_blocks < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
+    return PA_ERR_SHAPE;
+  if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (!prefix_tc_supported(dtype, Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if (B == 0 || T == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
+      !query_start)
+    return PA_ERR_NULL;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_ALIGN;
+  PrefillLaunch p{};
+  p.out = out; p.out_dtype = out_dtype; p.q = query;
+  p.k_cache = key_cache; p.v_cache = value_cache; p.dtype = dtype;
+  p.block_tables = block_tables; p.max_blocks = max_blocks_per_seq;
+  p.context_lens = context_lens; p.query_start = query_start;
+  p.B = B; p.max_query_len = max_query_len; p.Hq = Hq; p.Hkv = Hkv; p.bs = block_size;
+  p.num_blocks = num_blocks;
+  p.scale_log2 = scale * kLog2e;
+  p.max_context_len = max_context_len;
+  p.err_flag = err_flag;
+  return launch_prefill_tc(p, static_cast<cudaStream_t>(stream));
+}
+
 int pa_swap_blocks(void* dst_key, void* dst_value, const void* src_key, const void* src_value,
                    int dtype, const int64_t* block_mapping, int num_pairs, int Hkv, int D,
                    int block_size, int src_blocks, int dst_blocks, uint32_t* err_flag,

@@ -62,6 +62,25 @@ bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 int launch_merge(const DecodeArgs& a, cudaStream_t stream);
 bool prefix_tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 int prefix_chunks(int max_group_size, int G);
+
+// Paged prefill on the multi-query tensor-core kernel.
+struct PrefillLaunch {
+  void* out;
+  int out_dtype;
+  const void* q;                // [T, Hq, D]
+  const void* k_cache;
+  const void* v_cache;
+  int dtype;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;  // [B] tokens in the cache after the chunk
+  const int32_t* query_start;   // [B + 1]
+  int B, max_query_len, Hq, Hkv, bs, num_blocks;
+  float scale_log2;
+  int max_context_len;
+  uint32_t* err_flag;
+};
+int launch_prefill_tc(const PrefillLaunch& p, cudaStream_t stream);
 int launch_prefix_tc(const DecodeArgs& a, int dtype, const int32_t* group_offsets,
                      const int32_t* group_members, int num_groups, int max_group_size, int parts,
                      int part_tokens, cudaStream_t stream);

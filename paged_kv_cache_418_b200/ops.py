@@ -61,6 +61,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_shared_prefix.argtypes = [P, I, P, P, P, I, P, I, P, P, I, P, P, I, I, I, I, I,
                                             I, I, I, F, I, I, P, S, P, P]
     lib.pa_decode_shared_prefix.restype = I
+    lib.pa_prefill.argtypes = [P, I, P, P, P, I, P, I, P, P, I, I, I, I, I, I, I, I, F, I, P, P]
+    lib.pa_prefill.restype = I
     return lib
 
 
@@ -251,6 +253,24 @@ def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: t
         _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode_shared_prefix", rc)
+
+
+def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+               value_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor,
+               query_start: torch.Tensor, max_query_len: int, scale: float, max_context_len: int,
+               err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out [T,Hq,D] <- causal paged attention of the new tokens query [T,Hq,D] (see
+    pa_prefill in include/pa.h)."""
+    T, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    B = query_start.shape[0] - 1
+    rc = LIB.pa_prefill(_ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1],
+                        _ptr(context_lens), _ptr(query_start), B, T, int(max_query_len), Hq, Hkv,
+                        D, block_size, num_blocks, float(scale), int(max_context_len),
+                        _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_prefill", rc)
 
 
 def shared_prefix_workspace_for(query: torch.Tensor, key_cache: torch.Tensor,

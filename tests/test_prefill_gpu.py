@@ -1,0 +1,78 @@
+"""Paged prefill (causal, chunked) on the GPU against the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_418_b200 import ops
+from paged_kv_cache_418_b200 import workloads as W
+from pa_testlib import assert_attention_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(c, out_dtype=torch.float32, ctx=None):
+    t = W.prefill_to_torch(c, "cuda")
+    if ctx is not None:
+        t["context_lens"] = torch.from_numpy(np.asarray(ctx, dtype=np.int32)).cuda()
+    out = torch.full((c.T, c.Hq, c.D), float("nan"), dtype=out_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.pa_prefill(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                   t["query_start"], c.max_query_len, c.scale, c.max_context_len, err)
+    torch.cuda.synchronize()
+    return out, err
+
+
+SHAPES = [(dt, G, bs) for dt in (W.F16, W.BF16) for G in (1, 2, 4, 8, 16) for bs in (16, 32)]
+
+
+@pytest.mark.parametrize("dtype,G,bs", SHAPES)
+def test_prefill_every_shape(dtype, G, bs):
+    c = W.build_prefill_case("pf", dtype, Hq=2 * G, Hkv=2, D=128, block_size=bs,
+                             prior_lens=[0, 5, 130, bs, 300, 7], new_lens=[1, 40, 0, 2 * bs + 3, 129, 64],
+                             seed=G * 10 + bs + dtype)
+    out, err = _run(c)
+    ref = oracle.prefill(c.q, c.k_cache, c.v_cache, dtype, c.block_tables, c.context_lens,
+                         c.query_start, c.scale)
+    assert int(err.item()) == 0
+    assert_attention_close(out, ref, dtype, f"G={G} bs={bs}")
+
+
+def test_prefill_long_chunk_with_peaked_scores_and_16bit_output():
+    rng = np.random.default_rng(8)
+    c = W.build_prefill_case("pf-long", W.BF16, Hq=64, Hkv=8, D=128, block_size=16,
+                             prior_lens=[2000, 0], new_lens=[700, 300], seed=9)
+    # a few large K rows move the reference maxima mid-sequence (the lazy rescale)
+    kc = c.k_cache.view(np.uint16)
+    boost = W.round_to_storage((rng.standard_normal((40, 8, 128)) * 100).astype(np.float32), W.BF16)
+    rows = rng.choice(2700, 40, replace=False)
+    for i, tok in enumerate(rows):
+        kc[c.block_tables[0, tok // 16], tok % 16] = boost[i]
+    out, err = _run(c, out_dtype=torch.bfloat16)
+    ref = oracle.prefill(c.q, c.k_cache, c.v_cache, W.BF16, c.block_tables, c.context_lens,
+                         c.query_start, c.scale)
+    assert int(err.item()) == 0
+    assert_attention_close(out, ref, W.BF16, "long")
+
+
+def test_prefill_bad_lengths_are_flagged():
+    c = W.build_prefill_case("pf-bad", W.F16, Hq=8, Hkv=2, D=128, block_size=16,
+                             prior_lens=[10, 4], new_lens=[5, 6], seed=4)
+    out, err = _run(c, ctx=[15, 3])                 # the second sequence holds fewer than 6
+    assert int(err.item()) & ops.PA_DEV_BAD_CTX
+    ref = oracle.prefill(c.q, c.k_cache, c.v_cache, W.F16, c.block_tables, c.context_lens,
+                         c.query_start, c.scale)
+    assert_attention_close(out[:5], ref[:5], W.F16, "good sequence")
+
+
+def test_prefill_rejects_unsupported_shapes_before_launch():
+    c = W.build_prefill_case("pf-f32", W.F32, Hq=4, Hkv=4, D=128, block_size=16,
+                             prior_lens=[3], new_lens=[2], seed=1)
+    t = W.prefill_to_torch(c, "cuda")
+    out = torch.empty((c.T, c.Hq, c.D), dtype=torch.float32, device="cuda")
+    with pytest.raises(ops.PAError) as e:
+        ops.pa_prefill(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                       t["context_lens"], t["query_start"], c.max_query_len, c.scale,
+                       c.max_context_len)
+    assert e.value.status == 4
