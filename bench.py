@@ -256,7 +256,7 @@ def reference_arm(args, w: W.Workload, rank: int, world: int):
 # ----------------------------------------------------------------------------
 KERNEL_SOURCES = {
     "cuda-core": ["decode_simt.cu"],
-    "tcgen05": ["decode_tc.cu", "decode_simt.cu"],      # the merge kernel lives in decode_simt.cu
+    "tcgen05": ["decode_tc.cu", "tc_ptx.cuh", "decode_simt.cu"],  # merge kernel: decode_simt.cu
 }
 
 
