@@ -91,3 +91,58 @@ def test_null_alignment_and_workspace_checks():
     assert L.pa_copy_blocks(16, 16, 2, 16, 0, 8, 128, 16, 4, None, None) == 0
     assert L.pa_copy_blocks(16, 16, 2, 16, -1, 8, 128, 16, 4, None, None) == 2
     assert L.pa_copy_blocks(16, 16, 7, 16, 1, 8, 128, 16, 4, None, None) == 3
+
+
+def test_fp8_swap_prefill_and_shared_prefix_host_checks():
+    L = ops.LIB
+    # FP8 decode: bad query type, bad scale, NULL pool, B == 0 no-op
+    assert L.pa_decode_fp8(16, 0, 16, 7, 16, 16, 1.0, 1.0, 16, 1, 16, 2, 8, 2, 128, 16, 4, 0.1,
+                           16, 0, None, 0, None, None) == 3
+    assert L.pa_decode_fp8(16, 0, 16, 1, 16, 16, 0.0, 1.0, 16, 1, 16, 2, 8, 2, 128, 16, 4, 0.1,
+                           16, 0, None, 0, None, None) == 2
+    assert L.pa_decode_fp8(16, 0, 16, 1, None, 16, 1.0, 1.0, 16, 1, 16, 2, 8, 2, 128, 16, 4, 0.1,
+                           16, 0, None, 0, None, None) == 1
+    assert L.pa_decode_fp8(None, 0, None, 1, None, None, 1.0, 1.0, None, 1, None, 0, 8, 2, 128,
+                           16, 4, 0.1, 0, 0, None, 0, None, None) == 0
+    # FP8 scatter: NaN scale, unsupported head size, misaligned source
+    assert L.pa_reshape_and_cache_fp8(16, 16, 1, 16, 16, float("nan"), 1.0, 16, 2, 8, 128, 16, 4,
+                                      None, None) == 2
+    assert L.pa_reshape_and_cache_fp8(16, 16, 1, 16, 16, 1.0, 1.0, 16, 2, 8, 96, 16, 4,
+                                      None, None) == 4
+    assert L.pa_reshape_and_cache_fp8(24, 16, 1, 16, 16, 1.0, 1.0, 16, 2, 8, 128, 16, 4,
+                                      None, None) == 7
+    # swap: FP8 pools are allowed; an unknown type and negative pairs are not
+    assert L.pa_swap_blocks(16, 16, 16, 16, 3, 16, 0, 8, 128, 16, 4, 4, None, None) == 0
+    assert L.pa_swap_blocks(16, 16, 16, 16, 4, 16, 1, 8, 128, 16, 4, 4, None, None) == 3
+    assert L.pa_swap_blocks(16, 16, 16, 16, 2, 16, -1, 8, 128, 16, 4, 4, None, None) == 2
+    assert L.pa_swap_blocks(16, 16, None, 16, 2, 16, 1, 8, 128, 16, 4, 4, None, None) == 1
+    # prefill: f32 and D = 64 are not on the tensor-core kernel; NULL start offsets
+    assert L.pa_prefill(16, 0, 16, 16, 16, 0, 16, 1, 16, 16, 1, 4, 4, 8, 2, 128, 16, 4, 0.1, 16,
+                        None, None) == 4
+    assert L.pa_prefill(16, 0, 16, 16, 16, 2, 16, 1, 16, 16, 1, 4, 4, 8, 2, 64, 16, 4, 0.1, 16,
+                        None, None) == 4
+    assert L.pa_prefill(16, 0, 16, 16, 16, 2, 16, 1, 16, None, 1, 4, 4, 8, 2, 128, 16, 4, 0.1,
+                        16, None, None) == 1
+    assert L.pa_prefill(None, 0, None, None, None, 2, None, 1, None, None, 0, 0, 0, 8, 2, 128, 16,
+                        4, 0.1, 16, None, None) == 0
+    # shared prefix: more shared blocks than a table holds; NULL group arrays; no workspace
+    assert L.pa_decode_shared_prefix(16, 0, 16, 16, 16, 2, 16, 4, 16, 16, 1, 16, 16, 2, 5, 2, 8,
+                                     2, 128, 16, 4, 0.1, 64, 0, None, 0, None, None) == 2
+    assert L.pa_decode_shared_prefix(16, 0, 16, 16, 16, 2, 16, 4, 16, 16, 1, None, 16, 2, 2, 2, 8,
+                                     2, 128, 16, 4, 0.1, 64, 0, None, 0, None, None) == 1
+    assert L.pa_decode_shared_prefix(16, 0, 16, 16, 16, 2, 16, 4, 16, 16, 1, 16, 16, 2, 2, 2, 8,
+                                     2, 128, 16, 4, 0.1, 64, 0, None, 0, None, None) == 5
+
+
+def test_shared_prefix_workspace_and_fp8_plan():
+    # slots: one per 128-token tile of the largest shared prefix + the suffix partitions
+    up = lambda x: (x + 255) // 256 * 256
+    B, Hq, D = 256, 32, 128
+    n = ops.pa_shared_prefix_workspace_size(B, Hq, 8, D, 1547, 0, 16, 64)
+    P = 1024 // 128 + 4
+    rows = B * Hq * P
+    assert n == up(rows * D * 4) + 2 * up(rows * 4)
+    assert ops.pa_shared_prefix_workspace_size(B, Hq, 8, D, 1547, 0, 16, 0) == \
+        ops.pa_workspace_size(B, Hq, 8, D, 1547, 0)
+    # FP8 pools always plan the CUDA-core kernel
+    assert ops.pa_decode_plan(ops.PA_FP8_E4M3, 8, 64, 8, 128, 16, 4096)[0] == 1
