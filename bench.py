@@ -685,14 +685,44 @@ def prefill_arm(args, rank: int, world: int, local_rank: int):
     }
 
 
+def prefill_reference_arm(args):
+    """The oracle on the host cores for the prefill workload: a bounded sample of
+    each step (64 new tokens of one sequence), scaled to TFLOP/s of the sample."""
+    import oracle
+    c = prefill_case(0)
+    sub = W.build_prefill_case("sample", W.BF16, Hq=64, Hkv=8, D=128, block_size=16,
+                               prior_lens=[int(c.context_lens[0]) - 512], new_lens=[64], seed=1)
+    steps = max(1, min(args.steps, 5))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.prefill(sub.q, sub.k_cache, sub.v_cache, W.BF16, sub.block_tables,
+                       sub.context_lens, sub.query_start, sub.scale)
+    secs = time.perf_counter() - t0
+    value = sub.attention_flops() * steps / secs / 1e12
+    sample = f"64 new tokens of one sequence per step, {steps} step(s), {secs:.1f} s"
+    return {"impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6),
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": steps, "warmup": 0,
+            "ms_per_step": round(1e3 * secs / steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": c.name, "sample": sample},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                             "cores": oracle.max_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
 def main():
     args = parse()
     if args.prefill:
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
-        if args.impl == "reference" or world > 1:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(prefill_reference_arm(args)), flush=True)
+            return 0
+        if world > 1:
             return 0 if rank else (print(json.dumps({"impl": args.impl, "unavailable":
-                "prefill measurement runs on one GPU with --impl ours"})) or 0)
+                "prefill measurement runs on one GPU"})) or 0)
         print(json.dumps(prefill_arm(args, rank, world, int(os.environ.get("LOCAL_RANK", "0")))),
               flush=True)
         return 0
