@@ -31,9 +31,11 @@
 // q % G) at position pos0 + q / G attends keys [0, pos0 + q / G]; the unit
 // covers all of them and writes the normalised output rows directly.
 //
-// CTA = 6 warps, persistent over units u = blockIdx.x + k * gridDim.x:
-// warps 0-3 softmax and epilogue (TMEM lanes 0-127), warp 4 TMA producer,
-// warp 5 MMA issuer (it also owns the tensor memory). Every wait is bounded;
+// CTA = 10 warps, persistent over units u = blockIdx.x + k * gridDim.x:
+// warps 0-7 softmax and epilogue (warp w: TMEM lanes 32 (w % 4) .. + 31, query
+// columns 32 (w / 4) .. + 31, so each row's columns are split between two
+// warps and every scheduler runs two softmax warps), warp 8 TMA producer,
+// warp 9 MMA issuer (it also owns the tensor memory). Every wait is bounded;
 // one that gives up sets PA_DEV_TIMEOUT and the CTA drains and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -54,7 +56,9 @@ constexpr int kStage = 2 * kHalf;               // one K or V tile: 32 KB
 constexpr int kNST = 4;                         // ring stages
 constexpr int kNQ = 64;                         // query rows per unit (max)
 constexpr int kTile = 128;                      // tokens per tile
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                   // 8 softmax warps, producer, MMA issuer
+constexpr int kSoft = 256;                      // softmax threads: 2 per row, 32 columns each
+constexpr int kHalfCols = kNQ / 2;
 constexpr float kRescaleLog2 = 64.f;
 
 constexpr int OFF_Q = kNST * kStage;            // Q: 2 d-halves x kNQ rows x 128 B
@@ -154,9 +158,18 @@ __device__ __forceinline__ PUnit mq_unit(const PrefixArgs& a, int G, int mc, lon
   return PF ? prefill_unit(a, G, mc, u) : prefix_unit(a, G, mc, u);
 }
 
-// Named barrier of the 128 softmax threads; vote = OR of every thread's flag.
-__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-__device__ __forceinline__ bool sm_vote(bool x) { return wg_vote_or(x, 0); }
+// Named barrier of the 256 softmax threads; vote = OR of every thread's flag.
+__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool sm_vote(bool x) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, 1, 256, pi;"
+      " selp.u32 %0, 1, 0, po; }"
+      : "=r"(r)
+      : "r"((uint32_t)x)
+      : "memory");
+  return r != 0;
+}
 
 template <int FMT, int BS, bool PF>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -182,20 +195,20 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
       mbar_init(bar(B_FULL + s), 1);
       mbar_init(bar(B_EMPTY + s), 1);
     }
-    mbar_init(bar(B_QFULL), 128);
+    mbar_init(bar(B_QFULL), kSoft);
     mbar_init(bar(B_QEMPTY), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_SFREE + i), 128);
-      mbar_init(bar(B_PREADY + i), 128);
+      mbar_init(bar(B_SFREE + i), kSoft);
+      mbar_init(bar(B_PREADY + i), kSoft);
       mbar_init(bar(B_OFULL + i), 1);
     }
-    mbar_init(bar(B_ODONE), 128);
+    mbar_init(bar(B_ODONE), kSoft);
     mbar_init(bar(B_DONE), 1);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kTmemCols)
@@ -214,7 +227,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
   };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int tc_ = 0, issued = 0;
@@ -270,7 +283,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         while (!mbar_try(bar(B_FULL + s), (seq / kNST) & 1) && globaltimer() - t0 < kWaitNs) {}
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int tc_ = 0, ua = 0;
@@ -334,8 +347,10 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int r = threadIdx.x;                   // token row of S^T; d row of O^T
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int r = threadIdx.x & 127;             // token row of S^T; d row of O^T
+    const int c0 = (warp >> 2) * kHalfCols;      // first query column of this thread
+    const int st = threadIdx.x;                  // 0 .. 255
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float* mref = reinterpret_cast<float*>(smem + OFF_MREF);
     float* mold = mref + kNQ;
     float* mnew = mold + kNQ;
@@ -346,22 +361,22 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     auto wait_pv = [&](int t) {                  // output product of tile t has completed
       if (!mbar_wait(bar(B_OFULL + (t & 1)), (t >> 1) & 1, abort_flag)) failed = true;
     };
-    // exact column maxima of s[] over the 128 rows -> dst[q]
+    // exact column maxima of s[] (this thread's columns c0 + i) over the 128 rows -> dst[q]
     auto col_max = [&](const float* s, float* dst) {
 #pragma unroll
-      for (int q = 0; q < kNQ; ++q) {
-        float v = s[q];
+      for (int i = 0; i < kHalfCols; ++i) {
+        float v = s[i];
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0) red[warp * kNQ + q] = v;
+        if (lane == 0) red[(warp & 3) * kNQ + c0 + i] = v;
       }
       sm_sync();
-      if (r < kNQ) dst[r] = fmaxf(fmaxf(red[r], red[kNQ + r]), fmaxf(red[2 * kNQ + r], red[3 * kNQ + r]));
+      if (st < kNQ) dst[st] = fmaxf(fmaxf(red[st], red[kNQ + st]), fmaxf(red[2 * kNQ + st], red[3 * kNQ + st]));
       sm_sync();
     };
     for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
       const PUnit x = mq_unit<PF>(a, G, mc, u);
-      if (PF && x.bad && x.h == 0 && r == 0 && (u / a.Hkv) % a.chunks == 0)
+      if (PF && x.bad && x.h == 0 && st == 0 && (u / a.Hkv) % a.chunks == 0)
         flag_error(a.err_flag, PA_DEV_BAD_CTX);
       if (x.nm <= 0) continue;
       // the (query token, head) row q of the unit in the query matrix
@@ -376,16 +391,17 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
       };
       if (!PF && x.ntiles == 0) {
         // this partition of the prefix holds no tokens: an empty partial
-        for (int q = 0; q < x.nq; ++q) a.ws_acc[slot_row(q) * kD + r] = 0.f;
-        if (r < x.nq) {
-          a.ws_m[slot_row(r)] = -CUDART_INF_F;
-          a.ws_l[slot_row(r)] = 0.f;
+        for (int i = 0; i < kHalfCols; ++i)
+          if (c0 + i < x.nq) a.ws_acc[slot_row(c0 + i) * kD + r] = 0.f;
+        if (st < x.nq) {
+          a.ws_m[slot_row(st)] = -CUDART_INF_F;
+          a.ws_l[slot_row(st)] = 0.f;
         }
         continue;
       }
       // Q rows of the unit into the K-major 128-byte-swizzled operand
       if (ua > 0 && !mbar_wait(bar(B_QEMPTY), (ua - 1) & 1, abort_flag)) failed = true;
-      for (int c = r; c < x.nqp * 16; c += 128) {
+      for (int c = st; c < x.nqp * 16; c += kSoft) {
         const int q = c >> 4, k16 = c & 15, hh = k16 >> 3, kk = k16 & 7;
         uint4 v = make_uint4(0, 0, 0, 0);
         if (q < x.nq)
@@ -393,14 +409,14 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
                                               k16 * 16);
         *reinterpret_cast<uint4*>(smem + OFF_Q + hh * (kNQ * 128) + q * 128 + ((kk ^ (q & 7)) << 4)) = v;
       }
-      if (PF && r < kNQ) lim[r] = x.pos0 + r / G;   // causal: the last key of column r
+      if (PF && st < kNQ) lim[st] = x.pos0 + st / G;   // causal: the last key of column st
       fence_proxy_async();
       mbar_arrive(bar(B_QFULL));
       if (PF) sm_sync();
 
-      float l[kNQ];
+      float l[kHalfCols];                        // partial exp-sums of columns c0 + i
 #pragma unroll
-      for (int q = 0; q < kNQ; ++q) l[q] = 0.f;
+      for (int i = 0; i < kHalfCols; ++i) l[i] = 0.f;
       const int32_t* table = a.block_tables + (size_t)x.b0 * a.max_blocks;
       for (int k = 0; k < x.ntiles; ++k, ++tc_) {
         const int ts = x.t0 + k * kTile;
@@ -412,50 +428,53 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         }
         if (!mbar_wait(bar(B_SFULL + (tc_ & 1)), (tc_ >> 1) & 1, abort_flag)) failed = true;
         tc_fence_after();
-        float s[kNQ];
+        float s[kHalfCols];
 #pragma unroll
-        for (int c = 0; c < kNQ; c += 16) tmem_ld16(tmem_s + lane_off + (tc_ & 1) * kNQ + c, s + c);
+        for (int c = 0; c < kHalfCols; c += 16)
+          tmem_ld16(tmem_s + lane_off + (tc_ & 1) * kNQ + c0 + c, s + c);
         tc_fence_before();
         mbar_arrive(bar(B_SFREE + (tc_ & 1)));
 #pragma unroll
-        for (int q = 0; q < kNQ; ++q)
-          s[q] = (valid && q < x.nq && (!PF || tok <= lim[q])) ? s[q] * a.scale_log2 : -CUDART_INF_F;
+        for (int i = 0; i < kHalfCols; ++i) {
+          const int q = c0 + i;
+          s[i] = (valid && q < x.nq && (!PF || tok <= lim[q])) ? s[i] * a.scale_log2 : -CUDART_INF_F;
+        }
         if (sm_vote(failed)) { stop = true; break; }
         if (k == 0) {
           col_max(s, mref);
         } else {
           bool exceed = false;
 #pragma unroll
-          for (int q = 0; q < kNQ; ++q) exceed |= s[q] > mref[q] + kRescaleLog2;
+          for (int i = 0; i < kHalfCols; ++i) exceed |= s[i] > mref[c0 + i] + kRescaleLog2;
           if (sm_vote(exceed)) {
             // rare: move the references of the columns that passed them, and
             // rescale those columns of O (all earlier products included) and l
             col_max(s, mnew);
-            if (r < kNQ) {
-              mold[r] = mref[r];
-              mnew[r] = mnew[r] > mref[r] + kRescaleLog2 ? mnew[r] : mref[r];
+            if (st < kNQ) {
+              mold[st] = mref[st];
+              mnew[st] = mnew[st] > mref[st] + kRescaleLog2 ? mnew[st] : mref[st];
             }
             sm_sync();
             wait_pv(tc_ - 1);
             tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < kNQ; c += 16) {
+            for (int c = 0; c < kHalfCols; c += 16) {
               float o[16];
-              tmem_ld16(tmem_o + lane_off + c, o);
+              tmem_ld16(tmem_o + lane_off + c0 + c, o);
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
-                const int q = c + e;
+                const int q = c0 + c + e;
                 if (mnew[q] != mold[q] && mold[q] != -CUDART_INF_F) {
                   const float f = exp2f(mold[q] - mnew[q]);
                   o[e] *= f;
-                  l[q] *= f;
+                  l[c + e] *= f;
                 }
               }
-              tmem_st16(tmem_o + lane_off + c, o);
+              tmem_st16(tmem_o + lane_off + c0 + c, o);
             }
             tc_fence_before();
             sm_sync();
-            if (r < kNQ) mref[r] = mnew[r];
+            if (st < kNQ) mref[st] = mnew[st];
             sm_sync();
           }
         }
@@ -464,17 +483,18 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         uint8_t* pb = smem + OFF_P + (tc_ & 1) * kPBuf + (r >> 6) * (kNQ * 128);
         const int pc = (r & 63) >> 3, pbyte = (r & 7) * 2;
 #pragma unroll
-        for (int q = 0; q < kNQ; ++q) {
+        for (int i = 0; i < kHalfCols; ++i) {
+          const int q = c0 + i;
           const float m = mref[q];
-          const float p = (s[q] != -CUDART_INF_F && m != -CUDART_INF_F) ? exp2f(s[q] - m) : 0.f;
-          l[q] += p;
+          const float p = (s[i] != -CUDART_INF_F && m != -CUDART_INF_F) ? exp2f(s[i] - m) : 0.f;
+          l[i] += p;
           uint16_t hi, lo;
           split_16<FMT>(p, hi, lo);
           const int off = q * 128 + ((pc ^ (q & 7)) << 4) + pbyte;
           *reinterpret_cast<uint16_t*>(pb + off) = hi;
           *reinterpret_cast<uint16_t*>(pb + kPPart + off) = lo;
         }
-        if (!valid) {
+        if (!valid && c0 == 0) {
           // a row with weight 0 still enters the product: it must hold finite values
           const int seq = 2 * tc_ + 1, sv = seq % kNST;
           if (!mbar_wait(bar(B_FULL + sv), (seq / kNST) & 1, abort_flag)) failed = true;
@@ -492,35 +512,36 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
       wait_pv(tc_ - 1);
       if (sm_vote(failed)) break;
 #pragma unroll
-      for (int q = 0; q < kNQ; ++q) {
-        float v = l[q];
+      for (int i = 0; i < kHalfCols; ++i) {
+        float v = l[i];
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[warp * kNQ + q] = v;
+        if (lane == 0) red[(warp & 3) * kNQ + c0 + i] = v;
       }
       sm_sync();
       if (PF) {
         // prefill: each column's exp-sum, then normalised rows straight to the output
-        if (r < kNQ) mold[r] = red[r] + red[kNQ + r] + red[2 * kNQ + r] + red[3 * kNQ + r];
+        if (st < kNQ) mold[st] = red[st] + red[kNQ + st] + red[2 * kNQ + st] + red[3 * kNQ + st];
         sm_sync();
-      } else if (r < x.nq) {
-        const size_t sr = slot_row(r);
-        a.ws_m[sr] = mref[r];
-        a.ws_l[sr] = red[r] + red[kNQ + r] + red[2 * kNQ + r] + red[3 * kNQ + r];
+      } else if (st < x.nq) {
+        const size_t sr = slot_row(st);
+        a.ws_m[sr] = mref[st];
+        a.ws_l[sr] = red[st] + red[kNQ + st] + red[2 * kNQ + st] + red[3 * kNQ + st];
       }
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kNQ; c += 16) {
+      for (int c = 0; c < kHalfCols; c += 16) {
         float o[16];
-        tmem_ld16(tmem_o + lane_off + c, o);
+        tmem_ld16(tmem_o + lane_off + c0 + c, o);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          if (c + e >= x.nq) continue;
+          const int q = c0 + c + e;
+          if (q >= x.nq) continue;
           if (PF) {
-            const float L = mold[c + e];
-            store_out(a.out, q_row(c + e) * kD + r, L > 0.f ? o[e] / L : 0.f, a.out_dtype);
+            const float L = mold[q];
+            store_out(a.out, q_row(q) * kD + r, L > 0.f ? o[e] / L : 0.f, a.out_dtype);
           } else {
-            a.ws_acc[slot_row(c + e) * kD + r] = o[e];
+            a.ws_acc[slot_row(q) * kD + r] = o[e];
           }
         }
       }
@@ -534,7 +555,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
