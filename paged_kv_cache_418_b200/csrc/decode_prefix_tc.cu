@@ -31,11 +31,11 @@
 // q % G) at position pos0 + q / G attends keys [0, pos0 + q / G]; the unit
 // covers all of them and writes the normalised output rows directly.
 //
-// CTA = 10 warps, persistent over units u = blockIdx.x + k * gridDim.x:
-// warps 0-7 softmax and epilogue (warp w: TMEM lanes 32 (w % 4) .. + 31, query
-// columns 32 (w / 4) .. + 31, so each row's columns are split between two
-// warps and every scheduler runs two softmax warps), warp 8 TMA producer,
-// warp 9 MMA issuer (it also owns the tensor memory). Every wait is bounded;
+// CTA = 18 warps, persistent over units u = blockIdx.x + k * gridDim.x:
+// warps 0-15 softmax and epilogue (warp w: TMEM lanes 32 (w % 4) .. + 31, query
+// columns 16 (w / 4) .. + 15, so each row's columns are split among four
+// warps and every scheduler runs four softmax warps), warp 16 TMA producer,
+// warp 17 MMA issuer (it also owns the tensor memory). Every wait is bounded;
 // one that gives up sets PA_DEV_TIMEOUT and the CTA drains and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -56,9 +56,11 @@ constexpr int kStage = 2 * kHalf;               // one K or V tile: 32 KB
 constexpr int kNST = 4;                         // ring stages
 constexpr int kNQ = 64;                         // query rows per unit (max)
 constexpr int kTile = 128;                      // tokens per tile
-constexpr int kThreads = 320;                   // 8 softmax warps, producer, MMA issuer
-constexpr int kSoft = 256;                      // softmax threads: 2 per row, 32 columns each
-constexpr int kHalfCols = kNQ / 2;
+constexpr int kSplit = 4;                       // softmax threads per row of S^T
+constexpr int kSoft = 128 * kSplit;             // softmax threads
+constexpr int kHalfCols = kNQ / kSplit;         // query columns per softmax thread
+constexpr int kSoftWarps = kSoft / 32;
+constexpr int kThreads = kSoft + 64;            // + TMA producer warp + MMA warp
 constexpr float kRescaleLog2 = 64.f;
 
 constexpr int OFF_Q = kNST * kStage;            // Q: 2 d-halves x kNQ rows x 128 B
@@ -158,15 +160,15 @@ __device__ __forceinline__ PUnit mq_unit(const PrefixArgs& a, int G, int mc, lon
   return PF ? prefill_unit(a, G, mc, u) : prefix_unit(a, G, mc, u);
 }
 
-// Named barrier of the 256 softmax threads; vote = OR of every thread's flag.
-__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Named barrier of the kSoft softmax threads; vote = OR of every thread's flag.
+__device__ __forceinline__ void sm_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSoft) : "memory"); }
 __device__ __forceinline__ bool sm_vote(bool x) {
   uint32_t r;
   asm volatile(
-      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, 1, 256, pi;"
+      "{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, 1, %2, pi;"
       " selp.u32 %0, 1, 0, po; }"
       : "=r"(r)
-      : "r"((uint32_t)x)
+      : "r"((uint32_t)x), "n"(kSoft)
       : "memory");
   return r != 0;
 }
@@ -208,7 +210,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 9) {
+  if (warp == kSoftWarps + 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kTmemCols)
@@ -227,7 +229,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
   };
 
-  if (warp == 8) {
+  if (warp == kSoftWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int tc_ = 0, issued = 0;
@@ -283,7 +285,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         while (!mbar_try(bar(B_FULL + s), (seq / kNST) & 1) && globaltimer() - t0 < kWaitNs) {}
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kSoftWarps + 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int tc_ = 0, ua = 0;
@@ -349,7 +351,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     // ------------------------------------------------------------ softmax + epilogue
     const int r = threadIdx.x & 127;             // token row of S^T; d row of O^T
     const int c0 = (warp >> 2) * kHalfCols;      // first query column of this thread
-    const int st = threadIdx.x;                  // 0 .. 255
+    const int st = threadIdx.x;                  // 0 .. kSoft - 1
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     float* mref = reinterpret_cast<float*>(smem + OFF_MREF);
     float* mold = mref + kNQ;
@@ -555,7 +557,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kSoftWarps + 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
