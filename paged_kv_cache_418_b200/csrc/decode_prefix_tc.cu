@@ -70,8 +70,7 @@ constexpr int kPPart = 2 * kNQ * 128;
 constexpr int kPBuf = 2 * kPPart;
 constexpr int OFF_MREF = OFF_P + 2 * kPBuf;     // [3][kNQ] reference, old, new maxima
 constexpr int OFF_RED = OFF_MREF + 3 * kNQ * 4; // [4 warps][kNQ]
-constexpr int OFF_LIM = OFF_RED + 4 * kNQ * 4;  // [kNQ] prefill causal limits
-constexpr int OFF_BAR = OFF_LIM + kNQ * 4;
+constexpr int OFF_BAR = OFF_RED + 4 * kNQ * 4;
 enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY, B_SFULL, B_SFREE = B_SFULL + 2,
        B_PREADY = B_SFREE + 2, B_OFULL = B_PREADY + 2, B_ODONE = B_OFULL + 2, B_DONE, B_COUNT };
 constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
@@ -158,6 +157,15 @@ __device__ __forceinline__ PUnit prefix_unit(const PrefixArgs& a, int G, int mc,
 template <bool PF>
 __device__ __forceinline__ PUnit mq_unit(const PrefixArgs& a, int G, int mc, long long u) {
   return PF ? prefill_unit(a, G, mc, u) : prefix_unit(a, G, mc, u);
+}
+
+// 2^x by the multi-function unit's approximation (relative error ~2^-22, flushes
+// subnormal results to 0; -inf gives +0): the weights then go through the hi/lo
+// 16-bit split, which keeps far less than that.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Named barrier of the kSoft softmax threads; vote = OR of every thread's flag.
@@ -357,7 +365,6 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     float* mold = mref + kNQ;
     float* mnew = mold + kNQ;
     float* red = reinterpret_cast<float*>(smem + OFF_RED);
-    int* lim = reinterpret_cast<int*>(smem + OFF_LIM);   // prefill: last key of each column
     bool failed = false, stop = false;
     int tc_ = 0, ua = 0;
     auto wait_pv = [&](int t) {                  // output product of tile t has completed
@@ -411,10 +418,8 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
                                               k16 * 16);
         *reinterpret_cast<uint4*>(smem + OFF_Q + hh * (kNQ * 128) + q * 128 + ((kk ^ (q & 7)) << 4)) = v;
       }
-      if (PF && st < kNQ) lim[st] = x.pos0 + st / G;   // causal: the last key of column st
       fence_proxy_async();
       mbar_arrive(bar(B_QFULL));
-      if (PF) sm_sync();
 
       float l[kHalfCols];                        // partial exp-sums of columns c0 + i
 #pragma unroll
@@ -424,6 +429,8 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         const int ts = x.t0 + k * kTile;
         const int tok = ts + r;
         bool valid = tok < x.t1;
+        // prefill: column q (position pos0 + q / G) sees this key iff q >= qmin
+        const int qmin = PF ? max(0, (tok - x.pos0) * G) : 0;
         if (valid) {
           const int32_t p = __ldg(table + tok / BS);
           valid = p >= 0 && p < a.num_blocks;
@@ -439,7 +446,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
 #pragma unroll
         for (int i = 0; i < kHalfCols; ++i) {
           const int q = c0 + i;
-          s[i] = (valid && q < x.nq && (!PF || tok <= lim[q])) ? s[i] * a.scale_log2 : -CUDART_INF_F;
+          s[i] = (valid && q < x.nq && q >= qmin) ? s[i] * a.scale_log2 : -CUDART_INF_F;
         }
         if (sm_vote(failed)) { stop = true; break; }
         if (k == 0) {
@@ -488,7 +495,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         for (int i = 0; i < kHalfCols; ++i) {
           const int q = c0 + i;
           const float m = mref[q];
-          const float p = (s[i] != -CUDART_INF_F && m != -CUDART_INF_F) ? exp2f(s[i] - m) : 0.f;
+          const float p = (s[i] != -CUDART_INF_F && m != -CUDART_INF_F) ? fast_exp2(s[i] - m) : 0.f;
           l[i] += p;
           uint16_t hi, lo;
           split_16<FMT>(p, hi, lo);
