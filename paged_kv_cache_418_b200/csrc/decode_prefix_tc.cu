@@ -41,6 +41,8 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <cfloat>
+
 #include "pa_internal.h"
 #include "tc_ptx.cuh"
 
@@ -370,7 +372,9 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     auto wait_pv = [&](int t) {                  // output product of tile t has completed
       if (!mbar_wait(bar(B_OFULL + (t & 1)), (t >> 1) & 1, abort_flag)) failed = true;
     };
-    // exact column maxima of s[] (this thread's columns c0 + i) over the 128 rows -> dst[q]
+    // column maxima of s[] (this thread's columns c0 + i) over the 128 rows -> dst[q],
+    // floored at -FLT_MAX: a column with no visible key keeps a finite reference, so
+    // score - reference is -inf exactly where the score is masked
     auto col_max = [&](const float* s, float* dst) {
 #pragma unroll
       for (int i = 0; i < kHalfCols; ++i) {
@@ -380,7 +384,9 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         if (lane == 0) red[(warp & 3) * kNQ + c0 + i] = v;
       }
       sm_sync();
-      if (st < kNQ) dst[st] = fmaxf(fmaxf(red[st], red[kNQ + st]), fmaxf(red[2 * kNQ + st], red[3 * kNQ + st]));
+      if (st < kNQ)
+        dst[st] = fmaxf(fmaxf(fmaxf(red[st], red[kNQ + st]), fmaxf(red[2 * kNQ + st], red[3 * kNQ + st])),
+                        -FLT_MAX);
       sm_sync();
     };
     for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
@@ -429,12 +435,16 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         const int ts = x.t0 + k * kTile;
         const int tok = ts + r;
         bool valid = tok < x.t1;
-        // prefill: column q (position pos0 + q / G) sees this key iff q >= qmin
-        const int qmin = PF ? max(0, (tok - x.pos0) * G) : 0;
         if (valid) {
           const int32_t p = __ldg(table + tok / BS);
           valid = p >= 0 && p < a.num_blocks;
         }
+        // bit i of mk: column c0 + i is a real query row that sees this key (prefill:
+        // column q, at position pos0 + q / G, sees key tok iff q >= (tok - pos0) * G)
+        const int qlo = PF ? min(max((tok - x.pos0) * G - c0, 0), kHalfCols) : 0;
+        const int qhi = valid ? min(max(x.nq - c0, 0), kHalfCols) : 0;
+        const uint32_t mk = qhi > qlo ? ((1u << qhi) - 1u) & ~((1u << qlo) - 1u) : 0u;
+        const bool full = __all_sync(0xffffffffu, mk == (1u << kHalfCols) - 1u);
         if (!mbar_wait(bar(B_SFULL + (tc_ & 1)), (tc_ >> 1) & 1, abort_flag)) failed = true;
         tc_fence_after();
         float s[kHalfCols];
@@ -443,26 +453,40 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
           tmem_ld16(tmem_s + lane_off + (tc_ & 1) * kNQ + c0 + c, s + c);
         tc_fence_before();
         mbar_arrive(bar(B_SFREE + (tc_ & 1)));
-#pragma unroll
-        for (int i = 0; i < kHalfCols; ++i) {
-          const int q = c0 + i;
-          s[i] = (valid && q < x.nq && q >= qmin) ? s[i] * a.scale_log2 : -CUDART_INF_F;
-        }
         if (sm_vote(failed)) { stop = true; break; }
+        // s[i] becomes the scaled score of column c0 + i minus the column's reference
+        // maximum (log2 units): -inf where the key is masked
         if (k == 0) {
-          col_max(s, mref);
-        } else {
-          bool exceed = false;
 #pragma unroll
-          for (int i = 0; i < kHalfCols; ++i) exceed |= s[i] > mref[c0 + i] + kRescaleLog2;
-          if (sm_vote(exceed)) {
-            // rare: move the references of the columns that passed them, and
-            // rescale those columns of O (all earlier products included) and l
+          for (int i = 0; i < kHalfCols; ++i)
+            s[i] = ((mk >> i) & 1u) ? s[i] * a.scale_log2 : -CUDART_INF_F;
+          col_max(s, mref);
+#pragma unroll
+          for (int i = 0; i < kHalfCols; ++i) s[i] -= mref[c0 + i];
+        } else {
+          const float4* m4 = reinterpret_cast<const float4*>(mref + c0);
+#pragma unroll
+          for (int j = 0; j < kHalfCols / 4; ++j) {
+            const float4 m = m4[j];
+            s[4 * j] = fmaf(s[4 * j], a.scale_log2, -m.x);
+            s[4 * j + 1] = fmaf(s[4 * j + 1], a.scale_log2, -m.y);
+            s[4 * j + 2] = fmaf(s[4 * j + 2], a.scale_log2, -m.z);
+            s[4 * j + 3] = fmaf(s[4 * j + 3], a.scale_log2, -m.w);
+          }
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < kHalfCols; ++i)
+              if (!((mk >> i) & 1u)) s[i] = -CUDART_INF_F;
+          }
+          float mx = s[0];
+#pragma unroll
+          for (int i = 1; i < kHalfCols; ++i) mx = fmaxf(mx, s[i]);
+          if (sm_vote(mx > kRescaleLog2)) {
+            // rare: some column passed its reference by more than 2^64. Its reference
+            // moves up by the tile's maximum d of that column (relative to it), and its
+            // O (all earlier products included) and l are scaled by 2^-d
             col_max(s, mnew);
-            if (st < kNQ) {
-              mold[st] = mref[st];
-              mnew[st] = mnew[st] > mref[st] + kRescaleLog2 ? mnew[st] : mref[st];
-            }
+            if (st < kNQ) mold[st] = mnew[st] > kRescaleLog2 ? mnew[st] : 0.f;
             sm_sync();
             wait_pv(tc_ - 1);
             tc_fence_after();
@@ -472,9 +496,9 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
               tmem_ld16(tmem_o + lane_off + c0 + c, o);
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
-                const int q = c0 + c + e;
-                if (mnew[q] != mold[q] && mold[q] != -CUDART_INF_F) {
-                  const float f = exp2f(mold[q] - mnew[q]);
+                const float d = mold[c0 + c + e];
+                if (d != 0.f) {
+                  const float f = exp2f(-d);
                   o[e] *= f;
                   l[c + e] *= f;
                 }
@@ -482,8 +506,10 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
               tmem_st16(tmem_o + lane_off + c0 + c, o);
             }
             tc_fence_before();
+#pragma unroll
+            for (int i = 0; i < kHalfCols; ++i) s[i] -= mold[c0 + i];
             sm_sync();
-            if (st < kNQ) mref[st] = mnew[st];
+            if (st < kNQ) mref[st] += mold[st];
             sm_sync();
           }
         }
@@ -494,8 +520,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
 #pragma unroll
         for (int i = 0; i < kHalfCols; ++i) {
           const int q = c0 + i;
-          const float m = mref[q];
-          const float p = (s[i] != -CUDART_INF_F && m != -CUDART_INF_F) ? fast_exp2(s[i] - m) : 0.f;
+          const float p = fast_exp2(s[i]);        // 0 where masked
           l[i] += p;
           uint16_t hi, lo;
           split_16<FMT>(p, hi, lo);
@@ -534,7 +559,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         sm_sync();
       } else if (st < x.nq) {
         const size_t sr = slot_row(st);
-        a.ws_m[sr] = mref[st];
+        a.ws_m[sr] = mref[st] == -FLT_MAX ? -CUDART_INF_F : mref[st];
         a.ws_l[sr] = red[st] + red[kNQ + st] + red[2 * kNQ + st] + red[3 * kNQ + st];
       }
       tc_fence_after();
