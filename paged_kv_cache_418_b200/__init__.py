@@ -3,7 +3,10 @@
 Decode-step attention of one query token per sequence over a KV cache kept in
 fixed-size physical blocks and reached through per-sequence block tables,
 plus ``reshape_and_cache`` (write each new token's K/V to its slot) and
-``copy_blocks`` (copy-on-write of a shared block).
+``copy_blocks`` (copy-on-write of a shared block). Beside the decode step:
+FP8 (E4M3) pools with per-pool scales, ``swap_blocks`` between device and
+host pools, a shared-prefix decode that streams a group's common blocks once
+for the whole group, and paged (chunked) prefill with a causal mask.
 
 Modules:
   ops            thin ctypes binding of the C-ABI library ``libpa.so``

@@ -21,7 +21,11 @@
 // column is set on the unit's first tile (an exact column max) and moves only
 // when a score passes it by 2^64 (then O's columns are rescaled in TMEM), so a
 // tile needs no reduction across threads; the column sums l are per-thread
-// partial sums reduced once per unit.
+// partial sums reduced once per unit. A score enters as one FMA against its
+// column's reference (s * scale - m, log2 units); a 16-bit mask per token row
+// says which of the thread's columns see the key (all of them on most tiles,
+// one warp-uniform test), and references are floored at -FLT_MAX so a masked
+// score stays -inf and its weight 2^-inf = 0 needs no guard.
 //
 // The same kernel runs paged prefill (PF = true): a chunk of a sequence's new
 // query tokens attends, causally, to the sequence's own blocks — the prompt
