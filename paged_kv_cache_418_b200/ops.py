@@ -1,9 +1,9 @@
 """ctypes binding of libpa.so (the C ABI declared in include/pa.h).
 
 Argument marshalling only: every function here checks nothing the library does
-not check itself, reads the sizes off torch tensor shapes, passes raw device
-pointers and the current CUDA stream, and turns a nonzero status into
-``PAError``. All of the computing happens in the CUDA kernels. There is no
+not check itself (except, in debug mode, the cache ops' caller preconditions),
+reads the sizes off torch tensor shapes, passes raw device pointers and the
+current CUDA stream, and turns a nonzero status into ``PAError``. All of the computing happens in the CUDA kernels. There is no
 fallback: if the library cannot be built or loaded, importing this module
 raises.
 """
@@ -11,6 +11,7 @@ raises.
 from __future__ import annotations
 
 import ctypes
+import os
 from typing import Optional, Tuple
 
 import torch
@@ -68,6 +69,39 @@ def _load() -> ctypes.CDLL:
 
 LIB = _load()
 LIB_PATH = _build.LIB
+
+
+# Debug mode (PA_DEBUG=1 in the environment, or set_debug(True)): before each
+# cache op the binding reads the mapping back to the host and rejects the
+# inputs the library leaves to the caller (two tokens on one slot; a copy
+# destination named twice or also used as a source). It costs a device-to-host
+# copy and a sync per call, so it is off by default.
+DEBUG = os.environ.get("PA_DEBUG", "0") not in ("", "0")
+
+
+def set_debug(on: bool) -> None:
+    global DEBUG
+    DEBUG = bool(on)
+
+
+def check_slot_mapping(slot_mapping: torch.Tensor, fn: str = "pa_reshape_and_cache") -> None:
+    """ValueError if two tokens name the same (non-negative) slot."""
+    s = slot_mapping.detach().to("cpu", torch.int64).reshape(-1)
+    s = s[s >= 0]
+    if torch.unique(s).numel() != s.numel():
+        raise ValueError(f"{fn}: two tokens name the same slot in slot_mapping")
+
+
+def check_block_mapping(block_mapping: torch.Tensor, fn: str = "pa_copy_blocks",
+                        same_pool: bool = True) -> None:
+    """ValueError if a destination block is named twice or, within one pool, is
+    also a source of the same call."""
+    m = block_mapping.detach().to("cpu", torch.int64).reshape(-1, 2)
+    src, dst = m[:, 0], m[:, 1]
+    if torch.unique(dst).numel() != dst.numel():
+        raise ValueError(f"{fn}: a destination block is named twice")
+    if same_pool and bool(torch.isin(dst, src).any()):
+        raise ValueError(f"{fn}: a destination block is also a source")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -151,6 +185,8 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torc
                          value_cache: torch.Tensor, slot_mapping: torch.Tensor,
                          err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
     """Scatter new K/V rows [T,Hkv,D] into the pools at slot_mapping [T] (int64)."""
+    if DEBUG:
+        check_slot_mapping(slot_mapping)
     num_blocks, block_size, Hkv, D = key_cache.shape
     T = slot_mapping.shape[0]
     rc = LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache),
@@ -164,6 +200,8 @@ def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor,
                    block_mapping: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
                    stream=None) -> None:
     """Copy whole blocks src -> dst for each (src, dst) row of block_mapping [P,2] (int64)."""
+    if DEBUG:
+        check_block_mapping(block_mapping)
     num_blocks, block_size, Hkv, D = key_cache.shape
     P = block_mapping.shape[0]
     rc = LIB.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), pa_dtype(key_cache),
@@ -198,6 +236,8 @@ def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: 
                              slot_mapping: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
                              stream=None) -> None:
     """Quantise new K/V rows [T,Hkv,D] to E4M3 codes and scatter them into the pools."""
+    if DEBUG:
+        check_slot_mapping(slot_mapping, "pa_reshape_and_cache_fp8")
     num_blocks, block_size, Hkv, D = key_cache.shape
     T = slot_mapping.shape[0]
     rc = LIB.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), pa_dtype(key), _ptr(key_cache),
@@ -213,6 +253,8 @@ def pa_swap_blocks(dst_key: torch.Tensor, dst_value: torch.Tensor, src_key: torc
                    err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
     """Copy whole blocks src pool -> dst pool ((src id, dst id) rows of block_mapping);
     either pool may be pinned host memory."""
+    if DEBUG:
+        check_block_mapping(block_mapping, "pa_swap_blocks", same_pool=False)
     src_blocks, block_size, Hkv, D = src_key.shape
     dst_blocks = dst_key.shape[0]
     P = block_mapping.shape[0]
