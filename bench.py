@@ -229,14 +229,27 @@ def reference_arm(args, w: W.Workload, rank: int, world: int):
         return None
     import oracle
     cores = oracle.max_threads()
-    rows = oracle_sample_rows(w, budget_s=3.0)
+    steps = max(1, args.steps)
+    # each step a bounded sample: about 2 minutes of oracle time for the whole run
+    rows = oracle_sample_rows(w, budget_s=max(0.05, min(3.0, 120.0 / steps)))
     for _ in range(max(0, min(args.warmup, 1))):
         run_oracle(w, rows[:4])
-    secs, byts = run_oracle(w, rows, reps=args.steps)
+    secs, byts = run_oracle(w, rows, reps=steps)
     value = byts / secs / 1e9
     sample = (f"{len(rows)} of {w.B * w.Hq} (sequence, query head) rows per step "
               f"({100.0 * len(rows) / (w.B * w.Hq):.1f}%), plus the step's full "
               f"reshape_and_cache/copy_blocks; value scaled by the rows' share of KV bytes")
+    # the same oracle on one core: decode of a ~3 s sample of rows
+    rows1 = oracle_sample_rows(w, budget_s=3.0 / max(1, cores), rng_seed=1)
+    t = time.perf_counter()
+    oracle.decode_kv(w.q, w.dtype, w.k_cache, w.v_cache, w.kv_dtype, w.k_scale, w.v_scale,
+                     w.block_tables, w.context_lens, w.scale, rows=rows1, n_threads=1)
+    secs1 = time.perf_counter() - t
+    oracle.decode_kv(w.q, w.dtype, w.k_cache, w.v_cache, w.kv_dtype, w.k_scale, w.v_scale,
+                     w.block_tables, w.context_lens, w.scale, rows=rows1[:1], n_threads=cores)
+    frac1 = float(w.context_lens[rows1[:, 0]].sum()) / (w.Hq * float(w.context_lens.sum()))
+    one_core = {"value": round(w.kv_bytes() * frac1 / secs1 / 1e9, 4), "unit": "GB/s",
+                "sample": f"decode of {len(rows1)} rows on 1 thread, {secs1:.1f} s"}
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -244,7 +257,7 @@ def reference_arm(args, w: W.Workload, rank: int, world: int):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, 1, "host memory"),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
-                         "kind": "oracle", "sample": sample},
+                         "kind": "oracle", "sample": sample, "one_core": one_core},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

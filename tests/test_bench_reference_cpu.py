@@ -1,0 +1,40 @@
+"""The benchmark's reference arm (the oracle on the host cores) runs without a
+GPU and prints one JSON line of the contract: CPU only, on the tiny workload
+and on the prefill sample."""
+
+from __future__ import annotations
+
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _line(*args):
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        *args], capture_output=True, text=True, cwd=ROOT, timeout=600,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert r.returncode == 0, r.stderr
+    lines = [x for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    return json.loads(lines[0])
+
+
+def test_decode_reference_line():
+    d = _line("--workload", "1", "--steps", "3", "--warmup", "1")
+    assert d["impl"] == "reference" and d["metric"] == "paged decode attention KV GB/s"
+    assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["steps"] == 3
+    assert d["value"] > 0 and d["value"] == d["cpu_baseline"]["value"] == d["e2e"]["value"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["one_core"]["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "tiny-fp32"
+
+
+def test_prefill_reference_line():
+    d = _line("--prefill", "--steps", "1", "--warmup", "0")
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle"
