@@ -181,8 +181,8 @@ int pa_decode_static(void* out, int out_dtype, const void* query, const void* ke
 
 /*
  * FP8 KV cache. The pages give halving the bytes per cached token as the
- * reason to keep K and V in 8 bits ("vLLM与PagedAttention：大模型推理内存优化
- * 技术解析" section 6.2; "vLLM 与 LLM 推理部署实战" section 6.1) and fix no
+ * reason to keep K and V in 8 bits ("vLLM 与 LLM 推理部署实战" section 6.2;
+ * "vLLM与PagedAttention：大模型推理内存优化技术解析" section 6.1) and fix no
  * format. Here an FP8 pool holds OCP FP8 E4M3 codes, one byte per element
  * (sign, 4-bit exponent with bias 7, 3 fraction bits, no infinities, largest
  * finite value 448), with one float scale per pool: code c stands for
@@ -233,8 +233,8 @@ int pa_decode_fp8(void* out, int out_dtype, const void* query, int q_dtype, cons
 /*
  * pa_swap_blocks -- preemption by swapping: copy whole blocks (K and V)
  * between two pools, typically the device pool and a pool in page-locked host
- * memory ("vLLM与PagedAttention：大模型推理内存优化技术解析" section 三: under
- * memory pressure the block manager moves blocks out to CPU memory, and back).
+ * memory ("vLLM 与 LLM 推理部署实战" section 三: under memory pressure the
+ * block manager moves blocks out to CPU memory, and back).
  * dst_key, dst_value  [dst_blocks, block_size, Hkv, D] destination pools;
  * src_key, src_value  [src_blocks, block_size, Hkv, D] source pools;
  *               each pool is device memory or page-locked host memory that

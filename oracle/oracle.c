@@ -53,14 +53,14 @@
  *                     prompt's self-attention.
  *  oracle_swap_blocks The same whole-block copy between two different pools
  *                     (host and device memory): preemption by swapping moves
- *                     a sequence's blocks to CPU memory and back. "vLLM与
- *                     PagedAttention：大模型推理内存优化技术解析" section 三
- *                     (preemption: swapping blocks to CPU memory).
+ *                     a sequence's blocks to CPU memory and back. "vLLM 与
+ *                     LLM 推理部署实战" section 三 (preemption: the block
+ *                     manager swaps blocks out to CPU memory).
  *  FP8 KV cache       The pools may hold 8-bit codes instead of 16/32-bit
  *                     values: halving the bytes per token is the stated
- *                     point ("vLLM与PagedAttention：大模型推理内存优化技术解析"
- *                     section 6.2; "vLLM 与 LLM 推理部署实战" section 6.1,
- *                     which also names fp8 K with bf16 V). The pages fix no
+ *                     point ("vLLM 与 LLM 推理部署实战" section 6.2; "vLLM与
+ *                     PagedAttention：大模型推理内存优化技术解析" section 6.1
+ *                     names fp8 K with bf16 V). The pages fix no
  *                     format; the reading here is OCP FP8 E4M3 (bias 7, no
  *                     infinities, 448 the largest finite value) with one
  *                     float scale per pool: stored code = E4M3(x / scale),
