@@ -38,3 +38,18 @@ def test_prefill_reference_line():
     d = _line("--prefill", "--steps", "1", "--warmup", "0")
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_reference_line_under_torchrun_comes_from_rank_0_only():
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", "29581", os.path.join(ROOT, "bench.py"), "--impl",
+                        "reference", "--gpus", "2", "--workload", "1", "--steps", "2",
+                        "--warmup", "1"],
+                       capture_output=True, text=True, cwd=ROOT, timeout=600,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES="", OMP_NUM_THREADS="2"))
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.strip().startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0
