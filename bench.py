@@ -3,7 +3,8 @@
 step has copy-on-write pairs) + paged decode attention, on synthetic workloads.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|ID]
-                    [--impl ours|reference]
+                    [--impl ours|reference] [--batch B] [--e2e-steps E]
+                    [--shared-prefix | --prefill | --swap]
 
 One step = one pass of the whole hot path over one batch: the step's
 copy_blocks, then reshape_and_cache of the new tokens, then decode attention
@@ -22,6 +23,12 @@ there is) on a bounded sample of the same workload, on rank 0.
 --swap measures swap_blocks instead (preemption by swapping): whole blocks of
 the Llama-2-7B-shaped pool moved device -> page-locked host and back, against
 a plain cudaMemcpyAsync of the same bytes timed in the same run.
+
+--shared-prefix (with --workload 5) runs the step's decode with
+pa_decode_shared_prefix: each group's shared blocks are read once per group.
+
+--prefill measures paged chunked prefill in TFLOP/s: 8 sequences with
+U[0, 2048] cached tokens each take a 512-token chunk (Llama-3-70B-shaped, bf16).
 """
 
 from __future__ import annotations
