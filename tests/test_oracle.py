@@ -507,3 +507,26 @@ def test_prefill_first_token_of_an_empty_sequence_is_its_v_row():
         bad = c.context_lens.copy()
         bad[0] = 3                                   # fewer tokens than the chunk holds
         oracle.prefill(c.q, c.k_cache, c.v_cache, BF16, c.block_tables, bad, c.query_start, c.scale)
+
+
+def test_prefill_row_ignores_keys_after_its_position():
+    """Causality as an invariance: overwriting the K/V of every position after a
+    new token's own leaves that token's output bit-identical, and the output of
+    the chunk's last token (which sees everything) changes."""
+    from paged_kv_cache_418_b200.workloads import build_prefill_case
+    c = build_prefill_case("pf-causal", BF16, 8, 2, 32, 4, prior_lens=[6], new_lens=[9], seed=77)
+    out = oracle.prefill(c.q, c.k_cache, c.v_cache, BF16, c.block_tables, c.context_lens,
+                         c.query_start, c.scale)
+    ctx, n, bs = int(c.context_lens[0]), 9, 4
+    rng = RNG(5)
+    for i in range(n - 1):                       # new token i sits at position ctx - n + i
+        pos = ctx - n + i
+        kc, vc = c.k_cache.copy(), c.v_cache.copy()
+        for t in range(pos + 1, ctx):
+            blk = c.block_tables[0, t // bs]
+            kc[blk, t % bs] = _rand(rng, kc.shape[2:], BF16, 3.0)
+            vc[blk, t % bs] = _rand(rng, vc.shape[2:], BF16, 3.0)
+        out2 = oracle.prefill(c.q, kc, vc, BF16, c.block_tables, c.context_lens,
+                              c.query_start, c.scale)
+        assert np.array_equal(out2[:i + 1], out[:i + 1])
+        assert not np.allclose(out2[n - 1], out[n - 1])
