@@ -6,6 +6,7 @@ from __future__ import annotations
 
 import json
 import os
+import socket
 import subprocess
 import sys
 
@@ -40,10 +41,16 @@ def test_prefill_reference_line():
     assert d["cpu_baseline"]["kind"] == "oracle"
 
 
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def test_reference_line_under_torchrun_comes_from_rank_0_only():
     r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
                         "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
-                        "--master-port", "29581", os.path.join(ROOT, "bench.py"), "--impl",
+                        "--master-port", str(_free_port()), os.path.join(ROOT, "bench.py"), "--impl",
                         "reference", "--gpus", "2", "--workload", "1", "--steps", "2",
                         "--warmup", "1"],
                        capture_output=True, text=True, cwd=ROOT, timeout=600,
