@@ -93,3 +93,49 @@ def test_shrunk_shapes():
                 4: (64, 8, 128, 32, W.BF16)}[k]
         assert (w.Hq, w.Hkv, w.D, w.block_size, w.dtype) == full
         assert w.kv_bytes() == int(w.context_lens.sum()) * 2 * w.Hkv * w.D * 2
+
+
+def _cached_rows(w, pool):
+    """[tokens, Hkv, D] rows of every sequence's first ctx - 1 tokens (the cached part)."""
+    bs = w.block_size
+    out = []
+    for b in range(w.B):
+        n = int(w.context_lens[b]) - 1
+        for t in range(n):
+            out.append(pool[w.block_tables[b, t // bs], t % bs])
+    return np.stack(out)
+
+
+def test_length_recipes():
+    # bounds are about 5 standard errors of 48 draws wide
+    w2 = W.make_workload(2, batch=48)
+    assert w2.context_lens.min() >= 128 and w2.context_lens.max() <= 2048
+    assert 680 < float(w2.context_lens.mean()) < 1500               # U[128, 2048]: mean 1088
+    w3 = W.make_workload(3, batch=48)
+    assert w3.context_lens.min() >= 16 and w3.context_lens.max() <= 8192
+    assert 450 < float(np.median(w3.context_lens)) < 2200             # LogNormal(ln 1200, 0.8)
+
+
+def test_one_percent_of_k_rows_are_scaled_by_eight():
+    w = W.make_workload(4, batch=1)
+    assert list(w.context_lens) == [32768]
+    k = W.storage_to_float64(_cached_rows(w, w.k_cache), w.dtype)    # [tokens, Hkv, D]
+    norm = np.sqrt((k * k).sum(-1)).ravel()
+    big = norm > 4.0 * np.median(norm)                                # N(0,1)·8 rows stand out
+    n = norm.size
+    assert abs(int(big.sum()) - 0.01 * n) < 5 * np.sqrt(0.01 * n)     # binomial, 5 sigma
+    # a scaled row is exactly 8 times representable bf16 values (exact in bf16)
+    rows = k.reshape(-1, w.D)[big]
+    assert np.array_equal(W.storage_to_float64(W.round_to_storage(
+        (rows / 8).astype(np.float32), w.dtype), w.dtype) * 8, rows)
+
+
+def test_fp8_pool_codes_follow_the_recipe():
+    w = W.make_workload(6, batch=4)
+    assert w.fp8 and w.kv_dtype == W.FP8
+    for pool in (w.k_cache, w.v_cache):
+        codes = _cached_rows(w, pool).ravel()
+        e = (codes >> 3) & 15
+        assert e.min() >= 3 and e.max() <= 10                          # exponent field clipped
+        assert not np.isin(codes, [0x7F, 0xFF]).any()                  # no NaN in cached data
+        assert 0.4 < float((codes >> 7).mean()) < 0.6                  # both signs
