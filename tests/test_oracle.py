@@ -530,3 +530,20 @@ def test_prefill_row_ignores_keys_after_its_position():
                               c.query_start, c.scale)
         assert np.array_equal(out2[:i + 1], out[:i + 1])
         assert not np.allclose(out2[n - 1], out[n - 1])
+
+
+def test_oracle_result_does_not_depend_on_the_thread_count():
+    """Each (sequence, head) row is computed alone, so one thread and many give
+    the same bits (the CPU baseline may use either)."""
+    rng = RNG(11)
+    B, Hq, Hkv, D, bs = 5, 8, 2, 32, 4
+    ctx = [1, 7, 13, 4, 9]
+    kc = [_rand(rng, (n, Hkv, D), BF16) for n in ctx]
+    vc = [_rand(rng, (n, Hkv, D), BF16) for n in ctx]
+    kp, vp, tables = _paged_from_contiguous(kc, vc, bs, BF16, rng)
+    q = _rand(rng, (B, Hq, D), BF16)
+    cl = np.array(ctx, dtype=np.int32)
+    one = oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=1)
+    many = oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=4)
+    assert np.array_equal(one, many)
+    oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=oracle.max_threads())
