@@ -535,6 +535,7 @@ def test_prefill_row_ignores_keys_after_its_position():
 def test_oracle_result_does_not_depend_on_the_thread_count():
     """Each (sequence, head) row is computed alone, so one thread and many give
     the same bits (the CPU baseline may use either)."""
+    threads = oracle.max_threads()
     rng = RNG(11)
     B, Hq, Hkv, D, bs = 5, 8, 2, 32, 4
     ctx = [1, 7, 13, 4, 9]
@@ -546,4 +547,5 @@ def test_oracle_result_does_not_depend_on_the_thread_count():
     one = oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=1)
     many = oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=4)
     assert np.array_equal(one, many)
-    oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=oracle.max_threads())
+    oracle.decode(q, kp, vp, BF16, tables, cl, 0.2, n_threads=threads)    # restore the pool size
+    assert oracle.max_threads() == threads
