@@ -9,8 +9,16 @@ step has copy-on-write pairs) + paged decode attention, on synthetic workloads.
 One step = one pass of the whole hot path over one batch: the step's
 copy_blocks, then reshape_and_cache of the new tokens, then decode attention
 of every sequence's new query over its paged context (inputs resident in HBM).
-The default workload is the Llama-2-7B-shaped fp16 batch (64 sequences, 32
+The headline workload is the Llama-2-7B-shaped fp16 batch (64 sequences, 32
 heads x 128, contexts U[128, 2048], 16-token blocks, pool of 8192 blocks).
+With no --workload, the same JSON line also carries (one GPU only):
+  per_workload  the same step and fields on every other decode workload at full
+                size (Llama-3-70B-shaped GQA, long context, shared-prefix
+                sampling with plain and with shared-prefix decode, FP8 pools),
+                with the CUDA-core kernel timed beside the tensor-core one on
+                the GQA shapes (kernel_ab);
+  warm_l2       decode of a batch that fits the L2, with and without a flush;
+  paging_cost   decode on contiguous block tables against shuffled ones.
 
 Under torchrun (N > 1) every rank runs its own replica of the workload on its
 own GPU (weak scaling; the path has no exchange step, so there is no
@@ -54,6 +62,7 @@ from paged_kv_cache_418_b200 import workloads as W  # noqa: E402
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 METRIC = "paged decode attention KV GB/s"
+HEADLINE = "llama2-7b-fp16"
 
 
 def parse():
@@ -61,7 +70,11 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="llama2-7b-fp16")
+    p.add_argument("--workload", default=None,
+                   help="measure this workload alone (default: the Llama-2-7B-shaped batch as "
+                        "the headline, plus every other decode workload in per_workload)")
+    p.add_argument("--no-suite", action="store_true",
+                   help="default run: measure the headline workload only")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=None)
     p.add_argument("--batch", type=int, default=None,
@@ -307,32 +320,112 @@ def traffic_record(kernel: str, w: W.Workload):
     return rec.get("dram_bytes_per_launch")
 
 
-def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
+class Decoder:
+    """One workload's device tensors and its decode step through the C ABI."""
+
+    def __init__(self, w: W.Workload, dev, cascade: bool = False):
+        import torch
+        from paged_kv_cache_418_b200 import ops
+        self.w, self.dev, self.cascade, self.ops = w, dev, cascade, ops
+        self.t = W.to_torch(w, dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.out = torch.empty((w.B, w.Hq, w.D), dtype=self.t["torch_dtype"], device=dev)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        t = self.t
+        if cascade:
+            if "prefix_blocks" not in w.meta:
+                raise SystemExit("--shared-prefix needs a workload with groups "
+                                 "(shared-prefix-sampling-bf16)")
+            ng, nc, pb = w.meta["groups"], w.meta["children"], w.meta["prefix_blocks"]
+            self.group = (torch.full((w.B,), pb, dtype=torch.int32, device=dev),
+                          torch.arange(0, ng * nc + 1, nc, dtype=torch.int32, device=dev),
+                          torch.arange(ng * nc, dtype=torch.int32, device=dev), nc, pb)
+            self.ws = ops.shared_prefix_workspace_for(t["q"], t["k_cache"], w.max_context_len, pb,
+                                                      w.partition_size)
+        else:
+            self.ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len, w.partition_size)
+
+    def plan(self):
+        w = self.w
+        return self.ops.pa_decode_plan(w.kv_dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
+                                       w.max_context_len, w.partition_size)
+
+    def cache_ops(self):
+        w, t, ops = self.w, self.t, self.ops
+        if len(w.block_mapping):
+            ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], self.err, self.stream)
+        if w.fp8:
+            ops.pa_reshape_and_cache_fp8(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                         w.k_scale, w.v_scale, t["slot_mapping"], self.err,
+                                         self.stream)
+        else:
+            ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                     t["slot_mapping"], self.err, self.stream)
+
+    def decode(self):
+        w, t, ops = self.w, self.t, self.ops
+        if self.cascade:
+            g_shared, g_off, g_mem, nc, pb = self.group
+            ops.pa_decode_shared_prefix(self.out, t["q"], t["k_cache"], t["v_cache"],
+                                        t["block_tables"], t["context_lens"], g_shared, g_off,
+                                        g_mem, nc, pb, w.scale, w.max_context_len,
+                                        w.partition_size, self.ws, self.err, self.stream)
+        elif w.fp8:
+            ops.pa_decode_fp8(self.out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
+                              t["block_tables"], t["context_lens"], w.scale, w.max_context_len,
+                              w.partition_size, self.ws, self.err, self.stream)
+        else:
+            ops.pa_decode(self.out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                          t["context_lens"], w.scale, w.max_context_len, w.partition_size,
+                          self.ws, self.err, self.stream)
+
+    def step(self, ev=None):
+        """One step: the step's copy-on-write pairs, its new tokens, then decode."""
+        self.cache_ops()
+        if ev is not None:
+            ev[0].record(self.stream)
+        self.decode()
+        if ev is not None:
+            ev[1].record(self.stream)
+
+    def check(self, when: str):
+        import torch
+        torch.cuda.synchronize(self.dev)
+        if int(self.err.item()) != 0:
+            raise RuntimeError(f"{self.w.name}: device error flag {int(self.err.item())} {when}")
+
+
+def time_decode_only(d: Decoder, K: int, flush_buf=None) -> float:
+    """Mean event-timed duration (ms) of K back-to-back decode calls (L2 flushed
+    before each when flush_buf is given)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    for _ in range(3):
+        d.decode()
+    for e0, e1 in evs:
+        if flush_buf is not None:
+            flush_buf.zero_()
+        e0.record(d.stream)
+        d.decode()
+        e1.record(d.stream)
+    d.check("while timing decode")
+    return sum(a.elapsed_time(b) for a, b in evs) / K
+
+
+def measure(args, w: W.Workload, rank: int, world: int, local_rank: int, *,
+            cascade: bool = False, cuda_core_ab: bool = False):
+    """Time the step on one workload: W warm-up steps, K timed steps (barrier and
+    synchronize on both sides, max over ranks), then the end-to-end loop through
+    the same API with host buffers. Returns rank 0's fields (None elsewhere)."""
     import torch
     import torch.distributed as dist
-    from paged_kv_cache_418_b200 import _build, ops
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    t = W.to_torch(w, dev)
-    tdt = t["torch_dtype"]
-    stream = torch.cuda.current_stream(dev)
-    out = torch.empty((w.B, w.Hq, w.D), dtype=tdt, device=dev)
-    cascade = bool(getattr(args, "shared_prefix", False))
-    if cascade:
-        if "prefix_blocks" not in w.meta:
-            raise SystemExit("--shared-prefix needs a workload with groups (shared-prefix-sampling-bf16)")
-        ng, nc, pb = w.meta["groups"], w.meta["children"], w.meta["prefix_blocks"]
-        g_off = torch.arange(0, ng * nc + 1, nc, dtype=torch.int32, device=dev)
-        g_mem = torch.arange(ng * nc, dtype=torch.int32, device=dev)
-        g_shared = torch.full((w.B,), pb, dtype=torch.int32, device=dev)
-        ws = ops.shared_prefix_workspace_for(t["q"], t["k_cache"], w.max_context_len, pb,
-                                             w.partition_size)
-    else:
-        ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len, w.partition_size)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    kernel, P, psize = ops.pa_decode_plan(w.kv_dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
-                                          w.max_context_len, w.partition_size)
+    d = Decoder(w, dev, cascade)
+    t, stream = d.t, d.stream
+    kernel, P, psize = d.plan()
     launches_per_step = (1 if len(w.block_mapping) else 0) + 1 + 1 + (1 if P > 1 or cascade else 0) \
         + (1 if cascade else 0)
     unique = w.unique_kv_bytes()
@@ -341,41 +434,13 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
                f"inputs larger than L2 (KV {unique / 1e9:.2f} GB distinct > 126 MB)")
     flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
 
-    def step(ev=None):
-        if len(w.block_mapping):
-            ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err, stream)
-        if w.fp8:
-            ops.pa_reshape_and_cache_fp8(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
-                                         w.k_scale, w.v_scale, t["slot_mapping"], err, stream)
-        else:
-            ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
-                                     t["slot_mapping"], err, stream)
-        if ev is not None:
-            ev[0].record(stream)
-        if cascade:
-            ops.pa_decode_shared_prefix(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                                        t["context_lens"], g_shared, g_off, g_mem, nc, pb, w.scale,
-                                        w.max_context_len, w.partition_size, ws, err, stream)
-        elif w.fp8:
-            ops.pa_decode_fp8(out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
-                              t["block_tables"], t["context_lens"], w.scale, w.max_context_len,
-                              w.partition_size, ws, err, stream)
-        else:
-            ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
-                          t["context_lens"], w.scale, w.max_context_len, w.partition_size, ws,
-                          err, stream)
-        if ev is not None:
-            ev[1].record(stream)
-
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local_rank])
 
     for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    if int(err.item()) != 0:
-        raise RuntimeError(f"device error flag {int(err.item())} during warm-up")
+        d.step()
+    d.check("during warm-up")
 
     K = args.steps
     dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -394,7 +459,7 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
         if flush:
             flush_buf.zero_()
             step_ev[i][0].record(stream)
-        step(dec_ev[i])
+        d.step(dec_ev[i])
         if flush:
             step_ev[i][1].record(stream)
     t_end.record(stream)
@@ -407,22 +472,21 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
         ms = t_start.elapsed_time(t_end)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev) / K
     ms, dec_ms = max_over_ranks([ms, dec_ms], world, dev)
-    if int(err.item()) != 0:
-        raise RuntimeError(f"device error flag {int(err.item())} during timing")
+    d.check("during timing")
 
     # end to end through the public API: pinned host inputs -> device -> step -> host result
     host = {k: v.cpu().pin_memory() for k, v in t.items()
             if k in ("q", "new_key", "new_value", "slot_mapping", "block_tables",
                      "context_lens", "block_mapping")}
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    out_host = torch.empty(d.out.shape, dtype=d.out.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out.numel() * out.element_size()
+    d2h = d.out.numel() * d.out.element_size()
     Ke = args.e2e_steps or max(1, min(K, 200))
     for _ in range(2):
         for k, v in host.items():
             t[k].copy_(v, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
+        d.step()
+        out_host.copy_(d.out, non_blocking=True)
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -433,13 +497,26 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
         e0.record(stream)
         for k, v in host.items():
             t[k].copy_(v, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
+        d.step()
+        out_host.copy_(d.out, non_blocking=True)
         e1.record(stream)
         e1.synchronize()
         e_ms += e0.elapsed_time(e1)
     (e_ms,) = max_over_ranks([e_ms], world, dev)
     barrier()
+
+    # the same decode forced onto the CUDA-core kernel (evidence for the tensor-core choice)
+    ab = None
+    if cuda_core_ab and kernel == 2 and not cascade and rank == 0 and world == 1:
+        tc_us = 1e3 * time_decode_only(d, K, flush_buf)
+        os.environ["PA_DECODE_KERNEL"] = "simt"
+        try:
+            cc_us = 1e3 * time_decode_only(d, K, flush_buf)
+        finally:
+            del os.environ["PA_DECODE_KERNEL"]
+        ab = {"decode_us_tcgen05": round(tc_us, 2), "decode_us_cuda_core": round(cc_us, 2),
+              "cuda_core_over_tcgen05": round(cc_us / tc_us, 3),
+              "how": f"{K} decode calls back to back per kernel, same inputs, same loop"}
     if rank != 0:
         return None
 
@@ -448,7 +525,7 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
     peak, peak_src = peaks()
     kname = {1: "cuda-core", 2: "tcgen05"}[kernel] if not cascade else "shared-prefix"
     # the cascade reads each distinct K/V byte once: its algorithmic bytes are the distinct ones
-    alg = w.unique_kv_bytes() if cascade else kv
+    alg = unique if cascade else kv
     achieved = alg / (dec_ms / 1e3) / 1e9
     traffic = traffic_record(kname, w)
     e2e_value = job_value(kv, Ke, world, e_ms)
@@ -466,7 +543,9 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
                         "partition_tokens": psize},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "peak_source": f"hbm_gbs ({peak_src})",
+                     "traffic": traffic,
+                     "traffic_ratio": round(traffic / alg, 4) if traffic else None,
+                     "peak_source": f"hbm_gbs ({peak_src})",
                      "kernel": ("pa_decode_shared_prefix (suffix pass + prefix pass + merge)"
                                 if cascade else "pa_decode (partition pass + merge)") + ", per launch",
                      "algorithmic_bytes": alg},
@@ -475,7 +554,92 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke},
     }
+    if ab is not None:
+        line["kernel_ab"] = ab
+    del d
+    torch.cuda.empty_cache()
     return line
+
+
+def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
+    return measure(args, w, rank, world, local_rank,
+                   cascade=bool(getattr(args, "shared_prefix", False)))
+
+
+SUITE = [  # (workload id, shared-prefix decode) measured beside the headline by default
+    (3, False), (4, False), (5, False), (5, True), (6, False)]
+
+
+def suite(args, local_rank: int):
+    """Every other decode workload at full size, one GPU: the same step and
+    fields as the headline (plus the CUDA-core A/B on the tensor-core shapes),
+    each with a bounded oracle sample as its CPU baseline."""
+    out = {}
+    for k, cascade in SUITE:
+        w = W.make_workload(k, seed=rank_seed(k, 0))
+        line = measure(args, w, 0, 1, local_rank, cascade=cascade, cuda_core_ab=True)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=3.0)
+        keep = ("value", "unit", "ms_per_step", "decode_us", "kernel_ab",
+                "seq_steps_per_s", "pct_of_hbm_peak", "decode_plan",
+                "roofline", "gpu_launches", "clocks", "e2e", "cpu_baseline", "config", "dtype")
+        out[w.name + (" (pa_decode_shared_prefix)" if cascade else "")] = \
+            {k2: line[k2] for k2 in keep if k2 in line}
+        del w
+    return out
+
+
+def warm_l2(args, local_rank: int):
+    """Decode of a Llama-2-7B-shaped batch small enough for the 126 MB L2 (4
+    sequences), back to back without a flush (warm) and with the L2 flushed
+    before each call (cold)."""
+    import torch
+    dev = torch.device("cuda", local_rank)
+    w = W.make_workload(2, seed=rank_seed(2, 0), batch=4)
+    d = Decoder(w, dev)
+    d.cache_ops()
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    K = max(20, args.steps)
+    warm = time_decode_only(d, K)
+    cold = time_decode_only(d, K, flush_buf)
+    kv = w.kv_bytes()
+    peak, _ = peaks()
+    del d, flush_buf
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "kv_bytes": kv, "calls": K,
+            "decode_us_warm": round(warm * 1e3, 2), "gbs_warm": round(kv / (warm / 1e3) / 1e9, 1),
+            "decode_us_cold": round(cold * 1e3, 2), "gbs_cold": round(kv / (cold / 1e3) / 1e9, 1),
+            "frac_of_hbm_peak_warm": round(kv / (warm / 1e3) / 1e9 / peak, 4),
+            "note": "decode calls back to back; warm = no flush (the batch stays in L2), "
+                    "cold = 252 MB written before each call"}
+
+
+def paging_cost(args, local_rank: int):
+    """The same decode on the same lengths and bytes, with each sequence's
+    blocks contiguous (identity-like table) instead of popped from a shuffled
+    free list: what non-contiguous physical blocks cost the kernel."""
+    import torch
+    dev = torch.device("cuda", local_rank)
+    res = {}
+    for k in (2, 3):
+        K = max(20, args.steps)
+        times = {}
+        for layout in ("contiguous", "shuffled"):
+            w = W.make_workload(k, seed=rank_seed(k, 0), contiguous=layout == "contiguous")
+            d = Decoder(w, dev)
+            d.cache_ops()
+            times[layout] = time_decode_only(d, K)
+            kv = w.kv_bytes()
+            del d, w
+            torch.cuda.empty_cache()
+        res[W.WORKLOADS[k]] = {
+            "decode_us_contiguous": round(times["contiguous"] * 1e3, 2),
+            "decode_us_shuffled": round(times["shuffled"] * 1e3, 2),
+            "paging_overhead_pct": round(100.0 * (times["shuffled"] / times["contiguous"] - 1), 2),
+            "kv_bytes": kv, "calls": K}
+    res["note"] = ("decode calls back to back (inputs larger than L2); contiguous = every "
+                   "sequence's blocks are consecutive physical ids, shuffled = ids popped from "
+                   "a seeded permutation of the pool (the benchmark's layout)")
+    return res
 
 
 def rank_seed(k: int, rank: int) -> int:
@@ -758,7 +922,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    k = workload_id(args.workload)
+    default_run = args.workload is None
+    k = workload_id(args.workload or HEADLINE)
     seed = rank_seed(k, rank)
     if args.impl == "reference":
         if rank != 0:
@@ -785,6 +950,15 @@ def main():
     finally:
         if world > 1:
             dist.destroy_process_group()
+    del w
+    if rank == 0 and default_run and not args.no_suite:
+        if world == 1 and args.batch is None:
+            # the other workloads of the same step, and two reference measurements
+            line["per_workload"] = suite(args, local_rank)
+            line["warm_l2"] = warm_l2(args, local_rank)
+            line["paging_cost"] = paging_cost(args, local_rank)
+        else:
+            line["per_workload"] = {"note": "measured at N=1 only (one GPU)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0

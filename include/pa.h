@@ -165,11 +165,15 @@ int pa_copy_blocks(void* key_cache, void* value_cache, int dtype, const int64_t*
  *  - Sizes whose pa_workspace_size(...) exceeds PA_STATIC_SCRATCH_BYTES are
  *    rejected with PA_ERR_WORKSPACE before anything is launched.
  *  - Every GPU that loads the array keeps those bytes until the process exits.
- *  - The first call on a device (with that device current) looks up the
- *    array's device address; make that first call before any stream capture.
- *  - All calls on a device share the one array and it keeps the last call's
- *    contents (nothing in it needs to start at zero); calls that overlap on
- *    the GPU race on it, so order them (one stream, or events).
+ *  - The array's device address belongs to the CUDA context the library was
+ *    loaded into. Each call looks it up in the context current at that call
+ *    (so a second context on the device, or a device reset, gets its own
+ *    array), except while `stream` is capturing: then the address found by
+ *    the last call made outside capture in the same context is reused, and
+ *    with none the call fails (PA_ERR_CUDA). Make a first call outside capture.
+ *  - All calls in one context share the one array and it keeps the last
+ *    call's contents (nothing in it needs to start at zero); calls that
+ *    overlap on the GPU race on it, so order them (one stream, or events).
  * Returns a pa_status like pa_decode (PA_ERR_CUDA if the address lookup fails).
  */
 #define PA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)

@@ -10,6 +10,7 @@ raises.
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional, Tuple
@@ -108,6 +109,15 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _on_device_of(*tensors):
+    """Make the device of the first CUDA tensor current for the call, so the
+    default stream (and, for pa_decode_static, the scratch) is that device's."""
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return torch.cuda.device(t.device)
+    return contextlib.nullcontext()
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -148,17 +158,19 @@ def pa_decode(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
     """out [B,Hq,D] <- paged decode attention (see pa_decode in include/pa.h)."""
     B, Hq, D = query.shape
     num_blocks, block_size, Hkv, _ = key_cache.shape
-    rc = LIB.pa_decode(
-        _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-        B, Hq, Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
-        int(partition_size), _ptr(workspace),
-        0 if workspace is None else workspace.numel() * workspace.element_size(),
-        _ptr(err_flag), _stream(stream))
+    with _on_device_of(query):
+        rc = LIB.pa_decode(
+            _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+            pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+            B, Hq, Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
+            int(partition_size), _ptr(workspace),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode", rc)
 
 
+# PA_STATIC_SCRATCH_BYTES of include/pa.h (a CPU test checks the two agree)
 PA_STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
@@ -172,11 +184,12 @@ def pa_decode_static(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Te
     in include/pa.h: one shared scratch per device, calls must not overlap)."""
     B, Hq, D = query.shape
     num_blocks, block_size, Hkv, _ = key_cache.shape
-    rc = LIB.pa_decode_static(
-        _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-        B, Hq, Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
-        int(partition_size), _ptr(err_flag), _stream(stream))
+    with _on_device_of(query):
+        rc = LIB.pa_decode_static(
+            _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+            pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+            B, Hq, Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
+            int(partition_size), _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode_static", rc)
 
@@ -189,9 +202,10 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, key_cache: torc
         check_slot_mapping(slot_mapping)
     num_blocks, block_size, Hkv, D = key_cache.shape
     T = slot_mapping.shape[0]
-    rc = LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache),
-                                  pa_dtype(key_cache), _ptr(slot_mapping), T, Hkv, D,
-                                  block_size, num_blocks, _ptr(err_flag), _stream(stream))
+    with _on_device_of(key_cache):
+        rc = LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache),
+                                      pa_dtype(key_cache), _ptr(slot_mapping), T, Hkv, D,
+                                      block_size, num_blocks, _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_reshape_and_cache", rc)
 
@@ -204,9 +218,10 @@ def pa_copy_blocks(key_cache: torch.Tensor, value_cache: torch.Tensor,
         check_block_mapping(block_mapping)
     num_blocks, block_size, Hkv, D = key_cache.shape
     P = block_mapping.shape[0]
-    rc = LIB.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), pa_dtype(key_cache),
-                            _ptr(block_mapping), P, Hkv, D, block_size, num_blocks,
-                            _ptr(err_flag), _stream(stream))
+    with _on_device_of(key_cache):
+        rc = LIB.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), pa_dtype(key_cache),
+                                _ptr(block_mapping), P, Hkv, D, block_size, num_blocks,
+                                _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_copy_blocks", rc)
 
@@ -220,13 +235,14 @@ def pa_decode_fp8(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tenso
     """out [B,Hq,D] <- paged decode attention over FP8 E4M3 pools (uint8 codes)."""
     B, Hq, D = query.shape
     num_blocks, block_size, Hkv, _ = key_cache.shape
-    rc = LIB.pa_decode_fp8(
-        _ptr(out), pa_dtype(out), _ptr(query), pa_dtype(query), _ptr(key_cache),
-        _ptr(value_cache), float(k_scale), float(v_scale), _ptr(block_tables),
-        block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, block_size, num_blocks,
-        float(scale), int(max_context_len), int(partition_size), _ptr(workspace),
-        0 if workspace is None else workspace.numel() * workspace.element_size(),
-        _ptr(err_flag), _stream(stream))
+    with _on_device_of(query):
+        rc = LIB.pa_decode_fp8(
+            _ptr(out), pa_dtype(out), _ptr(query), pa_dtype(query), _ptr(key_cache),
+            _ptr(value_cache), float(k_scale), float(v_scale), _ptr(block_tables),
+            block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, block_size, num_blocks,
+            float(scale), int(max_context_len), int(partition_size), _ptr(workspace),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode_fp8", rc)
 
@@ -240,10 +256,11 @@ def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: 
         check_slot_mapping(slot_mapping, "pa_reshape_and_cache_fp8")
     num_blocks, block_size, Hkv, D = key_cache.shape
     T = slot_mapping.shape[0]
-    rc = LIB.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), pa_dtype(key), _ptr(key_cache),
-                                      _ptr(value_cache), float(k_scale), float(v_scale),
-                                      _ptr(slot_mapping), T, Hkv, D, block_size, num_blocks,
-                                      _ptr(err_flag), _stream(stream))
+    with _on_device_of(key_cache):
+        rc = LIB.pa_reshape_and_cache_fp8(_ptr(key), _ptr(value), pa_dtype(key), _ptr(key_cache),
+                                          _ptr(value_cache), float(k_scale), float(v_scale),
+                                          _ptr(slot_mapping), T, Hkv, D, block_size, num_blocks,
+                                          _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_reshape_and_cache_fp8", rc)
 
@@ -258,9 +275,10 @@ def pa_swap_blocks(dst_key: torch.Tensor, dst_value: torch.Tensor, src_key: torc
     src_blocks, block_size, Hkv, D = src_key.shape
     dst_blocks = dst_key.shape[0]
     P = block_mapping.shape[0]
-    rc = LIB.pa_swap_blocks(_ptr(dst_key), _ptr(dst_value), _ptr(src_key), _ptr(src_value),
-                            pa_dtype(src_key), _ptr(block_mapping), P, Hkv, D, block_size,
-                            src_blocks, dst_blocks, _ptr(err_flag), _stream(stream))
+    with _on_device_of(dst_key, src_key):
+        rc = LIB.pa_swap_blocks(_ptr(dst_key), _ptr(dst_value), _ptr(src_key), _ptr(src_value),
+                                pa_dtype(src_key), _ptr(block_mapping), P, Hkv, D, block_size,
+                                src_blocks, dst_blocks, _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_swap_blocks", rc)
 
@@ -285,14 +303,15 @@ def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: t
     pa_decode_shared_prefix in include/pa.h): shared blocks read once per group."""
     B, Hq, D = query.shape
     num_blocks, block_size, Hkv, _ = key_cache.shape
-    rc = LIB.pa_decode_shared_prefix(
-        _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-        _ptr(shared_blocks), group_offsets.shape[0] - 1, _ptr(group_offsets), _ptr(group_members),
-        int(max_group_size), int(max_shared_blocks), B, Hq, Hkv, D, block_size, num_blocks,
-        float(scale), int(max_context_len), int(partition_size), _ptr(workspace),
-        0 if workspace is None else workspace.numel() * workspace.element_size(),
-        _ptr(err_flag), _stream(stream))
+    with _on_device_of(query):
+        rc = LIB.pa_decode_shared_prefix(
+            _ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+            pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+            _ptr(shared_blocks), group_offsets.shape[0] - 1, _ptr(group_offsets), _ptr(group_members),
+            int(max_group_size), int(max_shared_blocks), B, Hq, Hkv, D, block_size, num_blocks,
+            float(scale), int(max_context_len), int(partition_size), _ptr(workspace),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode_shared_prefix", rc)
 
@@ -306,11 +325,12 @@ def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
     T, Hq, D = query.shape
     num_blocks, block_size, Hkv, _ = key_cache.shape
     B = query_start.shape[0] - 1
-    rc = LIB.pa_prefill(_ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-                        pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1],
-                        _ptr(context_lens), _ptr(query_start), B, T, int(max_query_len), Hq, Hkv,
-                        D, block_size, num_blocks, float(scale), int(max_context_len),
-                        _ptr(err_flag), _stream(stream))
+    with _on_device_of(query):
+        rc = LIB.pa_prefill(_ptr(out), pa_dtype(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                            pa_dtype(key_cache), _ptr(block_tables), block_tables.shape[1],
+                            _ptr(context_lens), _ptr(query_start), B, T, int(max_query_len), Hq, Hkv,
+                            D, block_size, num_blocks, float(scale), int(max_context_len),
+                            _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_prefill", rc)
 

@@ -92,10 +92,11 @@ def random_e4m3_codes(rng: np.random.Generator, shape, lo: int = 3, hi: int = 10
 
     The exponent field lies in [lo, hi]; lo=0, hi=15 reaches every finite code.
     """
-    sign = rng.integers(0, 2, size=shape, dtype=np.int64)
-    ex = np.clip(np.rint(rng.normal(7.0, 1.0, size=shape)), lo, hi).astype(np.int64)
-    frac = rng.integers(0, 8, size=shape, dtype=np.int64)
-    frac = np.where((ex == 15) & (frac == 7), 6, frac)
+    sign = rng.integers(0, 2, size=shape, dtype=np.uint8)
+    ex = np.clip(np.rint(rng.standard_normal(size=shape, dtype=np.float32) + np.float32(7.0)),
+                 lo, hi).astype(np.uint8)
+    frac = rng.integers(0, 8, size=shape, dtype=np.uint8)
+    frac = np.where((ex == 15) & (frac == 7), np.uint8(6), frac)
     return ((sign << 7) | (ex << 3) | frac).astype(np.uint8)
 
 
@@ -208,13 +209,22 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
         raise ValueError("need B context lengths, each >= 1")
     order = rng.permutation(num_blocks) if shuffle else np.arange(num_blocks)
     bm = BlockManager(num_blocks, block_size, order)
-    for b in range(B):
-        bm.allocate_prefill(b, int(ctx[b]) - 1)
     slots = np.empty(B, dtype=np.int64)
-    for b in range(B):
-        slot, cow = bm.append_token(b)
-        assert cow is None
-        slots[b] = slot
+    if shuffle:
+        for b in range(B):
+            bm.allocate_prefill(b, int(ctx[b]) - 1)
+        for b in range(B):
+            slot, cow = bm.append_token(b)
+            assert cow is None
+            slots[b] = slot
+    else:
+        # contiguous layout: each sequence's blocks, the appended token's
+        # included, are one run of consecutive physical ids
+        for b in range(B):
+            bm.allocate_prefill(b, int(ctx[b]) - 1)
+            slot, cow = bm.append_token(b)
+            assert cow is None
+            slots[b] = slot
     need = max(len(bm.seqs[b].block_table) for b in range(B))
     MB = need if max_blocks is None else int(max_blocks)
     if MB < need:
@@ -478,13 +488,24 @@ WORKLOADS = {
 WORKLOAD_IDS = {v: k for k, v in WORKLOADS.items()}
 
 
-def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None) -> Workload:
-    """Build workload ``which`` (1..5 or its name); seed defaults to 1000 + id.
+def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None,
+                  contiguous: bool = False) -> Workload:
+    """Build workload ``which`` (1..6 or its name); seed defaults to 1000 + id.
 
     ``batch`` (profiling runs) keeps every distribution and shape but uses that
     many sequences (groups of 16 for the shared-prefix workload) and a pool
     scaled down with them.
+
+    ``contiguous`` (workloads 2, 3 and 6, full size) gives every sequence one
+    run of consecutive physical blocks instead of ids popped from a shuffled
+    free list: the same lengths and bytes, with paging reduced to an identity
+    table (for measuring what non-contiguous blocks cost).
     """
+    if contiguous:
+        k = WORKLOAD_IDS[which] if isinstance(which, str) else int(which)
+        if k not in (2, 3, 6) or batch is not None:
+            raise ValueError("contiguous layouts are built for workloads 2, 3 and 6 at full size")
+        return _make_contiguous(k, 1000 + k if seed is None else int(seed))
     k = WORKLOAD_IDS[which] if isinstance(which, str) else int(which)
     seed = 1000 + k if seed is None else int(seed)
     name = WORKLOADS[k] if batch is None else f"{WORKLOADS[k]}-b{int(batch)}"
@@ -523,6 +544,21 @@ def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None
                                  num_blocks=8192, context_lens=ctx, seed=seed, rng=rng,
                                  max_blocks=128, kv_fp8=True)
     raise KeyError(which)
+
+
+def _make_contiguous(k: int, seed: int) -> Workload:
+    rng = np.random.Generator(np.random.PCG64(seed))
+    name = WORKLOADS[k] + "-contiguous"
+    if k in (2, 6):
+        ctx = rng.integers(128, 2049, size=64)
+        return build_decode_case(name, F16, B=64, Hq=32, Hkv=32, D=128, block_size=16,
+                                 num_blocks=8192, context_lens=ctx, seed=seed, rng=rng,
+                                 max_blocks=128, kv_fp8=k == 6, shuffle=False)
+    ln = rng.lognormal(mean=math.log(1200.0), sigma=0.8, size=128)
+    ctx = np.clip(np.rint(ln), 16, 8192).astype(np.int64)
+    return build_decode_case(name, BF16, B=128, Hq=64, Hkv=8, D=128, block_size=16,
+                             num_blocks=65536, context_lens=ctx, seed=seed, rng=rng,
+                             max_blocks=512, shuffle=False)
 
 
 def _make_batch(k: int, name: str, seed: int, B: int) -> Workload:

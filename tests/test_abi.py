@@ -34,6 +34,14 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(ops, n), n           # the binding keeps the same names
 
 
+def test_binding_scratch_size_matches_the_header():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    m = re.search(r"#define PA_STATIC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", src)
+    assert m, "PA_STATIC_SCRATCH_BYTES not found in include/pa.h"
+    a, b, c = (int(x) for x in m.groups())
+    assert ops.PA_STATIC_SCRATCH_BYTES == a * b * c
+
+
 def test_status_strings():
     assert ops.pa_status_string(0) == "ok"
     for s in range(1, 8):
