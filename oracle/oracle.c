@@ -68,7 +68,10 @@
  *                     even, saturating at +-448; value read = code * scale.
  *                     oracle_reshape_and_cache_fp8 quantises that way and
  *                     oracle_decode_kv reads the codes times their scale
- *                     (exact in double).
+ *                     (exact in double). The explainer's mixed configuration
+ *                     (K in fp8, V in bf16) takes one element type per pool:
+ *                     oracle_decode_mixed, oracle_prefill_mixed and
+ *                     oracle_reshape_and_cache_mixed.
  *
  * Inputs are read exactly: f32 as is; f16 and bf16 are widened to double from
  * their bit patterns by the IEEE-754 definitions of those formats.
@@ -177,11 +180,12 @@ int oracle_gather(double* out, const void* pool, int dtype, const int32_t* table
   return OR_OK;
 }
 
-/* One (b, hq) output row by the textbook two-pass softmax. */
-static int attend_row(double* o, const void* q, int qdt, const void* kpool, const void* vpool,
-                      int kvdt, double kscale, double vscale, const int32_t* table, int ctx,
-                      int Hq, int Hkv, int D, int bs, int num_blocks, double scale, int b,
-                      int hq) {
+/* One (b, hq) output row by the textbook two-pass softmax (K and V pools may
+   hold different element types). */
+static int attend_row(double* o, const void* q, int qdt, const void* kpool, int kdt,
+                      double kscale, const void* vpool, int vdt, double vscale,
+                      const int32_t* table, int ctx, int Hq, int Hkv, int D, int bs,
+                      int num_blocks, double scale, int b, int hq) {
   int G = Hq / Hkv, h = hq / G;
   for (int d = 0; d < D; ++d) o[d] = 0.0;
   if (ctx <= 0) return OR_OK;
@@ -191,9 +195,9 @@ static int attend_row(double* o, const void* q, int qdt, const void* kpool, cons
   double* qv = (double*)malloc(sizeof(double) * (size_t)D);
   int rc = OR_ERR_NOMEM;
   if (K && V && s && qv) {
-    rc = gather_head(K, kpool, kvdt, kscale, table, ctx, Hkv, h, D, bs, num_blocks);
+    rc = gather_head(K, kpool, kdt, kscale, table, ctx, Hkv, h, D, bs, num_blocks);
     if (rc == OR_OK)
-      rc = gather_head(V, vpool, kvdt, vscale, table, ctx, Hkv, h, D, bs, num_blocks);
+      rc = gather_head(V, vpool, vdt, vscale, table, ctx, Hkv, h, D, bs, num_blocks);
   }
   if (rc == OR_OK) {
     for (int d = 0; d < D; ++d) qv[d] = elem(q, ((size_t)b * Hq + hq) * D + d, qdt);
@@ -230,16 +234,20 @@ static int check_decode_args(const void* q, const void* kp, const void* vp, int 
 
 /*
  * out: [n_rows, D] (rows != NULL: rows holds n_rows (b, hq) pairs) or
- *      [B, Hq, D] (rows == NULL).
+ *      [B, Hq, D] (rows == NULL). The K pool holds k_dtype elements (read times
+ * k_scale), the V pool v_dtype elements (times v_scale): an FP8 K pool with a
+ * 16-bit V pool is the mixed configuration of "vLLM与PagedAttention：大模型推理
+ * 内存优化技术解析" section 6.1.
  * Returns OR_OK, or an error code (first error wins); n_threads <= 0 = all.
  */
-int oracle_decode_kv(double* out, const void* q, int q_dtype, const void* kpool,
-                     const void* vpool, int kv_dtype, double k_scale, double v_scale,
-                     const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
-                     int B, int Hq, int Hkv, int D, int bs, int num_blocks, double scale,
-                     const int32_t* rows, int n_rows, int n_threads) {
+int oracle_decode_mixed(double* out, const void* q, int q_dtype, const void* kpool, int k_dtype,
+                        double k_scale, const void* vpool, int v_dtype, double v_scale,
+                        const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                        int B, int Hq, int Hkv, int D, int bs, int num_blocks, double scale,
+                        const int32_t* rows, int n_rows, int n_threads) {
   if (q_dtype < OR_F32 || q_dtype > OR_BF16) return OR_ERR_ARG;
-  int rc = check_decode_args(q, kpool, vpool, kv_dtype, block_tables, max_blocks, context_lens,
+  if (v_dtype < OR_F32 || v_dtype > OR_FP8) return OR_ERR_ARG;
+  int rc = check_decode_args(q, kpool, vpool, k_dtype, block_tables, max_blocks, context_lens,
                              B, Hq, Hkv, D, bs);
   if (rc != OR_OK || !out) return rc ? rc : OR_ERR_ARG;
   long long n = rows ? n_rows : (long long)B * Hq;
@@ -254,7 +262,7 @@ int oracle_decode_kv(double* out, const void* q, int q_dtype, const void* kpool,
     int e;
     if (b < 0 || b >= B || hq < 0 || hq >= Hq) e = OR_ERR_ARG;
     else
-      e = attend_row(out + r * D, q, q_dtype, kpool, vpool, kv_dtype, k_scale, v_scale,
+      e = attend_row(out + r * D, q, q_dtype, kpool, k_dtype, k_scale, vpool, v_dtype, v_scale,
                      block_tables + (size_t)b * max_blocks, context_lens[b], Hq, Hkv, D, bs,
                      num_blocks, scale, b, hq);
     if (e != OR_OK) {
@@ -267,18 +275,32 @@ int oracle_decode_kv(double* out, const void* q, int q_dtype, const void* kpool,
   return err;
 }
 
+/* Both pools of one element type (kv_dtype), the query of q_dtype. */
+int oracle_decode_kv(double* out, const void* q, int q_dtype, const void* kpool,
+                     const void* vpool, int kv_dtype, double k_scale, double v_scale,
+                     const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                     int B, int Hq, int Hkv, int D, int bs, int num_blocks, double scale,
+                     const int32_t* rows, int n_rows, int n_threads) {
+  return oracle_decode_mixed(out, q, q_dtype, kpool, kv_dtype, k_scale, vpool, kv_dtype, v_scale,
+                             block_tables, max_blocks, context_lens, B, Hq, Hkv, D, bs,
+                             num_blocks, scale, rows, n_rows, n_threads);
+}
+
 /*
  * Causal prefill: out [T, Hq, D]; query [T, Hq, D] (packed new tokens, rows
  * query_start[b] .. query_start[b+1] of sequence b); context_lens after the chunk.
  */
-int oracle_prefill(double* out, const void* q, const void* kpool, const void* vpool, int dtype,
-                   const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
-                   const int32_t* query_start, int B, int Hq, int Hkv, int D, int bs,
-                   int num_blocks, double scale, int n_threads) {
+int oracle_prefill_mixed(double* out, const void* q, int q_dtype, const void* kpool,
+                         int k_dtype, double k_scale, const void* vpool, int v_dtype,
+                         double v_scale, const int32_t* block_tables, int max_blocks,
+                         const int32_t* context_lens, const int32_t* query_start, int B, int Hq,
+                         int Hkv, int D, int bs, int num_blocks, double scale, int n_threads) {
   if (!out || !query_start) return OR_ERR_ARG;
-  int rc = check_decode_args(q, kpool, vpool, dtype, block_tables, max_blocks, context_lens, B,
+  if (q_dtype < OR_F32 || q_dtype > OR_BF16 || v_dtype < OR_F32 || v_dtype > OR_FP8)
+    return OR_ERR_ARG;
+  int rc = check_decode_args(q, kpool, vpool, k_dtype, block_tables, max_blocks, context_lens, B,
                              Hq, Hkv, D, bs);
-  if (rc != OR_OK || dtype == OR_FP8) return rc ? rc : OR_ERR_ARG;
+  if (rc != OR_OK) return rc;
   for (int b = 0; b < B; ++b) {
     int n = query_start[b + 1] - query_start[b];
     if (n < 0 || n > context_lens[b]) return OR_ERR_ARG;
@@ -295,7 +317,7 @@ int oracle_prefill(double* out, const void* q, const void* kpool, const void* vp
     while (query_start[b + 1] <= t) ++b;                /* the sequence of query row t */
     int n = query_start[b + 1] - query_start[b];
     int pos = context_lens[b] - n + (int)(t - query_start[b]);
-    int e = attend_row(out + r * D, q, dtype, kpool, vpool, dtype, 1.0, 1.0,
+    int e = attend_row(out + r * D, q, q_dtype, kpool, k_dtype, k_scale, vpool, v_dtype, v_scale,
                        block_tables + (size_t)b * max_blocks, pos + 1, Hq, Hkv, D, bs,
                        num_blocks, scale, (int)t, hq);
     if (e != OR_OK) {
@@ -306,6 +328,17 @@ int oracle_prefill(double* out, const void* q, const void* kpool, const void* vp
     }
   }
   return err;
+}
+
+/* One element type for the query and both pools (16/32-bit). */
+int oracle_prefill(double* out, const void* q, const void* kpool, const void* vpool, int dtype,
+                   const int32_t* block_tables, int max_blocks, const int32_t* context_lens,
+                   const int32_t* query_start, int B, int Hq, int Hkv, int D, int bs,
+                   int num_blocks, double scale, int n_threads) {
+  if (dtype == OR_FP8) return OR_ERR_ARG;
+  return oracle_prefill_mixed(out, q, dtype, kpool, dtype, 1.0, vpool, dtype, 1.0, block_tables,
+                              max_blocks, context_lens, query_start, B, Hq, Hkv, D, bs,
+                              num_blocks, scale, n_threads);
 }
 
 /* Same element type for q, K and V (16/32-bit pools). */
@@ -451,6 +484,46 @@ int oracle_reshape_and_cache_fp8(uint8_t* kpool, uint8_t* vpool, const void* key
       float vx = (float)elem(value, (size_t)t * row + i, src_dtype);
       kpool[(size_t)s * row + i] = e4m3_from_float(kx / k_scale);
       vpool[(size_t)s * row + i] = e4m3_from_float(vx / v_scale);
+    }
+  }
+  return OR_OK;
+}
+
+/* Scatter into pools of per-pool element types: a pool of the source type gets
+   the row copied bit for bit, an FP8 pool gets codes E4M3(float(x) / scale)
+   (the two cases above, one per pool). */
+int oracle_reshape_and_cache_mixed(void* kpool, void* vpool, const void* key, const void* value,
+                                   int src_dtype, int k_dtype, int v_dtype, float k_scale,
+                                   float v_scale, const int64_t* slot_mapping, int T, int Hkv,
+                                   int D, int bs, int num_blocks) {
+  if (!kpool || !vpool || (T > 0 && (!key || !value || !slot_mapping))) return OR_ERR_ARG;
+  if (T < 0 || Hkv <= 0 || D <= 0 || bs <= 0 || num_blocks <= 0) return OR_ERR_ARG;
+  if (src_dtype < OR_F32 || src_dtype > OR_BF16) return OR_ERR_ARG;
+  if ((k_dtype != src_dtype && k_dtype != OR_FP8) || (v_dtype != src_dtype && v_dtype != OR_FP8))
+    return OR_ERR_ARG;
+  if ((k_dtype == OR_FP8 && !(k_scale > 0.f)) || (v_dtype == OR_FP8 && !(v_scale > 0.f)))
+    return OR_ERR_ARG;
+  size_t row = (size_t)Hkv * D;
+  long long nslots = (long long)num_blocks * bs;
+  for (int t = 0; t < T; ++t)
+    if (slot_mapping[t] >= nslots) return OR_ERR_SLOT;
+  for (int t = 0; t < T; ++t) {
+    int64_t s = slot_mapping[t];
+    if (s < 0) continue;
+    for (int which = 0; which < 2; ++which) {
+      const void* src = which ? value : key;
+      void* pool = which ? vpool : kpool;
+      int pdt = which ? v_dtype : k_dtype;
+      float sc = which ? v_scale : k_scale;
+      if (pdt == OR_FP8) {
+        for (size_t i = 0; i < row; ++i) {
+          float x = (float)elem(src, (size_t)t * row + i, src_dtype);
+          ((uint8_t*)pool)[(size_t)s * row + i] = e4m3_from_float(x / sc);
+        }
+      } else {
+        size_t rb = row * esize_of(pdt);
+        memcpy((char*)pool + (size_t)s * rb, (const char*)src + (size_t)t * rb, rb);
+      }
     }
   }
   return OR_OK;

@@ -27,6 +27,8 @@
 // 3.2); the tiling and vector layout here are this library's own.
 #include <math_constants.h>
 
+#include <cstdlib>
+
 #include "pa_internal.h"
 
 namespace pa {
@@ -54,8 +56,9 @@ __device__ __forceinline__ void load_q(const TQ* p, float* f) {
   for (int c = 0; c < VEC / N; ++c) widen16<TQ>(*reinterpret_cast<const uint4*>(p + c * N), f + c * N);
 }
 
-// TQ: query element type; TC: pool element type (TQ, or FP8 E4M3 codes).
-template <typename TQ, typename TC, int D, int BS, int GC>
+// TQ: query element type; TC: pool element type (TQ, or FP8 E4M3 codes);
+// PF: issue the loads of each warp's next tile before computing the current one.
+template <typename TQ, typename TC, int D, int BS, int GC, bool PF>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_simt_kernel(const DecodeArgs a) {
   using T = TC;
@@ -130,33 +133,27 @@ decode_simt_kernel(const DecodeArgs a) {
   const int tile_begin = tok_begin / TILE;
   const int tile_end = (tok_end + TILE - 1) / TILE;
 
-  int t = tile_begin + warp;
-  int phys_next = t < tile_end ? __ldg(table + (t * TILE) / BS) : 0;
-  for (; t < tile_end; t += kWarps) {
-    const int phys = phys_next;
-    const int tn = t + kWarps;
-    if (tn < tile_end) phys_next = __ldg(table + (tn * TILE) / BS);
-    const int token0 = t * TILE;
-    if (phys < 0 || phys >= a.num_blocks) {
-      if (lane == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
-      continue;
-    }
+  // rows of tile tt of block ph into k / v (zeros past the context or for a bad block)
+  auto issue = [&](int tt, int ph, uint4* k, uint4* v) {
+    const int token0 = tt * TILE;
+    const bool ok = ph >= 0 && ph < a.num_blocks;
     const size_t base =
-        ((size_t)phys * BS + (token0 % BS)) * row_stride + (size_t)h * D + ci * VEC;
-
-    uint4 kr[RG], vr[RG];
+        ((size_t)(ok ? ph : 0) * BS + (token0 % BS)) * row_stride + (size_t)h * D + ci * VEC;
 #pragma unroll
     for (int r = 0; r < RG; ++r) {
       const int row = r * RPI + rs;
-      if (token0 + row < tok_end) {
-        kr[r] = ld_stream16(kc + base + row * row_stride);
-        vr[r] = ld_stream16(vc + base + row * row_stride);
+      if (ok && token0 + row < tok_end) {
+        k[r] = ld_stream16(kc + base + row * row_stride);
+        v[r] = ld_stream16(vc + base + row * row_stride);
       } else {
-        kr[r] = make_uint4(0, 0, 0, 0);
-        vr[r] = make_uint4(0, 0, 0, 0);
+        k[r] = make_uint4(0, 0, 0, 0);
+        v[r] = make_uint4(0, 0, 0, 0);
       }
     }
-
+  };
+  // scores, online softmax and P.V of tile tt
+  auto consume = [&](int tt, const uint4* kr, const uint4* vr) {
+    const int token0 = tt * TILE;
     // scores of the lane's RG rows, reduced over the row's LPR lanes
     float s[RG][GC];
 #pragma unroll
@@ -224,6 +221,46 @@ decode_simt_kernel(const DecodeArgs a) {
         }
       }
     }
+  };
+  auto block_of = [&](int tt) { return __ldg(table + (tt * TILE) / BS); };
+  auto bad_block = [&](int ph) {
+    if (ph < 0 || ph >= a.num_blocks) {
+      if (lane == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+      return true;
+    }
+    return false;
+  };
+
+  int t = tile_begin + warp;
+  if constexpr (PF) {
+    // Loads of the warp's next tile are issued before this tile is computed, so
+    // each warp always has a tile's K and V in flight (block ids two tiles ahead).
+    uint4 kr[RG], vr[RG];
+    int phys = t < tile_end ? block_of(t) : -1;
+    int phys_n = t + kWarps < tile_end ? block_of(t + kWarps) : -1;
+    if (t < tile_end) issue(t, phys, kr, vr);
+    for (; t < tile_end; t += kWarps) {
+      const int tn = t + kWarps;
+      const int ph = phys;
+      uint4 kn[RG], vn[RG];
+      if (tn < tile_end) issue(tn, phys_n, kn, vn);
+      phys = phys_n;
+      phys_n = tn + kWarps < tile_end ? block_of(tn + kWarps) : -1;
+      if (!bad_block(ph)) consume(t, kr, vr);
+#pragma unroll
+      for (int r = 0; r < RG; ++r) { kr[r] = kn[r]; vr[r] = vn[r]; }
+    }
+  } else {
+    int phys_next = t < tile_end ? block_of(t) : 0;
+    for (; t < tile_end; t += kWarps) {
+      const int phys = phys_next;
+      const int tn = t + kWarps;
+      if (tn < tile_end) phys_next = block_of(tn);
+      if (bad_block(phys)) continue;
+      uint4 kr[RG], vr[RG];
+      issue(t, phys, kr, vr);
+      consume(t, kr, vr);
+    }
   }
 
   // combine the RPI row slots of the warp (same vector index, different rows)
@@ -274,12 +311,26 @@ decode_simt_kernel(const DecodeArgs a) {
   }
 }
 
+// Prefetching the next tile (PF) pays where a warp's tile carries few bytes
+// (FP8 pools: half the bytes of a 16-bit tile per load); PA_SIMT_PREFETCH=0/1
+// overrides the choice, for measurements.
+int prefetch_override() {
+  const char* s = std::getenv("PA_SIMT_PREFETCH");
+  if (!s || !*s) return -1;
+  return s[0] == '1' ? 1 : 0;
+}
+
 template <typename TQ, typename TC, int D, int BS, int GC>
 int launch_t(const DecodeArgs& a, cudaStream_t stream) {
   const int chunks = (a.Hq / a.Hkv) / GC;
   dim3 grid((unsigned)(a.P * chunks), (unsigned)a.Hkv, (unsigned)a.B);
-  const cudaError_t e = launch_k(decode_simt_kernel<TQ, TC, D, BS, GC>, grid, dim3(kWarps * 32),
-                                 0, stream, a);
+  const int ov = prefetch_override();
+  const bool pf = ov >= 0 ? ov == 1 : sizeof(TC) == 1;
+  const cudaError_t e =
+      pf ? launch_k(decode_simt_kernel<TQ, TC, D, BS, GC, true>, grid, dim3(kWarps * 32), 0,
+                    stream, a)
+         : launch_k(decode_simt_kernel<TQ, TC, D, BS, GC, false>, grid, dim3(kWarps * 32), 0,
+                    stream, a);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

@@ -9,7 +9,6 @@
 // FMAs per byte of K/V at G = 8, close to the FP32 pipe's limit at HBM speed;
 // on tcgen05 it is a few MMAs per tile.
 //
-// Work unit = (sequence, partition of the context, group of HG KV heads).
 // Tile = 128 rows of K (or V): HG heads x Rt = 128 / HG tokens, taken from
 // whole physical blocks. A 5-D TMA tensor map views the pool as
 // [num_blocks][2 d-halves][Hkv][block_size][64 d] (strides of the real
@@ -18,6 +17,19 @@
 // canonical 128-byte-swizzled layout the MMA reads (rows = (head, token),
 // 128 B each; the two d-halves 16 KB apart). Bigger boxes matter: streaming
 // the same bytes as 2-4 KB per-head boxes is limited by TMA issue, not HBM.
+//
+// Work split: the tiles of all (sequence b, group h of HG KV heads) pairs,
+// in (b, h, tile) order, form one list of T tiles, and CTA c takes the tiles
+// [floor(c T / grid), floor((c + 1) T / grid)): every CTA streams the same
+// number of tiles (+-1), whatever the mix of context lengths, so no CTA
+// finishes a long sequence alone at the end. A CTA's share is a run of units:
+// whole pairs in the middle, and at each end possibly a piece of a pair that
+// continues in the neighbouring CTA. A whole pair is written to the output
+// directly. A piece is written as (reference max, exp-sum, unnormalised
+// output) into its CTA's piece slot, then takes a ticket on its pair; the
+// piece that finishes last reads every piece of the pair back (from L2) and
+// merges them: M = max m_p, L = sum l_p 2^(m_p - M), o = sum 2^(m_p - M) o_p / L.
+// No CTA waits for another, and no separate merge launch is needed.
 //
 // Per tile (swap-AB, rows of the tile on the MMA's M = 128):
 //   scores  S^T[128 x HG*G]   = K_tile . Q_grp^T         (all query heads of the group)
@@ -33,7 +45,7 @@
 // columns are read, scaled and written back. Exact in real arithmetic: O and
 // l always share the same reference.
 //
-// CTA = 10 warps, persistent over its list of units:
+// CTA = 10 warps, persistent over its share:
 //   warps 0-7  two softmax groups; group w takes tiles t with t % 2 == w, so
 //              every SM sub-partition runs two independent softmax warps; at
 //              the end of a unit the group that did not take its last tile
@@ -46,10 +58,12 @@
 //   warp 8     TMA producer (one lane): Q of the unit, K and V tiles through a
 //              ring of 32 KB stages;
 //   warp 9     MMA issuer (one lane): S(t), then O(t-1).
-// Every pipeline wait is bounded (1 s); a wait that gives up sets the
-// PA_DEV_TIMEOUT bit, raises a CTA-wide abort flag, and all roles leave their
-// loops (the softmax warps of a group only together, at a named-barrier vote),
-// wait for their own asynchronous work, free tensor memory and return.
+// Every pipeline wait is bounded (DecodeArgs::wait_ns, 1 s unless a caller's
+// test shortens it); a wait that gives up sets the PA_DEV_TIMEOUT bit, raises
+// a CTA-wide abort flag, and all roles leave their loops (the softmax warps
+// of a group only together, at a named-barrier vote), wait for their own
+// asynchronous work (those waits keep the full 1 s bound, so no copy or MMA is
+// left in flight), free tensor memory and return.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
@@ -70,10 +84,11 @@ constexpr int kStageBytes = 2 * kHalf;          // one K or V tile: 32 KB
 constexpr int kHG = 4;                          // KV heads per unit
 constexpr int kRt = kRows / kHG;                // tokens per head per tile (32)
 constexpr int kThreads = 320;
-constexpr int kMaxUnits = 320;                  // work units one CTA can hold in its list
-constexpr int kScanChunk = 1024;                // sequences scanned per pass (stage 0 as scratch)
+constexpr int kScanChunk = 1024;                // sequences per pass of the first prologue scan
 constexpr float kRescaleLog2 = 64.f;            // lazy rescale threshold (log2 units): p <= 2^64,
                                                 // far from fp32 overflow in l and O
+constexpr int kEpochShift = 24;                 // ticket word: epoch << 24 | pieces arrived
+constexpr unsigned long long kCountMask = (1ull << kEpochShift) - 1;
 
 template <int G> struct TcShape {
   static constexpr int NS = kHG * G;                         // N of the score MMA
@@ -95,9 +110,8 @@ template <int G> struct TcShape {
   static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
   static constexpr int OFF_MREF = OFF_REDL + 2 * 2 * 8 * GP * 4;  // [group][3][NS] references
   static constexpr int OFF_COEF = OFF_MREF + 2 * 3 * NS * 4;   // [group][2][NS] merge weights
-  static constexpr int OFF_REC = (OFF_COEF + 2 * 2 * NS * 4 + 15) / 16 * 16;
-  static constexpr int OFF_MISC = OFF_REC + kMaxUnits * 16;
-  static constexpr int BYTES = OFF_MISC + 32;
+  static constexpr int OFF_MISC = (OFF_COEF + 2 * 2 * NS * 4 + 15) / 16 * 16;
+  static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   static_assert(2 * NS + 4 * NO <= kTmemCols, "tensor memory columns");
@@ -113,180 +127,286 @@ template <int NST> struct Bars {
                        ODONE = XFREE + 2, DONE = ODONE + 2;
 };
 
-// ---------------------------------------------------------------- work units
-// A unit is (sequence b, partition j, group h of kHG KV heads). Units exist
-// only for partitions that hold tokens. Units are spread over the CTAs like
-// longest-first list scheduling: they are ranked by size class (16 classes of
-// tile count, whole partitions first), and rank r goes to round r / grid of a
-// zig-zag over the CTAs (even rounds CTA 0, 1, ..., odd rounds backwards), so
-// every CTA gets its big units first and the small ones even out the end.
-// Every CTA builds its own list at start, in shared memory, so the roles never
-// touch global memory to find their next unit.
-struct __align__(16) URec {
-  int b, hj, ctx, start;      // hj = KV-head group | partition << 16; start = first token of the pass
+// Shared words written by the prologue (OFF_MISC).
+struct Misc {
+  uint32_t tmem;        // tensor-memory base address
+  uint32_t abort_flag;
+  int32_t valid;        // this CTA's share holds tiles
+  int32_t b0, h0, k0;   // first unit: sequence, KV-head group, first tile in the pair
+  int32_t found;        // prologue scan: the first unit has been located
+  int32_t last[2];      // per softmax group: this piece was the last of its pair
+  int32_t pad;
+  long long r0, r1;     // the share: global tiles [r0, r1)
+  long long T;          // tiles of all pairs
 };
+static_assert(sizeof(Misc) <= 64, "misc words");
+
+// ---------------------------------------------------------------- the work list
+// First global tile of CTA c: floor(c * T / grid), without 64-bit overflow.
+__device__ __forceinline__ long long share_begin(long long c, long long T, long long grid) {
+  return (T / grid) * c + ((T % grid) * c) / grid;
+}
+// The CTA whose share holds global tile x (the largest c with share_begin(c) <= x).
+__device__ __forceinline__ int share_owner(long long x, long long T, long long grid) {
+  return (int)(((x + 1) * grid - 1) / T);
+}
+
+// CTAs that hold a piece of the pair whose tiles are [pair0, pair0 + ntp):
+// the owners of its first and last tile and every CTA between them whose
+// share is not empty (shares are empty only when there are fewer tiles than
+// CTAs).
+__device__ __forceinline__ int pair_pieces(long long pair0, int ntp, long long T, int grid) {
+  const int c0 = share_owner(pair0, T, grid), c1 = share_owner(pair0 + ntp - 1, T, grid);
+  int n = 0;
+  for (int c = c0; c <= c1; ++c) n += share_begin(c + 1, T, grid) > share_begin(c, T, grid);
+  return n;
+}
+
+// Tiles of sequence b in this pass (0 for an empty pass or a bad length).
+template <int BS>
+__device__ __forceinline__ int seq_tiles(const DecodeArgs& a, int b, int& ctx, int& start) {
+  ctx = __ldg(a.context_lens + b);
+  start = a.start_blocks ? __ldg(a.start_blocks + b) * BS : 0;
+  if (ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len || start < 0 || start > ctx)
+    return 0;
+  return (ctx - start + kRt - 1) / kRt;
+}
+template <int BS>
+__device__ __forceinline__ bool seq_bad(const DecodeArgs& a, int ctx, int start) {
+  return ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len || start < 0 ||
+         start > ctx;
+}
+
+// A walk over this CTA's share, one unit (a pair, or a piece of one) at a time.
+struct Cursor {
+  int b, h;             // current pair
+  int k0, k1;           // tiles [k0, k1) of the pair in this unit
+  int ntp;              // tiles of the pair
+  int ctx, start;       // the sequence's length and the first token of the pass
+  long long g0;         // global index of the unit's first tile
+  long long left;       // tiles of the share after this unit
+  bool valid;
+};
+
+__device__ __forceinline__ void cur_fill(Cursor& c, int k0, long long budget) {
+  c.k0 = k0;
+  const long long n = min((long long)(c.ntp - k0), budget);
+  c.k1 = k0 + (int)n;
+  c.left = budget - n;
+}
+
+template <int BS>
+__device__ __forceinline__ void cur_init(const DecodeArgs& a, Cursor& c, const Misc* ms) {
+  c.valid = ms->valid != 0;
+  if (!c.valid) return;
+  c.b = ms->b0;
+  c.h = ms->h0;
+  c.ntp = seq_tiles<BS>(a, c.b, c.ctx, c.start);
+  c.g0 = ms->r0;
+  cur_fill(c, ms->k0, ms->r1 - ms->r0);
+}
+
+// Move to the next unit of the share (pairs with no tiles are skipped).
+template <int BS>
+__device__ __forceinline__ void cur_next(const DecodeArgs& a, int nhg, Cursor& c) {
+  if (!c.valid) return;
+  if (c.left <= 0) { c.valid = false; return; }
+  c.g0 += c.k1 - c.k0;
+  if (++c.h >= nhg) {
+    c.h = 0;
+    int n = 0;
+    do {
+      if (++c.b >= a.B) { c.valid = false; return; }
+      n = seq_tiles<BS>(a, c.b, c.ctx, c.start);
+    } while (n == 0);
+    c.ntp = n;
+  }
+  cur_fill(c, 0, c.left);
+}
 
 struct Unit {
-  int b, h, j, ctx, t0, t1, ntiles, nparts;
+  int b, h, ctx, t0, t1, ntiles, ntp;
+  bool whole;           // the unit is its whole pair
+  long long g0;         // global index of its first tile
+  long long pair0;      // global index of the pair's first tile
 };
 
-__device__ __forceinline__ Unit unit_from(const URec& r, int psize) {
+__device__ __forceinline__ Unit unit_of(const Cursor& c) {
   Unit x;
-  x.b = r.b; x.h = r.hj & 0xffff; x.j = r.hj >> 16; x.ctx = r.ctx;
-  x.t0 = r.start + x.j * psize;
-  x.t1 = min(r.ctx, x.t0 + psize);
-  x.ntiles = (x.t1 - x.t0 + kRt - 1) / kRt;
-  x.nparts = (r.ctx - r.start + psize - 1) / psize;
+  x.b = c.b; x.h = c.h; x.ctx = c.ctx; x.ntp = c.ntp;
+  x.t0 = c.start + c.k0 * kRt;
+  x.t1 = min(c.ctx, c.start + c.k1 * kRt);
+  x.ntiles = c.k1 - c.k0;
+  x.whole = c.k0 == 0 && c.k1 == c.ntp;
+  x.g0 = c.g0;
+  x.pair0 = c.g0 - c.k0;
   return x;
 }
 
-// Build this CTA's unit list (128 threads of warps 0-3, stage 0 as scratch).
-// Sequences with no tokens (or a context length the table cannot hold) get no
-// units; their output rows are zeroed here by CTA b % grid. Thread t of a pass
-// over kScanChunk sequences owns sequences t, t + 128, ... of the chunk, and
-// ranks within a class follow (pass, thread, sequence) order. Every loop here
-// is short and independent across threads: this runs before any K/V moves.
+// A tile position of the walk (for look-ahead of block ids).
+struct TilePos {
+  Cursor c;
+  int k;                // tile within the unit
+};
 template <int BS>
-__device__ void build_unit_list(const DecodeArgs& a, int nhg, uint8_t* scratch, URec* recs,
-                                int* my_units) {
-  constexpr int NC = 16;                                  // size classes
-  constexpr int PER = kScanChunk / 128;                   // sequences per thread and pass
+__device__ __forceinline__ void next_tile(const DecodeArgs& a, int nhg, TilePos& p) {
+  if (!p.c.valid) return;
+  if (++p.k >= p.c.k1 - p.c.k0) { p.k = 0; cur_next<BS>(a, nhg, p.c); }
+}
+
+// Prologue (the 128 threads of warps 0-3; stage 0 as scratch): count the
+// tiles of all pairs, zero the output rows of sequences with none (CTA
+// b % grid owns sequence b's rows), and find where this CTA's share starts.
+// Two short passes over context_lens, each a block-wide reduction or scan.
+template <int BS>
+__device__ void plan_share(const DecodeArgs& a, int nhg, uint8_t* scratch, Misc* ms) {
+  constexpr int PER = kScanChunk / 128;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
-  int* ctx_s = reinterpret_cast<int*>(scratch);           // [kScanChunk]
-  int* start_s = ctx_s + kScanChunk;                      // [kScanChunk] first token of the pass
-  int* next_s = start_s + kScanChunk;                     // [NC][128] next rank per class
-  int* hist = next_s + NC * 128;                          // [NC] units per class
-  int* cbase = hist + NC;                                 // [NC] first rank of each class
-  int* carry = cbase + NC;                                // [NC] ranks used by earlier passes
-  int* wsum = carry + NC;                                 // [4][NC]
-  int* nempty = wsum + 4 * NC;                            // sequences to zero in this pass
-  int* empty_s = nempty + 4;                              // [kScanChunk]
-  const int TP = (a.psize + kRt - 1) / kRt;               // tiles of a whole partition
-  // a context length (or pass start) the table cannot hold
-  auto bad = [&](int ctx, int start) {
-    return ctx < 0 || ctx > a.max_blocks * BS || ctx > a.max_context_len || start < 0 ||
-           start > ctx;
-  };
-  // partitions of the pass [start, ctx) and tiles of its last one; false: no units
-  auto shape = [&](int ctx, int start, int& np, int& tl) -> bool {
-    if (bad(ctx, start) || ctx == start) return false;
-    np = (ctx - start + a.psize - 1) / a.psize;
-    tl = (ctx - start - (np - 1) * a.psize + kRt - 1) / kRt;
-    return true;
-  };
-  auto start_of = [&](int b) { return a.start_blocks ? __ldg(a.start_blocks + b) * BS : 0; };
-  auto cls = [&](int nt) { return min(NC - 1, (nt * NC + TP - 1) / TP - 1); };
+  int* empty_s = reinterpret_cast<int*>(scratch);                   // [kScanChunk]
+  int* nempty = empty_s + kScanChunk;
+  long long* wsum = reinterpret_cast<long long*>(scratch + 4 * kScanChunk + 64);   // [4]
   auto bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
 
-  if (tid < NC) { hist[tid] = 0; carry[tid] = 0; }
-  bar();
-  for (int b = tid; b < a.B; b += 128) {
-    int np, tl;
-    if (!shape(__ldg(a.context_lens + b), start_of(b), np, tl)) continue;
-    if (np > 1) atomicAdd(&hist[NC - 1], (np - 1) * nhg);
-    atomicAdd(&hist[cls(tl)], nhg);
-  }
-  bar();
-  if (tid == 0) {
-    int r = 0;
-    for (int q = NC - 1; q >= 0; --q) { cbase[q] = r; r += hist[q]; }
-    const int full = r / grid, rem = r - full * grid;
-    const bool extra = rem > 0 && ((full & 1) ? cta >= grid - rem : cta < rem);
-    *my_units = min(full + (extra ? 1 : 0), kMaxUnits);
-  }
+  // pass 1: tiles of every sequence (per KV-head group); rows of empty ones
+  long long mine = 0;
   for (int b0 = 0; b0 < a.B; b0 += kScanChunk) {
-    const int n = min(kScanChunk, a.B - b0);
     if (tid == 0) *nempty = 0;
-#pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      const int i = e * 128 + tid;
-      ctx_s[i] = i < n ? __ldg(a.context_lens + b0 + i) : 0;
-      start_s[i] = i < n ? start_of(b0 + i) : 0;
-    }
-    bar();
-    // units per class of this thread's sequences, then a block-wide scan per class
-    int v[NC];
-#pragma unroll
-    for (int q = 0; q < NC; ++q) v[q] = 0;
-    for (int e = 0; e < PER; ++e) {
-      int np, tl;
-      const int i = e * 128 + tid;
-      if (!shape(ctx_s[i], start_s[i], np, tl)) {
-        if (i < n && ((b0 + i) % grid) == cta) empty_s[atomicAdd(nempty, 1)] = i;
-        continue;
-      }
-      const int c = cls(tl);
-#pragma unroll
-      for (int q = 0; q < NC; ++q) v[q] += (q == NC - 1 ? (np - 1) * nhg : 0) + (q == c ? nhg : 0);
-    }
-    int incl[NC];
-#pragma unroll
-    for (int q = 0; q < NC; ++q) {
-      incl[q] = v[q];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl[q], o);
-        if (lane >= o) incl[q] += t;
-      }
-      if (lane == 31) wsum[warp * NC + q] = incl[q];
-    }
     bar();
 #pragma unroll
-    for (int q = 0; q < NC; ++q) {
-      int wpre = 0;
-      for (int w = 0; w < warp; ++w) wpre += wsum[w * NC + q];
-      next_s[q * 128 + tid] = cbase[q] + carry[q] + wpre + incl[q] - v[q];
-    }
-    bar();
-    if (tid < NC) carry[tid] += wsum[tid] + wsum[NC + tid] + wsum[2 * NC + tid] + wsum[3 * NC + tid];
-    // walk the units in the order they were counted; keep the ones that land here
     for (int e = 0; e < PER; ++e) {
-      const int li = e * 128 + tid;
-      int np, tl;
-      if (!shape(ctx_s[li], start_s[li], np, tl)) continue;
-      if (np > 1) {
-        // whole partitions: consecutive ranks r0 .. r0 + nf - 1 (unit j * nhg + h);
-        // visit only the rounds they span and this CTA's slot in each
-        int* nx = next_s + (NC - 1) * 128 + tid;
-        const int r0 = *nx, nf = (np - 1) * nhg;
-        *nx = r0 + nf;
-        for (int round = r0 / grid; round * grid < r0 + nf && round < kMaxUnits; ++round) {
-          const int r = round * grid + ((round & 1) ? grid - 1 - cta : cta);
-          if (r < r0 || r >= r0 + nf) continue;
-          recs[round] = URec{b0 + li, ((r - r0) % nhg) | (((r - r0) / nhg) << 16), ctx_s[li],
-                             start_s[li]};
-        }
-      }
-      int* nx = next_s + cls(tl) * 128 + tid;               // the last partition
-      for (int h = 0; h < nhg; ++h) {
-        const int r = (*nx)++;
-        const int round = r / grid, pos = r - round * grid;
-        const int owner = (round & 1) ? grid - 1 - pos : pos;
-        if (owner == cta && round < kMaxUnits)
-          recs[round] = URec{b0 + li, h | ((np - 1) << 16), ctx_s[li], start_s[li]};
-      }
+      const int b = b0 + e * 128 + tid;
+      if (b >= a.B) break;
+      int ctx, st;
+      const int n = seq_tiles<BS>(a, b, ctx, st);
+      mine += n;
+      if (n == 0 && (b % grid) == cta) empty_s[atomicAdd(nempty, 1)] = b;
     }
-    // zero the output rows of empty / bad sequences this CTA owns
     bar();
     for (int k = 0; k < *nempty; ++k) {
-      const int li = empty_s[k], b = b0 + li;
-      if (bad(ctx_s[li], start_s[li]) && tid == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
+      const int b = empty_s[k];
+      int ctx, st;
+      (void)seq_tiles<BS>(a, b, ctx, st);
+      if (seq_bad<BS>(a, ctx, st) && tid == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
       if (!a.force_split)                 // the split-only pass leaves every row to the merge
         for (int i = tid; i < a.Hq * kD; i += 128)
           store_out(a.out, (size_t)b * a.Hq * kD + i, 0.f, a.out_dtype);
     }
     bar();
   }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  if (lane == 0) wsum[warp] = mine;
+  bar();
+  const long long T = (long long)nhg * (wsum[0] + wsum[1] + wsum[2] + wsum[3]);
+  const long long r0 = T > 0 ? share_begin(cta, T, grid) : 0;
+  const long long r1 = T > 0 ? share_begin(cta + 1, T, grid) : 0;
+  if (tid == 0) {
+    ms->T = T; ms->r0 = r0; ms->r1 = r1;
+    ms->valid = 0; ms->found = 0;
+  }
+  bar();
+  if (r0 >= r1) return;                   // an empty share (fewer tiles than CTAs)
+
+  // pass 2: the sequence whose tiles hold global tile r0 (a scan, 128 sequences a round)
+  long long carry = 0;                    // tiles per group of the sequences before this round
+  for (int b0 = 0; b0 < a.B; b0 += 128) {
+    const int b = b0 + tid;
+    int ctx = 0, st = 0;
+    const int n = b < a.B ? seq_tiles<BS>(a, b, ctx, st) : 0;
+    long long incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    bar();
+    long long wpre = 0;
+    for (int w = 0; w < warp; ++w) wpre += wsum[w];
+    const long long before = carry + wpre + incl - n;         // tiles per group before b
+    const long long lo = (long long)nhg * before;
+    if (n > 0 && lo <= r0 && r0 < lo + (long long)nhg * n) {
+      const long long d = r0 - lo;
+      ms->b0 = b;
+      ms->h0 = (int)(d / n);
+      ms->k0 = (int)(d % n);
+      ms->valid = 1;
+      ms->found = 1;
+    }
+    carry += wsum[0] + wsum[1] + wsum[2] + wsum[3];
+    bar();
+    if (ms->found) break;
+  }
 }
 
-// Advance (i, k) to the next tile of the CTA's unit list (i == nu: past the end).
-__device__ __forceinline__ void next_tile(const URec* recs, int nu, int psize, int& i, int& k) {
-  if (i >= nu) return;
-  const Unit x = unit_from(recs[i], psize);
-  if (++k >= x.ntiles) { k = 0; ++i; }
+// Take a ticket on a pair: true for the piece that arrives last. Lock-free
+// (every failed exchange means another piece succeeded), bounded anyway.
+__device__ __forceinline__ bool take_ticket(unsigned long long* word, unsigned long long epoch,
+                                            int npieces, uint32_t* err_flag) {
+  unsigned long long cur = atomicAdd(word, 0ull);
+#pragma unroll 1
+  for (int it = 0; it < (1 << 20); ++it) {
+    const unsigned long long cnt = (cur >> kEpochShift) == epoch ? (cur & kCountMask) : 0ull;
+    const unsigned long long want = (epoch << kEpochShift) | (cnt + 1);
+    const unsigned long long prev = atomicCAS(word, cur, want);
+    if (prev == cur) return (int)(cnt + 1) == npieces;
+    cur = prev;
+  }
+  flag_error(err_flag, PA_DEV_TIMEOUT);
+  return false;
 }
 
+// The last piece of a pair: merge every piece's (m, l, o) of the group's NS
+// query heads. 128 threads: thread `row` takes query head n = row / TPR and
+// DPT consecutive d. Writes the staging buffer (normalised output rows in the
+// output type, or, in the split-only pass, fp32 rows plus M and L).
+template <int G>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs& a, const Unit& x, int row,
+                                             uint8_t* stg, long long T, int grid, bool final_out,
+                                             size_t cas_row0) {
+  constexpr int NS = kHG * G, TPR = 128 / NS, DPT = kD / TPR;
+  const int n = row / TPR, d0 = (row % TPR) * DPT;
+  const int c0 = share_owner(x.pair0, T, grid);
+  const int c1 = share_owner(x.pair0 + x.ntp - 1, T, grid);
+  float M = -CUDART_INF_F, L = 0.f, o[DPT];
+#pragma unroll
+  for (int e = 0; e < DPT; ++e) o[e] = 0.f;
+#pragma unroll 1
+  for (int c = c0; c <= c1; ++c) {
+    const long long sb = share_begin(c, T, grid);
+    if (share_begin(c + 1, T, grid) <= sb) continue;       // an empty share: no piece
+    const size_t s = 2 * (size_t)c + (sb < x.pair0 ? 1 : 0);
+    const float m = __ldcg(a.sk_m + s * NS + n);
+    if (m == -CUDART_INF_F) continue;                       // no valid token in that piece
+    const float l = __ldcg(a.sk_l + s * NS + n);
+    const float Mn = fmaxf(M, m);
+    const float ca = exp2f(M - Mn), cb = exp2f(m - Mn);     // M = -inf gives ca = 0
+    L = fmaf(L, ca, l * cb);
+    const float4* src = reinterpret_cast<const float4*>(a.sk_acc + (s * NS + n) * kD + d0);
+#pragma unroll
+    for (int e = 0; e < DPT / 4; ++e) {
+      const float4 v = __ldcg(src + e);
+      o[4 * e + 0] = fmaf(o[4 * e + 0], ca, v.x * cb);
+      o[4 * e + 1] = fmaf(o[4 * e + 1], ca, v.y * cb);
+      o[4 * e + 2] = fmaf(o[4 * e + 2], ca, v.z * cb);
+      o[4 * e + 3] = fmaf(o[4 * e + 3], ca, v.w * cb);
+    }
+    M = Mn;
+  }
+  if (final_out) {
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+    for (int e = 0; e < DPT; ++e) store_out(stg, (size_t)n * kD + d0 + e, o[e] * inv, a.out_dtype);
+  } else {
+#pragma unroll
+    for (int e = 0; e < DPT; ++e) reinterpret_cast<float*>(stg)[n * kD + d0 + e] = o[e];
+    if (row % TPR == 0) {
+      a.ws_m[cas_row0 + n] = M;
+      a.ws_l[cas_row0 + n] = L;
+    }
+  }
+}
 
 template <int FMT, int BS, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -310,11 +430,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + S::OFF_BAR;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  const URec* recs = reinterpret_cast<const URec*>(smem + S::OFF_REC);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::OFF_MISC);
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + S::OFF_MISC + 4);
-  int* my_units_s = reinterpret_cast<int*>(smem + S::OFF_MISC + 8);
+  Misc* ms = reinterpret_cast<Misc*>(smem + S::OFF_MISC);
+  volatile uint32_t* abort_flag = &ms->abort_flag;
   const int nhg = a.Hkv / kHG;
+  const uint64_t wait_ns = a.wait_ns;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
@@ -337,31 +456,32 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     mbar_init(bar(Bx::ODONE), 128);
     mbar_init(bar(Bx::ODONE + 1), 128);
     mbar_init(bar(Bx::DONE), 1);
-    *abort_flag = 0u;
+    ms->abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 8) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_addr(tmem_slot)),
+                     smem_addr(&ms->tmem)),
                  "r"(S::kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   pdl_wait();                            // global memory from here on
   if (warp < 4) {
-    build_unit_list<BS>(a, nhg, smem, const_cast<URec*>(recs), my_units_s);
+    plan_share<BS>(a, nhg, smem, ms);
     fence_proxy_async();                 // stage 0 served as scratch; TMA writes it next
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = ms->tmem;
   const uint32_t tmem_s = tmem;                 // S buffers: [0, NS) and [NS, 2NS)
   // O accumulators from column 2NS: [unit parity][group], NO columns each, so the
   // next unit accumulates while the previous one is merged
   const uint32_t tmem_o = tmem + 2 * NS;
   auto obuf = [&](int ui, int g) { return tmem_o + (uint32_t)((2 * (ui & 1) + g) * NO); };
-  const int nu = *my_units_s;
+  const long long T = ms->T, r0 = ms->r0;
+  const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
   auto give_up = [&]() {
     *abort_flag = 1u;
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
@@ -378,19 +498,28 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     if (lane == 0) {
       int tc = 0, issued = 0;
       int phys_next[NQ];
-      auto load_ids = [&](int i, int k, int* ph) {
-        const Unit x = unit_from(recs[i], a.psize);
+      // block ids of the tile at p (-1 past the share's end)
+      auto load_ids = [&](const TilePos& p, int* ph) {
+        if (!p.c.valid) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) ph[q] = -1;
+          return;
+        }
+        const Unit x = unit_of(p.c);
         int ts, te, nql;
-        tile_span(x, k, ts, te, nql);
+        tile_span(x, p.k, ts, te, nql);
         const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) ph[q] = q < nql ? __ldg(table + (ts + q * RB) / BS) : -1;
       };
-      if (nu > 0) load_ids(0, 0, phys_next);
-      for (int i = 0; i < nu; ++i) {
-        const Unit x = unit_from(recs[i], a.psize);
+      Cursor cur;
+      cur_init<BS>(a, cur, ms);
+      TilePos ahead{cur, 0};
+      load_ids(ahead, phys_next);
+      for (int i = 0; cur.valid; ++i, cur_next<BS>(a, nhg, cur)) {
+        const Unit x = unit_of(cur);
         const int qi = i & 1;
-        if (!mbar_wait(bar(Bx::QEMPTY + qi), ((i >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+        if (!mbar_wait(bar(Bx::QEMPTY + qi), ((i >> 1) & 1) ^ 1, abort_flag, wait_ns)) { give_up(); goto prod_done; }
         mbar_expect_tx(bar(Bx::QFULL + qi), 2u * NS * 128u);
         for (int hh = 0; hh < 2; ++hh)
           tma_load_2d(sbase + S::OFF_Q + qi * S::kQBytes + hh * (NS * 128), &tmQ, hh * 64,
@@ -405,19 +534,19 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             phys[q] = phys_next[q];
             if (phys[q] >= 0 && phys[q] < a.num_blocks) bytes += 2u * RB * kHG * 128u;
           }
-          if (k + 1 < x.ntiles) load_ids(i, k + 1, phys_next);
-          else if (i + 1 < nu) load_ids(i + 1, 0, phys_next);
+          next_tile<BS>(a, nhg, ahead);
+          load_ids(ahead, phys_next);
           for (int kv = 0; kv < 2; ++kv) {
             const int seq = 2 * tc + kv, s = seq % NST;
-            if (!mbar_wait(bar(Bx::EMPTY + s), ((seq / NST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+            if (!mbar_wait(bar(Bx::EMPTY + s), ((seq / NST) & 1) ^ 1, abort_flag, wait_ns)) { give_up(); goto prod_done; }
             mbar_expect_tx(bar(Bx::FULL + s), bytes);
             const uint32_t dst = sbase + s * kStageBytes;
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
               if (phys[q] < 0 || phys[q] >= a.num_blocks) continue;
-              const int r0 = (ts + q * RB) % BS;
+              const int rr0 = (ts + q * RB) % BS;
               for (int hh = 0; hh < 2; ++hh)
-                tma_load_5d(dst + hh * kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, r0,
+                tma_load_5d(dst + hh * kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, rr0,
                             x.h * kHG, hh, phys[q], bar(Bx::FULL + s));
             }
             ++issued;
@@ -441,13 +570,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       // output product of tile tt (unit ui, tile kk of the unit, nql boxes with tokens)
       auto issue_pv = [&](int tt, int ui, int kk, int nql) -> bool {
         const int pb = tt & 1;
-        if (!mbar_wait(bar(Bx::PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(Bx::PREADY + pb), (tt >> 1) & 1, abort_flag, wait_ns)) return false;
         const bool first = kk <= 1;                   // this group's first tile of the unit
         // the unit's accumulators were last used by unit ui - 2: wait for its merge
-        if (first && ui >= 2 && !mbar_wait(bar(Bx::ODONE + (ui & 1)), ((ui - 2) >> 1) & 1, abort_flag))
+        if (first && ui >= 2 &&
+            !mbar_wait(bar(Bx::ODONE + (ui & 1)), ((ui - 2) >> 1) & 1, abort_flag, wait_ns))
           return false;
         const int seq = 2 * tt + 1, s = seq % NST;
-        if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) return false;
         tc_fence_after();
         const uint32_t vst = sbase + s * kStageBytes;
         const uint32_t pst = sbase + S::OFF_P + pb * S::kPBytes;
@@ -472,10 +602,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       };
       int pui = 0, pkk = 0, pnql = 0;                // the tile waiting for its output product
       bool pending = false;                          // tile tc - 1 still needs its output product
-      for (int i = 0; i < nu && ok; ++i) {
-        const Unit x = unit_from(recs[i], a.psize);
+      Cursor cur;
+      cur_init<BS>(a, cur, ms);
+      for (int i = 0; cur.valid && ok; ++i, cur_next<BS>(a, nhg, cur)) {
+        const Unit x = unit_of(cur);
         const int qi = i & 1;
-        if (!mbar_wait(bar(Bx::QFULL + qi), (i >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(Bx::QFULL + qi), (i >> 1) & 1, abort_flag, wait_ns)) { ok = false; break; }
         const uint32_t qst = sbase + S::OFF_Q + qi * S::kQBytes;
         for (int k = 0; k < x.ntiles; ++k) {
           int ts, te, nql;
@@ -496,12 +628,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
               if (mbar_test(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1) &&
                   mbar_test(bar(Bx::FULL + s), (seq / NST) & 1))
                 break;
-              if (*abort_flag || globaltimer() - t0 > kWaitNs) { ok = false; break; }
+              if (*abort_flag || globaltimer() - t0 > wait_ns) { ok = false; break; }
             }
             if (!ok) break;
           }
-          if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag, wait_ns)) { ok = false; break; }
+          if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + s * kStageBytes;
 #pragma unroll
@@ -555,20 +687,23 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     // the phase before t's (the group has seen S of a tile >= t, and the
     // issuer puts S(t) after O(t - 2) on the same in-order tensor pipe).
     auto wait_pv = [&](int t) {
-      if (!mbar_wait(bar(Bx::OFULL + grp), (t >> 1) & 1, abort_flag)) failed = true;
+      if (!mbar_wait(bar(Bx::OFULL + grp), (t >> 1) & 1, abort_flag, wait_ns)) failed = true;
     };
-    auto row_id = [&](int i, int k) -> int {
-      const Unit x = unit_from(recs[i], a.psize);
+    auto row_id = [&](const TilePos& p) -> int {
+      if (!p.c.valid) return -1;
+      const Unit x = unit_of(p.c);
       int ts, te, nql;
-      tile_span(x, k, ts, te, nql);
+      tile_span(x, p.k, ts, te, nql);
       return rq < nql ? __ldg(a.block_tables + (size_t)x.b * a.max_blocks + (ts + rq * RB) / BS) : -1;
     };
-    int ni = 0, nk = 0;
-    if (nu > 0 && grp == 1) next_tile(recs, nu, a.psize, ni, nk);       // group 1 starts at tile 1
-    int phys_next = (nu > 0 && ni < nu) ? row_id(ni, nk) : -1;
+    Cursor cur;
+    cur_init<BS>(a, cur, ms);
+    TilePos ahead{cur, 0};
+    if (grp == 1) next_tile<BS>(a, nhg, ahead);              // group 1 starts at tile 1
+    int phys_next = row_id(ahead);
     bool stop = false;
-    for (int i = 0; i < nu && !stop; ++i) {
-      const Unit x = unit_from(recs[i], a.psize);
+    for (int i = 0; cur.valid && !stop; ++i, cur_next<BS>(a, nhg, cur)) {
+      const Unit x = unit_of(cur);
       float mo[G], l[G];                           // this row's head: reference max, exp-sum
 #pragma unroll
       for (int g = 0; g < G; ++g) { mo[g] = -CUDART_INF_F; l[g] = 0.f; }
@@ -579,16 +714,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         tile_span(x, k, ts, te, nql);
         const bool in_range = rq < nql;
         const int phys = phys_next;
-        next_tile(recs, nu, a.psize, ni, nk);                 // two tiles ahead: the next own tile
-        next_tile(recs, nu, a.psize, ni, nk);
-        if (ni < nu) phys_next = row_id(ni, nk);
+        next_tile<BS>(a, nhg, ahead);                         // two tiles ahead: the next own tile
+        next_tile<BS>(a, nhg, ahead);
+        phys_next = row_id(ahead);
         const bool blk_ok = phys >= 0 && phys < a.num_blocks;
         const bool valid = in_range && blk_ok && ts + tt_row < te;
         if (in_range && !blk_ok && rr == 0 && rh == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
         const bool first = my_last < 0;
 
         const int par = (tc >> 1) & 1;                        // use count of this group's buffers
-        if (!mbar_wait(bar(Bx::SFULL + grp), par, abort_flag)) failed = true;
+        if (!mbar_wait(bar(Bx::SFULL + grp), par, abort_flag, wait_ns)) failed = true;
         tc_fence_after();
         constexpr int SVN = ((32 / RB) * G + 15) / 16 * 16;  // S columns this warp loads
         float sv[SVN];
@@ -674,11 +809,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         if (in_range && !valid) {
           // this V row enters the output product with weight 0: it must hold finite values
           const int seq = 2 * tc + 1, sv_ = seq % NST;
-          if (!mbar_wait(bar(Bx::FULL + sv_), (seq / NST) & 1, abort_flag)) failed = true;
-          uint4* r0 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + row * 128);
-          uint4* r1 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + kHalf + row * 128);
+          if (!mbar_wait(bar(Bx::FULL + sv_), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
+          uint4* z0 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + row * 128);
+          uint4* z1 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + kHalf + row * 128);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) { r0[c] = make_uint4(0, 0, 0, 0); r1[c] = make_uint4(0, 0, 0, 0); }
+          for (int c = 0; c < 8; ++c) { z0[c] = make_uint4(0, 0, 0, 0); z1[c] = make_uint4(0, 0, 0, 0); }
         }
         fence_proxy_async();
         mbar_arrive(bar(Bx::PREADY + grp));
@@ -702,7 +837,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       const int last_grp = (tc - 1) & 1;                    // group of the unit's last tile
       if (grp != last_grp) {
         if (my_last >= 0) wait_pv(my_last);
-        if (!mbar_wait(bar(Bx::XFREE + xi), xpar ^ 1, abort_flag)) failed = true;
+        if (!mbar_wait(bar(Bx::XFREE + xi), xpar ^ 1, abort_flag, wait_ns)) failed = true;
         if (row < NS) {
           float L = 0.f;
 #pragma unroll
@@ -718,7 +853,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         mbar_arrive(bar(Bx::XFULL + xi));
       } else {
         wait_pv(my_last);
-        if (!mbar_wait(bar(Bx::XFULL + xi), xpar, abort_flag)) failed = true;
+        if (!mbar_wait(bar(Bx::XFULL + xi), xpar, abort_flag, wait_ns)) failed = true;
         if (rq == 0 && rr == 0) {
 #pragma unroll
           for (int g = 0; g < G; ++g) mown[rh * G + g] = mo[g];
@@ -726,15 +861,19 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         if (row == 0) bulk_wait_read();           // the group's previous rows have left staging
         wg_sync(grp);
         const bool has_p = xflag[xi] != 0;
-        // merged rows go to shared memory first, then out in one bulk copy per head:
-        // the unit's NS output rows are contiguous in out [B, Hq, D] and in the
-        // workspace [B, P, Hq, D]
-        const bool final_out = x.nparts == 1 && !a.force_split;
+        // Where the unit's rows go: a whole pair to the output (normalised), or,
+        // in the split-only pass, to its workspace slot; a piece to its CTA's
+        // piece slot. The NS rows are contiguous in each.
+        const bool piece = !x.whole;
+        const bool final_out = !piece && !a.force_split;
         const int osz = final_out && a.out_dtype != PA_F32 ? 2 : 4;
         uint8_t* stg = smem + S::OFF_STG + grp * S::kStgBytes;
-        const size_t row0 = final_out ? (size_t)x.b * a.Hq + (size_t)x.h * NS
-                                      : ((size_t)x.b * a.P + a.slot_base + x.j) * a.Hq +
-                                            (size_t)x.h * NS;
+        const size_t out_row0 = (size_t)x.b * a.Hq + (size_t)x.h * NS;
+        const size_t cas_row0 = ((size_t)x.b * a.P + a.slot_base) * a.Hq + (size_t)x.h * NS;
+        const size_t piece_row0 = (2 * (size_t)cta + (x.g0 == r0 ? 0 : 1)) * NS;
+        float* wm = piece ? a.sk_m : a.ws_m;
+        float* wl = piece ? a.sk_l : a.ws_l;
+        const size_t wrow0 = piece ? piece_row0 : cas_row0;
         float* coef = reinterpret_cast<float*>(smem + S::OFF_COEF) + grp * 2 * NS;
         if (row < NS) {
           // query head n: combined max and exp-sum, and the weights of the two
@@ -757,8 +896,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             c *= inv;
             cp *= inv;
           } else {
-            a.ws_m[row0 + n] = M;
-            a.ws_l[row0 + n] = Lt;
+            wm[wrow0 + n] = M;
+            wl[wrow0 + n] = Lt;
           }
           coef[n] = c;
           coef[NS + n] = cp;
@@ -792,13 +931,46 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         mbar_arrive(bar(Bx::ODONE + (i & 1)));
         fence_proxy_async();                      // staging writes -> the bulk copy's proxy
         wg_sync(grp);                             // (mown is rewritten at the next merge, too)
+        const uint32_t hb = (uint32_t)(G * kD * osz);
         if (row == 0) {
-          uint8_t* dst = final_out ? static_cast<uint8_t*>(a.out) + row0 * kD * osz
-                                   : reinterpret_cast<uint8_t*>(a.ws_acc) + row0 * kD * 4;
-          const uint32_t hb = (uint32_t)(G * kD * osz);
+          uint8_t* dst = final_out ? static_cast<uint8_t*>(a.out) + out_row0 * kD * osz
+                       : piece     ? reinterpret_cast<uint8_t*>(a.sk_acc) + piece_row0 * kD * 4
+                                   : reinterpret_cast<uint8_t*>(a.ws_acc) + cas_row0 * kD * 4;
 #pragma unroll
           for (int h = 0; h < kHG; ++h) bulk_store(dst + h * hb, smem_addr(stg) + h * hb, hb);
           bulk_commit();
+        }
+        if (piece) {
+          // publish the piece (its m, l stores and its bulk copy), then take a
+          // ticket; the last piece of the pair merges all of them
+          __threadfence();
+          wg_sync(grp);
+          if (row == 0) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            __threadfence();
+            const int np = pair_pieces(x.pair0, x.ntp, T, grid);
+            ms->last[grp] =
+                take_ticket(a.tickets + (size_t)x.b * nhg + x.h, a.epoch, np, a.err_flag) ? 1 : 0;
+          }
+          wg_sync(grp);
+          if (ms->last[grp]) {
+            __threadfence();
+            merge_pieces<G>(a, x, row, stg, T, grid, !a.force_split, cas_row0);
+            fence_proxy_async();
+            wg_sync(grp);
+            if (row == 0) {
+              const int osz2 = a.force_split || a.out_dtype == PA_F32 ? 4 : 2;
+              const uint32_t hb2 = (uint32_t)(G * kD * osz2);
+              uint8_t* dst = a.force_split ? reinterpret_cast<uint8_t*>(a.ws_acc) + cas_row0 * kD * 4
+                                           : static_cast<uint8_t*>(a.out) + out_row0 * kD * osz2;
+#pragma unroll
+              for (int h = 0; h < kHG; ++h) bulk_store(dst + h * hb2, smem_addr(stg) + h * hb2, hb2);
+              bulk_commit();
+              // every piece has arrived: leave the ticket at zero for this epoch
+              atomicExch(a.tickets + (size_t)x.b * nhg + x.h, a.epoch << kEpochShift);
+            }
+          }
         }
       }
     }
@@ -861,12 +1033,10 @@ bool make_maps(const DecodeArgs& a, int dtype, int G, CUtensorMap* k, CUtensorMa
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return kSMs;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-    return kSMs;
-  return n;
+// Upper bound of the tiles of a call (every sequence at max_context_len).
+long long max_tiles(const DecodeArgs& a) {
+  const long long per = ((long long)(a.max_context_len > 0 ? a.max_context_len : 1) + kRt - 1) / kRt;
+  return (long long)a.B * (a.Hkv / kHG) * per;
 }
 
 template <int FMT, int BS, int G>
@@ -881,12 +1051,10 @@ int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
       return PA_ERR_CUDA;
     attr = true;
   }
-  // Units that hold tokens number at most B * (Hkv / kHG) * P; a CTA's list holds kMaxUnits.
-  const long long units = (long long)a.B * (a.Hkv / kHG) * a.P;
-  if (units <= 0) return PA_OK;
-  long long grid = units < sm_count() ? units : sm_count();
-  if ((units + grid - 1) / grid > kMaxUnits) grid = (units + kMaxUnits - 1) / kMaxUnits;
-  if (grid > 0x7fffffffLL) return PA_ERR_UNSUPPORTED;
+  // one CTA per SM (at most one per tile): the workspace's piece slots are sized for that
+  const long long tiles = max_tiles(a);
+  const long long grid = tiles < sm_count_cached() ? tiles : sm_count_cached();
+  if (grid <= 0) return PA_OK;
   return launch_k(kern, dim3((unsigned)grid), dim3(kThreads), smem, stream, a, k, v, q) ==
                  cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -901,13 +1069,40 @@ int launch_tc_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
   return PA_ERR_UNSUPPORTED;
 }
 
+size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+
 }  // namespace
+
+bool tc_shape(int Hq, int Hkv, int D) {
+  if (D != kD || Hkv <= 0 || Hq % Hkv || Hkv % kHG) return false;
+  const int G = Hq / Hkv;
+  return G == 4 || G == 8;
+}
 
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs) {
   if (dtype != PA_F16 && dtype != PA_BF16) return false;
-  if (D != kD || (bs != 16 && bs != 32) || Hkv <= 0 || Hq % Hkv || Hkv % kHG) return false;
-  const int G = Hq / Hkv;
-  return G == 4 || G == 8;
+  return (bs == 16 || bs == 32) && tc_shape(Hq, Hkv, D);
+}
+
+// Piece slots for every CTA of the largest grid, then one ticket word per pair.
+size_t tc_workspace_bytes(int B, int Hq, int Hkv, int D) {
+  if (B <= 0 || !tc_shape(Hq, Hkv, D)) return 0;
+  const size_t ns = (size_t)kHG * (Hq / Hkv);
+  const size_t slots = 2 * (size_t)sm_count_cached();
+  return up256(slots * ns * kD * 4) + 2 * up256(slots * ns * 4) +
+         up256((size_t)B * (Hkv / kHG) * 8);
+}
+
+void tc_carve(DecodeArgs& a, char* base) {
+  const size_t ns = (size_t)kHG * (a.Hq / a.Hkv);
+  const size_t slots = 2 * (size_t)sm_count_cached();
+  a.sk_acc = reinterpret_cast<float*>(base);
+  base += up256(slots * ns * kD * 4);
+  a.sk_m = reinterpret_cast<float*>(base);
+  base += up256(slots * ns * 4);
+  a.sk_l = reinterpret_cast<float*>(base);
+  base += up256(slots * ns * 4);
+  a.tickets = reinterpret_cast<unsigned long long*>(base);
 }
 
 int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream) {

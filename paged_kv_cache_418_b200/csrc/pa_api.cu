@@ -1,6 +1,8 @@
 // pa_api.cu -- the extern "C" boundary of libpa.so: argument checks, launch
 // planning (split or not, which kernel), workspace carve-up, launches.
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -37,17 +39,6 @@ int max_prefix_slots(int max_shared_blocks, int block_size) {
   return (max_shared_blocks * block_size + kPrefixTile - 1) / kPrefixTile;
 }
 
-int sm_count_cached() {
-  static int n = 0;
-  if (n <= 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = kSMs;
-  }
-  return n;
-}
-
 // Kernel override for A/B measurements: PA_DECODE_KERNEL=simt|tc (unset = auto).
 int kernel_override() {
   const char* s = std::getenv("PA_DECODE_KERNEL");
@@ -57,7 +48,39 @@ int kernel_override() {
   return 0;
 }
 
+// Limit of every pipeline wait of the tensor-core kernels, in ns (1 s; the
+// environment variable PA_TC_WAIT_NS lowers it, for tests of the timeout path).
+unsigned long long tc_wait_ns() {
+  const char* s = std::getenv("PA_TC_WAIT_NS");
+  if (!s || !*s) return 1000000000ull;
+  char* end = nullptr;
+  const unsigned long long v = std::strtoull(s, &end, 10);
+  return (end && *end == 0 && v <= 1000000000ull) ? v : 1000000000ull;
+}
+
+// A number per call of the tensor-core path (40 bits; its tickets carry it).
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> n{
+      (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 2654435761ull};
+  return (n.fetch_add(1) + 1) & ((1ull << 40) - 1);
+}
+
 }  // namespace
+
+// SM count of the current device (148 on B200; also the fallback with no device).
+int sm_count_cached() {
+  static int n = 0;
+  if (n <= 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+      cudaGetLastError();
+      return kSMs;                       // not cached: a device may appear later
+    }
+    n = v;
+  }
+  return n;
+}
 
 DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max_ctx,
                        int partition_size) {
@@ -80,6 +103,12 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max
   const int ov = kernel_override();
   const bool tc = tc_supported(dtype, Hq, Hkv, D, bs);
   p.kernel = ov == 1 ? 1 : (ov == 2 ? (tc ? 2 : 1) : (tc ? 2 : 1));
+  if (p.kernel == 2) {
+    // the tensor-core kernel splits the work evenly over the SMs itself (pieces
+    // merged in the kernel): no fixed partitions, no merge launch
+    p.P = 1;
+    p.psize = ((mc + bs - 1) / bs) * bs;
+  }
   (void)B;
   return p;
 }
@@ -101,8 +130,10 @@ extern "C" {
 size_t pa_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len, int partition_size) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_context_len <= 0 || partition_size < 0)
     return 0;
+  // enough for either kernel: the CUDA-core split pass, or the tensor-core
+  // kernel's pieces and tickets (shapes it can take in a 16-bit type)
   DecodePlan p = plan_decode(PA_F32, B, Hq, Hkv, D, 16, max_context_len, partition_size);
-  return workspace_bytes_for(B, Hq, D, p.P);
+  return std::max(workspace_bytes_for(B, Hq, D, p.P), tc_workspace_bytes(B, Hq, Hkv, D));
 }
 
 const char* pa_status_string(int status) {
@@ -174,7 +205,15 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   a.max_context_len = max_context_len;
   a.P = p.P; a.psize = p.psize;
   a.err_flag = err_flag;
-  if (p.P > 1) {
+  const bool tc_path = kv_dtype != PA_FP8_E4M3 && p.kernel == 2;
+  if (tc_path) {
+    const size_t need = tc_workspace_bytes(B, Hq, Hkv, D);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return PA_ERR_WORKSPACE;
+    tc_carve(a, static_cast<char*>(workspace));
+    a.epoch = next_epoch();
+    a.wait_ns = tc_wait_ns();
+  } else if (p.P > 1) {
     const size_t need = workspace_bytes_for(B, Hq, D, p.P);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
       return PA_ERR_WORKSPACE;
@@ -247,7 +286,10 @@ size_t pa_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int max_co
     return 0;
   if (max_shared_blocks == 0) return pa_workspace_size(B, Hq, Hkv, D, max_context_len, partition_size);
   DecodePlan p = plan_decode(PA_F32, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
-  return workspace_bytes_for(B, Hq, D, max_prefix_slots(max_shared_blocks, block_size) + p.P);
+  // partial slots of the prefix and suffix passes, then the tensor-core suffix
+  // pass's pieces and tickets
+  return workspace_bytes_for(B, Hq, D, max_prefix_slots(max_shared_blocks, block_size) + p.P) +
+         tc_workspace_bytes(B, Hq, Hkv, D);
 }
 
 int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const void* key_cache,
@@ -306,7 +348,8 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   a.start_blocks = shared_blocks;        // the suffix pass starts after the shared blocks
   a.slot_base = parts;                   // slots [0, parts) hold the prefix partials
   a.force_split = 1;
-  const size_t need = workspace_bytes_for(B, Hq, D, a.P);
+  const size_t part_bytes = workspace_bytes_for(B, Hq, D, a.P);
+  const size_t need = part_bytes + (p.kernel == 2 ? tc_workspace_bytes(B, Hq, Hkv, D) : 0);
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PA_ERR_WORKSPACE;
   const size_t rows = (size_t)B * Hq * a.P;
@@ -315,6 +358,11 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   a.ws_acc = reinterpret_cast<float*>(w);
   a.ws_m = reinterpret_cast<float*>(w + up(rows * D * 4));
   a.ws_l = reinterpret_cast<float*>(w + up(rows * D * 4) + up(rows * 4));
+  if (p.kernel == 2) {
+    tc_carve(a, w + part_bytes);
+    a.epoch = next_epoch();
+    a.wait_ns = tc_wait_ns();
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, st) : launch_decode_simt(a, dtype, st);
   if (rc == PA_OK)

@@ -36,6 +36,18 @@ struct DecodeArgs {
   const int32_t* start_blocks;
   int slot_base;
   int force_split;
+  // Tensor-core path (work split evenly over the CTAs): a (sequence, group of
+  // 4 KV heads) whose tiles straddle CTAs is written as pieces, at most two
+  // per CTA (slot 2 * cta for its first unit, 2 * cta + 1 for its last), and
+  // the last piece to finish, chosen by a ticket per (sequence, group), merges
+  // them. A ticket word is (epoch << 24 | count): a word from another call (or
+  // uninitialised memory) has another epoch and counts as zero.
+  float* sk_acc;                  // [2 * grid][4 * G][D] unnormalised piece outputs
+  float* sk_m;                    // [2 * grid][4 * G] piece reference max (log2 domain)
+  float* sk_l;                    // [2 * grid][4 * G] piece exp-sums
+  unsigned long long* tickets;    // [B * (Hkv / 4)]
+  unsigned long long epoch;       // this call's number (40 bits)
+  unsigned long long wait_ns;     // limit of every pipeline wait of the tensor-core kernel
 };
 
 // Shared-prefix decode: the prefix is cut into partitions of a multiple of
@@ -59,6 +71,12 @@ int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream);
 int launch_decode_simt_fp8(const DecodeArgs& a, int q_dtype, cudaStream_t stream);
 int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream);
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
+// Shapes the tensor-core path can take for some 16-bit element type and block size.
+bool tc_shape(int Hq, int Hkv, int D);
+// Scratch of the tensor-core path (pieces and tickets), and its carve-up.
+size_t tc_workspace_bytes(int B, int Hq, int Hkv, int D);
+void tc_carve(DecodeArgs& a, char* base);
+int sm_count_cached();
 int launch_merge(const DecodeArgs& a, cudaStream_t stream);
 bool prefix_tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 int prefix_chunks(int max_group_size, int G);

@@ -53,12 +53,19 @@ def test_workspace_and_plan():
     # short contexts: one pass, no workspace
     assert ops.pa_workspace_size(64, 32, 32, 128, 512, 0) == 0
     assert ops.pa_decode_plan(1, 64, 32, 32, 128, 16, 512)[1:] == (1, 512)
-    # long contexts: 512-token partitions; workspace = acc + m + l (fp32, 256 B aligned)
-    k, P, psize = ops.pa_decode_plan(2, 8, 64, 8, 128, 32, 32768, 512)
-    assert (P, psize) == (64, 512)
+    # long contexts on the CUDA-core kernel: 512-token partitions; workspace =
+    # acc + m + l (fp32, 256 B aligned)
+    k, P, psize = ops.pa_decode_plan(0, 8, 64, 8, 128, 32, 32768, 512)
+    assert (k, P, psize) == (1, 64, 512)
     rows = 8 * 64 * 64
     up = lambda x: (x + 255) // 256 * 256
     assert ops.pa_workspace_size(8, 64, 8, 128, 32768, 512) == up(rows * 128 * 4) + 2 * up(rows * 4)
+    # the tensor-core kernel splits the work over the SMs itself: no fixed partitions
+    assert ops.pa_decode_plan(2, 8, 64, 8, 128, 32, 32768, 512) == (2, 1, 32768)
+    # ... and needs its piece slots (2 per SM: 148 without a device) and tickets even
+    # for short contexts
+    assert ops.pa_workspace_size(8, 64, 8, 128, 100, 0) == \
+        up(296 * 32 * 128 * 4) + 2 * up(296 * 32 * 4) + up(8 * 2 * 8)
     assert ops.pa_workspace_size(64, 32, 32, 128, 2048, 0) > 0
     assert ops.pa_decode_plan(1, 64, 32, 32, 128, 16, 2048)[1:] == (4, 512)
     assert ops.pa_workspace_size(0, 32, 32, 128, 2048, 0) == 0
@@ -149,7 +156,9 @@ def test_shared_prefix_workspace_and_fp8_plan():
     n = ops.pa_shared_prefix_workspace_size(B, Hq, 8, D, 1547, 0, 16, 64)
     P = 1024 // 128 + 4
     rows = B * Hq * P
-    assert n == up(rows * D * 4) + 2 * up(rows * 4)
+    # + the tensor-core suffix pass's piece slots (2 per SM, 148 here) and tickets
+    tc = up(296 * 16 * D * 4) + 2 * up(296 * 16 * 4) + up(B * 2 * 8)
+    assert n == up(rows * D * 4) + 2 * up(rows * 4) + tc
     assert ops.pa_shared_prefix_workspace_size(B, Hq, 8, D, 1547, 0, 16, 0) == \
         ops.pa_workspace_size(B, Hq, 8, D, 1547, 0)
     # FP8 pools always plan the CUDA-core kernel

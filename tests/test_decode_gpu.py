@@ -245,3 +245,75 @@ def test_full_size_workload_sampled_parity(which, full_workloads):
     assert_attention_close(got, ref, w.dtype, w.name)
     # every output finite (NaN poison never leaks)
     assert torch.isfinite(out.float()).all()
+
+
+# -- the tensor-core kernel's even split of the work over the SMs -------------------
+def _tc_case(ctx, seed, Hq=64, Hkv=8, bs=16):
+    nb = sum((c + bs - 1) // bs for c in ctx) + 4
+    w = W.build_decode_case("even-split", W.BF16, B=len(ctx), Hq=Hq, Hkv=Hkv, D=128,
+                            block_size=bs, num_blocks=nb, context_lens=ctx, seed=seed,
+                            k_boost_frac=0.02)
+    assert ops.pa_decode_plan(w.kv_dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
+                              w.max_context_len)[0] == 2
+    return w
+
+
+def _decode_with(w, t, ws, out_dtype=torch.float32, mcl=None):
+    out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=out_dtype, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                  w.scale, mcl or w.max_context_len, 0, ws, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return out
+
+
+@pytest.mark.parametrize("ctx,G,mcl", [
+    ([5000, 37, 1, 800, 4096, 33, 64, 3000] + [17] * 20 + [2049, 700], 8, None),  # many pieces
+    ([9000, 12, 1], 4, None),                    # one sequence in pieces over ~70 CTAs
+    ([1, 1, 1], 8, 4096),                        # fewer tiles than CTAs: empty shares between
+    ([40, 1, 70], 4, 8192),                      # pieces with empty shares between them
+    ([300 + 37 * i for i in range(150)], 4, None),   # many whole sequences per CTA
+])
+def test_even_split_pieces_merge_to_the_oracle(ctx, G, mcl):
+    """Sequences cut into pieces across CTAs (the last piece merges them), whole
+    sequences in one CTA, CTAs with nothing to do; the workspace starts full of
+    random bytes (tickets of no earlier call), and a second call on the same
+    workspace gives the same bits."""
+    w = _tc_case(ctx, seed=len(ctx) * 31 + G, Hq=8 * G, Hkv=8)
+    t = device_inputs(w)
+    ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                             t["slot_mapping"])
+    ws = ops.workspace_for(t["q"], t["k_cache"], mcl or w.max_context_len)
+    ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda"))
+    out1 = _decode_with(w, t, ws, mcl=mcl)
+    out2 = _decode_with(w, t, ws, mcl=mcl)
+    ref, _, _ = oracle_step(w)
+    assert_attention_close(out1, ref, w.dtype, f"even split {len(ctx)} seqs")
+    assert torch.equal(out1, out2)
+    out3 = _decode_with(w, t, ws, out_dtype=torch.bfloat16, mcl=mcl)   # 16-bit output path
+    assert_attention_close(out3, ref, w.dtype, "bf16 out")
+
+
+def test_pipeline_wait_limit_runs_out_and_the_next_launch_is_correct(monkeypatch):
+    """With the tensor-core kernel's pipeline-wait limit at 0 ns every wait that
+    is not already satisfied gives up: the launch reports PA_DEV_TIMEOUT (its
+    outputs are unspecified), every CTA drains its own copies and products,
+    frees tensor memory and returns; the next launch on the same stream, with
+    the normal limit, matches the oracle."""
+    w = _tc_case([700, 45, 1300], seed=5)
+    t = device_inputs(w)
+    ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                             t["slot_mapping"])
+    ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len)
+    out = torch.zeros((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    monkeypatch.setenv("PA_TC_WAIT_NS", "0")
+    ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                  w.scale, w.max_context_len, 0, ws, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 16, "no wait ran out"
+    monkeypatch.delenv("PA_TC_WAIT_NS")
+    out = _decode_with(w, t, ws)
+    ref, _, _ = oracle_step(w)
+    assert_attention_close(out, ref, w.dtype, "after a timed-out launch")
