@@ -81,10 +81,18 @@ def _load():
         lib.oracle_fp8_encode.argtypes = [P, P, LL]
         lib.oracle_swap_blocks.argtypes = [P, P, P, P, P, I, ctypes.c_size_t, I, I]
         lib.oracle_prefill.argtypes = [P, P, P, P, I, P, I, P, P, I, I, I, I, I, I, D, I]
+        lib.oracle_decode_mixed.argtypes = [P, P, I, P, I, D, P, I, D, P, I, P, I, I, I, I, I,
+                                            I, D, P, I, I]
+        lib.oracle_prefill_mixed.argtypes = [P, P, I, P, I, D, P, I, D, P, I, P, P, I, I, I, I,
+                                             I, I, D, I]
+        lib.oracle_reshape_and_cache_mixed.argtypes = [P, P, P, P, I, I, I, ctypes.c_float,
+                                                       ctypes.c_float, P, I, I, I, I, I]
         for fn in ("oracle_gather", "oracle_decode", "oracle_decode_partitioned",
                    "oracle_reshape_and_cache", "oracle_copy_blocks", "oracle_widen",
                    "oracle_max_threads", "oracle_decode_kv", "oracle_reshape_and_cache_fp8",
-                   "oracle_fp8_encode", "oracle_swap_blocks", "oracle_prefill"):
+                   "oracle_fp8_encode", "oracle_swap_blocks", "oracle_prefill",
+                   "oracle_decode_mixed", "oracle_prefill_mixed",
+                   "oracle_reshape_and_cache_mixed"):
             getattr(lib, fn).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -255,4 +263,60 @@ def prefill(q, k_cache, v_cache, dtype: int, block_tables, context_lens, query_s
     _check(_load().oracle_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), dtype,
                                   _ptr(bt), bt.shape[1], _ptr(cl), _ptr(qs), B, Hq, hkv, D, bs, nb,
                                   float(scale), int(n_threads)))
+    return out
+
+
+def decode_mixed(q, q_dtype: int, k_cache, k_dtype: int, k_scale: float, v_cache, v_dtype: int,
+                 v_scale: float, block_tables, context_lens, scale: float, rows=None,
+                 n_threads: int = 0) -> np.ndarray:
+    """Attention with one element type per pool (e.g. K as FP8 codes times
+    k_scale, V as bf16): [B, Hq, D] float64, or [len(rows), D]."""
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    bt, cl = _c(block_tables, np.int32), _c(context_lens, np.int32)
+    B, Hq, D = q.shape
+    nb, bs, hkv, d2 = k_cache.shape
+    assert d2 == D and v_cache.shape == k_cache.shape and bt.shape[0] == B
+    if rows is None:
+        out = np.empty((B, Hq, D), dtype=np.float64)
+        rp, nr = None, 0
+    else:
+        rows = _c(rows, np.int32).reshape(-1, 2)
+        out = np.empty((rows.shape[0], D), dtype=np.float64)
+        rp, nr = _ptr(rows), rows.shape[0]
+    _check(_load().oracle_decode_mixed(_ptr(out), _ptr(q), q_dtype, _ptr(k_cache), k_dtype,
+                                       float(k_scale), _ptr(v_cache), v_dtype, float(v_scale),
+                                       _ptr(bt), bt.shape[1], _ptr(cl), B, Hq, hkv, D, bs, nb,
+                                       float(scale), rp, nr, int(n_threads)))
+    return out
+
+
+def reshape_and_cache_mixed(k_pool: np.ndarray, v_pool: np.ndarray, key, value, src_dtype: int,
+                            k_dtype: int, v_dtype: int, k_scale: float, v_scale: float,
+                            slot_mapping) -> None:
+    """In place: each pool gets the new rows copied (pool type = src_dtype) or
+    quantised to E4M3 codes (pool type FP8, code = E4M3(float(x) / scale))."""
+    assert k_pool.flags.c_contiguous and v_pool.flags.c_contiguous
+    key, value, sm = _c(key), _c(value), _c(slot_mapping, np.int64)
+    nb, bs, hkv, d = k_pool.shape
+    assert v_pool.shape == k_pool.shape
+    _check(_load().oracle_reshape_and_cache_mixed(
+        _ptr(k_pool), _ptr(v_pool), _ptr(key), _ptr(value), src_dtype, k_dtype, v_dtype,
+        float(k_scale), float(v_scale), _ptr(sm), sm.shape[0], hkv, d, bs, nb))
+
+
+def prefill_mixed(q, q_dtype: int, k_cache, k_dtype: int, k_scale: float, v_cache, v_dtype: int,
+                  v_scale: float, block_tables, context_lens, query_start, scale: float,
+                  n_threads: int = 0) -> np.ndarray:
+    """Causal prefill attention with one element type per pool: [T, Hq, D] float64."""
+    q, k_cache, v_cache = _c(q), _c(k_cache), _c(v_cache)
+    bt, cl, qs = _c(block_tables, np.int32), _c(context_lens, np.int32), _c(query_start, np.int32)
+    T, Hq, D = q.shape
+    nb, bs, hkv, _ = k_cache.shape
+    B = cl.shape[0]
+    assert qs.shape[0] == B + 1 and int(qs[-1]) == T and v_cache.shape == k_cache.shape
+    out = np.empty((T, Hq, D), dtype=np.float64)
+    _check(_load().oracle_prefill_mixed(_ptr(out), _ptr(q), q_dtype, _ptr(k_cache), k_dtype,
+                                        float(k_scale), _ptr(v_cache), v_dtype, float(v_scale),
+                                        _ptr(bt), bt.shape[1], _ptr(cl), _ptr(qs), B, Hq, hkv, D,
+                                        bs, nb, float(scale), int(n_threads)))
     return out

@@ -187,6 +187,8 @@ static int attend_row(double* o, const void* q, int qdt, const void* kpool, int 
                       const int32_t* table, int ctx, int Hq, int Hkv, int D, int bs,
                       int num_blocks, double scale, int b, int hq) {
   int G = Hq / Hkv, h = hq / G;
+  if (kdt != OR_FP8) kscale = 1.0;             /* a scale belongs to FP8 codes only */
+  if (vdt != OR_FP8) vscale = 1.0;
   for (int d = 0; d < D; ++d) o[d] = 0.0;
   if (ctx <= 0) return OR_OK;
   double* K = (double*)malloc(sizeof(double) * (size_t)ctx * D);
@@ -235,7 +237,8 @@ static int check_decode_args(const void* q, const void* kp, const void* vp, int 
 /*
  * out: [n_rows, D] (rows != NULL: rows holds n_rows (b, hq) pairs) or
  *      [B, Hq, D] (rows == NULL). The K pool holds k_dtype elements (read times
- * k_scale), the V pool v_dtype elements (times v_scale): an FP8 K pool with a
+ * k_scale if they are FP8 codes), the V pool v_dtype elements (times v_scale
+ * if FP8; 16/32-bit pools are read as stored): an FP8 K pool with a
  * 16-bit V pool is the mixed configuration of "vLLM与PagedAttention：大模型推理
  * 内存优化技术解析" section 6.1.
  * Returns OR_OK, or an error code (first error wins); n_threads <= 0 = all.

@@ -448,6 +448,130 @@ def test_decode_kv_with_one_type_equals_decode():
     assert np.array_equal(a, b)
 
 
+# -- one element type per pool (K in FP8, V in 16 bits, or the reverse) -------------
+def _code_layout(rng, ctxs, bs, Hkv, D, k_fp8: bool, v_fp8: bool, dt):
+    """Per-sequence contiguous K/V (FP8 codes or dt values) scattered block-wise
+    into pools through a random permutation; empty slots hold NaN (0x7F for codes)."""
+    from paged_kv_cache_418_b200.workloads import random_e4m3_codes
+    mk = lambda fp8, n: (random_e4m3_codes(rng, (n, Hkv, D)) if fp8
+                         else _rand(rng, (n, Hkv, D), dt))
+    kc = [mk(k_fp8, n) for n in ctxs]
+    vc = [mk(v_fp8, n) for n in ctxs]
+    nblk = [(n + bs - 1) // bs for n in ctxs]
+    nb = sum(nblk) + 2
+    perm = rng.permutation(nb)
+    kp = nan_fill((nb, bs, Hkv, D), oracle.FP8 if k_fp8 else dt)
+    vp = nan_fill((nb, bs, Hkv, D), oracle.FP8 if v_fp8 else dt)
+    tables = np.full((len(ctxs), max(nblk)), -1, dtype=np.int32)
+    used = 0
+    for b, n in enumerate(ctxs):
+        ids = perm[used:used + nblk[b]]
+        used += nblk[b]
+        tables[b, :nblk[b]] = ids
+        pk = nan_fill((nblk[b] * bs, Hkv, D), oracle.FP8 if k_fp8 else dt)
+        pv = nan_fill((nblk[b] * bs, Hkv, D), oracle.FP8 if v_fp8 else dt)
+        pk[:n], pv[:n] = kc[b], vc[b]
+        kp[ids], vp[ids] = pk.reshape(-1, bs, Hkv, D), pv.reshape(-1, bs, Hkv, D)
+    return kc, vc, kp, vp, tables
+
+
+@pytest.mark.parametrize("k_fp8,v_fp8,dt,Hq,Hkv,D,bs", [
+    (True, False, BF16, 8, 2, 32, 4),      # the explainer's K fp8 / V bf16
+    (True, False, F16, 16, 2, 128, 16),
+    (False, True, BF16, 4, 4, 16, 8),      # and the reverse
+])
+def test_decode_mixed_pool_types_match_torch_sdpa(k_fp8, v_fp8, dt, Hq, Hkv, D, bs):
+    rng = RNG(61 + Hq + D)
+    ctxs = [1, 7, bs, bs + 3, 40]
+    kc, vc, kp, vp, tables = _code_layout(rng, ctxs, bs, Hkv, D, k_fp8, v_fp8, dt)
+    q = _rand(rng, (len(ctxs), Hq, D), dt)
+    ks, vs, scale = float(np.float32(0.3)), float(np.float32(0.7)), 1.0 / math.sqrt(D)
+    kdt, vdt = (oracle.FP8 if k_fp8 else dt), (oracle.FP8 if v_fp8 else dt)
+    out = oracle.decode_mixed(q, dt, kp, kdt, ks, vp, vdt, vs, tables, np.array(ctxs), scale)
+    for b in range(len(ctxs)):
+        k64 = _torch_e4m3_to_f64(kc[b]) * ks if k_fp8 else storage_to_float64(kc[b], dt)
+        v64 = _torch_e4m3_to_f64(vc[b]) * vs if v_fp8 else storage_to_float64(vc[b], dt)
+        ref = _sdpa(storage_to_float64(q[b], dt), k64, v64, scale)
+        np.testing.assert_allclose(out[b], ref, rtol=0, atol=1e-12)
+
+
+def test_decode_mixed_with_one_type_equals_decode_kv():
+    rng = RNG(62)
+    for fp8, dt in ((True, F16), (False, BF16)):
+        kc, vc, kp, vp, tables = _code_layout(rng, [3, 9, 17], 4, 2, 16, fp8, fp8, dt)
+        q = _rand(rng, (3, 4, 16), dt)
+        pdt = oracle.FP8 if fp8 else dt
+        a = oracle.decode_kv(q, dt, kp, vp, pdt, 0.5, 0.25, tables, [3, 9, 17], 0.3)
+        b = oracle.decode_mixed(q, dt, kp, pdt, 0.5, vp, pdt, 0.25, tables, [3, 9, 17], 0.3)
+        assert np.array_equal(a, b)
+
+
+def test_reshape_and_cache_mixed_quantises_one_pool_and_copies_the_other():
+    rng = RNG(63)
+    nb, bs, hkv, d, T = 6, 16, 2, 32, 5
+    ks, vs = np.float32(0.37), np.float32(0.6)
+    slots = np.array([37, -1, 0, 95, 50], dtype=np.int64)
+    for src in (F16, BF16):
+        key = _rand(rng, (T, hkv, d), src, scale=3.0)
+        val = _rand(rng, (T, hkv, d), src)
+        for k_fp8 in (True, False):
+            kp = nan_fill((nb, bs, hkv, d), oracle.FP8 if k_fp8 else src)
+            vp = nan_fill((nb, bs, hkv, d), src if k_fp8 else oracle.FP8)
+            k0, v0 = kp.copy(), vp.copy()
+            oracle.reshape_and_cache_mixed(kp, vp, key, val, src,
+                                           oracle.FP8 if k_fp8 else src,
+                                           src if k_fp8 else oracle.FP8, float(ks), float(vs),
+                                           slots)
+            q_src, q_pool, q_sc = (key, kp, ks) if k_fp8 else (val, vp, vs)
+            c_src, c_pool = (val, vp) if k_fp8 else (key, kp)
+            # the quantised pool: numpy float32 division, torch's E4M3 cast
+            x = (storage_to_float64(q_src, src).astype(np.float32) / q_sc).clip(-448, 448)
+            codes = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+            touched = np.zeros((nb, bs), dtype=bool)
+            for t, s in enumerate(slots):
+                if s < 0:
+                    continue
+                assert np.array_equal(q_pool[s // bs, s % bs], codes[t])
+                assert np.array_equal(c_pool[s // bs, s % bs].view(np.uint16),
+                                      c_src[t].view(np.uint16))          # bit for bit
+                touched[s // bs, s % bs] = True
+            assert np.array_equal(kp[~touched].view(np.uint8), k0[~touched].view(np.uint8))
+            assert np.array_equal(vp[~touched].view(np.uint8), v0[~touched].view(np.uint8))
+    with pytest.raises(oracle.OracleError):             # a 16-bit pool of another type
+        oracle.reshape_and_cache_mixed(nan_fill((nb, bs, hkv, d), oracle.FP8),
+                                       nan_fill((nb, bs, hkv, d), F16), key, val, BF16,
+                                       oracle.FP8, F16, 0.5, 0.5, slots)
+
+
+@pytest.mark.parametrize("k_fp8,v_fp8", [(True, True), (True, False)])
+def test_prefill_mixed_over_fp8_pools_matches_sdpa_with_a_causal_mask(k_fp8, v_fp8):
+    rng = RNG(64)
+    dt, Hq, Hkv, D, bs = BF16, 8, 2, 32, 4
+    prior, new = [0, 5, 17], [7, 1, 9]
+    ctxs = [p + n for p, n in zip(prior, new)]
+    kc, vc, kp, vp, tables = _code_layout(rng, ctxs, bs, Hkv, D, k_fp8, v_fp8, dt)
+    T = sum(new)
+    q = _rand(rng, (T, Hq, D), dt)
+    qs = np.concatenate([[0], np.cumsum(new)]).astype(np.int32)
+    ks, vs, scale = float(np.float32(0.4)), float(np.float32(0.9)), 1.0 / math.sqrt(D)
+    kdt, vdt = (oracle.FP8 if k_fp8 else dt), (oracle.FP8 if v_fp8 else dt)
+    out = oracle.prefill_mixed(q, dt, kp, kdt, ks, vp, vdt, vs, tables, np.array(ctxs), qs, scale)
+    for b in range(3):
+        n, ctx = new[b], ctxs[b]
+        k64 = _torch_e4m3_to_f64(kc[b]) * ks if k_fp8 else storage_to_float64(kc[b], dt)
+        v64 = _torch_e4m3_to_f64(vc[b]) * vs if v_fp8 else storage_to_float64(vc[b], dt)
+        q64 = storage_to_float64(q[qs[b]:qs[b + 1]], dt)
+        pos = ctx - n + np.arange(n)
+        mask = torch.from_numpy(np.arange(ctx)[None, :] <= pos[:, None])
+        qt = torch.from_numpy(np.ascontiguousarray(q64.transpose(1, 0, 2)))[None]
+        kt = torch.from_numpy(np.ascontiguousarray(k64.transpose(1, 0, 2)))[None]
+        vt = torch.from_numpy(np.ascontiguousarray(v64.transpose(1, 0, 2)))[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, attn_mask=mask, scale=scale, enable_gqa=True)[0].numpy()
+        got = out[qs[b]:qs[b + 1]].transpose(1, 0, 2)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
 # -- swap_blocks ---------------------------------------------------------------------
 def test_swap_blocks_moves_whole_blocks_between_pools():
     rng = RNG(45)

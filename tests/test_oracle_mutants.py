@@ -43,6 +43,10 @@ MUTANTS = [
      "size_t blk = (size_t)(s / bs), off = 0;"),
     ("copy-v-dropped", "    memcpy((char*)vpool + d * blk, snap + (2 * (size_t)p + 1) * blk, blk);\n", ""),
     ("swap-reads-dst-index", "(const char*)src_k + s * block_bytes", "(const char*)src_k + d * block_bytes"),
+    ("mixed-v-read-as-k-type", "rc = gather_head(V, vpool, vdt, vscale,", "rc = gather_head(V, vpool, kdt, vscale,"),
+    ("mixed-scatter-one-scale", "float sc = which ? v_scale : k_scale;", "float sc = k_scale;"),
+    ("mixed-prefill-v-unscaled", "kpool, k_dtype, k_scale, vpool, v_dtype, v_scale,\n                       block_tables",
+     "kpool, k_dtype, k_scale, vpool, v_dtype, 1.0,\n                       block_tables"),
 ]
 
 PLUGIN = '''
