@@ -101,8 +101,8 @@ def peaks():
 
 
 def config_of(w: W.Workload, world: int, l2_note: str):
-    extra = ({"kv_cache": W.DTYPE_NAMES[w.kv_dtype], "k_scale": w.k_scale, "v_scale": w.v_scale}
-             if w.fp8 else {})
+    extra = ({"k_cache": W.DTYPE_NAMES[w.kv_dtype], "v_cache": W.DTYPE_NAMES[w.v_dtype],
+              "k_scale": w.k_scale, "v_scale": w.v_scale} if w.fp8 else {})
     return {**extra,
         "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "head_dim": w.D,
         "block_size": w.block_size, "num_blocks": w.num_blocks, "dtype": W.DTYPE_NAMES[w.dtype],
@@ -213,7 +213,10 @@ def oracle_cache_ops(w: W.Workload, kc, vc):
     import oracle
     if len(w.block_mapping):
         oracle.copy_blocks(kc, vc, w.block_mapping, w.kv_dtype)
-    if w.fp8:
+    if w.mixed:
+        oracle.reshape_and_cache_mixed(kc, vc, w.new_key, w.new_value, w.dtype, w.kv_dtype,
+                                       w.v_dtype, w.k_scale, w.v_scale, w.slot_mapping)
+    elif w.fp8:
         oracle.reshape_and_cache_fp8(kc, vc, w.new_key, w.new_value, w.dtype, w.k_scale,
                                      w.v_scale, w.slot_mapping)
     else:
@@ -222,6 +225,9 @@ def oracle_cache_ops(w: W.Workload, kc, vc):
 
 def oracle_decode_rows(w: W.Workload, kc, vc, rows):
     import oracle
+    if w.mixed:
+        return oracle.decode_mixed(w.q, w.dtype, kc, w.kv_dtype, w.k_scale, vc, w.v_dtype,
+                                   w.v_scale, w.block_tables, w.context_lens, w.scale, rows=rows)
     if w.fp8:
         return oracle.decode_kv(w.q, w.dtype, kc, vc, oracle.FP8, w.k_scale, w.v_scale,
                                 w.block_tables, w.context_lens, w.scale, rows=rows)
@@ -262,11 +268,13 @@ def reference_arm(args, w: W.Workload, rank: int, world: int):
     # the same oracle on one core: decode of a ~3 s sample of rows
     rows1 = oracle_sample_rows(w, budget_s=3.0 / max(1, cores), rng_seed=1)
     t = time.perf_counter()
-    oracle.decode_kv(w.q, w.dtype, w.k_cache, w.v_cache, w.kv_dtype, w.k_scale, w.v_scale,
-                     w.block_tables, w.context_lens, w.scale, rows=rows1, n_threads=1)
+    oracle.decode_mixed(w.q, w.dtype, w.k_cache, w.kv_dtype, w.k_scale, w.v_cache, w.v_dtype,
+                        w.v_scale, w.block_tables, w.context_lens, w.scale, rows=rows1,
+                        n_threads=1)
     secs1 = time.perf_counter() - t
-    oracle.decode_kv(w.q, w.dtype, w.k_cache, w.v_cache, w.kv_dtype, w.k_scale, w.v_scale,
-                     w.block_tables, w.context_lens, w.scale, rows=rows1[:1], n_threads=cores)
+    oracle.decode_mixed(w.q, w.dtype, w.k_cache, w.kv_dtype, w.k_scale, w.v_cache, w.v_dtype,
+                        w.v_scale, w.block_tables, w.context_lens, w.scale, rows=rows1[:1],
+                        n_threads=cores)
     frac1 = float(w.context_lens[rows1[:, 0]].sum()) / (w.Hq * float(w.context_lens.sum()))
     one_core = {"value": round(w.kv_bytes() * frac1 / secs1 / 1e9, 4), "unit": "GB/s",
                 "sample": f"decode of {len(rows1)} rows on 1 thread, {secs1:.1f} s"}
@@ -347,14 +355,18 @@ class Decoder:
 
     def plan(self):
         w = self.w
-        return self.ops.pa_decode_plan(w.kv_dtype, w.B, w.Hq, w.Hkv, w.D, w.block_size,
-                                       w.max_context_len, w.partition_size)
+        return self.ops.pa_decode_plan(W.FP8 if w.fp8 else w.kv_dtype, w.B, w.Hq, w.Hkv, w.D,
+                                       w.block_size, w.max_context_len, w.partition_size)
 
     def cache_ops(self):
         w, t, ops = self.w, self.t, self.ops
         if len(w.block_mapping):
             ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], self.err, self.stream)
-        if w.fp8:
+        if w.mixed:
+            ops.pa_reshape_and_cache_kv(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                        w.k_scale, w.v_scale, t["slot_mapping"], self.err,
+                                        self.stream)
+        elif w.fp8:
             ops.pa_reshape_and_cache_fp8(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
                                          w.k_scale, w.v_scale, t["slot_mapping"], self.err,
                                          self.stream)
@@ -370,6 +382,10 @@ class Decoder:
                                         t["block_tables"], t["context_lens"], g_shared, g_off,
                                         g_mem, nc, pb, w.scale, w.max_context_len,
                                         w.partition_size, self.ws, self.err, self.stream)
+        elif w.mixed:
+            ops.pa_decode_kv(self.out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
+                             t["block_tables"], t["context_lens"], w.scale, w.max_context_len,
+                             w.partition_size, self.ws, self.err, self.stream)
         elif w.fp8:
             ops.pa_decode_fp8(self.out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
                               t["block_tables"], t["context_lens"], w.scale, w.max_context_len,
@@ -567,7 +583,7 @@ def ours_arm(args, w: W.Workload, rank: int, world: int, local_rank: int):
 
 
 SUITE = [  # (workload id, shared-prefix decode) measured beside the headline by default
-    (3, False), (4, False), (5, False), (5, True), (6, False)]
+    (3, False), (4, False), (5, False), (5, True), (6, False), (7, False), (8, False)]
 
 
 def suite(args, local_rank: int):

@@ -235,6 +235,46 @@ int pa_decode_fp8(void* out, int out_dtype, const void* query, int q_dtype, cons
                   void* workspace, size_t workspace_bytes, uint32_t* err_flag, void* stream);
 
 /*
+ * Mixed pools: one element type per pool. The explainer configures the key
+ * cache in fp8 and the value cache in bf16 ("vLLM与PagedAttention：大模型推理
+ * 内存优化技术解析" section 6.1, mixed-precision configuration); the two
+ * entry points below take each pool's type separately.
+ *
+ * pa_reshape_and_cache_kv -- pa_reshape_and_cache with per-pool types.
+ * key, value    [T, Hkv, D] of src_dtype (PA_F32, PA_F16 or PA_BF16);
+ * key_cache     [num_blocks, block_size, Hkv, D] of k_dtype: src_dtype (the
+ *               rows are copied bit for bit) or PA_FP8_E4M3 (quantised as in
+ *               pa_reshape_and_cache_fp8 with k_scale);
+ * value_cache   likewise with v_dtype and v_scale;
+ * a scale is checked (positive, finite) and used only for an FP8 pool.
+ * Other arguments and errors as pa_reshape_and_cache.
+ */
+int pa_reshape_and_cache_kv(const void* key, const void* value, int src_dtype, void* key_cache,
+                            int k_dtype, float k_scale, void* value_cache, int v_dtype,
+                            float v_scale, const int64_t* slot_mapping, int T, int Hkv, int D,
+                            int block_size, int num_blocks, uint32_t* err_flag, void* stream);
+
+/*
+ * pa_decode_kv -- pa_decode with per-pool types: each K element attended is
+ * the K pool's value (times k_scale if it holds FP8 codes), each V element
+ * likewise with v_scale.
+ * query         [B, Hq, D] of q_dtype (PA_F32, PA_F16 or PA_BF16);
+ * key_cache     of k_dtype, value_cache of v_dtype: each q_dtype or
+ *               PA_FP8_E4M3; one FP8 pool beside one of the query's type needs
+ *               a 16-bit query (otherwise PA_ERR_DTYPE);
+ * k_scale, v_scale  positive finite scales of the FP8 pools (ignored for others).
+ * Every other argument, the workspace (pa_workspace_size) and the errors are
+ * pa_decode's. Calls with both pools of the query's type are pa_decode; calls
+ * with an FP8 pool run on the CUDA-core decode kernel.
+ */
+int pa_decode_kv(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                 int k_dtype, float k_scale, const void* value_cache, int v_dtype, float v_scale,
+                 const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                 int B, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+                 int max_context_len, int partition_size, void* workspace,
+                 size_t workspace_bytes, uint32_t* err_flag, void* stream);
+
+/*
  * pa_swap_blocks -- preemption by swapping: copy whole blocks (K and V)
  * between two pools, typically the device pool and a pool in page-locked host
  * memory ("vLLM 与 LLM 推理部署实战" section 三: under memory pressure the

@@ -59,17 +59,34 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ key_cache, uint4* __restr
     d[i] = s[i];
 }
 
-// FP8 form of reshape_and_cache: one thread writes 16 codes (one 16-byte
-// vector) of one token's K row and the same 16 of its V row. The source
-// elements (TS = f32, f16 or bf16) are exact in fp32; each is divided by the
-// pool's scale (IEEE division) and rounded to E4M3, nearest even, saturating.
-template <typename TS>
-__global__ void reshape_and_cache_fp8_kernel(const TS* __restrict__ key, const TS* __restrict__ value,
-                                             uint4* __restrict__ key_cache,
-                                             uint4* __restrict__ value_cache, float k_scale,
-                                             float v_scale, const int64_t* __restrict__ slot_mapping,
-                                             int T, int row16, long long num_slots,
-                                             uint32_t* err_flag) {
+// reshape_and_cache into pools of per-pool element types: one thread takes 16
+// consecutive elements of one token's K row and the same 16 of its V row. A
+// pool marked FP8 (KQ / VQ) receives codes: each element (TS = f32, f16 or
+// bf16, exact in fp32) is divided by the pool's scale (IEEE division) and
+// rounded to E4M3, nearest even, saturating; the other pool receives the 16
+// elements bit for bit.
+__device__ __forceinline__ uint4 quantise16(const float* f, float scale) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __nv_fp8x2_storage_t c0 = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(f[4 * k], scale), __fdiv_rn(f[4 * k + 1], scale)), __NV_SATFINITE,
+        __NV_E4M3);
+    const __nv_fp8x2_storage_t c1 = __nv_cvt_float2_to_fp8x2(
+        make_float2(__fdiv_rn(f[4 * k + 2], scale), __fdiv_rn(f[4 * k + 3], scale)),
+        __NV_SATFINITE, __NV_E4M3);
+    w[k] = (uint32_t)c0 | ((uint32_t)c1 << 16);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename TS, bool KQ, bool VQ>
+__global__ void reshape_and_cache_kv_kernel(const TS* __restrict__ key,
+                                            const TS* __restrict__ value, void* __restrict__ key_cache,
+                                            void* __restrict__ value_cache, float k_scale,
+                                            float v_scale, const int64_t* __restrict__ slot_mapping,
+                                            int T, int row16, long long num_slots,
+                                            uint32_t* err_flag) {
   pdl_trigger();
   pdl_wait();
   constexpr int N = Vec<TS>::N;                  // source elements per 16-byte load
@@ -85,33 +102,26 @@ __global__ void reshape_and_cache_fp8_kernel(const TS* __restrict__ key, const T
       continue;
     }
     const size_t src = ((size_t)t * row16 + c) * 16;   // first of this thread's 16 elements
-    float kf[16], vf[16];
+    const size_t dst = ((size_t)s * row16 + c) * 16;   // the same element of the pool row
 #pragma unroll
-    for (int k = 0; k < 16 / N; ++k) {
-      widen16<TS>(*reinterpret_cast<const uint4*>(key + src + k * N), kf + k * N);
-      widen16<TS>(*reinterpret_cast<const uint4*>(value + src + k * N), vf + k * N);
-    }
-    uint32_t kw[4], vw[4];
+    for (int which = 0; which < 2; ++which) {
+      const TS* in = which ? value : key;
+      const bool q = which ? VQ : KQ;
+      void* pool = which ? value_cache : key_cache;
+      if (q) {
+        float f[16];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const __nv_fp8x2_storage_t k0 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fdiv_rn(kf[4 * k], k_scale), __fdiv_rn(kf[4 * k + 1], k_scale)),
-          __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t k1 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fdiv_rn(kf[4 * k + 2], k_scale), __fdiv_rn(kf[4 * k + 3], k_scale)),
-          __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t v0 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fdiv_rn(vf[4 * k], v_scale), __fdiv_rn(vf[4 * k + 1], v_scale)),
-          __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t v1 = __nv_cvt_float2_to_fp8x2(
-          make_float2(__fdiv_rn(vf[4 * k + 2], v_scale), __fdiv_rn(vf[4 * k + 3], v_scale)),
-          __NV_SATFINITE, __NV_E4M3);
-      kw[k] = (uint32_t)k0 | ((uint32_t)k1 << 16);
-      vw[k] = (uint32_t)v0 | ((uint32_t)v1 << 16);
+        for (int k = 0; k < 16 / N; ++k)
+          widen16<TS>(*reinterpret_cast<const uint4*>(in + src + k * N), f + k * N);
+        *reinterpret_cast<uint4*>(static_cast<uint8_t*>(pool) + dst) =
+            quantise16(f, which ? v_scale : k_scale);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16 / N; ++k)
+          reinterpret_cast<uint4*>(static_cast<TS*>(pool) + dst)[k] =
+              *reinterpret_cast<const uint4*>(in + src + k * N);
+      }
     }
-    const size_t dst = (size_t)s * row16 + c;
-    key_cache[dst] = make_uint4(kw[0], kw[1], kw[2], kw[3]);
-    value_cache[dst] = make_uint4(vw[0], vw[1], vw[2], vw[3]);
   }
 }
 
@@ -137,40 +147,49 @@ __global__ void swap_blocks_kernel(uint4* __restrict__ dst_k, uint4* __restrict_
     d[i] = s[i];
 }
 
-int launch_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype,
-                                 void* key_cache, void* value_cache, float k_scale,
-                                 float v_scale, const int64_t* slot_mapping, int T, int Hkv,
-                                 int D, int block_size, int num_blocks, uint32_t* err_flag,
-                                 cudaStream_t stream) {
-  if (T == 0) return PA_OK;
-  int row16 = Hkv * D / 16;                      // 16-code vectors per token row
+template <typename TS>
+int launch_rac_kv(const void* key, const void* value, void* key_cache, int k_fp8, float k_scale,
+                  void* value_cache, int v_fp8, float v_scale, const int64_t* slot_mapping, int T,
+                  int row16, long long slots, uint32_t* err_flag, cudaStream_t stream) {
   long long n = (long long)T * row16;
   int threads = 256;
   long long blocks = (n + threads - 1) / threads;
   if (blocks > 8 * kSMs) blocks = 8 * kSMs;
-  const long long slots = (long long)num_blocks * block_size;
+  const TS* k = static_cast<const TS*>(key);
+  const TS* v = static_cast<const TS*>(value);
+  auto go = [&](auto kern) {
+    return launch_k(kern, dim3((unsigned)blocks), dim3(threads), 0, stream, k, v, key_cache,
+                    value_cache, k_scale, v_scale, slot_mapping, T, row16, slots, err_flag);
+  };
   cudaError_t e;
+  if (k_fp8 && v_fp8) e = go(reshape_and_cache_kv_kernel<TS, true, true>);
+  else if (k_fp8) e = go(reshape_and_cache_kv_kernel<TS, true, false>);
+  else if (v_fp8) e = go(reshape_and_cache_kv_kernel<TS, false, true>);
+  else e = go(reshape_and_cache_kv_kernel<TS, false, false>);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int launch_reshape_and_cache_kv(const void* key, const void* value, int src_dtype,
+                                void* key_cache, int k_fp8, float k_scale, void* value_cache,
+                                int v_fp8, float v_scale, const int64_t* slot_mapping, int T,
+                                int Hkv, int D, int block_size, int num_blocks,
+                                uint32_t* err_flag, cudaStream_t stream) {
+  if (T == 0) return PA_OK;
+  const int row16 = Hkv * D / 16;                // 16-element groups per token row
+  const long long slots = (long long)num_blocks * block_size;
   switch (src_dtype) {
     case PA_F32:
-      e = launch_k(reshape_and_cache_fp8_kernel<float>, dim3((unsigned)blocks), dim3(threads), 0,
-                   stream, (const float*)key, (const float*)value, (uint4*)key_cache,
-                   (uint4*)value_cache, k_scale, v_scale, slot_mapping, T, row16, slots, err_flag);
-      break;
+      return launch_rac_kv<float>(key, value, key_cache, k_fp8, k_scale, value_cache, v_fp8,
+                                  v_scale, slot_mapping, T, row16, slots, err_flag, stream);
     case PA_F16:
-      e = launch_k(reshape_and_cache_fp8_kernel<__half>, dim3((unsigned)blocks), dim3(threads), 0,
-                   stream, (const __half*)key, (const __half*)value, (uint4*)key_cache,
-                   (uint4*)value_cache, k_scale, v_scale, slot_mapping, T, row16, slots, err_flag);
-      break;
+      return launch_rac_kv<__half>(key, value, key_cache, k_fp8, k_scale, value_cache, v_fp8,
+                                   v_scale, slot_mapping, T, row16, slots, err_flag, stream);
     case PA_BF16:
-      e = launch_k(reshape_and_cache_fp8_kernel<__nv_bfloat16>, dim3((unsigned)blocks),
-                   dim3(threads), 0, stream, (const __nv_bfloat16*)key,
-                   (const __nv_bfloat16*)value, (uint4*)key_cache, (uint4*)value_cache, k_scale,
-                   v_scale, slot_mapping, T, row16, slots, err_flag);
-      break;
-    default:
-      return PA_ERR_DTYPE;
+      return launch_rac_kv<__nv_bfloat16>(key, value, key_cache, k_fp8, k_scale, value_cache,
+                                          v_fp8, v_scale, slot_mapping, T, row16, slots, err_flag,
+                                          stream);
   }
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return PA_ERR_DTYPE;
 }
 
 int launch_swap_blocks(void* dst_key, void* dst_value, const void* src_key,

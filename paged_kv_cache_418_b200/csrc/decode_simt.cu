@@ -56,16 +56,22 @@ __device__ __forceinline__ void load_q(const TQ* p, float* f) {
   for (int c = 0; c < VEC / N; ++c) widen16<TQ>(*reinterpret_cast<const uint4*>(p + c * N), f + c * N);
 }
 
-// TQ: query element type; TC: pool element type (TQ, or FP8 E4M3 codes);
-// PF: issue the loads of each warp's next tile before computing the current one.
-template <typename TQ, typename TC, int D, int BS, int GC, bool PF>
+// TQ: query element type; TK, TV: K and V pool element types (TQ, or FP8
+// E4M3 codes; the two may differ); PF: issue the loads of each warp's next
+// tile before computing the current one.
+template <typename TQ, typename TK, typename TV, int D, int BS, int GC, bool PF>
 __global__ void __launch_bounds__(kWarps * 32)
 decode_simt_kernel(const DecodeArgs a) {
-  using T = TC;
-  constexpr int VEC = Vec<T>::N;               // elements per 16-byte vector
+  // elements per lane and row: a 16-byte slice of the wider pool's row (the
+  // narrower pool's slice is then 8 bytes)
+  constexpr int ESZ = sizeof(TK) > sizeof(TV) ? sizeof(TK) : sizeof(TV);
+  constexpr int VEC = 16 / ESZ;
+  constexpr int NBK = VEC * sizeof(TK), NBV = VEC * sizeof(TV);
+  using RK = typename Raw<NBK>::T;
+  using RV = typename Raw<NBV>::T;
   constexpr int LPR = D / VEC;                 // lanes per K/V row: 4, 8, 16 or 32
   constexpr int RPI = 32 / LPR;                // rows per warp instruction: 8, 4, 2 or 1
-  constexpr int RGMAX = sizeof(T) == 1 ? 4 : 8;           // registers: 16 floats per vector for FP8
+  constexpr int RGMAX = VEC == 16 ? 4 : 8;     // registers: 16 floats per slice for FP8 pools
   constexpr int RG = (BS / RPI) < RGMAX ? (BS / RPI) : RGMAX;   // row groups per tile
   constexpr int TILE = RG * RPI;               // tokens per tile (divides BS)
   static_assert(BS % TILE == 0, "tile must divide the block");
@@ -127,14 +133,14 @@ decode_simt_kernel(const DecodeArgs a) {
   }
 
   const int32_t* table = a.block_tables + (size_t)b * a.max_blocks;
-  const T* kc = reinterpret_cast<const T*>(a.k_cache);
-  const T* vc = reinterpret_cast<const T*>(a.v_cache);
+  const TK* kc = reinterpret_cast<const TK*>(a.k_cache);
+  const TV* vc = reinterpret_cast<const TV*>(a.v_cache);
   const size_t row_stride = (size_t)a.Hkv * D;          // elements between token rows
   const int tile_begin = tok_begin / TILE;
   const int tile_end = (tok_end + TILE - 1) / TILE;
 
   // rows of tile tt of block ph into k / v (zeros past the context or for a bad block)
-  auto issue = [&](int tt, int ph, uint4* k, uint4* v) {
+  auto issue = [&](int tt, int ph, RK* k, RV* v) {
     const int token0 = tt * TILE;
     const bool ok = ph >= 0 && ph < a.num_blocks;
     const size_t base =
@@ -143,26 +149,26 @@ decode_simt_kernel(const DecodeArgs a) {
     for (int r = 0; r < RG; ++r) {
       const int row = r * RPI + rs;
       if (ok && token0 + row < tok_end) {
-        k[r] = ld_stream16(kc + base + row * row_stride);
-        v[r] = ld_stream16(vc + base + row * row_stride);
+        k[r] = ld_stream<NBK>(kc + base + row * row_stride);
+        v[r] = ld_stream<NBV>(vc + base + row * row_stride);
       } else {
-        k[r] = make_uint4(0, 0, 0, 0);
-        v[r] = make_uint4(0, 0, 0, 0);
+        k[r] = raw_zero<NBK>();
+        v[r] = raw_zero<NBV>();
       }
     }
   };
   // scores, online softmax and P.V of tile tt
-  auto consume = [&](int tt, const uint4* kr, const uint4* vr) {
+  auto consume = [&](int tt, const RK* kr, const RV* vr) {
     const int token0 = tt * TILE;
     // scores of the lane's RG rows, reduced over the row's LPR lanes
     float s[RG][GC];
 #pragma unroll
     for (int r = 0; r < RG; ++r) {
       float kf[VEC];
-      widen16<T>(kr[r], kf);
+      widen_raw<TK, VEC>(kr[r], kf);
 #pragma unroll
       for (int g = 0; g < GC; ++g) {
-        if constexpr (sizeof(T) == 1) {
+        if constexpr (VEC == 16) {
           // FP8 rows carry twice the elements per byte: packed FMAs halve the issue
           float d0 = 0.f, d1 = 0.f;
 #pragma unroll
@@ -208,10 +214,10 @@ decode_simt_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int r = 0; r < RG; ++r) {
       float vf[VEC];
-      widen16<T>(vr[r], vf);
+      widen_raw<TV, VEC>(vr[r], vf);
 #pragma unroll
       for (int g = 0; g < GC; ++g) {
-        if constexpr (sizeof(T) == 1) {
+        if constexpr (VEC == 16) {
 #pragma unroll
           for (int e = 0; e < VEC; e += 2)
             fma2(acc[g][e], acc[g][e + 1], s[r][g], s[r][g], vf[e], vf[e + 1]);
@@ -235,14 +241,16 @@ decode_simt_kernel(const DecodeArgs a) {
   if constexpr (PF) {
     // Loads of the warp's next tile are issued before this tile is computed, so
     // each warp always has a tile's K and V in flight (block ids two tiles ahead).
-    uint4 kr[RG], vr[RG];
+    RK kr[RG];
+    RV vr[RG];
     int phys = t < tile_end ? block_of(t) : -1;
     int phys_n = t + kWarps < tile_end ? block_of(t + kWarps) : -1;
     if (t < tile_end) issue(t, phys, kr, vr);
     for (; t < tile_end; t += kWarps) {
       const int tn = t + kWarps;
       const int ph = phys;
-      uint4 kn[RG], vn[RG];
+      RK kn[RG];
+      RV vn[RG];
       if (tn < tile_end) issue(tn, phys_n, kn, vn);
       phys = phys_n;
       phys_n = tn + kWarps < tile_end ? block_of(tn + kWarps) : -1;
@@ -257,7 +265,8 @@ decode_simt_kernel(const DecodeArgs a) {
       const int tn = t + kWarps;
       if (tn < tile_end) phys_next = block_of(tn);
       if (bad_block(phys)) continue;
-      uint4 kr[RG], vr[RG];
+      RK kr[RG];
+      RV vr[RG];
       issue(t, phys, kr, vr);
       consume(t, kr, vr);
     }
@@ -320,40 +329,41 @@ int prefetch_override() {
   return s[0] == '1' ? 1 : 0;
 }
 
-template <typename TQ, typename TC, int D, int BS, int GC>
+template <typename TQ, typename TK, typename TV, int D, int BS, int GC>
 int launch_t(const DecodeArgs& a, cudaStream_t stream) {
   const int chunks = (a.Hq / a.Hkv) / GC;
   dim3 grid((unsigned)(a.P * chunks), (unsigned)a.Hkv, (unsigned)a.B);
   const int ov = prefetch_override();
-  const bool pf = ov >= 0 ? ov == 1 : sizeof(TC) == 1;
+  const bool pf = ov >= 0 ? ov == 1 : (sizeof(TK) == 1 || sizeof(TV) == 1);
   const cudaError_t e =
-      pf ? launch_k(decode_simt_kernel<TQ, TC, D, BS, GC, true>, grid, dim3(kWarps * 32), 0,
+      pf ? launch_k(decode_simt_kernel<TQ, TK, TV, D, BS, GC, true>, grid, dim3(kWarps * 32), 0,
                     stream, a)
-         : launch_k(decode_simt_kernel<TQ, TC, D, BS, GC, false>, grid, dim3(kWarps * 32), 0,
+         : launch_k(decode_simt_kernel<TQ, TK, TV, D, BS, GC, false>, grid, dim3(kWarps * 32), 0,
                     stream, a);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <typename TQ, typename TC, int D, int BS>
+template <typename TQ, typename TK, typename TV, int D, int BS>
 int launch_gc(const DecodeArgs& a, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
-  if (G == 1) return launch_t<TQ, TC, D, BS, 1>(a, stream);
-  if constexpr (sizeof(TC) == 1) {
-    return launch_t<TQ, TC, D, BS, 2>(a, stream);   // FP8: pairs of heads (registers)
+  if (G == 1) return launch_t<TQ, TK, TV, D, BS, 1>(a, stream);
+  if constexpr (sizeof(TK) == 1 && sizeof(TV) == 1) {
+    return launch_t<TQ, TK, TV, D, BS, 2>(a, stream);   // FP8: pairs of heads (registers)
   } else {
-    if (G == 2) return launch_t<TQ, TC, D, BS, 2>(a, stream);
-    return launch_t<TQ, TC, D, BS, 4>(a, stream);   // G = 4, 8, 16: chunks of 4 heads
+    if (G == 2) return launch_t<TQ, TK, TV, D, BS, 2>(a, stream);
+    return launch_t<TQ, TK, TV, D, BS, 4>(a, stream);   // G = 4, 8, 16: chunks of 4 heads
   }
 }
 
-template <typename TQ, typename TC, int D>
+template <typename TQ, typename TK, typename TV, int D>
 int launch_bs(const DecodeArgs& a, cudaStream_t stream) {
-  return a.bs == 16 ? launch_gc<TQ, TC, D, 16>(a, stream) : launch_gc<TQ, TC, D, 32>(a, stream);
+  return a.bs == 16 ? launch_gc<TQ, TK, TV, D, 16>(a, stream)
+                    : launch_gc<TQ, TK, TV, D, 32>(a, stream);
 }
 
-template <typename TQ, typename TC>
+template <typename TQ, typename TK, typename TV>
 int launch_d(const DecodeArgs& a, cudaStream_t stream) {
-  return a.D == 64 ? launch_bs<TQ, TC, 64>(a, stream) : launch_bs<TQ, TC, 128>(a, stream);
+  return a.D == 64 ? launch_bs<TQ, TK, TV, 64>(a, stream) : launch_bs<TQ, TK, TV, 128>(a, stream);
 }
 
 // Merge of the split pass, for each (b, hq) row with more than one partition:
@@ -489,19 +499,35 @@ int launch_merge_d(const DecodeArgs& a, cudaStream_t stream) {
 
 int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream) {
   switch (dtype) {
-    case PA_F32: return launch_d<float, float>(a, stream);
-    case PA_F16: return launch_d<__half, __half>(a, stream);
-    case PA_BF16: return launch_d<__nv_bfloat16, __nv_bfloat16>(a, stream);
+    case PA_F32: return launch_d<float, float, float>(a, stream);
+    case PA_F16: return launch_d<__half, __half, __half>(a, stream);
+    case PA_BF16: return launch_d<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(a, stream);
   }
   return PA_ERR_DTYPE;
 }
 
-int launch_decode_simt_fp8(const DecodeArgs& a, int q_dtype, cudaStream_t stream) {
-  switch (q_dtype) {
-    case PA_F32: return launch_d<float, __nv_fp8_e4m3>(a, stream);
-    case PA_F16: return launch_d<__half, __nv_fp8_e4m3>(a, stream);
-    case PA_BF16: return launch_d<__nv_bfloat16, __nv_fp8_e4m3>(a, stream);
+// Pools of other types than the query's: both FP8 (any query type), or one FP8
+// and the other of the query's 16-bit type.
+int launch_decode_simt_kv(const DecodeArgs& a, int q_dtype, int k_dtype, int v_dtype,
+                          cudaStream_t stream) {
+  using F8 = __nv_fp8_e4m3;
+  const bool kf = k_dtype == PA_FP8_E4M3, vf = v_dtype == PA_FP8_E4M3;
+  if (kf && vf) {
+    switch (q_dtype) {
+      case PA_F32: return launch_d<float, F8, F8>(a, stream);
+      case PA_F16: return launch_d<__half, F8, F8>(a, stream);
+      case PA_BF16: return launch_d<__nv_bfloat16, F8, F8>(a, stream);
+    }
+    return PA_ERR_DTYPE;
   }
+  if (q_dtype == PA_F16) {
+    if (kf && v_dtype == PA_F16) return launch_d<__half, F8, __half>(a, stream);
+    if (vf && k_dtype == PA_F16) return launch_d<__half, __half, F8>(a, stream);
+  } else if (q_dtype == PA_BF16) {
+    if (kf && v_dtype == PA_BF16) return launch_d<__nv_bfloat16, F8, __nv_bfloat16>(a, stream);
+    if (vf && k_dtype == PA_BF16) return launch_d<__nv_bfloat16, __nv_bfloat16, F8>(a, stream);
+  }
+  if (!kf && !vf && k_dtype == q_dtype && v_dtype == q_dtype) return launch_decode_simt(a, q_dtype, stream);
   return PA_ERR_DTYPE;
 }
 

@@ -169,15 +169,30 @@ namespace {
 
 bool scale_ok(float x) { return std::isfinite(x) && x > 0.f; }
 
-// Shared body of pa_decode and pa_decode_fp8. q_dtype: query element type;
-// kv_dtype: pool element type (q_dtype itself, or PA_FP8_E4M3 with scales).
+// Pool element types a decode takes for a query of q_dtype: both the query's
+// type; both FP8; or, for a 16-bit query, one FP8 pool and one of its type.
+bool pool_types_ok(int q_dtype, int k_dtype, int v_dtype) {
+  const bool kf = k_dtype == PA_FP8_E4M3, vf = v_dtype == PA_FP8_E4M3;
+  if (!kf && k_dtype != q_dtype) return false;
+  if (!vf && v_dtype != q_dtype) return false;
+  if (kf != vf && q_dtype == PA_F32) return false;
+  return true;
+}
+
+// Shared body of the decode entry points. q_dtype: query element type;
+// k_dtype / v_dtype: pool element types (q_dtype, or PA_FP8_E4M3 read times
+// k_scale / v_scale; a scale is used only by an FP8 pool).
 int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
-                const void* value_cache, int kv_dtype, float k_scale, float v_scale,
+                int k_dtype, float k_scale, const void* value_cache, int v_dtype, float v_scale,
                 const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
                 int B, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
                 int max_context_len, int partition_size, void* workspace,
                 size_t workspace_bytes, uint32_t* err_flag, void* stream) {
   if (q_dtype < PA_F32 || q_dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (!pool_types_ok(q_dtype, k_dtype, v_dtype)) return PA_ERR_DTYPE;
+  const bool k_fp8 = k_dtype == PA_FP8_E4M3, v_fp8 = v_dtype == PA_FP8_E4M3;
+  if (!k_fp8) k_scale = 1.f;
+  if (!v_fp8) v_scale = 1.f;
   if (out_dtype != PA_F32 && out_dtype != q_dtype) return PA_ERR_DTYPE;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0 ||
       max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
@@ -192,8 +207,9 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_ALIGN;
 
-  DecodePlan p =
-      plan_decode(kv_dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  // a pool of another type than the query's runs on the CUDA-core kernel
+  DecodePlan p = plan_decode(k_fp8 || v_fp8 ? PA_FP8_E4M3 : q_dtype, B, Hq, Hkv, D, block_size,
+                             max_context_len, partition_size);
   DecodeArgs a{};
   a.out = out; a.out_dtype = out_dtype; a.q = query;
   a.k_cache = key_cache; a.v_cache = value_cache;
@@ -205,7 +221,7 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   a.max_context_len = max_context_len;
   a.P = p.P; a.psize = p.psize;
   a.err_flag = err_flag;
-  const bool tc_path = kv_dtype != PA_FP8_E4M3 && p.kernel == 2;
+  const bool tc_path = p.kernel == 2;
   if (tc_path) {
     const size_t need = tc_workspace_bytes(B, Hq, Hkv, D);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -226,7 +242,7 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int rc;
-  if (kv_dtype == PA_FP8_E4M3) rc = launch_decode_simt_fp8(a, q_dtype, s);
+  if (k_fp8 || v_fp8) rc = launch_decode_simt_kv(a, q_dtype, k_dtype, v_dtype, s);
   else rc = p.kernel == 2 ? launch_decode_tc(a, q_dtype, s) : launch_decode_simt(a, q_dtype, s);
   if (rc == PA_OK && p.P > 1) rc = launch_merge(a, s);
   return rc;
@@ -243,7 +259,7 @@ int pa_decode(void* out, int out_dtype, const void* query, const void* key_cache
               int partition_size, void* workspace, size_t workspace_bytes, uint32_t* err_flag,
               void* stream) {
   if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
-  return decode_impl(out, out_dtype, query, dtype, key_cache, value_cache, dtype, 1.f, 1.f,
+  return decode_impl(out, out_dtype, query, dtype, key_cache, dtype, 1.f, value_cache, dtype, 1.f,
                      block_tables, max_blocks_per_seq, context_lens, B, Hq, Hkv, D, block_size,
                      num_blocks, scale, max_context_len, partition_size, workspace,
                      workspace_bytes, err_flag, stream);
@@ -255,10 +271,24 @@ int pa_decode_fp8(void* out, int out_dtype, const void* query, int q_dtype, cons
                   const int32_t* context_lens, int B, int Hq, int Hkv, int D, int block_size,
                   int num_blocks, float scale, int max_context_len, int partition_size,
                   void* workspace, size_t workspace_bytes, uint32_t* err_flag, void* stream) {
-  return decode_impl(out, out_dtype, query, q_dtype, key_cache, value_cache, PA_FP8_E4M3,
-                     k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens, B, Hq,
+  return decode_impl(out, out_dtype, query, q_dtype, key_cache, PA_FP8_E4M3, k_scale, value_cache,
+                     PA_FP8_E4M3, v_scale, block_tables, max_blocks_per_seq, context_lens, B, Hq,
                      Hkv, D, block_size, num_blocks, scale, max_context_len, partition_size,
                      workspace, workspace_bytes, err_flag, stream);
+}
+
+int pa_decode_kv(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                 int k_dtype, float k_scale, const void* value_cache, int v_dtype, float v_scale,
+                 const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                 int B, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+                 int max_context_len, int partition_size, void* workspace,
+                 size_t workspace_bytes, uint32_t* err_flag, void* stream) {
+  if (k_dtype < PA_F32 || k_dtype > PA_FP8_E4M3 || v_dtype < PA_F32 || v_dtype > PA_FP8_E4M3)
+    return PA_ERR_DTYPE;
+  return decode_impl(out, out_dtype, query, q_dtype, key_cache, k_dtype, k_scale, value_cache,
+                     v_dtype, v_scale, block_tables, max_blocks_per_seq, context_lens, B, Hq, Hkv,
+                     D, block_size, num_blocks, scale, max_context_len, partition_size, workspace,
+                     workspace_bytes, err_flag, stream);
 }
 
 int pa_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype, void* key_cache,
@@ -273,9 +303,28 @@ int pa_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype, 
   if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
   if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_ALIGN;
-  return launch_reshape_and_cache_fp8(key, value, src_dtype, key_cache, value_cache, k_scale,
+  return launch_reshape_and_cache_kv(key, value, src_dtype, key_cache, 1, k_scale, value_cache, 1,
                                       v_scale, slot_mapping, T, Hkv, D, block_size, num_blocks,
                                       err_flag, static_cast<cudaStream_t>(stream));
+}
+
+int pa_reshape_and_cache_kv(const void* key, const void* value, int src_dtype, void* key_cache,
+                            int k_dtype, float k_scale, void* value_cache, int v_dtype,
+                            float v_scale, const int64_t* slot_mapping, int T, int Hkv, int D,
+                            int block_size, int num_blocks, uint32_t* err_flag, void* stream) {
+  if (src_dtype < PA_F32 || src_dtype > PA_BF16) return PA_ERR_DTYPE;
+  const bool kf = k_dtype == PA_FP8_E4M3, vf = v_dtype == PA_FP8_E4M3;
+  if ((!kf && k_dtype != src_dtype) || (!vf && v_dtype != src_dtype)) return PA_ERR_DTYPE;
+  if (T < 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0) return PA_ERR_SHAPE;
+  if ((kf && !scale_ok(k_scale)) || (vf && !scale_ok(v_scale))) return PA_ERR_SHAPE;
+  if (!supported_shape(Hkv, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (T == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PA_ERR_ALIGN;
+  return launch_reshape_and_cache_kv(key, value, src_dtype, key_cache, kf, k_scale, value_cache,
+                                     vf, v_scale, slot_mapping, T, Hkv, D, block_size, num_blocks,
+                                     err_flag, static_cast<cudaStream_t>(stream));
 }
 
 size_t pa_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len,
@@ -307,7 +356,7 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   const bool share = max_shared_blocks > 0 && num_groups > 0 && B > 0 &&
                      prefix_tc_supported(dtype, Hq, Hkv, D, block_size);
   if (!share)   // nothing shared, or a shape the prefix kernel does not take: plain decode
-    return decode_impl(out, out_dtype, query, dtype, key_cache, value_cache, dtype, 1.f, 1.f,
+    return decode_impl(out, out_dtype, query, dtype, key_cache, dtype, 1.f, value_cache, dtype, 1.f,
                        block_tables, max_blocks_per_seq, context_lens, B, Hq, Hkv, D, block_size,
                        num_blocks, scale, max_context_len, partition_size, workspace,
                        workspace_bytes, err_flag, stream);

@@ -60,6 +60,37 @@ template <> __device__ __forceinline__ void widen16<__nv_fp8_e4m3>(const uint4& 
   }
 }
 
+// One lane's slice of a K or V row: 8 or 16 bytes, loaded in one instruction.
+template <int NB> struct Raw;
+template <> struct Raw<16> { using T = uint4; };
+template <> struct Raw<8> { using T = uint2; };
+
+template <int NB> __device__ __forceinline__ typename Raw<NB>::T raw_zero();
+template <> __device__ __forceinline__ uint4 raw_zero<16>() { return make_uint4(0, 0, 0, 0); }
+template <> __device__ __forceinline__ uint2 raw_zero<8>() { return make_uint2(0, 0); }
+
+// Widen E elements of type T held in E * sizeof(T) raw bytes to fp32.
+template <typename T, int E>
+__device__ __forceinline__ void widen_raw(const typename Raw<E * (int)sizeof(T)>::T& v, float* f) {
+  if constexpr (E * sizeof(T) == 16) {
+    widen16<T>(v, f);
+  } else {
+    static_assert(sizeof(T) == 1 && E == 8, "8-byte slices hold 8 FP8 codes");
+    const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(
+            static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * k)) & 0xffffu), __NV_E4M3);
+        const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        f[4 * i + 2 * k] = t.x;
+        f[4 * i + 2 * k + 1] = t.y;
+      }
+    }
+  }
+}
+
 // Round fp32 to the output type (round to nearest even) and store.
 __device__ __forceinline__ void store_out(void* base, size_t i, float x, int out_dtype) {
   if (out_dtype == PA_F32) reinterpret_cast<float*>(base)[i] = x;
@@ -73,6 +104,17 @@ __device__ __forceinline__ uint4 ld_stream16(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
+}
+
+__device__ __forceinline__ uint2 ld_stream8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+template <int NB> __device__ __forceinline__ typename Raw<NB>::T ld_stream(const void* p) {
+  if constexpr (NB == 16) return ld_stream16(p);
+  else return ld_stream8(p);
 }
 
 __device__ __forceinline__ void flag_error(uint32_t* err_flag, uint32_t bit) {

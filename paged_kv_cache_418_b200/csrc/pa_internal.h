@@ -67,8 +67,10 @@ DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max
 size_t workspace_bytes_for(int B, int Hq, int D, int P);
 
 int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream);
-// FP8 E4M3 pools, query of q_dtype
-int launch_decode_simt_fp8(const DecodeArgs& a, int q_dtype, cudaStream_t stream);
+// Pools whose element types differ from the query's: both FP8 E4M3 (any query
+// type), or one FP8 and the other of the query's 16-bit type.
+int launch_decode_simt_kv(const DecodeArgs& a, int q_dtype, int k_dtype, int v_dtype,
+                          cudaStream_t stream);
 int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream);
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 // Shapes the tensor-core path can take for some 16-bit element type and block size.
@@ -110,11 +112,13 @@ int launch_reshape_and_cache(const void* key, const void* value, void* key_cache
 int launch_copy_blocks(void* key_cache, void* value_cache, int esize,
                        const int64_t* block_mapping, int num_pairs, int Hkv, int D,
                        int block_size, int num_blocks, uint32_t* err_flag, cudaStream_t stream);
-int launch_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype,
-                                 void* key_cache, void* value_cache, float k_scale,
-                                 float v_scale, const int64_t* slot_mapping, int T, int Hkv,
-                                 int D, int block_size, int num_blocks, uint32_t* err_flag,
-                                 cudaStream_t stream);
+// Scatter with one element type per pool: a pool of the source type gets the
+// row copied, an FP8 pool gets it quantised (code = E4M3(x / scale)).
+int launch_reshape_and_cache_kv(const void* key, const void* value, int src_dtype,
+                                void* key_cache, int k_fp8, float k_scale, void* value_cache,
+                                int v_fp8, float v_scale, const int64_t* slot_mapping, int T,
+                                int Hkv, int D, int block_size, int num_blocks,
+                                uint32_t* err_flag, cudaStream_t stream);
 int launch_swap_blocks(void* dst_key, void* dst_value, const void* src_key,
                        const void* src_value, int esize, const int64_t* block_mapping,
                        int num_pairs, int Hkv, int D, int block_size, int src_blocks,

@@ -65,6 +65,11 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_shared_prefix.restype = I
     lib.pa_prefill.argtypes = [P, I, P, P, P, I, P, I, P, P, I, I, I, I, I, I, I, I, F, I, P, P]
     lib.pa_prefill.restype = I
+    lib.pa_decode_kv.argtypes = [P, I, P, I, P, I, F, P, I, F, P, I, P, I, I, I, I, I, I, F, I, I,
+                                 P, S, P, P]
+    lib.pa_decode_kv.restype = I
+    lib.pa_reshape_and_cache_kv.argtypes = [P, P, I, P, I, F, P, I, F, P, I, I, I, I, I, P, P]
+    lib.pa_reshape_and_cache_kv.restype = I
     return lib
 
 
@@ -263,6 +268,49 @@ def pa_reshape_and_cache_fp8(key: torch.Tensor, value: torch.Tensor, key_cache: 
                                           _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_reshape_and_cache_fp8", rc)
+
+
+def pa_decode_kv(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                 value_cache: torch.Tensor, k_scale: float, v_scale: float,
+                 block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                 max_context_len: int, partition_size: int = 0,
+                 workspace: Optional[torch.Tensor] = None,
+                 err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out [B,Hq,D] <- paged decode attention with one element type per pool
+    (uint8 = FP8 E4M3 codes read times the pool's scale; see pa_decode_kv)."""
+    B, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    with _on_device_of(query):
+        rc = LIB.pa_decode_kv(
+            _ptr(out), pa_dtype(out), _ptr(query), pa_dtype(query), _ptr(key_cache),
+            pa_dtype(key_cache), float(k_scale), _ptr(value_cache), pa_dtype(value_cache),
+            float(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), B, Hq,
+            Hkv, D, block_size, num_blocks, float(scale), int(max_context_len),
+            int(partition_size), _ptr(workspace),
+            0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_decode_kv", rc)
+
+
+def pa_reshape_and_cache_kv(key: torch.Tensor, value: torch.Tensor, key_cache: torch.Tensor,
+                            value_cache: torch.Tensor, k_scale: float, v_scale: float,
+                            slot_mapping: torch.Tensor, err_flag: Optional[torch.Tensor] = None,
+                            stream=None) -> None:
+    """Scatter new K/V rows [T,Hkv,D] into pools of per-pool types (an FP8 pool
+    gets E4M3 codes of x / scale, a pool of the rows' type gets them copied)."""
+    if DEBUG:
+        check_slot_mapping(slot_mapping, "pa_reshape_and_cache_kv")
+    num_blocks, block_size, Hkv, D = key_cache.shape
+    T = slot_mapping.shape[0]
+    with _on_device_of(key_cache):
+        rc = LIB.pa_reshape_and_cache_kv(_ptr(key), _ptr(value), pa_dtype(key), _ptr(key_cache),
+                                         pa_dtype(key_cache), float(k_scale), _ptr(value_cache),
+                                         pa_dtype(value_cache), float(v_scale),
+                                         _ptr(slot_mapping), T, Hkv, D, block_size, num_blocks,
+                                         _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_reshape_and_cache_kv", rc)
 
 
 def pa_swap_blocks(dst_key: torch.Tensor, dst_value: torch.Tensor, src_key: torch.Tensor,

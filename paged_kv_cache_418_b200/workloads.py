@@ -126,22 +126,31 @@ class Workload:
     block_mapping: np.ndarray   # [P, 2] int64 (src, dst) copy-on-write pairs
     seed: int = 0
     meta: Dict = field(default_factory=dict)
-    kv_dtype: int = -1          # pool element type: dtype, or FP8 (codes times the scales)
+    kv_dtype: int = -1          # K pool element type: dtype, or FP8 (codes times k_scale)
     k_scale: float = 1.0
     v_scale: float = 1.0
+    v_dtype: int = -1           # V pool element type (default: the K pool's)
 
     def __post_init__(self):
         if self.kv_dtype < 0:
             self.kv_dtype = self.dtype
+        if self.v_dtype < 0:
+            self.v_dtype = self.kv_dtype
 
     @property
     def fp8(self) -> bool:
-        return self.kv_dtype == FP8
+        """Some pool holds FP8 codes."""
+        return self.kv_dtype == FP8 or self.v_dtype == FP8
+
+    @property
+    def mixed(self) -> bool:
+        """The K and V pools hold different element types."""
+        return self.kv_dtype != self.v_dtype
 
     @property
     def esize(self) -> int:
-        """Bytes per cached K/V element."""
-        return ESIZE[self.kv_dtype]
+        """Bytes per cached K/V element (the average of the two pools)."""
+        return (ESIZE[self.kv_dtype] + ESIZE[self.v_dtype]) // 2
 
     @property
     def G(self) -> int:
@@ -153,7 +162,8 @@ class Workload:
 
     def kv_bytes(self) -> int:
         """Algorithmic K+V bytes one decode pass must read (attended tokens only)."""
-        return kv_bytes_for(self.context_lens, self.Hkv, self.D, self.esize)
+        tokens = int(np.asarray(self.context_lens, dtype=np.int64).sum())
+        return tokens * self.Hkv * self.D * (ESIZE[self.kv_dtype] + ESIZE[self.v_dtype])
 
     def unique_kv_bytes(self) -> int:
         """K+V bytes of the distinct physical slots attended (shared blocks once)."""
@@ -164,7 +174,7 @@ class Workload:
             for i in range((n + bs - 1) // bs):
                 slots.add((int(self.block_tables[b, i]), min(bs, n - i * bs)))
         rows = sum(r for _, r in slots)
-        return rows * self.Hkv * self.D * 2 * self.esize
+        return rows * self.Hkv * self.D * (ESIZE[self.kv_dtype] + ESIZE[self.v_dtype])
 
 
 def kv_bytes_for(context_lens, Hkv: int, D: int, esize: int) -> int:
@@ -195,12 +205,15 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
                       partition_size: int = 0, shuffle: bool = True,
                       k_boost_frac: float = 0.0, k_boost: float = 8.0,
                       kv_fp8: bool = False, k_scale: float = 0.3,
-                      v_scale: float = 0.7) -> Workload:
+                      v_scale: float = 0.7, v_fp8: Optional[bool] = None) -> Workload:
     """Independent sequences, each prefilled with ctx-1 tokens plus one append.
 
     kv_fp8: the pools hold E4M3 codes (value = code * k_scale / v_scale,
     scales rounded to float32); the query and the new rows keep ``dtype``.
+    v_fp8 (default kv_fp8) sets the V pool apart: kv_fp8=True, v_fp8=False
+    is an FP8 K pool beside a V pool of ``dtype``.
     """
+    v_fp8 = kv_fp8 if v_fp8 is None else bool(v_fp8)
     if Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
     rng = rng if rng is not None else np.random.Generator(np.random.PCG64(seed))
@@ -235,23 +248,26 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
         tables[b, :len(tb)] = tb
 
     st = _STORAGE[dtype]
-    kvdt = FP8 if kv_fp8 else dtype
+    kdt = FP8 if kv_fp8 else dtype
+    vdt = FP8 if v_fp8 else dtype
     q = round_to_storage(rng.standard_normal((B, Hq, D), dtype=np.float32), dtype).view(st)
-    kc = nan_fill((num_blocks, block_size, Hkv, D), kvdt)
-    vc = nan_fill((num_blocks, block_size, Hkv, D), kvdt)
+    kc = nan_fill((num_blocks, block_size, Hkv, D), kdt)
+    vc = nan_fill((num_blocks, block_size, Hkv, D), vdt)
     for b in range(B):
         n = int(ctx[b]) - 1
         if kv_fp8:
             _fill_rows(kc, tables[b], block_size, 0, random_e4m3_codes(rng, (n, Hkv, D)))
+        else:
+            k = rng.standard_normal((n, Hkv, D), dtype=np.float32)
+            if k_boost_frac > 0.0:
+                k *= np.where(rng.random((n, Hkv, 1)) < k_boost_frac, np.float32(k_boost),
+                              np.float32(1.0))
+            _fill_rows(kc, tables[b], block_size, 0, round_to_storage(k, dtype).view(st))
+        if v_fp8:
             _fill_rows(vc, tables[b], block_size, 0, random_e4m3_codes(rng, (n, Hkv, D)))
-            continue
-        k = rng.standard_normal((n, Hkv, D), dtype=np.float32)
-        if k_boost_frac > 0.0:
-            k *= np.where(rng.random((n, Hkv, 1)) < k_boost_frac, np.float32(k_boost),
-                          np.float32(1.0))
-        _fill_rows(kc, tables[b], block_size, 0, round_to_storage(k, dtype).view(st))
-        v = rng.standard_normal((n, Hkv, D), dtype=np.float32)
-        _fill_rows(vc, tables[b], block_size, 0, round_to_storage(v, dtype).view(st))
+        else:
+            v = rng.standard_normal((n, Hkv, D), dtype=np.float32)
+            _fill_rows(vc, tables[b], block_size, 0, round_to_storage(v, dtype).view(st))
     nk = round_to_storage(rng.standard_normal((B, Hkv, D), dtype=np.float32), dtype).view(st)
     nv = round_to_storage(rng.standard_normal((B, Hkv, D), dtype=np.float32), dtype).view(st)
     return Workload(
@@ -261,8 +277,8 @@ def build_decode_case(name: str, dtype: int, B: int, Hq: int, Hkv: int, D: int,
         partition_size=int(partition_size), q=q, k_cache=kc, v_cache=vc,
         block_tables=tables, context_lens=ctx.astype(np.int32), new_key=nk, new_value=nv,
         slot_mapping=slots, block_mapping=np.zeros((0, 2), dtype=np.int64), seed=seed,
-        kv_dtype=kvdt, k_scale=float(np.float32(k_scale)) if kv_fp8 else 1.0,
-        v_scale=float(np.float32(v_scale)) if kv_fp8 else 1.0)
+        kv_dtype=kdt, k_scale=float(np.float32(k_scale)) if kv_fp8 else 1.0,
+        v_scale=float(np.float32(v_scale)) if v_fp8 else 1.0, v_dtype=vdt)
 
 
 # --------------------------------------------------------------------------
@@ -484,6 +500,8 @@ WORKLOADS = {
     4: "long-context-splitk-bf16",
     5: "shared-prefix-sampling-bf16",
     6: "llama2-7b-fp8kv",
+    7: "llama2-7b-fp8k-bf16v",
+    8: "llama3-70b-gqa-fp8kv",
 }
 WORKLOAD_IDS = {v: k for k, v in WORKLOADS.items()}
 
@@ -509,7 +527,7 @@ def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None
     k = WORKLOAD_IDS[which] if isinstance(which, str) else int(which)
     seed = 1000 + k if seed is None else int(seed)
     name = WORKLOADS[k] if batch is None else f"{WORKLOADS[k]}-b{int(batch)}"
-    if batch is not None and k in (2, 3, 4, 5, 6):
+    if batch is not None and k in (2, 3, 4, 5, 6, 7, 8):
         return _make_batch(k, name, seed, int(batch))
     if k == 1:
         return build_decode_case(name, F32, B=4, Hq=4, Hkv=4, D=64, block_size=16,
@@ -543,6 +561,19 @@ def make_workload(which, seed: Optional[int] = None, batch: Optional[int] = None
         return build_decode_case(name, F16, B=64, Hq=32, Hkv=32, D=128, block_size=16,
                                  num_blocks=8192, context_lens=ctx, seed=seed, rng=rng,
                                  max_blocks=128, kv_fp8=True)
+    if k == 7:
+        # the same batch with the explainer's mixed cache: K in FP8, V and query in bf16
+        ctx = rng.integers(128, 2049, size=64)
+        return build_decode_case(name, BF16, B=64, Hq=32, Hkv=32, D=128, block_size=16,
+                                 num_blocks=8192, context_lens=ctx, seed=seed, rng=rng,
+                                 max_blocks=128, kv_fp8=True, v_fp8=False)
+    if k == 8:
+        # the Llama-3-70B-shaped GQA batch with an FP8 E4M3 cache (bf16 query)
+        ln = rng.lognormal(mean=math.log(1200.0), sigma=0.8, size=128)
+        ctx = np.clip(np.rint(ln), 16, 8192).astype(np.int64)
+        return build_decode_case(name, BF16, B=128, Hq=64, Hkv=8, D=128, block_size=16,
+                                 num_blocks=65536, context_lens=ctx, seed=seed, rng=rng,
+                                 max_blocks=512, kv_fp8=True)
     raise KeyError(which)
 
 
@@ -563,17 +594,18 @@ def _make_contiguous(k: int, seed: int) -> Workload:
 
 def _make_batch(k: int, name: str, seed: int, B: int) -> Workload:
     rng = np.random.Generator(np.random.PCG64(seed))
-    if k in (2, 6):
+    if k in (2, 6, 7):
         ctx = rng.integers(128, 2049, size=B)
-        return build_decode_case(name, F16, B=B, Hq=32, Hkv=32, D=128, block_size=16,
-                                 num_blocks=B * 128, context_lens=ctx, seed=seed, rng=rng,
-                                 max_blocks=128, kv_fp8=k == 6)
-    if k == 3:
+        return build_decode_case(name, BF16 if k == 7 else F16, B=B, Hq=32, Hkv=32, D=128,
+                                 block_size=16, num_blocks=B * 128, context_lens=ctx, seed=seed,
+                                 rng=rng, max_blocks=128, kv_fp8=k in (6, 7), v_fp8=k == 6)
+    if k in (3, 8):
         ln = rng.lognormal(mean=math.log(1200.0), sigma=0.8, size=B)
         ctx = np.clip(np.rint(ln), 16, 8192).astype(np.int64)
         return build_decode_case(name, BF16, B=B, Hq=64, Hkv=8, D=128, block_size=16,
                                  num_blocks=max(512, 2 * int(sum((c + 15) // 16 for c in ctx))),
-                                 context_lens=ctx, seed=seed, rng=rng, max_blocks=512)
+                                 context_lens=ctx, seed=seed, rng=rng, max_blocks=512,
+                                 kv_fp8=k == 8)
     if k == 4:
         return build_decode_case(name, BF16, B=B, Hq=64, Hkv=8, D=128, block_size=32,
                                  num_blocks=B * 2048, context_lens=[32768] * B, seed=seed,
@@ -621,12 +653,21 @@ def shrink_workload(which, seed: int, B: Optional[int] = None, max_ctx: Optional
                                         children=4, prefix_blocks=4, Hq=32, Hkv=8, D=128,
                                         block_size=16, num_blocks=96, max_suffix=40,
                                         seed=seed)
-    if k == 6:
+    if k in (6, 7):
         B = B or 6
         hi = max_ctx or 300
         ctx = rng.integers(1, hi + 1, size=B)
         nb = int(sum((c + 15) // 16 for c in ctx)) + 7
-        return build_decode_case("llama2-7b-fp8kv-small", F16, B=B, Hq=32, Hkv=32, D=128,
+        return build_decode_case(WORKLOADS[k] + "-small", F16 if k == 6 else BF16, B=B, Hq=32,
+                                 Hkv=32, D=128, block_size=16, num_blocks=nb, context_lens=ctx,
+                                 seed=seed, rng=rng, kv_fp8=True, v_fp8=k == 6)
+    if k == 8:
+        B = B or 6
+        hi = max_ctx or 700
+        ln = rng.lognormal(mean=math.log(hi / 3.0), sigma=0.8, size=B)
+        ctx = np.clip(np.rint(ln), 1, hi).astype(np.int64)
+        nb = int(sum((c + 15) // 16 for c in ctx)) + 5
+        return build_decode_case("llama3-70b-gqa-fp8kv-small", BF16, B=B, Hq=64, Hkv=8, D=128,
                                  block_size=16, num_blocks=nb, context_lens=ctx, seed=seed,
                                  rng=rng, kv_fp8=True)
     raise KeyError(which)

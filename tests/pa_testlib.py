@@ -37,7 +37,10 @@ def device_step(w: Workload, t=None, out_dtype=None, partition_size=None, err=No
     if do_cache_ops:
         if len(w.block_mapping):
             ops.pa_copy_blocks(t["k_cache"], t["v_cache"], t["block_mapping"], err, stream)
-        if w.fp8:
+        if w.mixed:
+            ops.pa_reshape_and_cache_kv(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                        w.k_scale, w.v_scale, t["slot_mapping"], err, stream)
+        elif w.fp8:
             ops.pa_reshape_and_cache_fp8(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
                                          w.k_scale, w.v_scale, t["slot_mapping"], err, stream)
         else:
@@ -48,7 +51,11 @@ def device_step(w: Workload, t=None, out_dtype=None, partition_size=None, err=No
     psize = w.partition_size if partition_size is None else partition_size
     mcl = w.max_context_len if max_context_len is None else max_context_len
     ws = ops.workspace_for(t["q"], t["k_cache"], mcl, psize)
-    if w.fp8:
+    if w.mixed:
+        ops.pa_decode_kv(out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
+                         t["block_tables"], t["context_lens"], w.scale, mcl, psize, ws, err,
+                         stream)
+    elif w.fp8:
         ops.pa_decode_fp8(out, t["q"], t["k_cache"], t["v_cache"], w.k_scale, w.v_scale,
                           t["block_tables"], t["context_lens"], w.scale, mcl, psize, ws, err,
                           stream)
@@ -65,13 +72,20 @@ def oracle_step(w: Workload, rows=None, do_cache_ops=True):
     kc, vc = w.k_cache.copy(), w.v_cache.copy()
     if do_cache_ops:
         if len(w.block_mapping):
+            assert not w.mixed, "copy-on-write pairs over pools of two element types"
             oracle.copy_blocks(kc, vc, w.block_mapping, w.kv_dtype)
-        if w.fp8:
+        if w.mixed:
+            oracle.reshape_and_cache_mixed(kc, vc, w.new_key, w.new_value, w.dtype, w.kv_dtype,
+                                           w.v_dtype, w.k_scale, w.v_scale, w.slot_mapping)
+        elif w.fp8:
             oracle.reshape_and_cache_fp8(kc, vc, w.new_key, w.new_value, w.dtype, w.k_scale,
                                          w.v_scale, w.slot_mapping)
         else:
             oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
-    if w.fp8:
+    if w.mixed:
+        out = oracle.decode_mixed(w.q, w.dtype, kc, w.kv_dtype, w.k_scale, vc, w.v_dtype,
+                                  w.v_scale, w.block_tables, w.context_lens, w.scale, rows=rows)
+    elif w.fp8:
         out = oracle.decode_kv(w.q, w.dtype, kc, vc, FP8, w.k_scale, w.v_scale, w.block_tables,
                                w.context_lens, w.scale, rows=rows)
     else:
