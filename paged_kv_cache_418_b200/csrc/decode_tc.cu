@@ -58,8 +58,9 @@
 //   warp 8     TMA producer (one lane): Q of the unit, K and V tiles through a
 //              ring of 32 KB stages;
 //   warp 9     MMA issuer (one lane): S(t), then O(t-1).
-// Every pipeline wait is bounded (DecodeArgs::wait_ns, 1 s unless a caller's
-// test shortens it); a wait that gives up sets the PA_DEV_TIMEOUT bit, raises
+// Every pipeline wait is bounded (DecodeArgs::wait_ns, 1 s unless a test
+// shortens it; the timeout-path test also withholds one query load, so that a
+// wait can only run out); a wait that gives up sets the PA_DEV_TIMEOUT bit, raises
 // a CTA-wide abort flag, and all roles leave their loops (the softmax warps
 // of a group only together, at a named-barrier vote), wait for their own
 // asynchronous work (those waits keep the full 1 s bound, so no copy or MMA is
@@ -497,6 +498,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int tc = 0, issued = 0;
+      int q_last[2] = {-1, -1};                    // last unit whose query went to buffer 0 / 1
       int phys_next[NQ];
       // block ids of the tile at p (-1 past the share's end)
       auto load_ids = [&](const TilePos& p, int* ph) {
@@ -520,10 +522,13 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         const Unit x = unit_of(cur);
         const int qi = i & 1;
         if (!mbar_wait(bar(Bx::QEMPTY + qi), ((i >> 1) & 1) ^ 1, abort_flag, wait_ns)) { give_up(); goto prod_done; }
-        mbar_expect_tx(bar(Bx::QFULL + qi), 2u * NS * 128u);
-        for (int hh = 0; hh < 2; ++hh)
-          tma_load_2d(sbase + S::OFF_Q + qi * S::kQBytes + hh * (NS * 128), &tmQ, hh * 64,
-                      x.b * a.Hq + x.h * kHG * G, bar(Bx::QFULL + qi));
+        if (!(a.test_withhold_q && i == 0)) {
+          mbar_expect_tx(bar(Bx::QFULL + qi), 2u * NS * 128u);
+          for (int hh = 0; hh < 2; ++hh)
+            tma_load_2d(sbase + S::OFF_Q + qi * S::kQBytes + hh * (NS * 128), &tmQ, hh * 64,
+                        x.b * a.Hq + x.h * kHG * G, bar(Bx::QFULL + qi));
+          q_last[qi] = i;
+        }
         for (int k = 0; k < x.ntiles; ++k) {
           int ts, te, nql;
           tile_span(x, k, ts, te, nql);
@@ -555,11 +560,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         }
       }
     prod_done:
-      // never leave with copies in flight: wait (bounded) for the last loads of every stage
+      // never leave with copies in flight: wait (bounded) for the last loads of
+      // every stage and of both query buffers
       for (int seq = max(0, issued - NST); seq < issued; ++seq) {
         const int s = seq % NST;
         const uint64_t t0 = globaltimer();
         while (!mbar_try(bar(Bx::FULL + s), (seq / NST) & 1) && globaltimer() - t0 < kWaitNs) {}
+      }
+      for (int qb = 0; qb < 2; ++qb) {
+        if (q_last[qb] < 0) continue;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(bar(Bx::QFULL + qb), (q_last[qb] >> 1) & 1) && globaltimer() - t0 < kWaitNs) {}
       }
     }
   } else if (warp == 9) {

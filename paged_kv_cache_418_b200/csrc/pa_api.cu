@@ -58,6 +58,13 @@ unsigned long long tc_wait_ns() {
   return (end && *end == 0 && v <= 1000000000ull) ? v : 1000000000ull;
 }
 
+// The timeout-path test's hook (PA_TC_TEST_WITHHOLD_Q=1): the tensor-core
+// kernel leaves the first unit's query unloaded, so the wait for it runs out.
+int tc_test_withhold_q() {
+  const char* s = std::getenv("PA_TC_TEST_WITHHOLD_Q");
+  return s && s[0] == '1' ? 1 : 0;
+}
+
 // A number per call of the tensor-core path (40 bits; its tickets carry it).
 unsigned long long next_epoch() {
   static std::atomic<unsigned long long> n{
@@ -229,6 +236,7 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
     tc_carve(a, static_cast<char*>(workspace));
     a.epoch = next_epoch();
     a.wait_ns = tc_wait_ns();
+    a.test_withhold_q = tc_test_withhold_q();
   } else if (p.P > 1) {
     const size_t need = workspace_bytes_for(B, Hq, D, p.P);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -411,6 +419,7 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
     tc_carve(a, w + part_bytes);
     a.epoch = next_epoch();
     a.wait_ns = tc_wait_ns();
+    a.test_withhold_q = tc_test_withhold_q();
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, st) : launch_decode_simt(a, dtype, st);

@@ -296,11 +296,11 @@ def test_even_split_pieces_merge_to_the_oracle(ctx, G, mcl):
 
 
 def test_pipeline_wait_limit_runs_out_and_the_next_launch_is_correct(monkeypatch):
-    """With the tensor-core kernel's pipeline-wait limit at 0 ns every wait that
-    is not already satisfied gives up: the launch reports PA_DEV_TIMEOUT (its
-    outputs are unspecified), every CTA drains its own copies and products,
-    frees tensor memory and returns; the next launch on the same stream, with
-    the normal limit, matches the oracle."""
+    """The tensor-core kernel's pipeline waits are bounded. Here one CTA's first
+    query load is withheld, so the wait for it can only run out (after 1 ms):
+    the launch reports PA_DEV_TIMEOUT (its outputs are unspecified), every CTA
+    drains its own copies and products, frees tensor memory and returns; the
+    next launch on the same stream, with the normal limit, matches the oracle."""
     w = _tc_case([700, 45, 1300], seed=5)
     t = device_inputs(w)
     ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
@@ -308,12 +308,14 @@ def test_pipeline_wait_limit_runs_out_and_the_next_launch_is_correct(monkeypatch
     ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len)
     out = torch.zeros((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    monkeypatch.setenv("PA_TC_WAIT_NS", "0")
+    monkeypatch.setenv("PA_TC_WAIT_NS", "1000000")
+    monkeypatch.setenv("PA_TC_TEST_WITHHOLD_Q", "1")
     ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
                   w.scale, w.max_context_len, 0, ws, err)
     torch.cuda.synchronize()
     assert int(err.item()) & 16, "no wait ran out"
     monkeypatch.delenv("PA_TC_WAIT_NS")
+    monkeypatch.delenv("PA_TC_TEST_WITHHOLD_Q")
     out = _decode_with(w, t, ws)
     ref, _, _ = oracle_step(w)
     assert_attention_close(out, ref, w.dtype, "after a timed-out launch")
