@@ -455,11 +455,17 @@ int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cach
   p.k_cache = key_cache; p.v_cache = value_cache; p.dtype = dtype;
   p.block_tables = block_tables; p.max_blocks = max_blocks_per_seq;
   p.context_lens = context_lens; p.query_start = query_start;
-  p.B = B; p.max_query_len = max_query_len; p.Hq = Hq; p.Hkv = Hkv; p.bs = block_size;
+  p.B = B; p.T = T; p.max_query_len = max_query_len; p.Hq = Hq; p.Hkv = Hkv; p.bs = block_size;
   p.num_blocks = num_blocks;
   p.scale_log2 = scale * kLog2e;
   p.max_context_len = max_context_len;
   p.err_flag = err_flag;
+  // the kernel with the query rows on the MMA's M, unless PA_PREFILL_KERNEL=mq
+  // asks for the multi-query kernel (for measurements)
+  const char* ov = std::getenv("PA_PREFILL_KERNEL");
+  const bool mq = ov && !std::strcmp(ov, "mq");
+  if (!mq && prefill_fa_supported(dtype, Hq, Hkv, D, block_size))
+    return launch_prefill_fa(p, static_cast<cudaStream_t>(stream));
   return launch_prefill_tc(p, static_cast<cudaStream_t>(stream));
 }
 

@@ -97,12 +97,15 @@ struct PrefillLaunch {
   int max_blocks;
   const int32_t* context_lens;  // [B] tokens in the cache after the chunk
   const int32_t* query_start;   // [B + 1]
-  int B, max_query_len, Hq, Hkv, bs, num_blocks;
+  int B, T, max_query_len, Hq, Hkv, bs, num_blocks;
   float scale_log2;
   int max_context_len;
   uint32_t* err_flag;
 };
 int launch_prefill_tc(const PrefillLaunch& p, cudaStream_t stream);
+// Paged prefill with the query rows on the MMA's M (prefill_tc.cu).
+bool prefill_fa_supported(int dtype, int Hq, int Hkv, int D, int bs);
+int launch_prefill_fa(const PrefillLaunch& p, cudaStream_t stream);
 int launch_prefix_tc(const DecodeArgs& a, int dtype, const int32_t* group_offsets,
                      const int32_t* group_members, int num_groups, int max_group_size, int parts,
                      int part_tokens, cudaStream_t stream);

@@ -1,0 +1,590 @@
+// prefill_tc.cu -- paged (chunked) prefill attention on the 5th-generation
+// tensor cores with the query rows on the MMA's M.
+//
+// A chunk of a sequence's new query tokens attends, causally, to the
+// sequence's cached tokens through its block table ("推理引擎内部机制——
+// PagedAttention、连续批处理、分块预填充", chunked prefill: a long prompt is cut
+// into chunks that run between decode steps). New token i of a chunk of n at
+// the end of a context of ctx tokens sits at position ctx - n + i and attends
+// positions 0 .. ctx - n + i.
+//
+// Work unit = (sequence b, chunk of TPU = 128 / G new tokens, KV head h).
+// Its 128 query rows are (token t, query head g of the group of h), row
+// r = t * G + g: one TMA box of the query [T][Hq][128] brings them in that
+// order. Tile = 128 keys of head h: one TMA box per physical block and 64-wide
+// d-half, 128-byte swizzled (block-sized boxes; a head's rows of a block are
+// contiguous, the heads of a block are not). Per tile:
+//   S[128 rows x 128 keys]  = Q . K_tile^T          (tensor memory, fp32)
+//   O[128 rows x 128 d]    += P_hi . V_tile + P_lo . V_tile
+// where the weights P (in tensor memory, written over S) enter as two 16-bit
+// parts, p = hi + lo, hi = RN(p), lo = RN(p - hi) (~16 significant bits, as
+// in the decode kernels), and the A operand of the output products is read
+// from tensor memory.
+//
+// A softmax thread owns one query row: it reads its row of S (128 scores)
+// into registers, so the row maximum and the row sum need no exchange with
+// other threads. The reference maximum of a row is its first tile's maximum
+// and moves only when a later tile exceeds it by 2^64 (then the row's O is
+// rescaled in tensor memory, which its own thread does); references are
+// floored at -FLT_MAX so masked scores (-inf) give weight 0 without a guard.
+// Keys past a row's position are masked; the V rows of keys that no row of
+// the unit attends (past its last position, or in a block with a bad id) are
+// zeroed in shared memory before the output product, so they add exact zeros.
+//
+// CTA = 6 warps, persistent over units u = blockIdx.x + k * gridDim.x (the
+// chunks late in their sequences, which attend the most keys, first):
+//   warps 0-3  softmax and epilogue (thread = query row = TMEM lane);
+//   warp 4     TMA producer: the unit's query (double-buffered by unit), the
+//              K and V tiles through a ring of 32 KB stages;
+//   warp 5     MMA issuer and owner of the tensor memory: S(t), then the
+//              output product of tile t - 1 (S is double-buffered by tile, O
+//              by unit, so a unit's epilogue overlaps the next unit's tiles).
+// Every pipeline wait is bounded (1 s); one that gives up sets PA_DEV_TIMEOUT,
+// raises the CTA's abort flag, and every role drains its asynchronous work,
+// frees tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <cfloat>
+#include <cstdlib>
+
+#include "pa_internal.h"
+#include "tc_ptx.cuh"
+
+namespace pa {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kD = 128;
+constexpr int kM = 128;                         // query rows per unit (the MMA's M)
+constexpr int kTile = 128;                      // keys per tile
+constexpr int kHalf = 128 * 128;                // one 64-wide d-half of a 128-row operand
+constexpr int kOp = 2 * kHalf;                  // one 128 x 128 16-bit operand: 32 KB
+constexpr int kNST = 4;                         // K / V ring stages
+constexpr int kThreads = 192;
+constexpr float kRescaleLog2 = 64.f;
+
+constexpr int OFF_Q = 0;                        // [2 units][32 KB]
+constexpr int OFF_KV = 2 * kOp;                 // [kNST][32 KB]
+constexpr int OFF_BAR = OFF_KV + kNST * kOp;
+enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY = B_QFULL + 2,
+       B_SFULL = B_QEMPTY + 2, B_PREADY = B_SFULL + 2, B_OSTEP = B_PREADY + 2,
+       B_ODONE = B_OSTEP + 1, B_DONE = B_ODONE + 2, B_COUNT };
+constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
+constexpr int kSmem = OFF_MISC + 16 + 1024;     // + alignment slack
+static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
+constexpr int kTmemCols = 512;                  // S/P x2 (by tile), O x2 (by unit)
+
+struct FaArgs {
+  void* out;
+  int out_dtype;
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* context_lens;
+  const int32_t* query_start;
+  int B, Hq, Hkv, bs, num_blocks, chunks;
+  float scale_log2;
+  int max_context_len;
+  uint32_t* err_flag;
+};
+
+struct FUnit {
+  int b, c, h;
+  int qrow0;            // first query row (token) of the chunk in [T]
+  int ntok;             // new tokens of the chunk (0: nothing to do)
+  int pos0;             // position of the chunk's first token
+  int t1;               // keys [0, t1) are attended by some row
+  int ntiles;
+  bool bad;             // the sequence's lengths are inconsistent
+};
+
+template <int G>
+__device__ __forceinline__ FUnit fa_unit(const FaArgs& a, long long u) {
+  constexpr int TPU = kM / G;
+  FUnit x;
+  x.h = (int)(u % a.Hkv);
+  const long long t = u / a.Hkv;
+  x.b = (int)(t % a.B);
+  x.c = a.chunks - 1 - (int)(t / a.B);
+  const int qs = __ldg(a.query_start + x.b), qe = __ldg(a.query_start + x.b + 1);
+  const int n = qe - qs, ctx = __ldg(a.context_lens + x.b);
+  x.bad = n < 0 || ctx < n || ctx > a.max_blocks * a.bs || ctx > a.max_context_len;
+  x.ntok = x.bad ? 0 : max(0, min(TPU, n - x.c * TPU));
+  x.qrow0 = qs + x.c * TPU;
+  x.pos0 = ctx - n + x.c * TPU;
+  x.t1 = x.ntok > 0 ? x.pos0 + x.ntok : 0;
+  x.ntiles = (x.t1 + kTile - 1) / kTile;
+  return x;
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two fp32 weights -> packed 16-bit hi parts and lo parts (element 0 in the low half).
+template <int FMT>
+__device__ __forceinline__ void split2(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  if (FMT == 1) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(p0 - hf.x, p1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+  } else {
+    const __half2 h = __floats2half2_rn(p0, p1);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(p0 - hf.x, p1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+  }
+}
+
+template <int FMT, int BS, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+  constexpr int NB_T = kTile / BS;               // physical blocks per tile
+  constexpr uint32_t IDESC_S = make_idesc(FMT, 0, 0, kTile, kM);
+  constexpr uint32_t IDESC_O = make_idesc(FMT, 0, 1, kD, kM);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  auto bar = [&](int i) { return sbase + OFF_BAR + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long U = (long long)a.B * a.chunks * a.Hkv;
+  pdl_trigger();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kNST; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_QFULL + i), 1);
+      mbar_init(bar(B_QEMPTY + i), 1);
+      mbar_init(bar(B_SFULL + i), 1);
+      mbar_init(bar(B_PREADY + i), 128);
+      mbar_init(bar(B_ODONE + i), 128);
+    }
+    mbar_init(bar(B_OSTEP), 1);
+    mbar_init(bar(B_DONE), 1);
+    *abort_flag = 0u;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_s = tmem;                  // S/P: [0, 128), [128, 256)
+  const uint32_t tmem_o = tmem + 2 * kTile;      // O: [256, 384), [384, 512)
+  auto give_up = [&]() {
+    *abort_flag = 1u;
+    flag_error(a.err_flag, PA_DEV_TIMEOUT);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int tc_ = 0, issued = 0, ui = 0;
+      int q_last[2] = {-1, -1};
+      for (long long u = blockIdx.x; u < U; u += gridDim.x) {
+        const FUnit x = fa_unit<G>(a, u);
+        if (x.bad && x.c == 0 && x.h == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
+        if (x.ntok <= 0) continue;
+        const int qi = ui & 1;
+        if (!mbar_wait(bar(B_QEMPTY + qi), ((ui >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+        mbar_expect_tx(bar(B_QFULL + qi), (uint32_t)kOp);
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_4d(sbase + OFF_Q + qi * kOp + hh * kHalf, &tmQ, 0, hh, x.h * G, x.qrow0,
+                      bar(B_QFULL + qi));
+        q_last[qi] = ui;
+        const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
+        for (int k = 0; k < x.ntiles; ++k, ++tc_) {
+          const int ts = k * kTile;
+          const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+          int phys[NB_T];
+          uint32_t bytes = 0;
+#pragma unroll
+          for (int q = 0; q < NB_T; ++q) {
+            phys[q] = q < nblk ? __ldg(table + ts / BS + q) : -1;
+            if (q < nblk && (phys[q] < 0 || phys[q] >= a.num_blocks)) {
+              flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+              phys[q] = -1;
+            }
+            if (phys[q] >= 0) bytes += 2u * BS * 128u;
+          }
+          for (int kv = 0; kv < 2; ++kv) {
+            const int seq = 2 * tc_ + kv, s = seq % kNST;
+            if (!mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
+            mbar_expect_tx(bar(B_FULL + s), bytes);
+            const uint32_t dst = sbase + OFF_KV + s * kOp;
+#pragma unroll
+            for (int q = 0; q < NB_T; ++q) {
+              if (phys[q] < 0) continue;
+              for (int hh = 0; hh < 2; ++hh)
+                tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
+                            phys[q], bar(B_FULL + s));
+            }
+            ++issued;
+          }
+        }
+        ++ui;
+      }
+    prod_done:
+      // never leave with copies in flight: the last loads of every stage and query buffer
+      for (int seq = max(0, issued - kNST); seq < issued; ++seq) {
+        const int s = seq % kNST;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(bar(B_FULL + s), (seq / kNST) & 1) && globaltimer() - t0 < kWaitNs) {}
+      }
+      for (int qb = 0; qb < 2; ++qb) {
+        if (q_last[qb] < 0) continue;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try(bar(B_QFULL + qb), (q_last[qb] >> 1) & 1) && globaltimer() - t0 < kWaitNs) {}
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int tc_ = 0, ui = 0;
+      bool ok = true;
+      // output product of tile tt (the unit's first if first) into O buffer ob
+      auto issue_pv = [&](int tt, bool first, int ob) -> bool {
+        const int pb = tt & 1;
+        if (!mbar_wait(bar(B_PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
+        // the O buffer was last used by unit ui - 2: wait for its epilogue
+        if (first && ui >= 2 && !mbar_wait(bar(B_ODONE + ob), ((ui - 2) >> 1) & 1, abort_flag))
+          return false;
+        const int seq = 2 * tt + 1, s = seq % kNST;
+        if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vst = sbase + OFF_KV + s * kOp;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            const uint64_t bd = sw128_desc(vst + kk * 16 * 128, kHalf, 1024);
+            mma_f16_ta(tmem_o + ob * kD, tmem_s + pb * kTile + part * 64 + kk * 8, bd, IDESC_O,
+                       (first && part == 0 && kk == 0) ? 0u : 1u);
+          }
+        }
+        mma_commit(bar(B_EMPTY + s));
+        mma_commit(bar(B_OSTEP));
+        return true;
+      };
+      for (long long u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const FUnit x = fa_unit<G>(a, u);
+        if (x.ntok <= 0) continue;
+        const int qi = ui & 1, ob = ui & 1;
+        if (!mbar_wait(bar(B_QFULL + qi), (ui >> 1) & 1, abort_flag)) { ok = false; break; }
+        const uint32_t qst = sbase + OFF_Q + qi * kOp;
+        for (int k = 0; k < x.ntiles; ++k, ++tc_) {
+          const int sb = tc_ & 1;
+          const int seq = 2 * tc_, s = seq % kNST;
+          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kst = sbase + OFF_KV + s * kOp;
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint64_t ad = sw128_desc(qst + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = sw128_desc(kst + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+            mma_f16(tmem_s + sb * kTile, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(B_EMPTY + s));
+          mma_commit(bar(B_SFULL + sb));
+          if (k == x.ntiles - 1) mma_commit(bar(B_QEMPTY + qi));
+          if (k > 0 && !issue_pv(tc_ - 1, k == 1, ob)) { ok = false; break; }
+        }
+        if (ok && !issue_pv(tc_ - 1, x.ntiles == 1, ob)) ok = false;
+        ++ui;
+      }
+      if (!ok) give_up();
+      mma_commit(bar(B_DONE));                   // every issued MMA done before TMEM is freed
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(bar(B_DONE), 0) && globaltimer() - t0 < kWaitNs) {}
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int r = threadIdx.x;                   // query row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int tl = r / G, g = r - (r / G) * G;   // token of the unit, head of the group
+    bool failed = false;
+    int tc_ = 0, ui = 0, ostep = 0;              // tiles seen, units done, O products issued
+    for (long long u = blockIdx.x; u < U && !failed; u += gridDim.x) {
+      const FUnit x = fa_unit<G>(a, u);
+      if (x.ntok <= 0) continue;
+      const int ob = ui & 1;
+      const bool row_ok = tl < x.ntok;
+      const int pos = x.pos0 + tl;               // this row attends keys [0, pos]
+      const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
+      float m = -CUDART_INF_F, l = 0.f;
+      for (int k = 0; k < x.ntiles; ++k, ++tc_) {
+        const int sb = tc_ & 1;
+        const int ts = k * kTile;
+        // keys of this tile in a block with a bad id (the producer loaded nothing there)
+        uint32_t badblk = 0;
+        const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+#pragma unroll
+        for (int q = 0; q < NB_T; ++q) {
+          if (q >= nblk) continue;
+          const int ph = __ldg(table + ts / BS + q);
+          if (ph < 0 || ph >= a.num_blocks) badblk |= 1u << q;
+        }
+        // V row r of the stage: zero if no row of the unit attends key ts + r
+        const bool zero_v = ts + r >= x.t1 || ((badblk >> (r / BS)) & 1u);
+        if (!mbar_wait(bar(B_SFULL + sb), (tc_ >> 1) & 1, abort_flag)) failed = true;
+        tc_fence_after();
+        uint32_t raw[kTile];
+#pragma unroll
+        for (int c = 0; c < kTile; c += 32) tmem_ld32(tmem_s + lane_off + sb * kTile + c, raw + c);
+        tmem_wait_ld();
+        float* sv = reinterpret_cast<float*>(raw);
+        // scores in the log2 domain, masked; the tile's row maximum
+        const bool full = row_ok && ts + kTile - 1 <= x.pos0 && badblk == 0;  // every key seen
+        float tm = -CUDART_INF_F;
+#pragma unroll
+        for (int j = 0; j < kTile; ++j) {
+          float v = sv[j] * a.scale_log2;
+          if (!full) {
+            const bool vis = row_ok && ts + j <= pos && !((badblk >> (j / BS)) & 1u);
+            v = vis ? v : -CUDART_INF_F;
+          }
+          sv[j] = v;
+          tm = fmaxf(tm, v);
+        }
+        float alpha = 1.f;
+        bool resc = false;
+        if (k == 0) {
+          m = fmaxf(tm, -FLT_MAX);
+        } else if (tm > m + kRescaleLog2) {
+          resc = true;
+          alpha = ex2(m - tm);
+          m = tm;
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // rare: this warp's rows move their reference; O holds the products of
+          // tiles up to k - 1: wait for the last one, rescale the rows in TMEM
+          if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < kD; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem_o + lane_off + ob * kD + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tmem_o + lane_off + ob * kD + c, o);
+          }
+          tmem_wait_st();
+          l *= alpha;
+        }
+        // weights, the row sum, and P = hi + lo over this tile's S columns
+#pragma unroll
+        for (int c = 0; c < kTile; c += 64) {
+          uint32_t hi[32], lo[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2(sv[c + 2 * e] - m), p1 = ex2(sv[c + 2 * e + 1] - m);
+            l += p0 + p1;
+            split2<FMT>(p0, p1, hi[e], lo[e]);
+          }
+          tmem_st32(tmem_s + lane_off + sb * kTile + c / 2, hi);
+          tmem_st32(tmem_s + lane_off + sb * kTile + 64 + c / 2, lo);
+        }
+        if (zero_v) {
+          // this V row enters the output product with weight 0: it must hold finite values
+          const int seq = 2 * tc_ + 1, s = seq % kNST;
+          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) failed = true;
+          uint4* z0 = reinterpret_cast<uint4*>(smem + OFF_KV + s * kOp + r * 128);
+          uint4* z1 = reinterpret_cast<uint4*>(smem + OFF_KV + s * kOp + kHalf + r * 128);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) { z0[q] = make_uint4(0, 0, 0, 0); z1[q] = make_uint4(0, 0, 0, 0); }
+        }
+        fence_proxy_async();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(B_PREADY + sb));
+        ++ostep;
+      }
+      // ---- epilogue: O / l of this row to the output. The products of the
+      // last two tiles may both be pending; a parity wait names one of two
+      // phases, so wait for them in order.
+      if (ostep >= 2 && !mbar_wait(bar(B_OSTEP), (ostep - 2) & 1, abort_flag)) failed = true;
+      if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const size_t orow = ((size_t)(x.qrow0 + tl) * a.Hq + (size_t)x.h * G + g) * kD;
+#pragma unroll 1
+      for (int c = 0; c < kD; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem_o + lane_off + ob * kD + c, o);
+        tmem_wait_ld();
+        if (row_ok && !failed) {
+          if (a.out_dtype == PA_F32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + c);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv, __uint_as_float(o[4 * e + 1]) * inv,
+                                   __uint_as_float(o[4 * e + 2]) * inv, __uint_as_float(o[4 * e + 3]) * inv);
+          } else {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float f0 = __uint_as_float(o[2 * e]) * inv, f1 = __uint_as_float(o[2 * e + 1]) * inv;
+              if (a.out_dtype == PA_BF16) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(f0, f1);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+              } else {
+                const __half2 h = __floats2half2_rn(f0, f1);
+                pk[e] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow + c);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_ODONE + ob));
+      ++ui;
+      // the warps of the group leave together
+      failed = wg_vote_or(failed, 0);
+    }
+    if (failed) give_up();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 fa_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Query [T][Hq][128] seen as [T][Hq][2 d-halves][64]: a box of TPU tokens x G
+// heads x one d-half lands as 128 rows (token-major, then head) of 128 B,
+// 128-byte swizzled. Pools [NB][bs][Hkv][128] seen as [NB][2][Hkv][bs][64]: a
+// box of one block's bs rows of one head and one d-half.
+bool make_fa_maps(const PrefillLaunch& p, int G, CUtensorMap* q, CUtensorMap* k, CUtensorMap* v) {
+  auto enc = fa_encode_fn();
+  if (!enc || p.num_blocks <= 0) return false;
+  const CUtensorMapDataType dt =
+      p.dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t qdims[4] = {64, 2, (cuuint64_t)p.Hq, (cuuint64_t)p.T};
+  const cuuint64_t qstr[3] = {128, (cuuint64_t)kD * 2, (cuuint64_t)p.Hq * kD * 2};
+  const cuuint32_t qbox[4] = {64, 1, (cuuint32_t)G, (cuuint32_t)(kM / G)};
+  const cuuint32_t es4[4] = {1, 1, 1, 1};
+  if (enc(q, dt, 4, const_cast<void*>(p.q), qdims, qstr, qbox, es4, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const cuuint64_t dims[5] = {64, (cuuint64_t)p.bs, (cuuint64_t)p.Hkv, 2, (cuuint64_t)p.num_blocks};
+  const cuuint64_t strides[4] = {(cuuint64_t)p.Hkv * kD * 2, (cuuint64_t)kD * 2, 128,
+                                 (cuuint64_t)p.bs * p.Hkv * kD * 2};
+  const cuuint32_t box[5] = {64, (cuuint32_t)p.bs, 1, 1, 1};
+  const cuuint32_t es5[5] = {1, 1, 1, 1, 1};
+  for (int i = 0; i < 2; ++i) {
+    if (enc(i == 0 ? k : v, dt, 5, const_cast<void*>(i == 0 ? p.k_cache : p.v_cache), dims,
+            strides, box, es5, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+template <int FMT, int BS, int G>
+int launch_fa_t(const FaArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                cudaStream_t stream) {
+  auto kern = prefill_fa_kernel<FMT, BS, G>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
+        cudaSuccess)
+      return PA_ERR_CUDA;
+    attr = true;
+  }
+  const long long U = (long long)a.B * a.chunks * a.Hkv;
+  if (U <= 0) return PA_OK;
+  const long long grid = U < sm_count_cached() ? U : sm_count_cached();
+  return launch_k(kern, dim3((unsigned)grid), dim3(kThreads), kSmem, stream, a, q, k, v) ==
+                 cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <int FMT, int BS>
+int launch_fa_g(const FaArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                cudaStream_t stream) {
+  switch (a.Hq / a.Hkv) {
+    case 1: return launch_fa_t<FMT, BS, 1>(a, q, k, v, stream);
+    case 2: return launch_fa_t<FMT, BS, 2>(a, q, k, v, stream);
+    case 4: return launch_fa_t<FMT, BS, 4>(a, q, k, v, stream);
+    case 8: return launch_fa_t<FMT, BS, 8>(a, q, k, v, stream);
+    case 16: return launch_fa_t<FMT, BS, 16>(a, q, k, v, stream);
+  }
+  return PA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+bool prefill_fa_supported(int dtype, int Hq, int Hkv, int D, int bs) {
+  if (dtype != PA_F16 && dtype != PA_BF16) return false;
+  if (D != kD || (bs != 16 && bs != 32) || Hkv <= 0 || Hq % Hkv) return false;
+  const int G = Hq / Hkv;
+  return G == 1 || G == 2 || G == 4 || G == 8 || G == 16;
+}
+
+int launch_prefill_fa(const PrefillLaunch& p, cudaStream_t stream) {
+  const int G = p.Hq / p.Hkv;
+  CUtensorMap q, k, v;
+  if (!make_fa_maps(p, G, &q, &k, &v)) return PA_ERR_CUDA;
+  FaArgs a{};
+  a.out = p.out;
+  a.out_dtype = p.out_dtype;
+  a.block_tables = p.block_tables;
+  a.max_blocks = p.max_blocks;
+  a.context_lens = p.context_lens;
+  a.query_start = p.query_start;
+  a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.bs = p.bs; a.num_blocks = p.num_blocks;
+  a.chunks = (p.max_query_len + kM / G - 1) / (kM / G);
+  a.scale_log2 = p.scale_log2;
+  a.max_context_len = p.max_context_len;
+  a.err_flag = p.err_flag;
+  if (p.dtype == PA_BF16)
+    return p.bs == 16 ? launch_fa_g<1, 16>(a, q, k, v, stream) : launch_fa_g<1, 32>(a, q, k, v, stream);
+  return p.bs == 16 ? launch_fa_g<0, 16>(a, q, k, v, stream) : launch_fa_g<0, 32>(a, q, k, v, stream);
+}
+
+}  // namespace pa

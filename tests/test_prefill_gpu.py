@@ -1,4 +1,6 @@
-"""Paged prefill (causal, chunked) on the GPU against the fp64 oracle."""
+"""Paged prefill (causal, chunked) on the GPU against the fp64 oracle, on both
+prefill kernels: the default one (query rows on the MMA's M) and the
+multi-query kernel (key rows on M), chosen with PA_PREFILL_KERNEL."""
 
 import numpy as np
 import pytest
@@ -10,6 +12,15 @@ from paged_kv_cache_418_b200 import workloads as W
 from pa_testlib import assert_attention_close
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, params=["rows-on-m", "multi-query"])
+def prefill_kernel(request, monkeypatch):
+    if request.param == "multi-query":
+        monkeypatch.setenv("PA_PREFILL_KERNEL", "mq")
+    else:
+        monkeypatch.delenv("PA_PREFILL_KERNEL", raising=False)
+    return request.param
 
 
 def _run(c, out_dtype=torch.float32, ctx=None):
@@ -76,3 +87,17 @@ def test_prefill_rejects_unsupported_shapes_before_launch():
                        t["context_lens"], t["query_start"], c.max_query_len, c.scale,
                        c.max_context_len)
     assert e.value.status == 4
+
+
+def test_prefill_bad_block_id_is_flagged_and_left_out():
+    c = W.build_prefill_case("pf-badblk", W.BF16, Hq=16, Hkv=2, D=128, block_size=16,
+                             prior_lens=[300], new_lens=[40], seed=12)
+    t = W.prefill_to_torch(c, "cuda")
+    t["block_tables"][0, 3] = c.num_blocks + 5              # tokens 48..63 unreachable
+    out = torch.full((c.T, c.Hq, c.D), float("nan"), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.pa_prefill(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"], t["context_lens"],
+                   t["query_start"], c.max_query_len, c.scale, c.max_context_len, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & ops.PA_DEV_BAD_BLOCK_ID
+    assert torch.isfinite(out).all()
