@@ -18,7 +18,9 @@ With no --workload, the same JSON line also carries (one GPU only):
                 with the CUDA-core kernel timed beside the tensor-core one on
                 the GQA shapes (kernel_ab);
   warm_l2       decode of a batch that fits the L2, with and without a flush;
-  paging_cost   decode on contiguous block tables against shuffled ones.
+  paging_cost   decode on contiguous block tables against shuffled ones;
+  prefill       paged chunked prefill (TFLOP/s), with the multi-query kernel beside it;
+  swap_blocks   blocks swapped out to page-locked host memory and back.
 
 Under torchrun (N > 1) every rank runs its own replica of the workload on its
 own GPU (weak scaling; the path has no exchange step, so there is no
@@ -837,6 +839,19 @@ def prefill_arm(args, rank: int, world: int, local_rank: int):
     (ms,) = max_over_ranks([ms], world, dev)
     flops = c.attention_flops()
     tflops = flops / (ms / 1e3) / 1e12
+    # the same calls on the multi-query kernel (key rows on the MMA's M), same loop
+    os.environ["PA_PREFILL_KERNEL"] = "mq"
+    try:
+        for _ in range(3):
+            run()
+        e0.record(stream)
+        for _ in range(K):
+            run()
+        e1.record(stream)
+        e1.synchronize()
+        ms_mq = e0.elapsed_time(e1) / K
+    finally:
+        del os.environ["PA_PREFILL_KERNEL"]
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     peak = float(json.load(open(path))["bf16_tflops"]) if os.path.exists(path) else 1590.0
     # end to end: query and tables from pinned host memory, output back, every call
@@ -872,8 +887,12 @@ def prefill_arm(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
                      "peak_source": "bf16_tflops (measured, burst)",
-                     "kernel": "multi_query_tc_kernel (prefill), per launch; algorithmic flops "
-                               "4*D per (query head, attended key)"},
+                     "kernel": "prefill_fa_kernel (query rows on the MMA's M), per launch; "
+                               "algorithmic flops 4*D per (query head, attended key)"},
+        "kernel_ab": {"tflops_rows_on_m": round(tflops, 2),
+                      "tflops_multi_query": round(flops / (ms_mq / 1e3) / 1e12, 2),
+                      "ms_rows_on_m": round(ms, 5), "ms_multi_query": round(ms_mq, 5),
+                      "how": f"{K} calls back to back per kernel, same inputs"},
         "gpu_launches": K,
         "clocks": clocks,
         "e2e": {"value": round(flops / (e_ms / 1e3) / 1e12 * world, 2), "unit": "TFLOP/s",
@@ -973,6 +992,13 @@ def main():
             line["per_workload"] = suite(args, local_rank)
             line["warm_l2"] = warm_l2(args, local_rank)
             line["paging_cost"] = paging_cost(args, local_rank)
+            keep = ("metric", "value", "unit", "ms_per_step", "roofline", "kernel_ab", "clocks",
+                    "e2e", "cpu_baseline", "config", "gpu_launches")
+            pf = prefill_arm(args, 0, 1, local_rank)
+            line["prefill"] = {k2: pf[k2] for k2 in keep if k2 in pf}
+            sw = swap_arm(args, 0, 1, local_rank)
+            line["swap_blocks"] = {k2: sw[k2] for k2 in keep + ("swap_out_gbs", "swap_in_gbs")
+                                   if k2 in sw}
         else:
             line["per_workload"] = {"note": "measured at N=1 only (one GPU)"}
     if rank == 0:
