@@ -105,9 +105,9 @@ template <int G> struct TcShape {
   static constexpr int OFF_STG = OFF_P + 2 * kPBytes;        // [2 groups] output staging
   static constexpr int OFF_X = OFF_STG + 2 * kStgBytes;      // [2][2][NS] reference max, exp-sum
   static constexpr int OFF_BAR = OFF_X + 2 * 2 * NS * 4 + 16;
-  static constexpr int NBAR = 2 * kStages + 20;
+  static constexpr int NBAR = 3 * kStages + 20;
   static constexpr int GP = G < 8 ? 8 : G;                  // per-chunk stride of the reductions
-  static constexpr int OFF_RED = OFF_BAR + 8 * NBAR;         // [group][2][8 chunks][GP] maxima
+  static constexpr int OFF_RED = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;  // [group][2][8][GP] maxima
   static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
   static constexpr int OFF_MREF = OFF_REDL + 2 * 2 * 8 * GP * 4;  // [group][3][NS] references
   static constexpr int OFF_COEF = OFF_MREF + 2 * 3 * NS * 4;   // [group][2][NS] merge weights
@@ -125,7 +125,7 @@ template <int NST> struct Bars {
   static constexpr int FULL = 0, EMPTY = NST, QFULL = 2 * NST, QEMPTY = QFULL + 2,
                        SFULL = QEMPTY + 2, SFREE = SFULL + 2, PREADY = SFREE + 2,
                        OFULL = PREADY + 2, XFULL = OFULL + 2, XFREE = XFULL + 2,
-                       ODONE = XFREE + 2, DONE = ODONE + 2;
+                       ODONE = XFREE + 2, DONE = ODONE + 2, CONV = DONE + 1;
 };
 
 // Shared words written by the prologue (OFF_MISC).
@@ -409,7 +409,57 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs& a, const Unit& x,
   }
 }
 
-template <int FMT, int BS, int G>
+// FP8 pools: two E4M3 codes (one 16-bit word) -> two 16-bit values of the
+// query's type, exactly. E4M3 -> f16 is exact (every E4M3 value is a normal
+// f16 or zero); f16 -> bf16 is then exact too (3 fraction bits, exponent in
+// range): the bf16 pattern is the f16 magnitude shifted right by 3 with the
+// exponent rebased (+112), zero staying zero.
+template <int FMT>
+__device__ __forceinline__ uint32_t widen2_e4m3(uint32_t codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xffffu),
+                                                   __NV_E4M3);
+  const uint32_t f = (uint32_t)h.x | ((uint32_t)h.y << 16);
+  if (FMT == 0) return f;
+  const uint32_t mag = f & 0x7fff7fffu;
+  const uint32_t b = (mag >> 3) + 0x38003800u;             // no carry between the halves
+  return (f & 0x80008000u) | (b & ~__vcmpeq2(mag, 0u));
+}
+
+// Widen tile row `row` of a stage in place: its 128 E4M3 codes sit at the
+// stage's upper 16 KB (one 128-byte-swizzled row, as TMA wrote them) and
+// become the row of both 64-wide d-halves of the 16-bit operand layout (the
+// second of which is that very line). Only this thread touches the row, and
+// it reads the whole line before it writes; zero writes zeros instead.
+template <int FMT>
+__device__ __forceinline__ void widen_row_fp8(uint8_t* stage, int row, bool zero) {
+  const int sw = row & 7;
+  uint8_t* src = stage + kHalf + row * 128;
+  uint4 c[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    c[j] = zero ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(src + ((j ^ sw) << 4));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // codes 16j .. 16j + 15 -> d-half j / 4, 16-byte chunks 2 (j % 4) and 2 (j % 4) + 1
+    const uint32_t w[4] = {c[j].x, c[j].y, c[j].z, c[j].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[2 * k] = widen2_e4m3<FMT>(w[k]);
+      o[2 * k + 1] = widen2_e4m3<FMT>(w[k] >> 16);
+    }
+    uint8_t* dst = stage + (j >> 2) * kHalf + row * 128;
+    const int c0 = 2 * (j & 3);
+    *reinterpret_cast<uint4*>(dst + ((c0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + (((c0 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// KV8: the pools hold FP8 E4M3 codes (K times k_scale, folded into the score
+// scale; V times v_scale, folded into the output weights). TMA brings a tile's
+// codes (half the bytes); the softmax group that owns the tile widens it in
+// place (widen_row_fp8) and only then releases it to the tensor cores.
+template <int FMT, int BS, int G, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ) {
@@ -457,6 +507,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     mbar_init(bar(Bx::ODONE), 128);
     mbar_init(bar(Bx::ODONE + 1), 128);
     mbar_init(bar(Bx::DONE), 1);
+    for (int s = 0; s < NST; ++s) mbar_init(bar(Bx::CONV + s), 128);
     ms->abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -488,6 +539,9 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
   };
   // token range of tile k of a unit, and how many of its boxes hold tokens
+  // a stage is ready for the tensor cores when TMA filled it (16-bit pools) or
+  // when its owning group widened it (FP8 pools)
+  auto ready_bar = [&](int s) { return bar((KV8 ? Bx::CONV : Bx::FULL) + s); };
   auto tile_span = [&](const Unit& x, int k, int& ts, int& te, int& nql) {
     ts = x.t0 + k * kRt;
     te = min(x.t1, ts + kRt);
@@ -537,7 +591,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
             phys[q] = phys_next[q];
-            if (phys[q] >= 0 && phys[q] < a.num_blocks) bytes += 2u * RB * kHG * 128u;
+            if (phys[q] >= 0 && phys[q] < a.num_blocks) bytes += (KV8 ? 1u : 2u) * RB * kHG * 128u;
           }
           next_tile<BS>(a, nhg, ahead);
           load_ids(ahead, phys_next);
@@ -550,9 +604,15 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             for (int q = 0; q < NQ; ++q) {
               if (phys[q] < 0 || phys[q] >= a.num_blocks) continue;
               const int rr0 = (ts + q * RB) % BS;
-              for (int hh = 0; hh < 2; ++hh)
-                tma_load_5d(dst + hh * kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, rr0,
-                            x.h * kHG, hh, phys[q], bar(Bx::FULL + s));
+              if (KV8) {
+                // all 128 codes of a row in one 128-byte line, at the stage's upper half
+                tma_load_4d(dst + kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, rr0,
+                            x.h * kHG, phys[q], bar(Bx::FULL + s));
+              } else {
+                for (int hh = 0; hh < 2; ++hh)
+                  tma_load_5d(dst + hh * kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, rr0,
+                              x.h * kHG, hh, phys[q], bar(Bx::FULL + s));
+              }
             }
             ++issued;
           }
@@ -588,7 +648,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             !mbar_wait(bar(Bx::ODONE + (ui & 1)), ((ui - 2) >> 1) & 1, abort_flag, wait_ns))
           return false;
         const int seq = 2 * tt + 1, s = seq % NST;
-        if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) return false;
+        if (!mbar_wait(ready_bar(s), (seq / NST) & 1, abort_flag, wait_ns)) return false;
         tc_fence_after();
         const uint32_t vst = sbase + s * kStageBytes;
         const uint32_t pst = sbase + S::OFF_P + pb * S::kPBytes;
@@ -637,14 +697,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                 break;
               }
               if (mbar_test(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1) &&
-                  mbar_test(bar(Bx::FULL + s), (seq / NST) & 1))
+                  mbar_test(ready_bar(s), (seq / NST) & 1))
                 break;
               if (*abort_flag || globaltimer() - t0 > wait_ns) { ok = false; break; }
             }
             if (!ok) break;
           }
           if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag, wait_ns)) { ok = false; break; }
-          if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) { ok = false; break; }
+          if (!mbar_wait(ready_bar(s), (seq / NST) & 1, abort_flag, wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + s * kStageBytes;
 #pragma unroll
@@ -732,6 +792,18 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         const bool valid = in_range && blk_ok && ts + tt_row < te;
         if (in_range && !blk_ok && rr == 0 && rh == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
         const bool first = my_last < 0;
+        if constexpr (KV8) {
+          // widen this tile's K and V rows (zeros for V rows that must not count)
+#pragma unroll 1
+          for (int kv = 0; kv < 2; ++kv) {
+            const int seq = 2 * tc + kv, s = seq % NST;
+            if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
+            if (in_range && !failed)
+              widen_row_fp8<FMT>(smem + s * kStageBytes, row, kv == 1 && !valid);
+            fence_proxy_async();
+            mbar_arrive(bar(Bx::CONV + s));
+          }
+        }
 
         const int par = (tc >> 1) & 1;                        // use count of this group's buffers
         if (!mbar_wait(bar(Bx::SFULL + grp), par, abort_flag, wait_ns)) failed = true;
@@ -817,7 +889,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           *reinterpret_cast<uint16_t*>(prow + g * 128 + ((pchunk ^ (g & 7)) << 4) + pbyte) = hi;
           *reinterpret_cast<uint16_t*>(prow + (G + g) * 128 + ((pchunk ^ ((G + g) & 7)) << 4) + pbyte) = lo;
         }
-        if (in_range && !valid) {
+        if (!KV8 && in_range && !valid) {
           // this V row enters the output product with weight 0: it must hold finite values
           const int seq = 2 * tc + 1, sv_ = seq % NST;
           if (!mbar_wait(bar(Bx::FULL + sv_), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
@@ -902,6 +974,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             if (has_p) cp = exp2f(mp - M);
           }
           const float Lt = L * c + (has_p ? xl[n] * cp : 0.f);
+          c *= a.v_scale;                       // 1 unless V holds FP8 codes
+          cp *= a.v_scale;
           if (final_out) {
             const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
             c *= inv;
@@ -1015,24 +1089,41 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_maps(const DecodeArgs& a, int dtype, int G, CUtensorMap* k, CUtensorMap* v,
+bool make_maps(const DecodeArgs& a, int dtype, bool kv8, int G, CUtensorMap* k, CUtensorMap* v,
                CUtensorMap* q) {
   auto enc = encode_fn();
   if (!enc || a.num_blocks <= 0) return false;
   const CUtensorMapDataType dt =
       dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  // the pool [num_blocks][bs][Hkv][D] seen as [num_blocks][2][Hkv][bs][64]: a box of
-  // RB rows x kHG heads x 64 d lands head-major, 128 B per row, 128-byte swizzled
   const int rb = a.bs < kRt ? a.bs : kRt;
-  const cuuint64_t dims[5] = {64, (cuuint64_t)a.bs, (cuuint64_t)a.Hkv, 2, (cuuint64_t)a.num_blocks};
-  const cuuint64_t strides[4] = {(cuuint64_t)a.Hkv * kD * 2, (cuuint64_t)kD * 2, 128,
-                                 (cuuint64_t)a.bs * a.Hkv * kD * 2};
-  const cuuint32_t box[5] = {64, (cuuint32_t)rb, (cuuint32_t)kHG, 1, 1};
-  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   for (int i = 0; i < 2; ++i) {
-    CUresult r = enc(i == 0 ? k : v, dt, 5, const_cast<void*>(i == 0 ? a.k_cache : a.v_cache), dims,
-                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r;
+    void* pool = const_cast<void*>(i == 0 ? a.k_cache : a.v_cache);
+    if (kv8) {
+      // FP8 pool [num_blocks][bs][Hkv][128 codes]: a box of RB rows x kHG heads
+      // lands head-major, one 128-byte line per row, 128-byte swizzled
+      const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)a.bs, (cuuint64_t)a.Hkv,
+                                  (cuuint64_t)a.num_blocks};
+      const cuuint64_t strides[3] = {(cuuint64_t)a.Hkv * kD, (cuuint64_t)kD,
+                                     (cuuint64_t)a.bs * a.Hkv * kD};
+      const cuuint32_t box[4] = {(cuuint32_t)kD, (cuuint32_t)rb, (cuuint32_t)kHG, 1};
+      const cuuint32_t es[4] = {1, 1, 1, 1};
+      r = enc(i == 0 ? k : v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, pool, dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+      // the pool [num_blocks][bs][Hkv][D] seen as [num_blocks][2][Hkv][bs][64]: a box of
+      // RB rows x kHG heads x 64 d lands head-major, 128 B per row, 128-byte swizzled
+      const cuuint64_t dims[5] = {64, (cuuint64_t)a.bs, (cuuint64_t)a.Hkv, 2,
+                                  (cuuint64_t)a.num_blocks};
+      const cuuint64_t strides[4] = {(cuuint64_t)a.Hkv * kD * 2, (cuuint64_t)kD * 2, 128,
+                                     (cuuint64_t)a.bs * a.Hkv * kD * 2};
+      const cuuint32_t box[5] = {64, (cuuint32_t)rb, (cuuint32_t)kHG, 1, 1};
+      const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+      r = enc(i == 0 ? k : v, dt, 5, pool, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     if (r != CUDA_SUCCESS) return false;
   }
   const cuuint64_t qdims[2] = {(cuuint64_t)kD, (cuuint64_t)a.B * a.Hq};
@@ -1050,10 +1141,10 @@ long long max_tiles(const DecodeArgs& a) {
   return (long long)a.B * (a.Hkv / kHG) * per;
 }
 
-template <int FMT, int BS, int G>
+template <int FMT, int BS, int G, bool KV8>
 int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                 const CUtensorMap& q, cudaStream_t stream) {
-  auto kern = decode_tc_kernel<FMT, BS, G>;
+  auto kern = decode_tc_kernel<FMT, BS, G, KV8>;
   constexpr int smem = TcShape<G>::SMEM;
   static bool attr = false;
   if (!attr) {
@@ -1070,14 +1161,24 @@ int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                  cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int FMT, int BS>
+template <int FMT, int BS, bool KV8>
 int launch_tc_g(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                 const CUtensorMap& q, cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {
-    case 4: return launch_tc_t<FMT, BS, 4>(a, k, v, q, stream);
-    case 8: return launch_tc_t<FMT, BS, 8>(a, k, v, q, stream);
+    case 4: return launch_tc_t<FMT, BS, 4, KV8>(a, k, v, q, stream);
+    case 8: return launch_tc_t<FMT, BS, 8, KV8>(a, k, v, q, stream);
   }
   return PA_ERR_UNSUPPORTED;
+}
+
+template <bool KV8>
+int launch_tc_all(const DecodeArgs& a, int dtype, const CUtensorMap& k, const CUtensorMap& v,
+                  const CUtensorMap& q, cudaStream_t stream) {
+  if (dtype == PA_BF16)
+    return a.bs == 16 ? launch_tc_g<1, 16, KV8>(a, k, v, q, stream)
+                      : launch_tc_g<1, 32, KV8>(a, k, v, q, stream);
+  return a.bs == 16 ? launch_tc_g<0, 16, KV8>(a, k, v, q, stream)
+                    : launch_tc_g<0, 32, KV8>(a, k, v, q, stream);
 }
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1091,7 +1192,8 @@ bool tc_shape(int Hq, int Hkv, int D) {
 }
 
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs) {
-  if (dtype != PA_F16 && dtype != PA_BF16) return false;
+  // 16-bit pools, or FP8 pools (with a 16-bit query: the caller checks that)
+  if (dtype != PA_F16 && dtype != PA_BF16 && dtype != PA_FP8_E4M3) return false;
   return (bs == 16 || bs == 32) && tc_shape(Hq, Hkv, D);
 }
 
@@ -1116,13 +1218,14 @@ void tc_carve(DecodeArgs& a, char* base) {
   a.tickets = reinterpret_cast<unsigned long long*>(base);
 }
 
-int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream) {
+int launch_decode_tc(const DecodeArgs& a, int dtype, bool kv8, cudaStream_t stream) {
   const int G = a.Hq / a.Hkv;
   CUtensorMap k, v, q;
-  if (!make_maps(a, dtype, G, &k, &v, &q)) return launch_decode_simt(a, dtype, stream);
-  if (dtype == PA_BF16)
-    return a.bs == 16 ? launch_tc_g<1, 16>(a, k, v, q, stream) : launch_tc_g<1, 32>(a, k, v, q, stream);
-  return a.bs == 16 ? launch_tc_g<0, 16>(a, k, v, q, stream) : launch_tc_g<0, 32>(a, k, v, q, stream);
+  if (!make_maps(a, dtype, kv8, G, &k, &v, &q))
+    return kv8 ? launch_decode_simt_kv(a, dtype, PA_FP8_E4M3, PA_FP8_E4M3, stream)
+               : launch_decode_simt(a, dtype, stream);
+  return kv8 ? launch_tc_all<true>(a, dtype, k, v, q, stream)
+             : launch_tc_all<false>(a, dtype, k, v, q, stream);
 }
 
 }  // namespace pa

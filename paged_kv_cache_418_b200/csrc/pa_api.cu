@@ -128,6 +128,10 @@ size_t workspace_bytes_for(int B, int Hq, int D, int P) {
   return up(rows * D * 4) + up(rows * 4) + up(rows * 4);
 }
 
+size_t decode_scratch_bytes(const DecodePlan& p, int B, int Hq, int Hkv, int D) {
+  return p.kernel == 2 ? tc_workspace_bytes(B, Hq, Hkv, D) : workspace_bytes_for(B, Hq, D, p.P);
+}
+
 }  // namespace pa
 
 using namespace pa;
@@ -214,9 +218,12 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_ALIGN;
 
-  // a pool of another type than the query's runs on the CUDA-core kernel
+  // pools of another type than the query's run on the CUDA-core kernel, except
+  // FP8 K and V with a 16-bit query (the tensor-core kernel widens the codes)
   DecodePlan p = plan_decode(k_fp8 || v_fp8 ? PA_FP8_E4M3 : q_dtype, B, Hq, Hkv, D, block_size,
                              max_context_len, partition_size);
+  if (p.kernel == 2 && (k_fp8 != v_fp8 || (k_fp8 && q_dtype == PA_F32)))
+    p = plan_decode(PA_F32, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
   DecodeArgs a{};
   a.out = out; a.out_dtype = out_dtype; a.q = query;
   a.k_cache = key_cache; a.v_cache = value_cache;
@@ -230,7 +237,7 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   a.err_flag = err_flag;
   const bool tc_path = p.kernel == 2;
   if (tc_path) {
-    const size_t need = tc_workspace_bytes(B, Hq, Hkv, D);
+    const size_t need = decode_scratch_bytes(p, B, Hq, Hkv, D);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
       return PA_ERR_WORKSPACE;
     tc_carve(a, static_cast<char*>(workspace));
@@ -238,7 +245,7 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
     a.wait_ns = tc_wait_ns();
     a.test_withhold_q = tc_test_withhold_q();
   } else if (p.P > 1) {
-    const size_t need = workspace_bytes_for(B, Hq, D, p.P);
+    const size_t need = decode_scratch_bytes(p, B, Hq, Hkv, D);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
       return PA_ERR_WORKSPACE;
     const size_t rows = (size_t)B * Hq * p.P;
@@ -250,8 +257,9 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int rc;
-  if (k_fp8 || v_fp8) rc = launch_decode_simt_kv(a, q_dtype, k_dtype, v_dtype, s);
-  else rc = p.kernel == 2 ? launch_decode_tc(a, q_dtype, s) : launch_decode_simt(a, q_dtype, s);
+  if (p.kernel == 2) rc = launch_decode_tc(a, q_dtype, k_fp8, s);
+  else if (k_fp8 || v_fp8) rc = launch_decode_simt_kv(a, q_dtype, k_dtype, v_dtype, s);
+  else rc = launch_decode_simt(a, q_dtype, s);
   if (rc == PA_OK && p.P > 1) rc = launch_merge(a, s);
   return rc;
 }
@@ -422,7 +430,7 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
     a.test_withhold_q = tc_test_withhold_q();
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, st) : launch_decode_simt(a, dtype, st);
+  int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, false, st) : launch_decode_simt(a, dtype, st);
   if (rc == PA_OK)
     rc = launch_prefix_tc(a, dtype, group_offsets, group_members, num_groups, max_group_size,
                           parts, part_tokens, st);

@@ -67,13 +67,17 @@ struct DecodePlan {
 DecodePlan plan_decode(int dtype, int B, int Hq, int Hkv, int D, int bs, int max_ctx,
                        int partition_size);
 size_t workspace_bytes_for(int B, int Hq, int D, int P);
+// Scratch a decode with this plan needs: the tensor-core kernel's pieces and
+// tickets, or the CUDA-core split pass's partials (0 for a single pass).
+size_t decode_scratch_bytes(const DecodePlan& p, int B, int Hq, int Hkv, int D);
 
 int launch_decode_simt(const DecodeArgs& a, int dtype, cudaStream_t stream);
 // Pools whose element types differ from the query's: both FP8 E4M3 (any query
 // type), or one FP8 and the other of the query's 16-bit type.
 int launch_decode_simt_kv(const DecodeArgs& a, int q_dtype, int k_dtype, int v_dtype,
                           cudaStream_t stream);
-int launch_decode_tc(const DecodeArgs& a, int dtype, cudaStream_t stream);
+// dtype: the query's (16-bit) type; kv8: both pools hold FP8 E4M3 codes.
+int launch_decode_tc(const DecodeArgs& a, int dtype, bool kv8, cudaStream_t stream);
 bool tc_supported(int dtype, int Hq, int Hkv, int D, int bs);
 // Shapes the tensor-core path can take for some 16-bit element type and block size.
 bool tc_shape(int Hq, int Hkv, int D);

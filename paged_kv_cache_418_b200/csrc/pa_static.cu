@@ -108,7 +108,7 @@ extern "C" int pa_decode_static(void* out, int out_dtype, const void* query,
   if (B > 0 && Hq > 0 && D > 0 && block_size > 0 && max_context_len >= 0 && partition_size >= 0) {
     const pa::DecodePlan p =
         pa::plan_decode(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
-    need = pa::workspace_bytes_for(B, Hq, D, p.P);
+    need = pa::decode_scratch_bytes(p, B, Hq, Hkv, D);
   }
   if (need > (size_t)PA_STATIC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
   void* scratch = nullptr;

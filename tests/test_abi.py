@@ -161,5 +161,7 @@ def test_shared_prefix_workspace_and_fp8_plan():
     assert n == up(rows * D * 4) + 2 * up(rows * 4) + tc
     assert ops.pa_shared_prefix_workspace_size(B, Hq, 8, D, 1547, 0, 16, 0) == \
         ops.pa_workspace_size(B, Hq, 8, D, 1547, 0)
-    # FP8 pools always plan the CUDA-core kernel
-    assert ops.pa_decode_plan(ops.PA_FP8_E4M3, 8, 64, 8, 128, 16, 4096)[0] == 1
+    # FP8 pools plan the tensor-core kernel on its GQA shapes (16-bit query), the
+    # CUDA-core kernel elsewhere
+    assert ops.pa_decode_plan(ops.PA_FP8_E4M3, 8, 64, 8, 128, 16, 4096)[0] == 2
+    assert ops.pa_decode_plan(ops.PA_FP8_E4M3, 8, 32, 32, 128, 16, 4096)[0] == 1

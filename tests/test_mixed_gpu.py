@@ -99,3 +99,46 @@ def test_mixed_pools_need_a_16_bit_query():
     with pytest.raises(ops.PAError) as e:
         ops.pa_decode_kv(out, qb, kc, vc16, 0.5, 1.0, tables, lens, 0.1, 16)
     assert e.value.status == 3
+
+
+# -- FP8 pools on the tensor cores (grouped-query shapes, 16-bit query) ------------
+@pytest.mark.parametrize("qdt", [W.F16, W.BF16])
+@pytest.mark.parametrize("G,Hkv", [(4, 4), (8, 8)])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_fp8_pools_on_the_tensor_cores(qdt, G, Hkv, bs):
+    ctx = [1, bs - 1, bs, 33, 129, 700, 2049, 64]
+    nb = sum((c + bs - 1) // bs for c in ctx) + 5
+    w = W.build_decode_case("fp8-tc", qdt, B=len(ctx), Hq=G * Hkv, Hkv=Hkv, D=128, block_size=bs,
+                            num_blocks=nb, context_lens=ctx, seed=G * 100 + bs + qdt, kv_fp8=True)
+    assert ops.pa_decode_plan(W.FP8, w.B, w.Hq, w.Hkv, w.D, bs, w.max_context_len)[0] == 2
+    for out_f32 in (True, False):
+        out, t = device_step(w, out_dtype=torch.float32 if out_f32 else None)
+        ref, _, _ = oracle_step(w)
+        torch.cuda.synchronize()
+        assert int(t["err"].item()) == 0
+        assert_attention_close(out, ref, qdt, f"G={G} bs={bs} f32={out_f32}")
+
+
+@pytest.mark.parametrize("qdt", [W.F16, W.BF16])
+def test_fp8_tensor_core_widening_is_exact_for_every_code(qdt):
+    """One token with weight exactly 1: o = value(code) * v_scale, for every finite
+    E4M3 code (subnormals and +-448 included), through the tensor-core kernel's
+    in-place widening of the codes to the query's 16-bit type."""
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    D, Hkv, G = 128, 4, 8
+    w = W.build_decode_case("fp8-tc-codes", qdt, B=1, Hq=G * Hkv, Hkv=Hkv, D=D, block_size=16,
+                            num_blocks=4, context_lens=[2], seed=13, kv_fp8=True, v_scale=0.37)
+    assert ops.pa_decode_plan(W.FP8, 1, G * Hkv, Hkv, D, 16, 2)[0] == 2
+    codes = np.concatenate([finite, finite, finite[:Hkv * D - 2 * len(finite)]]).reshape(Hkv, D)
+    blk = w.block_tables[0, 0]
+    w.v_cache[blk, 0] = codes
+    w.k_cache[blk, 0] = 0x00                                   # k0 = 0: score 0
+    one = W.round_to_storage(np.ones(1, dtype=np.float32), qdt)[0]
+    w.q[:] = one
+    w.new_key[:] = W.round_to_storage(np.full(1, -1e4, dtype=np.float32), qdt)[0]
+    out, t = device_step(w, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert int(t["err"].item()) == 0
+    exp = (oracle.widen(codes, oracle.FP8) * w.v_scale).astype(np.float32)   # [Hkv, D]
+    exp = np.repeat(exp[None], G, axis=0).transpose(1, 0, 2).reshape(1, G * Hkv, D)
+    assert torch.equal(out.cpu(), torch.from_numpy(exp))

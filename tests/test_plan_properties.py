@@ -2,7 +2,7 @@
 random shapes (CPU only; nothing is launched): the partitions cover every
 context exactly once, the workspace holds the partials of every partition (or
 the tensor-core kernel's pieces and tickets), and the tensor-core path is
-planned only for 16-bit pools."""
+planned only for 16-bit and FP8 pools on the shapes it takes."""
 
 from __future__ import annotations
 
@@ -37,8 +37,11 @@ def test_partitions_cover_each_context_once(shape):
     psize_in = pblocks * bs
     kernel, P, psize = ops.pa_decode_plan(dtype, B, Hq, Hkv, D, bs, mcl, psize_in)
     assert kernel in (1, 2)
-    if dtype in (ops.PA_F32, ops.PA_FP8_E4M3):
-        assert kernel == 1                    # tcgen05 path: 16-bit pools only
+    tc_shape = D == 128 and Hkv % 4 == 0 and G in (4, 8)
+    if dtype == ops.PA_F32 or not tc_shape:
+        assert kernel == 1                    # tcgen05 path: 16-bit or FP8 pools, its shapes
+    else:
+        assert kernel == 2
     if D != 128:
         assert kernel == 1
     assert P >= 1 and psize > 0 and psize % bs == 0

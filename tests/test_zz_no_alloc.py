@@ -132,13 +132,15 @@ def test_a_second_context_does_not_change_the_primary_contexts_scratch():
 
 
 def test_sizes_beyond_the_scratch_are_rejected_before_launch():
-    # 64 sequences x 64 heads x 128 partitions of 512 tokens needs ~270 MB of partials
+    # 64 sequences x 64 heads (no grouping: the CUDA-core split pass) x 128
+    # partitions of 512 tokens needs ~270 MB of partials
     q = torch.zeros(64, 64, 128, dtype=torch.bfloat16, device="cuda")
-    kc = torch.zeros(4, 16, 8, 128, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(4, 16, 64, 128, dtype=torch.bfloat16, device="cuda")
     tables = torch.zeros(64, 4096, dtype=torch.int32, device="cuda")
     lens = torch.ones(64, dtype=torch.int32, device="cuda")
     out = torch.zeros(64, 64, 128, dtype=torch.bfloat16, device="cuda")
-    assert ops.pa_workspace_size(64, 64, 8, 128, 65536, 512) > ops.PA_STATIC_SCRATCH_BYTES
+    assert ops.pa_decode_plan(ops.PA_BF16, 64, 64, 64, 128, 16, 65536, 512)[:2] == (1, 128)
+    assert ops.pa_workspace_size(64, 64, 64, 128, 65536, 512) > ops.PA_STATIC_SCRATCH_BYTES
     with pytest.raises(ops.PAError) as e:
         ops.pa_decode_static(out, q, kc, kc, tables, lens, 0.1, 65536, 512)
     assert e.value.status == 5
