@@ -77,6 +77,8 @@ def parse():
                         "the headline, plus every other decode workload in per_workload)")
     p.add_argument("--no-suite", action="store_true",
                    help="default run: measure the headline workload only")
+    p.add_argument("--skip-prefill", action="store_true",
+                   help="default run: leave out the prefill measurement")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=None)
     p.add_argument("--batch", type=int, default=None,
@@ -994,8 +996,9 @@ def main():
             line["paging_cost"] = paging_cost(args, local_rank)
             keep = ("metric", "value", "unit", "ms_per_step", "roofline", "kernel_ab", "clocks",
                     "e2e", "cpu_baseline", "config", "gpu_launches")
-            pf = prefill_arm(args, 0, 1, local_rank)
-            line["prefill"] = {k2: pf[k2] for k2 in keep if k2 in pf}
+            if not args.skip_prefill:
+                pf = prefill_arm(args, 0, 1, local_rank)
+                line["prefill"] = {k2: pf[k2] for k2 in keep if k2 in pf}
             sw = swap_arm(args, 0, 1, local_rank)
             line["swap_blocks"] = {k2: sw[k2] for k2 in keep + ("swap_out_gbs", "swap_in_gbs")
                                    if k2 in sw}
