@@ -61,21 +61,28 @@ typedef enum {
                                   > max_context_len: sequence b's output rows are zeros */
 #define PA_DEV_BAD_SLOT 4u     /* slot >= num_blocks * block_size: that token is not written */
 #define PA_DEV_BAD_PAIR 8u     /* src or dst outside [0, num_blocks): that pair is skipped */
-#define PA_DEV_TIMEOUT 16u     /* a pipeline wait inside the tensor-core decode kernel gave up
+#define PA_DEV_TIMEOUT 16u     /* a pipeline wait inside a tensor-core kernel gave up
                                   (bounded at 1 s): outputs of that launch are unspecified */
 
 /*
  * pa_workspace_size -- bytes of scratch pa_decode needs for these sizes.
  *
- * The split-context pass (used when contexts are long or the batch is too
- * small to fill the GPU) writes, per (sequence, query head, partition), the
- * partition's running max m, exp-sum l and unnormalised output (fp32), and a
- * merge kernel combines them: M = max m_j, L = sum l_j e^(m_j - M),
+ * Splitting one sequence's softmax sum over several workers needs scratch:
+ * each part's running max m, exp-sum l and unnormalised output (fp32), which
+ * are then combined: M = max m_j, L = sum l_j e^(m_j - M),
  * o = sum e^(m_j - M) o_j / L. This is not on the pages; it is the algebra of
- * splitting one softmax sum. Returns 0 when pa_decode will not split.
- * partition_size: 0 = let the library choose, else the partition length in
- * tokens (a multiple of block_size, used as given). Same arguments as the
- * pa_decode call it sizes; never fails (nonsense sizes give 0).
+ * splitting one softmax sum.
+ *  - The CUDA-core kernel splits long contexts into partitions (of
+ *    partition_size tokens: 0 = let the library choose, else a multiple of
+ *    block_size, used as given) and a merge kernel combines them.
+ *  - The tensor-core kernel (16-bit or FP8 pools, head size 128, Hq / Hkv in
+ *    {4, 8}, Hkv a multiple of 4) divides all the work evenly over the SMs;
+ *    a sequence cut between two of them is merged inside the kernel, through
+ *    per-SM slots and one word per (sequence, group of 4 KV heads). It does
+ *    not use partition_size. Its scratch (about 2.5 MB at G = 4, 5 MB at
+ *    G = 8) is needed on those shapes whatever the context length.
+ * Returns the larger of the two needs (0 when neither kernel needs any). Same
+ * arguments as the pa_decode call it sizes; never fails (nonsense sizes give 0).
  */
 size_t pa_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len,
                          int partition_size);
@@ -99,9 +106,11 @@ size_t pa_workspace_size(int B, int Hq, int Hkv, int D, int max_context_len,
  * scale         softmax scale (usually 1/sqrt(D)).
  * max_context_len  host-side upper bound of context_lens (no device read is
  *               needed to size the launch); a larger length is an error bit.
- * partition_size   0 = auto, else split into partitions of this many tokens.
+ * partition_size   0 = auto, else split into partitions of this many tokens
+ *               (CUDA-core kernel; the tensor-core kernel splits its own way).
  * workspace     device scratch of at least pa_workspace_size(...) bytes, or
- *               NULL when that size is 0. Overwritten; the caller owns it.
+ *               NULL when that size is 0. Overwritten; the caller owns it; its
+ *               initial contents do not matter.
  * err_flag      nullable device uint32, see PA_DEV_*.
  * stream        cudaStream_t.
  *
@@ -224,8 +233,10 @@ int pa_reshape_and_cache_fp8(const void* key, const void* value, int src_dtype, 
  * k_scale, v_scale
  *               positive finite scales (else PA_ERR_SHAPE).
  * Every other argument, the workspace (sized by pa_workspace_size), the
- * supported shapes and the error behaviour are those of pa_decode. All shapes
- * run on the CUDA-core decode kernel.
+ * supported shapes and the error behaviour are those of pa_decode. With a
+ * 16-bit query on the tensor-core kernel's shapes the codes are widened to the
+ * query's type on the chip (exactly) and the products run on the tensor cores;
+ * every other call runs on the CUDA-core decode kernel.
  */
 int pa_decode_fp8(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
                   const void* value_cache, float k_scale, float v_scale,
@@ -369,14 +380,35 @@ int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cach
                int num_blocks, float scale, int max_context_len, uint32_t* err_flag,
                void* stream);
 
+/*
+ * pa_prefill_kv -- pa_prefill over pools of other element types than the
+ * query's: FP8 E4M3 codes (times k_scale / v_scale) in either pool or both, the
+ * other pool of the query's 16-bit type. The FP8 KV cache and the mixed
+ * configuration of the explainer ("vLLM与PagedAttention：大模型推理内存优化技术
+ * 解析" section 6.1) hold the same tokens a prompt's chunks attend.
+ * query        [T, Hq, D] of q_dtype (PA_F16 or PA_BF16);
+ * key_cache    of k_dtype, value_cache of v_dtype: each q_dtype or PA_FP8_E4M3;
+ * k_scale, v_scale  positive finite scales of the FP8 pools (ignored for others).
+ * Every other argument and the errors are pa_prefill's. The codes are widened
+ * to the query's type on the chip, exactly.
+ */
+int pa_prefill_kv(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                  int k_dtype, float k_scale, const void* value_cache, int v_dtype, float v_scale,
+                  const int32_t* block_tables, int max_blocks_per_seq,
+                  const int32_t* context_lens, const int32_t* query_start, int B, int T,
+                  int max_query_len, int Hq, int Hkv, int D, int block_size, int num_blocks,
+                  float scale, int max_context_len, uint32_t* err_flag, void* stream);
+
 /* Static text for a pa_status value. */
 const char* pa_status_string(int status);
 
 /*
  * pa_decode_plan -- what pa_decode will launch for these arguments, for
- * tools and tests (dtype = PA_FP8_E4M3 plans pa_decode_fp8, whose pools hold
- * codes): *kernel = 1 (CUDA-core path) or 2 (tcgen05 GQA path),
- * *num_partitions = partitions per sequence in the split pass (1 = no split),
+ * tools and tests (dtype = PA_FP8_E4M3 plans pa_decode_fp8 with a 16-bit
+ * query; an fp32 query always takes the CUDA-core kernel): *kernel = 1
+ * (CUDA-core path) or 2 (tcgen05 GQA path), *num_partitions = partitions per
+ * sequence of the CUDA-core split pass (1 = no split; always 1 for the
+ * tensor-core kernel, which splits the work over the SMs itself),
  * *partition_tokens = their length. Any pointer may be NULL. Returns a
  * pa_status (PA_ERR_UNSUPPORTED etc. for the same reasons pa_decode would).
  */

@@ -438,20 +438,34 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   return rc;
 }
 
-int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cache,
-               const void* value_cache, int dtype, const int32_t* block_tables,
-               int max_blocks_per_seq, const int32_t* context_lens, const int32_t* query_start,
-               int B, int T, int max_query_len, int Hq, int Hkv, int D, int block_size,
-               int num_blocks, float scale, int max_context_len, uint32_t* err_flag,
-               void* stream) {
-  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
-  if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_DTYPE;
+}  // extern "C"
+
+namespace {
+
+// Shared body of pa_prefill and pa_prefill_kv.
+int prefill_impl(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                 int k_dtype, float k_scale, const void* value_cache, int v_dtype, float v_scale,
+                 const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                 const int32_t* query_start, int B, int T, int max_query_len, int Hq, int Hkv,
+                 int D, int block_size, int num_blocks, float scale, int max_context_len,
+                 uint32_t* err_flag, void* stream) {
+  if (q_dtype < PA_F32 || q_dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (out_dtype != PA_F32 && out_dtype != q_dtype) return PA_ERR_DTYPE;
+  const bool k8 = k_dtype == PA_FP8_E4M3, v8 = v_dtype == PA_FP8_E4M3;
+  if ((!k8 && k_dtype != q_dtype) || (!v8 && v_dtype != q_dtype)) return PA_ERR_DTYPE;
   if (B < 0 || T < 0 || max_query_len < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 ||
       num_blocks < 0 || max_blocks_per_seq <= 0 || max_context_len < 0)
     return PA_ERR_SHAPE;
   if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
-  if (!prefix_tc_supported(dtype, Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
+  if (!prefix_tc_supported(q_dtype, Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
   if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if ((k8 && !scale_ok(k_scale)) || (v8 && !scale_ok(v_scale))) return PA_ERR_SHAPE;
+  // the kernel with the query rows on the MMA's M, unless PA_PREFILL_KERNEL=mq
+  // asks for the multi-query kernel (for measurements; 16-bit pools only)
+  const char* ov = std::getenv("PA_PREFILL_KERNEL");
+  const bool mq = ov && !std::strcmp(ov, "mq");
+  const bool fa = prefill_fa_supported(q_dtype, Hq, Hkv, D, block_size) && !(mq && !k8 && !v8);
+  if ((k8 || v8) && !fa) return PA_ERR_UNSUPPORTED;
   if (B == 0 || T == 0 || max_query_len == 0) return PA_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
       !query_start)
@@ -460,21 +474,50 @@ int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cach
     return PA_ERR_ALIGN;
   PrefillLaunch p{};
   p.out = out; p.out_dtype = out_dtype; p.q = query;
-  p.k_cache = key_cache; p.v_cache = value_cache; p.dtype = dtype;
+  p.k_cache = key_cache; p.v_cache = value_cache; p.dtype = q_dtype;
+  p.k_dtype = k8 ? PA_FP8_E4M3 : q_dtype;
+  p.v_dtype = v8 ? PA_FP8_E4M3 : q_dtype;
+  p.v_scale = v8 ? v_scale : 1.f;
   p.block_tables = block_tables; p.max_blocks = max_blocks_per_seq;
   p.context_lens = context_lens; p.query_start = query_start;
   p.B = B; p.T = T; p.max_query_len = max_query_len; p.Hq = Hq; p.Hkv = Hkv; p.bs = block_size;
   p.num_blocks = num_blocks;
-  p.scale_log2 = scale * kLog2e;
+  p.scale_log2 = scale * kLog2e * (k8 ? k_scale : 1.f);
   p.max_context_len = max_context_len;
   p.err_flag = err_flag;
-  // the kernel with the query rows on the MMA's M, unless PA_PREFILL_KERNEL=mq
-  // asks for the multi-query kernel (for measurements)
-  const char* ov = std::getenv("PA_PREFILL_KERNEL");
-  const bool mq = ov && !std::strcmp(ov, "mq");
-  if (!mq && prefill_fa_supported(dtype, Hq, Hkv, D, block_size))
-    return launch_prefill_fa(p, static_cast<cudaStream_t>(stream));
+  if (fa) return launch_prefill_fa(p, static_cast<cudaStream_t>(stream));
   return launch_prefill_tc(p, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_prefill(void* out, int out_dtype, const void* query, const void* key_cache,
+               const void* value_cache, int dtype, const int32_t* block_tables,
+               int max_blocks_per_seq, const int32_t* context_lens, const int32_t* query_start,
+               int B, int T, int max_query_len, int Hq, int Hkv, int D, int block_size,
+               int num_blocks, float scale, int max_context_len, uint32_t* err_flag,
+               void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  return prefill_impl(out, out_dtype, query, dtype, key_cache, dtype, 1.f, value_cache, dtype, 1.f,
+                      block_tables, max_blocks_per_seq, context_lens, query_start, B, T,
+                      max_query_len, Hq, Hkv, D, block_size, num_blocks, scale, max_context_len,
+                      err_flag, stream);
+}
+
+int pa_prefill_kv(void* out, int out_dtype, const void* query, int q_dtype, const void* key_cache,
+                  int k_dtype, float k_scale, const void* value_cache, int v_dtype, float v_scale,
+                  const int32_t* block_tables, int max_blocks_per_seq,
+                  const int32_t* context_lens, const int32_t* query_start, int B, int T,
+                  int max_query_len, int Hq, int Hkv, int D, int block_size, int num_blocks,
+                  float scale, int max_context_len, uint32_t* err_flag, void* stream) {
+  if (k_dtype < PA_F32 || k_dtype > PA_FP8_E4M3 || v_dtype < PA_F32 || v_dtype > PA_FP8_E4M3)
+    return PA_ERR_DTYPE;
+  return prefill_impl(out, out_dtype, query, q_dtype, key_cache, k_dtype, k_scale, value_cache,
+                      v_dtype, v_scale, block_tables, max_blocks_per_seq, context_lens,
+                      query_start, B, T, max_query_len, Hq, Hkv, D, block_size, num_blocks,
+                      scale, max_context_len, err_flag, stream);
 }
 
 int pa_swap_blocks(void* dst_key, void* dst_value, const void* src_key, const void* src_value,

@@ -96,7 +96,9 @@ struct PrefillLaunch {
   const void* q;                // [T, Hq, D]
   const void* k_cache;
   const void* v_cache;
-  int dtype;
+  int dtype;                    // query type (16-bit)
+  int k_dtype, v_dtype;         // pool types: dtype, or PA_FP8_E4M3 (codes times the scale)
+  float v_scale;                // FP8 V pool's scale (K's is in scale_log2)
   const int32_t* block_tables;
   int max_blocks;
   const int32_t* context_lens;  // [B] tokens in the cache after the chunk

@@ -72,7 +72,8 @@ constexpr int OFF_KV = 2 * kOp;                 // [kNST][32 KB]
 constexpr int OFF_BAR = OFF_KV + kNST * kOp;
 enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY = B_QFULL + 2,
        B_SFULL = B_QEMPTY + 2, B_PREADY = B_SFULL + 2, B_OSTEP = B_PREADY + 2,
-       B_ODONE = B_OSTEP + 1, B_DONE = B_ODONE + 2, B_COUNT };
+       B_ODONE = B_OSTEP + 1, B_DONE = B_ODONE + 2, B_CONV = B_DONE + 1,
+       B_COUNT = B_CONV + kNST };
 constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
 constexpr int kSmem = OFF_MISC + 16 + 1024;     // + alignment slack
 static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
@@ -87,6 +88,7 @@ struct FaArgs {
   const int32_t* query_start;
   int B, Hq, Hkv, bs, num_blocks, chunks;
   float scale_log2;
+  float v_scale;        // value of one V unit (FP8 V pool; 1 otherwise)
   int max_context_len;
   uint32_t* err_flag;
 };
@@ -144,7 +146,13 @@ __device__ __forceinline__ void split2(float p0, float p1, uint32_t& hi, uint32_
   }
 }
 
-template <int FMT, int BS, int G>
+// K8 / V8: that pool holds FP8 E4M3 codes. TMA brings a tile's codes (one
+// 128-byte line per row, at the stage's upper half) and the softmax thread
+// that owns the tile row widens it in place to the query's 16-bit type
+// (exact) before the tile is released to the tensor cores. A unit's first
+// tile is widened before its scores; each later tile right after the weights
+// of the tile before it are handed over, beside that tile's output product.
+template <int FMT, int BS, int G, bool K8, bool V8>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
@@ -176,6 +184,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
     }
     mbar_init(bar(B_OSTEP), 1);
     mbar_init(bar(B_DONE), 1);
+    for (int s = 0; s < kNST; ++s) mbar_init(bar(B_CONV + s), 128);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -196,6 +205,11 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
   auto give_up = [&]() {
     *abort_flag = 1u;
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
+  };
+  // a stage holding K (kv = 0) or V (kv = 1) is ready for the tensor cores when
+  // TMA filled it (16-bit pool) or when the softmax group widened it (FP8 pool)
+  auto ready_bar = [&](int kv, int s) {
+    return bar(((kv ? V8 : K8) ? B_CONV : B_FULL) + s);
   };
 
   if (warp == 4) {
@@ -227,19 +241,25 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
               flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
               phys[q] = -1;
             }
-            if (phys[q] >= 0) bytes += 2u * BS * 128u;
+            if (phys[q] >= 0) bytes += BS * 128u;                // per 128-byte line of rows
           }
           for (int kv = 0; kv < 2; ++kv) {
             const int seq = 2 * tc_ + kv, s = seq % kNST;
+            const bool codes = kv ? V8 : K8;
             if (!mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-            mbar_expect_tx(bar(B_FULL + s), bytes);
+            mbar_expect_tx(bar(B_FULL + s), codes ? bytes : 2u * bytes);
             const uint32_t dst = sbase + OFF_KV + s * kOp;
 #pragma unroll
             for (int q = 0; q < NB_T; ++q) {
               if (phys[q] < 0) continue;
-              for (int hh = 0; hh < 2; ++hh)
-                tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
-                            phys[q], bar(B_FULL + s));
+              if (codes) {
+                tma_load_4d(dst + kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, phys[q],
+                            bar(B_FULL + s));
+              } else {
+                for (int hh = 0; hh < 2; ++hh)
+                  tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
+                              phys[q], bar(B_FULL + s));
+              }
             }
             ++issued;
           }
@@ -272,7 +292,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         if (first && ui >= 2 && !mbar_wait(bar(B_ODONE + ob), ((ui - 2) >> 1) & 1, abort_flag))
           return false;
         const int seq = 2 * tt + 1, s = seq % kNST;
-        if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) return false;
+        if (!mbar_wait(ready_bar(1, s), (seq / kNST) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vst = sbase + OFF_KV + s * kOp;
 #pragma unroll
@@ -297,7 +317,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         for (int k = 0; k < x.ntiles; ++k, ++tc_) {
           const int sb = tc_ & 1;
           const int seq = 2 * tc_, s = seq % kNST;
-          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(ready_bar(0, s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + OFF_KV + s * kOp;
 #pragma unroll
@@ -334,18 +354,40 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       const int pos = x.pos0 + tl;               // this row attends keys [0, pos]
       const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
       float m = -CUDART_INF_F, l = 0.f;
+      // blocks of tile j with a bad id (the producer loaded nothing there)
+      auto tile_bad = [&](int j) {
+        const int tsj = j * kTile;
+        const int nb = (min(x.t1, tsj + kTile) - tsj + BS - 1) / BS;
+        uint32_t bb = 0;
+#pragma unroll
+        for (int q = 0; q < NB_T; ++q) {
+          if (q >= nb) continue;
+          const int ph = __ldg(table + tsj / BS + q);
+          if (ph < 0 || ph >= a.num_blocks) bb |= 1u << q;
+        }
+        return bb;
+      };
+      // FP8 pools: widen row r of tile j's K and V stages (global tile tj); a V
+      // row no row of the unit attends becomes zeros
+      auto widen_tile = [&](int j, int tj) {
+        if constexpr (K8 || V8) {
+          const bool zv = j * kTile + r >= x.t1 || ((tile_bad(j) >> (r / BS)) & 1u);
+#pragma unroll 1
+          for (int kv = 0; kv < 2; ++kv) {
+            if (!(kv ? V8 : K8)) continue;
+            const int seq = 2 * tj + kv, s = seq % kNST;
+            if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) failed = true;
+            if (!failed) widen_row_fp8<FMT>(smem + OFF_KV + s * kOp, r, kv == 1 && zv);
+            fence_proxy_async();
+            mbar_arrive(bar(B_CONV + s));
+          }
+        }
+      };
+      widen_tile(0, tc_);
       for (int k = 0; k < x.ntiles; ++k, ++tc_) {
         const int sb = tc_ & 1;
         const int ts = k * kTile;
-        // keys of this tile in a block with a bad id (the producer loaded nothing there)
-        uint32_t badblk = 0;
-        const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
-#pragma unroll
-        for (int q = 0; q < NB_T; ++q) {
-          if (q >= nblk) continue;
-          const int ph = __ldg(table + ts / BS + q);
-          if (ph < 0 || ph >= a.num_blocks) badblk |= 1u << q;
-        }
+        const uint32_t badblk = tile_bad(k);
         // V row r of the stage: zero if no row of the unit attends key ts + r
         const bool zero_v = ts + r >= x.t1 || ((badblk >> (r / BS)) & 1u);
         if (!mbar_wait(bar(B_SFULL + sb), (tc_ >> 1) & 1, abort_flag)) failed = true;
@@ -407,7 +449,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           tmem_st32(tmem_s + lane_off + sb * kTile + c / 2, hi);
           tmem_st32(tmem_s + lane_off + sb * kTile + 64 + c / 2, lo);
         }
-        if (zero_v) {
+        if (!V8 && zero_v) {
           // this V row enters the output product with weight 0: it must hold finite values
           const int seq = 2 * tc_ + 1, s = seq % kNST;
           if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) failed = true;
@@ -421,6 +463,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         tc_fence_before();
         mbar_arrive(bar(B_PREADY + sb));
         ++ostep;
+        if (k + 1 < x.ntiles) widen_tile(k + 1, tc_ + 1);
       }
       // ---- epilogue: O / l of this row to the output. The products of the
       // last two tiles may both be pending; a parity wait names one of two
@@ -428,7 +471,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       if (ostep >= 2 && !mbar_wait(bar(B_OSTEP), (ostep - 2) & 1, abort_flag)) failed = true;
       if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? a.v_scale / l : 0.f;
       const size_t orow = ((size_t)(x.qrow0 + tl) * a.Hq + (size_t)x.h * G + g) * kD;
 #pragma unroll 1
       for (int c = 0; c < kD; c += 32) {
@@ -499,7 +542,8 @@ PFN_cuTensorMapEncodeTiled_v12000 fa_encode_fn() {
 // heads x one d-half lands as 128 rows (token-major, then head) of 128 B,
 // 128-byte swizzled. Pools [NB][bs][Hkv][128] seen as [NB][2][Hkv][bs][64]: a
 // box of one block's bs rows of one head and one d-half.
-bool make_fa_maps(const PrefillLaunch& p, int G, CUtensorMap* q, CUtensorMap* k, CUtensorMap* v) {
+bool make_fa_maps(const PrefillLaunch& p, int G, bool k8, bool v8, CUtensorMap* q, CUtensorMap* k,
+                  CUtensorMap* v) {
   auto enc = fa_encode_fn();
   if (!enc || p.num_blocks <= 0) return false;
   const CUtensorMapDataType dt =
@@ -517,19 +561,31 @@ bool make_fa_maps(const PrefillLaunch& p, int G, CUtensorMap* q, CUtensorMap* k,
                                  (cuuint64_t)p.bs * p.Hkv * kD * 2};
   const cuuint32_t box[5] = {64, (cuuint32_t)p.bs, 1, 1, 1};
   const cuuint32_t es5[5] = {1, 1, 1, 1, 1};
+  // FP8 pool [NB][bs][Hkv][128 codes]: a box of one block's bs rows of one head,
+  // one 128-byte line per row
+  const cuuint64_t cdims[4] = {(cuuint64_t)kD, (cuuint64_t)p.bs, (cuuint64_t)p.Hkv,
+                               (cuuint64_t)p.num_blocks};
+  const cuuint64_t cstr[3] = {(cuuint64_t)p.Hkv * kD, (cuuint64_t)kD, (cuuint64_t)p.bs * p.Hkv * kD};
+  const cuuint32_t cbox[4] = {(cuuint32_t)kD, (cuuint32_t)p.bs, 1, 1};
   for (int i = 0; i < 2; ++i) {
-    if (enc(i == 0 ? k : v, dt, 5, const_cast<void*>(i == 0 ? p.k_cache : p.v_cache), dims,
-            strides, box, es5, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return false;
+    void* pool = const_cast<void*>(i == 0 ? p.k_cache : p.v_cache);
+    const bool codes = i == 0 ? k8 : v8;
+    const CUresult r =
+        codes ? enc(i == 0 ? k : v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, pool, cdims, cstr, cbox, es4,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
+              : enc(i == 0 ? k : v, dt, 5, pool, dims, strides, box, es5,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
   }
   return true;
 }
 
-template <int FMT, int BS, int G>
+template <int FMT, int BS, int G, bool K8, bool V8>
 int launch_fa_t(const FaArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                 cudaStream_t stream) {
-  auto kern = prefill_fa_kernel<FMT, BS, G>;
+  auto kern = prefill_fa_kernel<FMT, BS, G, K8, V8>;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
@@ -544,17 +600,27 @@ int launch_fa_t(const FaArgs& a, const CUtensorMap& q, const CUtensorMap& k, con
                  cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-template <int FMT, int BS>
+template <int FMT, int BS, bool K8, bool V8>
 int launch_fa_g(const FaArgs& a, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                 cudaStream_t stream) {
   switch (a.Hq / a.Hkv) {
-    case 1: return launch_fa_t<FMT, BS, 1>(a, q, k, v, stream);
-    case 2: return launch_fa_t<FMT, BS, 2>(a, q, k, v, stream);
-    case 4: return launch_fa_t<FMT, BS, 4>(a, q, k, v, stream);
-    case 8: return launch_fa_t<FMT, BS, 8>(a, q, k, v, stream);
-    case 16: return launch_fa_t<FMT, BS, 16>(a, q, k, v, stream);
+    case 1: return launch_fa_t<FMT, BS, 1, K8, V8>(a, q, k, v, stream);
+    case 2: return launch_fa_t<FMT, BS, 2, K8, V8>(a, q, k, v, stream);
+    case 4: return launch_fa_t<FMT, BS, 4, K8, V8>(a, q, k, v, stream);
+    case 8: return launch_fa_t<FMT, BS, 8, K8, V8>(a, q, k, v, stream);
+    case 16: return launch_fa_t<FMT, BS, 16, K8, V8>(a, q, k, v, stream);
   }
   return PA_ERR_UNSUPPORTED;
+}
+
+template <bool K8, bool V8>
+int launch_fa_kv(const FaArgs& a, int dtype, int bs, const CUtensorMap& q, const CUtensorMap& k,
+                 const CUtensorMap& v, cudaStream_t stream) {
+  if (dtype == PA_BF16)
+    return bs == 16 ? launch_fa_g<1, 16, K8, V8>(a, q, k, v, stream)
+                    : launch_fa_g<1, 32, K8, V8>(a, q, k, v, stream);
+  return bs == 16 ? launch_fa_g<0, 16, K8, V8>(a, q, k, v, stream)
+                  : launch_fa_g<0, 32, K8, V8>(a, q, k, v, stream);
 }
 
 }  // namespace
@@ -568,8 +634,9 @@ bool prefill_fa_supported(int dtype, int Hq, int Hkv, int D, int bs) {
 
 int launch_prefill_fa(const PrefillLaunch& p, cudaStream_t stream) {
   const int G = p.Hq / p.Hkv;
+  const bool k8 = p.k_dtype == PA_FP8_E4M3, v8 = p.v_dtype == PA_FP8_E4M3;
   CUtensorMap q, k, v;
-  if (!make_fa_maps(p, G, &q, &k, &v)) return PA_ERR_CUDA;
+  if (!make_fa_maps(p, G, k8, v8, &q, &k, &v)) return PA_ERR_CUDA;
   FaArgs a{};
   a.out = p.out;
   a.out_dtype = p.out_dtype;
@@ -580,11 +647,13 @@ int launch_prefill_fa(const PrefillLaunch& p, cudaStream_t stream) {
   a.B = p.B; a.Hq = p.Hq; a.Hkv = p.Hkv; a.bs = p.bs; a.num_blocks = p.num_blocks;
   a.chunks = (p.max_query_len + kM / G - 1) / (kM / G);
   a.scale_log2 = p.scale_log2;
+  a.v_scale = v8 ? p.v_scale : 1.f;
   a.max_context_len = p.max_context_len;
   a.err_flag = p.err_flag;
-  if (p.dtype == PA_BF16)
-    return p.bs == 16 ? launch_fa_g<1, 16>(a, q, k, v, stream) : launch_fa_g<1, 32>(a, q, k, v, stream);
-  return p.bs == 16 ? launch_fa_g<0, 16>(a, q, k, v, stream) : launch_fa_g<0, 32>(a, q, k, v, stream);
+  if (k8 && v8) return launch_fa_kv<true, true>(a, p.dtype, p.bs, q, k, v, stream);
+  if (k8) return launch_fa_kv<true, false>(a, p.dtype, p.bs, q, k, v, stream);
+  if (v8) return launch_fa_kv<false, true>(a, p.dtype, p.bs, q, k, v, stream);
+  return launch_fa_kv<false, false>(a, p.dtype, p.bs, q, k, v, stream);
 }
 
 }  // namespace pa

@@ -6,6 +6,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace pa {
@@ -218,6 +219,53 @@ __device__ __forceinline__ void mma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, uin
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// FP8 pools: two E4M3 codes (one 16-bit word) -> two 16-bit values of the
+// query's type, exactly. E4M3 -> f16 is exact (every E4M3 value is a normal
+// f16 or zero); f16 -> bf16 is then exact too (3 fraction bits, exponent in
+// range): the bf16 pattern is the f16 magnitude shifted right by 3 with the
+// exponent rebased (+112), zero staying zero.
+template <int FMT>
+__device__ __forceinline__ uint32_t widen2_e4m3(uint32_t codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xffffu),
+                                                   __NV_E4M3);
+  const uint32_t f = (uint32_t)h.x | ((uint32_t)h.y << 16);
+  if (FMT == 0) return f;
+  const uint32_t mag = f & 0x7fff7fffu;
+  const uint32_t b = (mag >> 3) + 0x38003800u;             // no carry between the halves
+  return (f & 0x80008000u) | (b & ~__vcmpeq2(mag, 0u));
+}
+
+// Widen tile row `row` of a stage in place: its 128 E4M3 codes sit at the
+// stage's upper 16 KB (one 128-byte-swizzled row, as TMA wrote them) and
+// become the row of both 64-wide d-halves of the 16-bit operand layout (the
+// second of which is that very line). Only this thread touches the row, and
+// it reads the whole line before it writes; zero writes zeros instead.
+template <int FMT>
+__device__ __forceinline__ void widen_row_fp8(uint8_t* stage, int row, bool zero) {
+  constexpr int kHalf = 128 * 128;           // one 64-wide d-half of a 128-row operand
+  const int sw = row & 7;
+  uint8_t* src = stage + kHalf + row * 128;
+  uint4 c[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    c[j] = zero ? make_uint4(0, 0, 0, 0) : *reinterpret_cast<const uint4*>(src + ((j ^ sw) << 4));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // codes 16j .. 16j + 15 -> d-half j / 4, 16-byte chunks 2 (j % 4) and 2 (j % 4) + 1
+    const uint32_t w[4] = {c[j].x, c[j].y, c[j].z, c[j].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[2 * k] = widen2_e4m3<FMT>(w[k]);
+      o[2 * k + 1] = widen2_e4m3<FMT>(w[k] >> 16);
+    }
+    uint8_t* dst = stage + (j >> 2) * kHalf + row * 128;
+    const int c0 = 2 * (j & 3);
+    *reinterpret_cast<uint4*>(dst + ((c0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + (((c0 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
 // Plain named-barrier sync of one softmax group.
 __device__ __forceinline__ void wg_sync(int group) {
   asm volatile("bar.sync %0, 128;" ::"r"(1 + group) : "memory");

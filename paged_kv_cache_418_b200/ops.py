@@ -70,6 +70,9 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_kv.restype = I
     lib.pa_reshape_and_cache_kv.argtypes = [P, P, I, P, I, F, P, I, F, P, I, I, I, I, I, P, P]
     lib.pa_reshape_and_cache_kv.restype = I
+    lib.pa_prefill_kv.argtypes = [P, I, P, I, P, I, F, P, I, F, P, I, P, P, I, I, I, I, I, I, I, I,
+                                  F, I, P, P]
+    lib.pa_prefill_kv.restype = I
     return lib
 
 
@@ -381,6 +384,29 @@ def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
                             _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_prefill", rc)
+
+
+def pa_prefill_kv(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                  value_cache: torch.Tensor, k_scale: float, v_scale: float,
+                  block_tables: torch.Tensor, context_lens: torch.Tensor,
+                  query_start: torch.Tensor, max_query_len: int, scale: float,
+                  max_context_len: int, err_flag: Optional[torch.Tensor] = None,
+                  stream=None) -> None:
+    """pa_prefill over pools of per-pool types (uint8 = FP8 E4M3 codes read times
+    the pool's scale; see pa_prefill_kv in include/pa.h)."""
+    T, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    B = query_start.shape[0] - 1
+    with _on_device_of(query):
+        rc = LIB.pa_prefill_kv(_ptr(out), pa_dtype(out), _ptr(query), pa_dtype(query),
+                               _ptr(key_cache), pa_dtype(key_cache), float(k_scale),
+                               _ptr(value_cache), pa_dtype(value_cache), float(v_scale),
+                               _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                               _ptr(query_start), B, T, int(max_query_len), Hq, Hkv, D,
+                               block_size, num_blocks, float(scale), int(max_context_len),
+                               _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_prefill_kv", rc)
 
 
 def shared_prefix_workspace_for(query: torch.Tensor, key_cache: torch.Tensor,

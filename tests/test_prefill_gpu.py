@@ -101,3 +101,53 @@ def test_prefill_bad_block_id_is_flagged_and_left_out():
     torch.cuda.synchronize()
     assert int(err.item()) & ops.PA_DEV_BAD_BLOCK_ID
     assert torch.isfinite(out).all()
+
+
+def _codes_like(pool, dtype, rng):
+    """An FP8 code pool with the same filled rows as a 16-bit pool (random codes
+    there, the NaN code where the 16-bit pool holds NaN)."""
+    filled = ~np.isnan(W.storage_to_float64(pool, dtype)).any(axis=-1)
+    codes = np.full(pool.shape, 0x7F, dtype=np.uint8)
+    codes[filled] = W.random_e4m3_codes(rng, (int(filled.sum()), pool.shape[-1]))
+    return codes
+
+
+@pytest.mark.parametrize("k8,v8", [(True, True), (True, False), (False, True)])
+@pytest.mark.parametrize("qdt,G,bs", [(W.BF16, 8, 16), (W.F16, 1, 32), (W.BF16, 4, 32),
+                                      (W.F16, 16, 16)])
+def test_prefill_over_fp8_and_mixed_pools(k8, v8, qdt, G, bs, prefill_kernel):
+    if prefill_kernel == "multi-query":
+        pytest.skip("FP8 pools run on the kernel with the query rows on M")
+    rng = np.random.default_rng(G * 7 + bs + 3 * k8 + v8)
+    c = W.build_prefill_case("pf-fp8", qdt, Hq=2 * G, Hkv=2, D=128, block_size=bs,
+                             prior_lens=[0, 5, 130, 300], new_lens=[40, 1, 2 * bs + 3, 129],
+                             seed=G * 10 + bs + qdt)
+    kc = _codes_like(c.k_cache, qdt, rng) if k8 else c.k_cache
+    vc = _codes_like(c.v_cache, qdt, rng) if v8 else c.v_cache
+    ks, vs = float(np.float32(0.3)), float(np.float32(0.6))
+    t = W.prefill_to_torch(c, "cuda")
+    tk = torch.from_numpy(kc).cuda() if k8 else t["k_cache"]
+    tv = torch.from_numpy(vc).cuda() if v8 else t["v_cache"]
+    for out_dtype in (torch.float32, {W.BF16: torch.bfloat16, W.F16: torch.float16}[qdt]):
+        out = torch.full((c.T, c.Hq, c.D), float("nan"), dtype=out_dtype, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ops.pa_prefill_kv(out, t["q"], tk, tv, ks, vs, t["block_tables"], t["context_lens"],
+                          t["query_start"], c.max_query_len, c.scale, c.max_context_len, err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        ref = oracle.prefill_mixed(c.q, qdt, kc, oracle.FP8 if k8 else qdt, ks, vc,
+                                   oracle.FP8 if v8 else qdt, vs, c.block_tables, c.context_lens,
+                                   c.query_start, c.scale)
+        assert_attention_close(out, ref, qdt, f"k8={k8} v8={v8} G={G} out={out_dtype}")
+
+
+def test_prefill_kv_refuses_an_fp32_query(prefill_kernel):
+    q = torch.zeros(4, 8, 128, dtype=torch.float32, device="cuda")
+    kc = torch.zeros(4, 16, 2, 128, dtype=torch.uint8, device="cuda")
+    tables = torch.zeros(1, 4, dtype=torch.int32, device="cuda")
+    lens = torch.full((1,), 4, dtype=torch.int32, device="cuda")
+    qs = torch.tensor([0, 4], dtype=torch.int32, device="cuda")
+    out = torch.zeros(4, 8, 128, dtype=torch.float32, device="cuda")
+    with pytest.raises(ops.PAError) as e:
+        ops.pa_prefill_kv(out, q, kc, kc, 0.5, 0.5, tables, lens, qs, 4, 0.1, 64)
+    assert e.value.status in (3, 4)
