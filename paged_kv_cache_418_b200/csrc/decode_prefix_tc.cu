@@ -78,7 +78,8 @@ constexpr int OFF_MREF = OFF_P + 2 * kPBuf;     // [3][kNQ] reference, old, new 
 constexpr int OFF_RED = OFF_MREF + 3 * kNQ * 4; // [4 warps][kNQ]
 constexpr int OFF_BAR = OFF_RED + 4 * kNQ * 4;
 enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY, B_SFULL, B_SFREE = B_SFULL + 2,
-       B_PREADY = B_SFREE + 2, B_OFULL = B_PREADY + 2, B_ODONE = B_OFULL + 2, B_DONE, B_COUNT };
+       B_PREADY = B_SFREE + 2, B_OFULL = B_PREADY + 2, B_ODONE = B_OFULL + 2, B_DONE,
+       B_CONV, B_COUNT = B_CONV + kNST };
 constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
 constexpr int kSmem = OFF_MISC + 32 + 1024;
 static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
@@ -95,6 +96,7 @@ struct PrefixArgs {
   int part_tokens;                              // tokens per prefix partition (multiple of 128)
   int B, Hq, Hkv, bs, num_blocks;
   float scale_log2;
+  float v_scale;                                // value of one V unit (FP8 V pool; 1 otherwise)
   int P;                                        // workspace slots per sequence
   float* ws_acc;
   float* ws_m;
@@ -187,7 +189,11 @@ __device__ __forceinline__ bool sm_vote(bool x) {
   return r != 0;
 }
 
-template <int FMT, int BS, bool PF>
+// K8 / V8 (shared-prefix mode): that pool holds FP8 E4M3 codes. TMA brings a
+// tile's codes (one 128-byte line per row, at the stage's upper half) and the
+// threads of the first query columns (one per tile row) widen them in place
+// to the query's 16-bit type, exactly, before the tile goes to the tensor cores.
+template <int FMT, int BS, bool PF, bool K8 = false, bool V8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
 multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV) {
@@ -221,6 +227,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
     }
     mbar_init(bar(B_ODONE), kSoft);
     mbar_init(bar(B_DONE), 1);
+    for (int s = 0; s < kNST; ++s) mbar_init(bar(B_CONV + s), 128);
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -241,6 +248,11 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
   auto give_up = [&]() {
     *abort_flag = 1u;
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
+  };
+  // a stage holding K (kv = 0) or V (kv = 1) is ready for the tensor cores when
+  // TMA filled it (16-bit pool) or when its rows were widened (FP8 pool)
+  auto ready_bar = [&](int kv, int s) {
+    return bar(((kv ? V8 : K8) ? B_CONV : B_FULL) + s);
   };
 
   if (warp == kSoftWarps) {
@@ -274,19 +286,25 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
               flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
               phys[q] = -1;
             }
-            if (phys[q] >= 0) bytes += 2u * BS * 128u;
+            if (phys[q] >= 0) bytes += BS * 128u;                // per 128-byte line of rows
           }
           for (int kv = 0; kv < 2; ++kv) {
             const int seq = 2 * tc_ + kv, s = seq % kNST;
+            const bool codes = kv ? V8 : K8;
             if (!mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-            mbar_expect_tx(bar(B_FULL + s), bytes);
+            mbar_expect_tx(bar(B_FULL + s), codes ? bytes : 2u * bytes);
             const uint32_t dst = sbase + s * kStage;
 #pragma unroll
             for (int q = 0; q < NB_T; ++q) {
               if (phys[q] < 0) continue;
-              for (int hh = 0; hh < 2; ++hh)
-                tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
-                            phys[q], bar(B_FULL + s));
+              if (codes) {
+                tma_load_4d(dst + kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, phys[q],
+                            bar(B_FULL + s));
+              } else {
+                for (int hh = 0; hh < 2; ++hh)
+                  tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
+                              phys[q], bar(B_FULL + s));
+              }
             }
             ++issued;
           }
@@ -316,7 +334,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
           if (!mbar_wait(bar(B_PREADY + pb), (tt >> 1) & 1, abort_flag)) return false;
           if (first && ua > 0 && !mbar_wait(bar(B_ODONE), (ua - 1) & 1, abort_flag)) return false;
           const int seq = 2 * tt + 1, s = seq % kNST;
-          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) return false;
+          if (!mbar_wait(ready_bar(1, s), (seq / kNST) & 1, abort_flag)) return false;
           tc_fence_after();
           const uint32_t vst = sbase + s * kStage;
           const uint32_t pst = sbase + OFF_P + pb * kPBuf;
@@ -338,7 +356,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
           const int sb = tc_ & 1;
           if (!mbar_wait(bar(B_SFREE + sb), ((tc_ >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
           const int seq = 2 * tc_, s = seq % kNST;
-          if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(ready_bar(0, s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + s * kStage;
 #pragma unroll
@@ -449,6 +467,21 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
         const int qhi = valid ? min(max(x.nq - c0, 0), kHalfCols) : 0;
         const uint32_t mk = qhi > qlo ? ((1u << qhi) - 1u) & ~((1u << qlo) - 1u) : 0u;
         const bool full = __all_sync(0xffffffffu, mk == (1u << kHalfCols) - 1u);
+        if constexpr (K8 || V8) {
+          // widen this tile's rows (threads of the first column block, one per row);
+          // a V row that must not count becomes zeros
+          if (c0 == 0) {
+#pragma unroll 1
+            for (int kv = 0; kv < 2; ++kv) {
+              if (!(kv ? V8 : K8)) continue;
+              const int seq = 2 * tc_ + kv, s = seq % kNST;
+              if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) failed = true;
+              if (!failed) widen_row_fp8<FMT>(smem + s * kStage, r, kv == 1 && !valid);
+              fence_proxy_async();
+              mbar_arrive(bar(B_CONV + s));
+            }
+          }
+        }
         if (!mbar_wait(bar(B_SFULL + (tc_ & 1)), (tc_ >> 1) & 1, abort_flag)) failed = true;
         tc_fence_after();
         float s[kHalfCols];
@@ -532,7 +565,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
           *reinterpret_cast<uint16_t*>(pb + off) = hi;
           *reinterpret_cast<uint16_t*>(pb + kPPart + off) = lo;
         }
-        if (!valid && c0 == 0) {
+        if (!V8 && !valid && c0 == 0) {
           // a row with weight 0 still enters the product: it must hold finite values
           const int seq = 2 * tc_ + 1, sv = seq % kNST;
           if (!mbar_wait(bar(B_FULL + sv), (seq / kNST) & 1, abort_flag)) failed = true;
@@ -579,7 +612,7 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
             const float L = mold[q];
             store_out(a.out, q_row(q) * kD + r, L > 0.f ? o[e] / L : 0.f, a.out_dtype);
           } else {
-            a.ws_acc[slot_row(q) * kD + r] = o[e];
+            a.ws_acc[slot_row(q) * kD + r] = o[e] * a.v_scale;
           }
         }
       }
@@ -619,7 +652,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // The pool [NB][bs][Hkv][D] seen as [NB][2][Hkv][bs][64]: a box of one block's
 // bs rows of one head and one d-half, 128-byte swizzled.
 bool make_prefix_maps(const void* k_cache, const void* v_cache, int dtype, int bs, int Hkv,
-                      int num_blocks, CUtensorMap* k, CUtensorMap* v) {
+                      int num_blocks, CUtensorMap* k, CUtensorMap* v, bool k8 = false,
+                      bool v8 = false) {
   auto enc = encode_fn();
   if (!enc || num_blocks <= 0) return false;
   const CUtensorMapDataType dt =
@@ -629,19 +663,30 @@ bool make_prefix_maps(const void* k_cache, const void* v_cache, int dtype, int b
                                  (cuuint64_t)bs * Hkv * kD * 2};
   const cuuint32_t box[5] = {64, (cuuint32_t)bs, 1, 1, 1};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  // FP8 pool [NB][bs][Hkv][128 codes]: a box of one block's bs rows of one head
+  const cuuint64_t cdims[4] = {(cuuint64_t)kD, (cuuint64_t)bs, (cuuint64_t)Hkv,
+                               (cuuint64_t)num_blocks};
+  const cuuint64_t cstr[3] = {(cuuint64_t)Hkv * kD, (cuuint64_t)kD, (cuuint64_t)bs * Hkv * kD};
+  const cuuint32_t cbox[4] = {(cuuint32_t)kD, (cuuint32_t)bs, 1, 1};
   for (int i = 0; i < 2; ++i) {
-    CUresult r = enc(i == 0 ? k : v, dt, 5, const_cast<void*>(i == 0 ? k_cache : v_cache), dims,
-                     strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    void* pool = const_cast<void*>(i == 0 ? k_cache : v_cache);
+    const CUresult r =
+        (i == 0 ? k8 : v8)
+            ? enc(i == 0 ? k : v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, pool, cdims, cstr, cbox, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE)
+            : enc(i == 0 ? k : v, dt, 5, pool, dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
   }
   return true;
 }
 
-template <int FMT, int BS, bool PF>
+template <int FMT, int BS, bool PF, bool K8 = false, bool V8 = false>
 int launch_mq_t(const PrefixArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                 cudaStream_t stream) {
-  auto kern = multi_query_tc_kernel<FMT, BS, PF>;
+  auto kern = multi_query_tc_kernel<FMT, BS, PF, K8, V8>;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) !=
@@ -672,11 +717,20 @@ int prefix_chunks(int max_group_size, int G) {
   return (max_group_size + mc - 1) / mc;
 }
 
+template <int FMT, int BS>
+int launch_prefix_kv(const PrefixArgs& a, bool k8, bool v8, const CUtensorMap& k,
+                     const CUtensorMap& v, cudaStream_t stream) {
+  if (k8 && v8) return launch_mq_t<FMT, BS, false, true, true>(a, k, v, stream);
+  if (k8) return launch_mq_t<FMT, BS, false, true, false>(a, k, v, stream);
+  if (v8) return launch_mq_t<FMT, BS, false, false, true>(a, k, v, stream);
+  return launch_mq_t<FMT, BS, false>(a, k, v, stream);
+}
+
 int launch_prefix_tc(const DecodeArgs& d, int dtype, const int32_t* group_offsets,
                      const int32_t* group_members, int num_groups, int max_group_size,
-                     int parts, int part_tokens, cudaStream_t stream) {
+                     int parts, int part_tokens, cudaStream_t stream, bool k8, bool v8) {
   CUtensorMap k, v;
-  if (!make_prefix_maps(d.k_cache, d.v_cache, dtype, d.bs, d.Hkv, d.num_blocks, &k, &v))
+  if (!make_prefix_maps(d.k_cache, d.v_cache, dtype, d.bs, d.Hkv, d.num_blocks, &k, &v, k8, v8))
     return PA_ERR_CUDA;
   PrefixArgs a{};
   a.q = d.q;
@@ -694,11 +748,12 @@ int launch_prefix_tc(const DecodeArgs& d, int dtype, const int32_t* group_offset
   a.P = d.P;
   a.ws_acc = d.ws_acc; a.ws_m = d.ws_m; a.ws_l = d.ws_l;
   a.err_flag = d.err_flag;
+  a.v_scale = d.v_scale;
   if (dtype == PA_BF16)
-    return d.bs == 16 ? launch_mq_t<1, 16, false>(a, k, v, stream)
-                      : launch_mq_t<1, 32, false>(a, k, v, stream);
-  return d.bs == 16 ? launch_mq_t<0, 16, false>(a, k, v, stream)
-                    : launch_mq_t<0, 32, false>(a, k, v, stream);
+    return d.bs == 16 ? launch_prefix_kv<1, 16>(a, k8, v8, k, v, stream)
+                      : launch_prefix_kv<1, 32>(a, k8, v8, k, v, stream);
+  return d.bs == 16 ? launch_prefix_kv<0, 16>(a, k8, v8, k, v, stream)
+                    : launch_prefix_kv<0, 32>(a, k8, v8, k, v, stream);
 }
 
 int launch_prefill_tc(const PrefillLaunch& p, cudaStream_t stream) {
@@ -719,6 +774,7 @@ int launch_prefill_tc(const PrefillLaunch& p, cudaStream_t stream) {
   a.chunks = (p.max_query_len + kNQ / (p.Hq / p.Hkv) - 1) / (kNQ / (p.Hq / p.Hkv));
   a.parts = 1;
   a.err_flag = p.err_flag;
+  a.v_scale = 1.f;
   if (p.dtype == PA_BF16)
     return p.bs == 16 ? launch_mq_t<1, 16, true>(a, k, v, stream)
                       : launch_mq_t<1, 32, true>(a, k, v, stream);

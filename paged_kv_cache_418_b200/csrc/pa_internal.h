@@ -112,9 +112,10 @@ int launch_prefill_tc(const PrefillLaunch& p, cudaStream_t stream);
 // Paged prefill with the query rows on the MMA's M (prefill_tc.cu).
 bool prefill_fa_supported(int dtype, int Hq, int Hkv, int D, int bs);
 int launch_prefill_fa(const PrefillLaunch& p, cudaStream_t stream);
+// dtype: the query's (16-bit) type; k8 / v8: that pool holds FP8 E4M3 codes.
 int launch_prefix_tc(const DecodeArgs& a, int dtype, const int32_t* group_offsets,
                      const int32_t* group_members, int num_groups, int max_group_size, int parts,
-                     int part_tokens, cudaStream_t stream);
+                     int part_tokens, cudaStream_t stream, bool k8 = false, bool v8 = false);
 
 int launch_reshape_and_cache(const void* key, const void* value, void* key_cache,
                              void* value_cache, int esize, const int64_t* slot_mapping, int T,
