@@ -350,6 +350,28 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
                             size_t workspace_bytes, uint32_t* err_flag, void* stream);
 
 /*
+ * pa_decode_shared_prefix_kv -- pa_decode_shared_prefix over pools of other
+ * element types than the query's (FP8 E4M3 codes times k_scale / v_scale in
+ * either pool or both; see pa_decode_kv): parallel sampling over an FP8 cache,
+ * or over the explainer's mixed one, reads each group's shared blocks once.
+ * Arguments as pa_decode_shared_prefix, with q_dtype, k_dtype / k_scale and
+ * v_dtype / v_scale as in pa_decode_kv; the workspace is sized by
+ * pa_shared_prefix_workspace_size. Shapes the prefix kernel does not take run
+ * as pa_decode_kv.
+ */
+int pa_decode_shared_prefix_kv(void* out, int out_dtype, const void* query, int q_dtype,
+                               const void* key_cache, int k_dtype, float k_scale,
+                               const void* value_cache, int v_dtype, float v_scale,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* context_lens, const int32_t* shared_blocks,
+                               int num_groups, const int32_t* group_offsets,
+                               const int32_t* group_members, int max_group_size,
+                               int max_shared_blocks, int B, int Hq, int Hkv, int D,
+                               int block_size, int num_blocks, float scale, int max_context_len,
+                               int partition_size, void* workspace, size_t workspace_bytes,
+                               uint32_t* err_flag, void* stream);
+
+/*
  * pa_prefill -- paged prefill (prompt or chunked-prefill) attention: each new
  * query token attends, causally, to its sequence's cached tokens up to and
  * including itself. Long prompts are cut into chunks that run between decode

@@ -357,32 +357,40 @@ size_t pa_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D, int max_co
          tc_workspace_bytes(B, Hq, Hkv, D);
 }
 
-int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const void* key_cache,
-                            const void* value_cache, int dtype, const int32_t* block_tables,
-                            int max_blocks_per_seq, const int32_t* context_lens,
-                            const int32_t* shared_blocks, int num_groups,
-                            const int32_t* group_offsets, const int32_t* group_members,
-                            int max_group_size, int max_shared_blocks, int B, int Hq, int Hkv,
-                            int D, int block_size, int num_blocks, float scale,
-                            int max_context_len, int partition_size, void* workspace,
-                            size_t workspace_bytes, uint32_t* err_flag, void* stream) {
-  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+}  // extern "C"
+
+namespace {
+
+// Shared body of pa_decode_shared_prefix and pa_decode_shared_prefix_kv.
+int shared_prefix_impl(void* out, int out_dtype, const void* query, int q_dtype,
+                       const void* key_cache, int k_dtype, float k_scale, const void* value_cache,
+                       int v_dtype, float v_scale, const int32_t* block_tables,
+                       int max_blocks_per_seq, const int32_t* context_lens,
+                       const int32_t* shared_blocks, int num_groups, const int32_t* group_offsets,
+                       const int32_t* group_members, int max_group_size, int max_shared_blocks,
+                       int B, int Hq, int Hkv, int D, int block_size, int num_blocks, float scale,
+                       int max_context_len, int partition_size, void* workspace,
+                       size_t workspace_bytes, uint32_t* err_flag, void* stream) {
+  if (q_dtype < PA_F32 || q_dtype > PA_BF16) return PA_ERR_DTYPE;
+  if (!pool_types_ok(q_dtype, k_dtype, v_dtype)) return PA_ERR_DTYPE;
+  const bool k8 = k_dtype == PA_FP8_E4M3, v8 = v_dtype == PA_FP8_E4M3;
   if (num_groups < 0 || max_group_size < 0 || max_shared_blocks < 0) return PA_ERR_SHAPE;
   if (max_shared_blocks > max_blocks_per_seq) return PA_ERR_SHAPE;
   const bool share = max_shared_blocks > 0 && num_groups > 0 && B > 0 &&
-                     prefix_tc_supported(dtype, Hq, Hkv, D, block_size);
+                     prefix_tc_supported(q_dtype, Hq, Hkv, D, block_size);
   if (!share)   // nothing shared, or a shape the prefix kernel does not take: plain decode
-    return decode_impl(out, out_dtype, query, dtype, key_cache, dtype, 1.f, value_cache, dtype, 1.f,
-                       block_tables, max_blocks_per_seq, context_lens, B, Hq, Hkv, D, block_size,
-                       num_blocks, scale, max_context_len, partition_size, workspace,
-                       workspace_bytes, err_flag, stream);
-  if (out_dtype != PA_F32 && out_dtype != dtype) return PA_ERR_DTYPE;
+    return decode_impl(out, out_dtype, query, q_dtype, key_cache, k_dtype, k_scale, value_cache,
+                       v_dtype, v_scale, block_tables, max_blocks_per_seq, context_lens, B, Hq,
+                       Hkv, D, block_size, num_blocks, scale, max_context_len, partition_size,
+                       workspace, workspace_bytes, err_flag, stream);
+  if (out_dtype != PA_F32 && out_dtype != q_dtype) return PA_ERR_DTYPE;
   if (Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || num_blocks < 0 ||
       max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0 || max_group_size < 1)
     return PA_ERR_SHAPE;
   if (!supported_shape(Hq, Hkv, D, block_size)) return PA_ERR_UNSUPPORTED;
   if (partition_size > 0 && partition_size % block_size) return PA_ERR_SHAPE;
   if (!std::isfinite(scale)) return PA_ERR_SHAPE;
+  if ((k8 && !scale_ok(k_scale)) || (v8 && !scale_ok(v_scale))) return PA_ERR_SHAPE;
   if (B > 65535 || Hkv > 65535) return PA_ERR_UNSUPPORTED;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
       !shared_blocks || !group_offsets || !group_members)
@@ -390,7 +398,11 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache))
     return PA_ERR_ALIGN;
 
-  DecodePlan p = plan_decode(dtype, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
+  // the suffix pass runs on the kernel pa_decode_kv would take
+  DecodePlan p = plan_decode(k8 || v8 ? PA_FP8_E4M3 : q_dtype, B, Hq, Hkv, D, block_size,
+                             max_context_len, partition_size);
+  if (p.kernel == 2 && k8 != v8)
+    p = plan_decode(PA_F32, B, Hq, Hkv, D, block_size, max_context_len, partition_size);
   // Prefix partitions: as many as keep every (group, member chunk, KV head)
   // unit of all of them in one wave over the SMs, at least one tile each.
   const int tiles = max_prefix_slots(max_shared_blocks, block_size);
@@ -405,8 +417,8 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
   a.block_tables = block_tables; a.max_blocks = max_blocks_per_seq;
   a.context_lens = context_lens;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.bs = block_size; a.num_blocks = num_blocks;
-  a.scale_log2 = scale * kLog2e;
-  a.v_scale = 1.f;
+  a.scale_log2 = scale * kLog2e * (k8 ? k_scale : 1.f);
+  a.v_scale = v8 ? v_scale : 1.f;
   a.max_context_len = max_context_len;
   a.P = tiles + p.P; a.psize = p.psize;    // slot stride as sized by the workspace query
   a.err_flag = err_flag;
@@ -430,12 +442,58 @@ int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const v
     a.test_withhold_q = tc_test_withhold_q();
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int rc = p.kernel == 2 ? launch_decode_tc(a, dtype, false, st) : launch_decode_simt(a, dtype, st);
+  int rc;
+  if (p.kernel == 2) rc = launch_decode_tc(a, q_dtype, k8, st);
+  else if (k8 || v8) rc = launch_decode_simt_kv(a, q_dtype, k_dtype, v_dtype, st);
+  else rc = launch_decode_simt(a, q_dtype, st);
   if (rc == PA_OK)
-    rc = launch_prefix_tc(a, dtype, group_offsets, group_members, num_groups, max_group_size,
-                          parts, part_tokens, st);
+    rc = launch_prefix_tc(a, q_dtype, group_offsets, group_members, num_groups, max_group_size,
+                          parts, part_tokens, st, k8, v8);
   if (rc == PA_OK) rc = launch_merge(a, st);
   return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode_shared_prefix(void* out, int out_dtype, const void* query, const void* key_cache,
+                            const void* value_cache, int dtype, const int32_t* block_tables,
+                            int max_blocks_per_seq, const int32_t* context_lens,
+                            const int32_t* shared_blocks, int num_groups,
+                            const int32_t* group_offsets, const int32_t* group_members,
+                            int max_group_size, int max_shared_blocks, int B, int Hq, int Hkv,
+                            int D, int block_size, int num_blocks, float scale,
+                            int max_context_len, int partition_size, void* workspace,
+                            size_t workspace_bytes, uint32_t* err_flag, void* stream) {
+  if (dtype < PA_F32 || dtype > PA_BF16) return PA_ERR_DTYPE;
+  return shared_prefix_impl(out, out_dtype, query, dtype, key_cache, dtype, 1.f, value_cache,
+                            dtype, 1.f, block_tables, max_blocks_per_seq, context_lens,
+                            shared_blocks, num_groups, group_offsets, group_members,
+                            max_group_size, max_shared_blocks, B, Hq, Hkv, D, block_size,
+                            num_blocks, scale, max_context_len, partition_size, workspace,
+                            workspace_bytes, err_flag, stream);
+}
+
+int pa_decode_shared_prefix_kv(void* out, int out_dtype, const void* query, int q_dtype,
+                               const void* key_cache, int k_dtype, float k_scale,
+                               const void* value_cache, int v_dtype, float v_scale,
+                               const int32_t* block_tables, int max_blocks_per_seq,
+                               const int32_t* context_lens, const int32_t* shared_blocks,
+                               int num_groups, const int32_t* group_offsets,
+                               const int32_t* group_members, int max_group_size,
+                               int max_shared_blocks, int B, int Hq, int Hkv, int D,
+                               int block_size, int num_blocks, float scale, int max_context_len,
+                               int partition_size, void* workspace, size_t workspace_bytes,
+                               uint32_t* err_flag, void* stream) {
+  if (k_dtype < PA_F32 || k_dtype > PA_FP8_E4M3 || v_dtype < PA_F32 || v_dtype > PA_FP8_E4M3)
+    return PA_ERR_DTYPE;
+  return shared_prefix_impl(out, out_dtype, query, q_dtype, key_cache, k_dtype, k_scale,
+                            value_cache, v_dtype, v_scale, block_tables, max_blocks_per_seq,
+                            context_lens, shared_blocks, num_groups, group_offsets,
+                            group_members, max_group_size, max_shared_blocks, B, Hq, Hkv, D,
+                            block_size, num_blocks, scale, max_context_len, partition_size,
+                            workspace, workspace_bytes, err_flag, stream);
 }
 
 }  // extern "C"

@@ -70,6 +70,9 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_kv.restype = I
     lib.pa_reshape_and_cache_kv.argtypes = [P, P, I, P, I, F, P, I, F, P, I, I, I, I, I, P, P]
     lib.pa_reshape_and_cache_kv.restype = I
+    lib.pa_decode_shared_prefix_kv.argtypes = [P, I, P, I, P, I, F, P, I, F, P, I, P, P, I, P, P,
+                                               I, I, I, I, I, I, I, I, F, I, I, P, S, P, P]
+    lib.pa_decode_shared_prefix_kv.restype = I
     lib.pa_prefill_kv.argtypes = [P, I, P, I, P, I, F, P, I, F, P, I, P, P, I, I, I, I, I, I, I, I,
                                   F, I, P, P]
     lib.pa_prefill_kv.restype = I
@@ -365,6 +368,32 @@ def pa_decode_shared_prefix(out: torch.Tensor, query: torch.Tensor, key_cache: t
             _ptr(err_flag), _stream(stream))
     if rc:
         raise PAError("pa_decode_shared_prefix", rc)
+
+
+def pa_decode_shared_prefix_kv(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,
+                               value_cache: torch.Tensor, k_scale: float, v_scale: float,
+                               block_tables: torch.Tensor, context_lens: torch.Tensor,
+                               shared_blocks: torch.Tensor, group_offsets: torch.Tensor,
+                               group_members: torch.Tensor, max_group_size: int,
+                               max_shared_blocks: int, scale: float, max_context_len: int,
+                               partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                               err_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """pa_decode_shared_prefix over pools of per-pool types (uint8 = FP8 E4M3 codes
+    read times the pool's scale; see pa_decode_shared_prefix_kv in include/pa.h)."""
+    B, Hq, D = query.shape
+    num_blocks, block_size, Hkv, _ = key_cache.shape
+    with _on_device_of(query):
+        rc = LIB.pa_decode_shared_prefix_kv(
+            _ptr(out), pa_dtype(out), _ptr(query), pa_dtype(query), _ptr(key_cache),
+            pa_dtype(key_cache), float(k_scale), _ptr(value_cache), pa_dtype(value_cache),
+            float(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+            _ptr(shared_blocks), group_offsets.shape[0] - 1, _ptr(group_offsets),
+            _ptr(group_members), int(max_group_size), int(max_shared_blocks), B, Hq, Hkv, D,
+            block_size, num_blocks, float(scale), int(max_context_len), int(partition_size),
+            _ptr(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+            _ptr(err_flag), _stream(stream))
+    if rc:
+        raise PAError("pa_decode_shared_prefix_kv", rc)
 
 
 def pa_prefill(out: torch.Tensor, query: torch.Tensor, key_cache: torch.Tensor,

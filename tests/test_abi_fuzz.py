@@ -49,6 +49,9 @@ BASE = {
                      16, 256, 0.088, 1024, 0, A[6], 1 << 30, A[7], None],
     "pa_reshape_and_cache_kv": [A[0], A[1], 2, A[2], 3, 0.3, A[3], 2, 1.0, A[4], 4, 8, 128, 16,
                                 256, A[7], None],
+    "pa_decode_shared_prefix_kv": [A[0], 2, A[1], 2, A[2], 3, 0.3, A[3], 3, 0.7, A[4], 64, A[5],
+                                   A[8], 2, A[9], A[10], 16, 8, 32, 32, 8, 128, 16, 1024, 0.088,
+                                   1024, 0, A[6], 1 << 30, A[7], None],
     "pa_prefill_kv": [A[0], 2, A[1], 2, A[2], 3, 0.3, A[3], 3, 0.7, A[4], 64, A[5], A[8], 2, 64, 32,
                       64, 8, 128, 16, 1024, 0.088, 1024, A[7], None],
     "pa_prefill": [A[0], 2, A[1], A[2], A[3], 2, A[4], 64, A[5], A[8], 2, 64, 32, 64, 8, 128, 16,

@@ -152,3 +152,45 @@ def test_full_size_sampling_workload_sampled_parity():
     got = out[torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()]
     assert_attention_close(got, ref, w.dtype, w.name)
     assert torch.isfinite(out.float()).all()
+
+
+def _codes_like(pool, dtype, rng):
+    """An FP8 code pool with the same filled rows as a 16-bit pool."""
+    filled = ~np.isnan(W.storage_to_float64(pool, dtype)).any(axis=-1)
+    codes = np.full(pool.shape, 0x7F, dtype=np.uint8)
+    codes[filled] = W.random_e4m3_codes(rng, (int(filled.sum()), pool.shape[-1]))
+    return codes
+
+
+@pytest.mark.parametrize("k8,v8", [(True, True), (True, False), (False, True)])
+def test_shared_prefix_over_fp8_and_mixed_pools(k8, v8):
+    """Parallel sampling over an FP8 cache (and the mixed one): the pools after
+    the step's cache ops, with codes in the FP8 pools, decoded with the shared
+    prefix read once per group; the oracle decodes the same pools plainly."""
+    rng = np.random.default_rng(70 + 2 * k8 + v8)
+    w = W.shrink_workload(5, seed=517)
+    offsets, members, shared, c, pb = _groups_of(w)
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    oracle.copy_blocks(kc, vc, w.block_mapping, w.dtype)
+    oracle.reshape_and_cache(kc, vc, w.new_key, w.new_value, w.slot_mapping, w.dtype)
+    kp = _codes_like(kc, w.dtype, rng) if k8 else kc
+    vp = _codes_like(vc, w.dtype, rng) if v8 else vc
+    ks, vs = float(np.float32(0.4)), float(np.float32(0.9))
+    t = device_inputs(w)
+    el = lambda a, fp8: (torch.from_numpy(a).cuda() if fp8
+                         else torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda())
+    tk, tv = el(kp, k8), el(vp, v8)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    ws = ops.shared_prefix_workspace_for(t["q"], tk, w.max_context_len, pb)
+    ref = oracle.decode_mixed(w.q, w.dtype, kp, oracle.FP8 if k8 else w.dtype, ks, vp,
+                              oracle.FP8 if v8 else w.dtype, vs, w.block_tables, w.context_lens,
+                              w.scale)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        out = torch.full((w.B, w.Hq, w.D), float("nan"), dtype=out_dtype, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ops.pa_decode_shared_prefix_kv(out, t["q"], tk, tv, ks, vs, t["block_tables"],
+                                       t["context_lens"], dev(shared), dev(offsets), dev(members),
+                                       c, pb, w.scale, w.max_context_len, 0, ws, err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert_attention_close(out, ref, w.dtype, f"k8={k8} v8={v8} {out_dtype}")
