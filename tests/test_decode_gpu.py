@@ -319,3 +319,36 @@ def test_pipeline_wait_limit_runs_out_and_the_next_launch_is_correct(monkeypatch
     out = _decode_with(w, t, ws)
     ref, _, _ = oracle_step(w)
     assert_attention_close(out, ref, w.dtype, "after a timed-out launch")
+
+
+def test_tensor_core_decode_replays_from_a_cuda_graph():
+    """A captured call keeps its epoch; every replay must still merge its pieces
+    (the merger leaves its ticket at zero for that epoch). Three replays of a
+    graph holding the step's scatter and decode, each checked against the oracle."""
+    w = _tc_case([5000, 37, 1, 800, 4096, 33, 64, 3000], seed=91)
+    t = device_inputs(w)
+    ws = ops.workspace_for(t["q"], t["k_cache"], w.max_context_len)
+    out = torch.zeros((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):                      # warm-up outside capture
+        ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                 t["slot_mapping"], err)
+        ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                      t["context_lens"], w.scale, w.max_context_len, 0, ws, err)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
+                                 t["slot_mapping"], err)
+        ops.pa_decode(out, t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                      t["context_lens"], w.scale, w.max_context_len, 0, ws, err)
+    ref, _, _ = oracle_step(w)
+    for rep in range(3):
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert_attention_close(out, ref, w.dtype, f"replay {rep}")
