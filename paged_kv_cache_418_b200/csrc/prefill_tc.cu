@@ -19,11 +19,15 @@
 // where the weights P (in tensor memory, written over S) enter as two 16-bit
 // parts, p = hi + lo, hi = RN(p), lo = RN(p - hi) (~16 significant bits, as
 // in the decode kernels), and the A operand of the output products is read
-// from tensor memory.
+// from tensor memory: each 32-key chunk of S becomes 16 columns of hi parts
+// followed by 16 columns of lo parts (two keys per 32-bit column).
 //
-// A softmax thread owns one query row: it reads its row of S (128 scores)
-// into registers, so the row maximum and the row sum need no exchange with
-// other threads. The reference maximum of a row is its first tile's maximum
+// A softmax thread owns one query row, so the row maximum and the row sum
+// need no exchange with other threads. It reads its row of S twice, 32
+// columns at a time: once for the tile's maximum, once for the weights, which
+// it writes over the chunk it has just read. (Holding all 128 scores in
+// registers instead made the loop body four times longer and the softmax
+// warps stall on instruction fetch.) The reference maximum of a row is its first tile's maximum
 // and moves only when a later tile exceeds it by 2^64 (then the row's O is
 // rescaled in tensor memory, which its own thread does); references are
 // floored at -FLT_MAX so masked scores (-inf) give weight 0 without a guard.
@@ -157,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   constexpr int NB_T = kTile / BS;               // physical blocks per tile
+  constexpr uint32_t kBlkBits = (uint32_t)((1ull << BS) - 1ull);   // one block's keys in a chunk mask
   constexpr uint32_t IDESC_S = make_idesc(FMT, 0, 0, kTile, kM);
   constexpr uint32_t IDESC_O = make_idesc(FMT, 0, 1, kD, kM);
   extern __shared__ uint8_t smem_raw[];
@@ -300,7 +305,8 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; ++kk) {
             const uint64_t bd = sw128_desc(vst + kk * 16 * 128, kHalf, 1024);
-            mma_f16_ta(tmem_o + ob * kD, tmem_s + pb * kTile + part * 64 + kk * 8, bd, IDESC_O,
+            mma_f16_ta(tmem_o + ob * kD,
+                       tmem_s + pb * kTile + (kk >> 1) * 32 + part * 16 + (kk & 1) * 8, bd, IDESC_O,
                        (first && part == 0 && kk == 0) ? 0u : 1u);
           }
         }
@@ -392,23 +398,48 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         const bool zero_v = ts + r >= x.t1 || ((badblk >> (r / BS)) & 1u);
         if (!mbar_wait(bar(B_SFULL + sb), (tc_ >> 1) & 1, abort_flag)) failed = true;
         tc_fence_after();
-        uint32_t raw[kTile];
+        const uint32_t srow = tmem_s + lane_off + sb * kTile;
+        // scores in the log2 domain, masked: keys past the row's position and
+        // keys of blocks with a bad id get -inf. The visibility of a 32-key
+        // chunk is one bit per key, computed without branches; a chunk every
+        // row of the warp sees whole takes the loop without the mask (most
+        // chunks), so no per-key branch or select is left in the hot loops.
+        auto chunk_mask = [&](int c) -> uint32_t {
+          const int n = min(max(pos - (ts + c) + 1, 0), 32);      // keys up to the position
+          uint32_t msk = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
 #pragma unroll
-        for (int c = 0; c < kTile; c += 32) tmem_ld32(tmem_s + lane_off + sb * kTile + c, raw + c);
-        tmem_wait_ld();
-        float* sv = reinterpret_cast<float*>(raw);
-        // scores in the log2 domain, masked; the tile's row maximum
-        const bool full = row_ok && ts + kTile - 1 <= x.pos0 && badblk == 0;  // every key seen
+          for (int q = 0; q < 32 / BS; ++q)
+            msk &= ((badblk >> (c / BS + q)) & 1u) ? ~(kBlkBits << (q * BS)) : 0xffffffffu;
+          return row_ok ? msk : 0u;
+        };
+        const float sl2 = a.scale_log2;
+        // pass 1: the tile's row maximum, 32 columns of S at a time
         float tm = -CUDART_INF_F;
+#pragma unroll 1
+        for (int c = 0; c < kTile; c += 32) {
+          uint32_t raw[32];
+          tmem_ld32(srow + c, raw);
+          tmem_wait_ld();
+          const uint32_t vm = chunk_mask(c);
+          float t0 = -CUDART_INF_F, t1 = -CUDART_INF_F, t2 = -CUDART_INF_F, t3 = -CUDART_INF_F;
+          if (__all_sync(0xffffffffu, vm == 0xffffffffu)) {
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) {
-          float v = sv[j] * a.scale_log2;
-          if (!full) {
-            const bool vis = row_ok && ts + j <= pos && !((badblk >> (j / BS)) & 1u);
-            v = vis ? v : -CUDART_INF_F;
+            for (int j = 0; j < 32; j += 4) {
+              t0 = fmaxf(t0, __uint_as_float(raw[j]) * sl2);
+              t1 = fmaxf(t1, __uint_as_float(raw[j + 1]) * sl2);
+              t2 = fmaxf(t2, __uint_as_float(raw[j + 2]) * sl2);
+              t3 = fmaxf(t3, __uint_as_float(raw[j + 3]) * sl2);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              t0 = fmaxf(t0, ((vm >> j) & 1u) ? __uint_as_float(raw[j]) * sl2 : -CUDART_INF_F);
+              t1 = fmaxf(t1, ((vm >> (j + 1)) & 1u) ? __uint_as_float(raw[j + 1]) * sl2 : -CUDART_INF_F);
+              t2 = fmaxf(t2, ((vm >> (j + 2)) & 1u) ? __uint_as_float(raw[j + 2]) * sl2 : -CUDART_INF_F);
+              t3 = fmaxf(t3, ((vm >> (j + 3)) & 1u) ? __uint_as_float(raw[j + 3]) * sl2 : -CUDART_INF_F);
+            }
           }
-          sv[j] = v;
-          tm = fmaxf(tm, v);
+          tm = fmaxf(tm, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));
         }
         float alpha = 1.f;
         bool resc = false;
@@ -436,18 +467,40 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           tmem_wait_st();
           l *= alpha;
         }
-        // weights, the row sum, and P = hi + lo over this tile's S columns
+        // pass 2: weights and the row sum; each 32-column chunk of S is read
+        // again and overwritten by its weights' 16-bit parts, hi in the chunk's
+        // first 16 columns and lo in the next 16 (two keys per column)
+#pragma unroll 1
+        for (int c = 0; c < kTile; c += 32) {
+          uint32_t raw[32];
+          tmem_ld32(srow + c, raw);
+          tmem_wait_ld();
+          const uint32_t vm = chunk_mask(c);
+          uint32_t pk[32];
+          float l0 = 0.f, l1 = 0.f;
+          if (__all_sync(0xffffffffu, vm == 0xffffffffu)) {
 #pragma unroll
-        for (int c = 0; c < kTile; c += 64) {
-          uint32_t hi[32], lo[32];
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = ex2(__uint_as_float(raw[2 * e]) * sl2 - m);
+              const float p1 = ex2(__uint_as_float(raw[2 * e + 1]) * sl2 - m);
+              l0 += p0;
+              l1 += p1;
+              split2<FMT>(p0, p1, pk[e], pk[16 + e]);
+            }
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float p0 = ex2(sv[c + 2 * e] - m), p1 = ex2(sv[c + 2 * e + 1] - m);
-            l += p0 + p1;
-            split2<FMT>(p0, p1, hi[e], lo[e]);
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = __uint_as_float(raw[2 * e]) * sl2 - m;
+              const float x1 = __uint_as_float(raw[2 * e + 1]) * sl2 - m;
+              const float p0 = ex2(((vm >> (2 * e)) & 1u) ? x0 : -CUDART_INF_F);
+              const float p1 = ex2(((vm >> (2 * e + 1)) & 1u) ? x1 : -CUDART_INF_F);
+              l0 += p0;
+              l1 += p1;
+              split2<FMT>(p0, p1, pk[e], pk[16 + e]);
+            }
           }
-          tmem_st32(tmem_s + lane_off + sb * kTile + c / 2, hi);
-          tmem_st32(tmem_s + lane_off + sb * kTile + 64 + c / 2, lo);
+          l += l0 + l1;
+          tmem_st32(srow + c, pk);
         }
         if (!V8 && zero_v) {
           // this V row enters the output product with weight 0: it must hold finite values
