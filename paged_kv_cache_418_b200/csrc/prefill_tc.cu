@@ -234,14 +234,26 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
                       bar(B_QFULL + qi));
         q_last[qi] = ui;
         const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
+        // block-table entries of tile k, read one tile ahead so that their
+        // latency overlaps the current tile's copies
+        auto fetch = [&](int k, int (&ph)[NB_T]) {
+          const int ts = k * kTile;
+          const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+#pragma unroll
+          for (int q = 0; q < NB_T; ++q) ph[q] = q < nblk ? __ldg(table + ts / BS + q) : -1;
+        };
+        int ahead[NB_T];
+        fetch(0, ahead);
         for (int k = 0; k < x.ntiles; ++k, ++tc_) {
           const int ts = k * kTile;
           const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
           int phys[NB_T];
+#pragma unroll
+          for (int q = 0; q < NB_T; ++q) phys[q] = ahead[q];
+          if (k + 1 < x.ntiles) fetch(k + 1, ahead);
           uint32_t bytes = 0;
 #pragma unroll
           for (int q = 0; q < NB_T; ++q) {
-            phys[q] = q < nblk ? __ldg(table + ts / BS + q) : -1;
             if (q < nblk && (phys[q] < 0 || phys[q] >= a.num_blocks)) {
               flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
               phys[q] = -1;
