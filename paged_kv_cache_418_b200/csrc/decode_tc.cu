@@ -69,6 +69,8 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <cfloat>
+
 #include "pa_internal.h"
 #include "tc_ptx.cuh"
 
@@ -105,13 +107,14 @@ template <int G> struct TcShape {
   static constexpr int OFF_STG = OFF_P + 2 * kPBytes;        // [2 groups] output staging
   static constexpr int OFF_X = OFF_STG + 2 * kStgBytes;      // [2][2][NS] reference max, exp-sum
   static constexpr int OFF_BAR = OFF_X + 2 * 2 * NS * 4 + 16;
-  static constexpr int NBAR = 3 * kStages + 20;
+  static constexpr int NBAR = 3 * kStages + 24;
   static constexpr int GP = G < 8 ? 8 : G;                  // per-chunk stride of the reductions
   static constexpr int OFF_RED = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;  // [group][2][8][GP] maxima
   static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
   static constexpr int OFF_MREF = OFF_REDL + 2 * 2 * 8 * GP * 4;  // [group][3][NS] references
   static constexpr int OFF_COEF = OFF_MREF + 2 * 3 * NS * 4;   // [group][2][NS] merge weights
-  static constexpr int OFF_MISC = (OFF_COEF + 2 * 2 * NS * 4 + 15) / 16 * 16;
+  static constexpr int OFF_QSC = OFF_COEF + 2 * 2 * NS * 4;      // [2 query buffers][NS] score scales
+  static constexpr int OFF_MISC = (OFF_QSC + 2 * NS * 4 + 15) / 16 * 16;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -125,7 +128,8 @@ template <int NST> struct Bars {
   static constexpr int FULL = 0, EMPTY = NST, QFULL = 2 * NST, QEMPTY = QFULL + 2,
                        SFULL = QEMPTY + 2, SFREE = SFULL + 2, PREADY = SFREE + 2,
                        OFULL = PREADY + 2, XFULL = OFULL + 2, XFREE = XFULL + 2,
-                       ODONE = XFREE + 2, DONE = ODONE + 2, CONV = DONE + 1;
+                       ODONE = XFREE + 2, DONE = ODONE + 2, CONV = DONE + 1,
+                       QCONV = CONV + NST, QSREAD = QCONV + 2;
 };
 
 // Shared words written by the prologue (OFF_MISC).
@@ -425,8 +429,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   constexpr int NQ = kRt / RB;                   // boxes per d-half per tile
   constexpr int KS = kRt / 16;                   // output-MMA K steps per head per tile
   constexpr int NCH = NQ * kHG;                  // (box, head) row chunks per tile
-  constexpr uint32_t IDESC_S = make_idesc(FMT, 0, 0, NS, 128);
-  constexpr uint32_t IDESC_O = make_idesc(FMT, 1, 0, NOH, 128);
+  // FP8 pools run on f16 operands whatever the query type: E4M3 -> f16 is one
+  // conversion per pair of codes (bf16 would take several), and a bf16 query
+  // is brought to f16 in shared memory with an exact power-of-two scale per
+  // query head (QCNV), which the scores take back.
+  constexpr int CF = KV8 ? 0 : FMT;             // element type of the MMA operands
+  constexpr bool QCNV = KV8 && FMT == 1;
+  constexpr uint32_t IDESC_S = make_idesc(CF, 0, 0, NS, 128);
+  constexpr uint32_t IDESC_O = make_idesc(CF, 1, 0, NOH, 128);
   static_assert(NCH * RB == kRows && NCH <= 8, "tile geometry");
 
   extern __shared__ uint8_t smem_raw[];
@@ -462,6 +472,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     mbar_init(bar(Bx::ODONE + 1), 128);
     mbar_init(bar(Bx::DONE), 1);
     for (int s = 0; s < NST; ++s) mbar_init(bar(Bx::CONV + s), 128);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Bx::QCONV + i), 128);
+      mbar_init(bar(Bx::QSREAD + i), 256);
+    }
     ms->abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -633,6 +647,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         const Unit x = unit_of(cur);
         const int qi = i & 1;
         if (!mbar_wait(bar(Bx::QFULL + qi), (i >> 1) & 1, abort_flag, wait_ns)) { ok = false; break; }
+        if (QCNV && !mbar_wait(bar(Bx::QCONV + qi), (i >> 1) & 1, abort_flag, wait_ns)) { ok = false; break; }
         const uint32_t qst = sbase + S::OFF_Q + qi * S::kQBytes;
         for (int k = 0; k < x.ntiles; ++k) {
           int ts, te, nql;
@@ -733,6 +748,67 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
       for (int g = 0; g < G; ++g) { mo[g] = -CUDART_INF_F; l[g] = 0.f; }
       int my_last = -1;
+      float qcs[G];                                // score scale of each query head of this row's head
+      if constexpr (QCNV) {
+        // the group that takes the unit's first tile brings its bf16 query to f16:
+        // query head n is scaled by 2^-e_n (its largest |q| lands in [2^14, 2^15)),
+        // exactly for every element the f16 grid holds, and its score scale by 2^e_n
+        const int qi = i & 1;
+        float* qsc = reinterpret_cast<float*>(smem + S::OFF_QSC) + qi * NS;
+        if ((tc & 1) == grp) {
+          if (!mbar_wait(bar(Bx::QFULL + qi), (i >> 1) & 1, abort_flag, wait_ns)) failed = true;
+          // the scales of unit i - 2 (same buffer) have been read by both groups
+          if (i >= 2 && !mbar_wait(bar(Bx::QSREAD + qi), ((i - 2) >> 1) & 1, abort_flag, wait_ns))
+            failed = true;
+          if (!failed) {
+            constexpr int TPQ = 128 / NS, CPT = 16 / TPQ;     // threads per query head, chunks each
+            const int n = row / TPQ, part = row % TPQ;
+            uint8_t* qb = smem + S::OFF_Q + qi * S::kQBytes;
+            uint4 v[CPT];
+            float mx = 0.f;
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+              const int ch = part * CPT + j, hh = ch >> 3, c = ch & 7;
+              v[j] = *reinterpret_cast<const uint4*>(qb + hh * (NS * 128) + n * 128 + ((c ^ (n & 7)) << 4));
+              const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                mx = fmaxf(mx, fabsf(__uint_as_float(w[e] << 16)));
+                mx = fmaxf(mx, fabsf(__uint_as_float(w[e] & 0xffff0000u)));
+              }
+            }
+#pragma unroll
+            for (int o = TPQ / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            int e2 = 0;
+            if (mx > 0.f && mx <= FLT_MAX) e2 = min(max((int)((__float_as_uint(mx) >> 23) & 0xff) - 127 - 14, -100), 100);
+            const float down = __uint_as_float((uint32_t)(127 - e2) << 23);   // 2^-e2
+#pragma unroll
+            for (int j = 0; j < CPT; ++j) {
+              const int ch = part * CPT + j, hh = ch >> 3, c = ch & 7;
+              const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+              uint32_t h[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const __half2 f = __floats2half2_rn(__uint_as_float(w[e] << 16) * down,
+                                                    __uint_as_float(w[e] & 0xffff0000u) * down);
+                h[e] = *reinterpret_cast<const uint32_t*>(&f);
+              }
+              *reinterpret_cast<uint4*>(qb + hh * (NS * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
+                  make_uint4(h[0], h[1], h[2], h[3]);
+            }
+            if (part == 0) qsc[n] = a.scale_log2 * __uint_as_float((uint32_t)(127 + e2) << 23);
+          }
+          fence_proxy_async();                     // the converted query -> the tensor cores
+          mbar_arrive(bar(Bx::QCONV + qi));
+        }
+        if (!mbar_wait(bar(Bx::QCONV + qi), (i >> 1) & 1, abort_flag, wait_ns)) failed = true;
+#pragma unroll
+        for (int g = 0; g < G; ++g) qcs[g] = qsc[rh * G + g];
+        mbar_arrive(bar(Bx::QSREAD + qi));
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) qcs[g] = a.scale_log2;
+      }
       for (int k = 0; k < x.ntiles; ++k, ++tc) {
         if ((tc & 1) != grp) continue;
         int ts, te, nql;
@@ -753,7 +829,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             const int seq = 2 * tc + kv, s = seq % NST;
             if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
             if (in_range && !failed)
-              widen_row_fp8<FMT>(smem + s * kStageBytes, row, kv == 1 && !valid);
+              widen_row_fp8<CF>(smem + s * kStageBytes, row, kv == 1 && !valid);
             fence_proxy_async();
             mbar_arrive(bar(Bx::CONV + s));
           }
@@ -775,7 +851,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float raw = (RB < 32 && second) ? sv[(RB < 32 ? G : 0) + g] : sv[g];
-          s[g] = valid ? raw * a.scale_log2 : -CUDART_INF_F;
+          s[g] = valid ? raw * (QCNV ? qcs[g] : a.scale_log2) : -CUDART_INF_F;
           float v = s[g];
 #pragma unroll
           for (int o = RB / 2; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -839,7 +915,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           const float p = valid ? exp2f(s[g] - mo[g]) : 0.f;
           l[g] = fmaf(l[g], ao[g], p);
           uint16_t hi, lo;
-          split_16<FMT>(p, hi, lo);
+          split_16<CF>(p, hi, lo);
           *reinterpret_cast<uint16_t*>(prow + g * 128 + ((pchunk ^ (g & 7)) << 4) + pbyte) = hi;
           *reinterpret_cast<uint16_t*>(prow + (G + g) * 128 + ((pchunk ^ ((G + g) & 7)) << 4) + pbyte) = lo;
         }
