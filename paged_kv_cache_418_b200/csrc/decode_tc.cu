@@ -93,21 +93,29 @@ constexpr float kRescaleLog2 = 64.f;            // lazy rescale threshold (log2 
 constexpr int kEpochShift = 24;                 // ticket word: epoch << 24 | pieces arrived
 constexpr unsigned long long kCountMask = (1ull << kEpochShift) - 1;
 
-template <int G> struct TcShape {
+// 16-bit pools: a ring of 32 KB stages, each the K or V operand of one tile.
+// FP8 pools (KV8): a ring of 16 KB stages of codes (K or V of one tile, one
+// 128-byte line per row) and, per softmax group, a 32 KB buffer that holds the
+// V operand of the group's current tile widened to f16; the query buffer holds
+// the 16-bit query as loaded, then its E4M3 pieces.
+template <int G, bool KV8 = false> struct TcShape {
   static constexpr int NS = kHG * G;                         // N of the score MMA
   static constexpr int NOH = ((2 * G + 15) / 16) * 16;       // N of a head's output MMA
   static constexpr int NO = kHG * NOH;                       // output columns per group
   static constexpr int kStages = 5;
+  static constexpr int kStage = KV8 ? kHalf : kStageBytes;   // bytes per ring stage
   static constexpr int kTmemCols = 512;                      // S x2, O x (2 units x 2 groups)
-  static constexpr int kQBytes = 2 * NS * 128;               // Q operand: 2 d-halves x NS rows
+  static constexpr int kNP = 3;                              // E4M3 pieces of the query at most
+  static constexpr int kQBytes = (KV8 ? kNP : 2) * NS * 128; // Q operand: 2 d-halves x NS rows
   static constexpr int kPBytes = 2 * NOH * 128;              // P operand of one tile: 2 lines
   static constexpr int kStgBytes = NS * kD * 4;              // one group's merged rows (fp32)
-  static constexpr int OFF_Q = kStages * kStageBytes;
+  static constexpr int OFF_VOP = kStages * kStage;           // [2 groups] widened V (FP8 pools)
+  static constexpr int OFF_Q = OFF_VOP + (KV8 ? 2 * kStageBytes : 0);
   static constexpr int OFF_P = OFF_Q + 2 * kQBytes;
   static constexpr int OFF_STG = OFF_P + 2 * kPBytes;        // [2 groups] output staging
   static constexpr int OFF_X = OFF_STG + 2 * kStgBytes;      // [2][2][NS] reference max, exp-sum
   static constexpr int OFF_BAR = OFF_X + 2 * 2 * NS * 4 + 16;
-  static constexpr int NBAR = 3 * kStages + 24;
+  static constexpr int NBAR = 2 * kStages + 23;
   static constexpr int GP = G < 8 ? 8 : G;                  // per-chunk stride of the reductions
   static constexpr int OFF_RED = (OFF_BAR + 8 * NBAR + 15) / 16 * 16;  // [group][2][8][GP] maxima
   static constexpr int OFF_REDL = OFF_RED + 2 * 2 * 8 * GP * 4;   // [group][2][8][GP] sums
@@ -118,9 +126,13 @@ template <int G> struct TcShape {
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;                  // + alignment slack
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
-  static_assert(2 * NS + 4 * NO <= kTmemCols, "tensor memory columns");
+  // an S buffer: NS columns, or one block of NS per query piece (FP8 pools)
+  static constexpr int SW = (KV8 ? kNP : 1) * NS;
+  static_assert(2 * SW + 4 * NO <= kTmemCols, "tensor memory columns");
   static_assert(OFF_STG % 128 == 0, "bulk-copy source alignment");
   static_assert(OFF_COEF % 16 == 0, "vector loads of the merge weights");
+  static_assert(OFF_Q % 1024 == 0 && kQBytes % 1024 == 0 && (NS * 128) % 1024 == 0,
+                "128-byte-swizzled operands start on 1024-byte boundaries");
 };
 
 // barrier indices (the ring's full/empty pairs come first)
@@ -128,8 +140,8 @@ template <int NST> struct Bars {
   static constexpr int FULL = 0, EMPTY = NST, QFULL = 2 * NST, QEMPTY = QFULL + 2,
                        SFULL = QEMPTY + 2, SFREE = SFULL + 2, PREADY = SFREE + 2,
                        OFULL = PREADY + 2, XFULL = OFULL + 2, XFREE = XFULL + 2,
-                       ODONE = XFREE + 2, DONE = ODONE + 2, CONV = DONE + 1,
-                       QCONV = CONV + NST, QSREAD = QCONV + 2;
+                       ODONE = XFREE + 2, DONE = ODONE + 2, QCONV = DONE + 1,
+                       QSREAD = QCONV + 2;
 };
 
 // Shared words written by the prologue (OFF_MISC).
@@ -413,15 +425,23 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs& a, const Unit& x,
   }
 }
 
+// Two 16-bit query elements of a 32-bit word (element 0 in the low half) as fp32.
+template <int FMT>
+__device__ __forceinline__ float2 q_pair(uint32_t w) {
+  if (FMT == 1) return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
 // KV8: the pools hold FP8 E4M3 codes (K times k_scale, folded into the score
 // scale; V times v_scale, folded into the output weights). TMA brings a tile's
-// codes (half the bytes); the softmax group that owns the tile widens it in
-// place (widen_row_fp8) and only then releases it to the tensor cores.
+// codes into 16 KB stages; the score product reads the K codes as they are,
+// and the softmax group that owns the tile, once it has written the tile's
+// weights, widens the V codes into the group's V buffer and frees the stage.
 template <int FMT, int BS, int G, bool KV8>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ) {
-  using S = TcShape<G>;
+  using S = TcShape<G, KV8>;
   constexpr int NST = S::kStages;
   using Bx = Bars<NST>;
   constexpr int NS = S::NS, NOH = S::NOH, NO = S::NO;
@@ -429,13 +449,18 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   constexpr int NQ = kRt / RB;                   // boxes per d-half per tile
   constexpr int KS = kRt / 16;                   // output-MMA K steps per head per tile
   constexpr int NCH = NQ * kHG;                  // (box, head) row chunks per tile
-  // FP8 pools run on f16 operands whatever the query type: E4M3 -> f16 is one
-  // conversion per pair of codes (bf16 would take several), and a bf16 query
-  // is brought to f16 in shared memory with an exact power-of-two scale per
-  // query head (QCNV), which the scores take back.
-  constexpr int CF = KV8 ? 0 : FMT;             // element type of the MMA operands
-  constexpr bool QCNV = KV8 && FMT == 1;
-  constexpr uint32_t IDESC_S = make_idesc(CF, 0, 0, NS, 128);
+  // FP8 pools. The score product runs on the K codes themselves
+  // (kind::f8f6f4): the query of each head is scaled by an exact power of two
+  // and split into E4M3 pieces, q = 2^e (q1 + q2 [+ q3]), each the rounding of
+  // what the earlier ones leave; two pieces hold a bf16 value exactly (4 + 4
+  // significant bits), three an f16 value, unless an element lies below the
+  // E4M3 grid (2^-17 of the head's largest element). The scores take 2^e back.
+  // The output product runs on f16 operands whatever the query type: E4M3 ->
+  // f16 is one conversion per pair of codes (bf16 would take several).
+  constexpr int CF = KV8 ? 0 : FMT;             // element type of the output product
+  constexpr bool QCNV = KV8;                    // the query becomes E4M3 pieces
+  constexpr int NPU = FMT == 1 ? 2 : 3;         // pieces the score product uses
+  constexpr uint32_t IDESC_S = make_idesc(CF, 0, 0, KV8 ? NPU * NS : NS, 128);
   constexpr uint32_t IDESC_O = make_idesc(CF, 1, 0, NOH, 128);
   static_assert(NCH * RB == kRows && NCH <= 8, "tile geometry");
 
@@ -471,7 +496,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
     mbar_init(bar(Bx::ODONE), 128);
     mbar_init(bar(Bx::ODONE + 1), 128);
     mbar_init(bar(Bx::DONE), 1);
-    for (int s = 0; s < NST; ++s) mbar_init(bar(Bx::CONV + s), 128);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(Bx::QCONV + i), 128);
       mbar_init(bar(Bx::QSREAD + i), 256);
@@ -498,7 +522,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   const uint32_t tmem_s = tmem;                 // S buffers: [0, NS) and [NS, 2NS)
   // O accumulators from column 2NS: [unit parity][group], NO columns each, so the
   // next unit accumulates while the previous one is merged
-  const uint32_t tmem_o = tmem + 2 * NS;
+  const uint32_t tmem_o = tmem + 2 * S::SW;
   auto obuf = [&](int ui, int g) { return tmem_o + (uint32_t)((2 * (ui & 1) + g) * NO); };
   const long long T = ms->T, r0 = ms->r0;
   const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
@@ -509,7 +533,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   // token range of tile k of a unit, and how many of its boxes hold tokens
   // a stage is ready for the tensor cores when TMA filled it (16-bit pools) or
   // when its owning group widened it (FP8 pools)
-  auto ready_bar = [&](int s) { return bar((KV8 ? Bx::CONV : Bx::FULL) + s); };
+  // K of a tile is ready for the tensor cores when TMA has filled its stage. V
+  // is ready when TMA has filled its stage (16-bit pools), or, with FP8 pools,
+  // when the group that owns the tile has widened its codes into the group's V
+  // buffer, which it does before it hands over the tile's P (PREADY).
+  auto k_ready_bar = [&](int s) { return bar(Bx::FULL + s); };
   auto tile_span = [&](const Unit& x, int k, int& ts, int& te, int& nql) {
     ts = x.t0 + k * kRt;
     te = min(x.t1, ts + kRt);
@@ -567,14 +595,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             const int seq = 2 * tc + kv, s = seq % NST;
             if (!mbar_wait(bar(Bx::EMPTY + s), ((seq / NST) & 1) ^ 1, abort_flag, wait_ns)) { give_up(); goto prod_done; }
             mbar_expect_tx(bar(Bx::FULL + s), bytes);
-            const uint32_t dst = sbase + s * kStageBytes;
+            const uint32_t dst = sbase + s * S::kStage;
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
               if (phys[q] < 0 || phys[q] >= a.num_blocks) continue;
               const int rr0 = (ts + q * RB) % BS;
               if (KV8) {
-                // all 128 codes of a row in one 128-byte line, at the stage's upper half
-                tma_load_4d(dst + kHalf + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, rr0,
+                // all 128 codes of a row in one 128-byte line
+                tma_load_4d(dst + q * (kHG * RB * 128), kv ? &tmV : &tmK, 0, rr0,
                             x.h * kHG, phys[q], bar(Bx::FULL + s));
               } else {
                 for (int hh = 0; hh < 2; ++hh)
@@ -616,9 +644,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             !mbar_wait(bar(Bx::ODONE + (ui & 1)), ((ui - 2) >> 1) & 1, abort_flag, wait_ns))
           return false;
         const int seq = 2 * tt + 1, s = seq % NST;
-        if (!mbar_wait(ready_bar(s), (seq / NST) & 1, abort_flag, wait_ns)) return false;
+        // FP8 pools: the group widened V into its buffer before handing over P
+        if (!KV8 && !mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) return false;
         tc_fence_after();
-        const uint32_t vst = sbase + s * kStageBytes;
+        const uint32_t vst = KV8 ? sbase + S::OFF_VOP + pb * kStageBytes : sbase + s * S::kStage;
         const uint32_t pst = sbase + S::OFF_P + pb * S::kPBytes;
 #pragma unroll
         for (int h = 0; h < kHG; ++h) {
@@ -635,7 +664,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             mma_f16(obuf(ui, pb) + h * NOH, ad, bd, IDESC_O, (first && ks == 0) ? 0u : 1u);
           }
         }
-        mma_commit(bar(Bx::EMPTY + s));
+        if (!KV8) mma_commit(bar(Bx::EMPTY + s));   // FP8: the group freed the code stage
         mma_commit(bar(Bx::OFULL + pb));
         return true;
       };
@@ -666,21 +695,33 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
                 break;
               }
               if (mbar_test(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1) &&
-                  mbar_test(ready_bar(s), (seq / NST) & 1))
+                  mbar_test(k_ready_bar(s), (seq / NST) & 1))
                 break;
               if (*abort_flag || globaltimer() - t0 > wait_ns) { ok = false; break; }
             }
             if (!ok) break;
           }
           if (!mbar_wait(bar(Bx::SFREE + sb), ((tc >> 1) & 1) ^ 1, abort_flag, wait_ns)) { ok = false; break; }
-          if (!mbar_wait(ready_bar(s), (seq / NST) & 1, abort_flag, wait_ns)) { ok = false; break; }
+          if (!mbar_wait(k_ready_bar(s), (seq / NST) & 1, abort_flag, wait_ns)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kst = sbase + s * kStageBytes;
+          const uint32_t kst = sbase + s * S::kStage;
+          if constexpr (QCNV) {
+            // K codes (one 128-byte line per row) times the query pieces, which
+            // stand one after another as NPU * NS rows of B: each piece's scores
+            // land in their own NS columns (4 steps of 32 codes)
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint64_t ad = sw128_desc(kst + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
-            const uint64_t bd = sw128_desc(qst + (ks >> 2) * (NS * 128) + (ks & 3) * 32, 16, 1024);
-            mma_f16(tmem_s + sb * NS, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < kD / 32; ++ks) {
+              const uint64_t ad = sw128_desc(kst + ks * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(qst + ks * 32, 16, 1024);
+              mma_f8(tmem_s + sb * S::SW, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint64_t ad = sw128_desc(kst + (ks >> 2) * kHalf + (ks & 3) * 32, 16, 1024);
+              const uint64_t bd = sw128_desc(qst + (ks >> 2) * (NS * 128) + (ks & 3) * 32, 16, 1024);
+              mma_f16(tmem_s + sb * S::SW, ad, bd, IDESC_S, ks > 0 ? 1u : 0u);
+            }
           }
           mma_commit(bar(Bx::EMPTY + s));
           mma_commit(bar(Bx::SFULL + sb));
@@ -750,9 +791,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
       int my_last = -1;
       float qcs[G];                                // score scale of each query head of this row's head
       if constexpr (QCNV) {
-        // the group that takes the unit's first tile brings its bf16 query to f16:
-        // query head n is scaled by 2^-e_n (its largest |q| lands in [2^14, 2^15)),
-        // exactly for every element the f16 grid holds, and its score scale by 2^e_n
+        // the group that takes the unit's first tile turns its 16-bit query into
+        // E4M3 pieces in place: query head n is scaled by 2^-e_n (its largest |q|
+        // lands in [2^7, 2^8), below the E4M3 maximum 448) and split as
+        // q1 = RN(q), q2 = RN(q - q1), q3 = RN(q - q1 - q2); the head's score
+        // scale takes 2^e_n
         const int qi = i & 1;
         float* qsc = reinterpret_cast<float*>(smem + S::OFF_QSC) + qi * NS;
         if ((tc & 1) == grp) {
@@ -760,45 +803,66 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           // the scales of unit i - 2 (same buffer) have been read by both groups
           if (i >= 2 && !mbar_wait(bar(Bx::QSREAD + qi), ((i - 2) >> 1) & 1, abort_flag, wait_ns))
             failed = true;
-          if (!failed) {
-            constexpr int TPQ = 128 / NS, CPT = 16 / TPQ;     // threads per query head, chunks each
-            const int n = row / TPQ, part = row % TPQ;
-            uint8_t* qb = smem + S::OFF_Q + qi * S::kQBytes;
-            uint4 v[CPT];
-            float mx = 0.f;
+          constexpr int TPQ = 128 / NS, CPT = 16 / TPQ;       // threads per query head, chunks each
+          const int n = row / TPQ, part = row % TPQ;
+          uint8_t* qb = smem + S::OFF_Q + qi * S::kQBytes;
+          // the 16-bit query: [2 d-halves][NS rows][128 B], 128-byte swizzled
+          uint4 v[CPT];
+          float mx = 0.f;
 #pragma unroll
-            for (int j = 0; j < CPT; ++j) {
-              const int ch = part * CPT + j, hh = ch >> 3, c = ch & 7;
-              v[j] = *reinterpret_cast<const uint4*>(qb + hh * (NS * 128) + n * 128 + ((c ^ (n & 7)) << 4));
-              const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+          for (int j = 0; j < CPT; ++j) {
+            const int ch = part * CPT + j, hh = ch >> 3, c = ch & 7;
+            v[j] = *reinterpret_cast<const uint4*>(qb + hh * (NS * 128) + n * 128 + ((c ^ (n & 7)) << 4));
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                mx = fmaxf(mx, fabsf(__uint_as_float(w[e] << 16)));
-                mx = fmaxf(mx, fabsf(__uint_as_float(w[e] & 0xffff0000u)));
-              }
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = q_pair<FMT>(w[e]);
+              mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
             }
+          }
 #pragma unroll
-            for (int o = TPQ / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          for (int o = TPQ / 2; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          // every row has been read before the pieces overwrite the buffer
+          if (!wg_vote_or(failed, grp)) {
             int e2 = 0;
-            if (mx > 0.f && mx <= FLT_MAX) e2 = min(max((int)((__float_as_uint(mx) >> 23) & 0xff) - 127 - 14, -100), 100);
+            if (mx > 0.f && mx <= FLT_MAX)
+              e2 = min(max((int)((__float_as_uint(mx) >> 23) & 0xff) - 127 - 7, -100), 100);
             const float down = __uint_as_float((uint32_t)(127 - e2) << 23);   // 2^-e2
+            // the pieces: [NPU][NS rows][128 codes], 128-byte swizzled (K-major)
 #pragma unroll
             for (int j = 0; j < CPT; ++j) {
               const int ch = part * CPT + j, hh = ch >> 3, c = ch & 7;
+              const int d0 = hh * 64 + c * 8;                   // first of the chunk's 8 elements
               const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-              uint32_t h[4];
+              uint32_t pw[NPU][2];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const __half2 f = __floats2half2_rn(__uint_as_float(w[e] << 16) * down,
-                                                    __uint_as_float(w[e] & 0xffff0000u) * down);
-                h[e] = *reinterpret_cast<const uint32_t*>(&f);
+                const float2 f = q_pair<FMT>(w[e]);
+                float r0 = f.x * down, r1 = f.y * down;        // exact: a power of two
+#pragma unroll
+                for (int pc = 0; pc < NPU; ++pc) {
+                  const __nv_fp8x2_storage_t h =
+                      __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
+                  if ((e & 1) == 0) pw[pc][e >> 1] = 0u;
+                  pw[pc][e >> 1] |= (uint32_t)h << ((e & 1) * 16);
+                  if (pc + 1 < NPU) {                          // what this piece leaves (exact)
+                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(h, __NV_E4M3);
+                    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+                    r0 -= hf.x;
+                    r1 -= hf.y;
+                  }
+                }
               }
-              *reinterpret_cast<uint4*>(qb + hh * (NS * 128) + n * 128 + ((c ^ (n & 7)) << 4)) =
-                  make_uint4(h[0], h[1], h[2], h[3]);
+              const int off = n * 128 + (((d0 >> 4) ^ (n & 7)) << 4) + (d0 & 15);
+#pragma unroll
+              for (int pc = 0; pc < NPU; ++pc)
+                *reinterpret_cast<uint2*>(qb + pc * (NS * 128) + off) = make_uint2(pw[pc][0], pw[pc][1]);
             }
             if (part == 0) qsc[n] = a.scale_log2 * __uint_as_float((uint32_t)(127 + e2) << 23);
+          } else {
+            failed = true;
           }
-          fence_proxy_async();                     // the converted query -> the tensor cores
+          fence_proxy_async();                     // the pieces -> the tensor cores
           mbar_arrive(bar(Bx::QCONV + qi));
         }
         if (!mbar_wait(bar(Bx::QCONV + qi), (i >> 1) & 1, abort_flag, wait_ns)) failed = true;
@@ -822,18 +886,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         const bool valid = in_range && blk_ok && ts + tt_row < te;
         if (in_range && !blk_ok && rr == 0 && rh == 0) flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
         const bool first = my_last < 0;
-        if constexpr (KV8) {
-          // widen this tile's K and V rows (zeros for V rows that must not count)
-#pragma unroll 1
-          for (int kv = 0; kv < 2; ++kv) {
-            const int seq = 2 * tc + kv, s = seq % NST;
-            if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
-            if (in_range && !failed)
-              widen_row_fp8<CF>(smem + s * kStageBytes, row, kv == 1 && !valid);
-            fence_proxy_async();
-            mbar_arrive(bar(Bx::CONV + s));
-          }
-        }
 
         const int par = (tc >> 1) & 1;                        // use count of this group's buffers
         if (!mbar_wait(bar(Bx::SFULL + grp), par, abort_flag, wait_ns)) failed = true;
@@ -841,36 +893,58 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
         constexpr int SVN = ((32 / RB) * G + 15) / 16 * 16;  // S columns this warp loads
         float sv[SVN];
 #pragma unroll
-        for (int c = 0; c < SVN; c += 16) tmem_ld16(tmem_s + lane_off + grp * NS + col0 + c, sv + c);
+        for (int c = 0; c < SVN; c += 16) tmem_ld16(tmem_s + lane_off + grp * S::SW + col0 + c, sv + c);
+        if constexpr (KV8) {
+          // the query pieces' scores: S = S(q1) + S(q2) [+ S(q3)]
+#pragma unroll
+          for (int pc = 1; pc < NPU; ++pc) {
+            float sp[SVN];
+#pragma unroll
+            for (int c = 0; c < SVN; c += 16)
+              tmem_ld16(tmem_s + lane_off + grp * S::SW + pc * NS + col0 + c, sp + c);
+#pragma unroll
+            for (int c = 0; c < SVN; ++c) sv[c] += sp[c];
+          }
+        }
         tc_fence_before();
         mbar_arrive(bar(Bx::SFREE + grp));
 
         float s[G];
         const bool second = rh * G != col0;                   // this row's head is the 2nd loaded
         float* rb = red + par * 8 * S::GP;
+        bool exceed = false;                                  // a score passed its reference
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float raw = (RB < 32 && second) ? sv[(RB < 32 ? G : 0) + g] : sv[g];
           s[g] = valid ? raw * (QCNV ? qcs[g] : a.scale_log2) : -CUDART_INF_F;
-          float v = s[g];
-#pragma unroll
-          for (int o = RB / 2; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-          if (rr == 0) rb[(rq * kHG + rh) * S::GP + g] = v;
+          exceed |= s[g] > mo[g] + kRescaleLog2;
         }
-        if (wg_vote_or(failed, grp)) { stop = true; break; }
-        // this head's tile maxima; lazy update of the references (uniform per group)
+        // The references (uniform per query head over the group): the unit's first
+        // tile sets them to its maxima, a reduction over the group; a later tile
+        // only votes on whether some score passed its reference by 2^64, and
+        // reduces (then rescales) only in that rare case.
+        const bool reduce = wg_vote_or(failed || first || exceed, grp);
+        if (reduce && wg_vote_or(failed, grp)) { stop = true; break; }
         float tm[G], ao[G];
-        bool exceed = false;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          tm[g] = -CUDART_INF_F;
+        for (int g = 0; g < G; ++g) { tm[g] = -CUDART_INF_F; ao[g] = 1.f; }
+        if (reduce) {
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) tm[g] = fmaxf(tm[g], rb[(q * kHG + rh) * S::GP + g]);
-          ao[g] = 1.f;
-          if (first) mo[g] = tm[g];
-          else exceed |= tm[g] > mo[g] + kRescaleLog2;
+          for (int g = 0; g < G; ++g) {
+            float v = s[g];
+#pragma unroll
+            for (int o = RB / 2; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+            if (rr == 0) rb[(rq * kHG + rh) * S::GP + g] = v;
+          }
+          wg_sync(grp);
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) tm[g] = fmaxf(tm[g], rb[(q * kHG + rh) * S::GP + g]);
+            if (first) mo[g] = tm[g];
+          }
         }
-        if (!first && wg_vote_or(exceed, grp)) {
+        if (!first && reduce) {
           // rare: O holds earlier tiles' products; publish old and new references,
           // wait for the last product, rescale the moved columns in TMEM
           if (rq == 0 && rr == 0) {
@@ -910,6 +984,11 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           }
           wg_sync(grp);                           // mold / mnew may be rewritten next tile
         }
+        // this group's P buffer (and, with FP8 pools, its V buffer) was last read
+        // by the output product of its previous tile: the issuer put S(tc) after
+        // it on the in-order tensor pipe, so seeing S(tc) means it is complete
+        // (the wait below then returns at once; it keeps the order explicit)
+        if (tc >= 2) wait_pv(tc - 2);
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float p = valid ? exp2f(s[g] - mo[g]) : 0.f;
@@ -923,12 +1002,25 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
           // this V row enters the output product with weight 0: it must hold finite values
           const int seq = 2 * tc + 1, sv_ = seq % NST;
           if (!mbar_wait(bar(Bx::FULL + sv_), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
-          uint4* z0 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + row * 128);
-          uint4* z1 = reinterpret_cast<uint4*>(smem + sv_ * kStageBytes + kHalf + row * 128);
+          uint4* z0 = reinterpret_cast<uint4*>(smem + sv_ * S::kStage + row * 128);
+          uint4* z1 = reinterpret_cast<uint4*>(smem + sv_ * S::kStage + kHalf + row * 128);
 #pragma unroll
           for (int c = 0; c < 8; ++c) { z0[c] = make_uint4(0, 0, 0, 0); z1[c] = make_uint4(0, 0, 0, 0); }
         }
-        fence_proxy_async();
+        if constexpr (KV8) {
+          // V of this tile: its codes become the group's V buffer, widened to f16
+          // (zeros for rows that must not count); the output product of the
+          // group's previous tile, which read the buffer last, is complete (see
+          // above). The code stage is free again once every row has been read.
+          const int seq = 2 * tc + 1, s = seq % NST;
+          if (!mbar_wait(bar(Bx::FULL + s), (seq / NST) & 1, abort_flag, wait_ns)) failed = true;
+          if (in_range && !failed)
+            widen_row_fp8_to<CF>(smem + s * S::kStage, smem + S::OFF_VOP + grp * kStageBytes, row,
+                                 !valid);
+          wg_sync(grp);
+          if (row == 0) mbar_arrive(bar(Bx::EMPTY + s));
+        }
+        fence_proxy_async();                      // P (and the widened V) -> the tensor cores
         mbar_arrive(bar(Bx::PREADY + grp));
         my_last = tc;
       }
@@ -1175,7 +1267,7 @@ template <int FMT, int BS, int G, bool KV8>
 int launch_tc_t(const DecodeArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                 const CUtensorMap& q, cudaStream_t stream) {
   auto kern = decode_tc_kernel<FMT, BS, G, KV8>;
-  constexpr int smem = TcShape<G>::SMEM;
+  constexpr int smem = TcShape<G, KV8>::SMEM;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=

@@ -125,6 +125,17 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// kind::f8f6f4 MMA, both operands in shared memory (E4M3 codes here; the
+// instruction descriptor's type fields read 0 = E4M3): D[M x N] (+)= A . B
+// over K = 32 codes, i.e. the same 32 bytes of each row as one kind::f16 step.
+__device__ __forceinline__ void mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.u32 p, %4, 0;"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
@@ -235,16 +246,18 @@ __device__ __forceinline__ uint32_t widen2_e4m3(uint32_t codes) {
   return (f & 0x80008000u) | (b & ~__vcmpeq2(mag, 0u));
 }
 
-// Widen tile row `row` of a stage in place: its 128 E4M3 codes sit at the
-// stage's upper 16 KB (one 128-byte-swizzled row, as TMA wrote them) and
-// become the row of both 64-wide d-halves of the 16-bit operand layout (the
-// second of which is that very line). Only this thread touches the row, and
-// it reads the whole line before it writes; zero writes zeros instead.
+// Widen tile row `row` of FP8 codes into a 16-bit operand: the row's 128
+// E4M3 codes are one 128-byte-swizzled line at codes + row * 128 (as TMA
+// wrote them) and become the row of both 64-wide d-halves of the operand at
+// op (the halves 16 KB apart, 128-byte swizzled); zero writes zeros instead.
+// The thread reads the whole line before it writes, so the line may be the
+// operand's second half itself (widening in place: codes = op + 16 KB).
 template <int FMT>
-__device__ __forceinline__ void widen_row_fp8(uint8_t* stage, int row, bool zero) {
+__device__ __forceinline__ void widen_row_fp8_to(const uint8_t* codes, uint8_t* op, int row,
+                                                 bool zero) {
   constexpr int kHalf = 128 * 128;           // one 64-wide d-half of a 128-row operand
   const int sw = row & 7;
-  uint8_t* src = stage + kHalf + row * 128;
+  const uint8_t* src = codes + row * 128;
   uint4 c[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -259,11 +272,17 @@ __device__ __forceinline__ void widen_row_fp8(uint8_t* stage, int row, bool zero
       o[2 * k] = widen2_e4m3<FMT>(w[k]);
       o[2 * k + 1] = widen2_e4m3<FMT>(w[k] >> 16);
     }
-    uint8_t* dst = stage + (j >> 2) * kHalf + row * 128;
+    uint8_t* dst = op + (j >> 2) * kHalf + row * 128;
     const int c0 = 2 * (j & 3);
     *reinterpret_cast<uint4*>(dst + ((c0 ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     *reinterpret_cast<uint4*>(dst + (((c0 + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
   }
+}
+// The same in place: the codes sit at the stage's upper 16 KB, which is the
+// row's second d-half afterwards.
+template <int FMT>
+__device__ __forceinline__ void widen_row_fp8(uint8_t* stage, int row, bool zero) {
+  widen_row_fp8_to<FMT>(stage + 128 * 128, stage, row, zero);
 }
 
 // Plain named-barrier sync of one softmax group.

@@ -111,8 +111,12 @@ def test_fp8_one_token_is_the_scaled_v_row():
     assert torch.equal(out.cpu(), torch.from_numpy(exp))
 
 
-def test_full_size_fp8_workload_sampled_parity():
-    w = W.make_workload(6)
+@pytest.mark.parametrize("which", [6, 8])
+def test_full_size_fp8_workload_sampled_parity(which):
+    """The FP8 workloads at full size as the benchmark launches them: the MHA
+    batch (CUDA cores) and the Llama-3-70B-shaped GQA batch (tensor cores, every
+    CTA walking dozens of tiles through the stage ring)."""
+    w = W.make_workload(which)
     out, t = device_step(w)
     torch.cuda.synchronize()
     assert int(t["err"].item()) == 0
@@ -122,7 +126,7 @@ def test_full_size_fp8_workload_sampled_parity():
     for got, exp in ((t["k_cache"], kc), (t["v_cache"], vc)):
         assert torch.equal(got, torch.from_numpy(exp).to(got.device))
     del t
-    rows = sample_rows(w, 48, seed=6)
+    rows = sample_rows(w, 48, seed=which)
     ref = oracle.decode_kv(w.q, w.dtype, kc, vc, oracle.FP8, w.k_scale, w.v_scale,
                            w.block_tables, w.context_lens, w.scale, rows=rows)
     got = out[torch.from_numpy(rows[:, 0]).long(), torch.from_numpy(rows[:, 1]).long()]

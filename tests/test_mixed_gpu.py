@@ -120,6 +120,26 @@ def test_fp8_pools_on_the_tensor_cores(qdt, G, Hkv, bs):
 
 
 @pytest.mark.parametrize("qdt", [W.F16, W.BF16])
+@pytest.mark.parametrize("ctx,G", [
+    ([5000, 37, 1, 800, 4096, 33, 64, 3000] + [17] * 20 + [2049, 700], 8),   # many pieces
+    ([300 + 37 * i for i in range(150)], 4),           # many whole sequences per CTA
+])
+def test_fp8_tensor_cores_over_long_walks(qdt, ctx, G):
+    """Every CTA walks many tiles, so each stage of the ring serves K and V in
+    turn many times over, and sequences are cut into pieces across CTAs."""
+    nb = sum((c + 15) // 16 for c in ctx) + 5
+    w = W.build_decode_case("fp8-tc-long", qdt, B=len(ctx), Hq=G * 8, Hkv=8, D=128,
+                            block_size=16, num_blocks=nb, context_lens=ctx, seed=G + qdt,
+                            kv_fp8=True, k_boost_frac=0.02)
+    assert ops.pa_decode_plan(W.FP8, w.B, w.Hq, w.Hkv, w.D, 16, w.max_context_len)[0] == 2
+    out, t = device_step(w, out_dtype=torch.float32)
+    ref, _, _ = oracle_step(w)
+    torch.cuda.synchronize()
+    assert int(t["err"].item()) == 0
+    assert_attention_close(out, ref, qdt, f"G={G}")
+
+
+@pytest.mark.parametrize("qdt", [W.F16, W.BF16])
 def test_fp8_tensor_core_widening_is_exact_for_every_code(qdt):
     """One token with weight exactly 1: o = value(code) * v_scale, for every finite
     E4M3 code (subnormals and +-448 included), through the tensor-core kernel's
