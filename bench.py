@@ -302,6 +302,7 @@ def reference_arm(args, w: W.Workload, rank: int, world: int):
 KERNEL_SOURCES = {
     "cuda-core": ["decode_simt.cu"],
     "tcgen05": ["decode_tc.cu", "tc_ptx.cuh", "decode_simt.cu"],  # merge kernel: decode_simt.cu
+    "shared-prefix": ["decode_prefix_tc.cu", "decode_tc.cu", "tc_ptx.cuh", "decode_simt.cu"],
 }
 
 
