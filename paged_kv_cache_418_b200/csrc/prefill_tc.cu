@@ -67,7 +67,7 @@ constexpr int kM = 128;                         // query rows per unit (the MMA'
 constexpr int kTile = 128;                      // keys per tile
 constexpr int kHalf = 128 * 128;                // one 64-wide d-half of a 128-row operand
 constexpr int kOp = 2 * kHalf;                  // one 128 x 128 16-bit operand: 32 KB
-constexpr int kNST = 4;                         // K / V ring stages
+constexpr int kNST = 5;                         // K / V ring stages (odd: a stage serves K and V in turn)
 constexpr int kThreads = 192;
 constexpr float kRescaleLog2 = 64.f;
 
@@ -216,6 +216,16 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
   auto ready_bar = [&](int kv, int s) {
     return bar(((kv ? V8 : K8) ? B_CONV : B_FULL) + s);
   };
+  // Phase parity of ring position seq on its ready barrier. FULL completes a
+  // phase on every use of the stage, and so does CONV when both pools hold
+  // codes. With one FP8 pool only its uses are widened: the ring has an odd
+  // number of stages, so a stage's uses alternate K and V, and use u = seq /
+  // kNST of a stage is the (u / 2)-th of its kind.
+  static_assert(kNST % 2 == 1, "uses of a stage alternate K and V");
+  auto ready_parity = [&](int kv, int seq) -> uint32_t {
+    const int u = seq / kNST;
+    return (uint32_t)(((kv ? V8 : K8) && K8 != V8) ? u >> 1 : u) & 1u;
+  };
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -309,7 +319,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         if (first && ui >= 2 && !mbar_wait(bar(B_ODONE + ob), ((ui - 2) >> 1) & 1, abort_flag))
           return false;
         const int seq = 2 * tt + 1, s = seq % kNST;
-        if (!mbar_wait(ready_bar(1, s), (seq / kNST) & 1, abort_flag)) return false;
+        if (!mbar_wait(ready_bar(1, s), ready_parity(1, seq), abort_flag)) return false;
         tc_fence_after();
         const uint32_t vst = sbase + OFF_KV + s * kOp;
 #pragma unroll
@@ -335,7 +345,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         for (int k = 0; k < x.ntiles; ++k, ++tc_) {
           const int sb = tc_ & 1;
           const int seq = 2 * tc_, s = seq % kNST;
-          if (!mbar_wait(ready_bar(0, s), (seq / kNST) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(ready_bar(0, s), ready_parity(0, seq), abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t kst = sbase + OFF_KV + s * kOp;
 #pragma unroll
