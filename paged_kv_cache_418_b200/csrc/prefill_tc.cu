@@ -229,71 +229,76 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int tc_ = 0, issued = 0, ui = 0;
-      int q_last[2] = {-1, -1};
-      for (long long u = blockIdx.x; u < U; u += gridDim.x) {
-        const FUnit x = fa_unit<G>(a, u);
-        if (x.bad && x.c == 0 && x.h == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
-        if (x.ntok <= 0) continue;
-        const int qi = ui & 1;
-        if (!mbar_wait(bar(B_QEMPTY + qi), ((ui >> 1) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-        mbar_expect_tx(bar(B_QFULL + qi), (uint32_t)kOp);
-        for (int hh = 0; hh < 2; ++hh)
-          tma_load_4d(sbase + OFF_Q + qi * kOp + hh * kHalf, &tmQ, 0, hh, x.h * G, x.qrow0,
-                      bar(B_QFULL + qi));
-        q_last[qi] = ui;
-        const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
-        // block-table entries of tile k, read one tile ahead so that their
-        // latency overlaps the current tile's copies
-        auto fetch = [&](int k, int (&ph)[NB_T]) {
-          const int ts = k * kTile;
-          const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
-#pragma unroll
-          for (int q = 0; q < NB_T; ++q) ph[q] = q < nblk ? __ldg(table + ts / BS + q) : -1;
-        };
-        int ahead[NB_T];
-        fetch(0, ahead);
-        for (int k = 0; k < x.ntiles; ++k, ++tc_) {
-          const int ts = k * kTile;
-          const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
-          int phys[NB_T];
-#pragma unroll
-          for (int q = 0; q < NB_T; ++q) phys[q] = ahead[q];
-          if (k + 1 < x.ntiles) fetch(k + 1, ahead);
-          uint32_t bytes = 0;
-#pragma unroll
-          for (int q = 0; q < NB_T; ++q) {
-            if (q < nblk && (phys[q] < 0 || phys[q] >= a.num_blocks)) {
-              flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
-              phys[q] = -1;
-            }
-            if (phys[q] >= 0) bytes += BS * 128u;                // per 128-byte line of rows
-          }
-          for (int kv = 0; kv < 2; ++kv) {
-            const int seq = 2 * tc_ + kv, s = seq % kNST;
-            const bool codes = kv ? V8 : K8;
-            if (!mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-            mbar_expect_tx(bar(B_FULL + s), codes ? bytes : 2u * bytes);
-            const uint32_t dst = sbase + OFF_KV + s * kOp;
-#pragma unroll
-            for (int q = 0; q < NB_T; ++q) {
-              if (phys[q] < 0) continue;
-              if (codes) {
-                tma_load_4d(dst + kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, phys[q],
-                            bar(B_FULL + s));
-              } else {
-                for (int hh = 0; hh < 2; ++hh)
-                  tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
-                              phys[q], bar(B_FULL + s));
-              }
-            }
-            ++issued;
-          }
+    // The warp's lanes share a tile's copies: lane q < NB_T issues those of the
+    // tile's q-th block (one instruction starts them all, instead of one
+    // thread issuing 16-32 in a row) and reads that block's id a tile ahead;
+    // lane 0 waits for free stages, sets the expected bytes and loads the query.
+    int tc_ = 0, issued = 0, ui = 0;
+    int q_last[2] = {-1, -1};
+    bool stop = false;
+    for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
+      const FUnit x = fa_unit<G>(a, u);
+      if (lane == 0 && x.bad && x.c == 0 && x.h == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
+      if (x.ntok <= 0) continue;
+      const int qi = ui & 1;
+      bool ok = true;
+      if (lane == 0) {
+        ok = mbar_wait(bar(B_QEMPTY + qi), ((ui >> 1) & 1) ^ 1, abort_flag);
+        if (ok) {
+          mbar_expect_tx(bar(B_QFULL + qi), (uint32_t)kOp);
+          for (int hh = 0; hh < 2; ++hh)
+            tma_load_4d(sbase + OFF_Q + qi * kOp + hh * kHalf, &tmQ, 0, hh, x.h * G, x.qrow0,
+                        bar(B_QFULL + qi));
+          q_last[qi] = ui;
         }
-        ++ui;
       }
-    prod_done:
+      if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
+      const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
+      // this lane's block of tile k (-1 for none)
+      auto fetch = [&](int k) -> int {
+        const int ts = k * kTile;
+        const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+        return lane < nblk ? __ldg(table + ts / BS + lane) : -1;
+      };
+      int ahead = fetch(0);
+      for (int k = 0; k < x.ntiles && !stop; ++k, ++tc_) {
+        const int ts = k * kTile;
+        const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
+        int phys = ahead;
+        if (k + 1 < x.ntiles) ahead = fetch(k + 1);     // latency overlaps this tile's copies
+        if (lane < nblk && (phys < 0 || phys >= a.num_blocks)) {
+          flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+          phys = -1;
+        }
+        // per 128-byte line of rows of the blocks that are loaded
+        const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, phys >= 0)) * (BS * 128u);
+        for (int kv = 0; kv < 2; ++kv) {
+          const int seq = 2 * tc_ + kv, s = seq % kNST;
+          const bool codes = kv ? V8 : K8;
+          bool ok2 = true;
+          if (lane == 0) {
+            ok2 = mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag);
+            if (ok2) mbar_expect_tx(bar(B_FULL + s), codes ? bytes : 2u * bytes);
+          }
+          if (!__shfl_sync(0xffffffffu, ok2, 0)) { stop = true; break; }
+          const uint32_t dst = sbase + OFF_KV + s * kOp;
+          if (phys >= 0) {
+            if (codes) {
+              tma_load_4d(dst + kHalf + lane * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, phys,
+                          bar(B_FULL + s));
+            } else {
+              for (int hh = 0; hh < 2; ++hh)
+                tma_load_5d(dst + hh * kHalf + lane * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
+                            phys, bar(B_FULL + s));
+            }
+          }
+          ++issued;
+        }
+      }
+      ++ui;
+    }
+    if (lane == 0) {
+      if (stop) give_up();
       // never leave with copies in flight: the last loads of every stage and query buffer
       for (int seq = max(0, issued - kNST); seq < issued; ++seq) {
         const int s = seq % kNST;
