@@ -257,64 +257,66 @@ multi_query_tc_kernel(const PrefixArgs a, const __grid_constant__ CUtensorMap tm
 
   if (warp == kSoftWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The warp's lanes share a tile's copies: lane q < NB_T issues those of the
+    // tile's q-th block (one instruction starts them all) and reads that
+    // block's id a tile ahead; lane 0 waits for free stages and sets the
+    // expected bytes.
+    {
       int tc_ = 0, issued = 0;
-      for (long long u = blockIdx.x; u < U; u += gridDim.x) {
+      bool stop = false;
+      for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
         const PUnit x = mq_unit<PF>(a, G, mc, u);
         if (x.nm <= 0 || x.ntiles == 0) continue;
         const int32_t* table = a.block_tables + (size_t)x.b0 * a.max_blocks;
-        // block ids of tile k of this unit (-1: no block there)
-        auto load_ids = [&](int k, int* ph) {
+        // this lane's block of tile k of the unit (-1 for none)
+        auto load_id = [&](int k) -> int {
           const int ts = x.t0 + k * kTile;
           const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
-#pragma unroll
-          for (int q = 0; q < NB_T; ++q) ph[q] = q < nblk ? __ldg(table + ts / BS + q) : -1;
+          return lane < nblk ? __ldg(table + ts / BS + lane) : -1;
         };
-        int phys_next[NB_T];
-        load_ids(0, phys_next);
-        for (int k = 0; k < x.ntiles; ++k, ++tc_) {
+        int phys_next = load_id(0);
+        for (int k = 0; k < x.ntiles && !stop; ++k, ++tc_) {
           const int ts = x.t0 + k * kTile;
           const int nblk = (min(x.t1, ts + kTile) - ts + BS - 1) / BS;
-          int phys[NB_T];
-          uint32_t bytes = 0;
-#pragma unroll
-          for (int q = 0; q < NB_T; ++q) phys[q] = phys_next[q];
-          if (k + 1 < x.ntiles) load_ids(k + 1, phys_next);   // a tile ahead: off the issue path
-#pragma unroll
-          for (int q = 0; q < NB_T; ++q) {
-            if (q < nblk && (phys[q] < 0 || phys[q] >= a.num_blocks)) {
-              flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
-              phys[q] = -1;
-            }
-            if (phys[q] >= 0) bytes += BS * 128u;                // per 128-byte line of rows
+          int phys = phys_next;
+          if (k + 1 < x.ntiles) phys_next = load_id(k + 1);   // a tile ahead: off the issue path
+          if (lane < nblk && (phys < 0 || phys >= a.num_blocks)) {
+            flag_error(a.err_flag, PA_DEV_BAD_BLOCK_ID);
+            phys = -1;
           }
+          // per 128-byte line of rows of the blocks that are loaded
+          const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, phys >= 0)) * (BS * 128u);
           for (int kv = 0; kv < 2; ++kv) {
             const int seq = 2 * tc_ + kv, s = seq % kNST;
             const bool codes = kv ? V8 : K8;
-            if (!mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag)) { give_up(); goto prod_done; }
-            mbar_expect_tx(bar(B_FULL + s), codes ? bytes : 2u * bytes);
+            bool ok = true;
+            if (lane == 0) {
+              ok = mbar_wait(bar(B_EMPTY + s), ((seq / kNST) & 1) ^ 1, abort_flag);
+              if (ok) mbar_expect_tx(bar(B_FULL + s), codes ? bytes : 2u * bytes);
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) { stop = true; break; }
             const uint32_t dst = sbase + s * kStage;
-#pragma unroll
-            for (int q = 0; q < NB_T; ++q) {
-              if (phys[q] < 0) continue;
+            if (phys >= 0) {
               if (codes) {
-                tma_load_4d(dst + kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, phys[q],
+                tma_load_4d(dst + kHalf + lane * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, phys,
                             bar(B_FULL + s));
               } else {
                 for (int hh = 0; hh < 2; ++hh)
-                  tma_load_5d(dst + hh * kHalf + q * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
-                              phys[q], bar(B_FULL + s));
+                  tma_load_5d(dst + hh * kHalf + lane * (BS * 128), kv ? &tmV : &tmK, 0, 0, x.h, hh,
+                              phys, bar(B_FULL + s));
               }
             }
             ++issued;
           }
         }
       }
-    prod_done:
-      for (int seq = max(0, issued - kNST); seq < issued; ++seq) {
-        const int s = seq % kNST;
-        const uint64_t t0 = globaltimer();
-        while (!mbar_try(bar(B_FULL + s), (seq / kNST) & 1) && globaltimer() - t0 < kWaitNs) {}
+      if (lane == 0) {
+        if (stop) give_up();
+        for (int seq = max(0, issued - kNST); seq < issued; ++seq) {
+          const int s = seq % kNST;
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(bar(B_FULL + s), (seq / kNST) & 1) && globaltimer() - t0 < kWaitNs) {}
+        }
       }
     }
   } else if (warp == kSoftWarps + 1) {
