@@ -320,8 +320,10 @@ decode_simt_kernel(const DecodeArgs a) {
   }
 }
 
-// Prefetching the next tile (PF) pays where a warp's tile carries few bytes
-// (FP8 pools: half the bytes of a 16-bit tile per load); PA_SIMT_PREFETCH=0/1
+// Prefetching the next tile (PF) keeps two tiles of loads in flight per warp:
+// it pays where a warp's tile carries few bytes (FP8 pools: half the bytes of a
+// 16-bit tile per load) and on the MHA shape (one query head per CTA), where
+// the extra registers still leave enough warps per SM; PA_SIMT_PREFETCH=0/1
 // overrides the choice, for measurements.
 int prefetch_override() {
   const char* s = std::getenv("PA_SIMT_PREFETCH");
@@ -334,7 +336,10 @@ int launch_t(const DecodeArgs& a, cudaStream_t stream) {
   const int chunks = (a.Hq / a.Hkv) / GC;
   dim3 grid((unsigned)(a.P * chunks), (unsigned)a.Hkv, (unsigned)a.B);
   const int ov = prefetch_override();
-  const bool pf = ov >= 0 ? ov == 1 : (sizeof(TK) == 1 || sizeof(TV) == 1);
+  // loads of the next tile issued before the current one is computed: the default
+  // for one query head per CTA (MHA: the extra registers leave enough warps) and
+  // for pools of codes (half the bytes per row, so a warp needs two tiles in flight)
+  const bool pf = ov >= 0 ? ov == 1 : (GC == 1 || sizeof(TK) == 1 || sizeof(TV) == 1);
   const cudaError_t e =
       pf ? launch_k(decode_simt_kernel<TQ, TK, TV, D, BS, GC, true>, grid, dim3(kWarps * 32), 0,
                     stream, a)

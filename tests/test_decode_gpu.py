@@ -55,6 +55,21 @@ def test_shrunk_workloads_full_parity(which, out_f32, kernel_choice):
     assert torch.equal(bits(t["v_cache"]).cpu(), host_bits(vc))
 
 
+# -- both load schedules of the CUDA-core kernel on the 16-bit and fp32 MHA shapes ----
+@pytest.mark.parametrize("prefetch", ["0", "1"])
+@pytest.mark.parametrize("which", [1, 2])
+def test_cuda_core_load_schedules_agree_with_the_oracle(which, prefetch, monkeypatch):
+    """The CUDA-core kernel with and without the next tile's loads in flight
+    (the default differs by shape and pool type; both must be exact)."""
+    monkeypatch.setenv("PA_SIMT_PREFETCH", prefetch)
+    w = W.make_workload(1) if which == 1 else W.shrink_workload(which, seed=300 + which)
+    out, t = device_step(w, out_dtype=torch.float32)
+    ref, _, _ = oracle_step(w)
+    torch.cuda.synchronize()
+    assert int(t["err"].item()) == 0
+    assert_attention_close(out, ref, w.dtype, f"{w.name} prefetch={prefetch}")
+
+
 # -- every supported shape, ragged lengths across partition boundaries ------------
 SHAPES = [(dt, D, bs, G) for dt in (W.F32, W.F16, W.BF16) for D in (64, 128) for bs in (16, 32)
           for G in (1, 2, 4, 8, 16)]
