@@ -22,25 +22,32 @@
 // from tensor memory: each 32-key chunk of S becomes 16 columns of hi parts
 // followed by 16 columns of lo parts (two keys per 32-bit column).
 //
-// A softmax thread owns one query row, so the row maximum and the row sum
-// need no exchange with other threads. It reads its row of S twice, 32
-// columns at a time: once for the tile's maximum, once for the weights, which
-// it writes over the chunk it has just read. (Holding all 128 scores in
-// registers instead made the loop body four times longer and the softmax
-// warps stall on instruction fetch.) The reference maximum of a row is its first tile's maximum
+// Two softmax groups share a unit's 128 query rows: thread (group hf, row r)
+// owns row r's keys [64 hf, 64 hf + 64) of every tile and O's columns [64 hf,
+// 64 hf + 64), so a row needs only its two threads to agree: they exchange the
+// tile's row maximum (and, at the unit's end, their parts of the row sum)
+// through shared memory. A thread reads its scores twice, 32 columns at a
+// time: once for the maximum, once for the weights, which it writes over the
+// chunk it has just read. (Holding all of a row's scores in registers made the
+// loop body four times longer; a per-key mask branch inside the loops cost
+// more than the rest of the tile's softmax: the mask is one bit per key of a
+// 32-key chunk, and whole chunks take a loop without it.) The reference
+// maximum of a row is its first tile's maximum
 // and moves only when a later tile exceeds it by 2^64 (then the row's O is
-// rescaled in tensor memory, which its own thread does); references are
+// rescaled in tensor memory, each half by its thread); references are
 // floored at -FLT_MAX so masked scores (-inf) give weight 0 without a guard.
 // Keys past a row's position are masked; the V rows of keys that no row of
 // the unit attends (past its last position, or in a block with a bad id) are
 // zeroed in shared memory before the output product, so they add exact zeros.
 //
-// CTA = 6 warps, persistent over units u = blockIdx.x + k * gridDim.x (the
+// CTA = 10 warps, persistent over units u = blockIdx.x + k * gridDim.x (the
 // chunks late in their sequences, which attend the most keys, first):
-//   warps 0-3  softmax and epilogue (thread = query row = TMEM lane);
-//   warp 4     TMA producer: the unit's query (double-buffered by unit), the
-//              K and V tiles through a ring of 32 KB stages;
-//   warp 5     MMA issuer and owner of the tensor memory: S(t), then the
+//   warps 0-7  softmax and epilogue, two groups (thread = query row = TMEM
+//              lane; warps w and w + 4 reach the same lanes);
+//   warp 8     TMA producer: the unit's query (double-buffered by unit), the
+//              K and V tiles through a ring of 32 KB stages (its lanes issue
+//              the copies of a tile's blocks together);
+//   warp 9     MMA issuer and owner of the tensor memory: S(t), then the
 //              output product of tile t - 1 (S is double-buffered by tile, O
 //              by unit, so a unit's epilogue overlaps the next unit's tiles).
 // Every pipeline wait is bounded (1 s); one that gives up sets PA_DEV_TIMEOUT,
@@ -68,7 +75,8 @@ constexpr int kTile = 128;                      // keys per tile
 constexpr int kHalf = 128 * 128;                // one 64-wide d-half of a 128-row operand
 constexpr int kOp = 2 * kHalf;                  // one 128 x 128 16-bit operand: 32 KB
 constexpr int kNST = 5;                         // K / V ring stages (odd: a stage serves K and V in turn)
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;                   // two softmax groups, producer, MMA
+constexpr int kProdWarp = 8, kMmaWarp = 9;
 constexpr float kRescaleLog2 = 64.f;
 
 constexpr int OFF_Q = 0;                        // [2 units][32 KB]
@@ -79,7 +87,8 @@ enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY = B_QFULL + 2,
        B_ODONE = B_OSTEP + 1, B_DONE = B_ODONE + 2, B_CONV = B_DONE + 1,
        B_COUNT = B_CONV + kNST };
 constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
-constexpr int kSmem = OFF_MISC + 16 + 1024;     // + alignment slack
+constexpr int OFF_XCH = OFF_MISC + 16;          // [2 groups][128 rows]: row maxima, then row sums
+constexpr int kSmem = OFF_XCH + 2 * 128 * 4 + 1024;   // + alignment slack
 static_assert(kSmem <= 227 * 1024, "shared memory per CTA");
 constexpr int kTmemCols = 512;                  // S/P x2 (by tile), O x2 (by unit)
 
@@ -184,8 +193,8 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       mbar_init(bar(B_QFULL + i), 1);
       mbar_init(bar(B_QEMPTY + i), 1);
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_PREADY + i), 128);
-      mbar_init(bar(B_ODONE + i), 128);
+      mbar_init(bar(B_PREADY + i), 256);
+      mbar_init(bar(B_ODONE + i), 256);
     }
     mbar_init(bar(B_OSTEP), 1);
     mbar_init(bar(B_DONE), 1);
@@ -193,7 +202,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
     *abort_flag = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_slot)),
                  "r"(kTmemCols)
@@ -227,7 +236,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
     return (uint32_t)(((kv ? V8 : K8) && K8 != V8) ? u >> 1 : u) & 1u;
   };
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     // ------------------------------------------------------------ producer
     // The warp's lanes share a tile's copies: lane q < NB_T issues those of the
     // tile's q-th block (one instruction starts them all, instead of one
@@ -311,7 +320,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         while (!mbar_try(bar(B_QFULL + qb), (q_last[qb] >> 1) & 1) && globaltimer() - t0 < kWaitNs) {}
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int tc_ = 0, ui = 0;
@@ -374,9 +383,23 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int r = threadIdx.x;                   // query row = TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    // Two groups of four warps share the 128 query rows: thread (hf, r) owns row
+    // r's keys [64 hf, 64 hf + 64) of each tile and its O columns [64 hf, 64 hf +
+    // 64) (warps w and w + 4 reach the same tensor-memory lanes). The groups
+    // exchange each tile's row maxima and, at a unit's end, the row sums.
+    const int r = threadIdx.x & 127;             // query row = TMEM lane
+    const int hf = threadIdx.x >> 7;             // which half of the keys and of O
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const int tl = r / G, g = r - (r / G) * G;   // token of the unit, head of the group
+    float* xch = reinterpret_cast<float*>(smem + OFF_XCH);    // [2][128]
+    auto sync256 = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+    auto vote256 = [](bool v) -> bool {
+      uint32_t o;
+      asm volatile("{ .reg .pred pi, po; setp.ne.u32 pi, %1, 0; bar.red.or.pred po, 1, 256, pi;"
+                   " selp.u32 %0, 1, 0, po; }"
+                   : "=r"(o) : "r"((uint32_t)v) : "memory");
+      return o != 0;
+    };
     bool failed = false;
     int tc_ = 0, ui = 0, ostep = 0;              // tiles seen, units done, O products issued
     for (long long u = blockIdx.x; u < U && !failed; u += gridDim.x) {
@@ -386,7 +409,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       const bool row_ok = tl < x.ntok;
       const int pos = x.pos0 + tl;               // this row attends keys [0, pos]
       const int32_t* table = a.block_tables + (size_t)x.b * a.max_blocks;
-      float m = -CUDART_INF_F, l = 0.f;
+      float m = -CUDART_INF_F, l = 0.f;          // l: this half's part of the row sum
       // blocks of tile j with a bad id (the producer loaded nothing there)
       auto tile_bad = [&](int j) {
         const int tsj = j * kTile;
@@ -400,17 +423,16 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         }
         return bb;
       };
-      // FP8 pools: widen row r of tile j's K and V stages (global tile tj); a V
-      // row no row of the unit attends becomes zeros
+      // FP8 pools: widen row r of tile j's K stage (group 0) or V stage (group 1)
+      // (global tile tj); a V row no row of the unit attends becomes zeros
       auto widen_tile = [&](int j, int tj) {
         if constexpr (K8 || V8) {
-          const bool zv = j * kTile + r >= x.t1 || ((tile_bad(j) >> (r / BS)) & 1u);
-#pragma unroll 1
-          for (int kv = 0; kv < 2; ++kv) {
-            if (!(kv ? V8 : K8)) continue;
+          const int kv = hf;
+          if (kv ? V8 : K8) {
+            const bool zv = kv == 1 && (j * kTile + r >= x.t1 || ((tile_bad(j) >> (r / BS)) & 1u));
             const int seq = 2 * tj + kv, s = seq % kNST;
             if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) failed = true;
-            if (!failed) widen_row_fp8<FMT>(smem + OFF_KV + s * kOp, r, kv == 1 && zv);
+            if (!failed) widen_row_fp8<FMT>(smem + OFF_KV + s * kOp, r, zv);
             fence_proxy_async();
             mbar_arrive(bar(B_CONV + s));
           }
@@ -440,10 +462,11 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           return row_ok ? msk : 0u;
         };
         const float sl2 = a.scale_log2;
-        // pass 1: the tile's row maximum, 32 columns of S at a time
+        const int c_lo = 64 * hf;                // this half's first key column
+        // pass 1: the maximum over this half's 64 keys, 32 columns of S at a time
         float tm = -CUDART_INF_F;
 #pragma unroll 1
-        for (int c = 0; c < kTile; c += 32) {
+        for (int c = c_lo; c < c_lo + 64; c += 32) {
           uint32_t raw[32];
           tmem_ld32(srow + c, raw);
           tmem_wait_ld();
@@ -468,6 +491,12 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           }
           tm = fmaxf(tm, fmaxf(fmaxf(t0, t1), fmaxf(t2, t3)));
         }
+        // the row's tile maximum: both halves (the second barrier keeps the
+        // buffer until both have read it)
+        xch[hf * 128 + r] = tm;
+        sync256();
+        tm = fmaxf(xch[r], xch[128 + r]);
+        sync256();
         float alpha = 1.f;
         bool resc = false;
         if (k == 0) {
@@ -479,11 +508,12 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         }
         if (__any_sync(0xffffffffu, resc)) {
           // rare: this warp's rows move their reference; O holds the products of
-          // tiles up to k - 1: wait for the last one, rescale the rows in TMEM
+          // tiles up to k - 1: wait for the last one, rescale this half of the
+          // rows in TMEM (both halves of a row take the same decision)
           if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < kD; c += 32) {
+          for (int c = c_lo; c < c_lo + 64; c += 32) {
             uint32_t o[32];
             tmem_ld32(tmem_o + lane_off + ob * kD + c, o);
             tmem_wait_ld();
@@ -494,11 +524,11 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           tmem_wait_st();
           l *= alpha;
         }
-        // pass 2: weights and the row sum; each 32-column chunk of S is read
-        // again and overwritten by its weights' 16-bit parts, hi in the chunk's
-        // first 16 columns and lo in the next 16 (two keys per column)
+        // pass 2: weights and this half's part of the row sum; each 32-column
+        // chunk of S is read again and overwritten by its weights' 16-bit parts,
+        // hi in the chunk's first 16 columns and lo in the next 16
 #pragma unroll 1
-        for (int c = 0; c < kTile; c += 32) {
+        for (int c = c_lo; c < c_lo + 64; c += 32) {
           uint32_t raw[32];
           tmem_ld32(srow + c, raw);
           tmem_wait_ld();
@@ -530,13 +560,13 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           tmem_st32(srow + c, pk);
         }
         if (!V8 && zero_v) {
-          // this V row enters the output product with weight 0: it must hold finite values
+          // this V row enters the output product with weight 0: it must hold
+          // finite values (each group zeroes one d-half of the row)
           const int seq = 2 * tc_ + 1, s = seq % kNST;
           if (!mbar_wait(bar(B_FULL + s), (seq / kNST) & 1, abort_flag)) failed = true;
-          uint4* z0 = reinterpret_cast<uint4*>(smem + OFF_KV + s * kOp + r * 128);
-          uint4* z1 = reinterpret_cast<uint4*>(smem + OFF_KV + s * kOp + kHalf + r * 128);
+          uint4* z = reinterpret_cast<uint4*>(smem + OFF_KV + s * kOp + hf * kHalf + r * 128);
 #pragma unroll
-          for (int q = 0; q < 8; ++q) { z0[q] = make_uint4(0, 0, 0, 0); z1[q] = make_uint4(0, 0, 0, 0); }
+          for (int q = 0; q < 8; ++q) z[q] = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async();
         tmem_wait_st();
@@ -545,16 +575,20 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         ++ostep;
         if (k + 1 < x.ntiles) widen_tile(k + 1, tc_ + 1);
       }
-      // ---- epilogue: O / l of this row to the output. The products of the
-      // last two tiles may both be pending; a parity wait names one of two
-      // phases, so wait for them in order.
+      // ---- epilogue: O / l of this row to the output, each half its 64
+      // columns. The products of the last two tiles may both be pending; a
+      // parity wait names one of two phases, so wait for them in order.
+      xch[hf * 128 + r] = l;
+      sync256();
+      const float lrow = xch[r] + xch[128 + r];
+      sync256();
       if (ostep >= 2 && !mbar_wait(bar(B_OSTEP), (ostep - 2) & 1, abort_flag)) failed = true;
       if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
       tc_fence_after();
-      const float inv = l > 0.f ? a.v_scale / l : 0.f;
+      const float inv = lrow > 0.f ? a.v_scale / lrow : 0.f;
       const size_t orow = ((size_t)(x.qrow0 + tl) * a.Hq + (size_t)x.h * G + g) * kD;
 #pragma unroll 1
-      for (int c = 0; c < kD; c += 32) {
+      for (int c = 64 * hf; c < 64 * hf + 64; c += 32) {
         uint32_t o[32];
         tmem_ld32(tmem_o + lane_off + ob * kD + c, o);
         tmem_wait_ld();
@@ -587,15 +621,15 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       tc_fence_before();
       mbar_arrive(bar(B_ODONE + ob));
       ++ui;
-      // the warps of the group leave together
-      failed = wg_vote_or(failed, 0);
+      // the warps of both groups leave together
+      failed = vote256(failed);
     }
     if (failed) give_up();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
