@@ -40,8 +40,9 @@
 // the unit attends (past its last position, or in a block with a bad id) are
 // zeroed in shared memory before the output product, so they add exact zeros.
 //
-// CTA = 10 warps, persistent over units u = blockIdx.x + k * gridDim.x (the
-// chunks late in their sequences, which attend the most keys, first):
+// CTA = 10 warps, persistent over rounds of units taken in alternating
+// directions (fa_unit_of_cta; the chunks late in their sequences, which
+// attend the most keys, come first):
 //   warps 0-7  softmax and epilogue, two groups (thread = query row = TMEM
 //              lane; warps w and w + 4 reach the same lanes);
 //   warp 8     TMA producer: the unit's query (double-buffered by unit), the
@@ -133,6 +134,14 @@ __device__ __forceinline__ FUnit fa_unit(const FaArgs& a, long long u) {
   x.t1 = x.ntok > 0 ? x.pos0 + x.ntok : 0;
   x.ntiles = (x.t1 + kTile - 1) / kTile;
   return x;
+}
+
+// The k-th unit of CTA cta: rounds of grid units, taken in alternating
+// directions (CTA c gets unit c of even rounds and unit grid - 1 - c of odd
+// ones). Units come longest first, so plain round-robin would hand CTA 0 the
+// largest unit of every round.
+__device__ __forceinline__ long long fa_unit_of_cta(long long k, int cta, int grid) {
+  return k * grid + ((k & 1) ? grid - 1 - cta : cta);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -245,7 +254,9 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
     int tc_ = 0, issued = 0, ui = 0;
     int q_last[2] = {-1, -1};
     bool stop = false;
-    for (long long u = blockIdx.x; u < U && !stop; u += gridDim.x) {
+    for (long long kk = 0; !stop; ++kk) {
+      const long long u = fa_unit_of_cta(kk, blockIdx.x, gridDim.x);
+      if (u >= U) break;
       const FUnit x = fa_unit<G>(a, u);
       if (lane == 0 && x.bad && x.c == 0 && x.h == 0) flag_error(a.err_flag, PA_DEV_BAD_CTX);
       if (x.ntok <= 0) continue;
@@ -350,7 +361,9 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         mma_commit(bar(B_OSTEP));
         return true;
       };
-      for (long long u = blockIdx.x; u < U && ok; u += gridDim.x) {
+      for (long long kk = 0; ok; ++kk) {
+        const long long u = fa_unit_of_cta(kk, blockIdx.x, gridDim.x);
+        if (u >= U) break;
         const FUnit x = fa_unit<G>(a, u);
         if (x.ntok <= 0) continue;
         const int qi = ui & 1, ob = ui & 1;
@@ -402,7 +415,9 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
     };
     bool failed = false;
     int tc_ = 0, ui = 0, ostep = 0;              // tiles seen, units done, O products issued
-    for (long long u = blockIdx.x; u < U && !failed; u += gridDim.x) {
+    for (long long kk = 0; !failed; ++kk) {
+      const long long u = fa_unit_of_cta(kk, blockIdx.x, gridDim.x);
+      if (u >= U) break;
       const FUnit x = fa_unit<G>(a, u);
       if (x.ntok <= 0) continue;
       const int ob = ui & 1;
