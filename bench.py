@@ -303,11 +303,12 @@ KERNEL_SOURCES = {
     "cuda-core": ["decode_simt.cu"],
     "tcgen05": ["decode_tc.cu", "tc_ptx.cuh", "decode_simt.cu"],  # merge kernel: decode_simt.cu
     "shared-prefix": ["decode_prefix_tc.cu", "decode_tc.cu", "tc_ptx.cuh", "decode_simt.cu"],
+    "prefill": ["prefill_tc.cu", "tc_ptx.cuh"],
 }
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of what a decode path's device code is built from: its kernel files,
+    """Hash of what a kernel path's device code is built from: its kernel files,
     the device helpers, and the launch-argument struct (declarations of other
     entry points do not change the kernels, so they are left out)."""
     import re
@@ -316,18 +317,19 @@ def kernel_source_hash(kernel: str) -> str:
     for f in KERNEL_SOURCES[kernel] + ["pa_common.cuh"]:
         h.update(open(os.path.join(csrc, f), "rb").read())
     internal = open(os.path.join(csrc, "pa_internal.h")).read()
-    m = re.search(r"struct DecodeArgs \{.*?\};", internal, re.S)
+    struct = "PrefillLaunch" if kernel == "prefill" else "DecodeArgs"
+    m = re.search(r"struct " + struct + r" \{.*?\};", internal, re.S)
     h.update((m.group(0) if m else internal).encode())
     return h.hexdigest()[:16]
 
 
-def traffic_record(kernel: str, w: W.Workload):
-    """DRAM bytes per pa_decode launch from a committed ncu summary, or None when
-    there is none for this workload or the kernel's sources changed since."""
+def traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch of a workload's kernel from a committed ncu summary,
+    or None when there is none for it or the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(path):
         return None
-    rec = json.load(open(path)).get(w.name)
+    rec = json.load(open(path)).get(workload)
     if not rec or rec.get("kernel") != kernel or rec.get("source_hash") != kernel_source_hash(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -559,7 +561,7 @@ def measure(args, w: W.Workload, rank: int, world: int, local_rank: int, *,
     # the cascade reads each distinct K/V byte once: its algorithmic bytes are the distinct ones
     alg = unique if cascade else kv
     achieved = alg / (dec_ms / 1e3) / 1e9
-    traffic = traffic_record(kname, w)
+    traffic = traffic_record(kname, w.name)
     e2e_value = job_value(kv, Ke, world, e_ms)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -868,7 +870,7 @@ def prefill_arm(args, rank: int, world: int, local_rank: int):
         del os.environ["PA_PREFILL_KERNEL"]
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     peak = float(json.load(open(path))["bf16_tflops"]) if os.path.exists(path) else 1590.0
-    # end to end: query and tables from pinned host memory, output back, every call
+    # end to end: the query from pinned host memory, the output back, every call
     hq = t["q"].cpu().pin_memory()
     hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -899,7 +901,8 @@ def prefill_arm(args, rank: int, world: int, local_rank: int):
                    "flops_per_step": flops, "l2": "K/V of the batch read once per 8-token "
                    "query chunk; inputs resident, no flush (compute-bound)"},
         "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                     "traffic": traffic_record("prefill", c.name),
                      "peak_source": "bf16_tflops (measured, burst)",
                      "kernel": "prefill_fa_kernel (query rows on the MMA's M), per launch; "
                                "algorithmic flops 4*D per (query head, attended key)"},

@@ -85,7 +85,7 @@ constexpr int OFF_KV = 2 * kOp;                 // [kNST][32 KB]
 constexpr int OFF_BAR = OFF_KV + kNST * kOp;
 enum { B_FULL = 0, B_EMPTY = kNST, B_QFULL = 2 * kNST, B_QEMPTY = B_QFULL + 2,
        B_SFULL = B_QEMPTY + 2, B_PREADY = B_SFULL + 2, B_OSTEP = B_PREADY + 2,
-       B_ODONE = B_OSTEP + 1, B_DONE = B_ODONE + 2, B_CONV = B_DONE + 1,
+       B_ODONE = B_OSTEP + 2, B_DONE = B_ODONE + 2, B_CONV = B_DONE + 1,
        B_COUNT = B_CONV + kNST };
 constexpr int OFF_MISC = OFF_BAR + 8 * B_COUNT;
 constexpr int OFF_XCH = OFF_MISC + 16;          // [2 groups][128 rows]: row maxima, then row sums
@@ -203,9 +203,9 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       mbar_init(bar(B_QEMPTY + i), 1);
       mbar_init(bar(B_SFULL + i), 1);
       mbar_init(bar(B_PREADY + i), 256);
+      mbar_init(bar(B_OSTEP + i), 1);
       mbar_init(bar(B_ODONE + i), 256);
     }
-    mbar_init(bar(B_OSTEP), 1);
     mbar_init(bar(B_DONE), 1);
     for (int s = 0; s < kNST; ++s) mbar_init(bar(B_CONV + s), 128);
     *abort_flag = 0u;
@@ -358,7 +358,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           }
         }
         mma_commit(bar(B_EMPTY + s));
-        mma_commit(bar(B_OSTEP));
+        mma_commit(bar(B_OSTEP + pb));
         return true;
       };
       for (long long kk = 0; ok; ++kk) {
@@ -414,7 +414,17 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
       return o != 0;
     };
     bool failed = false;
-    int tc_ = 0, ui = 0, ostep = 0;              // tiles seen, units done, O products issued
+    int tc_ = 0, ui = 0;                         // tiles seen, units done
+    // Wait for the output product of tile t. Products alternate between two
+    // barriers by tile parity, so a parity wait is exact: the barrier of t has
+    // passed the phase before t's (this group has seen S of tile t or a later
+    // one, and the issuer puts S(t) after O(t - 2) on the in-order tensor pipe)
+    // and cannot pass t's own before the group hands over tile t + 2. (One
+    // barrier for every product could pass two phases while a slow warp had
+    // not yet looked, and a parity wait would then take the wrong phase.)
+    auto wait_o = [&](int t) {
+      if (!mbar_wait(bar(B_OSTEP + (t & 1)), (t >> 1) & 1, abort_flag)) failed = true;
+    };
     for (long long kk = 0; !failed; ++kk) {
       const long long u = fa_unit_of_cta(kk, blockIdx.x, gridDim.x);
       if (u >= U) break;
@@ -525,7 +535,7 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
           // rare: this warp's rows move their reference; O holds the products of
           // tiles up to k - 1: wait for the last one, rescale this half of the
           // rows in TMEM (both halves of a row take the same decision)
-          if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
+          wait_o(tc_ - 1);
           tc_fence_after();
 #pragma unroll 1
           for (int c = c_lo; c < c_lo + 64; c += 32) {
@@ -587,18 +597,16 @@ prefill_fa_kernel(const FaArgs a, const __grid_constant__ CUtensorMap tmQ,
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(B_PREADY + sb));
-        ++ostep;
         if (k + 1 < x.ntiles) widen_tile(k + 1, tc_ + 1);
       }
       // ---- epilogue: O / l of this row to the output, each half its 64
-      // columns. The products of the last two tiles may both be pending; a
-      // parity wait names one of two phases, so wait for them in order.
+      // columns. The products of the last two tiles may both be pending; the
+      // last one's commit tracks every earlier MMA, so one wait covers both.
       xch[hf * 128 + r] = l;
       sync256();
       const float lrow = xch[r] + xch[128 + r];
       sync256();
-      if (ostep >= 2 && !mbar_wait(bar(B_OSTEP), (ostep - 2) & 1, abort_flag)) failed = true;
-      if (!mbar_wait(bar(B_OSTEP), (ostep - 1) & 1, abort_flag)) failed = true;
+      wait_o(tc_ - 1);
       tc_fence_after();
       const float inv = lrow > 0.f ? a.v_scale / lrow : 0.f;
       const size_t orow = ((size_t)(x.qrow0 + tl) * a.Hq + (size_t)x.h * G + g) * kD;
