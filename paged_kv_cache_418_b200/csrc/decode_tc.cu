@@ -19,10 +19,16 @@
 // the same bytes as 2-4 KB per-head boxes is limited by TMA issue, not HBM.
 //
 // Work split: the tiles of all (sequence b, group h of HG KV heads) pairs,
-// in (b, h, tile) order, form one list of T tiles, and CTA c takes the tiles
-// [floor(c T / grid), floor((c + 1) T / grid)): every CTA streams the same
-// number of tiles (+-1), whatever the mix of context lengths, so no CTA
-// finishes a long sequence alone at the end. A CTA's share is a run of units:
+// in (b, h, tile) order, form one list of T tiles, and the CTAs take equal
+// shares of its cost: a tile costs kCostTile, and each pair adds
+// DecodeArgs::pair_cost for the work of starting and finishing a unit (the
+// query load, the first tile's reduction, the epilogue), so a CTA whose share
+// crosses many short pairs streams fewer tiles. Tile x of the p-th pair with
+// tiles sits at cost position kCostTile * x + pair_cost * (p + 1), and CTA c
+// takes the tiles whose positions lie in [floor(c C / grid),
+// floor((c + 1) C / grid)), C the total cost: every CTA does about the same
+// work whatever the mix of context lengths, so no CTA finishes a long
+// sequence alone at the end. A CTA's share is a run of units:
 // whole pairs in the middle, and at each end possibly a piece of a pair that
 // continues in the neighbouring CTA. A whole pair is written to the output
 // directly. A piece is written as (reference max, exp-sum, unnormalised
@@ -150,32 +156,65 @@ struct Misc {
   uint32_t abort_flag;
   int32_t valid;        // this CTA's share holds tiles
   int32_t b0, h0, k0;   // first unit: sequence, KV-head group, first tile in the pair
-  int32_t found;        // prologue scan: the first unit has been located
+  int32_t found;        // prologue scan: bit 0 the share's start located, bit 1 its end
   int32_t last[2];      // per softmax group: this piece was the last of its pair
-  int32_t pad;
+  int32_t p0;           // first unit's pair: its index among the pairs with tiles
   long long r0, r1;     // the share: global tiles [r0, r1)
-  long long T;          // tiles of all pairs
+  long long C;          // cost of all pairs
 };
 static_assert(sizeof(Misc) <= 64, "misc words");
 
 // ---------------------------------------------------------------- the work list
-// First global tile of CTA c: floor(c * T / grid), without 64-bit overflow.
-__device__ __forceinline__ long long share_begin(long long c, long long T, long long grid) {
-  return (T / grid) * c + ((T % grid) * c) / grid;
+constexpr long long kCostTile = 16;             // cost of one tile (pair_cost is in these units)
+
+// First cost position of CTA c's share: floor(c * C / grid), without 64-bit overflow.
+__device__ __forceinline__ long long share_begin(long long c, long long C, long long grid) {
+  return (C / grid) * c + ((C % grid) * c) / grid;
 }
-// The CTA whose share holds global tile x (the largest c with share_begin(c) <= x).
-__device__ __forceinline__ int share_owner(long long x, long long T, long long grid) {
-  return (int)(((x + 1) * grid - 1) / T);
+// The CTA whose share holds cost position x (the largest c with share_begin(c) <= x).
+__device__ __forceinline__ int share_owner(long long x, long long C, long long grid) {
+  return (int)(((x + 1) * grid - 1) / C);
+}
+// Cost position of global tile x of the p-th pair with tiles.
+__device__ __forceinline__ long long tile_cost(long long x, long long p, long long pair_cost) {
+  return kCostTile * x + pair_cost * (p + 1);
 }
 
-// CTAs that hold a piece of the pair whose tiles are [pair0, pair0 + ntp):
-// the owners of its first and last tile and every CTA between them whose
-// share is not empty (shares are empty only when there are fewer tiles than
-// CTAs).
-__device__ __forceinline__ int pair_pieces(long long pair0, int ntp, long long T, int grid) {
-  const int c0 = share_owner(pair0, T, grid), c1 = share_owner(pair0 + ntp - 1, T, grid);
+// The shares that hold tiles of one pair (tiles [pair0, pair0 + ntp), the p-th
+// pair with tiles): CTAs c0 .. c1, the owners of its first and last tile, and
+// each one's piece slot. A CTA between them whose share falls between two of
+// the pair's tiles holds no piece. c0's share starts before the pair when it
+// also holds the previous pair's last tile (global tile pair0 - 1, p - 1).
+struct PairShares {
+  long long pos0;       // cost position of the pair's first tile
+  long long pair0;
+  int ntp, c0, c1;
+  bool c0_before;       // the pair is c0's last unit (slot 2 c0 + 1), else its first
+};
+__device__ __forceinline__ PairShares pair_shares(long long pair0, int ntp, long long p,
+                                                  long long C, int grid, long long pair_cost) {
+  PairShares r;
+  r.pos0 = tile_cost(pair0, p, pair_cost);
+  r.pair0 = pair0;
+  r.ntp = ntp;
+  r.c0 = share_owner(r.pos0, C, grid);
+  r.c1 = share_owner(r.pos0 + kCostTile * (ntp - 1), C, grid);
+  r.c0_before = p > 0 && share_begin(r.c0, C, grid) <= tile_cost(pair0 - 1, p - 1, pair_cost);
+  return r;
+}
+// First tile of share c (c0 < c <= c1 + 1) inside the pair; the pair's end for c1 + 1.
+__device__ __forceinline__ long long share_first_tile(const PairShares& r, int c, long long C,
+                                                      int grid) {
+  if (c > r.c1) return r.pair0 + r.ntp;
+  return r.pair0 + (share_begin(c, C, grid) - r.pos0 + kCostTile - 1) / kCostTile;
+}
+// Does share c (c0 <= c <= c1) hold a tile of the pair?
+__device__ __forceinline__ bool share_holds(const PairShares& r, int c, long long C, int grid) {
+  return c == r.c0 || share_first_tile(r, c, C, grid) < share_first_tile(r, c + 1, C, grid);
+}
+__device__ __forceinline__ int pair_pieces(const PairShares& r, long long C, int grid) {
   int n = 0;
-  for (int c = c0; c <= c1; ++c) n += share_begin(c + 1, T, grid) > share_begin(c, T, grid);
+  for (int c = r.c0; c <= r.c1; ++c) n += share_holds(r, c, C, grid);
   return n;
 }
 
@@ -197,6 +236,7 @@ __device__ __forceinline__ bool seq_bad(const DecodeArgs& a, int ctx, int start)
 // A walk over this CTA's share, one unit (a pair, or a piece of one) at a time.
 struct Cursor {
   int b, h;             // current pair
+  int p;                // its index among the pairs with tiles
   int k0, k1;           // tiles [k0, k1) of the pair in this unit
   int ntp;              // tiles of the pair
   int ctx, start;       // the sequence's length and the first token of the pass
@@ -218,6 +258,7 @@ __device__ __forceinline__ void cur_init(const DecodeArgs& a, Cursor& c, const M
   if (!c.valid) return;
   c.b = ms->b0;
   c.h = ms->h0;
+  c.p = ms->p0;
   c.ntp = seq_tiles<BS>(a, c.b, c.ctx, c.start);
   c.g0 = ms->r0;
   cur_fill(c, ms->k0, ms->r1 - ms->r0);
@@ -229,6 +270,7 @@ __device__ __forceinline__ void cur_next(const DecodeArgs& a, int nhg, Cursor& c
   if (!c.valid) return;
   if (c.left <= 0) { c.valid = false; return; }
   c.g0 += c.k1 - c.k0;
+  ++c.p;
   if (++c.h >= nhg) {
     c.h = 0;
     int n = 0;
@@ -246,6 +288,7 @@ struct Unit {
   bool whole;           // the unit is its whole pair
   long long g0;         // global index of its first tile
   long long pair0;      // global index of the pair's first tile
+  int p;                // the pair's index among the pairs with tiles
 };
 
 __device__ __forceinline__ Unit unit_of(const Cursor& c) {
@@ -257,6 +300,7 @@ __device__ __forceinline__ Unit unit_of(const Cursor& c) {
   x.whole = c.k0 == 0 && c.k1 == c.ntp;
   x.g0 = c.g0;
   x.pair0 = c.g0 - c.k0;
+  x.p = c.p;
   return x;
 }
 
@@ -272,9 +316,10 @@ __device__ __forceinline__ void next_tile(const DecodeArgs& a, int nhg, TilePos&
 }
 
 // Prologue (the 128 threads of warps 0-3; stage 0 as scratch): count the
-// tiles of all pairs, zero the output rows of sequences with none (CTA
-// b % grid owns sequence b's rows), and find where this CTA's share starts.
-// Two short passes over context_lens, each a block-wide reduction or scan.
+// tiles and the pairs with tiles, zero the output rows of sequences with none
+// (CTA b % grid owns sequence b's rows), and find the global tiles where this
+// CTA's share starts and ends. Two short passes over context_lens, each a
+// block-wide reduction or scan.
 template <int BS>
 __device__ void plan_share(const DecodeArgs& a, int nhg, uint8_t* scratch, Misc* ms) {
   constexpr int PER = kScanChunk / 128;
@@ -282,11 +327,12 @@ __device__ void plan_share(const DecodeArgs& a, int nhg, uint8_t* scratch, Misc*
   const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
   int* empty_s = reinterpret_cast<int*>(scratch);                   // [kScanChunk]
   int* nempty = empty_s + kScanChunk;
-  long long* wsum = reinterpret_cast<long long*>(scratch + 4 * kScanChunk + 64);   // [4]
+  long long* wsum = reinterpret_cast<long long*>(scratch + 4 * kScanChunk + 64);   // [2][4 warps]
   auto bar = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
 
-  // pass 1: tiles of every sequence (per KV-head group); rows of empty ones
-  long long mine = 0;
+  // pass 1: tiles of every sequence (per KV-head group), sequences with tiles;
+  // rows of empty ones
+  long long mine = 0, mine_ne = 0;
   for (int b0 = 0; b0 < a.B; b0 += kScanChunk) {
     if (tid == 0) *nempty = 0;
     bar();
@@ -297,6 +343,7 @@ __device__ void plan_share(const DecodeArgs& a, int nhg, uint8_t* scratch, Misc*
       int ctx, st;
       const int n = seq_tiles<BS>(a, b, ctx, st);
       mine += n;
+      mine_ne += n > 0;
       if (n == 0 && (b % grid) == cta) empty_s[atomicAdd(nempty, 1)] = b;
     }
     bar();
@@ -312,49 +359,86 @@ __device__ void plan_share(const DecodeArgs& a, int nhg, uint8_t* scratch, Misc*
     bar();
   }
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
-  if (lane == 0) wsum[warp] = mine;
+  for (int o = 16; o >= 1; o >>= 1) {
+    mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    mine_ne += __shfl_xor_sync(0xffffffffu, mine_ne, o);
+  }
+  if (lane == 0) { wsum[warp] = mine; wsum[4 + warp] = mine_ne; }
   bar();
   const long long T = (long long)nhg * (wsum[0] + wsum[1] + wsum[2] + wsum[3]);
-  const long long r0 = T > 0 ? share_begin(cta, T, grid) : 0;
-  const long long r1 = T > 0 ? share_begin(cta + 1, T, grid) : 0;
+  const long long NP = (long long)nhg * (wsum[4] + wsum[5] + wsum[6] + wsum[7]);
+  const long long pc = a.pair_cost;
+  const long long C = kCostTile * T + pc * NP;
+  // the share: tiles whose cost positions lie in [t0, t1)
+  const long long t0 = T > 0 ? share_begin(cta, C, grid) : 0;
+  const long long t1 = T > 0 ? share_begin(cta + 1, C, grid) : 0;
+  bar();
   if (tid == 0) {
-    ms->T = T; ms->r0 = r0; ms->r1 = r1;
+    ms->C = C; ms->r0 = T; ms->r1 = T;
     ms->valid = 0; ms->found = 0;
   }
   bar();
-  if (r0 >= r1) return;                   // an empty share (fewer tiles than CTAs)
+  if (T == 0 || t0 >= t1) return;
 
-  // pass 2: the sequence whose tiles hold global tile r0 (a scan, 128 sequences a round)
-  long long carry = 0;                    // tiles per group of the sequences before this round
+  // pass 2: the first tile whose position is >= t0 (the share's first) and the
+  // first whose position is >= t1 (the next share's first), a scan over the
+  // sequences, 128 a round; each sequence with tiles holds the targets that
+  // lie after its predecessor's last tile position and up to its own last.
+  long long carry = 0, carry_ne = 0;      // tiles per group, sequences with tiles, before this round
   for (int b0 = 0; b0 < a.B; b0 += 128) {
     const int b = b0 + tid;
     int ctx = 0, st = 0;
     const int n = b < a.B ? seq_tiles<BS>(a, b, ctx, st) : 0;
-    long long incl = n;
+    long long incl = n, incl_ne = n > 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const long long t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
+      const long long u = __shfl_up_sync(0xffffffffu, incl_ne, o);
+      if (lane >= o) { incl += t; incl_ne += u; }
     }
-    if (lane == 31) wsum[warp] = incl;
+    if (lane == 31) { wsum[warp] = incl; wsum[4 + warp] = incl_ne; }
     bar();
-    long long wpre = 0;
-    for (int w = 0; w < warp; ++w) wpre += wsum[w];
-    const long long before = carry + wpre + incl - n;         // tiles per group before b
-    const long long lo = (long long)nhg * before;
-    if (n > 0 && lo <= r0 && r0 < lo + (long long)nhg * n) {
-      const long long d = r0 - lo;
-      ms->b0 = b;
-      ms->h0 = (int)(d / n);
-      ms->k0 = (int)(d % n);
-      ms->valid = 1;
-      ms->found = 1;
+    long long wpre = 0, wpre_ne = 0;
+    for (int w = 0; w < warp; ++w) { wpre += wsum[w]; wpre_ne += wsum[4 + w]; }
+    if (n > 0) {
+      const long long x0 = (long long)nhg * (carry + wpre + incl - n);     // its first global tile
+      const long long p0 = (long long)nhg * (carry_ne + wpre_ne + incl_ne - 1);   // its first pair
+      const long long last = tile_cost(x0 + (long long)nhg * n - 1, p0 + nhg - 1, pc);
+      const long long prev = p0 > 0 ? tile_cost(x0 - 1, p0 - 1, pc) : -1;
+      // the first tile of this sequence at position >= t (prev < t <= last)
+      auto locate = [&](long long t, int& h, int& k) {
+        h = 0;
+        while (h + 1 < nhg && tile_cost(x0 + (long long)(h + 1) * n - 1, p0 + h, pc) < t) ++h;
+        const long long first = tile_cost(x0 + (long long)h * n, p0 + h, pc);
+        k = t <= first ? 0 : (int)((t - first + kCostTile - 1) / kCostTile);
+      };
+      if (prev < t0 && t0 <= last) {
+        int h, k;
+        locate(t0, h, k);
+        ms->b0 = b;
+        ms->h0 = h;
+        ms->k0 = k;
+        ms->p0 = (int32_t)(p0 + h);
+        ms->r0 = x0 + (long long)h * n + k;
+        ms->valid = 1;
+        atomicOr(&ms->found, 1);
+      }
+      if (prev < t1 && t1 <= last) {
+        int h, k;
+        locate(t1, h, k);
+        ms->r1 = x0 + (long long)h * n + k;
+        atomicOr(&ms->found, 2);
+      }
     }
     carry += wsum[0] + wsum[1] + wsum[2] + wsum[3];
+    carry_ne += wsum[4] + wsum[5] + wsum[6] + wsum[7];
     bar();
-    if (ms->found) break;
+    if (ms->found == 3) break;
   }
+  bar();
+  // no tile at or after t1: the share runs to the end of the list
+  if (tid == 0 && ms->valid && ms->r0 >= ms->r1) ms->valid = 0;
+  bar();
 }
 
 // Take a ticket on a pair: true for the piece that arrives last. Lock-free
@@ -376,40 +460,51 @@ __device__ __forceinline__ bool take_ticket(unsigned long long* word, unsigned l
 
 // The last piece of a pair: merge every piece's (m, l, o) of the group's NS
 // query heads. 128 threads: thread `row` takes query head n = row / TPR and
-// DPT consecutive d. Writes the staging buffer (normalised output rows in the
-// output type, or, in the split-only pass, fp32 rows plus M and L).
+// DPT consecutive d. A piece's loads (m, l and its DPT values) are issued
+// together, and with DPT <= 16 two pieces' (more would cost registers the
+// CTA does not have). Writes the staging buffer (normalised output rows in
+// the output type, or, in the split-only pass, fp32 rows plus M and L).
 template <int G>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs& a, const Unit& x, int row,
-                                             uint8_t* stg, long long T, int grid, bool final_out,
+                                             uint8_t* stg, long long C, int grid, bool final_out,
                                              size_t cas_row0) {
   constexpr int NS = kHG * G, TPR = 128 / NS, DPT = kD / TPR;
+  constexpr int NB = DPT <= 16 ? 2 : 1;          // pieces whose loads are in flight together
   const int n = row / TPR, d0 = (row % TPR) * DPT;
-  const int c0 = share_owner(x.pair0, T, grid);
-  const int c1 = share_owner(x.pair0 + x.ntp - 1, T, grid);
+  const PairShares ps = pair_shares(x.pair0, x.ntp, x.p, C, grid, a.pair_cost);
   float M = -CUDART_INF_F, L = 0.f, o[DPT];
 #pragma unroll
   for (int e = 0; e < DPT; ++e) o[e] = 0.f;
 #pragma unroll 1
-  for (int c = c0; c <= c1; ++c) {
-    const long long sb = share_begin(c, T, grid);
-    if (share_begin(c + 1, T, grid) <= sb) continue;       // an empty share: no piece
-    const size_t s = 2 * (size_t)c + (sb < x.pair0 ? 1 : 0);
-    const float m = __ldcg(a.sk_m + s * NS + n);
-    if (m == -CUDART_INF_F) continue;                       // no valid token in that piece
-    const float l = __ldcg(a.sk_l + s * NS + n);
-    const float Mn = fmaxf(M, m);
-    const float ca = exp2f(M - Mn), cb = exp2f(m - Mn);     // M = -inf gives ca = 0
-    L = fmaf(L, ca, l * cb);
-    const float4* src = reinterpret_cast<const float4*>(a.sk_acc + (s * NS + n) * kD + d0);
+  for (int c = ps.c0; c <= ps.c1; c += NB) {
+    float m[NB], l[NB];
+    float4 v[NB][DPT / 4];
 #pragma unroll
-    for (int e = 0; e < DPT / 4; ++e) {
-      const float4 v = __ldcg(src + e);
-      o[4 * e + 0] = fmaf(o[4 * e + 0], ca, v.x * cb);
-      o[4 * e + 1] = fmaf(o[4 * e + 1], ca, v.y * cb);
-      o[4 * e + 2] = fmaf(o[4 * e + 2], ca, v.z * cb);
-      o[4 * e + 3] = fmaf(o[4 * e + 3], ca, v.w * cb);
+    for (int j = 0; j < NB; ++j) {
+      const int cj = c + j;
+      const bool has = cj <= ps.c1 && share_holds(ps, cj, C, grid);   // else no piece there
+      const size_t s = 2 * (size_t)cj + (cj == ps.c0 && ps.c0_before ? 1 : 0);
+      m[j] = has ? __ldcg(a.sk_m + s * NS + n) : -CUDART_INF_F;
+      l[j] = has ? __ldcg(a.sk_l + s * NS + n) : 0.f;
+      const float4* src = reinterpret_cast<const float4*>(a.sk_acc + (s * NS + n) * kD + d0);
+#pragma unroll
+      for (int e = 0; e < DPT / 4; ++e) v[j][e] = has ? __ldcg(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    M = Mn;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (m[j] == -CUDART_INF_F) continue;    // no piece, or no valid token in it
+      const float Mn = fmaxf(M, m[j]);
+      const float ca = exp2f(M - Mn), cb = exp2f(m[j] - Mn);   // M = -inf gives ca = 0
+      L = fmaf(L, ca, l[j] * cb);
+#pragma unroll
+      for (int e = 0; e < DPT / 4; ++e) {
+        o[4 * e + 0] = fmaf(o[4 * e + 0], ca, v[j][e].x * cb);
+        o[4 * e + 1] = fmaf(o[4 * e + 1], ca, v[j][e].y * cb);
+        o[4 * e + 2] = fmaf(o[4 * e + 2], ca, v[j][e].z * cb);
+        o[4 * e + 3] = fmaf(o[4 * e + 3], ca, v[j][e].w * cb);
+      }
+      M = Mn;
+    }
   }
   if (final_out) {
     const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -524,20 +619,18 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
   // next unit accumulates while the previous one is merged
   const uint32_t tmem_o = tmem + 2 * S::SW;
   auto obuf = [&](int ui, int g) { return tmem_o + (uint32_t)((2 * (ui & 1) + g) * NO); };
-  const long long T = ms->T, r0 = ms->r0;
+  const long long C = ms->C, r0 = ms->r0;
   const int grid = (int)gridDim.x, cta = (int)blockIdx.x;
   auto give_up = [&]() {
     *abort_flag = 1u;
     flag_error(a.err_flag, PA_DEV_TIMEOUT);
   };
-  // token range of tile k of a unit, and how many of its boxes hold tokens
-  // a stage is ready for the tensor cores when TMA filled it (16-bit pools) or
-  // when its owning group widened it (FP8 pools)
   // K of a tile is ready for the tensor cores when TMA has filled its stage. V
   // is ready when TMA has filled its stage (16-bit pools), or, with FP8 pools,
   // when the group that owns the tile has widened its codes into the group's V
   // buffer, which it does before it hands over the tile's P (PREADY).
   auto k_ready_bar = [&](int s) { return bar(Bx::FULL + s); };
+  // token range of tile k of a unit, and how many of its boxes hold tokens
   auto tile_span = [&](const Unit& x, int k, int& ts, int& te, int& nql) {
     ts = x.t0 + k * kRt;
     te = min(x.t1, ts + kRt);
@@ -1156,14 +1249,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmK,
             bulk_wait_all();
             fence_proxy_async_global();
             __threadfence();
-            const int np = pair_pieces(x.pair0, x.ntp, T, grid);
+            const int np = pair_pieces(pair_shares(x.pair0, x.ntp, x.p, C, grid, a.pair_cost), C, grid);
             ms->last[grp] =
                 take_ticket(a.tickets + (size_t)x.b * nhg + x.h, a.epoch, np, a.err_flag) ? 1 : 0;
           }
           wg_sync(grp);
           if (ms->last[grp]) {
             __threadfence();
-            merge_pieces<G>(a, x, row, stg, T, grid, !a.force_split, cas_row0);
+            merge_pieces<G>(a, x, row, stg, C, grid, !a.force_split, cas_row0);
             fence_proxy_async();
             wg_sync(grp);
             if (row == 0) {

@@ -65,6 +65,21 @@ int tc_test_withhold_q() {
   return s && s[0] == '1' ? 1 : 0;
 }
 
+// Cost of a pair's start and end in the tensor-core kernel's work split, in
+// 1/16 of a tile. Per-CTA timers on the Llama-3-70B-shaped batch put a unit's
+// query load, first-tile reduction and epilogue at 1.2-1.5 tiles' time; a
+// sweep of 0-60 on the GQA, FP8 GQA, long-context and shared-prefix batches
+// was fastest at 28 or within 1.5% of it. PA_TC_PAIR_COST overrides it (0 =
+// equal tile counts), for measurements.
+constexpr int kPairCostDefault = 28;
+int tc_pair_cost() {
+  const char* s = std::getenv("PA_TC_PAIR_COST");
+  if (!s || !*s) return kPairCostDefault;
+  char* end = nullptr;
+  const long v = std::strtol(s, &end, 10);
+  return (end && *end == 0 && v >= 0 && v <= 4096) ? (int)v : kPairCostDefault;
+}
+
 // A number per call of the tensor-core path (40 bits; its tickets carry it).
 unsigned long long next_epoch() {
   static std::atomic<unsigned long long> n{
@@ -243,6 +258,7 @@ int decode_impl(void* out, int out_dtype, const void* query, int q_dtype, const 
     tc_carve(a, static_cast<char*>(workspace));
     a.epoch = next_epoch();
     a.wait_ns = tc_wait_ns();
+    a.pair_cost = tc_pair_cost();
     a.test_withhold_q = tc_test_withhold_q();
   } else if (p.P > 1) {
     const size_t need = decode_scratch_bytes(p, B, Hq, Hkv, D);
@@ -439,6 +455,7 @@ int shared_prefix_impl(void* out, int out_dtype, const void* query, int q_dtype,
     tc_carve(a, w + part_bytes);
     a.epoch = next_epoch();
     a.wait_ns = tc_wait_ns();
+    a.pair_cost = tc_pair_cost();
     a.test_withhold_q = tc_test_withhold_q();
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -48,6 +48,8 @@ struct DecodeArgs {
   unsigned long long* tickets;    // [B * (Hkv / 4)]
   unsigned long long epoch;       // this call's number (40 bits)
   unsigned long long wait_ns;     // limit of every pipeline wait of the tensor-core kernel
+  int pair_cost;                  // work split: cost of a pair's start and end, in 1/16 of a
+                                  // tile's (the CTAs take equal shares of tiles + pair costs)
   int test_withhold_q;            // timeout-path test only: the first unit's query is never
                                   // loaded, so the wait for it can only run out
 };

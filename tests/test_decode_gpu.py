@@ -289,16 +289,25 @@ def _decode_with(w, t, ws, out_dtype=torch.float32, mcl=None):
     ([1, 1, 1], 8, 4096),                        # fewer tiles than CTAs: empty shares between
     ([40, 1, 70], 4, 8192),                      # pieces with empty shares between them
     ([300 + 37 * i for i in range(150)], 4, None),   # many whole sequences per CTA
+    ([0, 900, 0, 0, 17, 0, 2500] + [0, 33] * 12, 8, None),   # empty sequences between pairs
 ])
-def test_even_split_pieces_merge_to_the_oracle(ctx, G, mcl):
+@pytest.mark.parametrize("pair_cost", [None, "0", "400"])
+def test_even_split_pieces_merge_to_the_oracle(ctx, G, mcl, pair_cost, monkeypatch):
     """Sequences cut into pieces across CTAs (the last piece merges them), whole
     sequences in one CTA, CTAs with nothing to do; the workspace starts full of
     random bytes (tickets of no earlier call), and a second call on the same
-    workspace gives the same bits."""
-    w = _tc_case(ctx, seed=len(ctx) * 31 + G, Hq=8 * G, Hkv=8)
+    workspace gives the same bits. The split weighs each pair's start: with the
+    default weight, with none (equal tile counts), and with a weight of 25
+    tiles, under which shares also fall between two pairs' tiles."""
+    if pair_cost is not None:
+        monkeypatch.setenv("PA_TC_PAIR_COST", pair_cost)
+    w = _tc_case([max(c, 1) for c in ctx], seed=len(ctx) * 31 + G, Hq=8 * G, Hkv=8)
     t = device_inputs(w)
     ops.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"],
                              t["slot_mapping"])
+    if min(ctx) == 0:           # empty sequences attend nothing (their new token stays unread)
+        w.context_lens = np.array(ctx, dtype=w.context_lens.dtype)
+        t["context_lens"].copy_(torch.from_numpy(w.context_lens))
     ws = ops.workspace_for(t["q"], t["k_cache"], mcl or w.max_context_len)
     ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda"))
     out1 = _decode_with(w, t, ws, mcl=mcl)
