@@ -561,7 +561,7 @@ def measure(args, w: W.Workload, rank: int, world: int, local_rank: int, *,
     # the cascade reads each distinct K/V byte once: its algorithmic bytes are the distinct ones
     alg = unique if cascade else kv
     achieved = alg / (dec_ms / 1e3) / 1e9
-    traffic = traffic_record(kname, w.name)
+    traffic = traffic_record(kname, w.name + (" (pa_decode_shared_prefix)" if cascade else ""))
     e2e_value = job_value(kv, Ke, world, e_ms)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
